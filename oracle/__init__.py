@@ -1,0 +1,227 @@
+"""CPU oracle for headwise hybrid (SWA + sparse retrieval) attention.
+
+TEST INFRASTRUCTURE ONLY: the plain fp64 statement of what the attention
+path computes, used to check the CUDA library.  Only the tests, the package
+smoke check and the CPU-baseline leg of the benchmark import this module;
+the library never does, and this module never imports the library.
+
+The arithmetic lives in oracle.cpp (C++17, fp64, std::thread); this file
+compiles it with g++ on first use and marshals numpy arrays through ctypes.
+Each function states the passage of the RTPurbo / RTPurboV2 pages it
+follows (see the header of oracle.cpp for the page titles).
+
+Pinned by the not-gpu tests (tests/test_oracle_pins.py) against brute-force
+masked attention, torch's scaled-dot-product attention in fp64 on CPU,
+closed forms and invariants.  The pages print no worked example, so no
+value here is tied to the authors' own implementation.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+SWA, FULL, SPARSE = 0, 1, 2
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.cpp into liboracle.so (g++ -O2, fp64, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["g++", "-O2", "-std=c++17", "-shared", "-fPIC", "-pthread", "-Wall", "-o", _LIB, _SRC]
+        subprocess.run(cmd, check=True)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        _lib = ctypes.CDLL(_LIB)
+        P = ctypes.c_void_p
+        L = ctypes.c_long
+        I = ctypes.c_int
+        D = ctypes.c_double
+        _lib.oracle_project_rows.argtypes = [P, L, I, P, I, P]
+        _lib.oracle_centroids.argtypes = [P, L, I, I, P, I, P]
+        _lib.oracle_qbar.argtypes = [P, I, L, I, I, P, I, P]
+        _lib.oracle_scores.argtypes = [P, P, L, I, P]
+        _lib.oracle_select.argtypes = [P, P, L, I, P, L, I, I, I, P, P, P]
+        _lib.oracle_attention_rows.argtypes = [P, P, L, P, P, L, I, I, L, I, P, P, I, D, P]
+        _lib.oracle_attention_probs.argtypes = [P, L, P, L, I, I, L, I, P, P, I, D, P]
+        _lib.oracle_decode_head.argtypes = [P, I, P, P, L, I, P, L, P, I, I, L, I, I, I, I, I, P, P, P, D, P]
+        for f in ("oracle_project_rows", "oracle_centroids", "oracle_qbar", "oracle_scores", "oracle_select",
+                  "oracle_attention_rows", "oracle_attention_probs", "oracle_decode_head"):
+            getattr(_lib, f).restype = None
+    return _lib
+
+
+def _bf16_bits(x) -> np.ndarray:
+    """bf16 data as a C-contiguous uint16 array of its bit patterns.
+
+    Accepts a torch bf16 tensor (any device) or a uint16 numpy array.
+    """
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint16
+        return np.ascontiguousarray(x)
+    import torch
+
+    assert x.dtype == torch.bfloat16
+    return np.ascontiguousarray(x.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16))
+
+
+def _f32(x) -> np.ndarray:
+    if isinstance(x, np.ndarray):
+        return np.ascontiguousarray(x, dtype=np.float32)
+    return np.ascontiguousarray(x.detach().cpu().float().numpy())
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def project_rows(x, proj) -> np.ndarray:
+    """Low-rank projection of bf16 rows [n, 128] -> fp64 [n, 16] (RTPurboV2 page, r = 16)."""
+    xb = _bf16_bits(x).reshape(-1, 128)
+    p = _f32(proj)
+    r = p.shape[1]
+    out = np.empty((xb.shape[0], r), dtype=np.float64)
+    _load().oracle_project_rows(_ptr(xb), xb.shape[0], 128, _ptr(p), r, _ptr(out))
+    return out
+
+
+def centroids(k_head, block: int, proj) -> np.ndarray:
+    """Block centroids of one KV head's keys [N, 128] -> fp64 [N/B, 16] (RTPurboV2 page, clustering)."""
+    kb = _bf16_bits(k_head).reshape(-1, 128)
+    p = _f32(proj)
+    r = p.shape[1]
+    n = kb.shape[0]
+    out = np.empty((n // block, r), dtype=np.float64)
+    _load().oracle_centroids(_ptr(kb), n, 128, block, _ptr(p), r, _ptr(out))
+    return out
+
+
+def qbar(q_group, block: int, proj) -> np.ndarray:
+    """Query-block summaries of one group's heads [G, N, 128] -> fp64 [N/B, 16]."""
+    qb = _bf16_bits(q_group)
+    G = qb.shape[0]
+    qb = qb.reshape(G, -1, 128)
+    n = qb.shape[1]
+    p = _f32(proj)
+    r = p.shape[1]
+    out = np.empty((n // block, r), dtype=np.float64)
+    _load().oracle_qbar(_ptr(qb), G, n, 128, block, _ptr(p), r, _ptr(out))
+    return out
+
+
+def scores(qbar_row: np.ndarray, C: np.ndarray) -> np.ndarray:
+    """s_j = qbar . c_j for every block j (fp64)."""
+    q = np.ascontiguousarray(qbar_row, dtype=np.float64)
+    c = np.ascontiguousarray(C, dtype=np.float64)
+    out = np.empty(c.shape[0], dtype=np.float64)
+    _load().oracle_scores(_ptr(q), _ptr(c), c.shape[0], c.shape[1], _ptr(out))
+    return out
+
+
+def select(qbar_rows: np.ndarray, C: np.ndarray, t_list, topk: int, n_local: int):
+    """Block selection (sink + top-k by (score desc, index asc) + local).
+
+    Returns (sel [nq, kmax] int32 padded with -1, cnt [nq], kth_score [nq]).
+    """
+    q = np.ascontiguousarray(qbar_rows, dtype=np.float64)
+    c = np.ascontiguousarray(C, dtype=np.float64)
+    t = np.ascontiguousarray(t_list, dtype=np.int32)
+    nq = t.shape[0]
+    kmax = topk + 1 + n_local
+    sel = np.empty((nq, kmax), dtype=np.int32)
+    cnt = np.empty(nq, dtype=np.int32)
+    kth = np.empty(nq, dtype=np.float64)
+    _load().oracle_select(_ptr(q), _ptr(c), c.shape[0], c.shape[1], _ptr(t), nq, topk, n_local, kmax, _ptr(sel),
+                          _ptr(cnt), _ptr(kth))
+    return sel, cnt, kth
+
+
+def attention_rows(q_rows, pos, k_head, v_head, mode: int, window: int = 0, block: int = 64, sel=None, cnt=None,
+                   scale: float | None = None) -> np.ndarray:
+    """Exact softmax attention for given rows of one query head -> fp64 [n, 128].
+
+    mode 0 = SWA (i-W < j <= i), 1 = full causal, 2 = sparse over sel[t(i)].
+    """
+    qb = _bf16_bits(q_rows).reshape(-1, 128)
+    pp = np.ascontiguousarray(pos, dtype=np.int64)
+    kb = _bf16_bits(k_head).reshape(-1, 128)
+    vb = _bf16_bits(v_head).reshape(-1, 128)
+    n = kb.shape[0]
+    if sel is None:
+        sel = np.zeros((1, 1), dtype=np.int32)
+        cnt = np.zeros(1, dtype=np.int32)
+    s = np.ascontiguousarray(sel, dtype=np.int32)
+    c = np.ascontiguousarray(cnt, dtype=np.int32)
+    kmax = s.shape[-1]
+    sc = 1.0 / np.sqrt(128.0) if scale is None else float(scale)
+    out = np.empty((qb.shape[0], 128), dtype=np.float64)
+    _load().oracle_attention_rows(_ptr(qb), _ptr(pp), qb.shape[0], _ptr(kb), _ptr(vb), n, 128, mode, window, block,
+                                  _ptr(s), _ptr(c), kmax, sc, _ptr(out))
+    return out
+
+
+def attention_probs(q_row, i: int, k_head, mode: int, window: int = 0, block: int = 64, sel=None, cnt=None,
+                    scale: float | None = None) -> np.ndarray:
+    """Normalised attention weights of one row over all N keys (0 where invisible)."""
+    qb = _bf16_bits(q_row).reshape(128)
+    kb = _bf16_bits(k_head).reshape(-1, 128)
+    n = kb.shape[0]
+    if sel is None:
+        sel = np.zeros((1, 1), dtype=np.int32)
+        cnt = np.zeros(1, dtype=np.int32)
+    s = np.ascontiguousarray(sel, dtype=np.int32)
+    c = np.ascontiguousarray(cnt, dtype=np.int32)
+    sc = 1.0 / np.sqrt(128.0) if scale is None else float(scale)
+    out = np.empty(n, dtype=np.float64)
+    _load().oracle_attention_probs(_ptr(qb), i, _ptr(kb), n, 128, mode, window, block, _ptr(s), _ptr(c),
+                                   s.shape[-1], sc, _ptr(out))
+    return out
+
+
+def decode_head(q_group, kc_head, vc_head, C_head, proj, mode: int, window: int, block: int, topk: int,
+                n_local: int, sel=None, cnt=None, scale: float | None = None):
+    """Sparse / SWA decode of one sequence and one KV head (query at Lc-1).
+
+    q_group [G, 128] bf16; caches [Lc, 128] bf16; C_head [Lc/B, 16] fp32.
+    If sel/cnt are given (one row), that selection is used; otherwise the
+    oracle selects.  Returns (out [G,128] fp64, sel [kmax], cnt, kth_score).
+    """
+    qb = _bf16_bits(q_group).reshape(-1, 128)
+    G = qb.shape[0]
+    kb = _bf16_bits(kc_head).reshape(-1, 128)
+    vb = _bf16_bits(vc_head).reshape(-1, 128)
+    Lc = kb.shape[0]
+    Cf = _f32(C_head).reshape(-1, 16)
+    p = _f32(proj)
+    kmax = topk + 1 + n_local
+    use_given = sel is not None
+    s = np.full(kmax, -1, dtype=np.int32) if sel is None else np.ascontiguousarray(sel, dtype=np.int32).reshape(-1)
+    c = np.zeros(1, dtype=np.int32) if cnt is None else np.array([int(np.asarray(cnt).reshape(-1)[0])],
+                                                                  dtype=np.int32)
+    kth = np.zeros(1, dtype=np.float64)
+    sc = 1.0 / np.sqrt(128.0) if scale is None else float(scale)
+    out = np.empty((G, 128), dtype=np.float64)
+    _load().oracle_decode_head(_ptr(qb), G, _ptr(kb), _ptr(vb), Lc, 128, _ptr(Cf), Cf.shape[0], _ptr(p), 16, mode,
+                               window, block, topk, n_local, kmax, int(use_given), _ptr(s), _ptr(c), _ptr(kth), sc,
+                               _ptr(out))
+    return out, s, int(c[0]), float(kth[0])
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round fp64 values to the nearest bf16 (ties to even), returned as fp64."""
+    f = np.asarray(x, dtype=np.float64).astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)

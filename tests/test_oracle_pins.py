@@ -1,0 +1,328 @@
+"""Pins of the CPU oracle against things other than itself.
+
+The pages print no worked example, so the oracle is pinned by construction:
+  * brute-force dense attention over an explicit boolean mask built here from
+    the visibility rules (window, causal, selected blocks);
+  * torch's scaled_dot_product_attention on CPU in fp64 with the same mask;
+  * invariants: SWA with W >= N equals full causal, sparse attention whose
+    selection covers every block equals full causal, each row of weights is
+    a distribution, V = 1 gives O = 1, a single visible key returns its V row;
+  * projection/centroids: coordinate selection is exact, centroids are linear
+    (mean of projections = projection of the mean), random projector equals a
+    plain matrix product;
+  * selection: brute-force scoring + full sort with the (score desc, index asc)
+    rule, a planted dominant block, degenerate sizes;
+  * decode: equals the last prefill row when both use the same selection.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from swa_hybrid_attention_b200 import inputs
+
+SCALE = 1.0 / np.sqrt(128.0)
+
+
+def widen(x):
+    return x.float().double().cpu().numpy()
+
+
+def mask_matrix(n, mode, window=0, block=64, sel=None, cnt=None):
+    """Explicit [n, n] visibility mask, built from the rules directly."""
+    i = np.arange(n)[:, None]
+    j = np.arange(n)[None, :]
+    m = j <= i
+    if mode == oracle.SWA:
+        m = m & (j > i - window)
+    elif mode == oracle.SPARSE:
+        allowed = np.zeros((n // block + 1, n // block + 1), dtype=bool)
+        for t in range(n // block):
+            for e in range(cnt[t]):
+                allowed[t, sel[t, e]] = True
+        m = m & allowed[i // block, j // block]
+    return m
+
+
+def dense_reference(q, k, v, m):
+    s = (q @ k.T) * SCALE
+    s = np.where(m, s, -np.inf)
+    s = s - s.max(axis=1, keepdims=True)
+    p = np.exp(s)
+    p = p / p.sum(axis=1, keepdims=True)
+    return p @ v
+
+
+def random_selection(n, block, kmax, rng):
+    """A random valid selection per query block: diagonal always, sink, random earlier blocks."""
+    nb = n // block
+    sel = np.full((nb, kmax), -1, dtype=np.int32)
+    cnt = np.zeros(nb, dtype=np.int32)
+    for t in range(nb):
+        pool = list(range(1, t))
+        rng.shuffle(pool)
+        chosen = sorted(set([0, t] + pool[: kmax - 2]))
+        sel[t, : len(chosen)] = chosen
+        cnt[t] = len(chosen)
+    return sel, cnt
+
+
+@pytest.fixture(scope="module")
+def small():
+    return inputs.small_prefill(384, 2, 1, [oracle.FULL], seed=7)
+
+
+@pytest.mark.parametrize("n", [128, 384, 1024])
+@pytest.mark.parametrize("mode,window", [(oracle.FULL, 0), (oracle.SWA, 100), (oracle.SWA, 1), (oracle.SWA, 256)])
+def test_attention_matches_bruteforce(n, mode, window):
+    d = inputs.small_prefill(n, 1, 1, [mode], seed=11 + n)
+    q, k, v = d["q"][0, 0], d["k"][0, 0], d["v"][0, 0]
+    rows = np.arange(n)
+    got = oracle.attention_rows(q, rows, k, v, mode, window)
+    ref = dense_reference(widen(q), widen(k), widen(v), mask_matrix(n, mode, window))
+    assert np.max(np.abs(got - ref)) <= 1e-12
+
+
+@pytest.mark.parametrize("n,block", [(384, 64), (1024, 128), (1024, 64)])
+def test_sparse_attention_matches_bruteforce(n, block):
+    rng = np.random.default_rng(n + block)
+    d = inputs.small_prefill(n, 1, 1, [oracle.SPARSE], seed=3)
+    q, k, v = d["q"][0, 0], d["k"][0, 0], d["v"][0, 0]
+    sel, cnt = random_selection(n, block, 5, rng)
+    got = oracle.attention_rows(q, np.arange(n), k, v, oracle.SPARSE, 0, block, sel, cnt)
+    ref = dense_reference(widen(q), widen(k), widen(v), mask_matrix(n, oracle.SPARSE, 0, block, sel, cnt))
+    assert np.max(np.abs(got - ref)) <= 1e-12
+
+
+def test_attention_matches_torch_sdpa_fp64():
+    n, block = 512, 64
+    rng = np.random.default_rng(5)
+    d = inputs.small_prefill(n, 1, 1, [oracle.SPARSE], seed=21)
+    q, k, v = d["q"][0, 0], d["k"][0, 0], d["v"][0, 0]
+    sel, cnt = random_selection(n, block, 4, rng)
+    for mode, window in [(oracle.FULL, 0), (oracle.SWA, 77), (oracle.SPARSE, 0)]:
+        m = mask_matrix(n, mode, window, block, sel, cnt)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q.double()[None, None], k.double()[None, None], v.double()[None, None],
+            attn_mask=torch.from_numpy(m)[None, None], scale=SCALE)[0, 0].numpy()
+        got = oracle.attention_rows(q, np.arange(n), k, v, mode, window, block, sel, cnt)
+        assert np.max(np.abs(got - ref)) <= 1e-12
+
+
+def test_swa_with_window_ge_seq_is_full_bitwise(small):
+    q, k, v = small["q"][0, 0], small["k"][0, 0], small["v"][0, 0]
+    n = q.shape[0]
+    rows = np.arange(n)
+    full = oracle.attention_rows(q, rows, k, v, oracle.FULL)
+    for w in (n, n + 1, 10 * n):
+        swa = oracle.attention_rows(q, rows, k, v, oracle.SWA, w)
+        assert np.array_equal(full, swa)
+
+
+def test_sparse_covering_all_blocks_is_full_bitwise(small):
+    q, k, v = small["q"][0, 0], small["k"][0, 0], small["v"][0, 0]
+    n, block = q.shape[0], 64
+    nb = n // block
+    sel = np.tile(np.arange(nb, dtype=np.int32), (nb, 1))
+    cnt = np.full(nb, nb, dtype=np.int32)
+    rows = np.arange(n)
+    full = oracle.attention_rows(q, rows, k, v, oracle.FULL)
+    sp = oracle.attention_rows(q, rows, k, v, oracle.SPARSE, 0, block, sel, cnt)
+    assert np.array_equal(full, sp)
+
+
+@pytest.mark.parametrize("mode,window", [(oracle.FULL, 0), (oracle.SWA, 50)])
+def test_rows_are_distributions(small, mode, window):
+    q, k = small["q"][0, 0], small["k"][0, 0]
+    n = q.shape[0]
+    for i in (0, 1, 49, 50, 51, 200, n - 1):
+        p = oracle.attention_probs(q[i], i, k, mode, window)
+        assert abs(p.sum() - 1.0) <= 1e-12
+        vis = np.arange(n) <= i
+        if mode == oracle.SWA:
+            vis &= np.arange(n) > i - window
+        assert np.all(p[~vis] == 0.0) and np.all(p[vis] > 0.0)
+
+
+def test_ones_value_gives_ones(small):
+    q, k = small["q"][0, 0], small["k"][0, 0]
+    ones = torch.ones_like(k)
+    n = q.shape[0]
+    for mode, w in [(oracle.FULL, 0), (oracle.SWA, 7)]:
+        o = oracle.attention_rows(q, np.arange(n), k, ones, mode, w)
+        assert np.max(np.abs(o - 1.0)) <= 1e-14
+
+
+def test_single_visible_key_returns_its_value(small):
+    q, k, v = small["q"][0, 0], small["k"][0, 0], small["v"][0, 0]
+    # row 0 sees only key 0; with W = 1 every row sees only itself
+    o0 = oracle.attention_rows(q[:1], np.array([0]), k, v, oracle.FULL)
+    assert np.array_equal(o0[0], widen(v[0]))
+    n = q.shape[0]
+    o = oracle.attention_rows(q, np.arange(n), k, v, oracle.SWA, 1)
+    assert np.array_equal(o, widen(v))
+
+
+def test_scale_enters_the_logits():
+    d = inputs.small_prefill(128, 1, 1, [oracle.FULL], seed=2)
+    q, k, v = d["q"][0, 0], d["k"][0, 0], d["v"][0, 0]
+    m = mask_matrix(128, oracle.FULL)
+    s = (widen(q) @ widen(k).T) * 0.3
+    s = np.where(m, s, -np.inf)
+    p = np.exp(s - s.max(1, keepdims=True))
+    ref = (p / p.sum(1, keepdims=True)) @ widen(v)
+    got = oracle.attention_rows(q, np.arange(128), k, v, oracle.FULL, scale=0.3)
+    assert np.max(np.abs(got - ref)) <= 1e-12
+
+
+# ----------------------------------------------------------------- projection
+
+
+def test_lowfreq_projection_selects_coordinates_exactly():
+    d = inputs.small_prefill(256, 1, 1, [oracle.SPARSE], seed=9)
+    k = d["k"][0, 0]
+    got = oracle.project_rows(k, inputs.lowfreq_projector())
+    dims = list(range(56, 64)) + list(range(120, 128))
+    assert np.array_equal(got, widen(k)[:, dims])
+
+
+def test_random_projection_is_matrix_product():
+    d = inputs.small_prefill(256, 1, 1, [oracle.SPARSE], seed=4)
+    k = d["k"][0, 0]
+    p = inputs.random_projector(123)
+    got = oracle.project_rows(k, p)
+    ref = widen(k) @ p.double().numpy()
+    assert np.max(np.abs(got - ref)) <= 1e-12
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_centroids_are_linear(block):
+    d = inputs.small_prefill(1024, 1, 1, [oracle.SPARSE], seed=6)
+    k = d["k"][0, 0]
+    p = inputs.random_projector(5)
+    got = oracle.centroids(k, block, p)
+    mean_k = widen(k).reshape(-1, block, 128).mean(axis=1)
+    ref = mean_k @ p.double().numpy()
+    assert got.shape == (1024 // block, 16)
+    assert np.max(np.abs(got - ref)) <= 1e-12
+
+
+def test_qbar_is_sum_over_heads_of_block_means():
+    d = inputs.small_prefill(512, 4, 1, [oracle.SPARSE], seed=8)
+    q = d["q"][0]
+    p = inputs.random_projector(6)
+    got = oracle.qbar(q, 64, p)
+    qn = widen(q)  # [G, N, 128]
+    ref = sum(qn[h].reshape(-1, 64, 128).mean(axis=1) for h in range(4)) @ p.double().numpy()
+    assert np.max(np.abs(got - ref)) <= 1e-12
+
+
+# ------------------------------------------------------------------ selection
+
+
+def brute_select(qb, C, t, topk, n_local):
+    s = C @ qb
+    cands = list(range(1, t - n_local + 1))
+    if len(cands) > topk:
+        cands = sorted(cands, key=lambda j: (-s[j], j))[:topk]
+    chosen = set(cands) | {0} | set(range(max(0, t - n_local + 1), t + 1))
+    return sorted(chosen)
+
+
+@pytest.mark.parametrize("nb,topk,n_local", [(32, 16, 2), (40, 5, 3), (9, 4, 1), (64, 1, 0), (12, 20, 2)])
+def test_selection_matches_bruteforce(nb, topk, n_local):
+    rng = np.random.default_rng(nb * 100 + topk)
+    C = rng.standard_normal((nb, 16))
+    qb = rng.standard_normal((nb, 16))
+    # plant exact ties to exercise the index tie-break
+    C[5] = C[7]
+    C[nb - 2] = C[3]
+    sel, cnt, kth = oracle.select(qb, C, np.arange(nb), topk, n_local)
+    for t in range(nb):
+        ref = brute_select(qb[t], C, t, topk, n_local)
+        assert cnt[t] == len(ref)
+        assert list(sel[t, : cnt[t]]) == ref
+        assert np.all(sel[t, cnt[t]:] == -1)
+        ncand = max(0, t - n_local)
+        if ncand > topk:
+            s = C @ qb[t]
+            kept = [j for j in ref if 1 <= j <= t - n_local]
+            assert abs(kth[t] - min(s[j] for j in kept)) <= 1e-12 * (1 + abs(kth[t]))
+        else:
+            assert np.isnan(kth[t])
+
+
+def test_selection_picks_planted_block():
+    rng = np.random.default_rng(1)
+    nb = 64
+    C = rng.standard_normal((nb, 16)) * 0.01
+    qb = rng.standard_normal((nb, 16))
+    C[17] = qb[50] * 10.0  # dominates for query block 50
+    sel, cnt, _ = oracle.select(qb, C, np.arange(nb), 1, 2)
+    assert list(sel[50, : cnt[50]]) == [0, 17, 49, 50]
+
+
+def test_selection_small_t_is_full_causal():
+    rng = np.random.default_rng(2)
+    nb = 16
+    C = rng.standard_normal((nb, 16))
+    qb = rng.standard_normal((nb, 16))
+    sel, cnt, _ = oracle.select(qb, C, np.arange(nb), 8, 2)
+    for t in range(0, 11):  # t - L <= k: every earlier block is kept
+        assert list(sel[t, : cnt[t]]) == list(range(t + 1))
+
+
+# --------------------------------------------------------------------- decode
+
+
+def test_decode_equals_last_prefill_row():
+    Lc, block, G = 1024, 64, 4
+    d = inputs.small_prefill(Lc, G, 1, [oracle.SPARSE], seed=31)
+    q, k, v = d["q"][0], d["k"][0, 0], d["v"][0, 0]
+    p = inputs.lowfreq_projector()
+    C = oracle.centroids(k, block, p).astype(np.float32)
+    out, sel, cnt, _ = oracle.decode_head(q[:, Lc - 1], k, v, C, p, oracle.SPARSE, 0, block, 4, 2)
+    nb = Lc // block
+    t = nb - 1
+    sel_full = np.full((nb, sel.shape[0]), -1, dtype=np.int32)
+    cnt_full = np.ones(nb, dtype=np.int32)
+    sel_full[:, 0] = 0
+    sel_full[t] = sel
+    cnt_full[t] = cnt
+    for h in range(G):
+        ref = oracle.attention_rows(q[h, Lc - 1:Lc], np.array([Lc - 1]), k, v, oracle.SPARSE, 0, block, sel_full,
+                                    cnt_full)
+        assert np.array_equal(out[h], ref[0])
+    # the oracle's own selection is the brute-force one on the decode summary
+    qb = oracle.project_rows(q[:, Lc - 1], p).sum(axis=0)
+    assert list(sel[:cnt]) == brute_select(qb, C.astype(np.float64), t, 4, 2)
+
+
+def test_decode_swa_equals_window_row():
+    Lc, G, W = 700, 2, 300
+    d = inputs.small_prefill(Lc, G, 1, [oracle.SWA], seed=41)
+    q, k, v = d["q"][0], d["k"][0, 0], d["v"][0, 0]
+    C = np.zeros((Lc // 64, 16), dtype=np.float32)
+    out, _, _, _ = oracle.decode_head(q[:, Lc - 1], k, v, C, inputs.lowfreq_projector(), oracle.SWA, W, 64, 4, 2)
+    for h in range(G):
+        ref = oracle.attention_rows(q[h, Lc - 1:Lc], np.array([Lc - 1]), k, v, oracle.SWA, W)
+        assert np.array_equal(out[h], ref[0])
+
+
+def test_round_bf16():
+    x = np.array([1.0, 1.00390625, 1.005859375, -3.14159, 0.0, 65504.0])
+    got = oracle.round_bf16(x)
+    ref = torch.tensor(x, dtype=torch.float64).to(torch.bfloat16).double().numpy()
+    assert np.array_equal(got, ref)
+
+
+def test_selection_ties_at_the_cut_take_lower_indices():
+    nb, topk, L = 40, 6, 2
+    C = np.ones((nb, 16))
+    qb = np.ones((nb, 16))
+    C[30] = 2.0  # one clear winner, every other candidate ties
+    sel, cnt, kth = oracle.select(qb, C, np.arange(nb), topk, L)
+    t = 39
+    assert list(sel[t, : cnt[t]]) == [0, 1, 2, 3, 4, 5, 30, 38, 39]
+    assert kth[t] == 16.0
