@@ -267,7 +267,8 @@ void oracle_attention_probs(const uint16_t* q_row, long i, const uint16_t* k, lo
 //   q      [G][D] bf16: the group's query heads for this token,
 //   kc, vc [L_c][D] bf16: this KV head's cache,
 //   C      [nbc][r] fp32: cached block centroids (nbc = L_c / B, full blocks),
-//   mode   0 = SWA (last W keys), 2 = retrieval (selected blocks).
+//   mode   0 = SWA (last W keys), 1 = full (every cached key),
+//          2 = retrieval (selected blocks).
 // For mode 2 the query summary is qbar = sum_h P^T q_h, the selection rule is
 // the prefill one with t = (L_c-1)/B; if use_given_sel is non-zero the
 // selection in sel/cnt is used as given, otherwise it is computed and written
@@ -298,6 +299,8 @@ void oracle_decode_head(const uint16_t* q, int G, const uint16_t* kc, const uint
         for (long j = b * B; j < (b + 1) * B; ++j)
           if (j <= i) keys.push_back(j);
       }
+    } else if (mode == 1) {
+      for (long j = 0; j <= i; ++j) keys.push_back(j);
     } else {
       for (long j = std::max<long>(0, i - window + 1); j <= i; ++j) keys.push_back(j);
     }

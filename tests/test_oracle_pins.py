@@ -310,6 +310,18 @@ def test_decode_swa_equals_window_row():
         assert np.array_equal(out[h], ref[0])
 
 
+def test_decode_full_head_sees_whole_cache():
+    Lc, G = 700, 2
+    d = inputs.small_prefill(Lc, G, 1, [oracle.FULL], seed=43)
+    q, k, v = d["q"][0], d["k"][0, 0], d["v"][0, 0]
+    C = np.zeros((Lc // 64, 16), dtype=np.float32)
+    out, _, _, _ = oracle.decode_head(q[:, Lc - 1], k, v, C, inputs.lowfreq_projector(), oracle.FULL, 10, 64, 4, 2)
+    m = mask_matrix(Lc, oracle.FULL)[Lc - 1:Lc]
+    for h in range(G):
+        ref = dense_reference(widen(q[h, Lc - 1:Lc]), widen(k), widen(v), m)
+        assert np.max(np.abs(out[h] - ref[0])) <= 1e-12
+
+
 def test_round_bf16():
     x = np.array([1.0, 1.00390625, 1.005859375, -3.14159, 0.0, 65504.0])
     got = oracle.round_bf16(x)
