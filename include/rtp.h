@@ -1,0 +1,227 @@
+/*
+ * rtp.h — C ABI of librtp.so: headwise hybrid (SWA + sparse retrieval)
+ * attention for NVIDIA B200 (sm_100a).
+ *
+ * The method (RTPurbo / RTPurboV2) routes every (layer, KV head) to one of
+ * two head types:
+ *   - streaming heads run sliding-window attention (SWA): the pages
+ *     "阿里Qwen3 RTPurbo：15%全量Attention长文本5倍压缩方案" (opening section)
+ *     and "阿里RTPurboV2：Transformer再次崛起，百步训练实现10倍稀少把稳" (window
+ *     8192 for the streaming heads) drop the far tokens of these heads;
+ *   - retrieval heads (about 15 %) run either dense causal attention (V1) or,
+ *     in V2, block-sparse attention: a trained projector maps keys and
+ *     queries from D=128 to r=16 dimensions (RTPurboV2 page, "r=16"), keys
+ *     are grouped (clustered) and summarised by centroids, the best blocks
+ *     for each query block are selected and exact softmax attention runs on
+ *     the selected keys only (summary page of "Full Attention Strikes Back":
+ *     the 16-dim indexer is a cheap scout; real attention runs on the
+ *     selected set).
+ *
+ * The pages leave the selection policy open; this library fixes it:
+ *   - keys are grouped in contiguous blocks of `block` keys; a block's
+ *     centroid is the mean of its projected keys;
+ *   - one selection per (KV head, query block of `block` rows), shared by the
+ *     query heads of the group; the query summary of block t is the sum over
+ *     the group's heads of the mean over the block's rows of the projected
+ *     queries;
+ *   - query block t scores candidate blocks 1..t-n_local by the dot product
+ *     of its summary with their centroids, keeps the `topk` best by
+ *     (score descending, block index ascending) and adds block 0 (sink) and
+ *     the n_local local blocks max(0,t-n_local+1)..t; the list is sorted
+ *     ascending; if at most `topk` candidates exist, all blocks 0..t are
+ *     kept;
+ *   - causal masking j <= i applies inside every selected block;
+ *   - SWA: key j is visible to query i iff i-window < j <= i.
+ *
+ * Conventions
+ *   - Every tensor argument is a DEVICE pointer owned by the caller,
+ *     contiguous.  Q/K/V/O are bf16 [batch][heads][seq][128]
+ *     (`head_dim` must be 128).  All pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = default stream).
+ *     Calls are asynchronous on `stream`; none synchronises except the
+ *     set-up call rtp_route_heads and rtp_last_device_status.
+ *   - Arguments are validated before anything is launched; a bad argument
+ *     returns RTP_ERR_INVALID_ARG and launches nothing.  A CUDA launch error
+ *     returns RTP_ERR_CUDA.  No C++ exception crosses this boundary.
+ *   - Every device-side wait is bounded (about 2 s); a wait that gives up
+ *     ends its kernel early and sets a device status word that
+ *     rtp_last_device_status reports as RTP_ERR_TIMEOUT.
+ *   - A plan is immutable after creation and may be used from several
+ *     streams at once.
+ */
+#ifndef RTP_H_
+#define RTP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RTP_OK = 0,
+  RTP_ERR_INVALID_ARG = 1,
+  RTP_ERR_UNSUPPORTED = 2,
+  RTP_ERR_CUDA = 3,
+  RTP_ERR_TIMEOUT = 4,
+  RTP_ERR_NO_MEMORY = 5
+} rtp_status;
+
+/* Head kinds of the routing map (one byte per KV head). */
+enum { RTP_HEAD_SWA = 0, RTP_HEAD_FULL = 1, RTP_HEAD_SPARSE = 2 };
+
+typedef struct {
+  int batch;       /* sequences                                                  */
+  int seq;         /* tokens per sequence (prefill); multiple of `block`         */
+  int n_q_heads;   /* query heads                                                */
+  int n_kv_heads;  /* KV heads; group = n_q_heads / n_kv_heads must be an even
+                      integer <= 16 (prefill processes query heads in pairs)     */
+  int head_dim;    /* must be 128                                                */
+  int window;      /* SWA keys including self (i-window < j <= i); >= 1          */
+  int block;       /* key block = query block for selection: 64 or 128           */
+  int rank;        /* projector rank r; must be 16                               */
+  int topk;        /* selected candidate blocks per query block                  */
+  int n_sink;      /* sink blocks; must be 1 (block 0)                           */
+  int n_local;     /* local blocks (diagonal included); >= 1                     */
+  float scale;     /* softmax scale; 0 => 1/sqrt(head_dim)                       */
+} rtp_attn_cfg;
+
+typedef struct rtp_plan rtp_plan; /* opaque, library-owned */
+
+/* ------------------------------------------------------------------------
+ * rtp_route_heads — compile the routing map of one layer into a plan.
+ * Pages: RTPurbo page, "RTP-LLM：RTPurbo 在长文上的极致性能优化" (different
+ * head types have different costs; schedule heavy tiles first to cut tail
+ * latency).
+ *   cfg        shapes and selection constants (validated here).
+ *   kind_host  HOST array [cfg->n_kv_heads] of RTP_HEAD_* values.
+ *   stream     stream for the plan's one-time host-to-device upload.
+ *   out        receives the plan; release with rtp_plan_destroy.
+ * The plan holds the work list of the prefill kernel: one entry per
+ * (sequence, KV head, pair of query heads, 128-row query tile), ordered by
+ * descending cost (KV tiles to visit) so that a persistent grid takes the
+ * heaviest tiles first.  Retrieval heads of kind RTP_HEAD_SPARSE are
+ * numbered 0..n_sparse-1 in KV-head order ("retrieval slots"); the indexer
+ * and selection buffers are indexed by slot.
+ * This set-up call uploads the work list on `stream` and synchronises it
+ * before returning, so the plan may then be used on any stream.
+ * Errors: RTP_ERR_INVALID_ARG (bad cfg or kind), RTP_ERR_NO_MEMORY,
+ * RTP_ERR_CUDA.
+ * ---------------------------------------------------------------------- */
+rtp_status rtp_route_heads(const rtp_attn_cfg* cfg, const uint8_t* kind_host, void* stream, rtp_plan** out);
+void rtp_plan_destroy(rtp_plan* plan);
+
+/* Number of retrieval slots (KV heads of kind RTP_HEAD_SPARSE). */
+int rtp_plan_num_sparse(const rtp_plan* plan);
+/* Number of prefill work items (tiles) in the plan. */
+long rtp_plan_num_items(const rtp_plan* plan);
+/* Copies the KV-head index of each retrieval slot into slots_host
+ * [rtp_plan_num_sparse]. */
+rtp_status rtp_plan_sparse_heads(const rtp_plan* plan, int32_t* slots_host);
+/* Copies the plan's work list (HOST int32 [n_items][4] = {kind | slot<<8,
+ * sequence*n_kv_heads + kv_head, query-head pair, query tile}) in the order
+ * the prefill kernel consumes it. */
+rtp_status rtp_plan_work_items(const rtp_plan* plan, int32_t* items_host);
+
+/* ------------------------------------------------------------------------
+ * rtp_indexer_project — low-rank projection, block centroids and query-block
+ * summaries for every retrieval slot (RTPurboV2 page: the projector keeps
+ * the low-frequency rotary components in r=16 dimensions; clustering of the
+ * projected keys; summary page of "Full Attention Strikes Back": the 16-dim
+ * indexer).
+ *   q          bf16 [batch][n_q_heads][seq][128]
+ *   k          bf16 [batch][n_kv_heads][seq][128]
+ *   proj       fp32 [128][16], row d = input dimension
+ *   centroids  fp32 [batch][n_sparse][seq/block][16] (out):
+ *              c_b = (1/block) * sum_{j in block b} proj^T k_j
+ *   qbar       fp32 [batch][n_sparse][seq/block][16] (out):
+ *              qbar_t = sum_{h in group} (1/block) sum_{i in block t} proj^T q_{h,i}
+ * Reductions run in a fixed order (deterministic results).  A plan with no
+ * retrieval slot makes this a no-op.
+ * ---------------------------------------------------------------------- */
+rtp_status rtp_indexer_project(const rtp_plan* plan, const void* q, const void* k, const float* proj,
+                               float* centroids, float* qbar, void* stream);
+
+/* ------------------------------------------------------------------------
+ * rtp_block_select — per (retrieval slot, query block) selection
+ * (RTPurboV2 page: fixed top-k is the classic policy; the rule used is the
+ * one stated at the top of this file).
+ *   qbar, centroids  as written by rtp_indexer_project
+ *   sel      int32 [batch][n_sparse][seq/block][kmax] (out), kmax =
+ *            topk + 1 + n_local: selected block indices, ascending; unused
+ *            entries are -1
+ *   sel_cnt  int32 [batch][n_sparse][seq/block] (out): entries used
+ * Scores are fp32 with a fixed summation order; ties in score go to the
+ * lower block index.
+ * ---------------------------------------------------------------------- */
+rtp_status rtp_block_select(const rtp_plan* plan, const float* qbar, const float* centroids, int32_t* sel,
+                            int32_t* sel_cnt, void* stream);
+
+/* ------------------------------------------------------------------------
+ * rtp_hybrid_prefill — causal prefill attention over the routing map.
+ * RTPurbo page (streaming heads: SWA; full heads: dense causal) and
+ * RTPurboV2 page / "Full Attention Strikes Back" summary (sparse heads:
+ * exact softmax over the selected blocks).  For query head h (KV head
+ * h / group) and query i:  O_i = softmax_j(scale * q_i . k_j) V over the
+ * visible keys of the head's kind.
+ *   q, k, v  bf16 as in rtp_indexer_project
+ *   sel, sel_cnt  from rtp_block_select (may be NULL when the plan has no
+ *            retrieval slot)
+ *   o        bf16 [batch][n_q_heads][seq][128] (out)
+ * bf16 inputs, fp32 accumulation (tensor memory), bf16 output.
+ * ---------------------------------------------------------------------- */
+rtp_status rtp_hybrid_prefill(const rtp_plan* plan, const void* q, const void* k, const void* v,
+                              const int32_t* sel, const int32_t* sel_cnt, void* o, void* stream);
+
+/* ------------------------------------------------------------------------
+ * rtp_sparse_decode — one decode step (one new token per sequence) over a
+ * KV cache (RTPurboV2 page: retrieval heads are sparsified in decode; the
+ * streaming heads keep a window).  The new token's K/V are already the last
+ * cache entry, so the query sits at position cache_len-1.
+ *   cfg        batch, n_q_heads, n_kv_heads, head_dim, window, block, rank,
+ *              topk, n_sink, n_local, scale are used; seq is ignored
+ *   kind_host  HOST [n_kv_heads] (n_kv_heads <= 256): RTP_HEAD_SPARSE
+ *              (retrieval) or RTP_HEAD_SWA; RTP_HEAD_FULL attends to the
+ *              whole cache
+ *   q          bf16 [batch][n_q_heads][1][128]
+ *   kcache, vcache  bf16 [batch][n_kv_heads][cache_len][128]
+ *   centroids  fp32 [batch][n_kv_heads][cache_len/block][16]: centroid of
+ *              every complete cache block (entries of non-retrieval heads
+ *              are not read)
+ *   proj       fp32 [128][16]
+ *   o          bf16 [batch][n_q_heads][1][128] (out)
+ *   workspace  device scratch of at least rtp_decode_workspace_bytes bytes
+ *   sel_out, cnt_out  optional (may be NULL): int32 [batch][n_kv_heads][kmax]
+ *              and [batch][n_kv_heads]: the selected blocks of retrieval
+ *              heads (rows of other heads are left untouched)
+ * Retrieval heads score qbar = sum_{h in group} proj^T q_h against the
+ * centroids of blocks 1..t-n_local (t = (cache_len-1)/block) and attend to
+ * the selected blocks; split-K over blocks, merged by log-sum-exp.
+ * ---------------------------------------------------------------------- */
+size_t rtp_decode_workspace_bytes(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len);
+rtp_status rtp_sparse_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* q,
+                             const void* kcache, const void* vcache, const float* centroids, const float* proj,
+                             void* o, void* workspace, size_t ws_bytes, int32_t* sel_out, int32_t* cnt_out,
+                             void* stream);
+
+/* ------------------------------------------------------------------------
+ * rtp_last_device_status — synchronise `stream`, then read and clear the
+ * device status word of the current device.  Returns RTP_OK, RTP_ERR_TIMEOUT
+ * (a bounded wait gave up), RTP_ERR_INVALID_ARG (a kernel met an
+ * out-of-range block index and skipped it) or RTP_ERR_CUDA (the stream
+ * reported an error).
+ * ---------------------------------------------------------------------- */
+rtp_status rtp_last_device_status(void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* rtp_status_str(rtp_status s);
+
+/* Library version, (major << 16) | minor. */
+int rtp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RTP_H_ */

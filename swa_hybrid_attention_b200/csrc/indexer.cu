@@ -1,0 +1,121 @@
+// Fused low-rank indexer: block centroids of the keys and block summaries of
+// the queries for every retrieval slot.
+//
+// Page "阿里RTPurboV2：Transformer再次崛起，百步训练实现10倍稀少把稳": a projector
+// maps the D=128 features to r=16 (keeping the low-frequency rotary
+// components), and clustering the projected keys lets whole groups of
+// unrelated tokens be skipped; the summary of "Full Attention Strikes Back"
+// calls this 16-dim indexer a cheap scout.  Here:
+//   c_b    = (1/B) sum_{j in block b} P^T k_j
+//   qbar_t = sum_{h in group} (1/B) sum_{i in block t} P^T q_{h,i}
+// By linearity both equal P^T applied to a plain sum, so the kernel sums the
+// raw 128-dim rows (fp32) and projects once per block: the work is one pass
+// over K and the group's Q, i.e. HBM-bound.
+//
+// One CTA per (block, retrieval slot, sequence), 256 threads.  Each thread
+// reads 16 bytes (8 bf16) per row; 16 threads cover a row, so a warp reads two
+// full 256-byte rows per instruction (coalesced).  The 16 row-groups' partial
+// sums are reduced through shared memory in a fixed order, so results are
+// bit-reproducible.
+
+#include <cuda_bf16.h>
+
+#include "internal.cuh"
+
+namespace rtp {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kRowGroups = kThreads / 16;  // rows read per pass
+
+__device__ __forceinline__ void accum_row8(float (&acc)[8], const uint4 v) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    float2 f = __bfloat1622float2(h[e]);
+    acc[2 * e] += f.x;
+    acc[2 * e + 1] += f.y;
+  }
+}
+
+// Sum `rows` consecutive 128-wide bf16 rows starting at `base` into acc
+// (this thread's 8 columns), 4 loads in flight per thread.
+__device__ __forceinline__ void sum_rows(float (&acc)[8], const __nv_bfloat16* base, int rows, int rg, int cg) {
+  const uint4* p = reinterpret_cast<const uint4*>(base) + cg;
+  int r = rg;
+  for (; r + 3 * kRowGroups < rows; r += 4 * kRowGroups) {
+    uint4 v0 = __ldg(p + static_cast<size_t>(r) * 16);
+    uint4 v1 = __ldg(p + static_cast<size_t>(r + kRowGroups) * 16);
+    uint4 v2 = __ldg(p + static_cast<size_t>(r + 2 * kRowGroups) * 16);
+    uint4 v3 = __ldg(p + static_cast<size_t>(r + 3 * kRowGroups) * 16);
+    accum_row8(acc, v0);
+    accum_row8(acc, v1);
+    accum_row8(acc, v2);
+    accum_row8(acc, v3);
+  }
+  for (; r < rows; r += kRowGroups) accum_row8(acc, __ldg(p + static_cast<size_t>(r) * 16));
+}
+
+__global__ void __launch_bounds__(kThreads) indexer_kernel(const IndexerArgs a) {
+  __shared__ float part[2][kRowGroups][kHeadDim];
+  __shared__ float total[2][kHeadDim];
+  __shared__ float proj[kHeadDim * kRank];
+
+  const int blk = blockIdx.x, slot = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, rg = tid >> 4, cg = tid & 15;
+  const int kvh = a.slot_heads[slot];
+  const int B = a.block;
+
+  for (int e = tid; e < kHeadDim * kRank; e += kThreads) proj[e] = a.proj[e];
+
+  // keys of this block
+  float acck[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  const __nv_bfloat16* kbase =
+      a.k + ((static_cast<size_t>(b) * a.n_kv_heads + kvh) * a.seq + static_cast<size_t>(blk) * B) * kHeadDim;
+  sum_rows(acck, kbase, B, rg, cg);
+
+  // queries of this block, every head of the group (heads are consecutive)
+  float accq[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int h = 0; h < a.group; ++h) {
+    const int hq = kvh * a.group + h;
+    const __nv_bfloat16* qbase =
+        a.q + ((static_cast<size_t>(b) * a.n_q_heads + hq) * a.seq + static_cast<size_t>(blk) * B) * kHeadDim;
+    sum_rows(accq, qbase, B, rg, cg);
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    part[0][rg][cg * 8 + e] = acck[e];
+    part[1][rg][cg * 8 + e] = accq[e];
+  }
+  __syncthreads();
+  {
+    const int which = tid >> 7, col = tid & 127;  // 256 threads = 2 x 128 columns
+    float s = 0.f;
+#pragma unroll
+    for (int g = 0; g < kRowGroups; ++g) s += part[which][g][col];
+    total[which][col] = s;
+  }
+  __syncthreads();
+  if (tid < 2 * kRank) {
+    const int which = tid >> 4, c = tid & 15;
+    float s = 0.f;
+    for (int d = 0; d < kHeadDim; ++d) s = fmaf(proj[d * kRank + c], total[which][d], s);
+    s *= 1.0f / static_cast<float>(B);
+    const size_t o = ((static_cast<size_t>(b) * a.n_sparse + slot) * (a.seq / B) + blk) * kRank + c;
+    if (which == 0)
+      a.centroids[o] = s;
+    else
+      a.qbar[o] = s;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_indexer(const IndexerArgs& a, cudaStream_t stream) {
+  if (a.n_sparse == 0) return cudaSuccess;
+  dim3 grid(a.seq / a.block, a.n_sparse, a.batch);
+  indexer_kernel<<<grid, kThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace rtp

@@ -1,0 +1,77 @@
+// Internal interface between the C ABI layer (rtp_api.cu) and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace rtp {
+
+constexpr int kHeadDim = 128;
+constexpr int kRank = 16;
+
+enum : int { KIND_SWA = 0, KIND_FULL = 1, KIND_SPARSE = 2 };
+
+// One prefill work item: {kind | slot << 8, seq * n_kv_heads + kv_head,
+// query-head pair, 128-row query tile}.
+struct PrefillArgs {
+  const int4* items;
+  long n_items;
+  const int32_t* sel;  // [batch][n_sparse][nqb][kmax]
+  const int32_t* cnt;  // [batch][n_sparse][nqb]
+  __nv_bfloat16* o;    // [batch][n_q_heads][seq][128]
+  int batch, seq, n_q_heads, n_kv_heads, group, n_sparse;
+  int window, block, kmax, nqb;
+  float scale_log2;  // softmax scale * log2(e)
+  uint32_t* status;
+};
+
+struct IndexerArgs {
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  const float* proj;
+  float* centroids;  // [batch][n_sparse][nb][16]
+  float* qbar;       // [batch][n_sparse][nb][16]
+  const int32_t* slot_heads;  // device [n_sparse] -> kv head
+  int batch, seq, n_q_heads, n_kv_heads, group, n_sparse, block;
+};
+
+struct SelectArgs {
+  const float* qbar;
+  const float* centroids;
+  int32_t* sel;
+  int32_t* cnt;
+  int batch, n_sparse, nb, topk, n_local, kmax;
+};
+
+constexpr int kMaxDecodeKvHeads = 256;
+
+struct DecodeArgs {
+  const __nv_bfloat16* q;       // [batch][n_q_heads][128]
+  const __nv_bfloat16* kcache;  // [batch][n_kv_heads][cache_len][128]
+  const __nv_bfloat16* vcache;
+  const float* centroids;       // [batch][n_kv_heads][nbc][16]
+  const float* proj;
+  __nv_bfloat16* o;             // [batch][n_q_heads][128]
+  uint8_t kind[kMaxDecodeKvHeads];  // routing map, passed by value
+  int32_t* sel;                 // [batch][n_kv_heads][kmax] (workspace or caller)
+  int32_t* cnt;                 // [batch][n_kv_heads]
+  float* partial;               // [batch][n_kv_heads][max_splits][group][kPartStride]
+  int batch, n_q_heads, n_kv_heads, group, cache_len, nbc;
+  int window, block, topk, n_local, kmax, max_splits;
+  float scale_log2;
+  uint32_t* status;
+};
+constexpr int kPartStride = 132;  // m, l, pad, pad, o[128]
+
+// Launchers (return the launch error, never synchronise).
+cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                           int num_ctas, cudaStream_t stream);
+cudaError_t launch_indexer(const IndexerArgs& a, cudaStream_t stream);
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+
+// Shared-memory bytes the prefill kernel needs (host side, for the opt-in).
+size_t prefill_smem_bytes();
+
+}  // namespace rtp

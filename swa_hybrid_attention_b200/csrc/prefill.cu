@@ -1,0 +1,544 @@
+// Hybrid prefill attention (SWA / full causal / block-sparse heads) on the
+// sm_100a tensor cores.
+//
+// What it computes: for query head h (KV head h / group) and query i,
+//   O_i = softmax_j(scale * q_i . k_j) V   over the keys visible to the head:
+//   SWA i-W < j <= i, full j <= i, sparse j <= i with block(j) selected for
+//   i's query block.  (Pages: "阿里Qwen3 RTPurbo：15%全量Attention长文本5倍压缩方案"
+//   — streaming heads drop far tokens, long-range heads keep full attention;
+//   "阿里RTPurboV2：Transformer再次崛起，百步训练实现10倍稀少把稳" and the summary
+//   of "Full Attention Strikes Back" — exact attention on the selected set.)
+//
+// Design (B200-first; the pages describe a Hopper kernel, not reused here):
+//  * Persistent grid, one CTA per SM.  The work list (built on the host,
+//    heaviest tiles first — the RTPurbo page's "sparsity-aware scheduling")
+//    holds (KV head, pair of query heads of its group, 128-row query tile);
+//    CTA c takes items c, c+grid, ...
+//  * Both query heads of a pair visit the same KV tiles (same window, same
+//    selection: the selection is shared by the group), so every K/V tile
+//    loaded into shared memory feeds two S = Q K^T and two O += P V MMAs.
+//    The four pairs of a group run on neighbouring CTAs at the same time,
+//    so K/V are re-read from L2, not HBM.
+//  * Warp roles: warp 0 = TMA producer (Q tiles, then a 2-stage K/V ring),
+//    warp 1 = single-thread tcgen05.mma issuer, warp 2 = TMEM allocator,
+//    warps 4-7 / 8-11 = softmax for head 0 / head 1 of the pair (one thread
+//    per query row, the whole S row in registers: no cross-thread reduction).
+//  * TMEM (512 columns): S0 | S1 | O0 | O1, 128 fp32 columns each.  P (bf16)
+//    is written back over the first 64 columns of its S and fed to the PV
+//    MMA straight from TMEM (A operand in tensor memory).
+//  * Online softmax in the log2 domain with a lazy reference maximum: O is
+//    rescaled only when the row maximum grows by more than 2^8, so most
+//    tiles never touch O from the CUDA cores.
+//  * Masks are evaluated only on edge tiles (diagonal, window edge, sparse
+//    diagonal); interior tiles run mask-free.
+//  * Block size 64 (sparse heads): a 128-row query tile spans two query
+//    blocks with different selections; the tile's KV list is the union of
+//    both, loaded in 64-row halves, with a per-half membership mask.
+//  * Every mbarrier wait is bounded; a time-out sets the device status word
+//    and the CTA drains its in-flight copies/MMAs, frees TMEM and exits.
+
+#include <cuda_bf16.h>
+
+#include <climits>
+#include <cstdint>
+
+#include "internal.cuh"
+#include "sm100.cuh"
+
+namespace rtp {
+namespace {
+
+constexpr int kThreads = 384;
+constexpr int kStages = 2;
+constexpr uint32_t kTileBytes = 128 * 128 * 2;  // one 128x128 bf16 operand tile
+constexpr uint32_t kChunkBytes = 128 * 128;     // 64 columns x 128 rows
+constexpr int kNoWindow = 1 << 30;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows > 2^8
+constexpr uint32_t kMemberAll = 0x1Eu;
+
+struct __align__(1024) Smem {
+  uint8_t q[2][kTileBytes];
+  uint8_t k[kStages][kTileBytes];
+  uint8_t v[kStages][kTileBytes];
+  uint64_t q_full[2], q_empty[2];
+  uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+  uint64_t s_full[2], p_full[2], o_full[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct Item {
+  int kind, slot, b, kvh, bkv, pair, t;
+};
+
+__device__ __forceinline__ Item load_item(const int4* items, long idx, int n_kv_heads) {
+  int4 w = items[idx];
+  Item it;
+  it.kind = w.x & 0xFF;
+  it.slot = w.x >> 8;
+  it.bkv = w.y;
+  it.b = w.y / n_kv_heads;
+  it.kvh = w.y - it.b * n_kv_heads;
+  it.pair = w.z;
+  it.t = w.w;
+  return it;
+}
+
+// A KV tile: two 64-key halves starting at key positions row0 and row1.
+// flags bit 0: the tile needs the element mask.  Bits 1..4: membership of
+// (half 0, query half 0), (half 0, query half 1), (half 1, query half 0),
+// (half 1, query half 1) — only block-64 sparse tiles clear any of them.
+struct TileRef {
+  int row0, row1;
+  uint32_t flags;
+};
+
+// Enumerates the KV tiles of one work item in ascending key order.  The
+// producer, the MMA issuer and the softmax warps each run their own copy.
+struct TileIter {
+  int kind, t, n, lo, q0, window, j;
+  const int32_t* la;
+  const int32_t* lb;
+  int na, nb, ia, ib;
+  int nblocks;  // valid block indices are < nblocks
+  bool b64;
+  uint32_t* status;
+
+  __device__ void init(const Item& it, const PrefillArgs& a) {
+    kind = it.kind;
+    t = it.t;
+    j = 0;
+    q0 = 128 * t;
+    window = (kind == KIND_SWA) ? a.window : kNoWindow;
+    b64 = false;
+    status = a.status;
+    nblocks = a.nqb;
+    if (kind == KIND_FULL) {
+      lo = 0;
+      n = t + 1;
+    } else if (kind == KIND_SWA) {
+      int first = q0 - a.window + 1;
+      lo = first <= 0 ? 0 : first / 128;
+      n = t - lo + 1;
+    } else if (a.block == 128) {
+      long base = (static_cast<long>(it.b) * a.n_sparse + it.slot) * a.nqb + t;
+      la = a.sel + base * a.kmax;
+      na = min(max(a.cnt[base], 0), a.kmax);
+      n = na;
+    } else {
+      b64 = true;
+      long base = (static_cast<long>(it.b) * a.n_sparse + it.slot) * a.nqb + 2 * t;
+      la = a.sel + base * a.kmax;
+      na = min(max(a.cnt[base], 0), a.kmax);
+      if (2 * t + 1 < a.nqb) {
+        lb = la + a.kmax;
+        nb = min(max(a.cnt[base + 1], 0), a.kmax);
+      } else {
+        lb = la;
+        nb = 0;
+      }
+      // size of the union of the two ascending lists
+      int x = 0, y = 0, u = 0;
+      while (x < na || y < nb) {
+        int va = x < na ? la[x] : INT_MAX, vb = y < nb ? lb[y] : INT_MAX;
+        if (va <= vb) ++x;
+        if (vb <= va) ++y;
+        ++u;
+      }
+      n = (u + 1) / 2;
+      ia = ib = 0;
+    }
+    if (n < 1) {
+      // An empty selection cannot come from the selection kernel (the
+      // diagonal block is always kept); treat it as the diagonal tile only.
+      flag_error(status, RTP_DEVERR_INDEX);
+      kind = KIND_FULL;
+      window = kNoWindow;
+      lo = t;
+      n = 1;
+    }
+  }
+
+  __device__ int checked_block(int blk, int limit) {
+    if (blk < 0 || blk > limit) {
+      flag_error(status, RTP_DEVERR_INDEX);
+      return 0;
+    }
+    return blk;
+  }
+
+  // Next union entry (block-64 mode): value and membership (1 = A, 2 = B).
+  __device__ bool pick(int& v, uint32_t& mem) {
+    int va = ia < na ? la[ia] : INT_MAX, vb = ib < nb ? lb[ib] : INT_MAX;
+    if (va == INT_MAX && vb == INT_MAX) return false;
+    v = min(va, vb);
+    mem = (va == v ? 1u : 0u) | (vb == v ? 2u : 0u);
+    if (va == v) ++ia;
+    if (vb == v) ++ib;
+    return true;
+  }
+
+  __device__ TileRef next() {
+    TileRef r;
+    if (kind == KIND_FULL || kind == KIND_SWA) {
+      int k0 = 128 * (lo + j);
+      r.row0 = k0;
+      r.row1 = k0 + 64;
+      bool full_visible = (k0 + 127 <= q0) && (k0 > q0 + 127 - window);
+      r.flags = kMemberAll | (full_visible ? 0u : 1u);
+    } else if (!b64) {
+      int blk = checked_block(la[j], t);
+      r.row0 = 128 * blk;
+      r.row1 = r.row0 + 64;
+      r.flags = kMemberAll | (blk >= t ? 1u : 0u);
+    } else {
+      int v0 = 0, v1 = 0;
+      uint32_t m0 = 0, m1 = 0;
+      pick(v0, m0);
+      if (!pick(v1, m1)) {
+        v1 = v0;
+        m1 = 0;
+      }
+      v0 = checked_block(v0, 2 * t + 1);
+      v1 = checked_block(v1, 2 * t + 1);
+      r.row0 = 64 * v0;
+      r.row1 = 64 * v1;
+      r.flags = 1u | ((m0 & 1u) << 1) | ((m0 & 2u) << 1) | ((m1 & 1u) << 3) | ((m1 & 2u) << 3);
+    }
+    ++j;
+    return r;
+  }
+};
+
+// Bounded wait that ignores the abort flag (used while draining).
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
+  return mbar_wait(bar, parity, nullptr, status);
+}
+
+// One lane polls, the whole warp gets the (uniform) result.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* status) {
+  int ok = 1;
+  if (lane_id() == 0) ok = mbar_wait(bar, parity, abort, status) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  __syncwarp();
+  return ok != 0;
+}
+
+// ------------------------------------------------------------------ producer
+__device__ void run_producer(Smem& s, const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv,
+                             const PrefillArgs& a, volatile int* abort) {
+  uint32_t it = 0, gt = 0;
+  uint32_t q_issued = 0;  // bit h: Q of head h issued for the current item
+  for (long idx = blockIdx.x; idx < a.n_items; idx += gridDim.x, ++it) {
+    Item item = load_item(a.items, idx, a.n_kv_heads);
+    const int zq = item.b * a.n_q_heads + item.kvh * a.group + 2 * item.pair;
+    q_issued = 0;
+    for (int h = 0; h < 2; ++h) {
+      if (!mbar_wait(&s.q_empty[h], (it & 1u) ^ 1u, abort, a.status)) goto drain;
+      mbar_arrive_expect_tx(&s.q_full[h], kTileBytes);
+      tma_load_3d(s.q[h], mq, &s.q_full[h], 0, 128 * item.t, zq + h);
+      tma_load_3d(s.q[h] + kChunkBytes, mq, &s.q_full[h], 64, 128 * item.t, zq + h);
+      q_issued |= 1u << h;
+    }
+    {
+      TileIter ti;
+      ti.init(item, a);
+      for (int j = 0; j < ti.n; ++j, ++gt) {
+        TileRef tr = ti.next();
+        const int st = gt & 1;
+        const uint32_t use = gt >> 1;
+        if (!mbar_wait(&s.kv_empty[st], (use & 1u) ^ 1u, abort, a.status)) goto drain;
+        mbar_arrive_expect_tx(&s.k_full[st], kTileBytes);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(s.k[st] + c * kChunkBytes, mk, &s.k_full[st], 64 * c, tr.row0, item.bkv);
+          tma_load_3d(s.k[st] + c * kChunkBytes + kChunkBytes / 2, mk, &s.k_full[st], 64 * c, tr.row1, item.bkv);
+        }
+        mbar_arrive_expect_tx(&s.v_full[st], kTileBytes);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_3d(s.v[st] + c * kChunkBytes, mv, &s.v_full[st], 64 * c, tr.row0, item.bkv);
+          tma_load_3d(s.v[st] + c * kChunkBytes + kChunkBytes / 2, mv, &s.v_full[st], 64 * c, tr.row1, item.bkv);
+        }
+      }
+    }
+  }
+  return;
+drain:
+  // Give up: wait (bounded) for the copies already issued so that no TMA
+  // write lands in shared memory after the CTA has exited.
+  for (uint32_t x = 0; x < 2 && x < gt; ++x) {
+    uint32_t g = gt - 1 - x;
+    drain_wait(&s.k_full[g & 1], (g >> 1) & 1u, a.status);
+    drain_wait(&s.v_full[g & 1], (g >> 1) & 1u, a.status);
+  }
+  for (int h = 0; h < 2; ++h)
+    if (q_issued & (1u << h)) drain_wait(&s.q_full[h], it & 1u, a.status);
+}
+
+// ---------------------------------------------------------------- MMA issue
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem, uint32_t idesc) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
+    umma_ss(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024), smem_desc_sw128(k_smem + off, 16, 1024), idesc,
+            kk > 0 ? 1u : 0u);
+  }
+}
+
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, uint32_t idesc,
+                                         bool accumulate) {
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    umma_ts(d_tmem, p_tmem + kk * 8, smem_desc_sw128(v_smem + kk * 2048, kChunkBytes, 1024), idesc,
+            (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+__device__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& a, volatile int* abort) {
+  const uint32_t id_qk = idesc_bf16_f32(128, 128, false);
+  const uint32_t id_pv = idesc_bf16_f32(128, 128, true);
+  const uint32_t tS[2] = {tmem, tmem + 128};
+  const uint32_t tO[2] = {tmem + 256, tmem + 384};
+  const uint32_t sq[2] = {smem_u32(s.q[0]), smem_u32(s.q[1])};
+  uint32_t it = 0, gt = 0, pc = 0;
+  for (long idx = blockIdx.x; idx < a.n_items; idx += gridDim.x, ++it) {
+    Item item = load_item(a.items, idx, a.n_kv_heads);
+    TileIter ti;
+    ti.init(item, a);
+    const int n = ti.n;
+    if (!mbar_wait(&s.q_full[0], it & 1u, abort, a.status)) goto drain;
+    if (!mbar_wait(&s.q_full[1], it & 1u, abort, a.status)) goto drain;
+    {
+      const int st0 = gt & 1;
+      if (!mbar_wait(&s.k_full[st0], (gt >> 1) & 1u, abort, a.status)) goto drain;
+      tc_fence_after();
+      const uint32_t sk = smem_u32(s.k[st0]);
+      issue_qk(tS[0], sq[0], sk, id_qk);
+      umma_commit(&s.s_full[0]);
+      issue_qk(tS[1], sq[1], sk, id_qk);
+      umma_commit(&s.s_full[1]);
+      if (n == 1) {
+        umma_commit(&s.q_empty[0]);
+        umma_commit(&s.q_empty[1]);
+      }
+    }
+    for (int j = 0; j < n; ++j) {
+      const uint32_t g = gt + j;
+      const int st = g & 1;
+      const bool has_next = j + 1 < n;
+      const int st2 = (g + 1) & 1;
+      const uint32_t sv = smem_u32(s.v[st]);
+      const uint32_t sk2 = smem_u32(s.k[st2]);
+      if (!mbar_wait(&s.v_full[st], (g >> 1) & 1u, abort, a.status)) goto drain;
+      // head 0: O0 += P0 V ; then S0 for the next tile
+      if (!mbar_wait(&s.p_full[0], pc & 1u, abort, a.status)) goto drain;
+      tc_fence_after();
+      issue_pv(tO[0], tS[0], sv, id_pv, j > 0);
+      if (!has_next) {
+        umma_commit(&s.o_full[0]);
+      } else {
+        if (!mbar_wait(&s.k_full[st2], ((g + 1) >> 1) & 1u, abort, a.status)) goto drain;
+        tc_fence_after();
+        issue_qk(tS[0], sq[0], sk2, id_qk);
+        umma_commit(&s.s_full[0]);
+        if (j + 2 == n) umma_commit(&s.q_empty[0]);
+      }
+      // head 1
+      if (!mbar_wait(&s.p_full[1], pc & 1u, abort, a.status)) goto drain;
+      tc_fence_after();
+      issue_pv(tO[1], tS[1], sv, id_pv, j > 0);
+      umma_commit(&s.kv_empty[st]);
+      if (!has_next) {
+        umma_commit(&s.o_full[1]);
+      } else {
+        issue_qk(tS[1], sq[1], sk2, id_qk);
+        umma_commit(&s.s_full[1]);
+        if (j + 2 == n) umma_commit(&s.q_empty[1]);
+      }
+      ++pc;
+    }
+    gt += n;
+  }
+drain:
+  // All MMAs issued by this thread must finish before TMEM is released.
+  umma_commit(&s.drain);
+  drain_wait(&s.drain, 0, a.status);
+}
+
+// ------------------------------------------------------------------ softmax
+__device__ void run_softmax(Smem& s, uint32_t tmem, int h, const PrefillArgs& a, volatile int* abort) {
+  const int q4 = warp_id() & 3;
+  const int row = q4 * 32 + lane_id();
+  const uint32_t lane_bits = static_cast<uint32_t>(q4 * 32) << 16;
+  const uint32_t tS = tmem + 128 * h + lane_bits;
+  const uint32_t tO = tmem + 256 + 128 * h + lane_bits;
+  const float sl2 = a.scale_log2;
+  uint32_t it = 0, sc = 0;
+  for (long idx = blockIdx.x; idx < a.n_items; idx += gridDim.x, ++it) {
+    Item item = load_item(a.items, idx, a.n_kv_heads);
+    TileIter ti;
+    ti.init(item, a);
+    const int i = 128 * item.t + row;
+    const int rh = row >> 6;
+    float m_ref = -INFINITY, l = 0.f;
+    for (int j = 0; j < ti.n; ++j) {
+      const TileRef tr = ti.next();
+      if (!warp_wait(&s.s_full[h], sc & 1u, abort, a.status)) return;
+      ++sc;
+      tc_fence_after();
+      uint32_t r[128];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+      tmem_ld_wait();
+      if (tr.flags & 1u) {
+        const int lo_key = i - ti.window;  // visible iff lo_key < key <= i
+#pragma unroll
+        for (int c = 0; c < 128; ++c) {
+          const int half = c >> 6;
+          const int key = (half ? tr.row1 : tr.row0) + (c & 63);
+          const bool member = (tr.flags >> (1 + 2 * half + rh)) & 1u;
+          if (!(member && key <= i && key > lo_key)) r[c] = __float_as_uint(-INFINITY);
+        }
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(r[c]));
+      const float m_new = mx * sl2;
+      if (m_new > m_ref + kRescaleThreshold) {
+        if (j > 0 && m_ref != -INFINITY) {
+          const float alpha = exp2f(m_ref - m_new);
+          l *= alpha;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + 32 * c, o);
+          }
+        }
+        m_ref = m_new;
+      }
+      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      // P = exp2(s * scale*log2e - m) as packed bf16 pairs, written over the
+      // first 64 columns of S (the whole S row is already in registers).
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t p[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = exp2f(fmaf(__uint_as_float(r[32 * c + 2 * e]), sl2, -m_use));
+          const float p1 = exp2f(fmaf(__uint_as_float(r[32 * c + 2 * e + 1]), sl2, -m_use));
+          sum += p0 + p1;
+          p[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + 16 * c, p);
+      }
+      l += sum;
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&s.p_full[h]);
+    }
+    // epilogue: O / l -> bf16
+    if (!warp_wait(&s.o_full[h], it & 1u, abort, a.status)) return;
+    tc_fence_after();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    const int hq = item.kvh * a.group + 2 * item.pair + h;
+    __nv_bfloat16* orow =
+        a.o + ((static_cast<size_t>(item.b) * a.n_q_heads + hq) * static_cast<size_t>(a.seq) + i) * kHeadDim;
+    const bool valid = i < a.seq;
+#pragma unroll 1
+    for (int c = 0; c < 4; ++c) {
+      uint32_t o[32];
+      tmem_ld32(tO + 32 * c, o);
+      tmem_ld_wait();
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv, __uint_as_float(o[2 * e + 1]) * inv);
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+      }
+    }
+    tc_fence_before();
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    hybrid_prefill_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
+                          const __grid_constant__ CUtensorMap mv, const PrefillArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = warp_id();
+  if (threadIdx.x == 0) {
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&s.q_full[h], 1);
+      mbar_init(&s.q_empty[h], 1);
+      mbar_init(&s.s_full[h], 1);
+      mbar_init(&s.p_full[h], 128);
+      mbar_init(&s.o_full[h], 1);
+    }
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&s.k_full[st], 1);
+      mbar_init(&s.v_full[st], 1);
+      mbar_init(&s.kv_empty[st], 1);
+    }
+    mbar_init(&s.drain, 1);
+    s.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane_id() == 0) {
+    tma_prefetch_desc(&mq);
+    tma_prefetch_desc(&mk);
+    tma_prefetch_desc(&mv);
+  }
+  if (warp == 2) {
+    tmem_alloc(&s.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  volatile int* abort = &s.abort_flag;
+
+  if (warp == 0) {
+    if (lane_id() == 0) run_producer(s, &mq, &mk, &mv, a, abort);
+  } else if (warp == 1) {
+    if (lane_id() == 0) run_mma(s, tmem, a, abort);
+  } else if (warp >= 4) {
+    run_softmax(s, tmem, (warp - 4) >> 2, a, abort);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+size_t prefill_smem_bytes() { return sizeof(Smem) + 1024; }
+
+cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                           int num_ctas, cudaStream_t stream) {
+  static int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    cudaError_t e = cudaFuncSetAttribute(hybrid_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(prefill_smem_bytes()));
+    if (e != cudaSuccess) return e;
+    configured_device = dev;
+  }
+  hybrid_prefill_kernel<<<num_ctas, kThreads, prefill_smem_bytes(), stream>>>(mq, mk, mv, a);
+  return cudaGetLastError();
+}
+
+}  // namespace rtp

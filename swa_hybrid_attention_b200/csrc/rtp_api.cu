@@ -1,0 +1,457 @@
+// C ABI of librtp.so (declared in include/rtp.h): argument validation, the
+// routing planner, TMA descriptor set-up and kernel dispatch.  No C++
+// exception crosses the boundary; every entry point returns an rtp_status.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "../../include/rtp.h"
+#include "internal.cuh"
+#include "sm100.cuh"
+
+using namespace rtp;
+
+struct rtp_plan {
+  rtp_attn_cfg cfg;
+  int device = 0;
+  int num_sms = 148;
+  int n_sparse = 0;
+  int nqt = 0;  // 128-row query tiles
+  int nqb = 0;  // query blocks of `block` rows
+  std::vector<uint8_t> kind;
+  std::vector<int32_t> slot_heads;
+  std::vector<int32_t> items_host;  // [n_items][4]
+  long n_items = 0;
+  void* d_mem = nullptr;
+  int4* d_items = nullptr;
+  int32_t* d_slot_heads = nullptr;
+  float scale = 0.f;
+};
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------- status word
+std::mutex g_status_mu;
+uint32_t* g_status[64] = {nullptr};
+
+uint32_t* status_word(int dev) {
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  if (!g_status[dev]) {
+    uint32_t* p = nullptr;
+    if (cudaMalloc(&p, sizeof(uint32_t)) != cudaSuccess) return nullptr;
+    if (cudaMemset(p, 0, sizeof(uint32_t)) != cudaSuccess) {
+      cudaFree(p);
+      return nullptr;
+    }
+    g_status[dev] = p;
+  }
+  return g_status[dev];
+}
+
+// ------------------------------------------------------------- TMA encoding
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 [slabs][rows][128] viewed as a 3-D tensor, 128-byte swizzled boxes of
+// 64 columns x box_rows rows.  Rows past `rows` read as zero.
+bool encode_bf16_3d(CUtensorMap* map, const void* base, long rows, long slabs, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(slabs)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim) * 2,
+                           static_cast<cuuint64_t>(kHeadDim) * 2 * static_cast<cuuint64_t>(rows)};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- validation
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool cfg_common_ok(const rtp_attn_cfg* c) {
+  if (!c) return false;
+  if (c->batch < 1 || c->n_q_heads < 1 || c->n_kv_heads < 1) return false;
+  if (c->head_dim != kHeadDim || c->rank != kRank || c->n_sink != 1) return false;
+  if (c->n_q_heads % c->n_kv_heads != 0) return false;
+  const int g = c->n_q_heads / c->n_kv_heads;
+  if (g > 16) return false;
+  if (c->window < 1 || c->n_local < 1 || c->topk < 0) return false;
+  if (c->block != 64 && c->block != 128) return false;
+  if (!(c->scale >= 0.f) || !std::isfinite(c->scale)) return false;
+  if (static_cast<long>(c->batch) * c->n_q_heads > (1L << 24)) return false;
+  return true;
+}
+
+bool cfg_prefill_ok(const rtp_attn_cfg* c) {
+  if (!cfg_common_ok(c)) return false;
+  if ((c->n_q_heads / c->n_kv_heads) % 2 != 0) return false;
+  if (c->seq < 1 || c->seq % c->block != 0) return false;
+  if (c->seq > (1 << 30) / 2) return false;
+  const long nb = c->seq / c->block;
+  if (nb * 4 > 200 * 1024) return false;  // selection keys live in shared memory
+  return true;
+}
+
+float effective_scale(const rtp_attn_cfg* c) {
+  return c->scale > 0.f ? c->scale : 1.0f / std::sqrt(static_cast<float>(c->head_dim));
+}
+
+// Selected-list length for a query block t with at least... (see rtp.h):
+// all blocks 0..t when there are at most topk candidates, else sink + topk +
+// local.
+long selected_count(long t, int topk, int n_local) {
+  long ncand = std::max<long>(0, t - n_local);
+  return ncand > topk ? 1L + topk + n_local : t + 1;
+}
+
+rtp_status cuda_status(cudaError_t e) { return e == cudaSuccess ? RTP_OK : RTP_ERR_CUDA; }
+
+int current_device() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return d;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rtp_status_str(rtp_status s) {
+  switch (s) {
+    case RTP_OK: return "RTP_OK";
+    case RTP_ERR_INVALID_ARG: return "RTP_ERR_INVALID_ARG";
+    case RTP_ERR_UNSUPPORTED: return "RTP_ERR_UNSUPPORTED";
+    case RTP_ERR_CUDA: return "RTP_ERR_CUDA";
+    case RTP_ERR_TIMEOUT: return "RTP_ERR_TIMEOUT";
+    case RTP_ERR_NO_MEMORY: return "RTP_ERR_NO_MEMORY";
+  }
+  return "RTP_ERR_UNKNOWN";
+}
+
+int rtp_version(void) { return (1 << 16) | 0; }
+
+rtp_status rtp_route_heads(const rtp_attn_cfg* cfg, const uint8_t* kind_host, void* stream, rtp_plan** out) {
+  if (!out) return RTP_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg_prefill_ok(cfg) || !kind_host) return RTP_ERR_INVALID_ARG;
+  for (int h = 0; h < cfg->n_kv_heads; ++h)
+    if (kind_host[h] > RTP_HEAD_SPARSE) return RTP_ERR_INVALID_ARG;
+
+  rtp_plan* p = new (std::nothrow) rtp_plan();
+  if (!p) return RTP_ERR_NO_MEMORY;
+  p->cfg = *cfg;
+  p->scale = effective_scale(cfg);
+  p->device = current_device();
+  cudaDeviceGetAttribute(&p->num_sms, cudaDevAttrMultiProcessorCount, p->device);
+  p->kind.assign(kind_host, kind_host + cfg->n_kv_heads);
+  std::vector<int> slot_of(cfg->n_kv_heads, -1);
+  for (int h = 0; h < cfg->n_kv_heads; ++h)
+    if (kind_host[h] == RTP_HEAD_SPARSE) {
+      slot_of[h] = static_cast<int>(p->slot_heads.size());
+      p->slot_heads.push_back(h);
+    }
+  p->n_sparse = static_cast<int>(p->slot_heads.size());
+  p->nqt = (cfg->seq + 127) / 128;
+  p->nqb = cfg->seq / cfg->block;
+  const int group = cfg->n_q_heads / cfg->n_kv_heads;
+  const int pairs = group / 2;
+
+  // Work items with their cost (KV tiles visited), then longest first.
+  struct W {
+    long cost;
+    int32_t v[4];
+  };
+  std::vector<W> work;
+  work.reserve(static_cast<size_t>(cfg->batch) * cfg->n_kv_heads * pairs * p->nqt);
+  for (int b = 0; b < cfg->batch; ++b)
+    for (int h = 0; h < cfg->n_kv_heads; ++h)
+      for (int t = 0; t < p->nqt; ++t) {
+        long cost;
+        const int kind = kind_host[h];
+        if (kind == RTP_HEAD_FULL) {
+          cost = t + 1;
+        } else if (kind == RTP_HEAD_SWA) {
+          long first = 128L * t - cfg->window + 1;
+          long lo = first <= 0 ? 0 : first / 128;
+          cost = t - lo + 1;
+        } else if (cfg->block == 128) {
+          cost = selected_count(t, cfg->topk, cfg->n_local);
+        } else {
+          long c0 = selected_count(2L * t, cfg->topk, cfg->n_local);
+          long c1 = 2L * t + 1 < p->nqb ? selected_count(2L * t + 1, cfg->topk, cfg->n_local) : 0;
+          cost = (c0 + c1 + 1) / 2;
+        }
+        const int slot = kind == RTP_HEAD_SPARSE ? slot_of[h] : 0;
+        for (int pr = 0; pr < pairs; ++pr)
+          work.push_back(W{cost, {kind | (slot << 8), b * cfg->n_kv_heads + h, pr, t}});
+      }
+  std::stable_sort(work.begin(), work.end(), [](const W& a, const W& b) { return a.cost > b.cost; });
+  p->n_items = static_cast<long>(work.size());
+  p->items_host.resize(work.size() * 4);
+  for (size_t i = 0; i < work.size(); ++i) std::memcpy(&p->items_host[i * 4], work[i].v, sizeof(work[i].v));
+
+  const size_t items_bytes = work.size() * sizeof(int4);
+  const size_t slots_bytes = std::max<size_t>(1, p->slot_heads.size()) * sizeof(int32_t);
+  if (cudaMalloc(&p->d_mem, items_bytes + 256 + slots_bytes) != cudaSuccess) {
+    delete p;
+    return RTP_ERR_NO_MEMORY;
+  }
+  p->d_items = reinterpret_cast<int4*>(p->d_mem);
+  p->d_slot_heads = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(p->d_mem) + ((items_bytes + 255) / 256) * 256);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(p->d_items, p->items_host.data(), items_bytes, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && !p->slot_heads.empty())
+    e = cudaMemcpyAsync(p->d_slot_heads, p->slot_heads.data(), p->slot_heads.size() * sizeof(int32_t),
+                        cudaMemcpyHostToDevice, s);
+  // The host arrays stay alive with the plan; make sure the upload finished
+  // before the call returns so that a caller may use the plan on any stream.
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) {
+    cudaFree(p->d_mem);
+    delete p;
+    return RTP_ERR_CUDA;
+  }
+  if (!status_word(p->device)) {
+    cudaFree(p->d_mem);
+    delete p;
+    return RTP_ERR_NO_MEMORY;
+  }
+  *out = p;
+  return RTP_OK;
+}
+
+void rtp_plan_destroy(rtp_plan* plan) {
+  if (!plan) return;
+  if (plan->d_mem) cudaFree(plan->d_mem);
+  delete plan;
+}
+
+int rtp_plan_num_sparse(const rtp_plan* plan) { return plan ? plan->n_sparse : -1; }
+
+long rtp_plan_num_items(const rtp_plan* plan) { return plan ? plan->n_items : -1; }
+
+rtp_status rtp_plan_sparse_heads(const rtp_plan* plan, int32_t* slots_host) {
+  if (!plan || (!slots_host && plan->n_sparse > 0)) return RTP_ERR_INVALID_ARG;
+  if (plan->n_sparse > 0) std::memcpy(slots_host, plan->slot_heads.data(), plan->slot_heads.size() * sizeof(int32_t));
+  return RTP_OK;
+}
+
+rtp_status rtp_plan_work_items(const rtp_plan* plan, int32_t* items_host) {
+  if (!plan || !items_host) return RTP_ERR_INVALID_ARG;
+  std::memcpy(items_host, plan->items_host.data(), plan->items_host.size() * sizeof(int32_t));
+  return RTP_OK;
+}
+
+rtp_status rtp_indexer_project(const rtp_plan* plan, const void* q, const void* k, const float* proj,
+                               float* centroids, float* qbar, void* stream) {
+  if (!plan) return RTP_ERR_INVALID_ARG;
+  if (plan->n_sparse == 0) return RTP_OK;
+  if (!q || !k || !proj || !centroids || !qbar) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(proj) || !aligned16(centroids) || !aligned16(qbar))
+    return RTP_ERR_INVALID_ARG;
+  const rtp_attn_cfg& c = plan->cfg;
+  IndexerArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.proj = proj;
+  a.centroids = centroids;
+  a.qbar = qbar;
+  a.slot_heads = plan->d_slot_heads;
+  a.batch = c.batch;
+  a.seq = c.seq;
+  a.n_q_heads = c.n_q_heads;
+  a.n_kv_heads = c.n_kv_heads;
+  a.group = c.n_q_heads / c.n_kv_heads;
+  a.n_sparse = plan->n_sparse;
+  a.block = c.block;
+  return cuda_status(launch_indexer(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rtp_status rtp_block_select(const rtp_plan* plan, const float* qbar, const float* centroids, int32_t* sel,
+                            int32_t* sel_cnt, void* stream) {
+  if (!plan) return RTP_ERR_INVALID_ARG;
+  if (plan->n_sparse == 0) return RTP_OK;
+  if (!qbar || !centroids || !sel || !sel_cnt) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(qbar) || !aligned16(centroids) || !aligned16(sel) || !aligned16(sel_cnt))
+    return RTP_ERR_INVALID_ARG;
+  const rtp_attn_cfg& c = plan->cfg;
+  SelectArgs a;
+  a.qbar = qbar;
+  a.centroids = centroids;
+  a.sel = sel;
+  a.cnt = sel_cnt;
+  a.batch = c.batch;
+  a.n_sparse = plan->n_sparse;
+  a.nb = plan->nqb;
+  a.topk = c.topk;
+  a.n_local = c.n_local;
+  a.kmax = c.topk + 1 + c.n_local;
+  return cuda_status(launch_select(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rtp_status rtp_hybrid_prefill(const rtp_plan* plan, const void* q, const void* k, const void* v,
+                              const int32_t* sel, const int32_t* sel_cnt, void* o, void* stream) {
+  if (!plan || !q || !k || !v || !o) return RTP_ERR_INVALID_ARG;
+  if (plan->n_sparse > 0 && (!sel || !sel_cnt)) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RTP_ERR_INVALID_ARG;
+  if (sel && !aligned16(sel)) return RTP_ERR_INVALID_ARG;
+  const rtp_attn_cfg& c = plan->cfg;
+  if (current_device() != plan->device) return RTP_ERR_INVALID_ARG;
+  CUtensorMap mq, mk, mv;
+  if (!encode_bf16_3d(&mq, q, c.seq, static_cast<long>(c.batch) * c.n_q_heads, 128) ||
+      !encode_bf16_3d(&mk, k, c.seq, static_cast<long>(c.batch) * c.n_kv_heads, 64) ||
+      !encode_bf16_3d(&mv, v, c.seq, static_cast<long>(c.batch) * c.n_kv_heads, 64))
+    return RTP_ERR_CUDA;
+  PrefillArgs a;
+  a.items = plan->d_items;
+  a.n_items = plan->n_items;
+  a.sel = sel;
+  a.cnt = sel_cnt;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.batch = c.batch;
+  a.seq = c.seq;
+  a.n_q_heads = c.n_q_heads;
+  a.n_kv_heads = c.n_kv_heads;
+  a.group = c.n_q_heads / c.n_kv_heads;
+  a.n_sparse = plan->n_sparse;
+  a.window = c.window;
+  a.block = c.block;
+  a.kmax = c.topk + 1 + c.n_local;
+  a.nqb = plan->nqb;
+  a.scale_log2 = plan->scale * kLog2e;
+  a.status = status_word(plan->device);
+  const int ctas = static_cast<int>(std::min<long>(plan->n_items, plan->num_sms));
+  if (ctas <= 0) return RTP_OK;
+  return cuda_status(launch_prefill(a, mq, mk, mv, ctas, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// Decode workspace: sel [batch][n_kv][kmax] int32 | cnt [batch][n_kv] int32 |
+// partials [batch][n_kv][max_splits][group][132] fp32, each 256-byte aligned.
+namespace {
+struct DecodeLayout {
+  size_t sel_off, cnt_off, part_off, total;
+  int max_splits, kmax;
+};
+
+bool decode_layout(const rtp_attn_cfg* c, const uint8_t* kind, int cache_len, DecodeLayout& L) {
+  if (!cfg_common_ok(c) || !kind || cache_len < 1) return false;
+  if (static_cast<long>(cache_len) / c->block * 4 > 200 * 1024) return false;
+  L.kmax = c->topk + 1 + c->n_local;
+  int ms = 1;
+  for (int h = 0; h < c->n_kv_heads; ++h) {
+    if (kind[h] > RTP_HEAD_SPARSE) return false;
+    int s;
+    if (kind[h] == RTP_HEAD_SPARSE)
+      s = L.kmax;
+    else if (kind[h] == RTP_HEAD_SWA)
+      s = (std::min(cache_len, c->window) + 127) / 128;
+    else
+      s = (cache_len + 127) / 128;
+    ms = std::max(ms, s);
+  }
+  L.max_splits = ms;
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t bk = static_cast<size_t>(c->batch) * c->n_kv_heads;
+  const int group = c->n_q_heads / c->n_kv_heads;
+  L.sel_off = 0;
+  L.cnt_off = up(bk * L.kmax * sizeof(int32_t));
+  L.part_off = L.cnt_off + up(bk * sizeof(int32_t));
+  L.total = L.part_off + up(bk * ms * group * kPartStride * sizeof(float));
+  return true;
+}
+}  // namespace
+
+size_t rtp_decode_workspace_bytes(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len) {
+  DecodeLayout L;
+  if (!decode_layout(cfg, kind_host, cache_len, L)) return 0;
+  return L.total;
+}
+
+rtp_status rtp_sparse_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* q,
+                             const void* kcache, const void* vcache, const float* centroids, const float* proj,
+                             void* o, void* workspace, size_t ws_bytes, int32_t* sel_out, int32_t* cnt_out,
+                             void* stream) {
+  DecodeLayout L;
+  if (!decode_layout(cfg, kind_host, cache_len, L)) return RTP_ERR_INVALID_ARG;
+  if (!q || !kcache || !vcache || !o || !workspace || ws_bytes < L.total) return RTP_ERR_INVALID_ARG;
+  bool any_sparse = false;
+  for (int h = 0; h < cfg->n_kv_heads; ++h) any_sparse |= kind_host[h] == RTP_HEAD_SPARSE;
+  if (any_sparse && (!centroids || !proj)) return RTP_ERR_INVALID_ARG;
+  if ((sel_out == nullptr) != (cnt_out == nullptr)) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o) || !aligned16(workspace))
+    return RTP_ERR_INVALID_ARG;
+  if ((centroids && !aligned16(centroids)) || (proj && !aligned16(proj))) return RTP_ERR_INVALID_ARG;
+  if (cfg->n_kv_heads > kMaxDecodeKvHeads) return RTP_ERR_INVALID_ARG;
+  DecodeArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.kcache = static_cast<const __nv_bfloat16*>(kcache);
+  a.vcache = static_cast<const __nv_bfloat16*>(vcache);
+  a.centroids = centroids;
+  a.proj = proj;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  std::memset(a.kind, 0, sizeof(a.kind));
+  std::memcpy(a.kind, kind_host, cfg->n_kv_heads);
+  char* ws = static_cast<char*>(workspace);
+  a.sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(ws + L.sel_off);
+  a.cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(ws + L.cnt_off);
+  a.partial = reinterpret_cast<float*>(ws + L.part_off);
+  a.batch = cfg->batch;
+  a.n_q_heads = cfg->n_q_heads;
+  a.n_kv_heads = cfg->n_kv_heads;
+  a.group = cfg->n_q_heads / cfg->n_kv_heads;
+  a.cache_len = cache_len;
+  a.nbc = cache_len / cfg->block;
+  a.window = cfg->window;
+  a.block = cfg->block;
+  a.topk = cfg->topk;
+  a.n_local = cfg->n_local;
+  a.kmax = L.kmax;
+  a.max_splits = L.max_splits;
+  a.scale_log2 = effective_scale(cfg) * kLog2e;
+  a.status = status_word(current_device());
+  if (!a.status) return RTP_ERR_NO_MEMORY;
+  return cuda_status(launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rtp_status rtp_last_device_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return RTP_ERR_CUDA;
+  uint32_t* w = status_word(current_device());
+  if (!w) return RTP_ERR_NO_MEMORY;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, w, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return RTP_ERR_CUDA;
+  if (v != 0 && cudaMemset(w, 0, sizeof(uint32_t)) != cudaSuccess) return RTP_ERR_CUDA;
+  if (v & RTP_DEVERR_TIMEOUT) return RTP_ERR_TIMEOUT;
+  if (v) return RTP_ERR_INVALID_ARG;
+  return RTP_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,160 @@
+// Block selection shared by the prefill selection kernel and the decode
+// step: sink + top-k candidates by (score desc, index asc) + local blocks.
+#pragma once
+#include <cstdint>
+
+#include "internal.cuh"
+
+namespace rtp {
+
+constexpr int kSelThreads = 256;
+
+struct SelectScratch {
+  uint32_t hist[256];
+  unsigned long long warp_sums[kSelThreads / 32];
+  uint32_t digit, need;
+};
+
+// Order-preserving map float -> uint32 (larger float, larger key); -0 and +0
+// map to the same key.
+__device__ __forceinline__ uint32_t order_key(float s) {
+  const uint32_t u = __float_as_uint(s + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ unsigned long long block_exclusive_scan(unsigned long long v, SelectScratch& sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned long long incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    unsigned long long y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) sh.warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned long long w = lane < kSelThreads / 32 ? sh.warp_sums[lane] : 0ull;
+    unsigned long long wi = w;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      unsigned long long y = __shfl_up_sync(0xffffffffu, wi, off);
+      if (lane >= off) wi += y;
+    }
+    if (lane < kSelThreads / 32) sh.warp_sums[lane] = wi - w;  // exclusive
+  }
+  __syncthreads();
+  return sh.warp_sums[warp] + incl - v;
+}
+
+// Selects the blocks of query block t.  Must be called by all kSelThreads
+// threads of the CTA.  q: the query summary (16 fp32); C: centroids of this
+// (slot, sequence), [>= t-n_local+1][16] fp32; keys: shared scratch of at
+// least max(0, t-n_local) words.  Writes out[0..kmax) (ascending, -1 padded)
+// and returns the number of entries used.
+__device__ inline int select_blocks(const float (&q)[kRank], const float* C, int t, int topk, int n_local, int kmax,
+                                    uint32_t* keys, SelectScratch& sh, int32_t* out) {
+  const int tid = threadIdx.x;
+  const int ncand = t - n_local > 0 ? t - n_local : 0;  // candidates are blocks 1..ncand
+  if (ncand <= topk) {
+    const int n = t + 1;
+    for (int e = tid; e < kmax; e += kSelThreads) out[e] = e < n ? e : -1;
+    return n;
+  }
+  // 1. scores -> order keys (fixed fma order over the 16 ranks)
+  for (int x = tid; x < ncand; x += kSelThreads) {
+    const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + 1) * kRank);
+    const float4 a0 = __ldg(c4), a1 = __ldg(c4 + 1), a2 = __ldg(c4 + 2), a3 = __ldg(c4 + 3);
+    float s = q[0] * a0.x;
+    s = fmaf(q[1], a0.y, s);
+    s = fmaf(q[2], a0.z, s);
+    s = fmaf(q[3], a0.w, s);
+    s = fmaf(q[4], a1.x, s);
+    s = fmaf(q[5], a1.y, s);
+    s = fmaf(q[6], a1.z, s);
+    s = fmaf(q[7], a1.w, s);
+    s = fmaf(q[8], a2.x, s);
+    s = fmaf(q[9], a2.y, s);
+    s = fmaf(q[10], a2.z, s);
+    s = fmaf(q[11], a2.w, s);
+    s = fmaf(q[12], a3.x, s);
+    s = fmaf(q[13], a3.y, s);
+    s = fmaf(q[14], a3.z, s);
+    s = fmaf(q[15], a3.w, s);
+    keys[x] = order_key(s);
+  }
+  __syncthreads();
+
+  // 2. radix select of the topk-th largest key, most significant byte first
+  uint32_t prefix = 0, need = static_cast<uint32_t>(topk);
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
+    for (int e = tid; e < 256; e += kSelThreads) sh.hist[e] = 0;
+    __syncthreads();
+    for (int x = tid; x < ncand; x += kSelThreads) {
+      const uint32_t k = keys[x];
+      if ((k & hi_mask) == prefix) atomicAdd(&sh.hist[(k >> shift) & 255u], 1u);
+    }
+    __syncthreads();
+    if (tid < 32) {
+      uint32_t cnt8[8], own = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        cnt8[e] = sh.hist[8 * tid + e];
+        own += cnt8[e];
+      }
+      uint32_t incl = own;  // count in bins of lanes >= this lane
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        uint32_t y = __shfl_down_sync(0xffffffffu, incl, off);
+        if (tid + off < 32) incl += y;
+      }
+      const uint32_t above = incl - own;
+      if (above < need && need <= incl) {
+        uint32_t acc = above;
+        for (int e = 7; e >= 0; --e) {
+          if (acc + cnt8[e] >= need) {
+            sh.digit = static_cast<uint32_t>(8 * tid + e);
+            sh.need = need - acc;
+            break;
+          }
+          acc += cnt8[e];
+        }
+      }
+    }
+    __syncthreads();
+    prefix |= sh.digit << shift;
+    need = sh.need;
+    __syncthreads();
+  }
+  const uint32_t T = prefix;  // key of the topk-th largest; `need` keys equal to T are kept
+
+  // 3. ordered compaction: contiguous run per thread + block-wide scan
+  const int per = (ncand + kSelThreads - 1) / kSelThreads;
+  const int x0 = min(ncand, tid * per), x1 = min(ncand, x0 + per);
+  uint32_t n_gt = 0, n_eq = 0;
+  for (int x = x0; x < x1; ++x) {
+    const uint32_t k = keys[x];
+    n_gt += k > T;
+    n_eq += k == T;
+  }
+  const unsigned long long excl =
+      block_exclusive_scan((static_cast<unsigned long long>(n_gt) << 32) | n_eq, sh);
+  uint32_t gt_before = static_cast<uint32_t>(excl >> 32), eq_before = static_cast<uint32_t>(excl & 0xFFFFFFFFu);
+  for (int x = x0; x < x1; ++x) {
+    const uint32_t k = keys[x];
+    if (k > T) {
+      out[1 + gt_before + min(eq_before, need)] = x + 1;
+      ++gt_before;
+    } else if (k == T) {
+      if (eq_before < need) out[1 + gt_before + eq_before] = x + 1;
+      ++eq_before;
+    }
+  }
+  if (tid == 0) out[0] = 0;
+  for (int m = tid; m < n_local; m += kSelThreads) out[1 + topk + m] = t - n_local + 1 + m;
+  for (int e = 1 + topk + n_local + tid; e < kmax; e += kSelThreads) out[e] = -1;
+  return 1 + topk + n_local;
+}
+
+}  // namespace rtp

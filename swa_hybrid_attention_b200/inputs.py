@@ -95,7 +95,7 @@ def workload(wid: int) -> Workload:
     if wid == 0:
         return Workload(0, "tiny-v2-2k", 1, 2048, 8, 2, 1, 512, 64, 16, 2, "lowfreq", 0, [[SPARSE, SWA]])
     if wid == 1:
-        return Workload(1, "qwen3-30b-a3b-v1-32k", 1, 32768, 32, 4, 48, 8192, 128, 0, 0, "none", 0,
+        return Workload(1, "qwen3-30b-a3b-v1-32k", 1, 32768, 32, 4, 48, 8192, 128, 0, 1, "none", 0,
                         _layered_map(48, 4, 29, FULL))
     if wid == 2:
         return Workload(2, "qwen3-30b-a3b-v2-128k", 1, 131072, 32, 4, 48, 8192, 128, 64, 4, "random", 256,

@@ -1,0 +1,285 @@
+"""Thin ctypes binding of librtp.so (C ABI in include/rtp.h).
+
+The functions below carry the C names and only marshal arguments: torch
+tensors become device pointers, the current torch stream becomes the
+cudaStream_t, the config becomes an ``rtp_attn_cfg`` struct.  Every step of
+the attention path runs in the library's CUDA kernels; there is no fallback.
+If librtp.so is missing or fails to load, importing this module raises.
+
+``hybrid_prefill_layer`` and ``sparse_decode_step`` chain the calls of one
+layer / one decode step and allocate their intermediate buffers with torch
+(device memory is the only thing torch is used for here).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librtp.so")
+
+RTP_OK, RTP_ERR_INVALID_ARG, RTP_ERR_UNSUPPORTED, RTP_ERR_CUDA, RTP_ERR_TIMEOUT, RTP_ERR_NO_MEMORY = range(6)
+RTP_HEAD_SWA, RTP_HEAD_FULL, RTP_HEAD_SPARSE = 0, 1, 2
+
+
+class RtpError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {status_str(status)} ({status})")
+        self.status = status
+
+
+class rtp_attn_cfg(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("batch", "seq", "n_q_heads", "n_kv_heads", "head_dim", "window",
+                                            "block", "rank", "topk", "n_sink", "n_local")] + [("scale", ctypes.c_float)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: run `python -m swa_hybrid_attention_b200.build` "
+                          "(the CUDA extension is required; there is no CPU path)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, L, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_long, ctypes.c_size_t
+    cfgp = ctypes.POINTER(rtp_attn_cfg)
+    sig = {
+        "rtp_route_heads": (I, [cfgp, P, P, ctypes.POINTER(P)]),
+        "rtp_plan_destroy": (None, [P]),
+        "rtp_plan_num_sparse": (I, [P]),
+        "rtp_plan_num_items": (L, [P]),
+        "rtp_plan_sparse_heads": (I, [P, P]),
+        "rtp_plan_work_items": (I, [P, P]),
+        "rtp_indexer_project": (I, [P, P, P, P, P, P, P]),
+        "rtp_block_select": (I, [P, P, P, P, P, P]),
+        "rtp_hybrid_prefill": (I, [P, P, P, P, P, P, P, P]),
+        "rtp_decode_workspace_bytes": (S, [cfgp, P, I]),
+        "rtp_sparse_decode": (I, [cfgp, P, I, P, P, P, P, P, P, P, S, P, P, P]),
+        "rtp_last_device_status": (I, [P]),
+        "rtp_status_str": (ctypes.c_char_p, [I]),
+        "rtp_version": (I, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+_lib = _load()
+EXPORTED = ("rtp_route_heads", "rtp_plan_destroy", "rtp_plan_num_sparse", "rtp_plan_num_items",
+            "rtp_plan_sparse_heads", "rtp_plan_work_items", "rtp_indexer_project", "rtp_block_select",
+            "rtp_hybrid_prefill", "rtp_decode_workspace_bytes", "rtp_sparse_decode", "rtp_last_device_status",
+            "rtp_status_str", "rtp_version")
+
+
+def status_str(s: int) -> str:
+    return _lib.rtp_status_str(int(s)).decode()
+
+
+def _check(name: str, s: int):
+    if s != RTP_OK:
+        raise RtpError(name, s)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, torch.Tensor):
+        if not t.is_contiguous():
+            raise ValueError("tensor arguments must be contiguous")
+        return t.data_ptr()
+    return int(t)
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        if torch.cuda.is_available():
+            return torch.cuda.current_stream().cuda_stream
+        return None
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _kinds(kinds) -> ctypes.Array:
+    return (ctypes.c_uint8 * len(kinds))(*[int(x) for x in kinds])
+
+
+@dataclass
+class AttnConfig:
+    batch: int
+    seq: int
+    n_q_heads: int
+    n_kv_heads: int
+    window: int
+    block: int = 128
+    topk: int = 0
+    n_local: int = 1
+    scale: float = 0.0
+    head_dim: int = 128
+    rank: int = 16
+    n_sink: int = 1
+
+    def c(self) -> rtp_attn_cfg:
+        return rtp_attn_cfg(self.batch, self.seq, self.n_q_heads, self.n_kv_heads, self.head_dim, self.window,
+                            self.block, self.rank, self.topk, self.n_sink, self.n_local, self.scale)
+
+    @property
+    def kmax(self) -> int:
+        return self.topk + 1 + self.n_local
+
+
+# ------------------------------------------------------------- C-named calls
+
+
+def rtp_route_heads(cfg: AttnConfig, kinds, stream=None) -> int:
+    """Returns an opaque plan handle (int); free with rtp_plan_destroy."""
+    out = ctypes.c_void_p()
+    c = cfg.c()
+    _check("rtp_route_heads", _lib.rtp_route_heads(ctypes.byref(c), _kinds(kinds), _stream(stream),
+                                                     ctypes.byref(out)))
+    return out.value
+
+
+def rtp_plan_destroy(plan: int) -> None:
+    _lib.rtp_plan_destroy(plan)
+
+
+def rtp_plan_num_sparse(plan: int) -> int:
+    return _lib.rtp_plan_num_sparse(plan)
+
+
+def rtp_plan_num_items(plan: int) -> int:
+    return _lib.rtp_plan_num_items(plan)
+
+
+def rtp_plan_sparse_heads(plan: int) -> list:
+    n = rtp_plan_num_sparse(plan)
+    buf = (ctypes.c_int32 * max(1, n))()
+    _check("rtp_plan_sparse_heads", _lib.rtp_plan_sparse_heads(plan, buf))
+    return list(buf)[:n]
+
+
+def rtp_plan_work_items(plan: int):
+    import numpy as np
+
+    n = rtp_plan_num_items(plan)
+    arr = np.empty((n, 4), dtype=np.int32)
+    _check("rtp_plan_work_items", _lib.rtp_plan_work_items(plan, arr.ctypes.data_as(ctypes.c_void_p)))
+    return arr
+
+
+def rtp_indexer_project(plan: int, q, k, proj, centroids, qbar, stream=None) -> None:
+    _check("rtp_indexer_project", _lib.rtp_indexer_project(plan, _ptr(q), _ptr(k), _ptr(proj), _ptr(centroids),
+                                                           _ptr(qbar), _stream(stream)))
+
+
+def rtp_block_select(plan: int, qbar, centroids, sel, sel_cnt, stream=None) -> None:
+    _check("rtp_block_select", _lib.rtp_block_select(plan, _ptr(qbar), _ptr(centroids), _ptr(sel), _ptr(sel_cnt),
+                                                     _stream(stream)))
+
+
+def rtp_hybrid_prefill(plan: int, q, k, v, sel, sel_cnt, o, stream=None) -> None:
+    _check("rtp_hybrid_prefill", _lib.rtp_hybrid_prefill(plan, _ptr(q), _ptr(k), _ptr(v), _ptr(sel), _ptr(sel_cnt),
+                                                         _ptr(o), _stream(stream)))
+
+
+def rtp_decode_workspace_bytes(cfg: AttnConfig, kinds, cache_len: int) -> int:
+    c = cfg.c()
+    return int(_lib.rtp_decode_workspace_bytes(ctypes.byref(c), _kinds(kinds), int(cache_len)))
+
+
+def rtp_sparse_decode(cfg: AttnConfig, kinds, cache_len: int, q, kcache, vcache, centroids, proj, o, workspace,
+                      ws_bytes: int, sel_out=None, cnt_out=None, stream=None) -> None:
+    c = cfg.c()
+    _check("rtp_sparse_decode", _lib.rtp_sparse_decode(ctypes.byref(c), _kinds(kinds), int(cache_len), _ptr(q),
+                                                       _ptr(kcache), _ptr(vcache), _ptr(centroids), _ptr(proj),
+                                                       _ptr(o), _ptr(workspace), int(ws_bytes), _ptr(sel_out),
+                                                       _ptr(cnt_out), _stream(stream)))
+
+
+def rtp_last_device_status(stream=None) -> int:
+    return int(_lib.rtp_last_device_status(_stream(stream)))
+
+
+def rtp_version() -> int:
+    return int(_lib.rtp_version())
+
+
+# ------------------------------------------------------------ conveniences
+
+
+class Plan:
+    """Owns a routing plan (rtp_route_heads / rtp_plan_destroy)."""
+
+    def __init__(self, cfg: AttnConfig, kinds, stream=None):
+        self.cfg = cfg
+        self.kinds = list(kinds)
+        self.handle = rtp_route_heads(cfg, kinds, stream)
+        self.n_sparse = rtp_plan_num_sparse(self.handle)
+        self.slot_heads = rtp_plan_sparse_heads(self.handle)
+
+    def close(self):
+        if self.handle:
+            rtp_plan_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def buffers(self, device) -> dict:
+        """Indexer / selection buffers for this plan (allocated with torch)."""
+        c = self.cfg
+        nb = c.seq // c.block
+        ns = max(self.n_sparse, 0)
+        return dict(
+            centroids=torch.empty(c.batch, ns, nb, 16, dtype=torch.float32, device=device),
+            qbar=torch.empty(c.batch, ns, nb, 16, dtype=torch.float32, device=device),
+            sel=torch.empty(c.batch, ns, nb, c.kmax, dtype=torch.int32, device=device),
+            sel_cnt=torch.empty(c.batch, ns, nb, dtype=torch.int32, device=device),
+        )
+
+    def run(self, q, k, v, proj, o, bufs: dict, stream=None) -> None:
+        """One layer: indexer + selection (if any retrieval slot) + prefill."""
+        if self.n_sparse > 0:
+            rtp_indexer_project(self.handle, q, k, proj, bufs["centroids"], bufs["qbar"], stream)
+            rtp_block_select(self.handle, bufs["qbar"], bufs["centroids"], bufs["sel"], bufs["sel_cnt"], stream)
+            rtp_hybrid_prefill(self.handle, q, k, v, bufs["sel"], bufs["sel_cnt"], o, stream)
+        else:
+            rtp_hybrid_prefill(self.handle, q, k, v, None, None, o, stream)
+
+
+def hybrid_prefill_layer(q, k, v, kinds, proj=None, *, window: int, block: int = 128, topk: int = 0,
+                         n_local: int = 1, scale: float = 0.0, stream=None):
+    """Prefill attention of one layer; returns (o, buffers)."""
+    cfg = AttnConfig(q.shape[0], q.shape[2], q.shape[1], k.shape[1], window, block, topk, n_local, scale)
+    plan = Plan(cfg, kinds, stream)
+    bufs = plan.buffers(q.device)
+    o = torch.empty_like(q)
+    if proj is None:
+        proj = torch.zeros(128, 16, dtype=torch.float32, device=q.device)
+    plan.run(q, k, v, proj, o, bufs, stream)
+    plan.close()
+    return o, bufs
+
+
+def sparse_decode_step(q, kcache, vcache, centroids, proj, kinds, *, window: int, block: int = 128, topk: int = 32,
+                       n_local: int = 4, scale: float = 0.0, stream=None, return_selection: bool = False):
+    """One decode step; returns o (and (sel, cnt) when asked)."""
+    B, Hq = q.shape[0], q.shape[1]
+    Hkv, Lc = kcache.shape[1], kcache.shape[2]
+    cfg = AttnConfig(B, 1, Hq, Hkv, window, block, topk, n_local, scale)
+    ws_bytes = rtp_decode_workspace_bytes(cfg, kinds, Lc)
+    if ws_bytes == 0:
+        raise RtpError("rtp_decode_workspace_bytes", RTP_ERR_INVALID_ARG)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    o = torch.empty_like(q)
+    sel = cnt = None
+    if return_selection:
+        sel = torch.full((B, Hkv, cfg.kmax), -1, dtype=torch.int32, device=q.device)
+        cnt = torch.zeros(B, Hkv, dtype=torch.int32, device=q.device)
+    rtp_sparse_decode(cfg, kinds, Lc, q, kcache, vcache, centroids, proj, o, ws, ws_bytes, sel, cnt, stream)
+    return (o, sel, cnt) if return_selection else o

@@ -1,0 +1,99 @@
+"""The C-ABI library loads, exports every symbol include/rtp.h declares, and
+rejects bad arguments before touching the GPU (runs without a GPU)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def rtp():
+    from swa_hybrid_attention_b200 import build
+
+    build.build()
+    from swa_hybrid_attention_b200 import rtp as mod
+
+    return mod
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "rtp.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(rtp_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(rtp):
+    lib = ctypes.CDLL(rtp.LIB_PATH)
+    names = declared_functions()
+    assert len(names) >= 14
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(rtp.EXPORTED)
+
+
+def test_status_strings(rtp):
+    assert rtp.status_str(0) == "RTP_OK"
+    assert rtp.status_str(1) == "RTP_ERR_INVALID_ARG"
+    assert rtp.status_str(4) == "RTP_ERR_TIMEOUT"
+    assert rtp.status_str(99) == "RTP_ERR_UNKNOWN"
+    assert rtp.rtp_version() >> 16 == 1
+
+
+BAD_CFGS = [
+    dict(head_dim=64),
+    dict(rank=8),
+    dict(n_sink=2),
+    dict(block=32),
+    dict(seq=1000),  # not a multiple of block
+    dict(n_q_heads=6, n_kv_heads=4),  # not a multiple
+    dict(n_q_heads=12, n_kv_heads=4),  # odd group
+    dict(n_q_heads=64, n_kv_heads=2),  # group > 16
+    dict(window=0),
+    dict(n_local=0),
+    dict(topk=-1),
+    dict(batch=0),
+    dict(scale=-1.0),
+]
+
+
+@pytest.mark.parametrize("bad", BAD_CFGS)
+def test_route_heads_rejects_bad_config(rtp, bad):
+    args = dict(batch=1, seq=1024, n_q_heads=8, n_kv_heads=2, window=256, block=64, topk=4, n_local=2)
+    extra = {k: v for k, v in bad.items() if k not in args}
+    args.update({k: v for k, v in bad.items() if k in args})
+    cfg = rtp.AttnConfig(**args)
+    for k, v in extra.items():
+        setattr(cfg, k, v)
+    with pytest.raises(rtp.RtpError) as e:
+        rtp.rtp_route_heads(cfg, [2, 0])
+    assert e.value.status == rtp.RTP_ERR_INVALID_ARG
+
+
+def test_route_heads_rejects_bad_kind(rtp):
+    cfg = rtp.AttnConfig(1, 1024, 8, 2, 256, 64, 4, 2)
+    with pytest.raises(rtp.RtpError) as e:
+        rtp.rtp_route_heads(cfg, [3, 0])
+    assert e.value.status == rtp.RTP_ERR_INVALID_ARG
+
+
+def test_decode_workspace_size_and_validation(rtp):
+    cfg = rtp.AttnConfig(8, 1, 32, 4, 8192, 128, 32, 4)
+    n = rtp.rtp_decode_workspace_bytes(cfg, [2, 2, 0, 2], 262144)
+    # sel + cnt + partials [8][4][max(37, 64)][8][132] fp32
+    assert n >= 8 * 4 * 64 * 8 * 132 * 4
+    assert rtp.rtp_decode_workspace_bytes(cfg, [2, 2, 0, 5], 262144) == 0
+    bad = rtp.AttnConfig(8, 1, 32, 4, 8192, 96, 32, 4)
+    assert rtp.rtp_decode_workspace_bytes(bad, [2, 2, 0, 2], 262144) == 0
+    with pytest.raises(rtp.RtpError) as e:
+        rtp.rtp_sparse_decode(cfg, [2, 2, 0, 2], 262144, 0, 0, 0, 0, 0, 0, 0, 0)
+    assert e.value.status == rtp.RTP_ERR_INVALID_ARG
+
+
+def test_null_plan_is_rejected(rtp):
+    for fn, nargs in [(rtp._lib.rtp_indexer_project, 7), (rtp._lib.rtp_block_select, 6),
+                      (rtp._lib.rtp_hybrid_prefill, 8)]:
+        assert fn(*([None] * nargs)) == rtp.RTP_ERR_INVALID_ARG

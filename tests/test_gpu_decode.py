@@ -1,0 +1,95 @@
+"""GPU parity of the sparse decode step against the CPU oracle (C ABI)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import O_MAX_ABS, O_MEAN_ABS, TIE_REL, cpu
+from swa_hybrid_attention_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def rtp(cuda_device):
+    from swa_hybrid_attention_b200 import build
+
+    build.build()
+    from swa_hybrid_attention_b200 import rtp as mod
+
+    return mod
+
+
+def oracle_centroids(kc, kinds, block, proj):
+    """Cached centroids of every retrieval head, computed by the oracle."""
+    B, H, Lc = kc.shape[0], kc.shape[1], kc.shape[2]
+    C = torch.zeros(B, H, Lc // block, 16, dtype=torch.float32)
+    for b in range(B):
+        for h in range(H):
+            if kinds[h] == 2:
+                C[b, h] = torch.from_numpy(oracle.centroids(cpu(kc[b, h]), block, cpu(proj)).astype(np.float32))
+    return C
+
+
+def check_decode(rtp, d, kinds, window, block, topk, n_local, device):
+    q, kc, vc = d["q"].to(device), d["kcache"].to(device), d["vcache"].to(device)
+    proj = d["proj"].to(device)
+    C = oracle_centroids(kc, kinds, block, proj)
+    o, sel, cnt = rtp.sparse_decode_step(q, kc, vc, C.to(device), proj, kinds, window=window, block=block, topk=topk,
+                                         n_local=n_local, return_selection=True)
+    torch.cuda.synchronize()
+    assert rtp.rtp_last_device_status() == rtp.RTP_OK
+    Bt, Hq, Hkv, Lc = q.shape[0], q.shape[1], kc.shape[1], kc.shape[2]
+    G = Hq // Hkv
+    sel, cnt, o = cpu(sel).numpy(), cpu(cnt).numpy(), cpu(o)
+    errs = []
+    for b in range(Bt):
+        for h in range(Hkv):
+            qg = cpu(q[b, h * G:(h + 1) * G, 0])
+            kh, vh = cpu(kc[b, h]), cpu(vc[b, h])
+            if kinds[h] == 2:
+                # the GPU's selection against the oracle's own
+                _, so, co, kth = oracle.decode_head(qg, kh, vh, C[b, h], cpu(proj), 2, window, block, topk, n_local)
+                g = [int(x) for x in sel[b, h, :cnt[b, h]]]
+                assert g == sorted(set(g)) and cnt[b, h] == co
+                if set(g) != set(so[:co].tolist()):
+                    qb = oracle.project_rows(qg, cpu(proj)).sum(axis=0)
+                    s = oracle.scores(qb, C[b, h].double().numpy())
+                    for blk in set(g) ^ set(so[:co].tolist()):
+                        assert abs(s[blk] - kth) <= TIE_REL * abs(kth)
+                ref, _, _, _ = oracle.decode_head(qg, kh, vh, C[b, h], cpu(proj), 2, window, block, topk, n_local,
+                                                  sel=sel[b, h], cnt=cnt[b, h])
+            else:
+                ref, _, _, _ = oracle.decode_head(qg, kh, vh, C[b, h], cpu(proj), kinds[h], window, block, topk,
+                                                  n_local)
+            got = o[b, h * G:(h + 1) * G, 0].double().numpy()
+            err = np.abs(got - oracle.round_bf16(ref))
+            errs.append(err)
+    e = np.stack(errs)
+    assert e.max() <= O_MAX_ABS and e.mean() <= O_MEAN_ABS, (e.max(), e.mean())
+
+
+DECODE_CASES = [
+    # batch, hq, hkv, kinds, cache_len, window, block, topk, n_local
+    (2, 16, 2, [2, 0], 4096, 1000, 128, 4, 2),
+    (2, 8, 4, [2, 2, 0, 1], 3000, 512, 64, 6, 2),    # ragged last block, full head, block 64
+    (1, 4, 1, [2], 640, 100, 128, 8, 1),            # fewer candidates than top-k
+    (3, 32, 4, [2, 0, 2, 2], 8192, 2048, 128, 16, 4),
+]
+
+
+@pytest.mark.parametrize("case", DECODE_CASES)
+def test_decode_small(rtp, cuda_device, case):
+    B, hq, hkv, kinds, Lc, window, block, topk, n_local = case
+    w = inputs.Workload(4, "t", B, 1, hq, hkv, 1, window, block, topk, n_local, "lowfreq", 0, [kinds],
+                        cache_len=Lc, decode=True)
+    d = inputs.decode_step(w, "cpu")
+    check_decode(rtp, d, kinds, window, block, topk, n_local, cuda_device)
+
+
+@pytest.mark.slow
+def test_decode_full_size(rtp, cuda_device):
+    w = inputs.workload(4)
+    d = inputs.decode_step(w, cuda_device)
+    check_decode(rtp, d, w.kinds[0], w.window, w.block, w.topk, w.n_local, cuda_device)

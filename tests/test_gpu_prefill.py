@@ -1,0 +1,173 @@
+"""GPU parity of the prefill path (indexer, selection, hybrid attention)
+against the CPU oracle, through the C ABI."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import check_indexer, check_prefill_rows, check_selection_rows, cpu
+from swa_hybrid_attention_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def rtp(cuda_device):
+    from swa_hybrid_attention_b200 import build
+
+    build.build()
+    from swa_hybrid_attention_b200 import rtp as mod
+
+    return mod
+
+
+def run_layer(rtp, d, window, block, topk, n_local, device, scale=0.0):
+    q, k, v = d["q"].to(device), d["k"].to(device), d["v"].to(device)
+    proj = d["proj"].to(device)
+    cfg = rtp.AttnConfig(q.shape[0], q.shape[2], q.shape[1], k.shape[1], window, block, topk, n_local, scale)
+    plan = rtp.Plan(cfg, d["kinds"])
+    bufs = plan.buffers(device)
+    o = torch.full_like(q, float("nan"))
+    plan.run(q, k, v, proj, o, bufs)
+    torch.cuda.synchronize()
+    assert rtp.rtp_last_device_status() == rtp.RTP_OK
+    return q, k, v, proj, o, bufs, plan
+
+
+def full_check(rtp, d, window, block, topk, n_local, device, scale=0.0):
+    q, k, v, proj, o, bufs, plan = run_layer(rtp, d, window, block, topk, n_local, device, scale)
+    group = q.shape[1] // k.shape[1]
+    n = q.shape[2]
+    nb = n // block
+    slot_of = {h: s for s, h in enumerate(plan.slot_heads)}
+    if plan.n_sparse:
+        C, Qb = check_indexer(bufs["centroids"], bufs["qbar"], q, k, proj, plan.slot_heads, block, group)
+        for s in range(plan.n_sparse):
+            check_selection_rows(cpu(bufs["sel"][0, s]).numpy(), cpu(bufs["sel_cnt"][0, s]).numpy(), Qb[s], C[s],
+                                 np.arange(nb), topk, n_local)
+    check_prefill_rows(o, q, k, v, d["kinds"], group, window, block, bufs["sel"], bufs["sel_cnt"], slot_of,
+                       lambda hq: np.arange(n), None if scale == 0.0 else scale)
+    plan.close()
+    return o
+
+
+def test_tiny_v2_layer(rtp, cuda_device):
+    w = inputs.workload(0)
+    d = inputs.prefill_layer(w, 0, "cpu")
+    full_check(rtp, d, w.window, w.block, w.topk, w.n_local, cuda_device)
+
+
+EDGE_CASES = [
+    # seq, hq, hkv, kinds, window, block, topk, n_local
+    (128, 2, 1, [1], 64, 128, 2, 1),            # one tile, full
+    (128, 2, 1, [0], 1, 128, 2, 1),             # window 1: each row sees itself
+    (192, 2, 1, [2], 64, 64, 1, 1),             # ragged last 128-row tile, block 64
+    (640, 4, 2, [0, 1], 100, 64, 2, 2),         # SWA window not a tile multiple
+    (640, 4, 2, [0, 1], 128, 128, 2, 2),        # window = one tile
+    (640, 4, 2, [0, 1], 129, 128, 2, 2),        # window = tile + 1
+    (640, 4, 2, [0, 2], 5000, 128, 1, 1),       # window > seq (SWA == full)
+    (1024, 16, 2, [2, 0], 256, 128, 2, 1),      # group 8, sparse block 128
+    (1024, 4, 2, [2, 2], 256, 64, 3, 2),        # two sparse slots, block 64
+    (1024, 4, 1, [2], 256, 128, 0, 1),          # top-k 0: sink + diagonal only
+    (1024, 4, 1, [2], 256, 128, 64, 1),         # top-k >= blocks: full causal
+    (1984, 8, 2, [2, 0], 300, 64, 5, 2),        # 31 blocks of 64: ragged tile
+]
+
+
+@pytest.mark.parametrize("case", EDGE_CASES, ids=[f"n{c[0]}-h{c[1]}x{c[2]}-k{''.join(map(str, c[3]))}-w{c[4]}-b{c[5]}"
+                                                  for c in EDGE_CASES])
+def test_edge_shapes(rtp, cuda_device, case):
+    seq, hq, hkv, kinds, window, block, topk, n_local = case
+    d = inputs.small_prefill(seq, hq, hkv, kinds, seed=100 + seq + hq)
+    full_check(rtp, d, window, block, topk, n_local, cuda_device)
+
+
+def test_batch_two_and_scale(rtp, cuda_device):
+    d0 = inputs.small_prefill(512, 4, 2, [2, 0], seed=5)
+    d1 = inputs.small_prefill(512, 4, 2, [2, 0], seed=6)
+    d = dict(q=torch.cat([d0["q"], d1["q"]]), k=torch.cat([d0["k"], d1["k"]]), v=torch.cat([d0["v"], d1["v"]]),
+             proj=d0["proj"], kinds=[2, 0])
+    q, k, v, proj, o, bufs, plan = run_layer(rtp, d, 200, 64, 2, 2, cuda_device, scale=0.05)
+    for b in range(2):
+        db = d0 if b == 0 else d1
+        sub = dict(centroids=bufs["centroids"][b:b + 1], sel=bufs["sel"][b:b + 1], sel_cnt=bufs["sel_cnt"][b:b + 1])
+        check_prefill_rows(o[b:b + 1], db["q"], db["k"], db["v"], [2, 0], 2, 200, 64, sub["sel"], sub["sel_cnt"],
+                           {0: 0}, lambda hq: np.arange(512), 0.05)
+    plan.close()
+
+
+def test_deterministic(rtp, cuda_device):
+    w = inputs.workload(0)
+    d = inputs.prefill_layer(w, 0, "cpu")
+    outs = []
+    for _ in range(2):
+        q, k, v, proj, o, bufs, plan = run_layer(rtp, d, w.window, w.block, w.topk, w.n_local, cuda_device)
+        outs.append((o.clone(), bufs["sel"].clone(), bufs["centroids"].clone()))
+        plan.close()
+    for a, b in zip(outs[0], outs[1]):
+        assert torch.equal(a, b)
+
+
+def sampled_rows(n, block, topk, n_local, rng, extra=()):
+    nb = n // block
+    blocks = sorted(set([0, 1, min(nb - 1, topk + n_local), min(nb - 1, topk + n_local + 1), nb - 1]
+                        + list(rng.integers(0, nb, 8))))
+    rows = []
+    for b in blocks:
+        rows += [b * block, b * block + block // 2, b * block + block - 1]
+    rows += list(rng.integers(0, n, 8)) + list(extra)
+    return np.array(sorted(set(int(r) for r in rows)), dtype=np.int64)
+
+
+def sampled_check(rtp, w, layer, device):
+    """Full-size layer: indexer and selection on sampled blocks, O on sampled rows."""
+    d = inputs.prefill_layer(w, layer, device)
+    q, k, v, proj, o, bufs, plan = run_layer(rtp, d, w.window, w.block, w.topk, w.n_local, device)
+    G, n, B = w.group, w.seq, w.block
+    nb = n // B
+    rng = np.random.default_rng(layer + 17)
+    slot_of = {h: s for s, h in enumerate(plan.slot_heads)}
+    needles_by_head = {}
+    for (kvh, qh, tq, j) in d["needles"]:
+        needles_by_head.setdefault(qh, []).append(tq)
+    for s, kvh in enumerate(plan.slot_heads):
+        C = oracle.centroids(cpu(k[0, kvh]), B, cpu(proj))
+        gc = cpu(bufs["centroids"][0, s]).double().numpy()
+        assert np.all(np.abs(gc - C) <= 2e-4 + 2e-4 * np.abs(C))
+        t_list = np.array(sorted(set([0, 1, w.topk + w.n_local, w.topk + w.n_local + 1, nb - 1]
+                                     + list(rng.integers(0, nb, 48)))), dtype=np.int32)
+        Qb = np.zeros((nb, 16))
+        for t in t_list:
+            Qb[t] = oracle.qbar(cpu(q[0, kvh * G:(kvh + 1) * G, t * B:(t + 1) * B]), B, cpu(proj))[0]
+        gq = cpu(bufs["qbar"][0, s]).double().numpy()[t_list]
+        assert np.all(np.abs(gq - Qb[t_list]) <= 2e-4 + 2e-4 * np.abs(Qb[t_list]))
+        sel = cpu(bufs["sel"][0, s]).numpy()
+        cnt = cpu(bufs["sel_cnt"][0, s]).numpy()
+        check_selection_rows(sel[t_list], cnt[t_list], Qb, C, t_list, w.topk, w.n_local)
+        # needle diagnostic: fraction of needles whose key block is selected for their query block
+        hits = sum(1 for (h, qh, tq, j) in d["needles"] if h == kvh and (j // B) in set(sel[tq // B][:cnt[tq // B]]))
+        tot = sum(1 for x in d["needles"] if x[0] == kvh)
+        print(f"needle recall slot {s}: {hits}/{tot}")
+    check_prefill_rows(o, q, k, v, d["kinds"], G, w.window, B, bufs["sel"], bufs["sel_cnt"], slot_of,
+                       lambda hq: sampled_rows(n, B, w.topk, w.n_local, rng, needles_by_head.get(hq, [])[:8]))
+    plan.close()
+
+
+@pytest.mark.slow
+def test_full_size_1m_v2_layer(rtp, cuda_device):
+    sampled_check(rtp, inputs.workload(3), 0, cuda_device)
+
+
+@pytest.mark.slow
+def test_full_size_128k_v2_layer(rtp, cuda_device):
+    w = inputs.workload(2)
+    layer = next(l for l in range(w.layers) if 2 in w.kinds[l])
+    sampled_check(rtp, w, layer, cuda_device)
+
+
+@pytest.mark.slow
+def test_full_size_32k_v1_layer(rtp, cuda_device):
+    w = inputs.workload(1)
+    layer = next(l for l in range(w.layers) if 1 in w.kinds[l])
+    sampled_check(rtp, w, layer, cuda_device)
