@@ -134,6 +134,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const DecodeA
     qs[e] = __bfloat162float(a.q[(static_cast<size_t>(b) * a.n_q_heads + kvh * G + h) * kHeadDim + d]);
   }
   if (tid == 0) ok_flag = mbar_wait(&bar, 0, nullptr, a.status) ? 1 : 0;
+  __syncwarp();  // warp 0 reconverges before the CTA barrier
   __syncthreads();
   if (!ok_flag) return;
 

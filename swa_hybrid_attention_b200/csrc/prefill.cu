@@ -404,22 +404,28 @@ __device__ void run_softmax(Smem& s, uint32_t tmem, int h, const PrefillArgs& a,
 #pragma unroll
       for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(r[c]));
       const float m_new = mx * sl2;
-      if (m_new > m_ref + kRescaleThreshold) {
-        if (j > 0 && m_ref != -INFINITY) {
-          const float alpha = exp2f(m_ref - m_new);
-          l *= alpha;
+      // Lazy rescale: a row moves its reference maximum only when the new
+      // maximum exceeds it by more than 2^8.  O lives in TMEM and the
+      // tcgen05.ld/st that rescale it are warp-collective, so the whole warp
+      // takes the rescale path when any of its rows needs it (alpha = 1 for
+      // the others).
+      const bool raise = m_new > m_ref + kRescaleThreshold;
+      const bool rescale_o = raise && j > 0 && m_ref != -INFINITY;
+      if (__any_sync(0xffffffffu, rescale_o)) {
+        const float alpha = rescale_o ? exp2f(m_ref - m_new) : 1.0f;
+        l *= alpha;
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tO + 32 * c, o);
-            tmem_ld_wait();
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + 32 * c, o);
-          }
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(tO + 32 * c, o);
         }
-        m_ref = m_new;
+        tmem_st_wait();
       }
+      if (raise) m_ref = m_new;
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
       // P = exp2(s * scale*log2e - m) as packed bf16 pairs, written over the
       // first 64 columns of S (the whole S row is already in registers).
@@ -496,6 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&mk);
     tma_prefetch_desc(&mv);
   }
+  __syncwarp();
   if (warp == 2) {
     tmem_alloc(&s.tmem_base, 512);
     tmem_relinquish();
@@ -506,10 +513,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
   volatile int* abort = &s.abort_flag;
 
+  // Single-lane roles: the other 31 lanes of warps 0 and 1 wait at
+  // __syncwarp so that every warp reaches the CTA barrier below converged.
   if (warp == 0) {
     if (lane_id() == 0) run_producer(s, &mq, &mk, &mv, a, abort);
+    __syncwarp();
   } else if (warp == 1) {
     if (lane_id() == 0) run_mma(s, tmem, a, abort);
+    __syncwarp();
   } else if (warp >= 4) {
     run_softmax(s, tmem, (warp - 4) >> 2, a, abort);
   }

@@ -121,6 +121,7 @@ __device__ inline int select_blocks(const float (&q)[kRank], const float* C, int
           acc += cnt8[e];
         }
       }
+      __syncwarp();
     }
     __syncthreads();
     prefix |= sh.digit << shift;
