@@ -206,6 +206,33 @@ rtp_status rtp_sparse_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, 
                              void* stream);
 
 /* ------------------------------------------------------------------------
+ * rtp_sparse_decode_noalloc — the decode step of rtp_sparse_decode for
+ * callers that cannot allocate device memory at call time: code running
+ * while a CUDA graph is being captured or replayed elsewhere in the
+ * process, real-time loops that must not enter the allocator (cudaMalloc
+ * synchronises the device), or hosts whose memory pools are owned by
+ * another runtime.  The paper has no counterpart to this entry point.
+ *   Arguments are those of rtp_sparse_decode without workspace/ws_bytes.
+ *   The split-K scratch (selection lists and per-split partial results)
+ *   lives in a fixed 16 MiB device array inside the library
+ *   (rtp_decode_workspace_bytes tells how much a shape needs); a shape that
+ *   needs more returns RTP_ERR_INVALID_ARG.  Nothing is allocated: no
+ *   cudaMalloc, cudaFree or allocating library call on this path.
+ *   The array is looked up once per device, on the first call made with
+ *   that device current; make that first call before any stream capture.
+ *   Every call shares the one array and it keeps the last call's contents
+ *   (every word a call reads is written earlier in the same call, so
+ *   nothing needs clearing); calls that overlap on the GPU — on different
+ *   streams, or from several host threads — race on it and must be
+ *   serialised by the caller.
+ *   Unlike rtp_sparse_decode this path has no device status word: an
+ *   out-of-range block index in the selection is skipped without a report.
+ * ---------------------------------------------------------------------- */
+rtp_status rtp_sparse_decode_noalloc(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* q,
+                                     const void* kcache, const void* vcache, const float* centroids,
+                                     const float* proj, void* o, int32_t* sel_out, int32_t* cnt_out, void* stream);
+
+/* ------------------------------------------------------------------------
  * rtp_last_device_status — synchronise `stream`, then read and clear the
  * device status word of the current device.  Returns RTP_OK, RTP_ERR_TIMEOUT
  * (a bounded wait gave up), RTP_ERR_INVALID_ARG (a kernel met an

@@ -22,6 +22,8 @@
 
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "internal.cuh"
 #include "select_common.cuh"
 #include "sm100.cuh"
@@ -250,7 +252,31 @@ __global__ void __launch_bounds__(kAttnThreads) decode_combine_kernel(const Deco
   a.o[(static_cast<size_t>(b) * a.n_q_heads + hq) * kHeadDim + d] = __float2bfloat16_rn(out);
 }
 
+// Scratch of the allocation-free decode entry point: a file-scope device
+// array that every GPU loading this library holds until the process exits.
+static __device__ __align__(256) unsigned char g_decode_static_scratch[kDecodeStaticScratchBytes];
+
 }  // namespace
+
+cudaError_t decode_static_scratch(void** ptr) {
+  // Host code may not use the array's name as a device address; look up the
+  // address once per device, with that device current, and reuse it.
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_static_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  return cudaSuccess;
+}
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
   const size_t sel_smem = static_cast<size_t>(a.nbc) * sizeof(uint32_t);

@@ -71,6 +71,12 @@ cudaError_t launch_indexer(const IndexerArgs& a, cudaStream_t stream);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 
+// Fixed-size device scratch used by the allocation-free decode entry point.
+constexpr size_t kDecodeStaticScratchBytes = size_t(16) << 20;
+// Device address of that scratch on the current device (looked up once per
+// device with cudaGetSymbolAddress; no allocation).
+cudaError_t decode_static_scratch(void** ptr);
+
 // Shared-memory bytes the prefill kernel needs (host side, for the opt-in).
 size_t prefill_smem_bytes();
 

@@ -441,6 +441,52 @@ rtp_status rtp_sparse_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, 
   return cuda_status(launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+rtp_status rtp_sparse_decode_noalloc(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* q,
+                                     const void* kcache, const void* vcache, const float* centroids,
+                                     const float* proj, void* o, int32_t* sel_out, int32_t* cnt_out, void* stream) {
+  DecodeLayout L;
+  if (!decode_layout(cfg, kind_host, cache_len, L)) return RTP_ERR_INVALID_ARG;
+  if (L.total > kDecodeStaticScratchBytes) return RTP_ERR_INVALID_ARG;  // beyond the fixed scratch
+  if (!q || !kcache || !vcache || !o) return RTP_ERR_INVALID_ARG;
+  bool any_sparse = false;
+  for (int h = 0; h < cfg->n_kv_heads; ++h) any_sparse |= kind_host[h] == RTP_HEAD_SPARSE;
+  if (any_sparse && (!centroids || !proj)) return RTP_ERR_INVALID_ARG;
+  if ((sel_out == nullptr) != (cnt_out == nullptr)) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o)) return RTP_ERR_INVALID_ARG;
+  if ((centroids && !aligned16(centroids)) || (proj && !aligned16(proj))) return RTP_ERR_INVALID_ARG;
+  if (cfg->n_kv_heads > kMaxDecodeKvHeads) return RTP_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  if (decode_static_scratch(&scratch) != cudaSuccess || !scratch) return RTP_ERR_CUDA;
+  DecodeArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.kcache = static_cast<const __nv_bfloat16*>(kcache);
+  a.vcache = static_cast<const __nv_bfloat16*>(vcache);
+  a.centroids = centroids;
+  a.proj = proj;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  std::memset(a.kind, 0, sizeof(a.kind));
+  std::memcpy(a.kind, kind_host, cfg->n_kv_heads);
+  char* ws = static_cast<char*>(scratch);
+  a.sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(ws + L.sel_off);
+  a.cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(ws + L.cnt_off);
+  a.partial = reinterpret_cast<float*>(ws + L.part_off);
+  a.batch = cfg->batch;
+  a.n_q_heads = cfg->n_q_heads;
+  a.n_kv_heads = cfg->n_kv_heads;
+  a.group = cfg->n_q_heads / cfg->n_kv_heads;
+  a.cache_len = cache_len;
+  a.nbc = cache_len / cfg->block;
+  a.window = cfg->window;
+  a.block = cfg->block;
+  a.topk = cfg->topk;
+  a.n_local = cfg->n_local;
+  a.kmax = L.kmax;
+  a.max_splits = L.max_splits;
+  a.scale_log2 = effective_scale(cfg) * kLog2e;
+  a.status = nullptr;  // no status word: getting one may allocate
+  return cuda_status(launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 rtp_status rtp_last_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return RTP_ERR_CUDA;

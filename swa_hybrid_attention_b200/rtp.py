@@ -56,6 +56,7 @@ def _load() -> ctypes.CDLL:
         "rtp_hybrid_prefill": (I, [P, P, P, P, P, P, P, P]),
         "rtp_decode_workspace_bytes": (S, [cfgp, P, I]),
         "rtp_sparse_decode": (I, [cfgp, P, I, P, P, P, P, P, P, P, S, P, P, P]),
+        "rtp_sparse_decode_noalloc": (I, [cfgp, P, I, P, P, P, P, P, P, P, P, P]),
         "rtp_last_device_status": (I, [P]),
         "rtp_status_str": (ctypes.c_char_p, [I]),
         "rtp_version": (I, []),
@@ -70,7 +71,8 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 EXPORTED = ("rtp_route_heads", "rtp_plan_destroy", "rtp_plan_num_sparse", "rtp_plan_num_items",
             "rtp_plan_sparse_heads", "rtp_plan_work_items", "rtp_indexer_project", "rtp_block_select",
-            "rtp_hybrid_prefill", "rtp_decode_workspace_bytes", "rtp_sparse_decode", "rtp_last_device_status",
+            "rtp_hybrid_prefill", "rtp_decode_workspace_bytes", "rtp_sparse_decode", "rtp_sparse_decode_noalloc",
+            "rtp_last_device_status",
             "rtp_status_str", "rtp_version")
 
 
@@ -196,6 +198,16 @@ def rtp_sparse_decode(cfg: AttnConfig, kinds, cache_len: int, q, kcache, vcache,
                                                        _ptr(kcache), _ptr(vcache), _ptr(centroids), _ptr(proj),
                                                        _ptr(o), _ptr(workspace), int(ws_bytes), _ptr(sel_out),
                                                        _ptr(cnt_out), _stream(stream)))
+
+
+def rtp_sparse_decode_noalloc(cfg: AttnConfig, kinds, cache_len: int, q, kcache, vcache, centroids, proj, o,
+                              sel_out=None, cnt_out=None, stream=None) -> None:
+    """Decode step whose scratch is the library's fixed device array (no allocation)."""
+    c = cfg.c()
+    _check("rtp_sparse_decode_noalloc",
+           _lib.rtp_sparse_decode_noalloc(ctypes.byref(c), _kinds(kinds), int(cache_len), _ptr(q), _ptr(kcache),
+                                          _ptr(vcache), _ptr(centroids), _ptr(proj), _ptr(o), _ptr(sel_out),
+                                          _ptr(cnt_out), _stream(stream)))
 
 
 def rtp_last_device_status(stream=None) -> int:
