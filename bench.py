@@ -482,7 +482,16 @@ def run_ours(args, rank, world, local):
 
     device = torch.device("cuda", local)
     peaks, peak_src = load_peaks()
+    if args.only == "decode":
+        if rank == 0:
+            print(json.dumps({"decode_8x256k": time_decode(rtp, args.decode_steps, device)}), flush=True)
+        return
     w = inputs.workload(3)
+    if args.seq:
+        # same head structure at a shorter length (profiling runs)
+        w.seq = args.seq
+        w.name = f"{w.name}@{args.seq}"
+        w.needles = max(1, w.needles * args.seq // 1048576)
     res = time_primary(rtp, w, rank, args.steps, args.warmup, device, world)
     algo, execd = layer_flops(w, res["kinds"])
     step_ms = max_over_ranks(res["total_ms"] / args.steps, world)
@@ -560,6 +569,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=10.0)
     ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--seq", type=int, default=0, help="override the primary workload's length (profiling)")
+    ap.add_argument("--only", choices=["all", "decode"], default="all", help="run only part of the bench")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

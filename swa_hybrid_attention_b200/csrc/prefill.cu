@@ -42,6 +42,7 @@
 #include <climits>
 #include <cstdint>
 
+#include "exp2_poly.cuh"
 #include "internal.cuh"
 #include "sm100.cuh"
 
@@ -49,12 +50,31 @@ namespace rtp {
 namespace {
 
 constexpr int kThreads = 384;
+// Register split between roles (setmaxnreg): warpgroup 0 (producer, MMA,
+// allocator, spare) gives registers to the two softmax warpgroups, which hold
+// a whole 128-column S row each.  The split must fit in what the block is
+// launched with (kThreads x kLaunchRegs), or the increase would wait forever;
+// launch_prefill checks the compiled count.  The roles are separate
+// (non-inlined) functions so that each is register-allocated for its own
+// budget; each runs once per CTA.
+constexpr int kLaunchRegs = 168;
+constexpr int kLowRegs = 88;
+constexpr int kHighRegs = 200;
+static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split must fit the launch");
 constexpr int kStages = 2;
 constexpr uint32_t kTileBytes = 128 * 128 * 2;  // one 128x128 bf16 operand tile
 constexpr uint32_t kChunkBytes = 128 * 128;     // 64 columns x 128 rows
 constexpr int kNoWindow = 1 << 30;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows > 2^8
 constexpr uint32_t kMemberAll = 0x1Eu;
+// Column pairs (k mod 8) whose exponentials use the FMA-pipe polynomial
+// instead of the MUFU: bit k set => pair k.  Default: none — measured on B200
+// (1M-token layer) the polynomial costs more issue slots than the MUFU time
+// it frees (1/8: +2.7 %, 1/4: +5.4 %, 3/8: +17 % kernel time).
+#ifndef RTP_POLY_PAIRS
+#define RTP_POLY_PAIRS 0x00u
+#endif
+constexpr uint32_t kPolyPairs = RTP_POLY_PAIRS;
 
 struct __align__(1024) Smem {
   uint8_t q[2][kTileBytes];
@@ -226,7 +246,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // ------------------------------------------------------------------ producer
-__device__ void run_producer(Smem& s, const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv,
+__device__ __noinline__ void run_producer(Smem& s, const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv,
                              const PrefillArgs& a, volatile int* abort) {
   uint32_t it = 0, gt = 0;
   uint32_t q_issued = 0;  // bit h: Q of head h issued for the current item
@@ -294,7 +314,7 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint3
   }
 }
 
-__device__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& a, volatile int* abort) {
+__device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& a, volatile int* abort) {
   const uint32_t id_qk = idesc_bf16_f32(128, 128, false);
   const uint32_t id_pv = idesc_bf16_f32(128, 128, true);
   const uint32_t tS[2] = {tmem, tmem + 128};
@@ -366,7 +386,7 @@ drain:
 }
 
 // ------------------------------------------------------------------ softmax
-__device__ void run_softmax(Smem& s, uint32_t tmem, int h, const PrefillArgs& a, volatile int* abort) {
+__device__ __noinline__ void run_softmax(Smem& s, uint32_t tmem, int h, const PrefillArgs& a, volatile int* abort) {
   const int q4 = warp_id() & 3;
   const int row = q4 * 32 + lane_id();
   const uint32_t lane_bits = static_cast<uint32_t>(q4 * 32) << 16;
@@ -400,9 +420,13 @@ __device__ void run_softmax(Smem& s, uint32_t tmem, int h, const PrefillArgs& a,
           if (!(member && key <= i && key > lo_key)) r[c] = __float_as_uint(-INFINITY);
         }
       }
-      float mx = -INFINITY;
+      // row maximum: three-input max, four independent chains
+      float m4[4];
 #pragma unroll
-      for (int c = 0; c < 128; ++c) mx = fmaxf(mx, __uint_as_float(r[c]));
+      for (int e = 0; e < 4; ++e) m4[e] = max3(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]), -INFINITY);
+#pragma unroll
+      for (int k = 4; k < 64; ++k) m4[k & 3] = max3(m4[k & 3], __uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+      const float mx = max3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
       const float m_new = mx * sl2;
       // Lazy rescale: a row moves its reference maximum only when the new
       // maximum exceeds it by more than 2^8.  O lives in TMEM and the
@@ -429,20 +453,32 @@ __device__ void run_softmax(Smem& s, uint32_t tmem, int h, const PrefillArgs& a,
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
       // P = exp2(s * scale*log2e - m) as packed bf16 pairs, written over the
       // first 64 columns of S (the whole S row is already in registers).
-      float sum = 0.f;
+      // Arithmetic runs on packed f32x2 pairs; the column pairs selected by
+      // kPolyPairs use the FMA-pipe polynomial, the others the MUFU ex2 (at
+      // full tensor rate the MUFU alone could not keep up).
+      const uint64_t sl2x2 = pack2(sl2, sl2), negm2 = pack2(-m_use, -m_use);
+      uint64_t s4[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t p[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = exp2f(fmaf(__uint_as_float(r[32 * c + 2 * e]), sl2, -m_use));
-          const float p1 = exp2f(fmaf(__uint_as_float(r[32 * c + 2 * e + 1]), sl2, -m_use));
-          sum += p0 + p1;
-          p[e] = pack_bf16x2(p0, p1);
+          const int k = 16 * c + e;  // column pair (2k, 2k+1)
+          const uint64_t x = fma2((static_cast<uint64_t>(r[2 * k + 1]) << 32) | r[2 * k], sl2x2, negm2);
+          uint64_t pe;
+          if ((kPolyPairs >> (k & 7)) & 1u)
+            pe = exp2_poly2(lo2(x), hi2(x));
+          else
+            pe = pack2(exp2f(lo2(x)), exp2f(hi2(x)));
+          s4[k & 3] = add2(s4[k & 3], pe);
+          p[e] = pack_bf16x2(lo2(pe), hi2(pe));
         }
         tmem_st16(tS + 16 * c, p);
       }
-      l += sum;
+      {
+        const uint64_t sa = add2(add2(s4[0], s4[1]), add2(s4[2], s4[3]));
+        l += lo2(sa) + hi2(sa);
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(&s.p_full[h]);
@@ -513,16 +549,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
   volatile int* abort = &s.abort_flag;
 
-  // Single-lane roles: the other 31 lanes of warps 0 and 1 wait at
-  // __syncwarp so that every warp reaches the CTA barrier below converged.
-  if (warp == 0) {
-    if (lane_id() == 0) run_producer(s, &mq, &mk, &mv, a, abort);
-    __syncwarp();
-  } else if (warp == 1) {
-    if (lane_id() == 0) run_mma(s, tmem, a, abort);
-    __syncwarp();
-  } else if (warp >= 4) {
+  // Each setmaxnreg sits inside its role's branch so that the raised budget
+  // dominates only the softmax code.  Single-lane roles: the other 31 lanes
+  // of warps 0 and 1 wait at __syncwarp so that every warp reaches the CTA
+  // barrier below converged.
+  if (warp >= 4) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
     run_softmax(s, tmem, (warp - 4) >> 2, a, abort);
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
+    if (warp == 0) {
+      if (lane_id() == 0) run_producer(s, &mq, &mk, &mv, a, abort);
+      __syncwarp();
+    } else if (warp == 1) {
+      if (lane_id() == 0) run_mma(s, tmem, a, abort);
+      __syncwarp();
+    }
   }
 
   tc_fence_before();
@@ -543,8 +585,14 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& mq, const CU
   int dev = 0;
   cudaGetDevice(&dev);
   if (configured_device != dev) {
-    cudaError_t e = cudaFuncSetAttribute(hybrid_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(prefill_smem_bytes()));
+    // The setmaxnreg split is only valid for the register count it was sized
+    // for; refuse to launch a build that compiled to anything else.
+    cudaFuncAttributes attr;
+    cudaError_t e = cudaFuncGetAttributes(&attr, hybrid_prefill_kernel);
+    if (e != cudaSuccess) return e;
+    if (attr.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(hybrid_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(prefill_smem_bytes()));
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }

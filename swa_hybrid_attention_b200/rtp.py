@@ -20,7 +20,9 @@ from dataclasses import dataclass
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "librtp.so")
+# RTP_LIB may name another build of the library (for example one compiled
+# with different tuning macros); by default the in-tree build is loaded.
+LIB_PATH = os.environ.get("RTP_LIB") or os.path.join(_HERE, "librtp.so")
 
 RTP_OK, RTP_ERR_INVALID_ARG, RTP_ERR_UNSUPPORTED, RTP_ERR_CUDA, RTP_ERR_TIMEOUT, RTP_ERR_NO_MEMORY = range(6)
 RTP_HEAD_SWA, RTP_HEAD_FULL, RTP_HEAD_SPARSE = 0, 1, 2
