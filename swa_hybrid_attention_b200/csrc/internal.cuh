@@ -69,7 +69,7 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& mq, const CU
                            int num_ctas, cudaStream_t stream);
 cudaError_t launch_indexer(const IndexerArgs& a, cudaStream_t stream);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
-cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t stream);
 
 // Fixed-size device scratch used by the allocation-free decode entry point.
 constexpr size_t kDecodeStaticScratchBytes = size_t(16) << 20;

@@ -351,7 +351,7 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
       const uint32_t sk2 = smem_u32(s.k[st2]);
       if (!mbar_wait(&s.v_full[st], (g >> 1) & 1u, abort, a.status)) goto drain;
       // head 0: O0 += P0 V ; then S0 for the next tile
-      if (!mbar_wait(&s.p_full[0], pc & 1u, abort, a.status)) goto drain;
+      if (!mbar_wait_spin(&s.p_full[0], pc & 1u, abort, a.status)) goto drain;
       tc_fence_after();
       issue_pv(tO[0], tS[0], sv, id_pv, j > 0);
       if (!has_next) {
@@ -364,7 +364,7 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
         if (j + 2 == n) umma_commit(&s.q_empty[0]);
       }
       // head 1
-      if (!mbar_wait(&s.p_full[1], pc & 1u, abort, a.status)) goto drain;
+      if (!mbar_wait_spin(&s.p_full[1], pc & 1u, abort, a.status)) goto drain;
       tc_fence_after();
       issue_pv(tO[1], tS[1], sv, id_pv, j > 0);
       umma_commit(&s.kv_empty[st]);

@@ -438,7 +438,11 @@ rtp_status rtp_sparse_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, 
   a.scale_log2 = effective_scale(cfg) * kLog2e;
   a.status = status_word(current_device());
   if (!a.status) return RTP_ERR_NO_MEMORY;
-  return cuda_status(launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+  CUtensorMap mk, mv;
+  if (!encode_bf16_3d(&mk, kcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64) ||
+      !encode_bf16_3d(&mv, vcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64))
+    return RTP_ERR_CUDA;
+  return cuda_status(launch_decode(a, mk, mv, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 rtp_status rtp_sparse_decode_noalloc(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* q,
@@ -484,7 +488,11 @@ rtp_status rtp_sparse_decode_noalloc(const rtp_attn_cfg* cfg, const uint8_t* kin
   a.max_splits = L.max_splits;
   a.scale_log2 = effective_scale(cfg) * kLog2e;
   a.status = nullptr;  // no status word: getting one may allocate
-  return cuda_status(launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+  CUtensorMap mk, mv;
+  if (!encode_bf16_3d(&mk, kcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64) ||
+      !encode_bf16_3d(&mv, vcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64))
+    return RTP_ERR_CUDA;
+  return cuda_status(launch_decode(a, mk, mv, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 rtp_status rtp_last_device_status(void* stream) {
