@@ -180,14 +180,33 @@ def barrier(world: int):
         dist.barrier()
 
 
+def _collective_device():
+    import torch.distributed as dist
+
+    return torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+
+
 def max_over_ranks(x: float, world: int) -> float:
+    """Max of a per-rank value (the step time) over all ranks."""
     if world == 1:
         return x
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_collective_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def shard_units(n_units: int, rank: int, world: int) -> list:
+    """Contiguous share of n_units independent units (layers, sequences) for a rank."""
+    per, extra = divmod(n_units, world)
+    start = rank * per + min(rank, extra)
+    return list(range(start, start + per + (1 if rank < extra else 0)))
+
+
+def rank_layer(rank: int) -> int:
+    """Each rank times its own independent layer of the primary workload (weak scaling)."""
+    return rank
 
 
 # ---------------------------------------------------------------- our arm
@@ -492,7 +511,7 @@ def run_ours(args, rank, world, local):
         w.seq = args.seq
         w.name = f"{w.name}@{args.seq}"
         w.needles = max(1, w.needles * args.seq // 1048576)
-    res = time_primary(rtp, w, rank, args.steps, args.warmup, device, world)
+    res = time_primary(rtp, w, rank_layer(rank), args.steps, args.warmup, device, world)
     algo, execd = layer_flops(w, res["kinds"])
     step_ms = max_over_ranks(res["total_ms"] / args.steps, world)
     pre_ms = statistics.mean(res["per"]["prefill"])
@@ -521,7 +540,7 @@ def run_ours(args, rank, world, local):
         del sample
         torch.cuda.empty_cache()
     secondary = {}
-    if not args.no_secondary:
+    if not args.no_secondary and world == 1:
         secondary["v2_128k_48_layers"] = time_secondary_128k(rtp, 2, device)
         secondary["decode_8x256k"] = time_decode(rtp, args.decode_steps, device)
     if rank != 0:

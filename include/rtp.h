@@ -241,6 +241,17 @@ rtp_status rtp_sparse_decode_noalloc(const rtp_attn_cfg* cfg, const uint8_t* kin
  * ---------------------------------------------------------------------- */
 rtp_status rtp_last_device_status(void* stream);
 
+/* ------------------------------------------------------------------------
+ * rtp_selftest_bounded_wait — diagnostic: launches a one-warp kernel that
+ * waits on an mbarrier nothing ever arrives on, using the same bounded wait
+ * as every kernel of the library but with a limit of `limit_ms`
+ * (1..10000).  The wait must give up, record the time-out in the device
+ * status word and let the kernel exit; the call then returns what
+ * rtp_last_device_status reports (RTP_ERR_TIMEOUT when the mechanism works)
+ * and the context stays usable.  Synchronises `stream`.
+ * ---------------------------------------------------------------------- */
+rtp_status rtp_selftest_bounded_wait(unsigned limit_ms, void* stream);
+
 /* Human-readable name of a status code (static string). */
 const char* rtp_status_str(rtp_status s);
 

@@ -37,27 +37,38 @@ constexpr int kMaxGroup = 16;
 __global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DecodeArgs a) {
   extern __shared__ uint32_t keys[];
   __shared__ SelectScratch sh;
-  __shared__ float proj_part[kMaxGroup][kRank];
+  __shared__ float qsum[kHeadDim];
+  __shared__ float part16[16][kRank];
   const int kvh = blockIdx.x, b = blockIdx.y;
   // The attention launch that follows may start now: its streaming-head
   // CTAs do not need the selection, its retrieval-head CTAs wait for it.
   griddep_launch_dependents();
   if (a.kind[kvh] != KIND_SPARSE) return;
-  // per-head projections P^T q_h (fixed order over d), then the sum over heads
+  // qbar = sum_h P^T q_h = P^T (sum_h q_h): sum the group's queries (fixed
+  // head order), then project with all threads: thread (j, c) takes dims
+  // [8j, 8j+8) of output c, and the 16 partials are added in a fixed order.
   const int tid = threadIdx.x;
-  for (int e = tid; e < a.group * kRank; e += kSelThreads) {
-    const int h = e / kRank, c = e % kRank;
-    const __nv_bfloat16* qh = a.q + (static_cast<size_t>(b) * a.n_q_heads + kvh * a.group + h) * kHeadDim;
-    float s = 0.f;
-    for (int d = 0; d < kHeadDim; ++d) s = fmaf(a.proj[d * kRank + c], __bfloat162float(qh[d]), s);
-    proj_part[h][c] = s;
+  if (tid < kHeadDim) {
+    const __nv_bfloat16* qg = a.q + (static_cast<size_t>(b) * a.n_q_heads + kvh * a.group) * kHeadDim + tid;
+    float sq = 0.f;
+    for (int h = 0; h < a.group; ++h) sq += __bfloat162float(qg[h * kHeadDim]);
+    qsum[tid] = sq;
+  }
+  __syncthreads();
+  {
+    const int j = tid >> 4, c = tid & 15;
+    float sp = 0.f;
+#pragma unroll
+    for (int d = 8 * j; d < 8 * j + 8; ++d) sp = fmaf(__ldg(a.proj + d * kRank + c), qsum[d], sp);
+    part16[j][c] = sp;
   }
   __syncthreads();
   float q[kRank];
 #pragma unroll
   for (int c = 0; c < kRank; ++c) {
     float s = 0.f;
-    for (int h = 0; h < a.group; ++h) s += proj_part[h][c];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) s += part16[j][c];
     q[c] = s;
   }
   const int t = (a.cache_len - 1) / a.block;

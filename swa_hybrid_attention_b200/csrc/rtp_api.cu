@@ -39,6 +39,21 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Self-test of the bounded wait used by every kernel: an mbarrier nobody
+// arrives on, waited for with a short limit.
+__global__ void bounded_wait_selftest_kernel(uint32_t* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, status, limit_ns);
+  __syncwarp();
+}
+
 // ---------------------------------------------------------------- status word
 std::mutex g_status_mu;
 uint32_t* g_status[64] = {nullptr};
@@ -493,6 +508,16 @@ rtp_status rtp_sparse_decode_noalloc(const rtp_attn_cfg* cfg, const uint8_t* kin
       !encode_bf16_3d(&mv, vcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64))
     return RTP_ERR_CUDA;
   return cuda_status(launch_decode(a, mk, mv, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rtp_status rtp_selftest_bounded_wait(unsigned limit_ms, void* stream) {
+  if (limit_ms < 1 || limit_ms > 10000) return RTP_ERR_INVALID_ARG;
+  uint32_t* st = status_word(current_device());
+  if (!st) return RTP_ERR_NO_MEMORY;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  bounded_wait_selftest_kernel<<<1, 32, 0, s>>>(st, static_cast<uint64_t>(limit_ms) * 1000000ull);
+  if (cudaGetLastError() != cudaSuccess) return RTP_ERR_CUDA;
+  return rtp_last_device_status(stream);
 }
 
 rtp_status rtp_last_device_status(void* stream) {

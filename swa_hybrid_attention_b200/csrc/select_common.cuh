@@ -60,27 +60,42 @@ __device__ inline int select_blocks(const float (&q)[kRank], const float* C, int
     for (int e = tid; e < kmax; e += kSelThreads) out[e] = e < n ? e : -1;
     return n;
   }
-  // 1. scores -> order keys (fixed fma order over the 16 ranks)
-  for (int x = tid; x < ncand; x += kSelThreads) {
-    const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + 1) * kRank);
-    const float4 a0 = __ldg(c4), a1 = __ldg(c4 + 1), a2 = __ldg(c4 + 2), a3 = __ldg(c4 + 3);
-    float s = q[0] * a0.x;
-    s = fmaf(q[1], a0.y, s);
-    s = fmaf(q[2], a0.z, s);
-    s = fmaf(q[3], a0.w, s);
-    s = fmaf(q[4], a1.x, s);
-    s = fmaf(q[5], a1.y, s);
-    s = fmaf(q[6], a1.z, s);
-    s = fmaf(q[7], a1.w, s);
-    s = fmaf(q[8], a2.x, s);
-    s = fmaf(q[9], a2.y, s);
-    s = fmaf(q[10], a2.z, s);
-    s = fmaf(q[11], a2.w, s);
-    s = fmaf(q[12], a3.x, s);
-    s = fmaf(q[13], a3.y, s);
-    s = fmaf(q[14], a3.z, s);
-    s = fmaf(q[15], a3.w, s);
-    keys[x] = order_key(s);
+  // 1. scores -> order keys (fixed fma order over the 16 ranks).  Four
+  // candidates per round with all their loads issued before any use, so a
+  // thread keeps 16 independent 16-byte loads in flight.
+  auto score = [&](const float4 (&v)[4]) {
+    float s = q[0] * v[0].x;
+    s = fmaf(q[1], v[0].y, s);
+    s = fmaf(q[2], v[0].z, s);
+    s = fmaf(q[3], v[0].w, s);
+    s = fmaf(q[4], v[1].x, s);
+    s = fmaf(q[5], v[1].y, s);
+    s = fmaf(q[6], v[1].z, s);
+    s = fmaf(q[7], v[1].w, s);
+    s = fmaf(q[8], v[2].x, s);
+    s = fmaf(q[9], v[2].y, s);
+    s = fmaf(q[10], v[2].z, s);
+    s = fmaf(q[11], v[2].w, s);
+    s = fmaf(q[12], v[3].x, s);
+    s = fmaf(q[13], v[3].y, s);
+    s = fmaf(q[14], v[3].z, s);
+    s = fmaf(q[15], v[3].w, s);
+    return s;
+  };
+  for (int x0 = tid; x0 < ncand; x0 += 4 * kSelThreads) {
+    float4 v[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int x = min(x0 + u * kSelThreads, ncand - 1);
+      const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + 1) * kRank);
+#pragma unroll
+      for (int w = 0; w < 4; ++w) v[u][w] = __ldg(c4 + w);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int x = x0 + u * kSelThreads;
+      if (x < ncand) keys[x] = order_key(score(v[u]));
+    }
   }
   __syncthreads();
 

@@ -103,14 +103,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for the phase with the given parity to complete.  Returns false when
 // the wait gave up (time limit) or when *abort became non-zero (another role
 // of the same CTA gave up first).  On a time-out the status word is flagged.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* status) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* status,
+                                          uint64_t limit_ns = RTP_WAIT_LIMIT_NS) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (abort && *abort) return false;
-    if (globaltimer_ns() - t0 > RTP_WAIT_LIMIT_NS) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       flag_error(status, RTP_DEVERR_TIMEOUT);
       if (abort) *abort = 1;
       return false;

@@ -60,6 +60,7 @@ def _load() -> ctypes.CDLL:
         "rtp_sparse_decode": (I, [cfgp, P, I, P, P, P, P, P, P, P, S, P, P, P]),
         "rtp_sparse_decode_noalloc": (I, [cfgp, P, I, P, P, P, P, P, P, P, P, P]),
         "rtp_last_device_status": (I, [P]),
+        "rtp_selftest_bounded_wait": (I, [ctypes.c_uint, P]),
         "rtp_status_str": (ctypes.c_char_p, [I]),
         "rtp_version": (I, []),
     }
@@ -74,7 +75,7 @@ _lib = _load()
 EXPORTED = ("rtp_route_heads", "rtp_plan_destroy", "rtp_plan_num_sparse", "rtp_plan_num_items",
             "rtp_plan_sparse_heads", "rtp_plan_work_items", "rtp_indexer_project", "rtp_block_select",
             "rtp_hybrid_prefill", "rtp_decode_workspace_bytes", "rtp_sparse_decode", "rtp_sparse_decode_noalloc",
-            "rtp_last_device_status",
+            "rtp_last_device_status", "rtp_selftest_bounded_wait",
             "rtp_status_str", "rtp_version")
 
 
@@ -214,6 +215,11 @@ def rtp_sparse_decode_noalloc(cfg: AttnConfig, kinds, cache_len: int, q, kcache,
 
 def rtp_last_device_status(stream=None) -> int:
     return int(_lib.rtp_last_device_status(_stream(stream)))
+
+
+def rtp_selftest_bounded_wait(limit_ms: int, stream=None) -> int:
+    """Runs the bounded-wait self-test; returns the status (RTP_ERR_TIMEOUT expected)."""
+    return int(_lib.rtp_selftest_bounded_wait(int(limit_ms), _stream(stream)))
 
 
 def rtp_version() -> int:
