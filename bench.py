@@ -90,6 +90,19 @@ def indexer_bytes(w, kinds) -> float:
     return float(ns * (w.seq * 128 * 2 * (1 + w.group) + 2 * nb * 16 * 4))
 
 
+def prefill_traffic(w):
+    """DRAM bytes per launch of the prefill kernel for the 1M-token layer, from
+    the committed ncu summary (captured at 128K and scaled by length); None
+    for any other length."""
+    p = os.path.join(ROOT, "profiles", "hybrid_prefill_kernel.md")
+    if w.seq != 1048576 or not os.path.exists(p):
+        return None
+    for line in open(p):
+        if line.startswith("prefill_traffic_bytes_per_launch_1m:"):
+            return float(line.split(":")[1])
+    return None
+
+
 def load_peaks() -> tuple[dict, str]:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -520,11 +533,7 @@ def run_ours(args, rank, world, local):
     value = world * algo / (step_ms * 1e-3) / 1e12
     achieved = execd / (pre_ms * 1e-3) / 1e12
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
-    traffic = None
-    tp = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(tp):
-        with open(tp) as f:
-            traffic = json.load(f).get("hybrid_prefill_kernel_bytes_per_launch")
+    traffic = prefill_traffic(w)
     extra = {}
     if not args.no_e2e:
         extra["e2e"] = time_e2e(rtp, w, res, max(2, min(args.steps, 3)), device)

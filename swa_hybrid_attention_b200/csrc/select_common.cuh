@@ -106,16 +106,9 @@ __device__ inline int select_blocks(const float (&q)[kRank], const float* C, int
     const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
     for (int e = tid; e < 256; e += kSelThreads) sh.hist[e] = 0;
     __syncthreads();
-    // Keys of similar magnitude share their top bytes, so lanes of a warp
-    // mostly hit the same bin: aggregate equal bins per warp (one atomic per
-    // distinct bin) instead of serialising 32 atomics on one address.
-    for (int x0 = tid - (tid & 31); x0 < ncand; x0 += kSelThreads) {
-      const int x = x0 + (tid & 31);
-      const uint32_t k = x < ncand ? keys[x] : 0u;
-      const bool hit = x < ncand && (k & hi_mask) == prefix;
-      const uint32_t bin = hit ? ((k >> shift) & 255u) : 256u;
-      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
-      if (hit && (tid & 31) == __ffs(peers) - 1) atomicAdd(&sh.hist[bin], static_cast<uint32_t>(__popc(peers)));
+    for (int x = tid; x < ncand; x += kSelThreads) {
+      const uint32_t k = keys[x];
+      if ((k & hi_mask) == prefix) atomicAdd(&sh.hist[(k >> shift) & 255u], 1u);
     }
     __syncthreads();
     if (tid < 32) {
