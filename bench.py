@@ -379,14 +379,18 @@ def time_decode(rtp, steps, device):
     o = torch.empty_like(d["q"])
     stream = torch.cuda.current_stream()
     args = (cfg, kinds, Lc, d["q"], d["kcache"], d["vcache"], C, d["proj"], o, ws, ws_bytes)
-    # L2 flush buffer (the selected K/V of one step, 95 MB, would otherwise stay in the 126 MB L2)
+    # L2 flush (the selected K/V of one step, 95 MB, would otherwise stay in the 126 MB L2): write
+    # 256 MB, then read another 256 MB so that L2 holds clean lines of unrelated data; with the
+    # write alone L2 would start the step full of dirty lines whose write-back the step would pay.
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
+    flush_read = torch.ones(64 * 1024 * 1024, dtype=torch.float32, device=device)
     for _ in range(5):
         rtp.rtp_sparse_decode(*args, stream=stream)
     torch.cuda.synchronize()
     times = []
     for _ in range(steps):
         flush.zero_()
+        flush_read.sum()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -404,7 +408,7 @@ def time_decode(rtp, steps, device):
     bytes_ = w.batch * (keys * 128 * 2 * 2 + ns * (Lc // w.block) * 16 * 4 + w.n_q_heads * 128 * 2 * 2)
     flops = w.batch * keys * G * 4 * 128
     return {"workload": w.name, "ms_per_step": ms, "algorithmic_bytes": bytes_, "gb_s": bytes_ / (ms * 1e-3) / 1e9,
-            "tflops_effective": flops / (ms * 1e-3) / 1e12, "l2": "flushed (256 MB write) before each step",
+            "tflops_effective": flops / (ms * 1e-3) / 1e12, "l2": "flushed before each step (256 MB write, then 256 MB read)",
             "launches_per_step": 3, "status": rtp.status_str(status)}
 
 

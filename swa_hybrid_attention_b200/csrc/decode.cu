@@ -9,19 +9,28 @@
 // with t = the block of the new token), and exact softmax attention runs
 // over the selected keys; streaming heads attend to the last `window` keys.
 //
-// Three launches on the caller's stream:
-//  1. decode_select_kernel  (seq, retrieval head): summary + selection.
-//  2. decode_attn_kernel    (split, kv head, seq): one span of <= 128 keys per
-//     CTA.  K and V rows of the span are contiguous in the cache and are
-//     brought into shared memory with two bulk copies on an mbarrier; QK runs
-//     one key per thread, PV one output dimension per thread, for all G query
-//     heads of the group at once (GQA: each K/V byte is read once per group).
-//     Writes an unnormalised partial (m, l, o) per head in the log2 domain.
-//  3. decode_combine_kernel (q head, seq): log-sum-exp merge of the splits.
-// The step is bound by HBM reads of the selected K/V.
+// Three launches on the caller's stream, chained by programmatic dependent
+// launch so each may start while its predecessor finishes:
+//  1. decode_select_kernel  (retrieval head, sequence): summary + selection.
+//  2. decode_attn_kernel    persistent, one CTA per SM.  The keys to visit are
+//     cut into spans of <= 128 (one selected block, or 128 consecutive keys
+//     of a window/full head) in two lists, window/full heads first; each CTA
+//     takes a contiguous range of each list, so it works through its window
+//     spans while the selection is still running and only then waits for it.
+//     A producer warp streams the spans' K and V through a 3-stage TMA ring;
+//     four consumer warps run S = Q K^T (each warp 32 keys), one softmax per
+//     span with a running maximum shared across the warps, and O += P V
+//     (each warp 32 output dimensions), on tensor cores (mma.sync m16n8k16,
+//     the group's query heads as the M rows: each K/V byte is read once per
+//     group).  Consecutive spans of one (sequence, head) merge online; a CTA
+//     writes one partial (m, l, o) per run of spans.
+//  3. decode_combine_kernel (query head, sequence): log-sum-exp merge of the
+//     runs of the head.
+// The step is bound by HBM reads of the selected K/V and the windows.
 
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "internal.cuh"
@@ -31,100 +40,394 @@
 namespace rtp {
 namespace {
 
-constexpr int kAttnThreads = 128;
-constexpr int kMaxGroup = 16;
+constexpr int kConsumerWarps = 4;
+constexpr int kAttnThreads = 32 * (kConsumerWarps + 1);  // + one producer warp
+constexpr int kCombineThreads = 128;
+constexpr int kRingStages = 3;
+constexpr uint32_t kHalfSpanBytes = 128 * 128 * 2;  // K (or V) of one span
+constexpr int kPRowElems = 128 + 8;  // P row pitch (bf16): 272 bytes, conflict-free
 
-__global__ void __launch_bounds__(kSelThreads) decode_select_kernel(const DecodeArgs a) {
-  extern __shared__ uint32_t keys[];
-  __shared__ SelectScratch sh;
-  __shared__ float qsum[kHeadDim];
-  __shared__ float part16[16][kRank];
-  const int kvh = blockIdx.x, b = blockIdx.y;
-  // The attention launch that follows may start now: its streaming-head
-  // CTAs do not need the selection, its retrieval-head CTAs wait for it.
-  griddep_launch_dependents();
-  if (a.kind[kvh] != KIND_SPARSE) return;
-  // qbar = sum_h P^T q_h = P^T (sum_h q_h): sum the group's queries (fixed
-  // head order), then project with all threads: thread (j, c) takes dims
-  // [8j, 8j+8) of output c, and the 16 partials are added in a fixed order.
-  const int tid = threadIdx.x;
-  if (tid < kHeadDim) {
-    const __nv_bfloat16* qg = a.q + (static_cast<size_t>(b) * a.n_q_heads + kvh * a.group) * kHeadDim + tid;
-    float sq = 0.f;
-    for (int h = 0; h < a.group; ++h) sq += __bfloat162float(qg[h * kHeadDim]);
-    qsum[tid] = sq;
-  }
-  __syncthreads();
-  {
-    const int j = tid >> 4, c = tid & 15;
-    float sp = 0.f;
-#pragma unroll
-    for (int d = 8 * j; d < 8 * j + 8; ++d) sp = fmaf(__ldg(a.proj + d * kRank + c), qsum[d], sp);
-    part16[j][c] = sp;
-  }
-  __syncthreads();
-  float q[kRank];
-#pragma unroll
-  for (int c = 0; c < kRank; ++c) {
-    float s = 0.f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) s += part16[j][c];
-    q[c] = s;
-  }
-  const int t = (a.cache_len - 1) / a.block;
-  const float* C = a.centroids + (static_cast<size_t>(b) * a.n_kv_heads + kvh) * a.nbc * kRank;
-  int32_t* out = a.sel + (static_cast<size_t>(b) * a.n_kv_heads + kvh) * a.kmax;
-  const int n = select_blocks(q, C, t, a.topk, a.n_local, a.kmax, keys, sh, out);
-  if (tid == 0) a.cnt[static_cast<size_t>(b) * a.n_kv_heads + kvh] = n;
+// ---------------------------------------------------------------- selection
+// One cluster of kSelCluster CTAs per (retrieval head, sequence).  CTA r of
+// the cluster scores its slice of the candidate blocks (one or two per
+// thread, one round of loads) and keeps its local top-k (radix select +
+// ordered compaction); the union of the local top-k lists holds the global
+// top-k.  After a cluster barrier CTA 0 gathers the lists from its peers'
+// shared memory, in slice order (= block order), and selects the final top-k
+// by the same rule, so ties still go to the lower block index.
+constexpr int kSelCluster = 8;
+constexpr int kDecSelThreads = 128;
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+// (No memory clobber: the loads of a gather may all be in flight together;
+// they are ordered after the cluster barrier, whose asm clobbers memory.)
+__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+// All threads of every CTA in the cluster: prior shared-memory writes become
+// visible to the peers (release/acquire).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Key span of split s for (b, kvh): [key0, key0 + nk).  nk <= 0: no work.
-__device__ __forceinline__ void span_of(const DecodeArgs& a, int b, int kvh, int s, int& key0, int& nk) {
-  const int kind = a.kind[kvh];
-  if (kind == KIND_SPARSE) {
-    const size_t bk = static_cast<size_t>(b) * a.n_kv_heads + kvh;
-    const int cnt = a.cnt[bk];
-    if (s >= cnt || s >= a.kmax) {
-      nk = 0;
-      key0 = 0;
-      return;
+__device__ __forceinline__ uint64_t ld_cluster_u64(uint32_t addr) {
+  uint64_t v;
+  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr));
+  return v;
+}
+
+// Top-k for k <= 32 on bitonic networks over the lanes of a warp.  A
+// candidate is the 64-bit key (order_key(score) << 32) | ~block: keys are
+// unique, and a larger key means a larger score or, for equal scores, a
+// lower block index -- the selection order.  0 is below every candidate.
+__device__ __forceinline__ uint64_t cand_key(float score, int block) {
+  return (static_cast<uint64_t>(order_key(score)) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(block));
+}
+__device__ __forceinline__ int cand_block(uint64_t key) { return static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key)); }
+
+// Two independent bitonic sorts of 32 keys (one per lane each), descending.
+__device__ __forceinline__ void warp_sort2_desc(uint64_t& x, uint64_t& y) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const uint64_t ox = __shfl_xor_sync(0xffffffffu, x, stride);
+      const uint64_t oy = __shfl_xor_sync(0xffffffffu, y, stride);
+      const bool take_max = ((lane & stride) == 0) == ((lane & size) == 0);
+      x = take_max ? max(x, ox) : min(x, ox);
+      y = take_max ? max(y, oy) : min(y, oy);
     }
-    int blk = a.sel[bk * a.kmax + s];
-    const int t = (a.cache_len - 1) / a.block;
-    if (blk < 0 || blk > t) {
-      flag_error(a.status, RTP_DEVERR_INDEX);
-      nk = 0;
-      key0 = 0;
-      return;
-    }
-    key0 = blk * a.block;
-    nk = min(a.block, a.cache_len - key0);
-  } else {
-    const int start = (kind == KIND_SWA) ? max(0, a.cache_len - a.window) : 0;
-    key0 = start + 128 * s;
-    nk = min(128, a.cache_len - key0);
   }
+}
+
+// x and y each sorted descending over the lanes: the 32 largest of the 64,
+// sorted descending (bitonic split against the reversed y, then merge).
+__device__ __forceinline__ uint64_t warp_merge_top32(uint64_t x, uint64_t y) {
+  const int lane = threadIdx.x & 31;
+  uint64_t v = max(x, __shfl_sync(0xffffffffu, y, 31 - lane));
+#pragma unroll
+  for (int stride = 16; stride > 0; stride >>= 1) {
+    const uint64_t o = __shfl_xor_sync(0xffffffffu, v, stride);
+    v = (lane & stride) == 0 ? max(v, o) : min(v, o);
+  }
+  return v;
+}
+
+// Bitonic sort of 32 values (one per lane), ascending.
+__device__ __forceinline__ uint32_t warp_sort_asc(uint32_t v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const uint32_t o = __shfl_xor_sync(0xffffffffu, v, stride);
+      const bool take_min = ((lane & stride) == 0) == ((lane & size) == 0);
+      v = take_min ? min(v, o) : max(v, o);
+    }
+  }
+  return v;
+}
+
+__global__ void __launch_bounds__(kDecSelThreads, 8) __cluster_dims__(kSelCluster, 1, 1)
+    decode_select_kernel(const __grid_constant__ DecodeArgs a) {
+  // dynamic: keys[chunk] | lkey[topk] | lidx[topk] | ukey[kSelCluster*topk] | uidx[kSelCluster*topk]
+  extern __shared__ uint32_t dsel[];
+  __shared__ SelectScratchT<kDecSelThreads> sh;
+  __shared__ float qpart[kDecSelThreads / 32][kRank];
+  __shared__ int n_kept;
+  __shared__ uint64_t wlist[kDecSelThreads / 32][32];  // per-warp top-32 lists
+  __shared__ uint64_t cta_top[32];                      // this CTA's top-32, read by CTA 0
+  const int kvh = blockIdx.x / kSelCluster, b = blockIdx.y;
+  // The attention launch that follows may start now: its window-head spans
+  // do not need the selection; its retrieval spans wait for this grid.
+  griddep_launch_dependents();
+  if (a.kind[kvh] != KIND_SPARSE) return;  // the whole cluster leaves
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t rank = cluster_ctarank();
+  const int t = (a.cache_len - 1) / a.block;
+  const int ncand = max(0, t - a.n_local);  // candidates are blocks 1..ncand
+  const size_t bk = static_cast<size_t>(b) * a.n_kv_heads + kvh;
+  int32_t* out = a.sel + bk * a.kmax;
+  if (ncand <= a.topk) {  // every block 0..t (uniform over the cluster)
+    if (rank == 0) {
+      for (int e = tid; e < a.kmax; e += kDecSelThreads) out[e] = e <= t ? e : -1;
+      if (tid == 0) a.cnt[bk] = t + 1;
+    }
+    return;
+  }
+  if (a.topk == 0) {  // sink and local blocks only
+    if (rank == 0) {
+      for (int e = tid; e < a.kmax; e += kDecSelThreads)
+        out[e] = e == 0 ? 0 : (e <= a.n_local ? t - a.n_local + e : -1);
+      if (tid == 0) a.cnt[bk] = 1 + a.n_local;
+    }
+    return;
+  }
+  const int chunk = (ncand + kSelCluster - 1) / kSelCluster;
+  const int lo = static_cast<int>(rank) * chunk;  // candidate x -> block x + 1
+  const int nl = max(0, min(ncand, lo + chunk) - lo);
+  uint32_t* keys = dsel;
+  uint32_t* lkey = keys + chunk;
+  uint32_t* lidx = lkey + a.topk;
+  uint32_t* ukey = lidx + a.topk;
+  uint32_t* uidx = ukey + kSelCluster * a.topk;
+  const float* C = a.centroids + bk * a.nbc * kRank;
+
+  // Loads first: this thread's first two centroid rows, its query dimension
+  // of the group's heads and its row of the projector.
+  float4 cv[2][4];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const int x = min(lo + min(tid + u * kDecSelThreads, max(nl - 1, 0)), ncand - 1);  // a valid row
+    const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + 1) * kRank);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) cv[u][w] = __ldg(c4 + w);
+  }
+  float4 pr[4];
+  {
+    const float4* p4 = reinterpret_cast<const float4*>(a.proj + tid * kRank);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) pr[w] = __ldg(p4 + w);
+  }
+  // qbar = P^T (sum_h q_h): thread d sums dimension d over the group's heads
+  // (fixed order), multiplies by row d of P, and the 128 rows are added by a
+  // warp butterfly and then over the four warps (fixed order).
+  float q[kRank];
+  {
+    const __nv_bfloat16* qg = a.q + (static_cast<size_t>(b) * a.n_q_heads + kvh * a.group) * kHeadDim + tid;
+    float qs = 0.f;
+    for (int h = 0; h < a.group; ++h) qs += __bfloat162float(qg[h * kHeadDim]);
+    const float prow[kRank] = {pr[0].x, pr[0].y, pr[0].z, pr[0].w, pr[1].x, pr[1].y, pr[1].z, pr[1].w,
+                               pr[2].x, pr[2].y, pr[2].z, pr[2].w, pr[3].x, pr[3].y, pr[3].z, pr[3].w};
+#pragma unroll
+    for (int c = 0; c < kRank; ++c) {
+      float v = prow[c] * qs;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (lane == 0) qpart[warp][c] = v;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int c = 0; c < kRank; ++c) q[c] = (qpart[0][c] + qpart[1][c]) + (qpart[2][c] + qpart[3][c]);
+  }
+  if (a.topk <= 32) {
+    // Warp w holds candidates x0 + 32w + lane and x0 + 128 + 32w + lane of
+    // each round; it keeps a running top-32 (sorted descending) of them.
+    uint64_t best = 0;
+    for (int x0 = 0; x0 < nl; x0 += 2 * kDecSelThreads) {
+      if (x0 > 0) {
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int x = lo + min(x0 + tid + u * kDecSelThreads, nl - 1);
+          const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + 1) * kRank);
+#pragma unroll
+          for (int w = 0; w < 4; ++w) cv[u][w] = __ldg(c4 + w);
+        }
+      }
+      const int xa = x0 + tid, xb = x0 + tid + kDecSelThreads;
+      uint64_t ka = xa < nl ? cand_key(score16(q, cv[0]), lo + xa + 1) : 0ull;
+      uint64_t kb = xb < nl ? cand_key(score16(q, cv[1]), lo + xb + 1) : 0ull;
+      warp_sort2_desc(ka, kb);
+      const uint64_t top = warp_merge_top32(ka, kb);
+      best = x0 == 0 ? top : warp_merge_top32(best, top);
+    }
+    // the four warps' lists -> the CTA's top-32
+    wlist[warp][lane] = best;
+    __syncthreads();
+    uint64_t v = 0;
+    if (warp < 2) v = warp_merge_top32(wlist[2 * warp][lane], wlist[2 * warp + 1][lane]);
+    __syncthreads();
+    if (warp < 2) wlist[warp][lane] = v;
+    __syncthreads();
+    if (warp == 0) cta_top[lane] = warp_merge_top32(wlist[0][lane], wlist[1][lane]);
+    cluster_sync();  // every CTA's top-32 is complete and visible to CTA 0
+    if (rank != 0) {
+      cluster_sync();  // CTA 0 has read the list
+      return;
+    }
+    // CTA 0: warp w merges the lists of CTAs 2w and 2w+1, then two rounds
+    // of merges in shared memory.
+    v = warp_merge_top32(ld_cluster_u64(map_to_rank(smem_u32(&cta_top[lane]), 2 * warp)),
+                         ld_cluster_u64(map_to_rank(smem_u32(&cta_top[lane]), 2 * warp + 1)));
+    wlist[warp][lane] = v;
+    __syncthreads();
+    cluster_sync();  // the peers may leave: their lists have been read
+    if (warp < 2) v = warp_merge_top32(wlist[2 * warp][lane], wlist[2 * warp + 1][lane]);
+    __syncthreads();
+    if (warp < 2) wlist[warp][lane] = v;
+    __syncthreads();
+    if (warp == 0) {
+      v = warp_merge_top32(wlist[0][lane], wlist[1][lane]);
+      // the first topk keys are the selection; put their blocks in order
+      const uint32_t blk = lane < a.topk ? static_cast<uint32_t>(cand_block(v)) : 0xFFFFFFFFu;
+      const uint32_t sorted = warp_sort_asc(blk);
+      if (lane < a.topk) out[1 + lane] = static_cast<int32_t>(sorted);
+    }
+    if (tid == 0) out[0] = 0;
+    for (int m = tid; m < a.n_local; m += kDecSelThreads) out[1 + a.topk + m] = t - a.n_local + 1 + m;
+    for (int e = 1 + a.topk + a.n_local + tid; e < a.kmax; e += kDecSelThreads) out[e] = -1;
+    if (tid == 0) a.cnt[bk] = 1 + a.topk + a.n_local;
+    return;
+  }
+  // k > 32: radix select.  Scores of this CTA's slice -> order keys.
+  for (int x0 = 0; x0 < nl; x0 += 2 * kDecSelThreads) {
+    if (x0 > 0) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int x = lo + min(x0 + tid + u * kDecSelThreads, nl - 1);
+        const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + 1) * kRank);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) cv[u][w] = __ldg(c4 + w);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int x = x0 + tid + u * kDecSelThreads;
+      if (x < nl) keys[x] = order_key(score16(q, cv[u]));
+    }
+  }
+  __syncthreads();
+  // Local top-k of the slice (all of it if it is small).
+  if (nl <= a.topk) {
+    for (int x = tid; x < nl; x += kDecSelThreads) {
+      lkey[x] = keys[x];
+      lidx[x] = static_cast<uint32_t>(lo + x + 1);
+    }
+    if (tid == 0) n_kept = nl;
+  } else {
+    uint32_t T, need;
+    radix_threshold<kDecSelThreads>(keys, nl, a.topk, sh, T, need);
+    ordered_select<kDecSelThreads>(keys, nl, T, need, sh, [&](int r, int x) {
+      lkey[r] = keys[x];
+      lidx[r] = static_cast<uint32_t>(lo + x + 1);
+    });
+    if (tid == 0) n_kept = a.topk;
+  }
+  cluster_sync();  // local lists complete and visible to CTA 0
+  if (rank == 0) {
+    int off[kSelCluster + 1];
+    off[0] = 0;
+#pragma unroll
+    for (int r = 0; r < kSelCluster; ++r)
+      off[r + 1] = off[r] + static_cast<int>(ld_cluster_u32(map_to_rank(smem_u32(&n_kept), r)));
+    for (int e0 = 0; e0 < a.topk; e0 += kDecSelThreads) {
+      const int e = e0 + tid;
+      uint32_t vk[kSelCluster], vi[kSelCluster];
+#pragma unroll
+      for (int r = 0; r < kSelCluster; ++r) {  // all loads first, then the stores
+        const bool in = e < off[r + 1] - off[r];
+        vk[r] = in ? ld_cluster_u32(map_to_rank(smem_u32(lkey + e), r)) : 0u;
+        vi[r] = in ? ld_cluster_u32(map_to_rank(smem_u32(lidx + e), r)) : 0u;
+      }
+#pragma unroll
+      for (int r = 0; r < kSelCluster; ++r) {
+        if (e < off[r + 1] - off[r]) {
+          ukey[off[r] + e] = vk[r];
+          uidx[off[r] + e] = vi[r];
+        }
+      }
+    }
+    __syncthreads();
+    cluster_sync();  // the peers may leave: their lists have been read
+    const int U = off[kSelCluster];
+    uint32_t T, need;
+    radix_threshold<kDecSelThreads>(ukey, U, a.topk, sh, T, need);
+    ordered_select<kDecSelThreads>(ukey, U, T, need, sh,
+                                   [&](int r, int x) { out[1 + r] = static_cast<int32_t>(uidx[x]); });
+    if (tid == 0) out[0] = 0;
+    for (int m = tid; m < a.n_local; m += kDecSelThreads) out[1 + a.topk + m] = t - a.n_local + 1 + m;
+    for (int e = 1 + a.topk + a.n_local + tid; e < a.kmax; e += kDecSelThreads) out[e] = -1;
+    if (tid == 0) a.cnt[bk] = 1 + a.topk + a.n_local;
+  } else {
+    cluster_sync();
+  }
+}
+
+// Dynamic shared memory of the selection kernel (host side).
+size_t decode_select_smem(const DecodeArgs& a) {
+  if (a.topk <= 32) return 0;  // static arrays suffice
+  const int t = (a.cache_len - 1) / a.block;
+  const int ncand = std::max(0, t - a.n_local);
+  const int chunk = (ncand + kSelCluster - 1) / kSelCluster;
+  return (static_cast<size_t>(chunk) + 2 * static_cast<size_t>(a.topk) * (1 + kSelCluster)) * sizeof(uint32_t);
+}
+
+// ---------------------------------------------------------------- schedule
+__device__ __forceinline__ int list_of(const DecodeArgs& a, int kvh) { return a.kind[kvh] == KIND_SPARSE ? 1 : 0; }
+
+// Spans of one (sequence, head): kmax selected blocks, or the visible keys of
+// a window/full head in 128-key pieces.
+__device__ __forceinline__ int n_spans_of(const DecodeArgs& a, int kvh) {
+  const int kind = a.kind[kvh];
+  if (kind == KIND_SPARSE) return a.kmax;
+  const int len = kind == KIND_SWA ? min(a.cache_len, a.window) : a.cache_len;
+  return (len + 127) / 128;
+}
+
+__device__ __forceinline__ long list_len(const DecodeArgs& a, int list) {
+  return static_cast<long>(a.batch) * a.per_b[list];
+}
+
+// First span of CTA c in a list of length n: floor(c * n / n_ctas).
+__device__ __forceinline__ long range_lo(const DecodeArgs& a, long n, int c) {
+  return static_cast<long>((static_cast<long long>(c) * n) / a.n_ctas);
+}
+
+// The CTA whose range holds span x: the largest c with range_lo(c) <= x.
+__device__ __forceinline__ int owner_of(const DecodeArgs& a, long n, long x) {
+  return static_cast<int>(((static_cast<long long>(x) + 1) * a.n_ctas - 1) / n);
+}
+
+// Span x of a list -> (sequence, head, span index within the head).
+__device__ __forceinline__ void locate(const DecodeArgs& a, int list, long x, int& b, int& kvh, int& s) {
+  b = static_cast<int>(x / a.per_b[list]);
+  const int r = static_cast<int>(x - static_cast<long>(b) * a.per_b[list]);
+  kvh = 0;
+  s = 0;
+  for (int h = 0; h < a.n_kv_heads; ++h) {
+    if (list_of(a, h) != list) continue;
+    const int off = a.span_off[h];
+    if (r >= off && r < off + n_spans_of(a, h)) {
+      kvh = h;
+      s = r - off;
+      return;
+    }
+  }
+}
+
+// Partial-result slot of the run that starts at span x of a list.
+__device__ __forceinline__ float* run_partial(const DecodeArgs& a, int list, long x) {
+  const long slot = (list == 1 ? list_len(a, 0) : 0) + x;
+  return a.partial + slot * a.group * kPartStride;
 }
 
 // --------------------------------------------------------------- attention
-// One CTA per (span of <= 128 keys, KV head, sequence); 4 warps, warp w owns
-// keys [32w, 32w+32) of the span.  K and V of the span arrive by TMA in
-// 128-byte-swizzled 64x64 boxes (rows past the cache read as zero).  Per warp,
-// tensor-core MMAs (m16n8k16, bf16 -> fp32) with the group's query heads as
-// the 16 M rows (rows >= G are zero):
-//   S = Q K^T   (A = Q fragments in registers, B = K via ldmatrix),
-//   P = exp2(S * scale*log2e - m_warp) kept in registers as the A operand,
-//   O = P V     (B = V via ldmatrix.trans).
-// The four warps' (m, l, O) are merged in shared memory (reusing the K
-// buffer) and the CTA writes one partial per head.
 struct __align__(1024) DecSmem {
-  uint8_t k[32768];  // 128 keys x 128 dims, two 64-column swizzled chunks
-  uint8_t v[32768];
-  uint64_t bar;
-  float wm[4][16], wl[4][16];
-  int ok;
+  uint8_t k[kRingStages][kHalfSpanBytes];  // 128 keys x 128 dims: two 64-column SW128 chunks
+  uint8_t v[kRingStages][kHalfSpanBytes];
+  __nv_bfloat16 p[16][kPRowElems];         // P of the current span: 16 rows x 128 keys
+  uint64_t k_full[kRingStages], v_full[kRingStages], empty[kRingStages];
+  int k_ok, v_ok;                          // results of the consumers' K / V waits
+  int nk[kRingStages];                     // valid keys of the span in each stage
+  float red_m[kConsumerWarps][16];
+  float red_l[kConsumerWarps][16];
+  int abort_flag;
 };
-constexpr size_t kDecSmemBytes = sizeof(DecSmem) + 1024;
+constexpr size_t kDecSmemBytes = sizeof(DecSmem) + 1024;  // + alignment slack
+static_assert(kDecSmemBytes <= 210 * 1024, "leave room for a selection CTA on the same SM");
 
 __device__ __forceinline__ uint32_t sw128(uint32_t base, int row, int dim) {
   return base + (dim >> 6) * 16384 + row * 128 + ((((dim & 63) >> 3) ^ (row & 7)) << 4);
@@ -148,240 +451,404 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const __grid_constant__ CUtensorMap mk,
-                                                                    const __grid_constant__ CUtensorMap mv,
-                                                                    const DecodeArgs a) {
-  extern __shared__ uint8_t dsmem[];
-  DecSmem& sm = *reinterpret_cast<DecSmem*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
-  const int s = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = lane >> 2, c = lane & 3;
-  const int G = a.group;
-  // Only retrieval heads read the selection written by the preceding launch.
-  if (a.kind[kvh] == KIND_SPARSE) griddep_wait();
-  float* part = a.partial + ((static_cast<size_t>(b) * a.n_kv_heads + kvh) * a.max_splits + s) * G * kPartStride;
-  int key0, nk;
-  span_of(a, b, kvh, s, key0, nk);
-  if (nk <= 0) {
-    for (int h = 0; h < G; ++h) {
-      if (tid == 0) {
-        part[h * kPartStride + 0] = -INFINITY;
-        part[h * kPartStride + 1] = 0.f;
-      }
-      part[h * kPartStride + 4 + tid] = 0.f;
-    }
-    return;
-  }
-  const uint32_t ks = smem_u32(sm.k), vs = smem_u32(sm.v);
-  const int slab = b * a.n_kv_heads + kvh;
-  if (tid == 0) {
-    mbar_init(&sm.bar, 1);
-    fence_mbar_init();
-    mbar_arrive_expect_tx(&sm.bar, 65536);
-    for (int cc = 0; cc < 2; ++cc)
-      for (int hh = 0; hh < 2; ++hh) {
-        tma_load_3d(sm.k + cc * 16384 + hh * 8192, &mk, &sm.bar, 64 * cc, key0 + 64 * hh, slab);
-        tma_load_3d(sm.v + cc * 16384 + hh * 8192, &mv, &sm.bar, 64 * cc, key0 + 64 * hh, slab);
-      }
-  }
-  // Q as A fragments: rows g and g+8 are query heads g and g+8 of the group
-  // (zero beyond G); 8 K steps of 16 dims.
-  uint32_t qa[8][4];
-  {
-    const __nv_bfloat16* qb = a.q + (static_cast<size_t>(b) * a.n_q_heads + kvh * G) * kHeadDim;
-#pragma unroll
-    for (int kk = 0; kk < 8; ++kk) {
-      const int d0 = 16 * kk + 2 * c;
-      qa[kk][0] = g < G ? *reinterpret_cast<const uint32_t*>(qb + g * kHeadDim + d0) : 0u;
-      qa[kk][1] = g + 8 < G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * kHeadDim + d0) : 0u;
-      qa[kk][2] = g < G ? *reinterpret_cast<const uint32_t*>(qb + g * kHeadDim + d0 + 8) : 0u;
-      qa[kk][3] = g + 8 < G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * kHeadDim + d0 + 8) : 0u;
-    }
-  }
-  if (tid == 0) sm.ok = mbar_wait(&sm.bar, 0, nullptr, a.status) ? 1 : 0;
-  __syncwarp();
-  __syncthreads();
-  if (!sm.ok) return;
+// Named barrier over the 128 consumer threads (the producer warp never
+// joins it): a hardware barrier, so waiting threads take no issue slots.
+__device__ __forceinline__ void consumers_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsumerWarps) : "memory");
+}
 
-  // S = Q K^T over this warp's 32 keys: 4 n-tiles of 8 keys
-  float sacc[4][4];
-#pragma unroll
-  for (int n = 0; n < 4; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
-  const int kbase = 32 * warp;
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-#pragma unroll
-    for (int np = 0; np < 2; ++np) {
-      uint32_t r[4];
-      const int key = kbase + 16 * np + (lane >> 4) * 8 + (lane & 7);
-      const int dim = 16 * kk + ((lane >> 3) & 1) * 8;
-      ldsm_x4(sw128(ks, key, dim), r);
-      mma_bf16(sacc[2 * np], qa[kk], r[0], r[1]);
-      mma_bf16(sacc[2 * np + 1], qa[kk], r[2], r[3]);
+// Consumer thread 0 alone polls an mbarrier (bounded wait); after the next
+// consumers_sync every thread reads the shared result and, when the phase is
+// complete, tests it once itself (it completes at once), which gives each
+// thread acquire ordering for the data the phase guards.
+__device__ __forceinline__ bool checked_phase(uint64_t* bar, uint32_t parity, int ok) {
+  if (ok) mbar_test(bar, parity);
+  return ok != 0;
+}
+// Producer warp: walks the CTA's spans in consumption order and streams K
+// and V of each into the ring (four 64x64 boxes each, 128-byte swizzle; rows
+// past the cache read as zero).  Block indices of retrieval spans are read
+// 32 at a time by the whole warp; lane 0 waits for free stages and issues.
+__device__ __forceinline__ void attn_producer(DecSmem& sm, const CUtensorMap* mk, const CUtensorMap* mv,
+                                              const DecodeArgs& a, volatile int* abort) {
+  const int lane = lane_id();
+  const int tq = (a.cache_len - 1) / a.block;  // block of the new token
+  uint32_t issued = 0;
+  bool ok = true;
+  for (int list = 0; list < 2 && ok; ++list) {
+    const long n = list_len(a, list);
+    if (n == 0) continue;
+    if (list == 1) griddep_wait();  // the selection is complete and visible
+    const long hi = range_lo(a, n, blockIdx.x + 1);
+    long x = range_lo(a, n, blockIdx.x);
+    while (x < hi && ok) {
+      int b, kvh, s;
+      locate(a, list, x, b, kvh, s);
+      const long run_end = min(hi, x - s + n_spans_of(a, kvh));
+      const size_t bk = static_cast<size_t>(b) * a.n_kv_heads + kvh;
+      const int cnt = list == 1 ? max(0, min(a.cnt[bk], a.kmax)) : a.kmax + (1 << 30);
+      const int s_end = min(s + static_cast<int>(run_end - x), cnt);
+      const int start = a.kind[kvh] == KIND_SWA ? max(0, a.cache_len - a.window) : 0;
+      for (int s0 = s; s0 < s_end && ok; s0 += 32) {
+        int blk_l = 0;
+        if (list == 1 && s0 + lane < s_end) blk_l = a.sel[bk * a.kmax + s0 + lane];
+        const int m = min(32, s_end - s0);
+        for (int i = 0; i < m; ++i) {
+          int key0, nk;
+          if (list == 1) {
+            const int blk = __shfl_sync(0xffffffffu, blk_l, i);
+            if (blk < 0 || blk > tq) {  // not a valid selection: the span contributes nothing
+              if (lane == 0) flag_error(a.status, RTP_DEVERR_INDEX);
+              key0 = 0;
+              nk = 0;
+            } else {
+              key0 = blk * a.block;
+              nk = min(a.block, a.cache_len - key0);
+            }
+          } else {
+            key0 = start + 128 * (s0 + i);
+            nk = min(128, a.cache_len - key0);
+          }
+          const uint32_t st = issued % kRingStages, ph = (issued / kRingStages) & 1u;
+          int okl = 1;
+          if (lane == 0) {
+            okl = mbar_wait(&sm.empty[st], ph ^ 1u, abort, a.status) ? 1 : 0;
+            if (okl) {
+              sm.nk[st] = nk;
+              mbar_arrive_expect_tx(&sm.k_full[st], kHalfSpanBytes);
+              for (int cc = 0; cc < 2; ++cc)
+                for (int hh = 0; hh < 2; ++hh)
+                  tma_load_3d(sm.k[st] + cc * 16384 + hh * 8192, mk, &sm.k_full[st], 64 * cc, key0 + 64 * hh,
+                              static_cast<int>(bk));
+              mbar_arrive_expect_tx(&sm.v_full[st], kHalfSpanBytes);
+              for (int cc = 0; cc < 2; ++cc)
+                for (int hh = 0; hh < 2; ++hh)
+                  tma_load_3d(sm.v[st] + cc * 16384 + hh * 8192, mv, &sm.v_full[st], 64 * cc, key0 + 64 * hh,
+                              static_cast<int>(bk));
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+          if (!ok) break;
+          ++issued;
+        }
+      }
+      x = run_end;
     }
   }
-  // scale to log2 units, mask keys past the span, row maxima (rows g, g+8)
-  const float sl2 = a.scale_log2;
-  float mrow[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-  for (int n = 0; n < 4; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int key = kbase + 8 * n + 2 * c + (e & 1);
-      const float v = key < nk ? sacc[n][e] * sl2 : -INFINITY;
-      sacc[n][e] = v;
-      mrow[e >> 1] = fmaxf(mrow[e >> 1], v);
-    }
-#pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    mrow[rr] = fmaxf(mrow[rr], __shfl_xor_sync(0xffffffffu, mrow[rr], 1));
-    mrow[rr] = fmaxf(mrow[rr], __shfl_xor_sync(0xffffffffu, mrow[rr], 2));
-  }
-  const float muse[2] = {mrow[0] == -INFINITY ? 0.f : mrow[0], mrow[1] == -INFINITY ? 0.f : mrow[1]};
-  float lrow[2] = {0.f, 0.f};
-#pragma unroll
-  for (int n = 0; n < 4; ++n)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float p = exp2f(sacc[n][e] - muse[e >> 1]);
-      sacc[n][e] = p;
-      lrow[e >> 1] += p;
-    }
-#pragma unroll
-  for (int rr = 0; rr < 2; ++rr) {
-    lrow[rr] += __shfl_xor_sync(0xffffffffu, lrow[rr], 1);
-    lrow[rr] += __shfl_xor_sync(0xffffffffu, lrow[rr], 2);
-  }
-  // O = P V: 16 n-tiles of 8 dims, 2 K steps of 16 keys
-  float oacc[16][4];
-#pragma unroll
-  for (int n = 0; n < 16; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
-#pragma unroll
-  for (int kk = 0; kk < 2; ++kk) {
-    uint32_t pa[4];
-    pa[0] = pack_bf16x2(sacc[2 * kk][0], sacc[2 * kk][1]);
-    pa[1] = pack_bf16x2(sacc[2 * kk][2], sacc[2 * kk][3]);
-    pa[2] = pack_bf16x2(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1]);
-    pa[3] = pack_bf16x2(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3]);
-#pragma unroll
-    for (int dp = 0; dp < 8; ++dp) {
-      uint32_t r[4];
-      const int key = kbase + 16 * kk + ((lane >> 3) & 1) * 8 + (lane & 7);
-      const int dim = 16 * dp + (lane >> 4) * 8;
-      ldsm_x4_t(sw128(vs, key, dim), r);
-      mma_bf16(oacc[2 * dp], pa, r[0], r[1]);
-      mma_bf16(oacc[2 * dp + 1], pa, r[2], r[3]);
-    }
-  }
-  // merge the four warps (K buffer reused as [warp][row][dim] fp32)
-  __syncthreads();
-  float (*wo)[16][128] = reinterpret_cast<float (*)[16][128]>(sm.k);
-  if (c == 0) {
-    sm.wm[warp][g] = mrow[0];
-    sm.wm[warp][g + 8] = mrow[1];
-    sm.wl[warp][g] = lrow[0];
-    sm.wl[warp][g + 8] = lrow[1];
-  }
-#pragma unroll
-  for (int n = 0; n < 16; ++n) {
-    *reinterpret_cast<float2*>(&wo[warp][g][8 * n + 2 * c]) = make_float2(oacc[n][0], oacc[n][1]);
-    *reinterpret_cast<float2*>(&wo[warp][g + 8][8 * n + 2 * c]) = make_float2(oacc[n][2], oacc[n][3]);
-  }
-  __syncthreads();
-  const int d = tid;  // one output dimension per thread
-  for (int h = 0; h < G; ++h) {
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm.wm[w][h]);
-    float L = 0.f, o = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float f = sm.wm[w][h] == -INFINITY ? 0.f : exp2f(sm.wm[w][h] - M);
-      L = fmaf(f, sm.wl[w][h], L);
-      o = fmaf(f, wo[w][h][d], o);
-    }
-    part[h * kPartStride + 4 + d] = o;
-    if (d == 0) {
-      part[h * kPartStride + 0] = M;
-      part[h * kPartStride + 1] = L;
+  // Wait (bounded) for the copies that may still be in flight so that no TMA
+  // write lands in shared memory after the CTA has exited.
+  if (lane == 0) {
+    for (uint32_t d = 0; d < kRingStages && d < issued; ++d) {
+      const uint32_t e = issued - 1 - d;
+      mbar_wait(&sm.k_full[e % kRingStages], (e / kRingStages) & 1u, nullptr, a.status);
+      mbar_wait(&sm.v_full[e % kRingStages], (e / kRingStages) & 1u, nullptr, a.status);
     }
   }
 }
 
-// Log-sum-exp merge of the splits of one query head: the split statistics
-// (m, l) are loaded in parallel and reduced in shared memory, then each
-// thread streams one output dimension over the splits (independent,
-// coalesced loads, four in flight).
-__global__ void __launch_bounds__(kAttnThreads) decode_combine_kernel(const DecodeArgs a) {
-  extern __shared__ float wsh[];  // [max_splits] split weights
-  __shared__ float red[kAttnThreads / 32];
-  __shared__ float Msh, Lsh;
+// Consumer warps 0-3.  Per span: S = Q K^T (warp w: keys [32w, 32w+32)),
+// scale and mask, the span's row maxima posted and combined across the four
+// warps, one running maximum per row (identical in every warp), P = exp2(S -
+// m) into shared memory, then O += P V (warp w: output dims [32w, 32w+32)).
+// At the end of a run the row sums are combined and the CTA writes the run's
+// partial (m, l, o) for the group's query heads.
+__device__ __forceinline__ void attn_consumer(DecSmem& sm, const DecodeArgs& a, volatile int* abort) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, c = lane & 3;
+  const int G = a.group;
+  const float sl2 = a.scale_log2;
+  const uint32_t p_base = smem_u32(&sm.p[0][0]);
+  const int kbase = 32 * warp, dbase = 32 * warp;
+  uint32_t used = 0;  // spans consumed
+  for (int list = 0; list < 2; ++list) {
+    const long n = list_len(a, list);
+    if (n == 0) continue;
+    if (list == 1) griddep_wait();
+    const long hi = range_lo(a, n, blockIdx.x + 1);
+    long x = range_lo(a, n, blockIdx.x);
+    while (x < hi) {
+      int b, kvh, s;
+      locate(a, list, x, b, kvh, s);
+      const long run_start = x, run_end = min(hi, x - s + n_spans_of(a, kvh));
+      const size_t bk = static_cast<size_t>(b) * a.n_kv_heads + kvh;
+      const int cnt = list == 1 ? max(0, min(a.cnt[bk], a.kmax)) : a.kmax + (1 << 30);
+      const int s_end = min(s + static_cast<int>(run_end - x), cnt);
+      // Q as A fragments: rows g and g+8 are query heads g and g+8 of the
+      // group (zero beyond G); 8 K steps of 16 dims.
+      uint32_t qa[8][4];
+      {
+        const __nv_bfloat16* qb = a.q + (static_cast<size_t>(b) * a.n_q_heads + kvh * G) * kHeadDim;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int d0 = 16 * kk + 2 * c;
+          qa[kk][0] = g < G ? *reinterpret_cast<const uint32_t*>(qb + g * kHeadDim + d0) : 0u;
+          qa[kk][1] = g + 8 < G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * kHeadDim + d0) : 0u;
+          qa[kk][2] = g < G ? *reinterpret_cast<const uint32_t*>(qb + g * kHeadDim + d0 + 8) : 0u;
+          qa[kk][3] = g + 8 < G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * kHeadDim + d0 + 8) : 0u;
+        }
+      }
+      float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
+      float oacc[4][4];
+#pragma unroll
+      for (int nn = 0; nn < 4; ++nn) oacc[nn][0] = oacc[nn][1] = oacc[nn][2] = oacc[nn][3] = 0.f;
+      for (; s < s_end; ++s, ++used) {
+        const uint32_t st = used % kRingStages, ph = (used / kRingStages) & 1u;
+        if (tid == 0) sm.k_ok = mbar_wait(&sm.k_full[st], ph, abort, a.status) ? 1 : 0;
+        consumers_sync();
+        if (!checked_phase(&sm.k_full[st], ph, sm.k_ok)) return;
+        const int nk = sm.nk[st];
+        const uint32_t ks = smem_u32(sm.k[st]), vs = smem_u32(sm.v[st]);
+        // S = Q K^T over this warp's 32 keys: 4 n-tiles of 8 keys.  The head
+        // dims are split in two halves with their own accumulators, so each
+        // dependent chain of MMAs is 4 long instead of 8.
+        float sacc[4][4], sac2[4][4];
+#pragma unroll
+        for (int nn = 0; nn < 4; ++nn)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sacc[nn][e] = sac2[nn][e] = 0.f;
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+#pragma unroll
+          for (int half = 0; half < 2; ++half) {
+            const int kk = k4 + 4 * half;
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+              uint32_t r[4];
+              const int key = kbase + 16 * np + (lane >> 4) * 8 + (lane & 7);
+              const int dim = 16 * kk + ((lane >> 3) & 1) * 8;
+              ldsm_x4(sw128(ks, key, dim), r);
+              float (&acc)[4][4] = half ? sac2 : sacc;
+              mma_bf16(acc[2 * np], qa[kk], r[0], r[1]);
+              mma_bf16(acc[2 * np + 1], qa[kk], r[2], r[3]);
+            }
+          }
+        }
+#pragma unroll
+        for (int nn = 0; nn < 4; ++nn)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sacc[nn][e] += sac2[nn][e];
+        // scale to log2 units, mask keys past the span, this warp's maxima
+        float mw[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int nn = 0; nn < 4; ++nn)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int key = kbase + 8 * nn + 2 * c + (e & 1);
+            const float v = key < nk ? sacc[nn][e] * sl2 : -INFINITY;
+            sacc[nn][e] = v;
+            mw[e >> 1] = fmaxf(mw[e >> 1], v);
+          }
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          mw[rr] = fmaxf(mw[rr], __shfl_xor_sync(0xffffffffu, mw[rr], 1));
+          mw[rr] = fmaxf(mw[rr], __shfl_xor_sync(0xffffffffu, mw[rr], 2));
+        }
+        if (c == 0) {
+          sm.red_m[warp][g] = mw[0];
+          sm.red_m[warp][g + 8] = mw[1];
+        }
+        consumers_sync();  // every warp's maxima are posted
+        float mref[2];
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          float ms = sm.red_m[0][g + 8 * rr];
+#pragma unroll
+          for (int w = 1; w < kConsumerWarps; ++w) ms = fmaxf(ms, sm.red_m[w][g + 8 * rr]);
+          const float m_new = fmaxf(m_run[rr], ms);
+          mref[rr] = m_new == -INFINITY ? 0.f : m_new;
+          const float alpha = exp2f(m_run[rr] - mref[rr]);  // 0 while nothing was visible
+          m_run[rr] = m_new;
+          l_run[rr] *= alpha;
+#pragma unroll
+          for (int nn = 0; nn < 4; ++nn) {
+            oacc[nn][2 * rr] *= alpha;
+            oacc[nn][2 * rr + 1] *= alpha;
+          }
+        }
+        // P = exp2(S - m) as bf16 into shared memory; row sums in fp32
+#pragma unroll
+        for (int nn = 0; nn < 4; ++nn) {
+          const float p0 = exp2f(sacc[nn][0] - mref[0]), p1 = exp2f(sacc[nn][1] - mref[0]);
+          const float p2 = exp2f(sacc[nn][2] - mref[1]), p3 = exp2f(sacc[nn][3] - mref[1]);
+          l_run[0] += p0 + p1;
+          l_run[1] += p2 + p3;
+          const int key = kbase + 8 * nn + 2 * c;
+          *reinterpret_cast<uint32_t*>(&sm.p[g][key]) = pack_bf16x2(p0, p1);
+          *reinterpret_cast<uint32_t*>(&sm.p[g + 8][key]) = pack_bf16x2(p2, p3);
+        }
+        if (tid == 0) sm.v_ok = mbar_wait(&sm.v_full[st], ph, abort, a.status) ? 1 : 0;
+        consumers_sync();  // P is complete; V has arrived
+        if (!checked_phase(&sm.v_full[st], ph, sm.v_ok)) return;
+        // O += P V over all 128 keys of the span for this warp's 32 dims;
+        // odd key steps accumulate separately (two chains of 4 MMAs).
+        float ob[4][4];
+#pragma unroll
+        for (int nn = 0; nn < 4; ++nn) ob[nn][0] = ob[nn][1] = ob[nn][2] = ob[nn][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          uint32_t pa[4];
+          const int prow = (lane & 7) + ((lane >> 3) & 1) * 8;
+          ldsm_x4(p_base + static_cast<uint32_t>(prow * kPRowElems + 16 * kk + (lane >> 4) * 8) * 2u, pa);
+#pragma unroll
+          for (int dp = 0; dp < 2; ++dp) {
+            uint32_t r[4];
+            const int key = 16 * kk + ((lane >> 3) & 1) * 8 + (lane & 7);
+            const int dim = dbase + 16 * dp + (lane >> 4) * 8;
+            ldsm_x4_t(sw128(vs, key, dim), r);
+            float (&acc)[4][4] = (kk & 1) ? ob : oacc;
+            mma_bf16(acc[2 * dp], pa, r[0], r[1]);
+            mma_bf16(acc[2 * dp + 1], pa, r[2], r[3]);
+          }
+        }
+#pragma unroll
+        for (int nn = 0; nn < 4; ++nn)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) oacc[nn][e] += ob[nn][e];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.empty[st]);
+      }
+      // end of the run: row sums over the quad, then over the four warps
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 1);
+        l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 2);
+      }
+      if (c == 0) {
+        sm.red_l[warp][g] = l_run[0];
+        sm.red_l[warp][g + 8] = l_run[1];
+      }
+      consumers_sync();  // every warp's row sums are posted
+      float* part = run_partial(a, list, run_start);
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int row = g + 8 * rr;
+        if (row < G) {
+          float* pr = part + row * kPartStride;
+          if (warp == 0 && c == 0) {
+            float L = 0.f;
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) L += sm.red_l[w][row];
+            pr[0] = m_run[rr];
+            pr[1] = L;
+          }
+#pragma unroll
+          for (int nn = 0; nn < 4; ++nn)
+            *reinterpret_cast<float2*>(pr + 4 + dbase + 8 * nn + 2 * c) =
+                make_float2(oacc[nn][2 * rr], oacc[nn][2 * rr + 1]);
+        }
+      }
+      consumers_sync();  // red_l is free again
+      x = run_end;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 2) decode_attn_kernel(const __grid_constant__ CUtensorMap mk,
+                                                                       const __grid_constant__ CUtensorMap mv,
+                                                                       const __grid_constant__ DecodeArgs a) {
+  extern __shared__ uint8_t dsmem[];
+  DecSmem& sm = *reinterpret_cast<DecSmem*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
+  const int warp = warp_id();
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRingStages; ++i) {
+      mbar_init(&sm.k_full[i], 1);
+      mbar_init(&sm.v_full[i], 1);
+      mbar_init(&sm.empty[i], kConsumerWarps);
+    }
+    sm.abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // The combine launch may be scheduled now; it waits for this grid.
+  griddep_launch_dependents();
+  volatile int* abort = &sm.abort_flag;
+  if (warp == kConsumerWarps) {
+    if (lane_id() == 0) {
+      tma_prefetch_desc(&mk);
+      tma_prefetch_desc(&mv);
+    }
+    attn_producer(sm, &mk, &mv, a, abort);
+  } else {
+    attn_consumer(sm, a, abort);
+  }
+}
+
+// Log-sum-exp merge of the runs of one query head.  The runs of (sequence,
+// head) are those of the CTAs whose ranges meet the head's spans [x0, x1]:
+// the owner of x0 (its run starts at x0) and every later CTA up to the owner
+// of x1 that has work (its run starts at its range's first span).  Warp w
+// merges runs w, w+4, ... (lane l: dims 4l..4l+3, four runs' loads in
+// flight at a time); the four warps' results are merged in shared memory.
+__device__ __forceinline__ long run_slot(const DecodeArgs& a, long n, long x0, int c0, int r) {
+  if (r == 0) return x0;
+  const long lo = range_lo(a, n, c0 + r);
+  return lo == range_lo(a, n, c0 + r + 1) ? -1 : lo;  // -1: this CTA has no span
+}
+
+__global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const __grid_constant__ DecodeArgs a) {
+  constexpr int kWarps = kCombineThreads / 32;
+  __shared__ float wm[kWarps], wl[kWarps];
+  __shared__ float4 wo[kWarps][32];
   griddep_wait();  // partials of the preceding attention launch
   const int hq = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int kvh = hq / a.group, h = hq % a.group;
-  const int kind = a.kind[kvh];
-  int nsplit;
-  if (kind == KIND_SPARSE) {
-    nsplit = min(a.cnt[static_cast<size_t>(b) * a.n_kv_heads + kvh], a.kmax);
-  } else {
-    const int start = (kind == KIND_SWA) ? max(0, a.cache_len - a.window) : 0;
-    nsplit = (a.cache_len - start + 127) / 128;
-  }
-  nsplit = max(0, min(nsplit, a.max_splits));
-  const float* base = a.partial + (static_cast<size_t>(b) * a.n_kv_heads + kvh) * a.max_splits * a.group * kPartStride;
-  // 1. M = max of the split maxima
-  float m = -INFINITY;
-  for (int sp = tid; sp < nsplit; sp += kAttnThreads) {
-    const float v = base[(sp * a.group + h) * kPartStride];
-    wsh[sp] = v;
-    m = fmaxf(m, v);
-  }
+  const int list = list_of(a, kvh);
+  const long n = list_len(a, list);
+  const long x0 = static_cast<long>(b) * a.per_b[list] + a.span_off[kvh];
+  const long x1 = x0 + n_spans_of(a, kvh) - 1;
+  const int c0 = owner_of(a, n, x0);
+  const int nr = owner_of(a, n, x1) - c0 + 1;
+  float M = -INFINITY, L = 0.f;
+  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int r0 = warp; r0 < nr; r0 += 4 * kWarps) {
+    float mr[4], lr[4];
+    float4 orr[4];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  if (lane == 0) red[warp] = m;
-  __syncthreads();
-  if (tid == 0) {
-    float M = red[0];
-    for (int w = 1; w < kAttnThreads / 32; ++w) M = fmaxf(M, red[w]);
-    Msh = M;
-  }
-  __syncthreads();
-  const float M = Msh;
-  // 2. weights w_s = 2^(m_s - M) and L = sum w_s l_s
-  float lsum = 0.f;
-  for (int sp = tid; sp < nsplit; sp += kAttnThreads) {
-    const float ms = wsh[sp];
-    const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);
-    wsh[sp] = w;
-    lsum = fmaf(w, base[(sp * a.group + h) * kPartStride + 1], lsum);
-  }
+    for (int u = 0; u < 4; ++u) {
+      const int r = r0 + u * kWarps;
+      const long slot = r < nr ? run_slot(a, n, x0, c0, r) : -1;
+      mr[u] = -INFINITY;
+      lr[u] = 0.f;
+      orr[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (slot >= 0) {
+        const float* p = run_partial(a, list, slot) + h * kPartStride;
+        mr[u] = p[0];
+        lr[u] = p[1];
+        orr[u] = *reinterpret_cast<const float4*>(p + 4 + 4 * lane);
+      }
+    }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
-  __syncthreads();
-  if (lane == 0) red[warp] = lsum;
-  __syncthreads();
-  if (tid == 0) {
-    float L = 0.f;
-    for (int w = 0; w < kAttnThreads / 32; ++w) L += red[w];
-    Lsh = L;
+    for (int u = 0; u < 4; ++u) {
+      if (mr[u] == -INFINITY) continue;  // no run, or no visible key in it
+      const float mn = fmaxf(M, mr[u]);
+      const float fa = exp2f(M - mn), fb = exp2f(mr[u] - mn);
+      L = fmaf(L, fa, lr[u] * fb);
+      o.x = fmaf(o.x, fa, orr[u].x * fb);
+      o.y = fmaf(o.y, fa, orr[u].y * fb);
+      o.z = fmaf(o.z, fa, orr[u].z * fb);
+      o.w = fmaf(o.w, fa, orr[u].w * fb);
+      M = mn;
+    }
   }
+  if (lane == 0) {
+    wm[warp] = M;
+    wl[warp] = L;
+  }
+  wo[warp][lane] = o;
   __syncthreads();
-  // 3. o_d = sum_s w_s o_s[d] / L
+  // thread d: output dimension d
   const int d = tid;
-  const float* od = base + h * kPartStride + 4 + d;
-  const size_t stride = static_cast<size_t>(a.group) * kPartStride;
-  float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-  int sp = 0;
-  for (; sp + 3 < nsplit; sp += 4) {
-    const float v0 = od[sp * stride], v1 = od[(sp + 1) * stride], v2 = od[(sp + 2) * stride], v3 = od[(sp + 3) * stride];
-    acc0 = fmaf(wsh[sp], v0, acc0);
-    acc1 = fmaf(wsh[sp + 1], v1, acc1);
-    acc2 = fmaf(wsh[sp + 2], v2, acc2);
-    acc3 = fmaf(wsh[sp + 3], v3, acc3);
+  float Mt = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) Mt = fmaxf(Mt, wm[w]);
+  float Lt = 0.f, ot = 0.f;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const float f = wm[w] == -INFINITY ? 0.f : exp2f(wm[w] - Mt);
+    Lt = fmaf(f, wl[w], Lt);
+    ot = fmaf(f, reinterpret_cast<const float*>(&wo[w][d >> 2])[d & 3], ot);
   }
-  for (; sp < nsplit; ++sp) acc0 = fmaf(wsh[sp], od[sp * stride], acc0);
-  const float L = Lsh;
-  const float out = L > 0.f ? ((acc0 + acc1) + (acc2 + acc3)) / L : 0.f;
+  const float out = Lt > 0.f ? ot / Lt : 0.f;
   a.o[(static_cast<size_t>(b) * a.n_q_heads + hq) * kHeadDim + d] = __float2bfloat16_rn(out);
 }
 
@@ -412,13 +879,23 @@ cudaError_t decode_static_scratch(void** ptr) {
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t stream) {
-  const size_t sel_smem = static_cast<size_t>(a.nbc) * sizeof(uint32_t);
+  // All three kernels prefer the largest shared-memory carveout: an SM that
+  // a selection or combine CTA has configured for little shared memory could
+  // not take an attention CTA until it drains.
+  for (const void* fn : {reinterpret_cast<const void*>(decode_select_kernel),
+                         reinterpret_cast<const void*>(decode_attn_kernel),
+                         reinterpret_cast<const void*>(decode_combine_kernel)}) {
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         static_cast<int>(cudaSharedmemCarveoutMaxShared));
+    if (e != cudaSuccess) return e;
+  }
+  const size_t sel_smem = decode_select_smem(a);
   if (sel_smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(decode_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(sel_smem));
     if (e != cudaSuccess) return e;
   }
-  decode_select_kernel<<<dim3(a.n_kv_heads, a.batch), kSelThreads, sel_smem, stream>>>(a);
+  decode_select_kernel<<<dim3(kSelCluster * a.n_kv_heads, a.batch), kDecSelThreads, sel_smem, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -430,7 +907,7 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUte
   pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   pdl[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.max_splits, a.n_kv_heads, a.batch);
+  cfg.gridDim = dim3(a.n_ctas);
   cfg.blockDim = dim3(kAttnThreads);
   cfg.dynamicSmemBytes = kDecSmemBytes;
   cfg.stream = stream;
@@ -439,12 +916,8 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUte
   e = cudaLaunchKernelEx(&cfg, decode_attn_kernel, mk, mv, a);
   if (e != cudaSuccess) return e;
   cfg.gridDim = dim3(a.n_q_heads, a.batch);
-  cfg.dynamicSmemBytes = static_cast<size_t>(a.max_splits) * sizeof(float);
-  if (cfg.dynamicSmemBytes > 48 * 1024) {
-    e = cudaFuncSetAttribute(decode_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(cfg.dynamicSmemBytes));
-    if (e != cudaSuccess) return e;
-  }
+  cfg.blockDim = dim3(kCombineThreads);
+  cfg.dynamicSmemBytes = 0;
   return cudaLaunchKernelEx(&cfg, decode_combine_kernel, a);
 }
 

@@ -56,11 +56,20 @@ struct DecodeArgs {
   uint8_t kind[kMaxDecodeKvHeads];  // routing map, passed by value
   int32_t* sel;                 // [batch][n_kv_heads][kmax] (workspace or caller)
   int32_t* cnt;                 // [batch][n_kv_heads]
-  float* partial;               // [batch][n_kv_heads][max_splits][group][kPartStride]
+  float* partial;               // [n_spans of both lists][group][kPartStride]
   int batch, n_q_heads, n_kv_heads, group, cache_len, nbc;
-  int window, block, topk, n_local, kmax, max_splits;
+  int window, block, topk, n_local, kmax;
   float scale_log2;
   uint32_t* status;
+  // Schedule of the attention launch.  The work is cut into spans of at most
+  // 128 keys (one selected block of a retrieval head, or 128 consecutive keys
+  // of a window/full head) kept in two lists, list 0 = window and full heads,
+  // list 1 = retrieval heads, each ordered (sequence, head, span).  CTA c of
+  // n_ctas takes the contiguous range [c*N/n_ctas, (c+1)*N/n_ctas) of each
+  // list (N = the list's length).
+  int n_ctas;
+  int per_b[2];                           // spans per sequence in each list
+  int span_off[kMaxDecodeKvHeads];        // first span of a head within its sequence's part of its list
 };
 constexpr int kPartStride = 132;  // m, l, pad, pad, o[128]
 

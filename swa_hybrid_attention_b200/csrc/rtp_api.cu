@@ -369,37 +369,76 @@ rtp_status rtp_hybrid_prefill(const rtp_plan* plan, const void* q, const void* k
 }
 
 // Decode workspace: sel [batch][n_kv][kmax] int32 | cnt [batch][n_kv] int32 |
-// partials [batch][n_kv][max_splits][group][132] fp32, each 256-byte aligned.
+// partials [spans of both lists][group][132] fp32, each 256-byte aligned.
+// The spans (<= 128 keys each) form two lists ordered (sequence, head, span):
+// list 0 = window and full heads, list 1 = retrieval heads (kmax spans each).
 namespace {
 struct DecodeLayout {
   size_t sel_off, cnt_off, part_off, total;
-  int max_splits, kmax;
+  int kmax;
+  int per_b[2];
+  int span_off[kMaxDecodeKvHeads];
 };
 
 bool decode_layout(const rtp_attn_cfg* c, const uint8_t* kind, int cache_len, DecodeLayout& L) {
   if (!cfg_common_ok(c) || !kind || cache_len < 1) return false;
   if (static_cast<long>(cache_len) / c->block * 4 > 200 * 1024) return false;
+  if (c->n_kv_heads > kMaxDecodeKvHeads) return false;
   L.kmax = c->topk + 1 + c->n_local;
-  int ms = 1;
+  long per_b[2] = {0, 0};
   for (int h = 0; h < c->n_kv_heads; ++h) {
     if (kind[h] > RTP_HEAD_SPARSE) return false;
-    int s;
+    long s;
     if (kind[h] == RTP_HEAD_SPARSE)
       s = L.kmax;
     else if (kind[h] == RTP_HEAD_SWA)
       s = (std::min(cache_len, c->window) + 127) / 128;
     else
       s = (cache_len + 127) / 128;
-    ms = std::max(ms, s);
+    const int list = kind[h] == RTP_HEAD_SPARSE ? 1 : 0;
+    L.span_off[h] = static_cast<int>(per_b[list]);
+    per_b[list] += s;
   }
-  L.max_splits = ms;
+  if (per_b[0] > (1L << 30) || per_b[1] > (1L << 30)) return false;
+  L.per_b[0] = static_cast<int>(per_b[0]);
+  L.per_b[1] = static_cast<int>(per_b[1]);
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t bk = static_cast<size_t>(c->batch) * c->n_kv_heads;
+  const size_t spans = static_cast<size_t>(c->batch) * (per_b[0] + per_b[1]);
   const int group = c->n_q_heads / c->n_kv_heads;
   L.sel_off = 0;
   L.cnt_off = up(bk * L.kmax * sizeof(int32_t));
   L.part_off = L.cnt_off + up(bk * sizeof(int32_t));
-  L.total = L.part_off + up(bk * ms * group * kPartStride * sizeof(float));
+  L.total = L.part_off + up(spans * group * kPartStride * sizeof(float));
+  return true;
+}
+
+// SM count of the current device (looked up once per device).
+int device_sms() {
+  static std::mutex mu;
+  static int sms[64] = {0};
+  const int dev = current_device();
+  if (dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lk(mu);
+  if (sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    sms[dev] = n;
+  }
+  return sms[dev];
+}
+
+// The attention launch's schedule: one CTA per SM, no more CTAs than spans
+// in the longer list.
+bool decode_schedule(const rtp_attn_cfg* c, const DecodeLayout& L, DecodeArgs& a) {
+  const int sms = device_sms();
+  if (sms <= 0) return false;
+  const long n0 = static_cast<long>(c->batch) * L.per_b[0], n1 = static_cast<long>(c->batch) * L.per_b[1];
+  a.n_ctas = static_cast<int>(std::max(1L, std::min<long>(std::min(sms, 1024), std::max(n0, n1))));
+  a.per_b[0] = L.per_b[0];
+  a.per_b[1] = L.per_b[1];
+  std::memset(a.span_off, 0, sizeof(a.span_off));
+  std::memcpy(a.span_off, L.span_off, sizeof(int) * c->n_kv_heads);
   return true;
 }
 }  // namespace
@@ -449,8 +488,8 @@ rtp_status rtp_sparse_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, 
   a.topk = cfg->topk;
   a.n_local = cfg->n_local;
   a.kmax = L.kmax;
-  a.max_splits = L.max_splits;
   a.scale_log2 = effective_scale(cfg) * kLog2e;
+  if (!decode_schedule(cfg, L, a)) return RTP_ERR_CUDA;
   a.status = status_word(current_device());
   if (!a.status) return RTP_ERR_NO_MEMORY;
   CUtensorMap mk, mv;
@@ -500,8 +539,8 @@ rtp_status rtp_sparse_decode_noalloc(const rtp_attn_cfg* cfg, const uint8_t* kin
   a.topk = cfg->topk;
   a.n_local = cfg->n_local;
   a.kmax = L.kmax;
-  a.max_splits = L.max_splits;
   a.scale_log2 = effective_scale(cfg) * kLog2e;
+  if (!decode_schedule(cfg, L, a)) return RTP_ERR_CUDA;
   a.status = nullptr;  // no status word: getting one may allocate
   CUtensorMap mk, mv;
   if (!encode_bf16_3d(&mk, kcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64) ||

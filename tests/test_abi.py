@@ -83,8 +83,11 @@ def test_route_heads_rejects_bad_kind(rtp):
 def test_decode_workspace_size_and_validation(rtp):
     cfg = rtp.AttnConfig(8, 1, 32, 4, 8192, 128, 32, 4)
     n = rtp.rtp_decode_workspace_bytes(cfg, [2, 2, 0, 2], 262144)
-    # sel + cnt + partials [8][4][max(37, 64)][8][132] fp32
-    assert n >= 8 * 4 * 64 * 8 * 132 * 4
+    # sel [8][4][37] int32 | cnt [8][4] int32 | one partial slot per span:
+    # 8 sequences x (3 x 37 selected blocks + 8192 / 128 window pieces), each
+    # [8 heads][132] fp32; every part rounded up to 256 bytes
+    up = lambda x: (x + 255) // 256 * 256
+    assert n == up(8 * 4 * 37 * 4) + up(8 * 4 * 4) + up(8 * (3 * 37 + 64) * 8 * 132 * 4)
     assert rtp.rtp_decode_workspace_bytes(cfg, [2, 2, 0, 5], 262144) == 0
     bad = rtp.AttnConfig(8, 1, 32, 4, 8192, 96, 32, 4)
     assert rtp.rtp_decode_workspace_bytes(bad, [2, 2, 0, 2], 262144) == 0

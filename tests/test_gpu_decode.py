@@ -76,6 +76,11 @@ DECODE_CASES = [
     (2, 8, 4, [2, 2, 0, 1], 3000, 512, 64, 6, 2),    # ragged last block, full head, block 64
     (1, 4, 1, [2], 640, 100, 128, 8, 1),            # fewer candidates than top-k
     (3, 32, 4, [2, 0, 2, 2], 8192, 2048, 128, 16, 4),
+    # top-k 32 (bitonic path) with more candidates than one scoring round per CTA
+    (1, 8, 2, [2, 0], 196608, 4096, 64, 32, 4),
+    # top-k above 32 (radix path): one round, then several rounds per CTA
+    (1, 8, 2, [2, 0], 8192, 1024, 128, 40, 2),
+    (1, 4, 1, [2], 196608, 128, 64, 48, 2),
 ]
 
 
