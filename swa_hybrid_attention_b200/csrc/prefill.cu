@@ -296,22 +296,30 @@ drain:
 }
 
 // ---------------------------------------------------------------- MMA issue
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem, uint32_t idesc) {
+// The single issuing thread shares its scheduler with two busy softmax warps
+// and the tensor pipe buffers very few MMAs, so the issue path is kept short:
+// operand descriptors are built once per kernel and an operand at base + off
+// is the base descriptor plus off >> 4 (the 14-bit start-address field counts
+// 16-byte units; every shared address here is below 256 KB, so it never
+// carries).  Stages and heads are picked with selects, not runtime-indexed
+// arrays, which would live in local memory.
+__device__ __forceinline__ constexpr uint64_t desc_off(uint32_t off_bytes) { return off_bytes >> 4; }
+
+// S = Q K^T: M=128, N=128, K=128 (8 steps of 16); both operands K-major SW128.
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t qd, uint64_t kd, uint32_t idesc) {
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-    umma_ss(d_tmem, smem_desc_sw128(q_smem + off, 16, 1024), smem_desc_sw128(k_smem + off, 16, 1024), idesc,
-            kk > 0 ? 1u : 0u);
+    const uint64_t off = desc_off((kk >> 2) * kChunkBytes + (kk & 3) * 32);
+    umma_ss(d_tmem, qd + off, kd + off, idesc, kk > 0 ? 1u : 0u);
   }
 }
-
-__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint32_t v_smem, uint32_t idesc,
+// O += P V: P (bf16) from TMEM; V MN-major (16 keys = 2048 bytes per K-step,
+// the two 64-dim chunks kChunkBytes apart).
+__device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t vd, uint32_t idesc,
                                          bool accumulate) {
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    umma_ts(d_tmem, p_tmem + kk * 8, smem_desc_sw128(v_smem + kk * 2048, kChunkBytes, 1024), idesc,
-            (accumulate || kk > 0) ? 1u : 0u);
-  }
+  for (int kk = 0; kk < 8; ++kk)
+    umma_ts(d_tmem, p_tmem + kk * 8, vd + desc_off(kk * 2048), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& a, volatile int* abort) {
@@ -319,7 +327,10 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
   const uint32_t id_pv = idesc_bf16_f32(128, 128, true);
   const uint32_t tS[2] = {tmem, tmem + 128};
   const uint32_t tO[2] = {tmem + 256, tmem + 384};
-  const uint32_t sq[2] = {smem_u32(s.q[0]), smem_u32(s.q[1])};
+  const uint64_t qd0 = smem_desc_sw128(smem_u32(s.q[0]), 16, 1024), qd1 = smem_desc_sw128(smem_u32(s.q[1]), 16, 1024);
+  const uint64_t kd0 = smem_desc_sw128(smem_u32(s.k[0]), 16, 1024), kd1 = smem_desc_sw128(smem_u32(s.k[1]), 16, 1024);
+  const uint64_t vd0 = smem_desc_sw128(smem_u32(s.v[0]), kChunkBytes, 1024);
+  const uint64_t vd1 = smem_desc_sw128(smem_u32(s.v[1]), kChunkBytes, 1024);
   uint32_t it = 0, gt = 0, pc = 0;
   for (long idx = blockIdx.x; idx < a.n_items; idx += gridDim.x, ++it) {
     Item item = load_item(a.items, idx, a.n_kv_heads);
@@ -332,10 +343,10 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
       const int st0 = gt & 1;
       if (!mbar_wait(&s.k_full[st0], (gt >> 1) & 1u, abort, a.status)) goto drain;
       tc_fence_after();
-      const uint32_t sk = smem_u32(s.k[st0]);
-      issue_qk(tS[0], sq[0], sk, id_qk);
+      const uint64_t sk = st0 ? kd1 : kd0;
+      issue_qk(tS[0], qd0, sk, id_qk);
       umma_commit(&s.s_full[0]);
-      issue_qk(tS[1], sq[1], sk, id_qk);
+      issue_qk(tS[1], qd1, sk, id_qk);
       umma_commit(&s.s_full[1]);
       if (n == 1) {
         umma_commit(&s.q_empty[0]);
@@ -347,8 +358,8 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
       const int st = g & 1;
       const bool has_next = j + 1 < n;
       const int st2 = (g + 1) & 1;
-      const uint32_t sv = smem_u32(s.v[st]);
-      const uint32_t sk2 = smem_u32(s.k[st2]);
+      const uint64_t sv = st ? vd1 : vd0;
+      const uint64_t sk2 = st2 ? kd1 : kd0;
       if (!mbar_wait(&s.v_full[st], (g >> 1) & 1u, abort, a.status)) goto drain;
       // head 0: O0 += P0 V ; then S0 for the next tile
       if (!mbar_wait_spin(&s.p_full[0], pc & 1u, abort, a.status)) goto drain;
@@ -359,7 +370,7 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
       } else {
         if (!mbar_wait(&s.k_full[st2], ((g + 1) >> 1) & 1u, abort, a.status)) goto drain;
         tc_fence_after();
-        issue_qk(tS[0], sq[0], sk2, id_qk);
+        issue_qk(tS[0], qd0, sk2, id_qk);
         umma_commit(&s.s_full[0]);
         if (j + 2 == n) umma_commit(&s.q_empty[0]);
       }
@@ -371,7 +382,7 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
       if (!has_next) {
         umma_commit(&s.o_full[1]);
       } else {
-        issue_qk(tS[1], sq[1], sk2, id_qk);
+        issue_qk(tS[1], qd1, sk2, id_qk);
         umma_commit(&s.s_full[1]);
         if (j + 2 == n) umma_commit(&s.q_empty[1]);
       }
@@ -512,7 +523,7 @@ __device__ __noinline__ void run_softmax(Smem& s, uint32_t tmem, int h, const Pr
 
 __global__ void __launch_bounds__(kThreads, 1)
     hybrid_prefill_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
-                          const __grid_constant__ CUtensorMap mv, const PrefillArgs a) {
+                          const __grid_constant__ CUtensorMap mv, const __grid_constant__ PrefillArgs a) {
   extern __shared__ uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = warp_id();
