@@ -366,15 +366,26 @@ size_t decode_select_smem(const DecodeArgs& a) {
 }
 
 // ---------------------------------------------------------------- schedule
-__device__ __forceinline__ int list_of(const DecodeArgs& a, int kvh) { return a.kind[kvh] == KIND_SPARSE ? 1 : 0; }
+// Block of the new token, and the number of blocks every selection keeps
+// whatever the scores: the sink and the local blocks {0} u {t-L+1..t}.
+__device__ __forceinline__ int decode_t(const DecodeArgs& a) { return (a.cache_len - 1) / a.block; }
+__device__ __forceinline__ int n_fixed(const DecodeArgs& a) { return min(decode_t(a) + 1, a.n_local + 1); }
 
-// Spans of one (sequence, head): kmax selected blocks, or the visible keys of
-// a window/full head in 128-key pieces.
-__device__ __forceinline__ int n_spans_of(const DecodeArgs& a, int kvh) {
+// Spans of one (sequence, head) in a list: list 0 holds a window/full head's
+// visible keys in 128-key pieces, or a retrieval head's sink and local
+// blocks; list 1 holds the rest of a retrieval head's kmax selected blocks.
+__device__ __forceinline__ int n_spans_in(const DecodeArgs& a, int list, int kvh) {
   const int kind = a.kind[kvh];
-  if (kind == KIND_SPARSE) return a.kmax;
+  if (kind == KIND_SPARSE) return list == 0 ? n_fixed(a) : a.kmax - n_fixed(a);
+  if (list == 1) return 0;
   const int len = kind == KIND_SWA ? min(a.cache_len, a.window) : a.cache_len;
   return (len + 127) / 128;
+}
+
+// Fixed block s (0 <= s < n_fixed) of a retrieval head, ascending.
+__device__ __forceinline__ int fixed_block(const DecodeArgs& a, int s) {
+  const int t = decode_t(a);
+  return (t <= a.n_local || s == 0) ? s : t - a.n_local + s;
 }
 
 __device__ __forceinline__ long list_len(const DecodeArgs& a, int list) {
@@ -391,16 +402,15 @@ __device__ __forceinline__ int owner_of(const DecodeArgs& a, long n, long x) {
   return static_cast<int>(((static_cast<long long>(x) + 1) * a.n_ctas - 1) / n);
 }
 
-// Span x of a list -> (sequence, head, span index within the head).
+// Span x of a list -> (sequence, head, span index within the head's part).
 __device__ __forceinline__ void locate(const DecodeArgs& a, int list, long x, int& b, int& kvh, int& s) {
   b = static_cast<int>(x / a.per_b[list]);
   const int r = static_cast<int>(x - static_cast<long>(b) * a.per_b[list]);
   kvh = 0;
   s = 0;
   for (int h = 0; h < a.n_kv_heads; ++h) {
-    if (list_of(a, h) != list) continue;
-    const int off = a.span_off[h];
-    if (r >= off && r < off + n_spans_of(a, h)) {
+    const int off = a.span_off[list][h];
+    if (r >= off && r < off + n_spans_in(a, list, h)) {
       kvh = h;
       s = r - off;
       return;
@@ -484,14 +494,17 @@ __device__ __forceinline__ void attn_producer(DecSmem& sm, const CUtensorMap* mk
     while (x < hi && ok) {
       int b, kvh, s;
       locate(a, list, x, b, kvh, s);
-      const long run_end = min(hi, x - s + n_spans_of(a, kvh));
+      const int nsp = n_spans_in(a, list, kvh);
+      const long run_end = min(hi, x - s + nsp);
       const size_t bk = static_cast<size_t>(b) * a.n_kv_heads + kvh;
-      const int cnt = list == 1 ? max(0, min(a.cnt[bk], a.kmax)) : a.kmax + (1 << 30);
+      // list 1: the first cnt - n_fixed of the head's spans hold selected blocks
+      const int cnt = list == 1 ? max(0, min(a.cnt[bk], a.kmax) - n_fixed(a)) : nsp;
       const int s_end = min(s + static_cast<int>(run_end - x), cnt);
+      const bool sparse = a.kind[kvh] == KIND_SPARSE;
       const int start = a.kind[kvh] == KIND_SWA ? max(0, a.cache_len - a.window) : 0;
       for (int s0 = s; s0 < s_end && ok; s0 += 32) {
-        int blk_l = 0;
-        if (list == 1 && s0 + lane < s_end) blk_l = a.sel[bk * a.kmax + s0 + lane];
+        int blk_l = 0;  // the selection keeps its sink first: span s is entry 1 + s
+        if (list == 1 && s0 + lane < s_end) blk_l = a.sel[bk * a.kmax + 1 + s0 + lane];
         const int m = min(32, s_end - s0);
         for (int i = 0; i < m; ++i) {
           int key0, nk;
@@ -505,6 +518,9 @@ __device__ __forceinline__ void attn_producer(DecSmem& sm, const CUtensorMap* mk
               key0 = blk * a.block;
               nk = min(a.block, a.cache_len - key0);
             }
+          } else if (sparse) {
+            key0 = fixed_block(a, s0 + i) * a.block;
+            nk = min(a.block, a.cache_len - key0);
           } else {
             key0 = start + 128 * (s0 + i);
             nk = min(128, a.cache_len - key0);
@@ -569,9 +585,10 @@ __device__ __forceinline__ void attn_consumer(DecSmem& sm, const DecodeArgs& a, 
     while (x < hi) {
       int b, kvh, s;
       locate(a, list, x, b, kvh, s);
-      const long run_start = x, run_end = min(hi, x - s + n_spans_of(a, kvh));
+      const int nsp = n_spans_in(a, list, kvh);
+      const long run_start = x, run_end = min(hi, x - s + nsp);
       const size_t bk = static_cast<size_t>(b) * a.n_kv_heads + kvh;
-      const int cnt = list == 1 ? max(0, min(a.cnt[bk], a.kmax)) : a.kmax + (1 << 30);
+      const int cnt = list == 1 ? max(0, min(a.cnt[bk], a.kmax) - n_fixed(a)) : nsp;
       const int s_end = min(s + static_cast<int>(run_end - x), cnt);
       // Q as A fragments: rows g and g+8 are query heads g and g+8 of the
       // group (zero beyond G); 8 K steps of 16 dims.
@@ -773,8 +790,9 @@ __global__ void __launch_bounds__(kAttnThreads, 2) decode_attn_kernel(const __gr
   }
 }
 
-// Log-sum-exp merge of the runs of one query head.  The runs of (sequence,
-// head) are those of the CTAs whose ranges meet the head's spans [x0, x1]:
+// Log-sum-exp merge of the runs of one query head.  In each list, the runs
+// of (sequence, head) are those of the CTAs whose ranges meet the head's
+// spans [x0, x1]:
 // the owner of x0 (its run starts at x0) and every later CTA up to the owner
 // of x1 that has work (its run starts at its range's first span).  Warp w
 // merges runs w, w+4, ... (lane l: dims 4l..4l+3, four runs' loads in
@@ -792,12 +810,23 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const _
   griddep_wait();  // partials of the preceding attention launch
   const int hq = blockIdx.x, b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int kvh = hq / a.group, h = hq % a.group;
-  const int list = list_of(a, kvh);
-  const long n = list_len(a, list);
-  const long x0 = static_cast<long>(b) * a.per_b[list] + a.span_off[kvh];
-  const long x1 = x0 + n_spans_of(a, kvh) - 1;
-  const int c0 = owner_of(a, n, x0);
-  const int nr = owner_of(a, n, x1) - c0 + 1;
+  // The head's runs: those of list 0, then those of list 1 (a retrieval head
+  // has spans in both; a window/full head only in list 0).
+  long n0 = 0, x00 = 0, n1 = 0, x01 = 0;
+  int c00 = 0, nr0 = 0, c01 = 0, nr1 = 0;
+  if (const int ns = n_spans_in(a, 0, kvh); ns > 0) {
+    n0 = list_len(a, 0);
+    x00 = static_cast<long>(b) * a.per_b[0] + a.span_off[0][kvh];
+    c00 = owner_of(a, n0, x00);
+    nr0 = owner_of(a, n0, x00 + ns - 1) - c00 + 1;
+  }
+  if (const int ns = n_spans_in(a, 1, kvh); ns > 0) {
+    n1 = list_len(a, 1);
+    x01 = static_cast<long>(b) * a.per_b[1] + a.span_off[1][kvh];
+    c01 = owner_of(a, n1, x01);
+    nr1 = owner_of(a, n1, x01 + ns - 1) - c01 + 1;
+  }
+  const int nr = nr0 + nr1;
   float M = -INFINITY, L = 0.f;
   float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int r0 = warp; r0 < nr; r0 += 4 * kWarps) {
@@ -806,7 +835,9 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const _
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int r = r0 + u * kWarps;
-      const long slot = r < nr ? run_slot(a, n, x0, c0, r) : -1;
+      const int list = r < nr0 ? 0 : 1;
+      const long slot = r >= nr ? -1
+                        : (list == 0 ? run_slot(a, n0, x00, c00, r) : run_slot(a, n1, x01, c01, r - nr0));
       mr[u] = -INFINITY;
       lr[u] = 0.f;
       orr[u] = make_float4(0.f, 0.f, 0.f, 0.f);

@@ -62,14 +62,15 @@ struct DecodeArgs {
   float scale_log2;
   uint32_t* status;
   // Schedule of the attention launch.  The work is cut into spans of at most
-  // 128 keys (one selected block of a retrieval head, or 128 consecutive keys
-  // of a window/full head) kept in two lists, list 0 = window and full heads,
-  // list 1 = retrieval heads, each ordered (sequence, head, span).  CTA c of
-  // n_ctas takes the contiguous range [c*N/n_ctas, (c+1)*N/n_ctas) of each
-  // list (N = the list's length).
+  // 128 keys (one block of a retrieval head, or 128 consecutive keys of a
+  // window/full head) kept in two lists, each ordered (sequence, head, span):
+  // list 0 = what needs no selection (window and full heads, and each
+  // retrieval head's sink and local blocks), list 1 = the blocks a retrieval
+  // head's top-k picked.  CTA c of n_ctas takes the contiguous range
+  // [c*N/n_ctas, (c+1)*N/n_ctas) of each list (N = the list's length).
   int n_ctas;
   int per_b[2];                           // spans per sequence in each list
-  int span_off[kMaxDecodeKvHeads];        // first span of a head within its sequence's part of its list
+  int span_off[2][kMaxDecodeKvHeads];     // first span of a head within its sequence's part of each list
 };
 constexpr int kPartStride = 132;  // m, l, pad, pad, o[128]
 

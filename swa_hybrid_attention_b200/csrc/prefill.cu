@@ -75,6 +75,14 @@ constexpr uint32_t kMemberAll = 0x1Eu;
 #define RTP_POLY_PAIRS 0x00u
 #endif
 constexpr uint32_t kPolyPairs = RTP_POLY_PAIRS;
+// P is handed to the MMA issuer in kPChunks pieces of 128/kPChunks keys, so
+// O += P V starts on the first keys while the softmax still exponentiates
+// the rest (the P V of a tile then ends shortly after its softmax).
+#ifndef RTP_P_CHUNKS
+#define RTP_P_CHUNKS 2
+#endif
+constexpr int kPChunks = RTP_P_CHUNKS;
+static_assert(kPChunks == 1 || kPChunks == 2 || kPChunks == 4, "P chunks must divide the four 32-key groups");
 
 struct __align__(1024) Smem {
   uint8_t q[2][kTileBytes];
@@ -82,7 +90,8 @@ struct __align__(1024) Smem {
   uint8_t v[kStages][kTileBytes];
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
-  uint64_t s_full[2], p_full[2], o_full[2];
+  uint64_t s_full[2], o_full[2];
+  uint64_t p_full[2][kPChunks];  // [head][chunk of keys]: that part of P is in TMEM
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -313,13 +322,27 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint64_t qd, uint64_t 
     umma_ss(d_tmem, qd + off, kd + off, idesc, kk > 0 ? 1u : 0u);
   }
 }
-// O += P V: P (bf16) from TMEM; V MN-major (16 keys = 2048 bytes per K-step,
-// the two 64-dim chunks kChunkBytes apart).
+// O += P V for key steps [kk0, kk1): P (bf16) from TMEM; V MN-major (16 keys
+// = 2048 bytes per K-step, the two 64-dim chunks kChunkBytes apart).
 __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, uint64_t vd, uint32_t idesc,
-                                         bool accumulate) {
+                                         bool accumulate, int kk0, int kk1) {
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk)
+  for (int kk = kk0; kk < kk1; ++kk)
     umma_ts(d_tmem, p_tmem + kk * 8, vd + desc_off(kk * 2048), idesc, (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// O += P V of one head, each chunk of keys issued as soon as its part of P is
+// in TMEM.  Returns false if a wait gave up.
+__device__ __forceinline__ bool issue_pv_chunked(Smem& s, int h, uint32_t parity, uint32_t d_tmem, uint32_t p_tmem,
+                                                 uint64_t vd, uint32_t idesc, bool accumulate, volatile int* abort,
+                                                 uint32_t* status) {
+#pragma unroll
+  for (int q = 0; q < kPChunks; ++q) {
+    if (!mbar_wait_spin(&s.p_full[h][q], parity, abort, status)) return false;
+    tc_fence_after();
+    issue_pv(d_tmem, p_tmem, vd, idesc, accumulate, q * (8 / kPChunks), (q + 1) * (8 / kPChunks));
+  }
+  return true;
 }
 
 __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& a, volatile int* abort) {
@@ -362,9 +385,7 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
       const uint64_t sk2 = st2 ? kd1 : kd0;
       if (!mbar_wait(&s.v_full[st], (g >> 1) & 1u, abort, a.status)) goto drain;
       // head 0: O0 += P0 V ; then S0 for the next tile
-      if (!mbar_wait_spin(&s.p_full[0], pc & 1u, abort, a.status)) goto drain;
-      tc_fence_after();
-      issue_pv(tO[0], tS[0], sv, id_pv, j > 0);
+      if (!issue_pv_chunked(s, 0, pc & 1u, tO[0], tS[0], sv, id_pv, j > 0, abort, a.status)) goto drain;
       if (!has_next) {
         umma_commit(&s.o_full[0]);
       } else {
@@ -375,9 +396,7 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
         if (j + 2 == n) umma_commit(&s.q_empty[0]);
       }
       // head 1
-      if (!mbar_wait_spin(&s.p_full[1], pc & 1u, abort, a.status)) goto drain;
-      tc_fence_after();
-      issue_pv(tO[1], tS[1], sv, id_pv, j > 0);
+      if (!issue_pv_chunked(s, 1, pc & 1u, tO[1], tS[1], sv, id_pv, j > 0, abort, a.status)) goto drain;
       umma_commit(&s.kv_empty[st]);
       if (!has_next) {
         umma_commit(&s.o_full[1]);
@@ -485,14 +504,16 @@ __device__ __noinline__ void run_softmax(Smem& s, uint32_t tmem, int h, const Pr
           p[e] = pack_bf16x2(lo2(pe), hi2(pe));
         }
         tmem_st16(tS + 16 * c, p);
+        if ((c + 1) % (4 / kPChunks) == 0) {  // a chunk of P is complete
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&s.p_full[h][c / (4 / kPChunks)]);
+        }
       }
       {
         const uint64_t sa = add2(add2(s4[0], s4[1]), add2(s4[2], s4[3]));
         l += lo2(sa) + hi2(sa);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&s.p_full[h]);
     }
     // epilogue: O / l -> bf16
     if (!warp_wait(&s.o_full[h], it & 1u, abort, a.status)) return;
@@ -532,7 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.q_full[h], 1);
       mbar_init(&s.q_empty[h], 1);
       mbar_init(&s.s_full[h], 1);
-      mbar_init(&s.p_full[h], 128);
+      for (int q = 0; q < kPChunks; ++q) mbar_init(&s.p_full[h][q], 128);
       mbar_init(&s.o_full[h], 1);
     }
     for (int st = 0; st < kStages; ++st) {

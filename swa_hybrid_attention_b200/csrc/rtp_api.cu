@@ -371,13 +371,15 @@ rtp_status rtp_hybrid_prefill(const rtp_plan* plan, const void* q, const void* k
 // Decode workspace: sel [batch][n_kv][kmax] int32 | cnt [batch][n_kv] int32 |
 // partials [spans of both lists][group][132] fp32, each 256-byte aligned.
 // The spans (<= 128 keys each) form two lists ordered (sequence, head, span):
-// list 0 = window and full heads, list 1 = retrieval heads (kmax spans each).
+// list 0 = window and full heads plus each retrieval head's sink and local
+// blocks (known before the selection), list 1 = the retrieval heads' top-k
+// blocks.
 namespace {
 struct DecodeLayout {
   size_t sel_off, cnt_off, part_off, total;
   int kmax;
   int per_b[2];
-  int span_off[kMaxDecodeKvHeads];
+  int span_off[2][kMaxDecodeKvHeads];
 };
 
 bool decode_layout(const rtp_attn_cfg* c, const uint8_t* kind, int cache_len, DecodeLayout& L) {
@@ -385,19 +387,24 @@ bool decode_layout(const rtp_attn_cfg* c, const uint8_t* kind, int cache_len, De
   if (static_cast<long>(cache_len) / c->block * 4 > 200 * 1024) return false;
   if (c->n_kv_heads > kMaxDecodeKvHeads) return false;
   L.kmax = c->topk + 1 + c->n_local;
+  const long t = (cache_len - 1) / c->block;                      // block of the new token
+  const long nfix = std::min<long>(t + 1, c->n_local + 1);       // sink + local blocks
   long per_b[2] = {0, 0};
   for (int h = 0; h < c->n_kv_heads; ++h) {
     if (kind[h] > RTP_HEAD_SPARSE) return false;
-    long s;
-    if (kind[h] == RTP_HEAD_SPARSE)
-      s = L.kmax;
-    else if (kind[h] == RTP_HEAD_SWA)
-      s = (std::min(cache_len, c->window) + 127) / 128;
-    else
-      s = (cache_len + 127) / 128;
-    const int list = kind[h] == RTP_HEAD_SPARSE ? 1 : 0;
-    L.span_off[h] = static_cast<int>(per_b[list]);
-    per_b[list] += s;
+    long s0 = 0, s1 = 0;
+    if (kind[h] == RTP_HEAD_SPARSE) {
+      s0 = nfix;
+      s1 = L.kmax - nfix;
+    } else if (kind[h] == RTP_HEAD_SWA) {
+      s0 = (std::min(cache_len, c->window) + 127) / 128;
+    } else {
+      s0 = (cache_len + 127) / 128;
+    }
+    L.span_off[0][h] = static_cast<int>(per_b[0]);
+    L.span_off[1][h] = static_cast<int>(per_b[1]);
+    per_b[0] += s0;
+    per_b[1] += s1;
   }
   if (per_b[0] > (1L << 30) || per_b[1] > (1L << 30)) return false;
   L.per_b[0] = static_cast<int>(per_b[0]);
@@ -438,7 +445,7 @@ bool decode_schedule(const rtp_attn_cfg* c, const DecodeLayout& L, DecodeArgs& a
   a.per_b[0] = L.per_b[0];
   a.per_b[1] = L.per_b[1];
   std::memset(a.span_off, 0, sizeof(a.span_off));
-  std::memcpy(a.span_off, L.span_off, sizeof(int) * c->n_kv_heads);
+  for (int l = 0; l < 2; ++l) std::memcpy(a.span_off[l], L.span_off[l], sizeof(int) * c->n_kv_heads);
   return true;
 }
 }  // namespace
