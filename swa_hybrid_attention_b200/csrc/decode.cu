@@ -18,12 +18,12 @@
 //     takes a contiguous range of each list, so it works through its window
 //     spans while the selection is still running and only then waits for it.
 //     A producer warp streams the spans' K and V through a 3-stage TMA ring;
-//     four consumer warps run S = Q K^T (each warp 32 keys), one softmax per
-//     span with a running maximum shared across the warps, and O += P V
-//     (each warp 32 output dimensions), on tensor cores (mma.sync m16n8k16,
-//     the group's query heads as the M rows: each K/V byte is read once per
-//     group).  Consecutive spans of one (sequence, head) merge online; a CTA
-//     writes one partial (m, l, o) per run of spans.
+//     four consumer warps each take 32 keys of every span and run S^T =
+//     K Q^T, their own online softmax and O^T += V^T P^T on tensor cores
+//     (mma.sync m16n8k16 with keys, then head dims, as M and the group's
+//     query heads as N: each K/V byte is read once per group, no row is
+//     padding).  Consecutive spans of one (sequence, head) merge online; the
+//     warps merge at the end of a run, which writes one partial (m, l, o).
 //  3. decode_combine_kernel (query head, sequence): log-sum-exp merge of the
 //     runs of the head.
 // The step is bound by HBM reads of the selected K/V and the windows.
@@ -44,8 +44,12 @@ constexpr int kConsumerWarps = 4;
 constexpr int kAttnThreads = 32 * (kConsumerWarps + 1);  // + one producer warp
 constexpr int kCombineThreads = 128;
 constexpr int kRingStages = 3;
+// The producer prefetches the K/V rows of the spans this many steps ahead of
+// the ones it loads into the ring into L2 (bulk prefetch): their page walks
+// and DRAM latency overlap without shared memory.  148 CTAs x 8 spans x 64 KB
+// = 76 MB stays well inside the 126 MB L2.
+constexpr int kPrefetchAhead = 8;
 constexpr uint32_t kHalfSpanBytes = 128 * 128 * 2;  // K (or V) of one span
-constexpr int kPRowElems = 128 + 8;  // P row pitch (bf16): 272 bytes, conflict-free
 
 // ---------------------------------------------------------------- selection
 // One cluster of kSelCluster CTAs per (retrieval head, sequence).  CTA r of
@@ -428,12 +432,10 @@ __device__ __forceinline__ float* run_partial(const DecodeArgs& a, int list, lon
 struct __align__(1024) DecSmem {
   uint8_t k[kRingStages][kHalfSpanBytes];  // 128 keys x 128 dims: two 64-column SW128 chunks
   uint8_t v[kRingStages][kHalfSpanBytes];
-  __nv_bfloat16 p[16][kPRowElems];         // P of the current span: 16 rows x 128 keys
+  float wo[kConsumerWarps][kHeadDim][8];   // run-end merge: each warp's O^T for 8 heads
+  float wm[kConsumerWarps][8], wl[kConsumerWarps][8];
   uint64_t k_full[kRingStages], v_full[kRingStages], empty[kRingStages];
-  int k_ok, v_ok;                          // results of the consumers' K / V waits
   int nk[kRingStages];                     // valid keys of the span in each stage
-  float red_m[kConsumerWarps][16];
-  float red_l[kConsumerWarps][16];
   int abort_flag;
 };
 constexpr size_t kDecSmemBytes = sizeof(DecSmem) + 1024;  // + alignment slack
@@ -461,24 +463,17 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Named barrier over the 128 consumer threads (the producer warp never
-// joins it): a hardware barrier, so waiting threads take no issue slots.
-__device__ __forceinline__ void consumers_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsumerWarps) : "memory");
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(p)), "r"(bytes)
+               : "memory");
 }
 
-// Consumer thread 0 alone polls an mbarrier (bounded wait); after the next
-// consumers_sync every thread reads the shared result and, when the phase is
-// complete, tests it once itself (it completes at once), which gives each
-// thread acquire ordering for the data the phase guards.
-__device__ __forceinline__ bool checked_phase(uint64_t* bar, uint32_t parity, int ok) {
-  if (ok) mbar_test(bar, parity);
-  return ok != 0;
-}
 // Producer warp: walks the CTA's spans in consumption order and streams K
 // and V of each into the ring (four 64x64 boxes each, 128-byte swizzle; rows
-// past the cache read as zero).  Block indices of retrieval spans are read
-// 32 at a time by the whole warp; lane 0 waits for free stages and issues.
+// past the cache read as zero).  The spans are taken 32 at a time: lane l
+// works out the key range of span l of the chunk (reading the selection for
+// retrieval spans), lanes prefetch the rows of the spans kPrefetchAhead ahead
+// into L2, and lane 0 waits for free stages and issues the loads.
 __device__ __forceinline__ void attn_producer(DecSmem& sm, const CUtensorMap* mk, const CUtensorMap* mv,
                                               const DecodeArgs& a, volatile int* abort) {
   const int lane = lane_id();
@@ -502,29 +497,42 @@ __device__ __forceinline__ void attn_producer(DecSmem& sm, const CUtensorMap* mk
       const int s_end = min(s + static_cast<int>(run_end - x), cnt);
       const bool sparse = a.kind[kvh] == KIND_SPARSE;
       const int start = a.kind[kvh] == KIND_SWA ? max(0, a.cache_len - a.window) : 0;
+      const __nv_bfloat16* kbase = a.kcache + bk * static_cast<size_t>(a.cache_len) * kHeadDim;
+      const __nv_bfloat16* vbase = a.vcache + bk * static_cast<size_t>(a.cache_len) * kHeadDim;
       for (int s0 = s; s0 < s_end && ok; s0 += 32) {
-        int blk_l = 0;  // the selection keeps its sink first: span s is entry 1 + s
-        if (list == 1 && s0 + lane < s_end) blk_l = a.sel[bk * a.kmax + 1 + s0 + lane];
         const int m = min(32, s_end - s0);
-        for (int i = 0; i < m; ++i) {
-          int key0, nk;
+        // lane l: key range of span s0 + l
+        int key0_l = 0, nk_l = 0;
+        if (lane < m) {
           if (list == 1) {
-            const int blk = __shfl_sync(0xffffffffu, blk_l, i);
+            const int blk = a.sel[bk * a.kmax + 1 + s0 + lane];  // the sink is entry 0
             if (blk < 0 || blk > tq) {  // not a valid selection: the span contributes nothing
-              if (lane == 0) flag_error(a.status, RTP_DEVERR_INDEX);
-              key0 = 0;
-              nk = 0;
+              flag_error(a.status, RTP_DEVERR_INDEX);
             } else {
-              key0 = blk * a.block;
-              nk = min(a.block, a.cache_len - key0);
+              key0_l = blk * a.block;
+              nk_l = min(a.block, a.cache_len - key0_l);
             }
           } else if (sparse) {
-            key0 = fixed_block(a, s0 + i) * a.block;
-            nk = min(a.block, a.cache_len - key0);
+            key0_l = fixed_block(a, s0 + lane) * a.block;
+            nk_l = min(a.block, a.cache_len - key0_l);
           } else {
-            key0 = start + 128 * (s0 + i);
-            nk = min(128, a.cache_len - key0);
+            key0_l = start + 128 * (s0 + lane);
+            nk_l = min(128, a.cache_len - key0_l);
           }
+        }
+        // rows the ring load will read: 128 from key0, within the cache
+        const uint32_t pf_bytes = static_cast<uint32_t>(max(0, min(128, a.cache_len - key0_l))) * kHeadDim * 2;
+        auto prefetch_span = [&]() {
+          if (pf_bytes > 0) {
+            prefetch_l2(kbase + static_cast<size_t>(key0_l) * kHeadDim, pf_bytes);
+            prefetch_l2(vbase + static_cast<size_t>(key0_l) * kHeadDim, pf_bytes);
+          }
+        };
+        if (lane < min(m, kPrefetchAhead)) prefetch_span();
+        for (int i = 0; i < m; ++i) {
+          const int key0 = __shfl_sync(0xffffffffu, key0_l, i);
+          const int nk = __shfl_sync(0xffffffffu, nk_l, i);
+          if (lane == i + kPrefetchAhead && lane < m) prefetch_span();
           const uint32_t st = issued % kRingStages, ph = (issued / kRingStages) & 1u;
           int okl = 1;
           if (lane == 0) {
@@ -562,20 +570,51 @@ __device__ __forceinline__ void attn_producer(DecSmem& sm, const CUtensorMap* mk
   }
 }
 
-// Consumer warps 0-3.  Per span: S = Q K^T (warp w: keys [32w, 32w+32)),
-// scale and mask, the span's row maxima posted and combined across the four
-// warps, one running maximum per row (identical in every warp), P = exp2(S -
-// m) into shared memory, then O += P V (warp w: output dims [32w, 32w+32)).
-// At the end of a run the row sums are combined and the CTA writes the run's
-// partial (m, l, o) for the group's query heads.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// All lanes of the warp wait (bounded) for a phase: lane 0 polls, then every
+// lane tests the completed phase once for its own acquire.  Uniform result.
+__device__ __forceinline__ bool warp_phase_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                                uint32_t* status) {
+  int ok = 1;
+  if (lane_id() == 0) ok = mbar_wait(bar, parity, abort, status) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  if (ok) mbar_test(bar, parity);
+  return ok != 0;
+}
+
+// Named barrier over the 128 consumer threads (the producer warp never
+// joins it).
+__device__ __forceinline__ void consumers_sync() {
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsumerWarps) : "memory");
+}
+
+// Consumer warps 0-3, each on its own: warp w takes keys [32w, 32w+32) of
+// every span and keeps its own running maximum, row sums and O for them
+// (flash-decoding inside the CTA); the four warps merge at the end of a run
+// through shared memory and the consumers' named barrier.  A warp whose
+// bounded wait gives up does not leave early: it walks the rest of the
+// schedule without waiting or computing, so every warp reaches every named
+// barrier and none can be left waiting at one.
+// The MMAs are transposed so that no row is padding: S^T = K Q^T with the 16
+// keys of an m16n8k16 tile as M and 8 query heads as N (NT tiles of 8 heads
+// for a group of up to 8 NT), then O^T += V^T P^T with 16 head dims as M,
+// where P^T comes straight from the S^T accumulators: each 8x8 block of
+// (key, head) values is transposed in registers (movmatrix) into the B
+// fragment layout.  Per span and warp: 16 NT MMAs for S^T and 16 NT for O^T.
+template <int NT>
 __device__ __forceinline__ void attn_consumer(DecSmem& sm, const DecodeArgs& a, volatile int* abort) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, c = lane & 3;
   const int G = a.group;
   const float sl2 = a.scale_log2;
-  const uint32_t p_base = smem_u32(&sm.p[0][0]);
-  const int kbase = 32 * warp, dbase = 32 * warp;
+  const int kbase = 32 * warp;
   uint32_t used = 0;  // spans consumed
+  bool dead = false;  // a wait gave up: no more waits or work, barriers only
   for (int list = 0; list < 2; ++list) {
     const long n = list_len(a, list);
     if (n == 0) continue;
@@ -590,176 +629,188 @@ __device__ __forceinline__ void attn_consumer(DecSmem& sm, const DecodeArgs& a, 
       const size_t bk = static_cast<size_t>(b) * a.n_kv_heads + kvh;
       const int cnt = list == 1 ? max(0, min(a.cnt[bk], a.kmax) - n_fixed(a)) : nsp;
       const int s_end = min(s + static_cast<int>(run_end - x), cnt);
-      // Q as A fragments: rows g and g+8 are query heads g and g+8 of the
-      // group (zero beyond G); 8 K steps of 16 dims.
-      uint32_t qa[8][4];
+      // Q^T as B fragments: lane (g, c) holds head 8nt+g, dims 16kk+2c(+1)
+      // and 16kk+2c+8(+9); zero for heads beyond the group.
+      uint32_t qb[NT][8][2];
       {
-        const __nv_bfloat16* qb = a.q + (static_cast<size_t>(b) * a.n_q_heads + kvh * G) * kHeadDim;
+        const __nv_bfloat16* qg = a.q + (static_cast<size_t>(b) * a.n_q_heads + kvh * G) * kHeadDim;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const int d0 = 16 * kk + 2 * c;
-          qa[kk][0] = g < G ? *reinterpret_cast<const uint32_t*>(qb + g * kHeadDim + d0) : 0u;
-          qa[kk][1] = g + 8 < G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * kHeadDim + d0) : 0u;
-          qa[kk][2] = g < G ? *reinterpret_cast<const uint32_t*>(qb + g * kHeadDim + d0 + 8) : 0u;
-          qa[kk][3] = g + 8 < G ? *reinterpret_cast<const uint32_t*>(qb + (g + 8) * kHeadDim + d0 + 8) : 0u;
+        for (int nt = 0; nt < NT; ++nt) {
+          const int head = 8 * nt + g;
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const __nv_bfloat16* qr = qg + head * kHeadDim + 16 * kk + 2 * c;
+            qb[nt][kk][0] = head < G ? *reinterpret_cast<const uint32_t*>(qr) : 0u;
+            qb[nt][kk][1] = head < G ? *reinterpret_cast<const uint32_t*>(qr + 8) : 0u;
+          }
         }
       }
-      float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.f, 0.f};
-      float oacc[4][4];
+      // running state of heads 8nt+2c and 8nt+2c+1 over this warp's keys
+      float m_run[NT][2], l_run[NT][2];
+      float oacc[NT][8][4];  // O^T tile dt: dims 16dt+g (+8), heads 8nt+2c (+1)
 #pragma unroll
-      for (int nn = 0; nn < 4; ++nn) oacc[nn][0] = oacc[nn][1] = oacc[nn][2] = oacc[nn][3] = 0.f;
+      for (int nt = 0; nt < NT; ++nt) {
+        m_run[nt][0] = m_run[nt][1] = -INFINITY;
+        l_run[nt][0] = l_run[nt][1] = 0.f;
+#pragma unroll
+        for (int dt = 0; dt < 8; ++dt) oacc[nt][dt][0] = oacc[nt][dt][1] = oacc[nt][dt][2] = oacc[nt][dt][3] = 0.f;
+      }
       for (; s < s_end; ++s, ++used) {
         const uint32_t st = used % kRingStages, ph = (used / kRingStages) & 1u;
-        if (tid == 0) sm.k_ok = mbar_wait(&sm.k_full[st], ph, abort, a.status) ? 1 : 0;
-        consumers_sync();
-        if (!checked_phase(&sm.k_full[st], ph, sm.k_ok)) return;
+        if (dead || !warp_phase_wait(&sm.k_full[st], ph, abort, a.status)) {
+          dead = true;
+          continue;
+        }
         const int nk = sm.nk[st];
         const uint32_t ks = smem_u32(sm.k[st]), vs = smem_u32(sm.v[st]);
-        // S = Q K^T over this warp's 32 keys: 4 n-tiles of 8 keys.  The head
-        // dims are split in two halves with their own accumulators, so each
-        // dependent chain of MMAs is 4 long instead of 8.
-        float sacc[4][4], sac2[4][4];
+        // S^T: tile mt holds keys kbase+16mt+g (rows d0,d1) and +8 (d2,d3);
+        // even and odd dim steps accumulate separately (chains of 4)
+        float sacc[NT][2][4], sac2[NT][2][4];
 #pragma unroll
-        for (int nn = 0; nn < 4; ++nn)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sacc[nn][e] = sac2[nn][e] = 0.f;
+          for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
+            for (int e = 0; e < 4; ++e) sacc[nt][mt][e] = sac2[nt][mt][e] = 0.f;
 #pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int kk = k4 + 4 * half;
+        for (int kk = 0; kk < 8; ++kk) {
 #pragma unroll
-            for (int np = 0; np < 2; ++np) {
-              uint32_t r[4];
-              const int key = kbase + 16 * np + (lane >> 4) * 8 + (lane & 7);
-              const int dim = 16 * kk + ((lane >> 3) & 1) * 8;
-              ldsm_x4(sw128(ks, key, dim), r);
-              float (&acc)[4][4] = half ? sac2 : sacc;
-              mma_bf16(acc[2 * np], qa[kk], r[0], r[1]);
-              mma_bf16(acc[2 * np + 1], qa[kk], r[2], r[3]);
+          for (int mt = 0; mt < 2; ++mt) {
+            uint32_t ra[4];
+            const int key = kbase + 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
+            const int dim = 16 * kk + (lane >> 4) * 8;
+            ldsm_x4(sw128(ks, key, dim), ra);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              float (&acc)[4] = (kk & 1) ? sac2[nt][mt] : sacc[nt][mt];
+              mma_bf16(acc, ra, qb[nt][kk][0], qb[nt][kk][1]);
             }
           }
         }
+        // scale, mask, per-head maximum over the warp's 32 keys
+        float mw[NT][2];
 #pragma unroll
-        for (int nn = 0; nn < 4; ++nn)
+        for (int nt = 0; nt < NT; ++nt) {
+          mw[nt][0] = mw[nt][1] = -INFINITY;
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sacc[nn][e] += sac2[nn][e];
-        // scale to log2 units, mask keys past the span, this warp's maxima
-        float mw[2] = {-INFINITY, -INFINITY};
+          for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
-        for (int nn = 0; nn < 4; ++nn)
+            for (int e = 0; e < 4; ++e) {
+              const int key = kbase + 16 * mt + g + 8 * (e >> 1);
+              const float v = key < nk ? (sacc[nt][mt][e] + sac2[nt][mt][e]) * sl2 : -INFINITY;
+              sacc[nt][mt][e] = v;
+              mw[nt][e & 1] = fmaxf(mw[nt][e & 1], v);
+            }
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int key = kbase + 8 * nn + 2 * c + (e & 1);
-            const float v = key < nk ? sacc[nn][e] * sl2 : -INFINITY;
-            sacc[nn][e] = v;
-            mw[e >> 1] = fmaxf(mw[e >> 1], v);
-          }
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          mw[rr] = fmaxf(mw[rr], __shfl_xor_sync(0xffffffffu, mw[rr], 1));
-          mw[rr] = fmaxf(mw[rr], __shfl_xor_sync(0xffffffffu, mw[rr], 2));
-        }
-        if (c == 0) {
-          sm.red_m[warp][g] = mw[0];
-          sm.red_m[warp][g + 8] = mw[1];
-        }
-        consumers_sync();  // every warp's maxima are posted
-        float mref[2];
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          float ms = sm.red_m[0][g + 8 * rr];
-#pragma unroll
-          for (int w = 1; w < kConsumerWarps; ++w) ms = fmaxf(ms, sm.red_m[w][g + 8 * rr]);
-          const float m_new = fmaxf(m_run[rr], ms);
-          mref[rr] = m_new == -INFINITY ? 0.f : m_new;
-          const float alpha = exp2f(m_run[rr] - mref[rr]);  // 0 while nothing was visible
-          m_run[rr] = m_new;
-          l_run[rr] *= alpha;
-#pragma unroll
-          for (int nn = 0; nn < 4; ++nn) {
-            oacc[nn][2 * rr] *= alpha;
-            oacc[nn][2 * rr + 1] *= alpha;
+          for (int hh = 0; hh < 2; ++hh) {
+            mw[nt][hh] = fmaxf(mw[nt][hh], __shfl_xor_sync(0xffffffffu, mw[nt][hh], 4));
+            mw[nt][hh] = fmaxf(mw[nt][hh], __shfl_xor_sync(0xffffffffu, mw[nt][hh], 8));
+            mw[nt][hh] = fmaxf(mw[nt][hh], __shfl_xor_sync(0xffffffffu, mw[nt][hh], 16));
           }
         }
-        // P = exp2(S - m) as bf16 into shared memory; row sums in fp32
+        // running maximum, rescale of O and l, P = exp2(S - m) as B fragments
+        uint32_t pb[NT][2][2];
 #pragma unroll
-        for (int nn = 0; nn < 4; ++nn) {
-          const float p0 = exp2f(sacc[nn][0] - mref[0]), p1 = exp2f(sacc[nn][1] - mref[0]);
-          const float p2 = exp2f(sacc[nn][2] - mref[1]), p3 = exp2f(sacc[nn][3] - mref[1]);
-          l_run[0] += p0 + p1;
-          l_run[1] += p2 + p3;
-          const int key = kbase + 8 * nn + 2 * c;
-          *reinterpret_cast<uint32_t*>(&sm.p[g][key]) = pack_bf16x2(p0, p1);
-          *reinterpret_cast<uint32_t*>(&sm.p[g + 8][key]) = pack_bf16x2(p2, p3);
-        }
-        if (tid == 0) sm.v_ok = mbar_wait(&sm.v_full[st], ph, abort, a.status) ? 1 : 0;
-        consumers_sync();  // P is complete; V has arrived
-        if (!checked_phase(&sm.v_full[st], ph, sm.v_ok)) return;
-        // O += P V over all 128 keys of the span for this warp's 32 dims;
-        // odd key steps accumulate separately (two chains of 4 MMAs).
-        float ob[4][4];
+        for (int nt = 0; nt < NT; ++nt) {
+          float mref[2];
 #pragma unroll
-        for (int nn = 0; nn < 4; ++nn) ob[nn][0] = ob[nn][1] = ob[nn][2] = ob[nn][3] = 0.f;
+          for (int hh = 0; hh < 2; ++hh) {
+            const float m_new = fmaxf(m_run[nt][hh], mw[nt][hh]);
+            mref[hh] = m_new == -INFINITY ? 0.f : m_new;
+            const float alpha = exp2f(m_run[nt][hh] - mref[hh]);  // 0 while nothing was visible
+            m_run[nt][hh] = m_new;
+            l_run[nt][hh] *= alpha;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          uint32_t pa[4];
-          const int prow = (lane & 7) + ((lane >> 3) & 1) * 8;
-          ldsm_x4(p_base + static_cast<uint32_t>(prow * kPRowElems + 16 * kk + (lane >> 4) * 8) * 2u, pa);
+            for (int dt = 0; dt < 8; ++dt) {
+              oacc[nt][dt][hh] *= alpha;
+              oacc[nt][dt][2 + hh] *= alpha;
+            }
+          }
 #pragma unroll
-          for (int dp = 0; dp < 2; ++dp) {
-            uint32_t r[4];
-            const int key = 16 * kk + ((lane >> 3) & 1) * 8 + (lane & 7);
-            const int dim = dbase + 16 * dp + (lane >> 4) * 8;
-            ldsm_x4_t(sw128(vs, key, dim), r);
-            float (&acc)[4][4] = (kk & 1) ? ob : oacc;
-            mma_bf16(acc[2 * dp], pa, r[0], r[1]);
-            mma_bf16(acc[2 * dp + 1], pa, r[2], r[3]);
+          for (int mt = 0; mt < 2; ++mt) {
+            const float p0 = exp2f(sacc[nt][mt][0] - mref[0]), p1 = exp2f(sacc[nt][mt][1] - mref[1]);
+            const float p2 = exp2f(sacc[nt][mt][2] - mref[0]), p3 = exp2f(sacc[nt][mt][3] - mref[1]);
+            l_run[nt][0] += p0 + p2;
+            l_run[nt][1] += p1 + p3;
+            // (key g, heads 2c..2c+1) and (key g+8, ...) -> (keys 2c..2c+1, head g), (keys 2c+8.., head g)
+            pb[nt][mt][0] = movmatrix_trans(pack_bf16x2(p0, p1));
+            pb[nt][mt][1] = movmatrix_trans(pack_bf16x2(p2, p3));
           }
         }
+        if (!warp_phase_wait(&sm.v_full[st], ph, abort, a.status)) {
+          dead = true;
+          continue;
+        }
+        // O^T += V^T P^T: A = V^T tile (dims 16dt.., keys 16mt..) by ldmatrix.trans
 #pragma unroll
-        for (int nn = 0; nn < 4; ++nn)
+        for (int dt = 0; dt < 8; ++dt) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) oacc[nn][e] += ob[nn][e];
+          for (int mt = 0; mt < 2; ++mt) {
+            uint32_t ra[4];
+            const int key = kbase + 16 * mt + (lane & 7) + ((lane >> 4) & 1) * 8;
+            const int dim = 16 * dt + ((lane >> 3) & 1) * 8;
+            ldsm_x4_t(sw128(vs, key, dim), ra);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_bf16(oacc[nt][dt], ra, pb[nt][mt][0], pb[nt][mt][1]);
+          }
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.empty[st]);
       }
-      // end of the run: row sums over the quad, then over the four warps
+      // end of the run: merge the four warps, 8 heads at a time
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 1);
-        l_run[rr] += __shfl_xor_sync(0xffffffffu, l_run[rr], 2);
-      }
-      if (c == 0) {
-        sm.red_l[warp][g] = l_run[0];
-        sm.red_l[warp][g + 8] = l_run[1];
-      }
-      consumers_sync();  // every warp's row sums are posted
-      float* part = run_partial(a, list, run_start);
+      for (int nt = 0; nt < NT; ++nt) {
+        float lsum[2];
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int row = g + 8 * rr;
-        if (row < G) {
-          float* pr = part + row * kPartStride;
-          if (warp == 0 && c == 0) {
-            float L = 0.f;
+        for (int hh = 0; hh < 2; ++hh) {
+          float v = l_run[nt][hh];
+          v += __shfl_xor_sync(0xffffffffu, v, 4);
+          v += __shfl_xor_sync(0xffffffffu, v, 8);
+          v += __shfl_xor_sync(0xffffffffu, v, 16);
+          lsum[hh] = v;
+        }
+        if (g == 0) {
+          sm.wm[warp][2 * c] = m_run[nt][0];
+          sm.wm[warp][2 * c + 1] = m_run[nt][1];
+          sm.wl[warp][2 * c] = lsum[0];
+          sm.wl[warp][2 * c + 1] = lsum[1];
+        }
 #pragma unroll
-            for (int w = 0; w < kConsumerWarps; ++w) L += sm.red_l[w][row];
-            pr[0] = m_run[rr];
+        for (int dt = 0; dt < 8; ++dt) {
+          *reinterpret_cast<float2*>(&sm.wo[warp][16 * dt + g][2 * c]) = make_float2(oacc[nt][dt][0], oacc[nt][dt][1]);
+          *reinterpret_cast<float2*>(&sm.wo[warp][16 * dt + g + 8][2 * c]) =
+              make_float2(oacc[nt][dt][2], oacc[nt][dt][3]);
+        }
+        consumers_sync();  // every warp's m, l and O^T are posted
+        // thread d: output dim d of the 8 heads
+        float* part = run_partial(a, list, run_start);
+        const int d = tid;
+        for (int hh = 0; hh < 8 && 8 * nt + hh < G; ++hh) {
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.wm[w][hh]);
+          float L = 0.f, o = 0.f;
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) {
+            const float f = sm.wm[w][hh] == -INFINITY ? 0.f : exp2f(sm.wm[w][hh] - M);
+            L = fmaf(f, sm.wl[w][hh], L);
+            o = fmaf(f, sm.wo[w][d][hh], o);
+          }
+          float* pr = part + (8 * nt + hh) * kPartStride;
+          pr[4 + d] = o;
+          if (d == 0) {
+            pr[0] = M;
             pr[1] = L;
           }
-#pragma unroll
-          for (int nn = 0; nn < 4; ++nn)
-            *reinterpret_cast<float2*>(pr + 4 + dbase + 8 * nn + 2 * c) =
-                make_float2(oacc[nn][2 * rr], oacc[nn][2 * rr + 1]);
         }
+        consumers_sync();  // wo, wm and wl are free again
       }
-      consumers_sync();  // red_l is free again
       x = run_end;
     }
   }
 }
 
+template <int NT>
 __global__ void __launch_bounds__(kAttnThreads, 2) decode_attn_kernel(const __grid_constant__ CUtensorMap mk,
                                                                        const __grid_constant__ CUtensorMap mv,
                                                                        const __grid_constant__ DecodeArgs a) {
@@ -786,7 +837,7 @@ __global__ void __launch_bounds__(kAttnThreads, 2) decode_attn_kernel(const __gr
     }
     attn_producer(sm, &mk, &mv, a, abort);
   } else {
-    attn_consumer(sm, a, abort);
+    attn_consumer<NT>(sm, a, abort);
   }
 }
 
@@ -913,8 +964,11 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUte
   // All three kernels prefer the largest shared-memory carveout: an SM that
   // a selection or combine CTA has configured for little shared memory could
   // not take an attention CTA until it drains.
-  for (const void* fn : {reinterpret_cast<const void*>(decode_select_kernel),
-                         reinterpret_cast<const void*>(decode_attn_kernel),
+  // The attention kernel is compiled for one or two tiles of 8 query heads.
+  const bool two_tiles = a.group > 8;
+  const void* attn = two_tiles ? reinterpret_cast<const void*>(decode_attn_kernel<2>)
+                               : reinterpret_cast<const void*>(decode_attn_kernel<1>);
+  for (const void* fn : {reinterpret_cast<const void*>(decode_select_kernel), attn,
                          reinterpret_cast<const void*>(decode_combine_kernel)}) {
     cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout,
                                          static_cast<int>(cudaSharedmemCarveoutMaxShared));
@@ -929,8 +983,7 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUte
   decode_select_kernel<<<dim3(kSelCluster * a.n_kv_heads, a.batch), kDecSelThreads, sel_smem, stream>>>(a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(kDecSmemBytes));
+  e = cudaFuncSetAttribute(attn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kDecSmemBytes));
   if (e != cudaSuccess) return e;
   // Programmatic dependent launches: each kernel may begin while the
   // previous one finishes; griddepcontrol.wait orders the data it reads.
@@ -944,7 +997,8 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUte
   cfg.stream = stream;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, decode_attn_kernel, mk, mv, a);
+  e = two_tiles ? cudaLaunchKernelEx(&cfg, decode_attn_kernel<2>, mk, mv, a)
+                : cudaLaunchKernelEx(&cfg, decode_attn_kernel<1>, mk, mv, a);
   if (e != cudaSuccess) return e;
   cfg.gridDim = dim3(a.n_q_heads, a.batch);
   cfg.blockDim = dim3(kCombineThreads);

@@ -81,6 +81,8 @@ DECODE_CASES = [
     # top-k above 32 (radix path): one round, then several rounds per CTA
     (1, 8, 2, [2, 0], 8192, 1024, 128, 40, 2),
     (1, 4, 1, [2], 196608, 128, 64, 48, 2),
+    # group of 16 query heads per KV head (two tiles of 8 heads in the attention MMAs)
+    (2, 32, 2, [2, 0], 4096, 1000, 128, 4, 2),
 ]
 
 
