@@ -360,20 +360,10 @@ def time_decode(rtp, steps, device):
     d = inputs.decode_step(w, device)
     kinds = d["kinds"]
     Lc = d["cache_len"]
-    # cached centroids come from the library's own indexer run over the cache
-    cfgp = rtp.AttnConfig(1, Lc, w.n_q_heads, w.n_kv_heads, w.window, w.block, w.topk, w.n_local)
+    # cached centroids: the library's bulk build over the whole cache (timed below)
+    cfg = rtp.AttnConfig(w.batch, Lc, w.n_q_heads, w.n_kv_heads, w.window, w.block, w.topk, w.n_local)
     C = torch.zeros(w.batch, w.n_kv_heads, Lc // w.block, 16, dtype=torch.float32, device=device)
-    qdummy = torch.zeros(1, w.n_q_heads, Lc, 128, dtype=torch.bfloat16, device=device)
-    for b in range(w.batch):
-        plan = rtp.Plan(cfgp, kinds)
-        bufs = plan.buffers(device)
-        rtp.rtp_indexer_project(plan.handle, qdummy, d["kcache"][b:b + 1].contiguous(), d["proj"],
-                                bufs["centroids"], bufs["qbar"])
-        for s, h in enumerate(plan.slot_heads):
-            C[b, h] = bufs["centroids"][0, s]
-        plan.close()
-    del qdummy
-    cfg = rtp.AttnConfig(w.batch, 1, w.n_q_heads, w.n_kv_heads, w.window, w.block, w.topk, w.n_local)
+    rtp.rtp_cache_centroids(cfg, kinds, Lc, d["kcache"], d["proj"], C)
     ws_bytes = rtp.rtp_decode_workspace_bytes(cfg, kinds, Lc)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
     o = torch.empty_like(d["q"])
@@ -400,6 +390,7 @@ def time_decode(rtp, steps, device):
     torch.cuda.synchronize()
     ms = statistics.median(a.elapsed_time(b) for a, b in times)
     status = rtp.rtp_last_device_status(stream)
+    upkeep = time_cache_upkeep(rtp, w, d, C, cfg, flush, flush_read, steps, stream)
     G = w.group
     ns = sum(1 for k in kinds if k == inputs.SPARSE)
     nsw = len(kinds) - ns
@@ -409,7 +400,49 @@ def time_decode(rtp, steps, device):
     flops = w.batch * keys * G * 4 * 128
     return {"workload": w.name, "ms_per_step": ms, "algorithmic_bytes": bytes_, "gb_s": bytes_ / (ms * 1e-3) / 1e9,
             "tflops_effective": flops / (ms * 1e-3) / 1e12, "l2": "flushed before each step (256 MB write, then 256 MB read)",
-            "launches_per_step": 3, "status": rtp.status_str(status)}
+            "launches_per_step": 3, "status": rtp.status_str(status), "cache_upkeep": upkeep}
+
+
+def time_cache_upkeep(rtp, w, d, C, cfg, flush, flush_read, steps, stream):
+    """The KV-cache calls on the decode workload: the bulk centroid build over
+    every cached block, and one append (new K/V row; the row completes a block,
+    so its centroid is recomputed for each retrieval head).  The appended row
+    is the cache's own last row, so the cache keeps its contents."""
+    kinds, Lc = d["kinds"], d["cache_len"]
+    ns = sum(1 for k in kinds if k == inputs.SPARSE)
+
+    def timed(fn, n):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        ev = []
+        for _ in range(n):
+            flush.zero_()
+            flush_read.sum()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            ev.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+    build_ms = timed(lambda: rtp.rtp_cache_centroids(cfg, kinds, Lc, d["kcache"], d["proj"], C, stream=stream), 10)
+    build_bytes = w.batch * ns * (Lc // w.block) * (w.block * 128 * 2 + 16 * 4)
+    k_new = d["kcache"][:, :, Lc - 1].contiguous()
+    v_new = d["vcache"][:, :, Lc - 1].contiguous()
+    app_ms = timed(lambda: rtp.rtp_cache_append(cfg, kinds, Lc - 1, k_new, v_new, d["kcache"], d["vcache"],
+                                                d["proj"], C, stream=stream), min(steps, 64))
+    app_bytes = w.batch * w.n_kv_heads * 4 * 128 * 2 + w.batch * ns * (w.block * 128 * 2 + 16 * 4)
+    k_mid = d["kcache"][:, :, Lc - 2].contiguous()
+    v_mid = d["vcache"][:, :, Lc - 2].contiguous()
+    row_ms = timed(lambda: rtp.rtp_cache_append(cfg, kinds, Lc - 2, k_mid, v_mid, d["kcache"], d["vcache"],
+                                                d["proj"], C, stream=stream), min(steps, 64))
+    return {"append_row_only_us": row_ms * 1e3,"centroid_build_ms": build_ms, "centroid_build_algorithmic_bytes": build_bytes,
+            "centroid_build_gb_s": build_bytes / (build_ms * 1e-3) / 1e9,
+            "append_us": app_ms * 1e3, "append_algorithmic_bytes": app_bytes,
+            "append_note": "row completes a block: its centroid is recomputed for every retrieval head"}
 
 
 # ---------------------------------------------------------------- oracle arm

@@ -73,7 +73,9 @@ enum { RTP_HEAD_SWA = 0, RTP_HEAD_FULL = 1, RTP_HEAD_SPARSE = 2 };
 
 typedef struct {
   int batch;       /* sequences                                                  */
-  int seq;         /* tokens per sequence (prefill); multiple of `block`         */
+  int seq;         /* tokens per sequence (prefill); multiple of `block`.
+                      Decode and cache calls: rows allocated per (sequence,
+                      KV head) in the cache (its capacity)                      */
   int n_q_heads;   /* query heads                                                */
   int n_kv_heads;  /* KV heads; group = n_q_heads / n_kv_heads must be an even
                       integer <= 16 (prefill processes query heads in pairs)     */
@@ -180,15 +182,19 @@ rtp_status rtp_hybrid_prefill(const rtp_plan* plan, const void* q, const void* k
  * streaming heads keep a window).  The new token's K/V are already the last
  * cache entry, so the query sits at position cache_len-1.
  *   cfg        batch, n_q_heads, n_kv_heads, head_dim, window, block, rank,
- *              topk, n_sink, n_local, scale are used; seq is ignored
+ *              topk, n_sink, n_local, scale are used; seq is the cache
+ *              capacity (see below)
  *   kind_host  HOST [n_kv_heads] (n_kv_heads <= 256): RTP_HEAD_SPARSE
  *              (retrieval) or RTP_HEAD_SWA; RTP_HEAD_FULL attends to the
  *              whole cache
  *   q          bf16 [batch][n_q_heads][1][128]
- *   kcache, vcache  bf16 [batch][n_kv_heads][cache_len][128]
- *   centroids  fp32 [batch][n_kv_heads][cache_len/block][16]: centroid of
- *              every complete cache block (entries of non-retrieval heads
- *              are not read)
+ *   kcache, vcache  bf16 [batch][n_kv_heads][cap][128], of which rows
+ *              0..cache_len-1 are read; cap = cfg->seq when cfg->seq >=
+ *              cache_len (a cache allocated once and filled by
+ *              rtp_cache_append), else cap = cache_len
+ *   centroids  fp32 [batch][n_kv_heads][cap/block][16]: centroid of every
+ *              complete cache block (entries of non-retrieval heads are not
+ *              read; see rtp_cache_centroids / rtp_cache_append)
  *   proj       fp32 [128][16]
  *   o          bf16 [batch][n_q_heads][1][128] (out)
  *   workspace  device scratch of at least rtp_decode_workspace_bytes bytes
@@ -231,6 +237,58 @@ rtp_status rtp_sparse_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, 
 rtp_status rtp_sparse_decode_noalloc(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* q,
                                      const void* kcache, const void* vcache, const float* centroids,
                                      const float* proj, void* o, int32_t* sel_out, int32_t* cnt_out, void* stream);
+
+/* ------------------------------------------------------------------------
+ * rtp_cache_centroids — block centroids of a KV cache in the layout the
+ * decode step reads (RTPurboV2 page: decode scores the centroids of the
+ * projected cached keys; the same page describes running full attention in
+ * prefill and clustering the K cache afterwards, which is this call after an
+ * rtp_hybrid_prefill with RTP_HEAD_FULL heads).
+ *   cfg        batch, n_kv_heads, head_dim, block, rank used (validated as
+ *              for rtp_sparse_decode); seq = cache capacity as there
+ *   kind_host  HOST [n_kv_heads]: only RTP_HEAD_SPARSE heads are written
+ *   cache_len  rows held per (sequence, KV head), >= 1; the complete blocks
+ *              0 .. cache_len/block - 1 are written
+ *   kcache     bf16 [batch][n_kv_heads][cap][128] (device)
+ *   proj       fp32 [128][16] (device)
+ *   centroids  fp32 [batch][n_kv_heads][cap/block][16] (device, out):
+ *              c_b = (1/block) sum_{j in block b} proj^T k_j, summed in the
+ *              fixed order of rtp_indexer_project (same fp32 value for the
+ *              same keys); other entries are left untouched
+ * centroids and proj may be NULL when no head is RTP_HEAD_SPARSE.
+ * Errors: RTP_ERR_INVALID_ARG (bad cfg, kind, length, NULL or unaligned
+ * pointer; nothing launched), RTP_ERR_CUDA (launch failure).
+ * ---------------------------------------------------------------------- */
+rtp_status rtp_cache_centroids(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* kcache,
+                               const float* proj, float* centroids, void* stream);
+
+/* ------------------------------------------------------------------------
+ * rtp_cache_append — append one token per sequence to a KV cache of fixed
+ * capacity and keep the centroids current (RTPurboV2 page: the centroids of
+ * the projected keys stand for their cache blocks in decode; a block's
+ * centroid is defined once its last row is cached, and the block of the
+ * newest token is always one of the local blocks the decode step reads in
+ * full).
+ *   cfg        as for rtp_cache_centroids; seq = capacity cap (rows
+ *              allocated per (sequence, KV head)), required
+ *   kind_host  HOST [n_kv_heads]
+ *   pos        row of the new token = rows already cached, 0 <= pos < cap
+ *   k_new, v_new  bf16 [batch][n_kv_heads][128] (device)
+ *   kcache, vcache  bf16 [batch][n_kv_heads][cap][128] (device, in/out):
+ *              row pos is written, no other row
+ *   proj       fp32 [128][16] (device)
+ *   centroids  fp32 [batch][n_kv_heads][cap/block][16] (device, in/out):
+ *              when (pos+1) % block == 0, entry (pos+1)/block - 1 of every
+ *              RTP_HEAD_SPARSE head is written (as rtp_cache_centroids
+ *              would write it); nothing else
+ * After the call, rtp_sparse_decode with cache_len = pos + 1 and the same
+ * cfg (seq = cap) decodes the new token.
+ * Errors: RTP_ERR_INVALID_ARG (bad cfg, kind, pos, NULL or unaligned
+ * pointer; nothing launched), RTP_ERR_CUDA (launch failure).
+ * ---------------------------------------------------------------------- */
+rtp_status rtp_cache_append(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int pos, const void* k_new,
+                            const void* v_new, void* kcache, void* vcache, const float* proj, float* centroids,
+                            void* stream);
 
 /* ------------------------------------------------------------------------
  * rtp_last_device_status — synchronise `stream`, then read and clear the

@@ -219,6 +219,52 @@ def decode_head(q_group, kc_head, vc_head, C_head, proj, mode: int, window: int,
     return out, s, int(c[0]), float(kth[0])
 
 
+def cache_centroids(kcache, cache_len: int, kinds, block: int, proj, C=None) -> np.ndarray:
+    """Centroids of the complete blocks of a KV cache (RTPurboV2 page: decode
+    scores the centroids of the projected cached keys; clustering the K cache
+    after a full-attention prefill).
+
+    kcache: bf16 [batch][H][cap][128] (torch tensor or uint16 bit array).
+    Returns fp64 [batch][H][cap // block][16]: for every head of kind SPARSE,
+    block b < cache_len // block holds the mean of P^T k_j over the block's
+    rows; every other entry is copied from C (NaN when C is None).
+    """
+    kb = _bf16_bits(kcache)
+    nb_, H, cap = kb.shape[0], kb.shape[1], kb.shape[2]
+    nbc = cap // block
+    out = np.full((nb_, H, nbc, 16), np.nan) if C is None else np.array(C, dtype=np.float64, copy=True)
+    n = (cache_len // block) * block
+    for b in range(nb_):
+        for h in range(H):
+            if int(kinds[h]) == SPARSE and n > 0:
+                out[b, h, : n // block] = centroids(kb[b, h, :n], block, proj)
+    return out
+
+
+def cache_append(kcache, vcache, C, kinds, pos: int, k_new, v_new, block: int, proj):
+    """One token appended to a KV cache of fixed capacity (RTPurboV2 page: a
+    block's centroid stands for its keys once all of them are cached).
+
+    Row `pos` of every (sequence, head) becomes k_new / v_new
+    ([batch][H][128]).  If that row is the last of its block, the block's
+    centroid is (re)computed for every SPARSE head from the cached rows of the
+    block; no other centroid changes.  Returns new arrays (kcache, vcache as
+    uint16 bf16 bits, C as fp64); the inputs are not modified.
+    """
+    kc = _bf16_bits(kcache).copy()
+    vc = _bf16_bits(vcache).copy()
+    Cn = np.array(C, dtype=np.float64, copy=True)
+    kc[:, :, pos] = _bf16_bits(k_new).reshape(kc.shape[0], kc.shape[1], 128)
+    vc[:, :, pos] = _bf16_bits(v_new).reshape(vc.shape[0], vc.shape[1], 128)
+    if (pos + 1) % block == 0:
+        blk = (pos + 1) // block - 1
+        for b in range(kc.shape[0]):
+            for h in range(kc.shape[1]):
+                if int(kinds[h]) == SPARSE:
+                    Cn[b, h, blk] = centroids(kc[b, h, blk * block:(blk + 1) * block], block, proj)[0]
+    return kc, vc, Cn
+
+
 def round_bf16(x: np.ndarray) -> np.ndarray:
     """Round fp64 values to the nearest bf16 (ties to even), returned as fp64."""
     f = np.asarray(x, dtype=np.float64).astype(np.float32)

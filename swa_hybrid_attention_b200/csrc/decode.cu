@@ -497,8 +497,8 @@ __device__ __forceinline__ void attn_producer(DecSmem& sm, const CUtensorMap* mk
       const int s_end = min(s + static_cast<int>(run_end - x), cnt);
       const bool sparse = a.kind[kvh] == KIND_SPARSE;
       const int start = a.kind[kvh] == KIND_SWA ? max(0, a.cache_len - a.window) : 0;
-      const __nv_bfloat16* kbase = a.kcache + bk * static_cast<size_t>(a.cache_len) * kHeadDim;
-      const __nv_bfloat16* vbase = a.vcache + bk * static_cast<size_t>(a.cache_len) * kHeadDim;
+      const __nv_bfloat16* kbase = a.kcache + bk * static_cast<size_t>(a.cache_cap) * kHeadDim;
+      const __nv_bfloat16* vbase = a.vcache + bk * static_cast<size_t>(a.cache_cap) * kHeadDim;
       for (int s0 = s; s0 < s_end && ok; s0 += 32) {
         const int m = min(32, s_end - s0);
         // lane l: key range of span s0 + l

@@ -16,45 +16,19 @@
 // reads 16 bytes (8 bf16) per row; 16 threads cover a row, so a warp reads two
 // full 256-byte rows per instruction (coalesced).  The 16 row-groups' partial
 // sums are reduced through shared memory in a fixed order, so results are
-// bit-reproducible.
+// bit-reproducible (and equal to the KV-cache centroids of cache.cu, which
+// use the same order).
 
 #include <cuda_bf16.h>
 
 #include "internal.cuh"
+#include "row_sum.cuh"
 
 namespace rtp {
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kRowGroups = kThreads / 16;  // rows read per pass
-
-__device__ __forceinline__ void accum_row8(float (&acc)[8], const uint4 v) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    float2 f = __bfloat1622float2(h[e]);
-    acc[2 * e] += f.x;
-    acc[2 * e + 1] += f.y;
-  }
-}
-
-// Sum `rows` consecutive 128-wide bf16 rows starting at `base` into acc
-// (this thread's 8 columns), 4 loads in flight per thread.
-__device__ __forceinline__ void sum_rows(float (&acc)[8], const __nv_bfloat16* base, int rows, int rg, int cg) {
-  const uint4* p = reinterpret_cast<const uint4*>(base) + cg;
-  int r = rg;
-  for (; r + 3 * kRowGroups < rows; r += 4 * kRowGroups) {
-    uint4 v0 = __ldg(p + static_cast<size_t>(r) * 16);
-    uint4 v1 = __ldg(p + static_cast<size_t>(r + kRowGroups) * 16);
-    uint4 v2 = __ldg(p + static_cast<size_t>(r + 2 * kRowGroups) * 16);
-    uint4 v3 = __ldg(p + static_cast<size_t>(r + 3 * kRowGroups) * 16);
-    accum_row8(acc, v0);
-    accum_row8(acc, v1);
-    accum_row8(acc, v2);
-    accum_row8(acc, v3);
-  }
-  for (; r < rows; r += kRowGroups) accum_row8(acc, __ldg(p + static_cast<size_t>(r) * 16));
-}
+constexpr int kThreads = kSumThreads;
+constexpr int kRowGroups = kSumRowGroups;  // rows read per pass
 
 __global__ void __launch_bounds__(kThreads) indexer_kernel(const IndexerArgs a) {
   __shared__ float part[2][kRowGroups][kHeadDim];

@@ -48,16 +48,16 @@ constexpr int kMaxDecodeKvHeads = 256;
 
 struct DecodeArgs {
   const __nv_bfloat16* q;       // [batch][n_q_heads][128]
-  const __nv_bfloat16* kcache;  // [batch][n_kv_heads][cache_len][128]
+  const __nv_bfloat16* kcache;  // [batch][n_kv_heads][cache_cap][128], rows < cache_len used
   const __nv_bfloat16* vcache;
-  const float* centroids;       // [batch][n_kv_heads][nbc][16]
+  const float* centroids;       // [batch][n_kv_heads][nbc][16], nbc = cache_cap / block
   const float* proj;
   __nv_bfloat16* o;             // [batch][n_q_heads][128]
   uint8_t kind[kMaxDecodeKvHeads];  // routing map, passed by value
   int32_t* sel;                 // [batch][n_kv_heads][kmax] (workspace or caller)
   int32_t* cnt;                 // [batch][n_kv_heads]
   float* partial;               // [n_spans of both lists][group][kPartStride]
-  int batch, n_q_heads, n_kv_heads, group, cache_len, nbc;
+  int batch, n_q_heads, n_kv_heads, group, cache_len, cache_cap, nbc;
   int window, block, topk, n_local, kmax;
   float scale_log2;
   uint32_t* status;
@@ -74,12 +74,29 @@ struct DecodeArgs {
 };
 constexpr int kPartStride = 132;  // m, l, pad, pad, o[128]
 
+// KV-cache maintenance: appending one token per sequence, and the block
+// centroids of retrieval heads in the layout the decode step reads.
+struct CacheArgs {
+  const __nv_bfloat16* k_new;  // [batch][n_kv_heads][128] (append only)
+  const __nv_bfloat16* v_new;
+  __nv_bfloat16* kcache;       // [batch][n_kv_heads][cache_cap][128]
+  __nv_bfloat16* vcache;
+  const float* proj;           // [128][16]
+  float* centroids;            // [batch][n_kv_heads][cache_cap / block][16]
+  uint8_t kind[kMaxDecodeKvHeads];
+  int batch, n_kv_heads, cache_cap, block;
+  int pos;       // append: row of the new token
+  int n_blocks;  // centroid build: complete blocks to write
+};
+
 // Launchers (return the launch error, never synchronise).
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                            int num_ctas, cudaStream_t stream);
 cudaError_t launch_indexer(const IndexerArgs& a, cudaStream_t stream);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t stream);
+cudaError_t launch_cache_append(const CacheArgs& a, cudaStream_t stream);
+cudaError_t launch_cache_centroids(const CacheArgs& a, cudaStream_t stream);
 
 // Fixed-size device scratch used by the allocation-free decode entry point.
 constexpr size_t kDecodeStaticScratchBytes = size_t(16) << 20;

@@ -91,15 +91,18 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 [slabs][rows][128] viewed as a 3-D tensor, 128-byte swizzled boxes of
-// 64 columns x box_rows rows.  Rows past `rows` read as zero.
-bool encode_bf16_3d(CUtensorMap* map, const void* base, long rows, long slabs, int box_rows) {
+// bf16 [slabs][slab_rows][128] viewed as a 3-D tensor of which the first
+// `rows` rows of each slab are used (slab_rows = 0 means rows), 128-byte
+// swizzled boxes of 64 columns x box_rows rows.  Rows past `rows` read as
+// zero.
+bool encode_bf16_3d(CUtensorMap* map, const void* base, long rows, long slabs, int box_rows, long slab_rows = 0) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
+  if (slab_rows < rows) slab_rows = rows;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(slabs)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim) * 2,
-                           static_cast<cuuint64_t>(kHeadDim) * 2 * static_cast<cuuint64_t>(rows)};
+                           static_cast<cuuint64_t>(kHeadDim) * 2 * static_cast<cuuint64_t>(slab_rows)};
   cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -382,6 +385,10 @@ struct DecodeLayout {
   int span_off[2][kMaxDecodeKvHeads];
 };
 
+// Rows allocated per (sequence, KV head) in a decode-time cache: cfg->seq
+// when it is at least cache_len, else exactly cache_len.
+int decode_capacity(const rtp_attn_cfg* c, int cache_len) { return c->seq > cache_len ? c->seq : cache_len; }
+
 bool decode_layout(const rtp_attn_cfg* c, const uint8_t* kind, int cache_len, DecodeLayout& L) {
   if (!cfg_common_ok(c) || !kind || cache_len < 1) return false;
   if (static_cast<long>(cache_len) / c->block * 4 > 200 * 1024) return false;
@@ -448,6 +455,36 @@ bool decode_schedule(const rtp_attn_cfg* c, const DecodeLayout& L, DecodeArgs& a
   for (int l = 0; l < 2; ++l) std::memcpy(a.span_off[l], L.span_off[l], sizeof(int) * c->n_kv_heads);
   return true;
 }
+
+// Shared validation of the KV-cache maintenance calls; fills the common
+// fields of CacheArgs.
+rtp_status cache_args(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cap, const void* kcache,
+                      const float* proj, float* centroids, CacheArgs& a) {
+  if (!cfg_common_ok(cfg) || !kind_host || !kcache) return RTP_ERR_INVALID_ARG;
+  if (cfg->n_kv_heads > kMaxDecodeKvHeads || cfg->batch > 65535 || cap < 1) return RTP_ERR_INVALID_ARG;
+  bool any_sparse = false;
+  for (int h = 0; h < cfg->n_kv_heads; ++h) {
+    if (kind_host[h] > RTP_HEAD_SPARSE) return RTP_ERR_INVALID_ARG;
+    any_sparse |= kind_host[h] == RTP_HEAD_SPARSE;
+  }
+  if (any_sparse && (!centroids || !proj)) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(kcache) || (centroids && !aligned16(centroids)) || (proj && !aligned16(proj)))
+    return RTP_ERR_INVALID_ARG;
+  std::memset(a.kind, 0, sizeof(a.kind));
+  std::memcpy(a.kind, kind_host, cfg->n_kv_heads);
+  a.kcache = static_cast<__nv_bfloat16*>(const_cast<void*>(kcache));
+  a.proj = proj;
+  a.centroids = centroids;
+  a.batch = cfg->batch;
+  a.n_kv_heads = cfg->n_kv_heads;
+  a.cache_cap = cap;
+  a.block = cfg->block;
+  a.k_new = a.v_new = nullptr;
+  a.vcache = nullptr;
+  a.pos = 0;
+  a.n_blocks = 0;
+  return RTP_OK;
+}
 }  // namespace
 
 size_t rtp_decode_workspace_bytes(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len) {
@@ -489,7 +526,8 @@ rtp_status rtp_sparse_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, 
   a.n_kv_heads = cfg->n_kv_heads;
   a.group = cfg->n_q_heads / cfg->n_kv_heads;
   a.cache_len = cache_len;
-  a.nbc = cache_len / cfg->block;
+  a.cache_cap = decode_capacity(cfg, cache_len);
+  a.nbc = a.cache_cap / cfg->block;
   a.window = cfg->window;
   a.block = cfg->block;
   a.topk = cfg->topk;
@@ -500,8 +538,8 @@ rtp_status rtp_sparse_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, 
   a.status = status_word(current_device());
   if (!a.status) return RTP_ERR_NO_MEMORY;
   CUtensorMap mk, mv;
-  if (!encode_bf16_3d(&mk, kcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64) ||
-      !encode_bf16_3d(&mv, vcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64))
+  if (!encode_bf16_3d(&mk, kcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64, a.cache_cap) ||
+      !encode_bf16_3d(&mv, vcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64, a.cache_cap))
     return RTP_ERR_CUDA;
   return cuda_status(launch_decode(a, mk, mv, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -540,7 +578,8 @@ rtp_status rtp_sparse_decode_noalloc(const rtp_attn_cfg* cfg, const uint8_t* kin
   a.n_kv_heads = cfg->n_kv_heads;
   a.group = cfg->n_q_heads / cfg->n_kv_heads;
   a.cache_len = cache_len;
-  a.nbc = cache_len / cfg->block;
+  a.cache_cap = decode_capacity(cfg, cache_len);
+  a.nbc = a.cache_cap / cfg->block;
   a.window = cfg->window;
   a.block = cfg->block;
   a.topk = cfg->topk;
@@ -550,10 +589,37 @@ rtp_status rtp_sparse_decode_noalloc(const rtp_attn_cfg* cfg, const uint8_t* kin
   if (!decode_schedule(cfg, L, a)) return RTP_ERR_CUDA;
   a.status = nullptr;  // no status word: getting one may allocate
   CUtensorMap mk, mv;
-  if (!encode_bf16_3d(&mk, kcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64) ||
-      !encode_bf16_3d(&mv, vcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64))
+  if (!encode_bf16_3d(&mk, kcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64, a.cache_cap) ||
+      !encode_bf16_3d(&mv, vcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64, a.cache_cap))
     return RTP_ERR_CUDA;
   return cuda_status(launch_decode(a, mk, mv, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+
+rtp_status rtp_cache_centroids(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* kcache,
+                               const float* proj, float* centroids, void* stream) {
+  if (!cfg || cache_len < 1) return RTP_ERR_INVALID_ARG;
+  CacheArgs a;
+  const rtp_status st = cache_args(cfg, kind_host, decode_capacity(cfg, cache_len), kcache, proj, centroids, a);
+  if (st != RTP_OK) return st;
+  a.n_blocks = cache_len / cfg->block;
+  return cuda_status(launch_cache_centroids(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rtp_status rtp_cache_append(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int pos, const void* k_new,
+                            const void* v_new, void* kcache, void* vcache, const float* proj, float* centroids,
+                            void* stream) {
+  if (!cfg || pos < 0 || pos >= cfg->seq) return RTP_ERR_INVALID_ARG;
+  CacheArgs a;
+  const rtp_status st = cache_args(cfg, kind_host, cfg->seq, kcache, proj, centroids, a);
+  if (st != RTP_OK) return st;
+  if (!k_new || !v_new || !vcache || !aligned16(k_new) || !aligned16(v_new) || !aligned16(vcache))
+    return RTP_ERR_INVALID_ARG;
+  a.k_new = static_cast<const __nv_bfloat16*>(k_new);
+  a.v_new = static_cast<const __nv_bfloat16*>(v_new);
+  a.vcache = static_cast<__nv_bfloat16*>(vcache);
+  a.pos = pos;
+  return cuda_status(launch_cache_append(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 rtp_status rtp_selftest_bounded_wait(unsigned limit_ms, void* stream) {

@@ -59,6 +59,8 @@ def _load() -> ctypes.CDLL:
         "rtp_decode_workspace_bytes": (S, [cfgp, P, I]),
         "rtp_sparse_decode": (I, [cfgp, P, I, P, P, P, P, P, P, P, S, P, P, P]),
         "rtp_sparse_decode_noalloc": (I, [cfgp, P, I, P, P, P, P, P, P, P, P, P]),
+        "rtp_cache_centroids": (I, [cfgp, P, I, P, P, P, P]),
+        "rtp_cache_append": (I, [cfgp, P, I, P, P, P, P, P, P, P]),
         "rtp_last_device_status": (I, [P]),
         "rtp_selftest_bounded_wait": (I, [ctypes.c_uint, P]),
         "rtp_status_str": (ctypes.c_char_p, [I]),
@@ -75,7 +77,7 @@ _lib = _load()
 EXPORTED = ("rtp_route_heads", "rtp_plan_destroy", "rtp_plan_num_sparse", "rtp_plan_num_items",
             "rtp_plan_sparse_heads", "rtp_plan_work_items", "rtp_indexer_project", "rtp_block_select",
             "rtp_hybrid_prefill", "rtp_decode_workspace_bytes", "rtp_sparse_decode", "rtp_sparse_decode_noalloc",
-            "rtp_last_device_status", "rtp_selftest_bounded_wait",
+            "rtp_cache_centroids", "rtp_cache_append", "rtp_last_device_status", "rtp_selftest_bounded_wait",
             "rtp_status_str", "rtp_version")
 
 
@@ -213,6 +215,23 @@ def rtp_sparse_decode_noalloc(cfg: AttnConfig, kinds, cache_len: int, q, kcache,
                                           _ptr(cnt_out), _stream(stream)))
 
 
+def rtp_cache_centroids(cfg: AttnConfig, kinds, cache_len: int, kcache, proj, centroids, stream=None) -> None:
+    """Centroids of every complete cache block of the retrieval heads (cfg.seq = cache capacity)."""
+    c = cfg.c()
+    _check("rtp_cache_centroids", _lib.rtp_cache_centroids(ctypes.byref(c), _kinds(kinds), int(cache_len),
+                                                           _ptr(kcache), _ptr(proj), _ptr(centroids),
+                                                           _stream(stream)))
+
+
+def rtp_cache_append(cfg: AttnConfig, kinds, pos: int, k_new, v_new, kcache, vcache, proj, centroids,
+                     stream=None) -> None:
+    """Writes cache row `pos`; completes the centroid of the block that row fills (cfg.seq = capacity)."""
+    c = cfg.c()
+    _check("rtp_cache_append", _lib.rtp_cache_append(ctypes.byref(c), _kinds(kinds), int(pos), _ptr(k_new),
+                                                     _ptr(v_new), _ptr(kcache), _ptr(vcache), _ptr(proj),
+                                                     _ptr(centroids), _stream(stream)))
+
+
 def rtp_last_device_status(stream=None) -> int:
     return int(_lib.rtp_last_device_status(_stream(stream)))
 
@@ -287,11 +306,19 @@ def hybrid_prefill_layer(q, k, v, kinds, proj=None, *, window: int, block: int =
 
 
 def sparse_decode_step(q, kcache, vcache, centroids, proj, kinds, *, window: int, block: int = 128, topk: int = 32,
-                       n_local: int = 4, scale: float = 0.0, stream=None, return_selection: bool = False):
-    """One decode step; returns o (and (sel, cnt) when asked)."""
+                       n_local: int = 4, scale: float = 0.0, stream=None, return_selection: bool = False,
+                       cache_len: int | None = None):
+    """One decode step; returns o (and (sel, cnt) when asked).
+
+    The caches are [batch][n_kv_heads][capacity][128]; the first `cache_len`
+    rows (default: all) are the cached tokens, the last of them the new one.
+    """
     B, Hq = q.shape[0], q.shape[1]
-    Hkv, Lc = kcache.shape[1], kcache.shape[2]
-    cfg = AttnConfig(B, 1, Hq, Hkv, window, block, topk, n_local, scale)
+    Hkv, cap = kcache.shape[1], kcache.shape[2]
+    Lc = cap if cache_len is None else int(cache_len)
+    if not 1 <= Lc <= cap:
+        raise RtpError("rtp_sparse_decode", RTP_ERR_INVALID_ARG)
+    cfg = AttnConfig(B, cap, Hq, Hkv, window, block, topk, n_local, scale)
     ws_bytes = rtp_decode_workspace_bytes(cfg, kinds, Lc)
     if ws_bytes == 0:
         raise RtpError("rtp_decode_workspace_bytes", RTP_ERR_INVALID_ARG)
@@ -303,3 +330,53 @@ def sparse_decode_step(q, kcache, vcache, centroids, proj, kinds, *, window: int
         cnt = torch.zeros(B, Hkv, dtype=torch.int32, device=q.device)
     rtp_sparse_decode(cfg, kinds, Lc, q, kcache, vcache, centroids, proj, o, ws, ws_bytes, sel, cnt, stream)
     return (o, sel, cnt) if return_selection else o
+
+
+class DecodeCache:
+    """A KV cache of fixed capacity with the block centroids decode scores.
+
+    Tensors are allocated once ([batch][n_kv_heads][capacity][128] bf16 K and
+    V, [batch][n_kv_heads][capacity // block][16] fp32 centroids); tokens are
+    added with `append` (rtp_cache_append) or in bulk with `load` (a prefill's
+    K/V, followed by rtp_cache_centroids), and `decode` runs rtp_sparse_decode
+    over the rows held so far.
+    """
+
+    def __init__(self, batch: int, n_kv_heads: int, capacity: int, kinds, proj, *, block: int = 128,
+                 device="cuda"):
+        self.kinds = [int(x) for x in kinds]
+        self.block = block
+        self.capacity = capacity
+        self.length = 0
+        self.proj = proj.to(device=device, dtype=torch.float32).contiguous()
+        self.k = torch.zeros(batch, n_kv_heads, capacity, 128, dtype=torch.bfloat16, device=device)
+        self.v = torch.zeros_like(self.k)
+        self.centroids = torch.zeros(batch, n_kv_heads, capacity // block, 16, dtype=torch.float32, device=device)
+
+    def _cfg(self, n_q_heads: int = 0, window: int = 1, topk: int = 0, n_local: int = 1, scale: float = 0.0):
+        B, H = self.k.shape[0], self.k.shape[1]
+        return AttnConfig(B, self.capacity, n_q_heads or H, H, window, self.block, topk, n_local, scale)
+
+    def load(self, k, v, stream=None) -> None:
+        """Replace the contents by k, v [batch][n_kv_heads][n][128] and build their centroids."""
+        n = k.shape[2]
+        if n > self.capacity:
+            raise RtpError("rtp_cache_centroids", RTP_ERR_INVALID_ARG)
+        self.k[:, :, :n].copy_(k)
+        self.v[:, :, :n].copy_(v)
+        self.length = n
+        if n > 0:
+            rtp_cache_centroids(self._cfg(), self.kinds, n, self.k, self.proj, self.centroids, stream)
+
+    def append(self, k_new, v_new, stream=None) -> None:
+        """Append one token per sequence (k_new, v_new [batch][n_kv_heads][128] or [..][1][128])."""
+        rtp_cache_append(self._cfg(), self.kinds, self.length, k_new.contiguous(), v_new.contiguous(), self.k, self.v,
+                         self.proj, self.centroids, stream)
+        self.length += 1
+
+    def decode(self, q, *, window: int, topk: int = 32, n_local: int = 4, scale: float = 0.0, stream=None,
+               return_selection: bool = False):
+        """One decode step for q [batch][n_q_heads][1][128] over the rows held."""
+        return sparse_decode_step(q, self.k, self.v, self.centroids, self.proj, self.kinds, window=window,
+                                  block=self.block, topk=topk, n_local=n_local, scale=scale, stream=stream,
+                                  return_selection=return_selection, cache_len=self.length)

@@ -100,3 +100,27 @@ def test_null_plan_is_rejected(rtp):
     for fn, nargs in [(rtp._lib.rtp_indexer_project, 7), (rtp._lib.rtp_block_select, 6),
                       (rtp._lib.rtp_hybrid_prefill, 8)]:
         assert fn(*([None] * nargs)) == rtp.RTP_ERR_INVALID_ARG
+
+
+def test_cache_calls_validate_before_launch(rtp):
+    """Bad arguments are refused without touching the GPU (no device needed)."""
+    cfg = rtp.AttnConfig(2, 1024, 8, 2, 256, 64, 4, 2)
+    fake = 1 << 20  # a 16-byte-aligned non-null address; never dereferenced on these paths
+    lib = rtp._lib
+    c = cfg.c()
+    kinds = rtp._kinds([2, 0])
+    inv = rtp.RTP_ERR_INVALID_ARG
+    # append: pos outside [0, capacity)
+    assert lib.rtp_cache_append(ctypes.byref(c), kinds, 1024, fake, fake, fake, fake, fake, fake, None) == inv
+    assert lib.rtp_cache_append(ctypes.byref(c), kinds, -1, fake, fake, fake, fake, fake, fake, None) == inv
+    # append: bad kind, null and unaligned pointers, missing centroids for a retrieval head
+    assert lib.rtp_cache_append(ctypes.byref(c), rtp._kinds([3, 0]), 5, fake, fake, fake, fake, fake, fake,
+                                None) == inv
+    assert lib.rtp_cache_append(ctypes.byref(c), kinds, 5, None, fake, fake, fake, fake, fake, None) == inv
+    assert lib.rtp_cache_append(ctypes.byref(c), kinds, 5, fake + 8, fake, fake, fake, fake, fake, None) == inv
+    assert lib.rtp_cache_append(ctypes.byref(c), kinds, 5, fake, fake, fake, fake, fake, None, None) == inv
+    # centroids: empty cache, bad block size
+    assert lib.rtp_cache_centroids(ctypes.byref(c), kinds, 0, fake, fake, fake, None) == inv
+    bad = rtp.AttnConfig(2, 1024, 8, 2, 256, 96, 4, 2).c()
+    assert lib.rtp_cache_centroids(ctypes.byref(bad), kinds, 512, fake, fake, fake, None) == inv
+    assert lib.rtp_cache_centroids(ctypes.byref(c), kinds, 512, None, fake, fake, None) == inv

@@ -12,7 +12,11 @@ The pages print no worked example, so the oracle is pinned by construction:
     plain matrix product;
   * selection: brute-force scoring + full sort with the (score desc, index asc)
     rule, a planted dominant block, degenerate sizes;
-  * decode: equals the last prefill row when both use the same selection.
+  * decode: equals the last prefill row when both use the same selection;
+  * KV-cache maintenance: filling a cache one append at a time gives the
+    centroids of a plain numpy mean-then-project of each complete block, only
+    the appended row and (on a block's last row) that block's centroid change,
+    and non-retrieval heads' centroids are never written.
 """
 
 import numpy as np
@@ -338,3 +342,68 @@ def test_selection_ties_at_the_cut_take_lower_indices():
     t = 39
     assert list(sel[t, : cnt[t]]) == [0, 1, 2, 3, 4, 5, 30, 38, 39]
     assert kth[t] == 16.0
+
+
+# ------------------------------------------------------------ KV-cache upkeep
+
+
+def _cache_case(batch, H, cap, seed):
+    d = inputs.small_prefill(cap, H, H, [oracle.SWA] * H, seed=seed)  # any bf16 keys/values of the right shape
+    k = d["k"].expand(batch, -1, -1, -1).clone() if batch > 1 else d["k"]
+    v = d["v"].expand(batch, -1, -1, -1).clone() if batch > 1 else d["v"]
+    return k, v
+
+
+@pytest.mark.parametrize("block", [64, 128])
+def test_appending_one_row_at_a_time_builds_block_means(block):
+    H, cap = 3, 5 * block + 17  # capacity not a multiple of the block
+    kinds = [oracle.SPARSE, oracle.SWA, oracle.SPARSE]
+    k_src, v_src = _cache_case(2, H, cap, seed=50 + block)
+    k_src[1] = torch.roll(k_src[1], 7, dims=1)  # the two sequences differ
+    p = inputs.random_projector(17)
+    kc = np.zeros((2, H, cap, 128), dtype=np.uint16)
+    vc = np.zeros((2, H, cap, 128), dtype=np.uint16)
+    sentinel = -12345.0
+    C = np.full((2, H, cap // block, 16), sentinel)
+    kb, vb = oracle._bf16_bits(k_src), oracle._bf16_bits(v_src)
+    for pos in range(cap):
+        kc2, vc2, C2 = oracle.cache_append(kc, vc, C, kinds, pos, kb[:, :, pos], vb[:, :, pos], block, p)
+        # only row pos changed in the caches
+        changed = np.any(kc2 != kc, axis=-1) | np.any(vc2 != vc, axis=-1)
+        assert not np.any(np.delete(changed, pos, axis=2))
+        assert np.array_equal(kc2[:, :, pos], kb[:, :, pos]) and np.array_equal(vc2[:, :, pos], vb[:, :, pos])
+        # a centroid changes only when its block completes, only for SPARSE heads
+        diff = np.any(C2 != C, axis=-1)
+        if (pos + 1) % block == 0:
+            blk = (pos + 1) // block - 1
+            expect = np.zeros_like(diff)
+            expect[:, [0, 2], blk] = True
+            assert np.array_equal(diff, expect)
+        else:
+            assert not diff.any()
+        kc, vc, C = kc2, vc2, C2
+    # after filling: complete blocks of SPARSE heads = numpy mean-then-project
+    nbc = cap // block
+    pn = p.double().numpy()
+    for b in range(2):
+        for h in range(H):
+            if kinds[h] == oracle.SPARSE:
+                ref = widen(k_src[b, h, : nbc * block]).reshape(nbc, block, 128).mean(axis=1) @ pn
+                assert np.max(np.abs(C[b, h] - ref)) <= 1e-12
+            else:
+                assert np.all(C[b, h] == sentinel)
+    # the bulk build agrees with the appended result, for every cache length
+    for L in (0, block - 1, block, 3 * block + 5, cap):
+        bulk = oracle.cache_centroids(k_src, L, kinds, block, p, C=np.full_like(C, sentinel))
+        full = L // block
+        assert np.array_equal(bulk[:, [0, 2], :full], C[:, [0, 2], :full])
+        assert np.all(bulk[:, [0, 2], full:] == sentinel) and np.all(bulk[:, 1] == sentinel)
+
+
+def test_cache_centroid_with_coordinate_projector_is_mean_of_coordinates():
+    block, cap = 64, 256
+    k_src, _ = _cache_case(1, 1, cap, seed=77)
+    got = oracle.cache_centroids(k_src, cap, [oracle.SPARSE], block, inputs.lowfreq_projector())
+    dims = list(range(56, 64)) + list(range(120, 128))
+    ref = widen(k_src[0, 0])[:, dims].reshape(-1, block, 16).mean(axis=1)
+    assert np.max(np.abs(got[0, 0] - ref)) <= 1e-15
