@@ -54,10 +54,12 @@ def _load():
         _lib.oracle_qbar.argtypes = [P, I, L, I, I, P, I, P]
         _lib.oracle_scores.argtypes = [P, P, L, I, P]
         _lib.oracle_select.argtypes = [P, P, L, I, P, L, I, I, I, P, P, P]
+        _lib.oracle_select_dynamic.argtypes = [P, P, L, I, P, L, I, I, I, D, I, D, P, P, P, P]
         _lib.oracle_attention_rows.argtypes = [P, P, L, P, P, L, I, I, L, I, P, P, I, D, P]
         _lib.oracle_attention_probs.argtypes = [P, L, P, L, I, I, L, I, P, P, I, D, P]
         _lib.oracle_decode_head.argtypes = [P, I, P, P, L, I, P, L, P, I, I, L, I, I, I, I, I, P, P, P, D, P]
         for f in ("oracle_project_rows", "oracle_centroids", "oracle_qbar", "oracle_scores", "oracle_select",
+                  "oracle_select_dynamic",
                   "oracle_attention_rows", "oracle_attention_probs", "oracle_decode_head"):
             getattr(_lib, f).restype = None
     return _lib
@@ -146,6 +148,32 @@ def select(qbar_rows: np.ndarray, C: np.ndarray, t_list, topk: int, n_local: int
     _load().oracle_select(_ptr(q), _ptr(c), c.shape[0], c.shape[1], _ptr(t), nq, topk, n_local, kmax, _ptr(sel),
                           _ptr(cnt), _ptr(kth))
     return sel, cnt, kth
+
+
+def select_dynamic(qbar_rows: np.ndarray, C: np.ndarray, t_list, cap: int, n_local: int, mass: float,
+                   min_k: int, beta: float):
+    """Dynamic block selection (RTPurboV2 page: the budget should vary by head,
+    length and query instead of a fixed top-k).
+
+    The shortest prefix of the candidates in (score desc, index asc) order
+    whose softmax weights exp(beta * (s - max s)) reach `mass` of their total,
+    clamped to [min_k, cap], plus the sink and local blocks.
+    Returns (sel [nq, cap+1+n_local] int32 padded with -1, cnt [nq],
+    cum_lo [nq], cum_hi [nq]): the selected mass fraction without / with the
+    last candidate taken.
+    """
+    q = np.ascontiguousarray(qbar_rows, dtype=np.float64)
+    c = np.ascontiguousarray(C, dtype=np.float64)
+    t = np.ascontiguousarray(t_list, dtype=np.int32)
+    nq = t.shape[0]
+    kmax = cap + 1 + n_local
+    sel = np.empty((nq, kmax), dtype=np.int32)
+    cnt = np.empty(nq, dtype=np.int32)
+    lo = np.empty(nq, dtype=np.float64)
+    hi = np.empty(nq, dtype=np.float64)
+    _load().oracle_select_dynamic(_ptr(q), _ptr(c), c.shape[0], c.shape[1], _ptr(t), nq, cap, n_local, kmax,
+                                  float(mass), int(min_k), float(beta), _ptr(sel), _ptr(cnt), _ptr(lo), _ptr(hi))
+    return sel, cnt, lo, hi
 
 
 def attention_rows(q_rows, pos, k_head, v_head, mode: int, window: int = 0, block: int = 64, sel=None, cnt=None,

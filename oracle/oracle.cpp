@@ -182,6 +182,69 @@ void oracle_select(const double* qbar, const double* C, long nb, int r, const in
   });
 }
 
+// [P2] dynamic budget instead of a fixed top-k (the page only says that
+// different heads, lengths and queries need very different numbers of
+// context tokens; the rule below is this library's reading).  For query
+// summary q (block t = t_list[q]):
+//   candidates j in [1, t-L] with scores s_j = qbar . c_j;
+//   weights    w_j = exp(beta * (s_j - max_j s_j));  Z = sum_j w_j;
+//   order      the candidates by (score desc, index asc);
+//   n*         the smallest n whose first n weights sum to >= mass * Z
+//              (all candidates if no prefix reaches it), then clamped to
+//              [min(min_k, #cand), min(cap, #cand)];
+//   selection  the first n* candidates, block 0 and the local blocks
+//              max(0,t-L+1)..t, de-duplicated and sorted ascending.
+// cum_lo[q] / cum_hi[q] receive the prefix sums / Z at n*-1 and n* (NaN
+// where undefined), so a caller can see how close the cut was.
+void oracle_select_dynamic(const double* qbar, const double* C, long nb, int r, const int32_t* t_list, long nq,
+                           int cap, int n_local, int kmax, double mass, int min_k, double beta, int32_t* sel,
+                           int32_t* cnt, double* cum_lo, double* cum_hi) {
+  parallel_for(nq, [&](long q) {
+    long t = t_list[q];
+    std::vector<double> s(nb);
+    oracle_scores(qbar + q * r, C, nb, r, s.data());
+    std::vector<long> cand;
+    for (long j = 1; j <= t - n_local; ++j) cand.push_back(j);
+    const long m = static_cast<long>(cand.size());
+    long nstar = 0;
+    cum_lo[q] = std::nan("");
+    cum_hi[q] = std::nan("");
+    if (m > 0) {
+      double smax = -INFINITY;
+      for (long j : cand) smax = std::max(smax, s[j]);
+      double Z = 0.0;
+      for (long j : cand) Z += std::exp(beta * (s[j] - smax));
+      std::sort(cand.begin(), cand.end(), [&](long a, long b) {
+        if (s[a] != s[b]) return s[a] > s[b];
+        return a < b;
+      });
+      std::vector<double> prefix(m);
+      double acc = 0.0;
+      for (long e = 0; e < m; ++e) {
+        acc += std::exp(beta * (s[cand[e]] - smax));
+        prefix[e] = acc;
+      }
+      nstar = m;
+      for (long e = 0; e < m; ++e)
+        if (prefix[e] >= mass * Z) {
+          nstar = e + 1;
+          break;
+        }
+      nstar = std::max(nstar, std::min<long>(min_k, m));
+      nstar = std::min(nstar, std::min<long>(cap, m));
+      cum_lo[q] = nstar >= 2 ? prefix[nstar - 2] / Z : (nstar == 1 ? 0.0 : std::nan(""));
+      cum_hi[q] = nstar >= 1 ? prefix[nstar - 1] / Z : std::nan("");
+    }
+    std::vector<long> all(cand.begin(), cand.begin() + nstar);
+    all.push_back(0);
+    for (long j = std::max<long>(0, t - n_local + 1); j <= t; ++j) all.push_back(j);
+    std::sort(all.begin(), all.end());
+    all.erase(std::unique(all.begin(), all.end()), all.end());
+    for (int i = 0; i < kmax; ++i) sel[q * kmax + i] = i < static_cast<int>(all.size()) ? static_cast<int32_t>(all[i]) : -1;
+    cnt[q] = static_cast<int32_t>(all.size());
+  });
+}
+
 // Visible keys of query position i for one head ([P1] SWA drops far tokens,
 // full heads see every earlier token, [P4] sparse heads see the selected set):
 //   mode 0 (SWA):    i-W < j <= i

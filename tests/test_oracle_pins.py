@@ -407,3 +407,92 @@ def test_cache_centroid_with_coordinate_projector_is_mean_of_coordinates():
     dims = list(range(56, 64)) + list(range(120, 128))
     ref = widen(k_src[0, 0])[:, dims].reshape(-1, block, 16).mean(axis=1)
     assert np.max(np.abs(got[0, 0] - ref)) <= 1e-15
+
+
+# ------------------------------------------------------- dynamic selection
+
+
+def pairwise_dynamic(qb, C, t, cap, n_local, mass, min_k, beta):
+    """Dynamic selection without sorting: candidate j is kept iff the weight of
+    the candidates ahead of it in (score desc, index asc) order is still below
+    mass * Z; then the count is clamped by dropping/adding in that order."""
+    s = C @ qb
+    cands = list(range(1, t - n_local + 1))
+    if not cands:
+        return sorted(set([0] + list(range(max(0, t - n_local + 1), t + 1))))
+    smax = max(s[j] for j in cands)
+    w = {j: np.exp(beta * (s[j] - smax)) for j in cands}
+    Z = sum(w.values())
+
+    def ahead(i, j):
+        return s[i] > s[j] or (s[i] == s[j] and i < j)
+
+    rank = {j: sum(1 for i in cands if ahead(i, j)) for j in cands}
+    kept = [j for j in cands if sum(w[i] for i in cands if ahead(i, j)) < mass * Z]
+    n = len(kept)
+    n = max(n, min(min_k, len(cands)))
+    n = min(n, cap, len(cands))
+    chosen = [j for j in cands if rank[j] < n]
+    return sorted(set(chosen) | {0} | set(range(max(0, t - n_local + 1), t + 1)))
+
+
+def _dyn_case(nb, seed):
+    rng = np.random.default_rng(seed)
+    return rng.normal(size=(nb, 16)), rng.normal(size=(nb, 16))
+
+
+@pytest.mark.parametrize("mass,beta,cap,min_k", [(0.5, 0.3, 40, 0), (0.9, 0.3, 40, 0), (0.9, 1.0, 8, 0),
+                                                 (0.99, 0.05, 60, 3), (0.2, 2.0, 40, 5), (1.0, 0.3, 12, 0)])
+def test_dynamic_selection_matches_pairwise_definition(mass, beta, cap, min_k):
+    nb, n_local = 64, 2
+    Q, C = _dyn_case(nb, 3)
+    ts = np.arange(nb, dtype=np.int32)
+    sel, cnt, lo, hi = oracle.select_dynamic(Q, C, ts, cap, n_local, mass, min_k, beta)
+    for t in range(nb):
+        ref = pairwise_dynamic(Q[t], C, t, cap, n_local, mass, min_k, beta)
+        assert list(sel[t, :cnt[t]]) == ref, (t, list(sel[t, :cnt[t]]), ref)
+        assert np.all(sel[t, cnt[t]:] == -1)
+
+
+def test_dynamic_selection_with_equal_weights_takes_ceil_of_mass():
+    """beta = 0: every candidate weighs the same, so n* = ceil(mass * m) and the
+    set is the fixed top-n* of the scores."""
+    nb, n_local = 48, 3
+    Q, C = _dyn_case(nb, 5)
+    for mass in (0.1, 0.25, 0.5, 0.77, 1.0):
+        for t in (10, 30, 47):
+            m = t - n_local
+            n = int(np.ceil(mass * m - 1e-12))
+            sel, cnt, _, _ = oracle.select_dynamic(Q[t:t + 1], C, [t], 1000, n_local, mass, 0, 0.0)
+            fsel, fcnt, _ = oracle.select(Q[t:t + 1], C, [t], n, n_local)
+            assert cnt[0] == 1 + n + n_local
+            assert list(sel[0, :cnt[0]]) == list(fsel[0, :fcnt[0]])
+
+
+def test_dynamic_selection_with_full_mass_equals_fixed_topk():
+    nb, n_local, cap = 80, 4, 10
+    Q, C = _dyn_case(nb, 8)
+    ts = np.arange(nb, dtype=np.int32)
+    sel, cnt, _, _ = oracle.select_dynamic(Q, C, ts, cap, n_local, 1.0, 0, 0.5)
+    fsel, fcnt, _ = oracle.select(Q, C, ts, cap, n_local)
+    for t in range(nb):
+        if t - n_local > cap:  # more candidates than the cap: the fixed rule keeps exactly the cap
+            assert list(sel[t, :cnt[t]]) == list(fsel[t, :fcnt[t]])
+
+
+def test_dynamic_selection_stops_at_planted_mass():
+    """Two dominant blocks hold almost all the mass: mass 0.9 keeps just them."""
+    nb, n_local = 40, 2
+    rng = np.random.default_rng(1)
+    C = rng.normal(scale=0.01, size=(nb, 16))
+    q = np.zeros(16)
+    q[0] = 1.0
+    C[7, 0] = C[23, 0] = 10.0
+    sel, cnt, lo, hi = oracle.select_dynamic(q[None], C, [39], 16, n_local, 0.9, 0, 1.0)
+    assert list(sel[0, :cnt[0]]) == [0, 7, 23, 38, 39]
+    assert hi[0] >= 0.9 > lo[0]
+    # min_k raises the count past the planted pair, cap lowers it
+    sel, cnt, _, _ = oracle.select_dynamic(q[None], C, [39], 16, n_local, 0.9, 4, 1.0)
+    assert cnt[0] == 1 + 4 + n_local
+    sel, cnt, _, _ = oracle.select_dynamic(q[None], C, [39], 1, n_local, 0.9, 0, 1.0)
+    assert list(sel[0, :cnt[0]]) == [0, 7, 38, 39]
