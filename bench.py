@@ -279,6 +279,70 @@ def time_primary(rtp, w, layer, steps, warmup, device, world):
     return res
 
 
+def needle_recall(needles, slot_of, sel, cnt, block) -> float | None:
+    """Fraction of planted needles whose key block is selected for the
+    query block of their target query (a diagnostic, not a pinned value)."""
+    if not needles:
+        return None
+    sel_c, cnt_c = sel.cpu(), cnt.cpu()
+    hit = 0
+    for kvh, _, tq, j in needles:
+        t = tq // block
+        row = sel_c[0, slot_of[kvh], t, :int(cnt_c[0, slot_of[kvh], t])]
+        hit += int((row == j // block).any())
+    return hit / len(needles)
+
+
+def time_dynamic(rtp, w, res, device, points=((0.9, None), (0.99, None), (0.9, 1.0)), reps=2):
+    """The layer of the main step with the dynamic (mass-threshold) selection
+    in place of the fixed top-k (cap = the workload's top-k, default beta):
+    selection and prefill times, blocks kept, and the executed FLOPs of the
+    prefill on that selection."""
+    plan, bufs = res["plan"], res["bufs"]
+    if not plan.n_sparse:
+        return None
+    q, k, v, o = res["q"], res["k"], res["v"], res["o"]
+    stream = torch.cuda.current_stream()
+    beta0 = rtp.default_selection_beta(plan.cfg)
+    slot_of = {h: s for s, h in enumerate(plan.slot_heads)}
+    B, G = w.block, w.group
+    nb = w.seq // B
+    out = {"cap": w.topk, "default_beta": beta0, "min_k": 0,
+           "fixed_needle_recall": needle_recall(res["needles"], slot_of, bufs["sel"], bufs["sel_cnt"], B)}
+    for mass, beta in points:
+        beta = beta0 if beta is None else beta
+        sel, cnt = torch.empty_like(bufs["sel"]), torch.empty_like(bufs["sel_cnt"])
+        for _ in range(2):
+            rtp.rtp_block_select_dynamic(plan.handle, bufs["qbar"], bufs["centroids"], mass, 0, beta, sel, cnt,
+                                         stream)
+            rtp.rtp_hybrid_prefill(plan.handle, q, k, v, sel, cnt, o, stream)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+        torch.cuda.synchronize()
+        for e in ev:
+            e[0].record(stream)
+            rtp.rtp_block_select_dynamic(plan.handle, bufs["qbar"], bufs["centroids"], mass, 0, beta, sel, cnt,
+                                         stream)
+            e[1].record(stream)
+            rtp.rtp_hybrid_prefill(plan.handle, q, k, v, sel, cnt, o, stream)
+            e[2].record(stream)
+        torch.cuda.synchronize()
+        sel_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+        pre_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+        c = cnt.cpu().long()  # [batch][n_sparse][nb]
+        # executed tiles of the sparse heads: one 128-key tile per selected block (block 128)
+        sparse_pairs = float(((c - 1) * B * B + B * (B + 1) // 2).sum()) * G
+        other_pairs = sum(algorithmic_pairs(kd, w.seq, w.window, B, w.topk, w.n_local)
+                          for kd in res["kinds"] if kd != inputs.SPARSE) * G
+        flops = (sparse_pairs + other_pairs) * 4 * 128
+        out[f"mass_{mass}_beta_{beta:.4g}"] = {
+            "select_ms": sel_ms, "prefill_ms": pre_ms,
+            "mean_blocks_per_query_block": float(c.float().mean()),
+            "fixed_blocks_per_query_block": float(np.mean([selected_count(t, w.topk, w.n_local) for t in range(nb)])),
+            "algorithmic_tflops": flops / (pre_ms * 1e-3) / 1e12,
+            "needle_recall": needle_recall(res["needles"], slot_of, sel, cnt, B)}
+    return out
+
+
 def time_e2e(rtp, w, res, steps, device):
     """Same step through the C ABI from pinned host buffers, copies included."""
     q, k, v = res["q"], res["k"], res["v"]
@@ -572,6 +636,8 @@ def run_ours(args, rank, world, local):
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     traffic = prefill_traffic(w)
     extra = {}
+    if not args.no_secondary and world == 1:
+        extra["dynamic"] = time_dynamic(rtp, w, res, device)
     if not args.no_e2e:
         extra["e2e"] = time_e2e(rtp, w, res, max(2, min(args.steps, 3)), device)
     for key in ("q", "k", "v", "o"):
@@ -589,6 +655,8 @@ def run_ours(args, rank, world, local):
     if not args.no_secondary and world == 1:
         secondary["v2_128k_48_layers"] = time_secondary_128k(rtp, 2, device)
         secondary["decode_8x256k"] = time_decode(rtp, args.decode_steps, device)
+        if extra.get("dynamic"):
+            secondary["dynamic_selection"] = extra["dynamic"]
     if rank != 0:
         return
     clocks = res["clocks"]

@@ -161,6 +161,35 @@ rtp_status rtp_block_select(const rtp_plan* plan, const float* qbar, const float
                             int32_t* sel_cnt, void* stream);
 
 /* ------------------------------------------------------------------------
+ * rtp_block_select_dynamic — selection with a per-query-block budget instead
+ * of a fixed top-k (RTPurboV2 page: the fixed top-k policy is criticised
+ * because heads, sequence lengths and queries need very different numbers of
+ * context tokens; the page gives no rule, so this is the library's):
+ *   candidates j = 1..t-n_local of query block t, scores s_j = qbar_t . c_j
+ *   (fp32, fixed order as in rtp_block_select), weights
+ *   w_j = exp(beta * (s_j - max s)), Z = sum w_j; keep the shortest prefix of
+ *   the candidates in (score desc, index asc) order whose weights sum to
+ *   >= mass * Z (all of them if no prefix does), clamped to
+ *   [min(min_k, #candidates), min(topk, #candidates)]; add block 0 and the
+ *   local blocks max(0,t-n_local+1)..t.
+ *   plan      its topk is the cap (<= 1024, else RTP_ERR_UNSUPPORTED)
+ *   mass      fraction of the candidates' weight to cover, 0 < mass <= 1
+ *   min_k     smallest number of candidates kept, 0 <= min_k <= topk
+ *   beta      inverse temperature on the low-rank scores, >= 0 (0: every
+ *             candidate weighs the same, so ceil(mass * #candidates) are
+ *             kept); the softmax scale divided by the group size weighs a
+ *             block like the mean over the group's heads of its logits
+ *   qbar, centroids, sel, sel_cnt  as in rtp_block_select (same layout,
+ *             kmax = topk + 1 + n_local; rows end with -1 padding), so the
+ *             result feeds rtp_hybrid_prefill unchanged
+ * Every sum runs in a fixed order: results are bit-reproducible.
+ * Errors: RTP_ERR_INVALID_ARG (bad plan, mass, min_k, beta or pointer;
+ * nothing launched), RTP_ERR_UNSUPPORTED (topk > 1024), RTP_ERR_CUDA.
+ * ---------------------------------------------------------------------- */
+rtp_status rtp_block_select_dynamic(const rtp_plan* plan, const float* qbar, const float* centroids, float mass,
+                                    int min_k, float beta, int32_t* sel, int32_t* sel_cnt, void* stream);
+
+/* ------------------------------------------------------------------------
  * rtp_hybrid_prefill — causal prefill attention over the routing map.
  * RTPurbo page (streaming heads: SWA; full heads: dense causal) and
  * RTPurboV2 page / "Full Attention Strikes Back" summary (sparse heads:

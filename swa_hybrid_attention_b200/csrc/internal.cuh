@@ -42,7 +42,12 @@ struct SelectArgs {
   int32_t* sel;
   int32_t* cnt;
   int batch, n_sparse, nb, topk, n_local, kmax;
+  // dynamic selection only: mass fraction, minimum count, beta * log2(e)
+  float mass;
+  int min_k;
+  float beta_log2;
 };
+constexpr int kDynMaxCap = 1024;  // largest top-k cap of the dynamic selection
 
 constexpr int kMaxDecodeKvHeads = 256;
 
@@ -94,6 +99,7 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& mq, const CU
                            int num_ctas, cudaStream_t stream);
 cudaError_t launch_indexer(const IndexerArgs& a, cudaStream_t stream);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
+cudaError_t launch_select_dynamic(const SelectArgs& a, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t stream);
 cudaError_t launch_cache_append(const CacheArgs& a, cudaStream_t stream);
 cudaError_t launch_cache_centroids(const CacheArgs& a, cudaStream_t stream);

@@ -335,6 +335,34 @@ rtp_status rtp_block_select(const rtp_plan* plan, const float* qbar, const float
   return cuda_status(launch_select(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+rtp_status rtp_block_select_dynamic(const rtp_plan* plan, const float* qbar, const float* centroids, float mass,
+                                    int min_k, float beta, int32_t* sel, int32_t* sel_cnt, void* stream) {
+  if (!plan) return RTP_ERR_INVALID_ARG;
+  const rtp_attn_cfg& c = plan->cfg;
+  if (!(mass > 0.f && mass <= 1.f) || !(beta >= 0.f) || !std::isfinite(beta)) return RTP_ERR_INVALID_ARG;
+  if (min_k < 0 || min_k > c.topk) return RTP_ERR_INVALID_ARG;
+  if (c.topk > kDynMaxCap) return RTP_ERR_UNSUPPORTED;
+  if (plan->n_sparse == 0) return RTP_OK;
+  if (!qbar || !centroids || !sel || !sel_cnt) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(qbar) || !aligned16(centroids) || !aligned16(sel) || !aligned16(sel_cnt))
+    return RTP_ERR_INVALID_ARG;
+  SelectArgs a;
+  a.qbar = qbar;
+  a.centroids = centroids;
+  a.sel = sel;
+  a.cnt = sel_cnt;
+  a.batch = c.batch;
+  a.n_sparse = plan->n_sparse;
+  a.nb = plan->nqb;
+  a.topk = c.topk;
+  a.n_local = c.n_local;
+  a.kmax = c.topk + 1 + c.n_local;
+  a.mass = mass;
+  a.min_k = min_k;
+  a.beta_log2 = beta * kLog2e;
+  return cuda_status(launch_select_dynamic(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 rtp_status rtp_hybrid_prefill(const rtp_plan* plan, const void* q, const void* k, const void* v,
                               const int32_t* sel, const int32_t* sel_cnt, void* o, void* stream) {
   if (!plan || !q || !k || !v || !o) return RTP_ERR_INVALID_ARG;

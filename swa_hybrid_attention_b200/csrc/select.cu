@@ -39,7 +39,227 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(const SelectA
   if (threadIdx.x == 0) a.cnt[row] = n;
 }
 
+// ------------------------------------------------------------ dynamic budget
+//
+// The same page argues that heads, lengths and queries need very different
+// numbers of context blocks.  Rule implemented here (the library's reading):
+// weights w_j = exp(beta (s_j - max s)) over the candidates, Z = sum w_j; the
+// shortest prefix of the candidates in (score desc, index asc) order whose
+// weights reach mass * Z, clamped to [min_k, cap]; plus sink and local blocks.
+//
+// Per CTA (one query block): scores -> keys (as above); max key and Z by
+// fixed-order reductions; the cap best candidates (radix select, or all of
+// them) are bitonic-sorted in shared memory by (key desc, index asc); a
+// fixed-order scan of their weights gives the cut n*; the cut is turned back
+// into a (threshold key, ties) pair and the ordered compaction of the fixed
+// kernel writes the kept blocks ascending.  Every reduction has a fixed
+// order, so results are bit-reproducible.
+
+__device__ __forceinline__ float key_score(uint32_t key) {  // inverse of order_key
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
+struct DynScratch {
+  unsigned long long srt[kDynMaxCap];  // (key << 32) | ~index, sorted descending
+  float red[kSelThreads / 32];
+  float warp_excl[kSelThreads / 32];
+  uint32_t kred[kSelThreads / 32];
+  int cut, first_eq;
+};
+
+// Sum over the CTA in a fixed order (butterfly inside each warp, lane 0's
+// value per warp, then the warps in index order).  Called by all threads.
+__device__ __forceinline__ float cta_sum_fixed(float v, DynScratch& d) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  if (lane == 0) d.red[warp] = v;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int w = 0; w < kSelThreads / 32; ++w) tot += d.red[w];
+  __syncthreads();
+  return tot;
+}
+
+__device__ __forceinline__ uint32_t cta_max_u32(uint32_t v, DynScratch& d) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, off));
+  if (lane == 0) d.kred[warp] = v;
+  __syncthreads();
+  uint32_t m = 0;
+#pragma unroll
+  for (int w = 0; w < kSelThreads / 32; ++w) m = max(m, d.kred[w]);
+  __syncthreads();
+  return m;
+}
+
+// Exclusive prefix sum of one float per thread, in thread order, fixed
+// association (shuffle scan inside warps, then over the warp totals).
+__device__ __forceinline__ float cta_exclusive_scan_fixed(float v, DynScratch& d) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  float incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const float y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) d.red[warp] = incl;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float acc = 0.f;
+    for (int w = 0; w < kSelThreads / 32; ++w) {
+      d.warp_excl[w] = acc;
+      acc += d.red[w];
+    }
+  }
+  __syncthreads();
+  const float r = d.warp_excl[warp] + (incl - v);
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kSelThreads) block_select_dynamic_kernel(const SelectArgs a) {
+  extern __shared__ uint32_t keys[];
+  __shared__ SelectScratch sh;
+  __shared__ DynScratch d;
+  const int tid = threadIdx.x;
+  const int t = blockIdx.x, slot = blockIdx.y, b = blockIdx.z;
+  const size_t row = (static_cast<size_t>(b) * a.n_sparse + slot) * a.nb + t;
+  int32_t* out = a.sel + row * a.kmax;
+  const float* C = a.centroids + (static_cast<size_t>(b) * a.n_sparse + slot) * a.nb * kRank;
+  const int ncand = t - a.n_local > 0 ? t - a.n_local : 0;  // candidates are blocks 1..ncand
+  if (ncand == 0) {  // only sink and local blocks exist: blocks 0..t
+    for (int e = tid; e < a.kmax; e += kSelThreads) out[e] = e <= t ? e : -1;
+    if (tid == 0) a.cnt[row] = t + 1;
+    return;
+  }
+  float q[kRank];
+#pragma unroll
+  for (int c = 0; c < kRank; ++c) q[c] = a.qbar[row * kRank + c];
+  // 1. scores -> order keys
+  for (int x0 = tid; x0 < ncand; x0 += 4 * kSelThreads) {
+    float4 v[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int x = min(x0 + u * kSelThreads, ncand - 1);
+      const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + 1) * kRank);
+#pragma unroll
+      for (int w = 0; w < 4; ++w) v[u][w] = __ldg(c4 + w);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int x = x0 + u * kSelThreads;
+      if (x < ncand) keys[x] = order_key(score16(q, v[u]));
+    }
+  }
+  __syncthreads();
+  // 2. max score and Z = sum of the weights (each thread a contiguous run)
+  const int per = (ncand + kSelThreads - 1) / kSelThreads;
+  const int x0 = min(ncand, tid * per), x1 = min(ncand, x0 + per);
+  uint32_t kmax_l = 0;
+  for (int x = x0; x < x1; ++x) kmax_l = max(kmax_l, keys[x]);
+  const float smax = key_score(cta_max_u32(kmax_l, d));
+  float zl = 0.f;
+  for (int x = x0; x < x1; ++x) zl += exp2f(a.beta_log2 * (key_score(keys[x]) - smax));
+  const float Z = cta_sum_fixed(zl, d);
+  // 3. the cap best candidates, sorted by (key desc, index asc)
+  const int m = min(ncand, a.topk);
+  int nstar = 0;
+  if (m > 0) {
+    int P = 1;
+    while (P < m) P <<= 1;
+    if (ncand > m) {
+      uint32_t T, need;
+      radix_threshold<kSelThreads>(keys, ncand, m, sh, T, need);
+      ordered_select<kSelThreads>(keys, ncand, T, need, sh, [&](int r, int x) {
+        d.srt[r] = (static_cast<unsigned long long>(keys[x]) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(x));
+      });
+    } else {
+      for (int x = tid; x < m; x += kSelThreads)
+        d.srt[x] = (static_cast<unsigned long long>(keys[x]) << 32) | (0xFFFFFFFFu - static_cast<uint32_t>(x));
+    }
+    for (int e = m + tid; e < P; e += kSelThreads) d.srt[e] = 0ull;  // sorts last
+    if (tid == 0) {
+      d.cut = 0x7FFFFFFF;
+      d.first_eq = 0x7FFFFFFF;
+    }
+    __syncthreads();
+    for (int k = 2; k <= P; k <<= 1) {
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int i = tid; i < P; i += kSelThreads) {
+          const int ixj = i ^ j;
+          if (ixj > i) {
+            const unsigned long long u = d.srt[i], w = d.srt[ixj];
+            if (((i & k) == 0) ? (u < w) : (u > w)) {
+              d.srt[i] = w;
+              d.srt[ixj] = u;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    // 4. prefix sums of the sorted weights; the first prefix >= mass * Z
+    const int rper = (m + kSelThreads - 1) / kSelThreads;  // <= 4
+    const int r0 = min(m, tid * rper), r1 = min(m, r0 + rper);
+    float wl[4];
+    float tot = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      wl[e] = 0.f;
+      if (r0 + e < r1) {
+        wl[e] = exp2f(a.beta_log2 * (key_score(static_cast<uint32_t>(d.srt[r0 + e] >> 32)) - smax));
+        tot += wl[e];
+      }
+    }
+    float acc = cta_exclusive_scan_fixed(tot, d);
+    const float thr = a.mass * Z;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (r0 + e < r1) {
+        acc += wl[e];
+        if (acc >= thr) {
+          atomicMin(&d.cut, r0 + e + 1);
+          break;
+        }
+      }
+    }
+    __syncthreads();
+    nstar = d.cut == 0x7FFFFFFF ? m : d.cut;
+    nstar = max(nstar, min(a.min_k, m));
+    nstar = min(nstar, m);
+    // 5. the cut as (threshold key, ties at it), then the ordered compaction
+    const uint32_t Tc = static_cast<uint32_t>(d.srt[nstar - 1] >> 32);
+    for (int r = tid; r < nstar; r += kSelThreads)
+      if (static_cast<uint32_t>(d.srt[r] >> 32) == Tc) atomicMin(&d.first_eq, r);
+    __syncthreads();
+    const uint32_t need_c = static_cast<uint32_t>(nstar - d.first_eq);
+    ordered_select<kSelThreads>(keys, ncand, Tc, need_c, sh, [&](int r, int x) { out[1 + r] = x + 1; });
+  }
+  if (tid == 0) {
+    out[0] = 0;
+    a.cnt[row] = 1 + nstar + a.n_local;
+  }
+  for (int e = tid; e < a.n_local; e += kSelThreads) out[1 + nstar + e] = t - a.n_local + 1 + e;
+  for (int e = 1 + nstar + a.n_local + tid; e < a.kmax; e += kSelThreads) out[e] = -1;
+}
+
 }  // namespace
+
+cudaError_t launch_select_dynamic(const SelectArgs& a, cudaStream_t stream) {
+  if (a.n_sparse == 0) return cudaSuccess;
+  const size_t smem = static_cast<size_t>(a.nb) * sizeof(uint32_t);
+  if (smem + sizeof(DynScratch) + sizeof(SelectScratch) > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(block_select_dynamic_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  dim3 grid(a.nb, a.n_sparse, a.batch);
+  block_select_dynamic_kernel<<<grid, kSelThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
   if (a.n_sparse == 0) return cudaSuccess;

@@ -14,6 +14,7 @@ layer / one decode step and allocate their intermediate buffers with torch
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 from dataclasses import dataclass
 
@@ -55,6 +56,7 @@ def _load() -> ctypes.CDLL:
         "rtp_plan_work_items": (I, [P, P]),
         "rtp_indexer_project": (I, [P, P, P, P, P, P, P]),
         "rtp_block_select": (I, [P, P, P, P, P, P]),
+        "rtp_block_select_dynamic": (I, [P, P, P, ctypes.c_float, I, ctypes.c_float, P, P, P]),
         "rtp_hybrid_prefill": (I, [P, P, P, P, P, P, P, P]),
         "rtp_decode_workspace_bytes": (S, [cfgp, P, I]),
         "rtp_sparse_decode": (I, [cfgp, P, I, P, P, P, P, P, P, P, S, P, P, P]),
@@ -76,6 +78,7 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 EXPORTED = ("rtp_route_heads", "rtp_plan_destroy", "rtp_plan_num_sparse", "rtp_plan_num_items",
             "rtp_plan_sparse_heads", "rtp_plan_work_items", "rtp_indexer_project", "rtp_block_select",
+            "rtp_block_select_dynamic",
             "rtp_hybrid_prefill", "rtp_decode_workspace_bytes", "rtp_sparse_decode", "rtp_sparse_decode_noalloc",
             "rtp_cache_centroids", "rtp_cache_append", "rtp_last_device_status", "rtp_selftest_bounded_wait",
             "rtp_status_str", "rtp_version")
@@ -186,6 +189,19 @@ def rtp_block_select(plan: int, qbar, centroids, sel, sel_cnt, stream=None) -> N
                                                      _stream(stream)))
 
 
+def rtp_block_select_dynamic(plan: int, qbar, centroids, mass: float, min_k: int, beta: float, sel, sel_cnt,
+                             stream=None) -> None:
+    _check("rtp_block_select_dynamic",
+           _lib.rtp_block_select_dynamic(plan, _ptr(qbar), _ptr(centroids), float(mass), int(min_k), float(beta),
+                                         _ptr(sel), _ptr(sel_cnt), _stream(stream)))
+
+
+def default_selection_beta(cfg: AttnConfig) -> float:
+    """Softmax scale / group: weighs a block like the group-mean of its attention logits."""
+    scale = cfg.scale if cfg.scale > 0 else 1.0 / math.sqrt(cfg.head_dim)
+    return scale / (cfg.n_q_heads // cfg.n_kv_heads)
+
+
 def rtp_hybrid_prefill(plan: int, q, k, v, sel, sel_cnt, o, stream=None) -> None:
     _check("rtp_hybrid_prefill", _lib.rtp_hybrid_prefill(plan, _ptr(q), _ptr(k), _ptr(v), _ptr(sel), _ptr(sel_cnt),
                                                          _ptr(o), _stream(stream)))
@@ -281,11 +297,23 @@ class Plan:
             sel_cnt=torch.empty(c.batch, ns, nb, dtype=torch.int32, device=device),
         )
 
-    def run(self, q, k, v, proj, o, bufs: dict, stream=None) -> None:
-        """One layer: indexer + selection (if any retrieval slot) + prefill."""
+    def run(self, q, k, v, proj, o, bufs: dict, stream=None, dynamic: dict | None = None) -> None:
+        """One layer: indexer + selection (if any retrieval slot) + prefill.
+
+        dynamic: None for the fixed top-k selection, else a dict with `mass`
+        and optionally `min_k` (default 0) and `beta` (default: softmax scale
+        / group) for rtp_block_select_dynamic (topk is then the cap).
+        """
         if self.n_sparse > 0:
             rtp_indexer_project(self.handle, q, k, proj, bufs["centroids"], bufs["qbar"], stream)
-            rtp_block_select(self.handle, bufs["qbar"], bufs["centroids"], bufs["sel"], bufs["sel_cnt"], stream)
+            if dynamic is None:
+                rtp_block_select(self.handle, bufs["qbar"], bufs["centroids"], bufs["sel"], bufs["sel_cnt"], stream)
+            else:
+                beta = dynamic.get("beta")
+                rtp_block_select_dynamic(self.handle, bufs["qbar"], bufs["centroids"], dynamic["mass"],
+                                         dynamic.get("min_k", 0),
+                                         default_selection_beta(self.cfg) if beta is None else beta, bufs["sel"],
+                                         bufs["sel_cnt"], stream)
             rtp_hybrid_prefill(self.handle, q, k, v, bufs["sel"], bufs["sel_cnt"], o, stream)
         else:
             rtp_hybrid_prefill(self.handle, q, k, v, None, None, o, stream)

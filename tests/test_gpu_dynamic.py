@@ -1,0 +1,133 @@
+"""GPU parity of the dynamic (mass-threshold) block selection against the CPU
+oracle, and prefill attention on its selection (C ABI)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from helpers import TIE_REL, check_indexer, check_prefill_rows, cpu
+from swa_hybrid_attention_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+# The cut n* is an integer decided by fp32 sums on the GPU and fp64 sums in
+# the oracle: a different count is accepted when the oracle's covered mass
+# fraction at the GPU's cut is within MASS_TOL of the target (the fp32 error
+# of up to 8K summed weights, each within ~1e-6 relative, is far smaller).
+MASS_TOL = 1e-4
+
+
+@pytest.fixture(scope="module")
+def rtp(cuda_device):
+    from swa_hybrid_attention_b200 import build
+
+    build.build()
+    from swa_hybrid_attention_b200 import rtp as mod
+
+    return mod
+
+
+def oracle_fractions(qb, C, t, n_local, beta):
+    """Candidates in (score desc, index asc) order and their covered mass fractions (fp64)."""
+    s = C @ qb
+    cands = np.arange(1, t - n_local + 1)
+    if cands.size == 0:
+        return cands, np.zeros(0), s
+    order = cands[np.lexsort((cands, -s[cands]))]
+    w = np.exp(beta * (s[order] - s[cands].max()))
+    return order, np.cumsum(w) / w.sum(), s
+
+
+def check_dynamic_rows(sel, cnt, Qb, C, nb, cap, n_local, mass, min_k, beta):
+    sel_o, cnt_o, _, _ = oracle.select_dynamic(Qb, C, np.arange(nb), cap, n_local, mass, min_k, beta)
+    differing = 0
+    for t in range(nb):
+        g = [int(x) for x in sel[t, :cnt[t]]]
+        assert g == sorted(set(g)) and all(x == -1 for x in sel[t, cnt[t]:]), t
+        assert 0 in g and all(b in g for b in range(max(0, t - n_local + 1), t + 1)), (t, g)
+        order, frac, s = oracle_fractions(Qb[t], C, t, n_local, beta)
+        m = order.size
+        n_g = len([x for x in g if 1 <= x <= t - n_local])
+        n_o = len([x for x in sel_o[t, :cnt_o[t]] if 1 <= x <= t - n_local])
+        lo, hi = min(min_k, m), min(cap, m)
+        assert lo <= n_g <= hi, (t, n_g, lo, hi)
+        if n_g != n_o:
+            differing += 1
+            if n_g < n_o:  # the GPU stopped earlier: its prefix must be within tolerance of the target
+                assert mass - frac[n_g - 1] <= MASS_TOL, (t, n_g, n_o, frac[n_g - 1])
+            else:  # the GPU went on: the shorter prefix must have been within tolerance of the target
+                assert frac[n_g - 2] - mass <= MASS_TOL, (t, n_g, n_o, frac[n_g - 2])
+        # the kept candidates are the n_g best by score, up to fp32/fp64 near-ties
+        if n_g:
+            best = set(int(x) for x in order[:n_g])
+            kth = s[order[n_g - 1]]
+            for b in best ^ set(x for x in g if 1 <= x <= t - n_local):
+                assert abs(s[b] - kth) <= TIE_REL * abs(kth), (t, b, s[b], kth)
+    return differing
+
+
+def run_dynamic(rtp, d, window, block, cap, n_local, device, mass, min_k, beta):
+    q, k, v = d["q"].to(device), d["k"].to(device), d["v"].to(device)
+    proj = d["proj"].to(device)
+    cfg = rtp.AttnConfig(1, q.shape[2], q.shape[1], k.shape[1], window, block, cap, n_local)
+    plan = rtp.Plan(cfg, d["kinds"])
+    bufs = plan.buffers(device)
+    o = torch.full_like(q, float("nan"))
+    plan.run(q, k, v, proj, o, bufs, dynamic=dict(mass=mass, min_k=min_k, beta=beta))
+    torch.cuda.synchronize()
+    assert rtp.rtp_last_device_status() == rtp.RTP_OK
+    return q, k, v, proj, o, bufs, plan, cfg
+
+
+CASES = [
+    # seq, block, cap, n_local, mass, min_k, beta (None = scale / group)
+    # (low-rank scores of these random inputs spread by ~0.1, so a small beta
+    # makes the weights nearly equal and a large one makes them peaked)
+    (8192, 64, 32, 2, 0.9, 0, None),     # radix path (more candidates than the cap) for most rows
+    (8192, 64, 32, 2, 0.5, 4, 20.0),     # peaked weights: the cut falls inside the cap
+    (8192, 64, 64, 2, 0.3, 0, 40.0),
+    (8192, 64, 200, 2, 0.95, 0, 5.0),    # cap above every candidate count: sort of all candidates
+    (8192, 128, 16, 4, 0.7, 2, 0.0),     # equal weights: ceil(mass * candidates)
+    (16384, 64, 1000, 1, 0.99, 0, 0.05),  # cap near the 1024 limit (1024-entry sort)
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_dynamic_selection_parity(rtp, cuda_device, case):
+    n, block, cap, n_local, mass, min_k, beta = case
+    G = 4
+    d = inputs.small_prefill(n, G, 1, [2], seed=n + cap)
+    d["proj"] = inputs.random_projector(13)
+    q, k, v, proj, o, bufs, plan, cfg = run_dynamic(rtp, d, 256, block, cap, n_local, cuda_device, mass, min_k, beta)
+    b = rtp.default_selection_beta(cfg) if beta is None else beta
+    C, Qb = check_indexer(bufs["centroids"], bufs["qbar"], q, k, proj, plan.slot_heads, block, G)
+    sel, cnt = cpu(bufs["sel"][0, 0]).numpy(), cpu(bufs["sel_cnt"][0, 0]).numpy()
+    nb = n // block
+    differing = check_dynamic_rows(sel, cnt, Qb[0], C[0], nb, cap, n_local, mass, min_k, b)
+    assert differing <= max(2, nb // 100)
+    # with peaked weights the budget really varies from row to row
+    if beta is not None and beta >= 5.0:
+        assert len(set(cnt[nb // 2:].tolist())) > 1
+    # bit-reproducible
+    sel2, cnt2 = torch.empty_like(bufs["sel"]), torch.empty_like(bufs["sel_cnt"])
+    rtp.rtp_block_select_dynamic(plan.handle, bufs["qbar"], bufs["centroids"], mass, min_k, b, sel2, cnt2)
+    torch.cuda.synchronize()
+    assert torch.equal(sel2, bufs["sel"]) and torch.equal(cnt2, bufs["sel_cnt"])
+    plan.close()
+
+
+def test_prefill_on_dynamic_selection(rtp, cuda_device):
+    """Attention over the dynamically selected blocks matches the oracle on that selection."""
+    n, block, cap, n_local = 4096, 64, 24, 2
+    d = inputs.small_prefill(n, 8, 2, [2, 0], seed=5)
+    q, k, v, proj, o, bufs, plan, cfg = run_dynamic(rtp, d, 300, block, cap, n_local, cuda_device, 0.8, 1, 20.0)
+    slot_of = {h: s for s, h in enumerate(plan.slot_heads)}
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([rng.integers(0, n, 384), np.arange(0, 130), np.arange(n - 130, n)]))
+    check_prefill_rows(o, q, k, v, d["kinds"], 4, 300, block, bufs["sel"], bufs["sel_cnt"], slot_of, lambda hq: rows)
+    # rows with more candidates than the cap that keep fewer than the cap
+    cnt = cpu(bufs["sel_cnt"][0, 0]).numpy()
+    many = np.arange(n // block) - n_local > cap
+    assert (cnt[many] < 1 + cap + n_local).any()
+    plan.close()
