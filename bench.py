@@ -293,7 +293,7 @@ def needle_recall(needles, slot_of, sel, cnt, block) -> float | None:
     return hit / len(needles)
 
 
-def time_dynamic(rtp, w, res, device, points=((0.9, None), (0.99, None), (0.9, 1.0)), reps=2):
+def time_dynamic(rtp, w, res, device, points=((0.9, None), (0.99, None), (0.9, 100.0)), reps=2):
     """The layer of the main step with the dynamic (mass-threshold) selection
     in place of the fixed top-k (cap = the workload's top-k, default beta):
     selection and prefill times, blocks kept, and the executed FLOPs of the
@@ -341,6 +341,54 @@ def time_dynamic(rtp, w, res, device, points=((0.9, None), (0.99, None), (0.9, 1
             "algorithmic_tflops": flops / (pre_ms * 1e-3) / 1e12,
             "needle_recall": needle_recall(res["needles"], slot_of, sel, cnt, B)}
     return out
+
+
+def time_cp_projection(rtp, w, res, device, world=8, link_gbs=770.0):
+    """Context-parallel prefill of the main layer split over `world` ranks,
+    projected from one GPU: each rank's ranged prefill is timed here on its own
+    rows (its K/V buffer holds every row it may read), and the K/V bytes it
+    would receive are counted from the row needs of its heads and selection.
+    Transfer time = bytes / the measured peer-copy bandwidth.  Not a
+    multi-GPU measurement."""
+    from swa_hybrid_attention_b200 import context_parallel as cp
+
+    plan, bufs = res["plan"], res["bufs"]
+    q, k, v = res["q"], res["k"], res["v"]
+    cfg = plan.cfg
+    stream = torch.cuda.current_stream()
+    slot_of = {h: s for s, h in enumerate(plan.slot_heads)}
+    sel = bufs["sel"].cpu() if plan.n_sparse else None
+    cnt = bufs["sel_cnt"].cpu() if plan.n_sparse else None
+    ranks = []
+    for qb, qe in cp.cp_ranges(cfg.seq, world):
+        pr = rtp.Plan(cfg, res["kinds"], q_range=(qb, qe))
+        needs = cp.kv_needs(res["kinds"], cfg.window, cfg.block, (qb, qe), cfg.batch, sel, cnt, slot_of)
+        kv_bytes = sum(hi - lo for iv in needs.values() for lo, hi in iv) * 2 * 128 * 2
+        q_loc = q[:, :, qb:qe].contiguous()
+        k_loc, v_loc = k[:, :, :qe].contiguous(), v[:, :, :qe].contiguous()
+        o_loc = torch.empty_like(q_loc)
+        args = (pr.handle, q_loc, k_loc, v_loc, bufs["sel"] if plan.n_sparse else None,
+                bufs["sel_cnt"] if plan.n_sparse else None, o_loc, stream)
+        rtp.rtp_hybrid_prefill(*args)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(2):
+            rtp.rtp_hybrid_prefill(*args)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / 2
+        ranks.append({"q_rows": qe - qb, "prefill_ms": ms, "kv_bytes_in": kv_bytes,
+                      "transfer_ms": kv_bytes / (link_gbs * 1e9) * 1e3})
+        pr.close()
+        del q_loc, k_loc, v_loc, o_loc
+        torch.cuda.empty_cache()
+    worst = max(r["prefill_ms"] + r["transfer_ms"] for r in ranks)
+    return {"world": world, "ranks": ranks, "compute_ms_max": max(r["prefill_ms"] for r in ranks),
+            "kv_bytes_in_max": max(r["kv_bytes_in"] for r in ranks), "link_gbs": link_gbs,
+            "projected_ms_no_overlap": worst,
+            "note": "projection from one GPU: per-rank prefill timed on its own rows; K/V transfer = bytes / "
+                    "measured 770 GB/s peer copy; the indexer, selection and centroid all-gather (<1 ms) are "
+                    "not included"}
 
 
 def time_e2e(rtp, w, res, steps, device):
@@ -638,6 +686,7 @@ def run_ours(args, rank, world, local):
     extra = {}
     if not args.no_secondary and world == 1:
         extra["dynamic"] = time_dynamic(rtp, w, res, device)
+        extra["cp"] = time_cp_projection(rtp, w, res, device)
     if not args.no_e2e:
         extra["e2e"] = time_e2e(rtp, w, res, max(2, min(args.steps, 3)), device)
     for key in ("q", "k", "v", "o"):
@@ -657,6 +706,8 @@ def run_ours(args, rank, world, local):
         secondary["decode_8x256k"] = time_decode(rtp, args.decode_steps, device)
         if extra.get("dynamic"):
             secondary["dynamic_selection"] = extra["dynamic"]
+        if extra.get("cp"):
+            secondary["context_parallel_projection"] = extra["cp"]
     if rank != 0:
         return
     clocks = res["clocks"]

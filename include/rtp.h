@@ -112,6 +112,32 @@ typedef struct rtp_plan rtp_plan; /* opaque, library-owned */
  * RTP_ERR_CUDA.
  * ---------------------------------------------------------------------- */
 rtp_status rtp_route_heads(const rtp_attn_cfg* cfg, const uint8_t* kind_host, void* stream, rtp_plan** out);
+
+/* ------------------------------------------------------------------------
+ * rtp_route_heads_range — a plan for the query rows [q_begin, q_end) of the
+ * sequence only: one rank's share under context parallelism (RTPurbo page,
+ * "RTP-LLM：RTPurbo 在长文上的极致性能优化": context parallelism instead of
+ * tensor parallelism, so that each GPU computes every head's attention for
+ * its part of the context).  rtp_route_heads(cfg, ...) is
+ * rtp_route_heads_range(cfg, ..., 0, cfg->seq, ...).
+ *   q_begin   multiple of 128, 0 <= q_begin < q_end
+ *   q_end     multiple of 128, or cfg->seq; q_end <= cfg->seq
+ * With a ranged plan the other calls work on that range:
+ *   rtp_indexer_project  q and k hold rows [q_begin, q_end) only
+ *       ([batch][heads][q_end-q_begin][128]); centroids / qbar keep their
+ *       whole-sequence layout and only the blocks q_begin/block ..
+ *       q_end/block-1 are written
+ *   rtp_block_select(_dynamic)  only the query blocks of the range are
+ *       selected (whole-sequence sel/cnt layout); the centroids of every
+ *       earlier block must be present (gathered from the other ranks)
+ *   rtp_hybrid_prefill  q and o hold rows [q_begin, q_end) only; k and v are
+ *       [batch][n_kv_heads][q_end][128] of which only the rows the range's
+ *       queries can see are read (the window before q_begin for SWA heads,
+ *       every earlier row for full heads, the selected blocks for sparse
+ *       heads, and the range itself)
+ * ---------------------------------------------------------------------- */
+rtp_status rtp_route_heads_range(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int q_begin, int q_end,
+                                 void* stream, rtp_plan** out);
 void rtp_plan_destroy(rtp_plan* plan);
 
 /* Number of retrieval slots (KV heads of kind RTP_HEAD_SPARSE). */

@@ -35,7 +35,8 @@ __global__ void __launch_bounds__(kThreads) indexer_kernel(const IndexerArgs a) 
   __shared__ float total[2][kHeadDim];
   __shared__ float proj[kHeadDim * kRank];
 
-  const int blk = blockIdx.x, slot = blockIdx.y, b = blockIdx.z;
+  const int blk = a.blk0 + static_cast<int>(blockIdx.x), slot = blockIdx.y, b = blockIdx.z;
+  const int lrow = static_cast<int>(blockIdx.x) * a.block;  // first row of the block in the q/k arrays
   const int tid = threadIdx.x, rg = tid >> 4, cg = tid & 15;
   const int kvh = a.slot_heads[slot];
   const int B = a.block;
@@ -45,7 +46,7 @@ __global__ void __launch_bounds__(kThreads) indexer_kernel(const IndexerArgs a) 
   // keys of this block
   float acck[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   const __nv_bfloat16* kbase =
-      a.k + ((static_cast<size_t>(b) * a.n_kv_heads + kvh) * a.seq + static_cast<size_t>(blk) * B) * kHeadDim;
+      a.k + ((static_cast<size_t>(b) * a.n_kv_heads + kvh) * a.rows + static_cast<size_t>(lrow)) * kHeadDim;
   sum_rows(acck, kbase, B, rg, cg);
 
   // queries of this block, every head of the group (heads are consecutive)
@@ -53,7 +54,7 @@ __global__ void __launch_bounds__(kThreads) indexer_kernel(const IndexerArgs a) 
   for (int h = 0; h < a.group; ++h) {
     const int hq = kvh * a.group + h;
     const __nv_bfloat16* qbase =
-        a.q + ((static_cast<size_t>(b) * a.n_q_heads + hq) * a.seq + static_cast<size_t>(blk) * B) * kHeadDim;
+        a.q + ((static_cast<size_t>(b) * a.n_q_heads + hq) * a.rows + static_cast<size_t>(lrow)) * kHeadDim;
     sum_rows(accq, qbase, B, rg, cg);
   }
 #pragma unroll
@@ -87,7 +88,8 @@ __global__ void __launch_bounds__(kThreads) indexer_kernel(const IndexerArgs a) 
 
 cudaError_t launch_indexer(const IndexerArgs& a, cudaStream_t stream) {
   if (a.n_sparse == 0) return cudaSuccess;
-  dim3 grid(a.seq / a.block, a.n_sparse, a.batch);
+  if (a.n_blocks == 0) return cudaSuccess;
+  dim3 grid(a.n_blocks, a.n_sparse, a.batch);
   indexer_kernel<<<grid, kThreads, 0, stream>>>(a);
   return cudaGetLastError();
 }

@@ -19,8 +19,9 @@ struct PrefillArgs {
   long n_items;
   const int32_t* sel;  // [batch][n_sparse][nqb][kmax]
   const int32_t* cnt;  // [batch][n_sparse][nqb]
-  __nv_bfloat16* o;    // [batch][n_q_heads][seq][128]
+  __nv_bfloat16* o;    // [batch][n_q_heads][q_rows][128]
   int batch, seq, n_q_heads, n_kv_heads, group, n_sparse;
+  int q_row0, q_rows;  // Q/O arrays hold query rows q_row0 .. q_row0 + q_rows - 1
   int window, block, kmax, nqb;
   float scale_log2;  // softmax scale * log2(e)
   uint32_t* status;
@@ -34,6 +35,8 @@ struct IndexerArgs {
   float* qbar;       // [batch][n_sparse][nb][16]
   const int32_t* slot_heads;  // device [n_sparse] -> kv head
   int batch, seq, n_q_heads, n_kv_heads, group, n_sparse, block;
+  int blk0, rows;  // q/k arrays hold rows blk0*block .. + rows - 1 (outputs use the whole-sequence index)
+  int n_blocks;    // blocks to process, starting at blk0
 };
 
 struct SelectArgs {
@@ -42,6 +45,7 @@ struct SelectArgs {
   int32_t* sel;
   int32_t* cnt;
   int batch, n_sparse, nb, topk, n_local, kmax;
+  int t0, n_rows;  // query blocks t0 .. t0 + n_rows - 1 are selected
   // dynamic selection only: mass fraction, minimum count, beta * log2(e)
   float mass;
   int min_k;

@@ -266,8 +266,8 @@ __device__ __noinline__ void run_producer(Smem& s, const CUtensorMap* mq, const 
     for (int h = 0; h < 2; ++h) {
       if (!mbar_wait(&s.q_empty[h], (it & 1u) ^ 1u, abort, a.status)) goto drain;
       mbar_arrive_expect_tx(&s.q_full[h], kTileBytes);
-      tma_load_3d(s.q[h], mq, &s.q_full[h], 0, 128 * item.t, zq + h);
-      tma_load_3d(s.q[h] + kChunkBytes, mq, &s.q_full[h], 64, 128 * item.t, zq + h);
+      tma_load_3d(s.q[h], mq, &s.q_full[h], 0, 128 * item.t - a.q_row0, zq + h);
+      tma_load_3d(s.q[h] + kChunkBytes, mq, &s.q_full[h], 64, 128 * item.t - a.q_row0, zq + h);
       q_issued |= 1u << h;
     }
     {
@@ -521,8 +521,9 @@ __device__ __noinline__ void run_softmax(Smem& s, uint32_t tmem, int h, const Pr
     const float inv = l > 0.f ? 1.f / l : 0.f;
     const int hq = item.kvh * a.group + 2 * item.pair + h;
     __nv_bfloat16* orow =
-        a.o + ((static_cast<size_t>(item.b) * a.n_q_heads + hq) * static_cast<size_t>(a.seq) + i) * kHeadDim;
-    const bool valid = i < a.seq;
+        a.o + ((static_cast<size_t>(item.b) * a.n_q_heads + hq) * static_cast<size_t>(a.q_rows) + (i - a.q_row0)) *
+                  kHeadDim;
+    const bool valid = i - a.q_row0 < a.q_rows;
 #pragma unroll 1
     for (int c = 0; c < 4; ++c) {
       uint32_t o[32];

@@ -25,6 +25,7 @@ struct rtp_plan {
   int n_sparse = 0;
   int nqt = 0;  // 128-row query tiles
   int nqb = 0;  // query blocks of `block` rows
+  int q_begin = 0, q_end = 0;  // query rows of this plan (whole sequence unless ranged)
   std::vector<uint8_t> kind;
   std::vector<int32_t> slot_heads;
   std::vector<int32_t> items_host;  // [n_items][4]
@@ -177,9 +178,21 @@ const char* rtp_status_str(rtp_status s) {
 int rtp_version(void) { return (1 << 16) | 0; }
 
 rtp_status rtp_route_heads(const rtp_attn_cfg* cfg, const uint8_t* kind_host, void* stream, rtp_plan** out) {
+  if (!cfg) {
+    if (out) *out = nullptr;
+    return RTP_ERR_INVALID_ARG;
+  }
+  return rtp_route_heads_range(cfg, kind_host, 0, cfg->seq, stream, out);
+}
+
+rtp_status rtp_route_heads_range(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int q_begin, int q_end,
+                                 void* stream, rtp_plan** out) {
   if (!out) return RTP_ERR_INVALID_ARG;
   *out = nullptr;
   if (!cfg_prefill_ok(cfg) || !kind_host) return RTP_ERR_INVALID_ARG;
+  if (q_begin < 0 || q_begin >= q_end || q_end > cfg->seq || q_begin % 128 != 0 ||
+      (q_end % 128 != 0 && q_end != cfg->seq))
+    return RTP_ERR_INVALID_ARG;
   for (int h = 0; h < cfg->n_kv_heads; ++h)
     if (kind_host[h] > RTP_HEAD_SPARSE) return RTP_ERR_INVALID_ARG;
 
@@ -199,6 +212,9 @@ rtp_status rtp_route_heads(const rtp_attn_cfg* cfg, const uint8_t* kind_host, vo
   p->n_sparse = static_cast<int>(p->slot_heads.size());
   p->nqt = (cfg->seq + 127) / 128;
   p->nqb = cfg->seq / cfg->block;
+  p->q_begin = q_begin;
+  p->q_end = q_end;
+  const int t_lo = q_begin / 128, t_hi = (q_end + 127) / 128;
   const int group = cfg->n_q_heads / cfg->n_kv_heads;
   const int pairs = group / 2;
 
@@ -208,10 +224,10 @@ rtp_status rtp_route_heads(const rtp_attn_cfg* cfg, const uint8_t* kind_host, vo
     int32_t v[4];
   };
   std::vector<W> work;
-  work.reserve(static_cast<size_t>(cfg->batch) * cfg->n_kv_heads * pairs * p->nqt);
+  work.reserve(static_cast<size_t>(cfg->batch) * cfg->n_kv_heads * pairs * (t_hi - t_lo));
   for (int b = 0; b < cfg->batch; ++b)
     for (int h = 0; h < cfg->n_kv_heads; ++h)
-      for (int t = 0; t < p->nqt; ++t) {
+      for (int t = t_lo; t < t_hi; ++t) {
         long cost;
         const int kind = kind_host[h];
         if (kind == RTP_HEAD_FULL) {
@@ -310,6 +326,9 @@ rtp_status rtp_indexer_project(const rtp_plan* plan, const void* q, const void* 
   a.group = c.n_q_heads / c.n_kv_heads;
   a.n_sparse = plan->n_sparse;
   a.block = c.block;
+  a.blk0 = plan->q_begin / c.block;
+  a.rows = plan->q_end - plan->q_begin;
+  a.n_blocks = plan->q_end / c.block - a.blk0;
   return cuda_status(launch_indexer(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -332,6 +351,8 @@ rtp_status rtp_block_select(const rtp_plan* plan, const float* qbar, const float
   a.topk = c.topk;
   a.n_local = c.n_local;
   a.kmax = c.topk + 1 + c.n_local;
+  a.t0 = plan->q_begin / c.block;
+  a.n_rows = plan->q_end / c.block - a.t0;
   return cuda_status(launch_select(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -357,6 +378,8 @@ rtp_status rtp_block_select_dynamic(const rtp_plan* plan, const float* qbar, con
   a.topk = c.topk;
   a.n_local = c.n_local;
   a.kmax = c.topk + 1 + c.n_local;
+  a.t0 = plan->q_begin / c.block;
+  a.n_rows = plan->q_end / c.block - a.t0;
   a.mass = mass;
   a.min_k = min_k;
   a.beta_log2 = beta * kLog2e;
@@ -372,9 +395,10 @@ rtp_status rtp_hybrid_prefill(const rtp_plan* plan, const void* q, const void* k
   const rtp_attn_cfg& c = plan->cfg;
   if (current_device() != plan->device) return RTP_ERR_INVALID_ARG;
   CUtensorMap mq, mk, mv;
-  if (!encode_bf16_3d(&mq, q, c.seq, static_cast<long>(c.batch) * c.n_q_heads, 128) ||
-      !encode_bf16_3d(&mk, k, c.seq, static_cast<long>(c.batch) * c.n_kv_heads, 64) ||
-      !encode_bf16_3d(&mv, v, c.seq, static_cast<long>(c.batch) * c.n_kv_heads, 64))
+  const int q_rows = plan->q_end - plan->q_begin;
+  if (!encode_bf16_3d(&mq, q, q_rows, static_cast<long>(c.batch) * c.n_q_heads, 128) ||
+      !encode_bf16_3d(&mk, k, plan->q_end, static_cast<long>(c.batch) * c.n_kv_heads, 64) ||
+      !encode_bf16_3d(&mv, v, plan->q_end, static_cast<long>(c.batch) * c.n_kv_heads, 64))
     return RTP_ERR_CUDA;
   PrefillArgs a;
   a.items = plan->d_items;
@@ -384,6 +408,8 @@ rtp_status rtp_hybrid_prefill(const rtp_plan* plan, const void* q, const void* k
   a.o = static_cast<__nv_bfloat16*>(o);
   a.batch = c.batch;
   a.seq = c.seq;
+  a.q_row0 = plan->q_begin;
+  a.q_rows = q_rows;
   a.n_q_heads = c.n_q_heads;
   a.n_kv_heads = c.n_kv_heads;
   a.group = c.n_q_heads / c.n_kv_heads;

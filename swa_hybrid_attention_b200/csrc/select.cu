@@ -28,7 +28,7 @@ namespace {
 __global__ void __launch_bounds__(kSelThreads) block_select_kernel(const SelectArgs a) {
   extern __shared__ uint32_t keys[];
   __shared__ SelectScratch sh;
-  const int t = blockIdx.x, slot = blockIdx.y, b = blockIdx.z;
+  const int t = a.t0 + static_cast<int>(blockIdx.x), slot = blockIdx.y, b = blockIdx.z;
   const size_t row = (static_cast<size_t>(b) * a.n_sparse + slot) * a.nb + t;
   int32_t* out = a.sel + row * a.kmax;
   const float* C = a.centroids + (static_cast<size_t>(b) * a.n_sparse + slot) * a.nb * kRank;
@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kSelThreads) block_select_dynamic_kernel(const
   __shared__ SelectScratch sh;
   __shared__ DynScratch d;
   const int tid = threadIdx.x;
-  const int t = blockIdx.x, slot = blockIdx.y, b = blockIdx.z;
+  const int t = a.t0 + static_cast<int>(blockIdx.x), slot = blockIdx.y, b = blockIdx.z;
   const size_t row = (static_cast<size_t>(b) * a.n_sparse + slot) * a.nb + t;
   int32_t* out = a.sel + row * a.kmax;
   const float* C = a.centroids + (static_cast<size_t>(b) * a.n_sparse + slot) * a.nb * kRank;
@@ -256,7 +256,8 @@ cudaError_t launch_select_dynamic(const SelectArgs& a, cudaStream_t stream) {
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  dim3 grid(a.nb, a.n_sparse, a.batch);
+  if (a.n_rows == 0) return cudaSuccess;
+  dim3 grid(a.n_rows, a.n_sparse, a.batch);
   block_select_dynamic_kernel<<<grid, kSelThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
@@ -269,7 +270,8 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream) {
         cudaFuncSetAttribute(block_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  dim3 grid(a.nb, a.n_sparse, a.batch);
+  if (a.n_rows == 0) return cudaSuccess;
+  dim3 grid(a.n_rows, a.n_sparse, a.batch);
   block_select_kernel<<<grid, kSelThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }

@@ -49,6 +49,7 @@ def _load() -> ctypes.CDLL:
     cfgp = ctypes.POINTER(rtp_attn_cfg)
     sig = {
         "rtp_route_heads": (I, [cfgp, P, P, ctypes.POINTER(P)]),
+        "rtp_route_heads_range": (I, [cfgp, P, I, I, P, ctypes.POINTER(P)]),
         "rtp_plan_destroy": (None, [P]),
         "rtp_plan_num_sparse": (I, [P]),
         "rtp_plan_num_items": (L, [P]),
@@ -76,7 +77,7 @@ def _load() -> ctypes.CDLL:
 
 
 _lib = _load()
-EXPORTED = ("rtp_route_heads", "rtp_plan_destroy", "rtp_plan_num_sparse", "rtp_plan_num_items",
+EXPORTED = ("rtp_route_heads", "rtp_route_heads_range", "rtp_plan_destroy", "rtp_plan_num_sparse", "rtp_plan_num_items",
             "rtp_plan_sparse_heads", "rtp_plan_work_items", "rtp_indexer_project", "rtp_block_select",
             "rtp_block_select_dynamic",
             "rtp_hybrid_prefill", "rtp_decode_workspace_bytes", "rtp_sparse_decode", "rtp_sparse_decode_noalloc",
@@ -148,6 +149,15 @@ def rtp_route_heads(cfg: AttnConfig, kinds, stream=None) -> int:
     c = cfg.c()
     _check("rtp_route_heads", _lib.rtp_route_heads(ctypes.byref(c), _kinds(kinds), _stream(stream),
                                                      ctypes.byref(out)))
+    return out.value
+
+
+def rtp_route_heads_range(cfg: AttnConfig, kinds, q_begin: int, q_end: int, stream=None) -> int:
+    """A plan for query rows [q_begin, q_end) only (one context-parallel rank's share)."""
+    out = ctypes.c_void_p()
+    c = cfg.c()
+    _check("rtp_route_heads_range", _lib.rtp_route_heads_range(ctypes.byref(c), _kinds(kinds), int(q_begin),
+                                                                 int(q_end), _stream(stream), ctypes.byref(out)))
     return out.value
 
 
@@ -267,10 +277,14 @@ def rtp_version() -> int:
 class Plan:
     """Owns a routing plan (rtp_route_heads / rtp_plan_destroy)."""
 
-    def __init__(self, cfg: AttnConfig, kinds, stream=None):
+    def __init__(self, cfg: AttnConfig, kinds, stream=None, q_range: tuple | None = None):
         self.cfg = cfg
         self.kinds = list(kinds)
-        self.handle = rtp_route_heads(cfg, kinds, stream)
+        self.q_range = (0, cfg.seq) if q_range is None else (int(q_range[0]), int(q_range[1]))
+        if q_range is None:
+            self.handle = rtp_route_heads(cfg, kinds, stream)
+        else:
+            self.handle = rtp_route_heads_range(cfg, kinds, self.q_range[0], self.q_range[1], stream)
         self.n_sparse = rtp_plan_num_sparse(self.handle)
         self.slot_heads = rtp_plan_sparse_heads(self.handle)
 
