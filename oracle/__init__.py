@@ -55,11 +55,13 @@ def _load():
         _lib.oracle_scores.argtypes = [P, P, L, I, P]
         _lib.oracle_select.argtypes = [P, P, L, I, P, L, I, I, I, P, P, P]
         _lib.oracle_select_dynamic.argtypes = [P, P, L, I, P, L, I, I, I, D, I, D, P, P, P, P]
+        _lib.oracle_kmeans.argtypes = [P, L, I, I, I, P, P]
+        _lib.oracle_attention_keys.argtypes = [P, I, P, P, I, P, L, D, P]
         _lib.oracle_attention_rows.argtypes = [P, P, L, P, P, L, I, I, L, I, P, P, I, D, P]
         _lib.oracle_attention_probs.argtypes = [P, L, P, L, I, I, L, I, P, P, I, D, P]
         _lib.oracle_decode_head.argtypes = [P, I, P, P, L, I, P, L, P, I, I, L, I, I, I, I, I, P, P, P, D, P]
         for f in ("oracle_project_rows", "oracle_centroids", "oracle_qbar", "oracle_scores", "oracle_select",
-                  "oracle_select_dynamic",
+                  "oracle_select_dynamic", "oracle_kmeans", "oracle_attention_keys",
                   "oracle_attention_rows", "oracle_attention_probs", "oracle_decode_head"):
             getattr(_lib, f).restype = None
     return _lib
@@ -291,6 +293,67 @@ def cache_append(kcache, vcache, C, kinds, pos: int, k_new, v_new, block: int, p
                 if int(kinds[h]) == SPARSE:
                     Cn[b, h, blk] = centroids(kc[b, h, blk * block:(blk + 1) * block], block, proj)[0]
     return kc, vc, Cn
+
+
+def kmeans(X: np.ndarray, n_clusters: int, iters: int):
+    """Lloyd's k-means on projected keys X [n, r] (RTPurboV2 page: clustering of
+    the projected keys).  Evenly spaced initial centroids, nearest centroid by
+    squared distance (ties to the lower index), empty clusters keep their
+    centroid.  Returns (centroids [nc, r] fp64, assignment [n] int32)."""
+    x = np.ascontiguousarray(X, dtype=np.float64)
+    n, r = x.shape
+    mu = np.empty((n_clusters, r), dtype=np.float64)
+    assign = np.zeros(n, dtype=np.int32)
+    _load().oracle_kmeans(_ptr(x), n, r, n_clusters, iters, _ptr(mu), _ptr(assign))
+    return mu, assign
+
+
+def cluster_chunks(assign: np.ndarray, row0: int, n_clusters: int, chunk: int = 128):
+    """Members of each cluster (key positions row0 + index, ascending) in
+    cluster order, and the cluster's members cut into chunks of at most
+    `chunk` keys.  Returns (members [n], offsets [nc+1], chunks: list of
+    (cluster, start, length) with start an index into members)."""
+    a = np.asarray(assign)
+    order = np.lexsort((np.arange(a.size), a))  # by cluster, then position
+    members = (order + row0).astype(np.int64)
+    counts = np.bincount(a, minlength=n_clusters)
+    offsets = np.concatenate([[0], np.cumsum(counts)])
+    chunks = []
+    for c in range(n_clusters):
+        for s0 in range(int(offsets[c]), int(offsets[c + 1]), chunk):
+            chunks.append((c, s0, min(chunk, int(offsets[c + 1]) - s0)))
+    return members, offsets, chunks
+
+
+def attention_keys(q_group, kc_head, vc_head, keys, scale: float | None = None) -> np.ndarray:
+    """Exact attention of the group's query rows [G, 128] over the listed cached keys -> fp64 [G, 128]."""
+    qb = _bf16_bits(q_group).reshape(-1, 128)
+    kb = _bf16_bits(kc_head).reshape(-1, 128)
+    vb = _bf16_bits(vc_head).reshape(-1, 128)
+    kk = np.ascontiguousarray(keys, dtype=np.int64)
+    sc = 1.0 / np.sqrt(128.0) if scale is None else float(scale)
+    out = np.empty((qb.shape[0], 128), dtype=np.float64)
+    _load().oracle_attention_keys(_ptr(qb), qb.shape[0], _ptr(kb), _ptr(vb), 128, _ptr(kk), kk.size, sc, _ptr(out))
+    return out
+
+
+def decode_clustered_keys(members, chunks, chosen, block: int, clu_end: int, cache_len: int) -> np.ndarray:
+    """Keys a clustered decode step attends to: the sink block, the keys of the
+    chosen chunks (all inside [block, clu_end)) and the unclustered tail
+    [clu_end, cache_len), ascending."""
+    keys = list(range(0, min(block, cache_len)))
+    for x in chosen:
+        _, s0, n = chunks[int(x)]
+        keys.extend(int(k) for k in members[s0:s0 + n])
+    keys.extend(range(clu_end, cache_len))
+    return np.array(sorted(keys), dtype=np.int64)
+
+
+def topk_chunks(qbar_row: np.ndarray, chunk_centroids: np.ndarray, topk: int) -> np.ndarray:
+    """The topk chunks by (score desc, index asc), ascending."""
+    s = scores(qbar_row, chunk_centroids)
+    order = np.lexsort((np.arange(s.size), -s))
+    return np.sort(order[:topk])
 
 
 def round_bf16(x: np.ndarray) -> np.ndarray:

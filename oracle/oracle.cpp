@@ -245,6 +245,73 @@ void oracle_select_dynamic(const double* qbar, const double* C, long nb, int r, 
   });
 }
 
+// [P2] clustering of the projected keys ("聚类中心"), read as k-means (Lloyd's
+// algorithm) on the r-dim projected keys X [n][r] (fp64):
+//   init      mu_c = X[floor((2c+1) n / (2 nc))], c = 0..nc-1 (evenly spaced);
+//   iterate   `iters` times: assign each point to the nearest centroid
+//             (squared Euclidean distance; ties to the lower index), then set
+//             each centroid to the mean of its points (a cluster with no
+//             point keeps its centroid).
+// Writes the final centroids [nc][r] and the last assignment [n].
+void oracle_kmeans(const double* X, long n, int r, int nc, int iters, double* mu, int32_t* assign) {
+  for (int c = 0; c < nc; ++c) {
+    const long j = (static_cast<long>(2 * c + 1) * n) / (2L * nc);
+    for (int d = 0; d < r; ++d) mu[c * r + d] = X[j * r + d];
+  }
+  for (int it = 0; it < iters; ++it) {
+    parallel_for(n, [&](long j) {
+      double best = INFINITY;
+      int bc = 0;
+      for (int c = 0; c < nc; ++c) {
+        double dist = 0.0;
+        for (int d = 0; d < r; ++d) {
+          const double e = X[j * r + d] - mu[c * r + d];
+          dist += e * e;
+        }
+        if (dist < best) {
+          best = dist;
+          bc = c;
+        }
+      }
+      assign[j] = bc;
+    });
+    std::vector<double> sum(static_cast<size_t>(nc) * r, 0.0);
+    std::vector<long> count(nc, 0);
+    for (long j = 0; j < n; ++j) {
+      ++count[assign[j]];
+      for (int d = 0; d < r; ++d) sum[assign[j] * r + d] += X[j * r + d];
+    }
+    for (int c = 0; c < nc; ++c)
+      if (count[c] > 0)
+        for (int d = 0; d < r; ++d) mu[c * r + d] = sum[c * r + d] / count[c];
+  }
+}
+
+// Exact attention of G query rows over an explicit list of cached keys
+// (used for decode over clustered keys): O_h = softmax_j(scale q_h . k_j) V
+// over j in keys[0..n_keys), fp64.  out [G][D].
+void oracle_attention_keys(const uint16_t* q, int G, const uint16_t* kc, const uint16_t* vc, int D,
+                           const int64_t* keys, long n_keys, double scale, double* out) {
+  for (int h = 0; h < G; ++h) {
+    std::vector<double> s(n_keys);
+    double m = -INFINITY;
+    for (long e = 0; e < n_keys; ++e) {
+      double acc = 0.0;
+      for (int d = 0; d < D; ++d) acc += widen_bf16(q[h * D + d]) * widen_bf16(kc[keys[e] * D + d]);
+      s[e] = acc * scale;
+      m = std::max(m, s[e]);
+    }
+    double l = 0.0;
+    std::vector<double> o(D, 0.0);
+    for (long e = 0; e < n_keys; ++e) {
+      const double p = std::exp(s[e] - m);
+      l += p;
+      for (int d = 0; d < D; ++d) o[d] += p * widen_bf16(vc[keys[e] * D + d]);
+    }
+    for (int d = 0; d < D; ++d) out[h * D + d] = o[d] / l;
+  }
+}
+
 // Visible keys of query position i for one head ([P1] SWA drops far tokens,
 // full heads see every earlier token, [P4] sparse heads see the selected set):
 //   mode 0 (SWA):    i-W < j <= i

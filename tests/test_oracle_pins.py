@@ -496,3 +496,79 @@ def test_dynamic_selection_stops_at_planted_mass():
     assert cnt[0] == 1 + 4 + n_local
     sel, cnt, _, _ = oracle.select_dynamic(q[None], C, [39], 1, n_local, 0.9, 0, 1.0)
     assert list(sel[0, :cnt[0]]) == [0, 7, 38, 39]
+
+
+# ------------------------------------------------------ k-means clustering
+
+
+def _objective(X, mu, assign):
+    return float(((X - mu[assign]) ** 2).sum())
+
+
+def test_kmeans_recovers_planted_blobs_in_one_step():
+    rng = np.random.default_rng(0)
+    nc, per, r = 6, 40, 16
+    centers = rng.normal(scale=20.0, size=(nc, r))
+    X = np.concatenate([centers[c] + rng.normal(scale=0.1, size=(per, r)) for c in range(nc)])
+    mu, assign = oracle.kmeans(X, nc, 1)  # the evenly spaced start puts one seed in each blob
+    assert np.array_equal(assign, np.repeat(np.arange(nc), per))
+    ref = X.reshape(nc, per, r).mean(axis=1)
+    assert np.max(np.abs(mu - ref)) <= 1e-12
+
+
+def test_kmeans_objective_never_increases_and_converges_to_nearest():
+    rng = np.random.default_rng(1)
+    X = rng.normal(size=(500, 16))
+    prev = np.inf
+    for it in range(1, 8):
+        mu, assign = oracle.kmeans(X, 12, it)
+        obj = _objective(X, mu, assign)
+        assert obj <= prev + 1e-9
+        prev = obj
+    mu, assign = oracle.kmeans(X, 12, 200)
+    mu2, assign2 = oracle.kmeans(X, 12, 201)
+    assert np.array_equal(assign, assign2)  # converged
+    d = ((X[:, None, :] - mu[None]) ** 2).sum(-1)
+    assert np.array_equal(np.argmin(d, axis=1), assign)  # every point sits with its nearest centroid
+
+
+def test_kmeans_degenerate_sizes():
+    rng = np.random.default_rng(2)
+    X = rng.normal(size=(9, 16))
+    mu, assign = oracle.kmeans(X, 9, 3)  # one point per cluster
+    assert np.array_equal(assign, np.arange(9)) and np.array_equal(mu, X)
+    mu0, _ = oracle.kmeans(X, 3, 0)  # no iteration: the evenly spaced seeds
+    assert np.array_equal(mu0, X[[1, 4, 7]])
+
+
+def test_cluster_chunks_cover_members_once():
+    rng = np.random.default_rng(3)
+    assign = rng.integers(0, 5, size=700)
+    assign[:300] = 2  # one cluster larger than two chunks
+    members, offsets, chunks = oracle.cluster_chunks(assign, 128, 5)
+    assert sorted(members.tolist()) == list(range(128, 828))
+    seen = []
+    for c, s0, n in chunks:
+        assert 1 <= n <= 128 and offsets[c] <= s0 and s0 + n <= offsets[c + 1]
+        block = members[s0:s0 + n]
+        assert np.all(assign[block - 128] == c) and np.all(np.diff(block) > 0)
+        seen.extend(block.tolist())
+    assert sorted(seen) == list(range(128, 828))
+
+
+def test_attention_over_key_list_matches_bruteforce_and_full_row():
+    Lc, G = 700, 2
+    d = inputs.small_prefill(Lc, G, 1, [oracle.FULL], seed=45)
+    q, k, v = d["q"][0], d["k"][0, 0], d["v"][0, 0]
+    rng = np.random.default_rng(4)
+    keys = np.sort(rng.choice(Lc, size=150, replace=False))
+    got = oracle.attention_keys(q[:, Lc - 1], k, v, keys)
+    m = np.zeros((1, Lc), dtype=bool)
+    m[0, keys] = True
+    for h in range(G):
+        ref = dense_reference(widen(q[h, Lc - 1:Lc]), widen(k), widen(v), m)
+        assert np.max(np.abs(got[h] - ref[0])) <= 1e-12
+    allk = oracle.attention_keys(q[:, Lc - 1], k, v, np.arange(Lc))
+    for h in range(G):
+        full = oracle.attention_rows(q[h, Lc - 1:Lc], np.array([Lc - 1]), k, v, oracle.FULL)
+        assert np.max(np.abs(allk[h] - full[0])) <= 1e-12
