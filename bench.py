@@ -503,6 +503,7 @@ def time_decode(rtp, steps, device):
     ms = statistics.median(a.elapsed_time(b) for a, b in times)
     status = rtp.rtp_last_device_status(stream)
     upkeep = time_cache_upkeep(rtp, w, d, C, cfg, flush, flush_read, steps, stream)
+    clustered = time_clustered_decode(rtp, w, d, flush, flush_read, steps, stream)
     G = w.group
     ns = sum(1 for k in kinds if k == inputs.SPARSE)
     nsw = len(kinds) - ns
@@ -512,7 +513,68 @@ def time_decode(rtp, steps, device):
     flops = w.batch * keys * G * 4 * 128
     return {"workload": w.name, "ms_per_step": ms, "algorithmic_bytes": bytes_, "gb_s": bytes_ / (ms * 1e-3) / 1e9,
             "tflops_effective": flops / (ms * 1e-3) / 1e12, "l2": "flushed before each step (256 MB write, then 256 MB read)",
-            "launches_per_step": 3, "status": rtp.status_str(status), "cache_upkeep": upkeep}
+            "launches_per_step": 3, "status": rtp.status_str(status), "cache_upkeep": upkeep,
+            "clustered": clustered}
+
+
+def time_clustered_decode(rtp, w, d, flush, flush_read, steps, stream, n_clusters=2048, iters=8):
+    """Decode with k-means-clustered retrieval heads on the decode workload:
+    the clustering of rows [block, clu_end) of every retrieval head (clu_end
+    leaves the last n_local blocks as the unclustered tail), then the decode
+    step selecting top-k chunks of <= 128 keys (L2 flushed as for the main
+    decode step)."""
+    kinds, Lc = d["kinds"], d["cache_len"]
+    B = w.block
+    clu_end = (Lc // B - w.n_local) * B
+    ns = sum(1 for k in kinds if k == inputs.SPARSE)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    cl = rtp.cluster_cache(d["kcache"], d["vcache"], d["proj"], kinds, clu_end=clu_end, n_clusters=n_clusters,
+                           iters=iters, block=B, stream=stream)
+    b.record(stream)
+    torch.cuda.synchronize()
+    km_ms = a.elapsed_time(b)
+    cfg = rtp.AttnConfig(w.batch, Lc, w.n_q_heads, w.n_kv_heads, w.window, B, w.topk, w.n_local)
+    ws_bytes = rtp.rtp_decode_clustered_workspace_bytes(cfg, kinds, Lc, clu_end)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=d["q"].device)
+    o = torch.empty_like(d["q"])
+    cnt = torch.zeros(w.batch, w.n_kv_heads, dtype=torch.int32, device=d["q"].device)
+    if ws_bytes == 0:
+        raise RuntimeError("clustered decode: rejected configuration")
+    sel = torch.full((w.batch, w.n_kv_heads, 1 + (Lc - clu_end + 127) // 128 + w.topk), -1,
+                     dtype=torch.int32, device=d["q"].device)
+    args = (cfg, kinds, Lc, d["q"], d["kcache"], d["vcache"], d["proj"], cl, o, ws, ws_bytes, sel, cnt)
+    for _ in range(5):
+        rtp.rtp_sparse_decode_clustered(*args, stream=stream)
+    torch.cuda.synchronize()
+    ev = []
+    for _ in range(steps):
+        flush.zero_()
+        flush_read.sum()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        rtp.rtp_sparse_decode_clustered(*args, stream=stream)
+        e1.record(stream)
+        ev.append((e0, e1))
+    torch.cuda.synchronize()
+    ms = statistics.median(x.elapsed_time(y) for x, y in ev)
+    status = rtp.rtp_last_device_status(stream)
+    # keys read: every retrieval head's sink block, tail and selected chunks, every window head's window
+    sel_c, cnt_c = sel.cpu(), cnt.cpu()
+    lens = cl.chunk_len.cpu()
+    keys = 0
+    for bb in range(w.batch):
+        for h, kind in enumerate(kinds):
+            if kind == inputs.SPARSE:
+                m = int(cnt_c[bb, h]) - 1 - (Lc - clu_end + 127) // 128
+                keys += B + (Lc - clu_end) + sum(int(lens[bb, h, int(x)]) for x in sel_c[bb, h, 1:1 + m])
+            else:
+                keys += min(w.window, Lc)
+    bytes_ = keys * 128 * 2 * 2 + w.batch * ns * cl.max_chunks * 16 * 4 + w.batch * w.n_q_heads * 128 * 2 * 2
+    chunks = cl.n_chunks.cpu()[:, [h for h, k in enumerate(kinds) if k == inputs.SPARSE]].float()
+    return {"n_clusters": n_clusters, "iters": iters, "clu_end": clu_end, "kmeans_ms": km_ms,
+            "mean_chunks_per_head": float(chunks.mean()), "ms_per_step": ms, "algorithmic_bytes": bytes_,
+            "gb_s": bytes_ / (ms * 1e-3) / 1e9, "status": rtp.status_str(status)}
 
 
 def time_cache_upkeep(rtp, w, d, C, cfg, flush, flush_read, steps, stream):

@@ -346,6 +346,74 @@ rtp_status rtp_cache_append(const rtp_attn_cfg* cfg, const uint8_t* kind_host, i
                             void* stream);
 
 /* ------------------------------------------------------------------------
+ * Clustered KV cache (RTPurboV2 page: clustering the projected keys lets
+ * decode skip whole groups of unrelated tokens; the page's deployment runs
+ * full attention in prefill, clusters the K cache, then decodes sparsely).
+ * Rows [block, clu_end) of every retrieval head are grouped by k-means of
+ * their projected keys P^T k; each cluster's keys (ascending positions) are
+ * cut into chunks of at most 128 keys, the units the decode step selects.
+ * All arrays are device memory owned by the caller; n = clu_end - block,
+ * max_chunks = n / 128 + n_clusters (an upper bound on the chunks of a head).
+ * Entries of non-retrieval heads are not written or read.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int clu_end;             /* rows [block, clu_end) are clustered: multiple of block, > block */
+  int n_clusters;          /* 1 .. 2048, <= n */
+  float* centroids;        /* fp32 [batch][n_kv_heads][n_clusters][16] */
+  int32_t* members;        /* [batch][n_kv_heads][n]: key rows grouped by cluster, ascending inside */
+  int32_t* offsets;        /* [batch][n_kv_heads][n_clusters + 1]: cluster c = members[offsets[c] ..] */
+  void* k_sorted;          /* bf16 [batch][n_kv_heads][n][128]: K rows in `members` order */
+  void* v_sorted;          /* bf16, likewise for V */
+  float* chunk_centroids;  /* fp32 [batch][n_kv_heads][max_chunks][16]: the centroid of the chunk's cluster */
+  int32_t* chunk_start;    /* [batch][n_kv_heads][max_chunks]: first row of the chunk in k_sorted */
+  int32_t* chunk_len;      /* [batch][n_kv_heads][max_chunks]: 1..128 */
+  int32_t* n_chunks;       /* [batch][n_kv_heads]: chunks in use, cluster-major order */
+} rtp_clusters;
+
+/* ------------------------------------------------------------------------
+ * rtp_cache_cluster — k-means of the projected cached keys of every
+ * retrieval head (the library's reading of the page's clustering):
+ * seeds mu_c = X[floor((2c+1) n / (2 n_clusters))] of X_j = P^T k_j
+ * (fp32, fixed order); `iters` rounds of: each key to the nearest centroid
+ * (squared distance, evaluated as |mu|^2 - 2 x.mu; ties to the lower
+ * index), each centroid to the mean of its keys (an empty cluster keeps its
+ * centroid).  Then the members, offsets, chunk table and the K/V rows in
+ * cluster order are written.  Deterministic (fixed-order sums, a stable
+ * counting sort).
+ *   cfg        batch, n_kv_heads, head_dim, block, rank used; seq = cache
+ *              capacity as for rtp_sparse_decode (must be >= clu_end)
+ *   kind_host  HOST [n_kv_heads]; RTP_HEAD_SPARSE heads are clustered
+ *   iters      rounds, 1 .. 1000
+ *   kcache, vcache, proj  as for rtp_sparse_decode
+ *   cl         clu_end, n_clusters and the output arrays
+ *   workspace  device scratch of rtp_cache_cluster_workspace_bytes bytes
+ * Errors: RTP_ERR_INVALID_ARG (nothing launched), RTP_ERR_CUDA.
+ * ---------------------------------------------------------------------- */
+size_t rtp_cache_cluster_workspace_bytes(const rtp_attn_cfg* cfg, int clu_end);
+rtp_status rtp_cache_cluster(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int iters, const void* kcache,
+                             const void* vcache, const float* proj, const rtp_clusters* cl, void* workspace,
+                             size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * rtp_sparse_decode_clustered — rtp_sparse_decode with clustered retrieval
+ * heads: such a head scores the chunks of its clusters by
+ * qbar . centroid(cluster) (qbar = sum_{h in group} P^T q_h), keeps the topk
+ * best by (score desc, chunk index asc) and attends exactly to their keys,
+ * to the sink block [0, block) and to every key of the unclustered tail
+ * [clu_end, cache_len) (tokens cached after clustering; clu_end <=
+ * cache_len).  Streaming (SWA) and full heads are as in rtp_sparse_decode.
+ * Arguments as rtp_sparse_decode (centroids replaced by `cl`); sel_out /
+ * cnt_out rows hold, for a retrieval head, entry 0 (the sink) then the
+ * selected chunk indices, and cnt = 1 + tail spans + chunks kept.
+ * ---------------------------------------------------------------------- */
+size_t rtp_decode_clustered_workspace_bytes(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len,
+                                            int clu_end);
+rtp_status rtp_sparse_decode_clustered(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len,
+                                       const void* q, const void* kcache, const void* vcache, const float* proj,
+                                       const rtp_clusters* cl, void* o, void* workspace, size_t ws_bytes,
+                                       int32_t* sel_out, int32_t* cnt_out, void* stream);
+
+/* ------------------------------------------------------------------------
  * rtp_last_device_status — synchronise `stream`, then read and clear the
  * device status word of the current device.  Returns RTP_OK, RTP_ERR_TIMEOUT
  * (a bounded wait gave up), RTP_ERR_INVALID_ARG (a kernel met an

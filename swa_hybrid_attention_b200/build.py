@@ -19,7 +19,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "librtp.so")
-SOURCES = ["rtp_api.cu", "prefill.cu", "indexer.cu", "select.cu", "decode.cu", "cache.cu"]
+SOURCES = ["rtp_api.cu", "prefill.cu", "indexer.cu", "select.cu", "decode.cu", "cache.cu", "kmeans.cu"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

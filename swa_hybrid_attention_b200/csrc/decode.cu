@@ -145,6 +145,27 @@ __device__ __forceinline__ uint32_t warp_sort_asc(uint32_t v) {
   return v;
 }
 
+// Block of the new token, and the number of spans every retrieval head
+// visits whatever the scores: the sink and the local blocks {0} u {t-L+1..t},
+// or, for clustered heads, the sink block and the unclustered tail
+// [clu_end, cache_len) in 128-key pieces.
+__device__ __forceinline__ int decode_t(const DecodeArgs& a) { return (a.cache_len - 1) / a.block; }
+__device__ __forceinline__ int n_fixed(const DecodeArgs& a) {
+  return a.clustered ? 1 + (a.cache_len - a.clu_end + 127) / 128 : min(decode_t(a) + 1, a.n_local + 1);
+}
+
+// Entries of a full selection row besides the topk picks out[1..topk]: the
+// sink marker, then the local blocks (contiguous mode) or nothing (clustered
+// mode, whose sink and tail spans need no entry); -1 after; and the count
+// the attention launch reads (n_fixed + topk).
+__device__ __forceinline__ void finish_selection(const DecodeArgs& a, int32_t* out, int t, size_t bk, int tid) {
+  const int n_loc = a.clustered ? 0 : a.n_local;
+  if (tid == 0) out[0] = 0;
+  for (int m = tid; m < n_loc; m += kDecSelThreads) out[1 + a.topk + m] = t - a.n_local + 1 + m;
+  for (int e = 1 + a.topk + n_loc + tid; e < a.kmax; e += kDecSelThreads) out[e] = -1;
+  if (tid == 0) a.cnt[bk] = a.clustered ? n_fixed(a) + a.topk : 1 + a.topk + a.n_local;
+}
+
 __global__ void __launch_bounds__(kDecSelThreads, 8) __cluster_dims__(kSelCluster, 1, 1)
     decode_select_kernel(const __grid_constant__ DecodeArgs a) {
   // dynamic: keys[chunk] | lkey[topk] | lidx[topk] | ukey[kSelCluster*topk] | uidx[kSelCluster*topk]
@@ -162,9 +183,20 @@ __global__ void __launch_bounds__(kDecSelThreads, 8) __cluster_dims__(kSelCluste
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t rank = cluster_ctarank();
   const int t = (a.cache_len - 1) / a.block;
-  const int ncand = max(0, t - a.n_local);  // candidates are blocks 1..ncand
   const size_t bk = static_cast<size_t>(b) * a.n_kv_heads + kvh;
+  // Candidates: blocks 1..t-L (candidate x is block x + 1, centroid row
+  // x + 1), or the chunks 0..n_chunks-1 of a clustered head (row x).
+  const int crow0 = a.clustered ? 0 : 1;
+  const int ncand = a.clustered ? min(max(a.n_chunks[bk], 0), a.max_chunks) : max(0, t - a.n_local);
   int32_t* out = a.sel + bk * a.kmax;
+  if (a.clustered && (ncand <= a.topk || a.topk == 0)) {  // every chunk (or none)
+    if (rank == 0) {
+      const int m = min(ncand, a.topk);
+      for (int e = tid; e < a.kmax; e += kDecSelThreads) out[e] = e == 0 ? 0 : (e <= m ? e - 1 : -1);
+      if (tid == 0) a.cnt[bk] = n_fixed(a) + m;
+    }
+    return;
+  }
   if (ncand <= a.topk) {  // every block 0..t (uniform over the cluster)
     if (rank == 0) {
       for (int e = tid; e < a.kmax; e += kDecSelThreads) out[e] = e <= t ? e : -1;
@@ -188,7 +220,7 @@ __global__ void __launch_bounds__(kDecSelThreads, 8) __cluster_dims__(kSelCluste
   uint32_t* lidx = lkey + a.topk;
   uint32_t* ukey = lidx + a.topk;
   uint32_t* uidx = ukey + kSelCluster * a.topk;
-  const float* C = a.centroids + bk * a.nbc * kRank;
+  const float* C = a.clustered ? a.chunk_centroids + bk * a.max_chunks * kRank : a.centroids + bk * a.nbc * kRank;
 
   // Loads first: this thread's first two centroid rows, its query dimension
   // of the group's heads and its row of the projector.
@@ -196,7 +228,7 @@ __global__ void __launch_bounds__(kDecSelThreads, 8) __cluster_dims__(kSelCluste
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
     const int x = min(lo + min(tid + u * kDecSelThreads, max(nl - 1, 0)), ncand - 1);  // a valid row
-    const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + 1) * kRank);
+    const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + crow0) * kRank);
 #pragma unroll
     for (int w = 0; w < 4; ++w) cv[u][w] = __ldg(c4 + w);
   }
@@ -236,14 +268,14 @@ __global__ void __launch_bounds__(kDecSelThreads, 8) __cluster_dims__(kSelCluste
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
           const int x = lo + min(x0 + tid + u * kDecSelThreads, nl - 1);
-          const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + 1) * kRank);
+          const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + crow0) * kRank);
 #pragma unroll
           for (int w = 0; w < 4; ++w) cv[u][w] = __ldg(c4 + w);
         }
       }
       const int xa = x0 + tid, xb = x0 + tid + kDecSelThreads;
-      uint64_t ka = xa < nl ? cand_key(score16(q, cv[0]), lo + xa + 1) : 0ull;
-      uint64_t kb = xb < nl ? cand_key(score16(q, cv[1]), lo + xb + 1) : 0ull;
+      uint64_t ka = xa < nl ? cand_key(score16(q, cv[0]), lo + xa + crow0) : 0ull;
+      uint64_t kb = xb < nl ? cand_key(score16(q, cv[1]), lo + xb + crow0) : 0ull;
       warp_sort2_desc(ka, kb);
       const uint64_t top = warp_merge_top32(ka, kb);
       best = x0 == 0 ? top : warp_merge_top32(best, top);
@@ -280,10 +312,7 @@ __global__ void __launch_bounds__(kDecSelThreads, 8) __cluster_dims__(kSelCluste
       const uint32_t sorted = warp_sort_asc(blk);
       if (lane < a.topk) out[1 + lane] = static_cast<int32_t>(sorted);
     }
-    if (tid == 0) out[0] = 0;
-    for (int m = tid; m < a.n_local; m += kDecSelThreads) out[1 + a.topk + m] = t - a.n_local + 1 + m;
-    for (int e = 1 + a.topk + a.n_local + tid; e < a.kmax; e += kDecSelThreads) out[e] = -1;
-    if (tid == 0) a.cnt[bk] = 1 + a.topk + a.n_local;
+    finish_selection(a, out, t, bk, tid);
     return;
   }
   // k > 32: radix select.  Scores of this CTA's slice -> order keys.
@@ -292,7 +321,7 @@ __global__ void __launch_bounds__(kDecSelThreads, 8) __cluster_dims__(kSelCluste
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int x = lo + min(x0 + tid + u * kDecSelThreads, nl - 1);
-        const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + 1) * kRank);
+        const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + crow0) * kRank);
 #pragma unroll
         for (int w = 0; w < 4; ++w) cv[u][w] = __ldg(c4 + w);
       }
@@ -308,7 +337,7 @@ __global__ void __launch_bounds__(kDecSelThreads, 8) __cluster_dims__(kSelCluste
   if (nl <= a.topk) {
     for (int x = tid; x < nl; x += kDecSelThreads) {
       lkey[x] = keys[x];
-      lidx[x] = static_cast<uint32_t>(lo + x + 1);
+      lidx[x] = static_cast<uint32_t>(lo + x + crow0);
     }
     if (tid == 0) n_kept = nl;
   } else {
@@ -316,7 +345,7 @@ __global__ void __launch_bounds__(kDecSelThreads, 8) __cluster_dims__(kSelCluste
     radix_threshold<kDecSelThreads>(keys, nl, a.topk, sh, T, need);
     ordered_select<kDecSelThreads>(keys, nl, T, need, sh, [&](int r, int x) {
       lkey[r] = keys[x];
-      lidx[r] = static_cast<uint32_t>(lo + x + 1);
+      lidx[r] = static_cast<uint32_t>(lo + x + crow0);
     });
     if (tid == 0) n_kept = a.topk;
   }
@@ -351,10 +380,7 @@ __global__ void __launch_bounds__(kDecSelThreads, 8) __cluster_dims__(kSelCluste
     radix_threshold<kDecSelThreads>(ukey, U, a.topk, sh, T, need);
     ordered_select<kDecSelThreads>(ukey, U, T, need, sh,
                                    [&](int r, int x) { out[1 + r] = static_cast<int32_t>(uidx[x]); });
-    if (tid == 0) out[0] = 0;
-    for (int m = tid; m < a.n_local; m += kDecSelThreads) out[1 + a.topk + m] = t - a.n_local + 1 + m;
-    for (int e = 1 + a.topk + a.n_local + tid; e < a.kmax; e += kDecSelThreads) out[e] = -1;
-    if (tid == 0) a.cnt[bk] = 1 + a.topk + a.n_local;
+    finish_selection(a, out, t, bk, tid);
   } else {
     cluster_sync();
   }
@@ -364,16 +390,12 @@ __global__ void __launch_bounds__(kDecSelThreads, 8) __cluster_dims__(kSelCluste
 size_t decode_select_smem(const DecodeArgs& a) {
   if (a.topk <= 32) return 0;  // static arrays suffice
   const int t = (a.cache_len - 1) / a.block;
-  const int ncand = std::max(0, t - a.n_local);
+  const int ncand = a.clustered ? a.max_chunks : std::max(0, t - a.n_local);
   const int chunk = (ncand + kSelCluster - 1) / kSelCluster;
   return (static_cast<size_t>(chunk) + 2 * static_cast<size_t>(a.topk) * (1 + kSelCluster)) * sizeof(uint32_t);
 }
 
 // ---------------------------------------------------------------- schedule
-// Block of the new token, and the number of blocks every selection keeps
-// whatever the scores: the sink and the local blocks {0} u {t-L+1..t}.
-__device__ __forceinline__ int decode_t(const DecodeArgs& a) { return (a.cache_len - 1) / a.block; }
-__device__ __forceinline__ int n_fixed(const DecodeArgs& a) { return min(decode_t(a) + 1, a.n_local + 1); }
 
 // Spans of one (sequence, head) in a list: list 0 holds a window/full head's
 // visible keys in 128-key pieces, or a retrieval head's sink and local
@@ -386,7 +408,7 @@ __device__ __forceinline__ int n_spans_in(const DecodeArgs& a, int list, int kvh
   return (len + 127) / 128;
 }
 
-// Fixed block s (0 <= s < n_fixed) of a retrieval head, ascending.
+// Fixed block s (0 <= s < n_fixed) of a retrieval head in contiguous mode, ascending.
 __device__ __forceinline__ int fixed_block(const DecodeArgs& a, int s) {
   const int t = decode_t(a);
   return (t <= a.n_local || s == 0) ? s : t - a.n_local + s;
@@ -475,7 +497,8 @@ __device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
 // retrieval spans), lanes prefetch the rows of the spans kPrefetchAhead ahead
 // into L2, and lane 0 waits for free stages and issues the loads.
 __device__ __forceinline__ void attn_producer(DecSmem& sm, const CUtensorMap* mk, const CUtensorMap* mv,
-                                              const DecodeArgs& a, volatile int* abort) {
+                                              const CUtensorMap* mks, const CUtensorMap* mvs, const DecodeArgs& a,
+                                              volatile int* abort) {
   const int lane = lane_id();
   const int tq = (a.cache_len - 1) / a.block;  // block of the new token
   uint32_t issued = 0;
@@ -497,14 +520,34 @@ __device__ __forceinline__ void attn_producer(DecSmem& sm, const CUtensorMap* mk
       const int s_end = min(s + static_cast<int>(run_end - x), cnt);
       const bool sparse = a.kind[kvh] == KIND_SPARSE;
       const int start = a.kind[kvh] == KIND_SWA ? max(0, a.cache_len - a.window) : 0;
-      const __nv_bfloat16* kbase = a.kcache + bk * static_cast<size_t>(a.cache_cap) * kHeadDim;
-      const __nv_bfloat16* vbase = a.vcache + bk * static_cast<size_t>(a.cache_cap) * kHeadDim;
+      // clustered list-1 spans come from the cluster-ordered K/V
+      const bool sorted_src = a.clustered && list == 1;
+      const __nv_bfloat16* kbase = sorted_src ? a.k_sorted + bk * static_cast<size_t>(a.clu_rows) * kHeadDim
+                                              : a.kcache + bk * static_cast<size_t>(a.cache_cap) * kHeadDim;
+      const __nv_bfloat16* vbase = sorted_src ? a.v_sorted + bk * static_cast<size_t>(a.clu_rows) * kHeadDim
+                                              : a.vcache + bk * static_cast<size_t>(a.cache_cap) * kHeadDim;
+      const int src_rows = sorted_src ? a.clu_rows : a.cache_len;
+      const CUtensorMap* tk = sorted_src ? mks : mk;
+      const CUtensorMap* tv = sorted_src ? mvs : mv;
       for (int s0 = s; s0 < s_end && ok; s0 += 32) {
         const int m = min(32, s_end - s0);
         // lane l: key range of span s0 + l
         int key0_l = 0, nk_l = 0;
         if (lane < m) {
-          if (list == 1) {
+          if (list == 1 && a.clustered) {
+            const int ch = a.sel[bk * a.kmax + 1 + s0 + lane];  // a chunk of the head's clusters
+            if (ch < 0 || ch >= min(a.n_chunks[bk], a.max_chunks)) {
+              flag_error(a.status, RTP_DEVERR_INDEX);
+            } else {
+              const size_t e = bk * a.max_chunks + ch;
+              key0_l = a.chunk_start[e];
+              nk_l = min(a.chunk_len[e], a.clu_rows - key0_l);
+              if (key0_l < 0 || nk_l < 0) {
+                flag_error(a.status, RTP_DEVERR_INDEX);
+                key0_l = nk_l = 0;
+              }
+            }
+          } else if (list == 1) {
             const int blk = a.sel[bk * a.kmax + 1 + s0 + lane];  // the sink is entry 0
             if (blk < 0 || blk > tq) {  // not a valid selection: the span contributes nothing
               flag_error(a.status, RTP_DEVERR_INDEX);
@@ -512,6 +555,10 @@ __device__ __forceinline__ void attn_producer(DecSmem& sm, const CUtensorMap* mk
               key0_l = blk * a.block;
               nk_l = min(a.block, a.cache_len - key0_l);
             }
+          } else if (sparse && a.clustered) {  // the sink block, then the unclustered tail
+            const int sp = s0 + lane;
+            key0_l = sp == 0 ? 0 : a.clu_end + 128 * (sp - 1);
+            nk_l = sp == 0 ? min(a.block, a.cache_len) : min(128, a.cache_len - key0_l);
           } else if (sparse) {
             key0_l = fixed_block(a, s0 + lane) * a.block;
             nk_l = min(a.block, a.cache_len - key0_l);
@@ -521,7 +568,7 @@ __device__ __forceinline__ void attn_producer(DecSmem& sm, const CUtensorMap* mk
           }
         }
         // rows the ring load will read: 128 from key0, within the cache
-        const uint32_t pf_bytes = static_cast<uint32_t>(max(0, min(128, a.cache_len - key0_l))) * kHeadDim * 2;
+        const uint32_t pf_bytes = static_cast<uint32_t>(max(0, min(128, src_rows - key0_l))) * kHeadDim * 2;
         auto prefetch_span = [&]() {
           if (pf_bytes > 0) {
             prefetch_l2(kbase + static_cast<size_t>(key0_l) * kHeadDim, pf_bytes);
@@ -542,12 +589,12 @@ __device__ __forceinline__ void attn_producer(DecSmem& sm, const CUtensorMap* mk
               mbar_arrive_expect_tx(&sm.k_full[st], kHalfSpanBytes);
               for (int cc = 0; cc < 2; ++cc)
                 for (int hh = 0; hh < 2; ++hh)
-                  tma_load_3d(sm.k[st] + cc * 16384 + hh * 8192, mk, &sm.k_full[st], 64 * cc, key0 + 64 * hh,
+                  tma_load_3d(sm.k[st] + cc * 16384 + hh * 8192, tk, &sm.k_full[st], 64 * cc, key0 + 64 * hh,
                               static_cast<int>(bk));
               mbar_arrive_expect_tx(&sm.v_full[st], kHalfSpanBytes);
               for (int cc = 0; cc < 2; ++cc)
                 for (int hh = 0; hh < 2; ++hh)
-                  tma_load_3d(sm.v[st] + cc * 16384 + hh * 8192, mv, &sm.v_full[st], 64 * cc, key0 + 64 * hh,
+                  tma_load_3d(sm.v[st] + cc * 16384 + hh * 8192, tv, &sm.v_full[st], 64 * cc, key0 + 64 * hh,
                               static_cast<int>(bk));
             }
           }
@@ -813,6 +860,8 @@ __device__ __forceinline__ void attn_consumer(DecSmem& sm, const DecodeArgs& a, 
 template <int NT>
 __global__ void __launch_bounds__(kAttnThreads, 2) decode_attn_kernel(const __grid_constant__ CUtensorMap mk,
                                                                        const __grid_constant__ CUtensorMap mv,
+                                                                       const __grid_constant__ CUtensorMap mks,
+                                                                       const __grid_constant__ CUtensorMap mvs,
                                                                        const __grid_constant__ DecodeArgs a) {
   extern __shared__ uint8_t dsmem[];
   DecSmem& sm = *reinterpret_cast<DecSmem*>((reinterpret_cast<uintptr_t>(dsmem) + 1023) & ~uintptr_t(1023));
@@ -834,8 +883,12 @@ __global__ void __launch_bounds__(kAttnThreads, 2) decode_attn_kernel(const __gr
     if (lane_id() == 0) {
       tma_prefetch_desc(&mk);
       tma_prefetch_desc(&mv);
+      if (a.clustered) {
+        tma_prefetch_desc(&mks);
+        tma_prefetch_desc(&mvs);
+      }
     }
-    attn_producer(sm, &mk, &mv, a, abort);
+    attn_producer(sm, &mk, &mv, &mks, &mvs, a, abort);
   } else {
     attn_consumer<NT>(sm, a, abort);
   }
@@ -960,7 +1013,8 @@ cudaError_t decode_static_scratch(void** ptr) {
   return cudaSuccess;
 }
 
-cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t stream) {
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mks,
+                          const CUtensorMap& mvs, cudaStream_t stream) {
   // All three kernels prefer the largest shared-memory carveout: an SM that
   // a selection or combine CTA has configured for little shared memory could
   // not take an attention CTA until it drains.
@@ -997,8 +1051,8 @@ cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUte
   cfg.stream = stream;
   cfg.attrs = pdl;
   cfg.numAttrs = 1;
-  e = two_tiles ? cudaLaunchKernelEx(&cfg, decode_attn_kernel<2>, mk, mv, a)
-                : cudaLaunchKernelEx(&cfg, decode_attn_kernel<1>, mk, mv, a);
+  e = two_tiles ? cudaLaunchKernelEx(&cfg, decode_attn_kernel<2>, mk, mv, mks, mvs, a)
+                : cudaLaunchKernelEx(&cfg, decode_attn_kernel<1>, mk, mv, mks, mvs, a);
   if (e != cudaSuccess) return e;
   cfg.gridDim = dim3(a.n_q_heads, a.batch);
   cfg.blockDim = dim3(kCombineThreads);

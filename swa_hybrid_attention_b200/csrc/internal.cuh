@@ -80,6 +80,18 @@ struct DecodeArgs {
   int n_ctas;
   int per_b[2];                           // spans per sequence in each list
   int span_off[2][kMaxDecodeKvHeads];     // first span of a head within its sequence's part of each list
+  // Clustered retrieval heads (k-means of the cache; 0 = contiguous blocks):
+  // a retrieval head attends to the sink block, the unclustered tail
+  // [clu_end, cache_len) (both in list 0) and the top-k chunks of its
+  // clusters (list 1), streamed from the cluster-ordered copy of K/V.
+  int clustered;
+  int clu_end, clu_rows, max_chunks;
+  const __nv_bfloat16* k_sorted;    // [batch][n_kv_heads][clu_rows][128]
+  const __nv_bfloat16* v_sorted;
+  const float* chunk_centroids;     // [batch][n_kv_heads][max_chunks][16]
+  const int32_t* chunk_start;       // [batch][n_kv_heads][max_chunks]
+  const int32_t* chunk_len;
+  const int32_t* n_chunks;          // [batch][n_kv_heads]
 };
 constexpr int kPartStride = 132;  // m, l, pad, pad, o[128]
 
@@ -98,14 +110,39 @@ struct CacheArgs {
   int n_blocks;  // centroid build: complete blocks to write
 };
 
+// k-means clustering of the projected keys of a KV cache (retrieval heads):
+// rows [block, clu_end) of each (sequence, KV head), n = clu_end - block.
+struct KmeansArgs {
+  const __nv_bfloat16* kcache;  // [batch][n_kv_heads][cache_cap][128]
+  const __nv_bfloat16* vcache;
+  const float* proj;            // [128][16]
+  float* X;                     // workspace [batch][n_kv_heads][n][16]: projected keys
+  int32_t* assign;              // workspace [batch][n_kv_heads][n]
+  float* centroids;             // [batch][n_kv_heads][nc][16]
+  int32_t* members;             // [batch][n_kv_heads][n]: key rows grouped by cluster, ascending inside
+  int32_t* offsets;             // [batch][n_kv_heads][nc + 1]
+  __nv_bfloat16* k_sorted;      // [batch][n_kv_heads][n][128]: K rows in `members` order
+  __nv_bfloat16* v_sorted;
+  float* chunk_centroids;       // [batch][n_kv_heads][max_chunks][16]
+  int32_t* chunk_start;         // [batch][n_kv_heads][max_chunks]: first row in the sorted K/V
+  int32_t* chunk_len;
+  int32_t* n_chunks;            // [batch][n_kv_heads]
+  uint8_t kind[kMaxDecodeKvHeads];
+  int batch, n_kv_heads, cache_cap, block, clu_end, n, nc, max_chunks;
+};
+constexpr int kMaxClusters = 2048;
+
 // Launchers (return the launch error, never synchronise).
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                            int num_ctas, cudaStream_t stream);
 cudaError_t launch_indexer(const IndexerArgs& a, cudaStream_t stream);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
 cudaError_t launch_select_dynamic(const SelectArgs& a, cudaStream_t stream);
-cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t stream);
+// mks / mvs: the cluster-ordered K/V of clustered mode (any valid map otherwise).
+cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mks,
+                          const CUtensorMap& mvs, cudaStream_t stream);
 cudaError_t launch_cache_append(const CacheArgs& a, cudaStream_t stream);
+cudaError_t launch_kmeans(const KmeansArgs& a, int iters, cudaStream_t stream);
 cudaError_t launch_cache_centroids(const CacheArgs& a, cudaStream_t stream);
 
 // Fixed-size device scratch used by the allocation-free decode entry point.

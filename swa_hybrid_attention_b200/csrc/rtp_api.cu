@@ -443,13 +443,17 @@ struct DecodeLayout {
 // when it is at least cache_len, else exactly cache_len.
 int decode_capacity(const rtp_attn_cfg* c, int cache_len) { return c->seq > cache_len ? c->seq : cache_len; }
 
-bool decode_layout(const rtp_attn_cfg* c, const uint8_t* kind, int cache_len, DecodeLayout& L) {
+// clu_end > 0: clustered retrieval heads (sink block + tail pieces fixed,
+// topk chunks selected).
+bool decode_layout(const rtp_attn_cfg* c, const uint8_t* kind, int cache_len, DecodeLayout& L, int clu_end = 0) {
   if (!cfg_common_ok(c) || !kind || cache_len < 1) return false;
   if (static_cast<long>(cache_len) / c->block * 4 > 200 * 1024) return false;
   if (c->n_kv_heads > kMaxDecodeKvHeads) return false;
-  L.kmax = c->topk + 1 + c->n_local;
-  const long t = (cache_len - 1) / c->block;                      // block of the new token
-  const long nfix = std::min<long>(t + 1, c->n_local + 1);       // sink + local blocks
+  if (clu_end > 0 && (clu_end % c->block != 0 || clu_end <= c->block || clu_end > cache_len)) return false;
+  const long t = (cache_len - 1) / c->block;  // block of the new token
+  const long nfix = clu_end > 0 ? 1 + (cache_len - clu_end + 127) / 128  // sink + unclustered tail
+                                : std::min<long>(t + 1, c->n_local + 1);   // sink + local blocks
+  L.kmax = clu_end > 0 ? static_cast<int>(nfix) + c->topk : c->topk + 1 + c->n_local;
   long per_b[2] = {0, 0};
   for (int h = 0; h < c->n_kv_heads; ++h) {
     if (kind[h] > RTP_HEAD_SPARSE) return false;
@@ -510,6 +514,99 @@ bool decode_schedule(const rtp_attn_cfg* c, const DecodeLayout& L, DecodeArgs& a
   return true;
 }
 
+// The arrays and sizes of a clustering description (cap = cache capacity).
+bool cluster_args_ok(const rtp_attn_cfg* c, const uint8_t* kind, const rtp_clusters* cl, int cap) {
+  if (!cfg_common_ok(c) || !kind || !cl || c->n_kv_heads > kMaxDecodeKvHeads || c->batch > 65535) return false;
+  for (int h = 0; h < c->n_kv_heads; ++h)
+    if (kind[h] > RTP_HEAD_SPARSE) return false;
+  if (cl->clu_end <= c->block || cl->clu_end % c->block != 0 || cl->clu_end > cap) return false;
+  const int n = cl->clu_end - c->block;
+  if (cl->n_clusters < 1 || cl->n_clusters > kMaxClusters || cl->n_clusters > n) return false;
+  if (!cl->centroids || !cl->members || !cl->offsets || !cl->k_sorted || !cl->v_sorted || !cl->chunk_centroids ||
+      !cl->chunk_start || !cl->chunk_len || !cl->n_chunks)
+    return false;
+  return aligned16(cl->centroids) && aligned16(cl->k_sorted) && aligned16(cl->v_sorted) &&
+         aligned16(cl->chunk_centroids);
+}
+
+// Argument checks and DecodeArgs of the decode entry points (cl: clustered
+// mode, else contiguous blocks with `centroids`).
+rtp_status prepare_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* q,
+                          const void* kcache, const void* vcache, const float* centroids, const float* proj,
+                          const rtp_clusters* cl, void* o, int32_t* sel_out, int32_t* cnt_out, DecodeLayout& L,
+                          DecodeArgs& a) {
+  if (!cfg) return RTP_ERR_INVALID_ARG;
+  if (!decode_layout(cfg, kind_host, cache_len, L, cl ? cl->clu_end : 0)) return RTP_ERR_INVALID_ARG;
+  if (!q || !kcache || !vcache || !o) return RTP_ERR_INVALID_ARG;
+  bool any_sparse = false;
+  for (int h = 0; h < cfg->n_kv_heads; ++h) any_sparse |= kind_host[h] == RTP_HEAD_SPARSE;
+  if (any_sparse && (!proj || (!cl && !centroids))) return RTP_ERR_INVALID_ARG;
+  if (cl && !cluster_args_ok(cfg, kind_host, cl, decode_capacity(cfg, cache_len))) return RTP_ERR_INVALID_ARG;
+  if ((sel_out == nullptr) != (cnt_out == nullptr)) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o)) return RTP_ERR_INVALID_ARG;
+  if ((centroids && !aligned16(centroids)) || (proj && !aligned16(proj))) return RTP_ERR_INVALID_ARG;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.kcache = static_cast<const __nv_bfloat16*>(kcache);
+  a.vcache = static_cast<const __nv_bfloat16*>(vcache);
+  a.centroids = centroids;
+  a.proj = proj;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  std::memset(a.kind, 0, sizeof(a.kind));
+  std::memcpy(a.kind, kind_host, cfg->n_kv_heads);
+  a.batch = cfg->batch;
+  a.n_q_heads = cfg->n_q_heads;
+  a.n_kv_heads = cfg->n_kv_heads;
+  a.group = cfg->n_q_heads / cfg->n_kv_heads;
+  a.cache_len = cache_len;
+  a.cache_cap = decode_capacity(cfg, cache_len);
+  a.nbc = a.cache_cap / cfg->block;
+  a.window = cfg->window;
+  a.block = cfg->block;
+  a.topk = cfg->topk;
+  a.n_local = cfg->n_local;
+  a.kmax = L.kmax;
+  a.scale_log2 = effective_scale(cfg) * kLog2e;
+  a.clustered = cl ? 1 : 0;
+  a.clu_end = cl ? cl->clu_end : 0;
+  a.clu_rows = cl ? cl->clu_end - cfg->block : 0;
+  a.max_chunks = cl ? a.clu_rows / 128 + cl->n_clusters : 0;
+  a.k_sorted = cl ? static_cast<const __nv_bfloat16*>(cl->k_sorted) : nullptr;
+  a.v_sorted = cl ? static_cast<const __nv_bfloat16*>(cl->v_sorted) : nullptr;
+  a.chunk_centroids = cl ? cl->chunk_centroids : nullptr;
+  a.chunk_start = cl ? cl->chunk_start : nullptr;
+  a.chunk_len = cl ? cl->chunk_len : nullptr;
+  a.n_chunks = cl ? cl->n_chunks : nullptr;
+  if (!decode_schedule(cfg, L, a)) return RTP_ERR_CUDA;
+  return RTP_OK;
+}
+
+// Scratch pointers, status word, TMA maps and the launch.
+rtp_status run_decode(DecodeArgs& a, const DecodeLayout& L, char* ws, int32_t* sel_out, int32_t* cnt_out,
+                      bool with_status, const rtp_clusters* cl, void* stream) {
+  a.sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(ws + L.sel_off);
+  a.cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(ws + L.cnt_off);
+  a.partial = reinterpret_cast<float*>(ws + L.part_off);
+  a.status = nullptr;
+  if (with_status) {
+    a.status = status_word(current_device());
+    if (!a.status) return RTP_ERR_NO_MEMORY;
+  }
+  const long slabs = static_cast<long>(a.batch) * a.n_kv_heads;
+  CUtensorMap mk, mv, mks, mvs;
+  if (!encode_bf16_3d(&mk, a.kcache, a.cache_len, slabs, 64, a.cache_cap) ||
+      !encode_bf16_3d(&mv, a.vcache, a.cache_len, slabs, 64, a.cache_cap))
+    return RTP_ERR_CUDA;
+  if (cl) {
+    if (!encode_bf16_3d(&mks, cl->k_sorted, a.clu_rows, slabs, 64) ||
+        !encode_bf16_3d(&mvs, cl->v_sorted, a.clu_rows, slabs, 64))
+      return RTP_ERR_CUDA;
+  } else {
+    mks = mk;
+    mvs = mv;
+  }
+  return cuda_status(launch_decode(a, mk, mv, mks, mvs, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 // Shared validation of the KV-cache maintenance calls; fills the common
 // fields of CacheArgs.
 rtp_status cache_args(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cap, const void* kcache,
@@ -547,108 +644,101 @@ size_t rtp_decode_workspace_bytes(const rtp_attn_cfg* cfg, const uint8_t* kind_h
   return L.total;
 }
 
+size_t rtp_decode_clustered_workspace_bytes(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len,
+                                            int clu_end) {
+  DecodeLayout L;
+  if (clu_end <= 0 || !decode_layout(cfg, kind_host, cache_len, L, clu_end)) return 0;
+  return L.total;
+}
+
 rtp_status rtp_sparse_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* q,
                              const void* kcache, const void* vcache, const float* centroids, const float* proj,
                              void* o, void* workspace, size_t ws_bytes, int32_t* sel_out, int32_t* cnt_out,
                              void* stream) {
   DecodeLayout L;
-  if (!decode_layout(cfg, kind_host, cache_len, L)) return RTP_ERR_INVALID_ARG;
-  if (!q || !kcache || !vcache || !o || !workspace || ws_bytes < L.total) return RTP_ERR_INVALID_ARG;
-  bool any_sparse = false;
-  for (int h = 0; h < cfg->n_kv_heads; ++h) any_sparse |= kind_host[h] == RTP_HEAD_SPARSE;
-  if (any_sparse && (!centroids || !proj)) return RTP_ERR_INVALID_ARG;
-  if ((sel_out == nullptr) != (cnt_out == nullptr)) return RTP_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o) || !aligned16(workspace))
-    return RTP_ERR_INVALID_ARG;
-  if ((centroids && !aligned16(centroids)) || (proj && !aligned16(proj))) return RTP_ERR_INVALID_ARG;
-  if (cfg->n_kv_heads > kMaxDecodeKvHeads) return RTP_ERR_INVALID_ARG;
   DecodeArgs a;
-  a.q = static_cast<const __nv_bfloat16*>(q);
-  a.kcache = static_cast<const __nv_bfloat16*>(kcache);
-  a.vcache = static_cast<const __nv_bfloat16*>(vcache);
-  a.centroids = centroids;
-  a.proj = proj;
-  a.o = static_cast<__nv_bfloat16*>(o);
-  std::memset(a.kind, 0, sizeof(a.kind));
-  std::memcpy(a.kind, kind_host, cfg->n_kv_heads);
-  char* ws = static_cast<char*>(workspace);
-  a.sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(ws + L.sel_off);
-  a.cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(ws + L.cnt_off);
-  a.partial = reinterpret_cast<float*>(ws + L.part_off);
-  a.batch = cfg->batch;
-  a.n_q_heads = cfg->n_q_heads;
-  a.n_kv_heads = cfg->n_kv_heads;
-  a.group = cfg->n_q_heads / cfg->n_kv_heads;
-  a.cache_len = cache_len;
-  a.cache_cap = decode_capacity(cfg, cache_len);
-  a.nbc = a.cache_cap / cfg->block;
-  a.window = cfg->window;
-  a.block = cfg->block;
-  a.topk = cfg->topk;
-  a.n_local = cfg->n_local;
-  a.kmax = L.kmax;
-  a.scale_log2 = effective_scale(cfg) * kLog2e;
-  if (!decode_schedule(cfg, L, a)) return RTP_ERR_CUDA;
-  a.status = status_word(current_device());
-  if (!a.status) return RTP_ERR_NO_MEMORY;
-  CUtensorMap mk, mv;
-  if (!encode_bf16_3d(&mk, kcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64, a.cache_cap) ||
-      !encode_bf16_3d(&mv, vcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64, a.cache_cap))
-    return RTP_ERR_CUDA;
-  return cuda_status(launch_decode(a, mk, mv, reinterpret_cast<cudaStream_t>(stream)));
+  rtp_status st = prepare_decode(cfg, kind_host, cache_len, q, kcache, vcache, centroids, proj, nullptr, o, sel_out,
+                                 cnt_out, L, a);
+  if (st != RTP_OK) return st;
+  if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return RTP_ERR_INVALID_ARG;
+  return run_decode(a, L, static_cast<char*>(workspace), sel_out, cnt_out, true, nullptr, stream);
+}
+
+rtp_status rtp_sparse_decode_clustered(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len,
+                                       const void* q, const void* kcache, const void* vcache, const float* proj,
+                                       const rtp_clusters* cl, void* o, void* workspace, size_t ws_bytes,
+                                       int32_t* sel_out, int32_t* cnt_out, void* stream) {
+  if (!cl) return RTP_ERR_INVALID_ARG;
+  DecodeLayout L;
+  DecodeArgs a;
+  rtp_status st =
+      prepare_decode(cfg, kind_host, cache_len, q, kcache, vcache, nullptr, proj, cl, o, sel_out, cnt_out, L, a);
+  if (st != RTP_OK) return st;
+  if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return RTP_ERR_INVALID_ARG;
+  return run_decode(a, L, static_cast<char*>(workspace), sel_out, cnt_out, true, cl, stream);
 }
 
 rtp_status rtp_sparse_decode_noalloc(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* q,
                                      const void* kcache, const void* vcache, const float* centroids,
                                      const float* proj, void* o, int32_t* sel_out, int32_t* cnt_out, void* stream) {
   DecodeLayout L;
-  if (!decode_layout(cfg, kind_host, cache_len, L)) return RTP_ERR_INVALID_ARG;
+  DecodeArgs a;
+  rtp_status st = prepare_decode(cfg, kind_host, cache_len, q, kcache, vcache, centroids, proj, nullptr, o, sel_out,
+                                 cnt_out, L, a);
+  if (st != RTP_OK) return st;
   if (L.total > kDecodeStaticScratchBytes) return RTP_ERR_INVALID_ARG;  // beyond the fixed scratch
-  if (!q || !kcache || !vcache || !o) return RTP_ERR_INVALID_ARG;
-  bool any_sparse = false;
-  for (int h = 0; h < cfg->n_kv_heads; ++h) any_sparse |= kind_host[h] == RTP_HEAD_SPARSE;
-  if (any_sparse && (!centroids || !proj)) return RTP_ERR_INVALID_ARG;
-  if ((sel_out == nullptr) != (cnt_out == nullptr)) return RTP_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(kcache) || !aligned16(vcache) || !aligned16(o)) return RTP_ERR_INVALID_ARG;
-  if ((centroids && !aligned16(centroids)) || (proj && !aligned16(proj))) return RTP_ERR_INVALID_ARG;
-  if (cfg->n_kv_heads > kMaxDecodeKvHeads) return RTP_ERR_INVALID_ARG;
   void* scratch = nullptr;
   if (decode_static_scratch(&scratch) != cudaSuccess || !scratch) return RTP_ERR_CUDA;
-  DecodeArgs a;
-  a.q = static_cast<const __nv_bfloat16*>(q);
-  a.kcache = static_cast<const __nv_bfloat16*>(kcache);
-  a.vcache = static_cast<const __nv_bfloat16*>(vcache);
-  a.centroids = centroids;
-  a.proj = proj;
-  a.o = static_cast<__nv_bfloat16*>(o);
-  std::memset(a.kind, 0, sizeof(a.kind));
-  std::memcpy(a.kind, kind_host, cfg->n_kv_heads);
-  char* ws = static_cast<char*>(scratch);
-  a.sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(ws + L.sel_off);
-  a.cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(ws + L.cnt_off);
-  a.partial = reinterpret_cast<float*>(ws + L.part_off);
-  a.batch = cfg->batch;
-  a.n_q_heads = cfg->n_q_heads;
-  a.n_kv_heads = cfg->n_kv_heads;
-  a.group = cfg->n_q_heads / cfg->n_kv_heads;
-  a.cache_len = cache_len;
-  a.cache_cap = decode_capacity(cfg, cache_len);
-  a.nbc = a.cache_cap / cfg->block;
-  a.window = cfg->window;
-  a.block = cfg->block;
-  a.topk = cfg->topk;
-  a.n_local = cfg->n_local;
-  a.kmax = L.kmax;
-  a.scale_log2 = effective_scale(cfg) * kLog2e;
-  if (!decode_schedule(cfg, L, a)) return RTP_ERR_CUDA;
-  a.status = nullptr;  // no status word: getting one may allocate
-  CUtensorMap mk, mv;
-  if (!encode_bf16_3d(&mk, kcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64, a.cache_cap) ||
-      !encode_bf16_3d(&mv, vcache, cache_len, static_cast<long>(cfg->batch) * cfg->n_kv_heads, 64, a.cache_cap))
-    return RTP_ERR_CUDA;
-  return cuda_status(launch_decode(a, mk, mv, reinterpret_cast<cudaStream_t>(stream)));
+  // no status word: getting one may allocate
+  return run_decode(a, L, static_cast<char*>(scratch), sel_out, cnt_out, false, nullptr, stream);
 }
 
+size_t rtp_cache_cluster_workspace_bytes(const rtp_attn_cfg* cfg, int clu_end) {
+  if (!cfg_common_ok(cfg) || clu_end <= cfg->block) return 0;
+  const size_t bk = static_cast<size_t>(cfg->batch) * cfg->n_kv_heads;
+  const size_t n = static_cast<size_t>(clu_end - cfg->block);
+  auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+  return up(bk * n * kRank * sizeof(float)) + up(bk * n * sizeof(int32_t));
+}
+
+rtp_status rtp_cache_cluster(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int iters, const void* kcache,
+                             const void* vcache, const float* proj, const rtp_clusters* cl, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  if (!cfg || !cl || iters < 1 || iters > 1000) return RTP_ERR_INVALID_ARG;
+  if (!cluster_args_ok(cfg, kind_host, cl, decode_capacity(cfg, cl->clu_end))) return RTP_ERR_INVALID_ARG;
+  if (!kcache || !vcache || !proj || !aligned16(kcache) || !aligned16(vcache) || !aligned16(proj))
+    return RTP_ERR_INVALID_ARG;
+  const size_t need = rtp_cache_cluster_workspace_bytes(cfg, cl->clu_end);
+  if (!workspace || ws_bytes < need || !aligned16(workspace)) return RTP_ERR_INVALID_ARG;
+  KmeansArgs a;
+  std::memset(a.kind, 0, sizeof(a.kind));
+  std::memcpy(a.kind, kind_host, cfg->n_kv_heads);
+  a.kcache = static_cast<const __nv_bfloat16*>(kcache);
+  a.vcache = static_cast<const __nv_bfloat16*>(vcache);
+  a.proj = proj;
+  a.batch = cfg->batch;
+  a.n_kv_heads = cfg->n_kv_heads;
+  a.cache_cap = decode_capacity(cfg, cl->clu_end);
+  a.block = cfg->block;
+  a.clu_end = cl->clu_end;
+  a.n = cl->clu_end - cfg->block;
+  a.nc = cl->n_clusters;
+  a.max_chunks = a.n / 128 + a.nc;
+  const size_t bk = static_cast<size_t>(cfg->batch) * cfg->n_kv_heads;
+  a.X = static_cast<float*>(workspace);
+  a.assign = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) +
+                                        (bk * a.n * kRank * sizeof(float) + 255) / 256 * 256);
+  a.centroids = cl->centroids;
+  a.members = cl->members;
+  a.offsets = cl->offsets;
+  a.k_sorted = static_cast<__nv_bfloat16*>(cl->k_sorted);
+  a.v_sorted = static_cast<__nv_bfloat16*>(cl->v_sorted);
+  a.chunk_centroids = cl->chunk_centroids;
+  a.chunk_start = cl->chunk_start;
+  a.chunk_len = cl->chunk_len;
+  a.n_chunks = cl->n_chunks;
+  return cuda_status(launch_kmeans(a, iters, reinterpret_cast<cudaStream_t>(stream)));
+}
 
 rtp_status rtp_cache_centroids(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* kcache,
                                const float* proj, float* centroids, void* stream) {

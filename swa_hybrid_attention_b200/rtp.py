@@ -40,6 +40,13 @@ class rtp_attn_cfg(ctypes.Structure):
                                             "block", "rank", "topk", "n_sink", "n_local")] + [("scale", ctypes.c_float)]
 
 
+class rtp_clusters(ctypes.Structure):
+    _fields_ = [("clu_end", ctypes.c_int), ("n_clusters", ctypes.c_int), ("centroids", ctypes.c_void_p),
+                ("members", ctypes.c_void_p), ("offsets", ctypes.c_void_p), ("k_sorted", ctypes.c_void_p),
+                ("v_sorted", ctypes.c_void_p), ("chunk_centroids", ctypes.c_void_p), ("chunk_start", ctypes.c_void_p),
+                ("chunk_len", ctypes.c_void_p), ("n_chunks", ctypes.c_void_p)]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: run `python -m swa_hybrid_attention_b200.build` "
@@ -64,6 +71,10 @@ def _load() -> ctypes.CDLL:
         "rtp_sparse_decode_noalloc": (I, [cfgp, P, I, P, P, P, P, P, P, P, P, P]),
         "rtp_cache_centroids": (I, [cfgp, P, I, P, P, P, P]),
         "rtp_cache_append": (I, [cfgp, P, I, P, P, P, P, P, P, P]),
+        "rtp_cache_cluster_workspace_bytes": (S, [cfgp, I]),
+        "rtp_cache_cluster": (I, [cfgp, P, I, P, P, P, ctypes.POINTER(rtp_clusters), P, S, P]),
+        "rtp_decode_clustered_workspace_bytes": (S, [cfgp, P, I, I]),
+        "rtp_sparse_decode_clustered": (I, [cfgp, P, I, P, P, P, P, ctypes.POINTER(rtp_clusters), P, P, S, P, P, P]),
         "rtp_last_device_status": (I, [P]),
         "rtp_selftest_bounded_wait": (I, [ctypes.c_uint, P]),
         "rtp_status_str": (ctypes.c_char_p, [I]),
@@ -81,7 +92,9 @@ EXPORTED = ("rtp_route_heads", "rtp_route_heads_range", "rtp_plan_destroy", "rtp
             "rtp_plan_sparse_heads", "rtp_plan_work_items", "rtp_indexer_project", "rtp_block_select",
             "rtp_block_select_dynamic",
             "rtp_hybrid_prefill", "rtp_decode_workspace_bytes", "rtp_sparse_decode", "rtp_sparse_decode_noalloc",
-            "rtp_cache_centroids", "rtp_cache_append", "rtp_last_device_status", "rtp_selftest_bounded_wait",
+            "rtp_cache_centroids", "rtp_cache_append", "rtp_cache_cluster_workspace_bytes", "rtp_cache_cluster",
+            "rtp_decode_clustered_workspace_bytes", "rtp_sparse_decode_clustered",
+            "rtp_last_device_status", "rtp_selftest_bounded_wait",
             "rtp_status_str", "rtp_version")
 
 
@@ -256,6 +269,96 @@ def rtp_cache_append(cfg: AttnConfig, kinds, pos: int, k_new, v_new, kcache, vca
     _check("rtp_cache_append", _lib.rtp_cache_append(ctypes.byref(c), _kinds(kinds), int(pos), _ptr(k_new),
                                                      _ptr(v_new), _ptr(kcache), _ptr(vcache), _ptr(proj),
                                                      _ptr(centroids), _stream(stream)))
+
+
+class Clusters:
+    """Device arrays of a clustered KV cache (rtp_clusters), allocated with torch."""
+
+    def __init__(self, batch: int, n_kv_heads: int, clu_end: int, n_clusters: int, block: int, device):
+        n = clu_end - block
+        self.clu_end, self.n_clusters, self.n = clu_end, n_clusters, n
+        self.max_chunks = n // 128 + n_clusters
+        i32 = dict(dtype=torch.int32, device=device)
+        self.centroids = torch.zeros(batch, n_kv_heads, n_clusters, 16, dtype=torch.float32, device=device)
+        self.members = torch.zeros(batch, n_kv_heads, n, **i32)
+        self.offsets = torch.zeros(batch, n_kv_heads, n_clusters + 1, **i32)
+        self.k_sorted = torch.zeros(batch, n_kv_heads, n, 128, dtype=torch.bfloat16, device=device)
+        self.v_sorted = torch.zeros_like(self.k_sorted)
+        self.chunk_centroids = torch.zeros(batch, n_kv_heads, self.max_chunks, 16, dtype=torch.float32,
+                                           device=device)
+        self.chunk_start = torch.zeros(batch, n_kv_heads, self.max_chunks, **i32)
+        self.chunk_len = torch.zeros(batch, n_kv_heads, self.max_chunks, **i32)
+        self.n_chunks = torch.zeros(batch, n_kv_heads, **i32)
+
+    def c(self) -> rtp_clusters:
+        return rtp_clusters(self.clu_end, self.n_clusters, _ptr(self.centroids), _ptr(self.members),
+                            _ptr(self.offsets), _ptr(self.k_sorted), _ptr(self.v_sorted), _ptr(self.chunk_centroids),
+                            _ptr(self.chunk_start), _ptr(self.chunk_len), _ptr(self.n_chunks))
+
+
+def rtp_cache_cluster_workspace_bytes(cfg: AttnConfig, clu_end: int) -> int:
+    c = cfg.c()
+    return int(_lib.rtp_cache_cluster_workspace_bytes(ctypes.byref(c), int(clu_end)))
+
+
+def rtp_cache_cluster(cfg: AttnConfig, kinds, iters: int, kcache, vcache, proj, clusters: Clusters, workspace,
+                      ws_bytes: int, stream=None) -> None:
+    c, cl = cfg.c(), clusters.c()
+    _check("rtp_cache_cluster", _lib.rtp_cache_cluster(ctypes.byref(c), _kinds(kinds), int(iters), _ptr(kcache),
+                                                       _ptr(vcache), _ptr(proj), ctypes.byref(cl), _ptr(workspace),
+                                                       int(ws_bytes), _stream(stream)))
+
+
+def rtp_decode_clustered_workspace_bytes(cfg: AttnConfig, kinds, cache_len: int, clu_end: int) -> int:
+    c = cfg.c()
+    return int(_lib.rtp_decode_clustered_workspace_bytes(ctypes.byref(c), _kinds(kinds), int(cache_len),
+                                                         int(clu_end)))
+
+
+def rtp_sparse_decode_clustered(cfg: AttnConfig, kinds, cache_len: int, q, kcache, vcache, proj, clusters: Clusters,
+                                o, workspace, ws_bytes: int, sel_out=None, cnt_out=None, stream=None) -> None:
+    c, cl = cfg.c(), clusters.c()
+    _check("rtp_sparse_decode_clustered",
+           _lib.rtp_sparse_decode_clustered(ctypes.byref(c), _kinds(kinds), int(cache_len), _ptr(q), _ptr(kcache),
+                                            _ptr(vcache), _ptr(proj), ctypes.byref(cl), _ptr(o), _ptr(workspace),
+                                            int(ws_bytes), _ptr(sel_out), _ptr(cnt_out), _stream(stream)))
+
+
+def cluster_cache(kcache, vcache, proj, kinds, *, clu_end: int, n_clusters: int, iters: int = 8, block: int = 128,
+                  stream=None) -> Clusters:
+    """k-means clustering of rows [block, clu_end) of the retrieval heads of a
+    cache [batch][n_kv_heads][capacity][128]; returns the Clusters arrays."""
+    B, H, cap = kcache.shape[0], kcache.shape[1], kcache.shape[2]
+    cfg = AttnConfig(B, cap, H, H, 1, block, 0, 1)
+    cl = Clusters(B, H, clu_end, n_clusters, block, kcache.device)
+    ws_bytes = rtp_cache_cluster_workspace_bytes(cfg, clu_end)
+    if ws_bytes == 0:
+        raise RtpError("rtp_cache_cluster_workspace_bytes", RTP_ERR_INVALID_ARG)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=kcache.device)
+    rtp_cache_cluster(cfg, kinds, iters, kcache, vcache, proj, cl, ws, ws_bytes, stream)
+    return cl
+
+
+def sparse_decode_clustered_step(q, kcache, vcache, proj, kinds, clusters: Clusters, *, window: int,
+                                 block: int = 128, topk: int = 32, scale: float = 0.0, cache_len: int | None = None,
+                                 stream=None, return_selection: bool = False):
+    """One decode step with clustered retrieval heads; returns o (and (sel, cnt))."""
+    B, Hq = q.shape[0], q.shape[1]
+    Hkv, cap = kcache.shape[1], kcache.shape[2]
+    Lc = cap if cache_len is None else int(cache_len)
+    cfg = AttnConfig(B, cap, Hq, Hkv, window, block, topk, 1, scale)
+    ws_bytes = rtp_decode_clustered_workspace_bytes(cfg, kinds, Lc, clusters.clu_end)
+    if ws_bytes == 0:
+        raise RtpError("rtp_decode_clustered_workspace_bytes", RTP_ERR_INVALID_ARG)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    o = torch.empty_like(q)
+    sel = cnt = None
+    if return_selection:
+        kmax = 1 + (Lc - clusters.clu_end + 127) // 128 + topk
+        sel = torch.full((B, Hkv, kmax), -1, dtype=torch.int32, device=q.device)
+        cnt = torch.zeros(B, Hkv, dtype=torch.int32, device=q.device)
+    rtp_sparse_decode_clustered(cfg, kinds, Lc, q, kcache, vcache, proj, clusters, o, ws, ws_bytes, sel, cnt, stream)
+    return (o, sel, cnt) if return_selection else o
 
 
 def rtp_last_device_status(stream=None) -> int:

@@ -124,3 +124,43 @@ def test_cache_calls_validate_before_launch(rtp):
     bad = rtp.AttnConfig(2, 1024, 8, 2, 256, 96, 4, 2).c()
     assert lib.rtp_cache_centroids(ctypes.byref(bad), kinds, 512, fake, fake, fake, None) == inv
     assert lib.rtp_cache_centroids(ctypes.byref(c), kinds, 512, None, fake, fake, None) == inv
+
+
+def test_library_has_no_unresolved_internal_symbols(rtp):
+    """Every kernel source is linked in (a missing one would leave rtp:: symbols undefined)."""
+    import subprocess
+
+    out = subprocess.run(["nm", "-D", "--undefined-only", rtp.LIB_PATH], capture_output=True, text=True).stdout
+    assert "_ZN3rtp" not in out
+
+
+def test_cluster_calls_validate_before_launch(rtp):
+    cfg = rtp.AttnConfig(2, 4096, 8, 2, 256, 128, 4, 2)
+    c = cfg.c()
+    lib = rtp._lib
+    fake = 1 << 20
+    inv = rtp.RTP_ERR_INVALID_ARG
+    good = dict(clu_end=2048, n_clusters=16)
+    ptrs = [fake] * 9
+
+    def cl(**kw):
+        d = dict(good, **kw)
+        return rtp.rtp_clusters(d["clu_end"], d["n_clusters"], *ptrs)
+
+    kinds = rtp._kinds([2, 0])
+    ws = rtp.rtp_cache_cluster_workspace_bytes(cfg, 2048)
+    assert ws == ((2 * 2 * 1920 * 16 * 4 + 255) // 256 * 256) + ((2 * 2 * 1920 * 4 + 255) // 256 * 256)
+    for bad in (dict(clu_end=128), dict(clu_end=2000), dict(clu_end=8192), dict(n_clusters=0),
+                dict(n_clusters=4096)):
+        x = cl(**bad)
+        assert lib.rtp_cache_cluster(ctypes.byref(c), kinds, 4, fake, fake, fake, ctypes.byref(x), fake, ws,
+                                     None) == inv, bad
+    x = cl()
+    assert lib.rtp_cache_cluster(ctypes.byref(c), kinds, 0, fake, fake, fake, ctypes.byref(x), fake, ws, None) == inv
+    assert lib.rtp_cache_cluster(ctypes.byref(c), kinds, 4, fake, fake, fake, ctypes.byref(x), fake, ws - 1,
+                                 None) == inv
+    # clustered decode: clustered rows beyond the cache, or a null clustering
+    assert rtp.rtp_decode_clustered_workspace_bytes(cfg, [2, 0], 1024, 2048) == 0
+    assert rtp.rtp_decode_clustered_workspace_bytes(cfg, [2, 0], 3000, 2048) > 0
+    assert lib.rtp_sparse_decode_clustered(ctypes.byref(c), kinds, 3000, fake, fake, fake, fake, None, fake, fake,
+                                           1 << 30, None, None, None) == inv
