@@ -19,7 +19,8 @@
 // Kernels (retrieval heads only; CTAs of other heads leave at once):
 //   km_project    one thread per key: X = P^T k (fixed order over d)
 //   km_seed       the evenly spaced seeds
-//   km_assign     one thread per key, the centroids in shared memory
+//   km_assign     four keys per thread against every centroid, the centroids
+//                 in shared memory
 //   km_group      one CTA of 1024 threads per (sequence, head): cluster sizes,
 //                 offsets (scan), stable placement of the keys (one warp,
 //                 32 keys per step with match_any), and the new centroids
@@ -83,6 +84,10 @@ __global__ void __launch_bounds__(kKmThreads) km_seed_kernel(const KmeansArgs a)
   }
 }
 
+// Keys per thread in km_assign: every centroid read from shared memory
+// serves this many keys (the loop is bound by shared-memory loads otherwise).
+constexpr int kAssignKeys = 4;
+
 __global__ void __launch_bounds__(kKmThreads) km_assign_kernel(const KmeansArgs a) {
   extern __shared__ float4 mu4[];  // [nc][4] centroids, then [nc] squared norms
   if (a.kind[blockIdx.y] != KIND_SPARSE) return;
@@ -104,39 +109,51 @@ __global__ void __launch_bounds__(kKmThreads) km_assign_kernel(const KmeansArgs 
     nrm[c] = s;
   }
   __syncthreads();
-  const int j = blockIdx.x * kKmThreads + threadIdx.x;
-  if (j >= a.n) return;
-  float x[kRank];
-  {
+  // keys j0 + u * kKmThreads, u < kAssignKeys (coalesced over the CTA)
+  const int j0 = blockIdx.x * kKmThreads * kAssignKeys + threadIdx.x;
+  float x[kAssignKeys][kRank];
+#pragma unroll
+  for (int u = 0; u < kAssignKeys; ++u) {
+    const int j = min(j0 + u * kKmThreads, a.n - 1);
     const float4* xr = reinterpret_cast<const float4*>(a.X + (bk * a.n + j) * kRank);
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       const float4 v = xr[w];
-      x[4 * w] = v.x;
-      x[4 * w + 1] = v.y;
-      x[4 * w + 2] = v.z;
-      x[4 * w + 3] = v.w;
+      x[u][4 * w] = v.x;
+      x[u][4 * w + 1] = v.y;
+      x[u][4 * w + 2] = v.z;
+      x[u][4 * w + 3] = v.w;
     }
   }
-  float best = INFINITY;
-  int bc = 0;
-  for (int c = 0; c < a.nc; ++c) {
-    float dot = 0.f;
+  float best[kAssignKeys];
+  int bc[kAssignKeys];
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      const float4 m = mu4[4 * c + w];
-      dot = fmaf(x[4 * w], m.x, dot);
-      dot = fmaf(x[4 * w + 1], m.y, dot);
-      dot = fmaf(x[4 * w + 2], m.z, dot);
-      dot = fmaf(x[4 * w + 3], m.w, dot);
-    }
-    const float dist = fmaf(-2.f, dot, nrm[c]);
-    if (dist < best) {
-      best = dist;
-      bc = c;
+  for (int u = 0; u < kAssignKeys; ++u) {
+    best[u] = INFINITY;
+    bc[u] = 0;
+  }
+  for (int c = 0; c < a.nc; ++c) {
+    const float4 m0 = mu4[4 * c], m1 = mu4[4 * c + 1], m2 = mu4[4 * c + 2], m3 = mu4[4 * c + 3];
+    const float nc2 = nrm[c];
+    const float m[kRank] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w,
+                            m2.x, m2.y, m2.z, m2.w, m3.x, m3.y, m3.z, m3.w};
+#pragma unroll
+    for (int u = 0; u < kAssignKeys; ++u) {
+      float dot = 0.f;
+#pragma unroll
+      for (int d = 0; d < kRank; ++d) dot = fmaf(x[u][d], m[d], dot);
+      const float dist = fmaf(-2.f, dot, nc2);
+      if (dist < best[u]) {
+        best[u] = dist;
+        bc[u] = c;
+      }
     }
   }
-  a.assign[bk * a.n + j] = bc;
+#pragma unroll
+  for (int u = 0; u < kAssignKeys; ++u) {
+    const int j = j0 + u * kKmThreads;
+    if (j < a.n) a.assign[bk * a.n + j] = bc[u];
+  }
 }
 
 // Exclusive scan of v over the CTA (kGroupThreads threads, thread order).
@@ -288,6 +305,7 @@ __global__ void __launch_bounds__(kKmThreads) km_permute_kernel(const KmeansArgs
 
 cudaError_t launch_kmeans(const KmeansArgs& a, int iters, cudaStream_t stream) {
   const dim3 per_key((a.n + kKmThreads - 1) / kKmThreads, a.n_kv_heads, a.batch);
+  const dim3 per_keys((a.n + kKmThreads * kAssignKeys - 1) / (kKmThreads * kAssignKeys), a.n_kv_heads, a.batch);
   const dim3 per_head(1, a.n_kv_heads, a.batch);
   km_project_kernel<<<per_key, kKmThreads, 0, stream>>>(a);
   km_seed_kernel<<<per_head, kKmThreads, 0, stream>>>(a);
@@ -298,7 +316,7 @@ cudaError_t launch_kmeans(const KmeansArgs& a, int iters, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
   }
   for (int it = 0; it < iters; ++it) {
-    km_assign_kernel<<<per_key, kKmThreads, smem, stream>>>(a);
+    km_assign_kernel<<<per_keys, kKmThreads, smem, stream>>>(a);
     km_group_kernel<<<per_head, kGroupThreads, 0, stream>>>(a);
   }
   km_chunks_kernel<<<per_head, kGroupThreads, 0, stream>>>(a);
