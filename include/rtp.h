@@ -232,6 +232,40 @@ rtp_status rtp_hybrid_prefill(const rtp_plan* plan, const void* q, const void* k
                               const int32_t* sel, const int32_t* sel_cnt, void* o, void* stream);
 
 /* ------------------------------------------------------------------------
+ * rtp_hybrid_prefill_host — the prefill of one layer whose Q, K, V and O are
+ * in host memory (a serving engine's view of a request).  The layer is cut
+ * into n_chunks runs of query rows (whole 128-row tiles); chunk c's Q, K and
+ * V rows go to the device on an upload stream, its indexer, selection and
+ * attention run on `stream` as soon as they have arrived (the attention of
+ * rows [begin, end) only reads K/V rows < end, all of them uploaded by then),
+ * and its O rows return on a download stream: uploads, kernels and
+ * downloads of different chunks overlap.  The result equals rtp_route_heads
+ * + rtp_indexer_project + rtp_block_select + rtp_hybrid_prefill on the same
+ * data, bit for bit (each tile is computed the same way).
+ *   rtp_pipeline_create  plans the chunks (one ranged plan each; uploads
+ *       them on `stream` and synchronises it, like rtp_route_heads)
+ *   q_host, k_host, v_host, o_host  HOST bf16 [batch][heads][seq][128];
+ *       page-locked memory lets the copies run asynchronously (other host
+ *       memory works, with copies that block)
+ *   proj       DEVICE fp32 [128][16]
+ *   q_dev .. o_dev  DEVICE staging of the same shapes
+ *   centroids, qbar, sel, sel_cnt  DEVICE, as for rtp_block_select (may be
+ *       NULL without retrieval heads)
+ * The call returns once everything is queued; `stream` completes after the
+ * last O rows have reached o_host.
+ * Errors: RTP_ERR_INVALID_ARG (bad cfg, chunk count, NULL or unaligned
+ * pointer), RTP_ERR_NO_MEMORY, RTP_ERR_CUDA.
+ * ---------------------------------------------------------------------- */
+typedef struct rtp_pipeline rtp_pipeline; /* opaque, library-owned */
+rtp_status rtp_pipeline_create(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int n_chunks, void* stream,
+                               rtp_pipeline** out);
+void rtp_pipeline_destroy(rtp_pipeline* pipeline);
+rtp_status rtp_hybrid_prefill_host(rtp_pipeline* pipeline, const void* q_host, const void* k_host, const void* v_host,
+                                   const float* proj, void* o_host, void* q_dev, void* k_dev, void* v_dev,
+                                   void* o_dev, float* centroids, float* qbar, int32_t* sel, int32_t* sel_cnt,
+                                   void* stream);
+
+/* ------------------------------------------------------------------------
  * rtp_sparse_decode — one decode step (one new token per sequence) over a
  * KV cache (RTPurboV2 page: retrieval heads are sparsified in decode; the
  * streaming heads keep a window).  The new token's K/V are already the last

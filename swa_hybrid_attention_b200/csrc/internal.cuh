@@ -22,6 +22,7 @@ struct PrefillArgs {
   __nv_bfloat16* o;    // [batch][n_q_heads][q_rows][128]
   int batch, seq, n_q_heads, n_kv_heads, group, n_sparse;
   int q_row0, q_rows;  // Q/O arrays hold query rows q_row0 .. q_row0 + q_rows - 1
+  int q_slab;          // rows between consecutive (sequence, head) slabs of Q/O (>= q_rows)
   int window, block, kmax, nqb;
   float scale_log2;  // softmax scale * log2(e)
   uint32_t* status;
@@ -35,7 +36,8 @@ struct IndexerArgs {
   float* qbar;       // [batch][n_sparse][nb][16]
   const int32_t* slot_heads;  // device [n_sparse] -> kv head
   int batch, seq, n_q_heads, n_kv_heads, group, n_sparse, block;
-  int blk0, rows;  // q/k arrays hold rows blk0*block .. + rows - 1 (outputs use the whole-sequence index)
+  int blk0, rows;  // q/k arrays start at row blk0*block; `rows` = rows between consecutive slabs
+                   // (outputs use the whole-sequence block index)
   int n_blocks;    // blocks to process, starting at blk0
 };
 

@@ -521,7 +521,7 @@ __device__ __noinline__ void run_softmax(Smem& s, uint32_t tmem, int h, const Pr
     const float inv = l > 0.f ? 1.f / l : 0.f;
     const int hq = item.kvh * a.group + 2 * item.pair + h;
     __nv_bfloat16* orow =
-        a.o + ((static_cast<size_t>(item.b) * a.n_q_heads + hq) * static_cast<size_t>(a.q_rows) + (i - a.q_row0)) *
+        a.o + ((static_cast<size_t>(item.b) * a.n_q_heads + hq) * static_cast<size_t>(a.q_slab) + (i - a.q_row0)) *
                   kHeadDim;
     const bool valid = i - a.q_row0 < a.q_rows;
 #pragma unroll 1

@@ -18,6 +18,18 @@
 
 using namespace rtp;
 
+struct rtp_plan;
+struct rtp_pipeline {
+  rtp_attn_cfg cfg;
+  int device = 0;
+  int n_sparse = 0;
+  std::vector<rtp_plan*> plans;  // one ranged plan per chunk of query rows
+  std::vector<int> begin, end;
+  cudaStream_t s_in = nullptr, s_out = nullptr;  // uploads, downloads
+  std::vector<cudaEvent_t> ev_in, ev_out;
+  cudaEvent_t ev_start = nullptr, ev_done = nullptr;
+};
+
 struct rtp_plan {
   rtp_attn_cfg cfg;
   int device = 0;
@@ -159,6 +171,77 @@ int current_device() {
   return d;
 }
 
+// The indexer of a (possibly ranged) plan; q and k point at the plan's first
+// row of slab 0 and consecutive (sequence, head) slabs are slab_rows apart.
+rtp_status indexer_run(const rtp_plan* plan, const void* q, const void* k, int slab_rows, const float* proj,
+                       float* centroids, float* qbar, void* stream) {
+  if (plan->n_sparse == 0) return RTP_OK;
+  if (!q || !k || !proj || !centroids || !qbar) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(proj) || !aligned16(centroids) || !aligned16(qbar))
+    return RTP_ERR_INVALID_ARG;
+  const rtp_attn_cfg& c = plan->cfg;
+  IndexerArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.proj = proj;
+  a.centroids = centroids;
+  a.qbar = qbar;
+  a.slot_heads = plan->d_slot_heads;
+  a.batch = c.batch;
+  a.seq = c.seq;
+  a.n_q_heads = c.n_q_heads;
+  a.n_kv_heads = c.n_kv_heads;
+  a.group = c.n_q_heads / c.n_kv_heads;
+  a.n_sparse = plan->n_sparse;
+  a.block = c.block;
+  a.blk0 = plan->q_begin / c.block;
+  a.rows = slab_rows;
+  a.n_blocks = plan->q_end / c.block - a.blk0;
+  return cuda_status(launch_indexer(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// The prefill of a (possibly ranged) plan.  q and o point at the plan's first
+// query row of slab 0, their slabs q_slab rows apart; k and v start at row 0,
+// their slabs kv_slab rows apart.
+rtp_status prefill_run(const rtp_plan* plan, const void* q, int q_slab, const void* k, const void* v, int kv_slab,
+                       const int32_t* sel, const int32_t* sel_cnt, void* o, void* stream) {
+  if (!q || !k || !v || !o) return RTP_ERR_INVALID_ARG;
+  if (plan->n_sparse > 0 && (!sel || !sel_cnt)) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RTP_ERR_INVALID_ARG;
+  if (sel && !aligned16(sel)) return RTP_ERR_INVALID_ARG;
+  const rtp_attn_cfg& c = plan->cfg;
+  if (current_device() != plan->device) return RTP_ERR_INVALID_ARG;
+  CUtensorMap mq, mk, mv;
+  const int q_rows = plan->q_end - plan->q_begin;
+  if (!encode_bf16_3d(&mq, q, q_rows, static_cast<long>(c.batch) * c.n_q_heads, 128, q_slab) ||
+      !encode_bf16_3d(&mk, k, plan->q_end, static_cast<long>(c.batch) * c.n_kv_heads, 64, kv_slab) ||
+      !encode_bf16_3d(&mv, v, plan->q_end, static_cast<long>(c.batch) * c.n_kv_heads, 64, kv_slab))
+    return RTP_ERR_CUDA;
+  PrefillArgs a;
+  a.items = plan->d_items;
+  a.n_items = plan->n_items;
+  a.sel = sel;
+  a.cnt = sel_cnt;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.batch = c.batch;
+  a.seq = c.seq;
+  a.q_row0 = plan->q_begin;
+  a.q_rows = q_rows;
+  a.q_slab = q_slab;
+  a.n_q_heads = c.n_q_heads;
+  a.n_kv_heads = c.n_kv_heads;
+  a.group = c.n_q_heads / c.n_kv_heads;
+  a.n_sparse = plan->n_sparse;
+  a.window = c.window;
+  a.block = c.block;
+  a.kmax = c.topk + 1 + c.n_local;
+  a.nqb = plan->nqb;
+  a.scale_log2 = plan->scale * kLog2e;
+  a.status = status_word(plan->device);
+  const int ctas = static_cast<int>(std::min<long>(plan->n_items, plan->num_sms));
+  if (ctas <= 0) return RTP_OK;
+  return cuda_status(launch_prefill(a, mq, mk, mv, ctas, reinterpret_cast<cudaStream_t>(stream)));
+}
 }  // namespace
 
 extern "C" {
@@ -307,30 +390,9 @@ rtp_status rtp_plan_work_items(const rtp_plan* plan, int32_t* items_host) {
 rtp_status rtp_indexer_project(const rtp_plan* plan, const void* q, const void* k, const float* proj,
                                float* centroids, float* qbar, void* stream) {
   if (!plan) return RTP_ERR_INVALID_ARG;
-  if (plan->n_sparse == 0) return RTP_OK;
-  if (!q || !k || !proj || !centroids || !qbar) return RTP_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(proj) || !aligned16(centroids) || !aligned16(qbar))
-    return RTP_ERR_INVALID_ARG;
-  const rtp_attn_cfg& c = plan->cfg;
-  IndexerArgs a;
-  a.q = static_cast<const __nv_bfloat16*>(q);
-  a.k = static_cast<const __nv_bfloat16*>(k);
-  a.proj = proj;
-  a.centroids = centroids;
-  a.qbar = qbar;
-  a.slot_heads = plan->d_slot_heads;
-  a.batch = c.batch;
-  a.seq = c.seq;
-  a.n_q_heads = c.n_q_heads;
-  a.n_kv_heads = c.n_kv_heads;
-  a.group = c.n_q_heads / c.n_kv_heads;
-  a.n_sparse = plan->n_sparse;
-  a.block = c.block;
-  a.blk0 = plan->q_begin / c.block;
-  a.rows = plan->q_end - plan->q_begin;
-  a.n_blocks = plan->q_end / c.block - a.blk0;
-  return cuda_status(launch_indexer(a, reinterpret_cast<cudaStream_t>(stream)));
+  return indexer_run(plan, q, k, plan->q_end - plan->q_begin, proj, centroids, qbar, stream);
 }
+
 
 rtp_status rtp_block_select(const rtp_plan* plan, const float* qbar, const float* centroids, int32_t* sel,
                             int32_t* sel_cnt, void* stream) {
@@ -388,42 +450,10 @@ rtp_status rtp_block_select_dynamic(const rtp_plan* plan, const float* qbar, con
 
 rtp_status rtp_hybrid_prefill(const rtp_plan* plan, const void* q, const void* k, const void* v,
                               const int32_t* sel, const int32_t* sel_cnt, void* o, void* stream) {
-  if (!plan || !q || !k || !v || !o) return RTP_ERR_INVALID_ARG;
-  if (plan->n_sparse > 0 && (!sel || !sel_cnt)) return RTP_ERR_INVALID_ARG;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RTP_ERR_INVALID_ARG;
-  if (sel && !aligned16(sel)) return RTP_ERR_INVALID_ARG;
-  const rtp_attn_cfg& c = plan->cfg;
-  if (current_device() != plan->device) return RTP_ERR_INVALID_ARG;
-  CUtensorMap mq, mk, mv;
-  const int q_rows = plan->q_end - plan->q_begin;
-  if (!encode_bf16_3d(&mq, q, q_rows, static_cast<long>(c.batch) * c.n_q_heads, 128) ||
-      !encode_bf16_3d(&mk, k, plan->q_end, static_cast<long>(c.batch) * c.n_kv_heads, 64) ||
-      !encode_bf16_3d(&mv, v, plan->q_end, static_cast<long>(c.batch) * c.n_kv_heads, 64))
-    return RTP_ERR_CUDA;
-  PrefillArgs a;
-  a.items = plan->d_items;
-  a.n_items = plan->n_items;
-  a.sel = sel;
-  a.cnt = sel_cnt;
-  a.o = static_cast<__nv_bfloat16*>(o);
-  a.batch = c.batch;
-  a.seq = c.seq;
-  a.q_row0 = plan->q_begin;
-  a.q_rows = q_rows;
-  a.n_q_heads = c.n_q_heads;
-  a.n_kv_heads = c.n_kv_heads;
-  a.group = c.n_q_heads / c.n_kv_heads;
-  a.n_sparse = plan->n_sparse;
-  a.window = c.window;
-  a.block = c.block;
-  a.kmax = c.topk + 1 + c.n_local;
-  a.nqb = plan->nqb;
-  a.scale_log2 = plan->scale * kLog2e;
-  a.status = status_word(plan->device);
-  const int ctas = static_cast<int>(std::min<long>(plan->n_items, plan->num_sms));
-  if (ctas <= 0) return RTP_OK;
-  return cuda_status(launch_prefill(a, mq, mk, mv, ctas, reinterpret_cast<cudaStream_t>(stream)));
+  if (!plan) return RTP_ERR_INVALID_ARG;
+  return prefill_run(plan, q, plan->q_end - plan->q_begin, k, v, plan->q_end, sel, sel_cnt, o, stream);
 }
+
 
 // Decode workspace: sel [batch][n_kv][kmax] int32 | cnt [batch][n_kv] int32 |
 // partials [spans of both lists][group][132] fp32, each 256-byte aligned.
@@ -764,6 +794,114 @@ rtp_status rtp_cache_append(const rtp_attn_cfg* cfg, const uint8_t* kind_host, i
   a.vcache = static_cast<__nv_bfloat16*>(vcache);
   a.pos = pos;
   return cuda_status(launch_cache_append(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// ------------------------------------------------------- host pipeline
+rtp_status rtp_pipeline_create(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int n_chunks, void* stream,
+                               rtp_pipeline** out) {
+  if (!out) return RTP_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg_prefill_ok(cfg) || !kind_host || n_chunks < 1 || n_chunks > 1024) return RTP_ERR_INVALID_ARG;
+  const int tiles = (cfg->seq + 127) / 128;
+  if (tiles < n_chunks) return RTP_ERR_INVALID_ARG;
+  rtp_pipeline* pl = new (std::nothrow) rtp_pipeline();
+  if (!pl) return RTP_ERR_NO_MEMORY;
+  pl->cfg = *cfg;
+  pl->device = current_device();
+  auto fail = [&](rtp_status st) {
+    rtp_pipeline_destroy(pl);
+    return st;
+  };
+  for (int c = 0; c < n_chunks; ++c) {
+    const int b = 128 * static_cast<int>(static_cast<long>(c) * tiles / n_chunks);
+    const int e = std::min(cfg->seq, 128 * static_cast<int>(static_cast<long>(c + 1) * tiles / n_chunks));
+    rtp_plan* p = nullptr;
+    const rtp_status st = rtp_route_heads_range(cfg, kind_host, b, e, stream, &p);
+    if (st != RTP_OK) return fail(st);
+    pl->plans.push_back(p);
+    pl->begin.push_back(b);
+    pl->end.push_back(e);
+  }
+  pl->n_sparse = pl->plans[0]->n_sparse;
+  if (cudaStreamCreateWithFlags(&pl->s_in, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&pl->s_out, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&pl->ev_start, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&pl->ev_done, cudaEventDisableTiming) != cudaSuccess)
+    return fail(RTP_ERR_CUDA);
+  pl->ev_in.assign(n_chunks, nullptr);
+  pl->ev_out.assign(n_chunks, nullptr);
+  for (int c = 0; c < n_chunks; ++c)
+    if (cudaEventCreateWithFlags(&pl->ev_in[c], cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&pl->ev_out[c], cudaEventDisableTiming) != cudaSuccess)
+      return fail(RTP_ERR_CUDA);
+  *out = pl;
+  return RTP_OK;
+}
+
+void rtp_pipeline_destroy(rtp_pipeline* pl) {
+  if (!pl) return;
+  for (rtp_plan* p : pl->plans) rtp_plan_destroy(p);
+  for (cudaEvent_t e : pl->ev_in)
+    if (e) cudaEventDestroy(e);
+  for (cudaEvent_t e : pl->ev_out)
+    if (e) cudaEventDestroy(e);
+  if (pl->ev_start) cudaEventDestroy(pl->ev_start);
+  if (pl->ev_done) cudaEventDestroy(pl->ev_done);
+  if (pl->s_in) cudaStreamDestroy(pl->s_in);
+  if (pl->s_out) cudaStreamDestroy(pl->s_out);
+  delete pl;
+}
+
+rtp_status rtp_hybrid_prefill_host(rtp_pipeline* pl, const void* q_host, const void* k_host, const void* v_host,
+                                   const float* proj, void* o_host, void* q_dev, void* k_dev, void* v_dev,
+                                   void* o_dev, float* centroids, float* qbar, int32_t* sel, int32_t* sel_cnt,
+                                   void* stream) {
+  if (!pl || !q_host || !k_host || !v_host || !o_host || !q_dev || !k_dev || !v_dev || !o_dev)
+    return RTP_ERR_INVALID_ARG;
+  if (pl->n_sparse > 0 && (!proj || !centroids || !qbar || !sel || !sel_cnt)) return RTP_ERR_INVALID_ARG;
+  if (current_device() != pl->device) return RTP_ERR_INVALID_ARG;
+  const rtp_attn_cfg& c = pl->cfg;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t row = kHeadDim * sizeof(__nv_bfloat16);
+  const size_t pitch = static_cast<size_t>(c.seq) * row;
+  const size_t q_slabs = static_cast<size_t>(c.batch) * c.n_q_heads, kv_slabs = static_cast<size_t>(c.batch) * c.n_kv_heads;
+  auto at = [&](const void* base, int r) { return static_cast<const char*>(base) + static_cast<size_t>(r) * row; };
+  auto atw = [&](void* base, int r) { return static_cast<char*>(base) + static_cast<size_t>(r) * row; };
+  // The copy streams start after the work already queued on `stream`.
+  if (cudaEventRecord(pl->ev_start, s) != cudaSuccess || cudaStreamWaitEvent(pl->s_in, pl->ev_start) != cudaSuccess ||
+      cudaStreamWaitEvent(pl->s_out, pl->ev_start) != cudaSuccess)
+    return RTP_ERR_CUDA;
+  for (size_t ci = 0; ci < pl->plans.size(); ++ci) {
+    const rtp_plan* p = pl->plans[ci];
+    const int b = pl->begin[ci], e = pl->end[ci];
+    const size_t width = static_cast<size_t>(e - b) * row;
+    // 1. this chunk's Q, K and V rows (every slab) to the device
+    if (cudaMemcpy2DAsync(atw(q_dev, b), pitch, at(q_host, b), pitch, width, q_slabs, cudaMemcpyHostToDevice,
+                          pl->s_in) != cudaSuccess ||
+        cudaMemcpy2DAsync(atw(k_dev, b), pitch, at(k_host, b), pitch, width, kv_slabs, cudaMemcpyHostToDevice,
+                          pl->s_in) != cudaSuccess ||
+        cudaMemcpy2DAsync(atw(v_dev, b), pitch, at(v_host, b), pitch, width, kv_slabs, cudaMemcpyHostToDevice,
+                          pl->s_in) != cudaSuccess ||
+        cudaEventRecord(pl->ev_in[ci], pl->s_in) != cudaSuccess || cudaStreamWaitEvent(s, pl->ev_in[ci]) != cudaSuccess)
+      return RTP_ERR_CUDA;
+    // 2. its kernels: every earlier row is already on the device
+    rtp_status st = RTP_OK;
+    if (pl->n_sparse > 0) {
+      st = indexer_run(p, atw(q_dev, b), atw(k_dev, b), c.seq, proj, centroids, qbar, stream);
+      if (st == RTP_OK) st = rtp_block_select(p, qbar, centroids, sel, sel_cnt, stream);
+    }
+    if (st == RTP_OK) st = prefill_run(p, atw(q_dev, b), c.seq, k_dev, v_dev, c.seq, sel, sel_cnt, atw(o_dev, b), stream);
+    if (st != RTP_OK) return st;
+    // 3. its O rows back to the host
+    if (cudaEventRecord(pl->ev_out[ci], s) != cudaSuccess || cudaStreamWaitEvent(pl->s_out, pl->ev_out[ci]) != cudaSuccess ||
+        cudaMemcpy2DAsync(atw(o_host, b), pitch, at(o_dev, b), pitch, width, q_slabs, cudaMemcpyDeviceToHost,
+                          pl->s_out) != cudaSuccess)
+      return RTP_ERR_CUDA;
+  }
+  // `stream` completes when the last download does
+  if (cudaEventRecord(pl->ev_done, pl->s_out) != cudaSuccess || cudaStreamWaitEvent(s, pl->ev_done) != cudaSuccess)
+    return RTP_ERR_CUDA;
+  return RTP_OK;
 }
 
 rtp_status rtp_selftest_bounded_wait(unsigned limit_ms, void* stream) {

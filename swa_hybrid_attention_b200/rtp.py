@@ -66,6 +66,9 @@ def _load() -> ctypes.CDLL:
         "rtp_block_select": (I, [P, P, P, P, P, P]),
         "rtp_block_select_dynamic": (I, [P, P, P, ctypes.c_float, I, ctypes.c_float, P, P, P]),
         "rtp_hybrid_prefill": (I, [P, P, P, P, P, P, P, P]),
+        "rtp_pipeline_create": (I, [cfgp, P, I, P, ctypes.POINTER(P)]),
+        "rtp_pipeline_destroy": (None, [P]),
+        "rtp_hybrid_prefill_host": (I, [P] * 15),
         "rtp_decode_workspace_bytes": (S, [cfgp, P, I]),
         "rtp_sparse_decode": (I, [cfgp, P, I, P, P, P, P, P, P, P, S, P, P, P]),
         "rtp_sparse_decode_noalloc": (I, [cfgp, P, I, P, P, P, P, P, P, P, P, P]),
@@ -90,7 +93,7 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 EXPORTED = ("rtp_route_heads", "rtp_route_heads_range", "rtp_plan_destroy", "rtp_plan_num_sparse", "rtp_plan_num_items",
             "rtp_plan_sparse_heads", "rtp_plan_work_items", "rtp_indexer_project", "rtp_block_select",
-            "rtp_block_select_dynamic",
+            "rtp_block_select_dynamic", "rtp_pipeline_create", "rtp_pipeline_destroy", "rtp_hybrid_prefill_host",
             "rtp_hybrid_prefill", "rtp_decode_workspace_bytes", "rtp_sparse_decode", "rtp_sparse_decode_noalloc",
             "rtp_cache_centroids", "rtp_cache_append", "rtp_cache_cluster_workspace_bytes", "rtp_cache_cluster",
             "rtp_decode_clustered_workspace_bytes", "rtp_sparse_decode_clustered",
@@ -228,6 +231,26 @@ def default_selection_beta(cfg: AttnConfig) -> float:
 def rtp_hybrid_prefill(plan: int, q, k, v, sel, sel_cnt, o, stream=None) -> None:
     _check("rtp_hybrid_prefill", _lib.rtp_hybrid_prefill(plan, _ptr(q), _ptr(k), _ptr(v), _ptr(sel), _ptr(sel_cnt),
                                                          _ptr(o), _stream(stream)))
+
+
+def rtp_pipeline_create(cfg: AttnConfig, kinds, n_chunks: int, stream=None) -> int:
+    out = ctypes.c_void_p()
+    c = cfg.c()
+    _check("rtp_pipeline_create", _lib.rtp_pipeline_create(ctypes.byref(c), _kinds(kinds), int(n_chunks),
+                                                             _stream(stream), ctypes.byref(out)))
+    return out.value
+
+
+def rtp_pipeline_destroy(pipeline: int) -> None:
+    _lib.rtp_pipeline_destroy(pipeline)
+
+
+def rtp_hybrid_prefill_host(pipeline: int, q_host, k_host, v_host, proj, o_host, q_dev, k_dev, v_dev, o_dev,
+                            centroids=None, qbar=None, sel=None, sel_cnt=None, stream=None) -> None:
+    _check("rtp_hybrid_prefill_host",
+           _lib.rtp_hybrid_prefill_host(pipeline, _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(proj),
+                                        _ptr(o_host), _ptr(q_dev), _ptr(k_dev), _ptr(v_dev), _ptr(o_dev),
+                                        _ptr(centroids), _ptr(qbar), _ptr(sel), _ptr(sel_cnt), _stream(stream)))
 
 
 def rtp_decode_workspace_bytes(cfg: AttnConfig, kinds, cache_len: int) -> int:
@@ -434,6 +457,41 @@ class Plan:
             rtp_hybrid_prefill(self.handle, q, k, v, bufs["sel"], bufs["sel_cnt"], o, stream)
         else:
             rtp_hybrid_prefill(self.handle, q, k, v, None, None, o, stream)
+
+
+class HostPipeline:
+    """Prefill of layers whose Q/K/V/O live in host memory, chunked so that
+    uploads, kernels and downloads overlap (rtp_pipeline_create /
+    rtp_hybrid_prefill_host).  Owns the device staging buffers."""
+
+    def __init__(self, cfg: AttnConfig, kinds, n_chunks: int = 8, device="cuda", stream=None):
+        self.cfg = cfg
+        self.handle = rtp_pipeline_create(cfg, kinds, n_chunks, stream)
+        c = cfg
+        qs = (c.batch, c.n_q_heads, c.seq, 128)
+        ks = (c.batch, c.n_kv_heads, c.seq, 128)
+        bf = dict(dtype=torch.bfloat16, device=device)
+        self.q, self.k, self.v, self.o = (torch.empty(qs, **bf), torch.empty(ks, **bf), torch.empty(ks, **bf),
+                                          torch.empty(qs, **bf))
+        self.plan = Plan(cfg, kinds, stream)  # for the shapes of the selection buffers
+        self.bufs = self.plan.buffers(device)
+        self.plan.close()
+
+    def run(self, q_host, k_host, v_host, proj, o_host, stream=None) -> None:
+        b = self.bufs
+        rtp_hybrid_prefill_host(self.handle, q_host, k_host, v_host, proj, o_host, self.q, self.k, self.v, self.o,
+                                b["centroids"], b["qbar"], b["sel"], b["sel_cnt"], stream)
+
+    def close(self):
+        if self.handle:
+            rtp_pipeline_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def hybrid_prefill_layer(q, k, v, kinds, proj=None, *, window: int, block: int = 128, topk: int = 0,
