@@ -131,3 +131,47 @@ def test_prefill_on_dynamic_selection(rtp, cuda_device):
     many = np.arange(n // block) - n_local > cap
     assert (cnt[many] < 1 + cap + n_local).any()
     plan.close()
+
+
+@pytest.mark.slow
+def test_dynamic_selection_full_size_1m(rtp, cuda_device):
+    """The 1M-token layer with the mass-threshold selection (peaked weights):
+    sampled query blocks against the oracle (R21), sampled output rows
+    against the oracle on the GPU's selection."""
+    w = inputs.workload(3)
+    d = inputs.prefill_layer(w, 0, cuda_device)
+    mass, beta = 0.9, 100.0
+    q, k, v, proj, o, bufs, plan, cfg = run_dynamic(rtp, d, w.window, w.block, w.topk, w.n_local, cuda_device,
+                                                    mass, 0, beta)
+    G, n, B = w.group, w.seq, w.block
+    nb = n // B
+    rng = np.random.default_rng(5)
+    t_list = np.array(sorted(set([0, 1, w.n_local + 1, w.topk + w.n_local + 1, nb - 1]
+                                 + list(rng.integers(0, nb, 40)))), dtype=np.int64)
+    kvh = plan.slot_heads[0]
+    C = oracle.centroids(cpu(k[0, kvh]), B, cpu(proj))
+    Qb = np.zeros((nb, 16))
+    for t in t_list:
+        Qb[t] = oracle.qbar(cpu(q[0, kvh * G:(kvh + 1) * G, t * B:(t + 1) * B]), B, cpu(proj))[0]
+    sel, cnt = cpu(bufs["sel"][0, 0]).numpy(), cpu(bufs["sel_cnt"][0, 0]).numpy()
+    sel_o, cnt_o, _, _ = oracle.select_dynamic(Qb[t_list], C, t_list, w.topk, w.n_local, mass, 0, beta)
+    for r, t in enumerate(t_list):
+        g = [int(x) for x in sel[t, :cnt[t]]]
+        assert g == sorted(set(g))
+        order, frac, s = oracle_fractions(Qb[t], C, int(t), w.n_local, beta)
+        n_g = len([x for x in g if 1 <= x <= t - w.n_local])
+        n_o = len([x for x in sel_o[r, :cnt_o[r]] if 1 <= x <= t - w.n_local])
+        if n_g < n_o:
+            assert mass - frac[n_g - 1] <= MASS_TOL
+        elif n_g > n_o:
+            assert frac[n_g - 2] - mass <= MASS_TOL
+        if n_g:
+            kth = s[order[n_g - 1]]
+            for b in set(int(x) for x in order[:n_g]) ^ set(x for x in g if 1 <= x <= t - w.n_local):
+                assert abs(s[b] - kth) <= TIE_REL * abs(kth)
+    assert cnt[nb // 2:].mean() < 1 + w.topk + w.n_local  # the budget shrank on average
+    slot_of = {h: s_ for s_, h in enumerate(plan.slot_heads)}
+    rows = np.unique(np.concatenate([t_list * B, t_list * B + B - 1, rng.integers(0, n, 16)]))
+    check_prefill_rows(o, q, k, v, d["kinds"], G, w.window, B, bufs["sel"], bufs["sel_cnt"], slot_of,
+                       lambda hq: rows)
+    plan.close()

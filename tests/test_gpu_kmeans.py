@@ -245,3 +245,47 @@ def test_gpu_clustering_then_decode_runs_clean(rtp, cuda_device):
         ref = oracle.attention_keys(cpu(q[b, :G, 0]), cpu(k[b, 0, :Lc]), cpu(v[b, 0, :Lc]), np.sort(keys))
         got = cpu(o[b, :G, 0]).double().numpy()
         assert np.max(np.abs(got - oracle.round_bf16(ref))) <= O_MAX_ABS
+
+
+@pytest.mark.slow
+def test_clustered_decode_full_size_cache(rtp, cuda_device):
+    """Two sequences of the 256K-token decode workload, clustered by the
+    oracle (256 clusters, 2 rounds) and decoded with the clustered kernels."""
+    w = inputs.workload(4)
+    d = inputs.decode_step(w, cuda_device, batch=2)
+    kinds, Lc, B = d["kinds"], d["cache_len"], w.block
+    clu_end = (Lc // B - w.n_local) * B
+    q, k, v, proj = d["q"], d["kcache"], d["vcache"], d["proj"]
+    cl, per_head = clusters_from_oracle(rtp, k, v, proj, kinds, clu_end, 256, 2, B)
+    o, sel, cnt = rtp.sparse_decode_clustered_step(q, k, v, proj, kinds, cl, window=w.window, block=B, topk=w.topk,
+                                                   return_selection=True)
+    torch.cuda.synchronize()
+    assert rtp.rtp_last_device_status() == rtp.RTP_OK
+    sel, cnt, o = cpu(sel).numpy(), cpu(cnt).numpy(), cpu(o)
+    G = w.group
+    n_tail = (Lc - clu_end + 127) // 128
+    errs = []
+    for b in range(2):
+        for h, kind in enumerate(kinds):
+            qg = cpu(q[b, h * G:(h + 1) * G, 0])
+            kh, vh = cpu(k[b, h]), cpu(v[b, h])
+            if kind == 2:
+                members, chunks, cc = per_head[(b, h)]
+                m = min(w.topk, len(chunks))
+                assert cnt[b, h] == 1 + n_tail + m
+                chosen = sel[b, h, 1:1 + m]
+                qb = oracle.project_rows(qg, cpu(proj)).sum(axis=0)
+                ref_sel = oracle.topk_chunks(qb, cc, m)
+                if set(chosen.tolist()) != set(ref_sel.tolist()):
+                    s = oracle.scores(qb, cc)
+                    kth = np.sort(s)[::-1][m - 1]
+                    for x in set(chosen.tolist()) ^ set(ref_sel.tolist()):
+                        assert abs(s[x] - kth) <= TIE_REL * abs(kth)
+                keys = oracle.decode_clustered_keys(members, chunks, chosen, B, clu_end, Lc)
+                ref = oracle.attention_keys(qg, kh, vh, keys)
+            else:
+                ref, _, _, _ = oracle.decode_head(qg, kh, vh, np.zeros((Lc // B, 16)), cpu(proj), kind, w.window, B,
+                                                  w.topk, w.n_local)
+            errs.append(np.abs(o[b, h * G:(h + 1) * G, 0].double().numpy() - oracle.round_bf16(ref)))
+    e = np.stack(errs)
+    assert e.max() <= O_MAX_ABS and e.mean() <= O_MEAN_ABS, (e.max(), e.mean())

@@ -53,3 +53,25 @@ def test_host_pipeline_equals_device_layer(rtp, cuda_device, case):
     if 2 in kinds:
         assert torch.equal(pl.bufs["sel"], bufs["sel"]) and torch.equal(pl.bufs["sel_cnt"], bufs["sel_cnt"])
     pl.close()
+
+
+@pytest.mark.slow
+def test_host_pipeline_full_size_1m_layer(rtp, cuda_device):
+    """The 1M-token layer from pinned host memory in 16 chunks equals the device-resident layer."""
+    w = inputs.workload(3)
+    d = inputs.prefill_layer(w, 0, cuda_device)
+    cfg = rtp.AttnConfig(1, w.seq, w.n_q_heads, w.n_kv_heads, w.window, w.block, w.topk, w.n_local)
+    plan = rtp.Plan(cfg, d["kinds"])
+    bufs = plan.buffers(cuda_device)
+    o_ref = torch.empty_like(d["q"])
+    plan.run(d["q"], d["k"], d["v"], d["proj"], o_ref, bufs)
+    torch.cuda.synchronize()
+    plan.close()
+    hq_, hk_, hv_ = (x.cpu().pin_memory() for x in (d["q"], d["k"], d["v"]))
+    ho = torch.empty(d["q"].shape, dtype=torch.bfloat16).pin_memory()
+    pl = rtp.HostPipeline(cfg, d["kinds"], 16, device=cuda_device)
+    pl.run(hq_, hk_, hv_, d["proj"], ho)
+    torch.cuda.synchronize()
+    assert rtp.rtp_last_device_status() == rtp.RTP_OK
+    assert torch.equal(ho.to(cuda_device), o_ref)
+    pl.close()
