@@ -12,6 +12,8 @@
 #include <new>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/rtp.h"
 #include "internal.cuh"
 #include "sm100.cuh"
@@ -51,6 +53,13 @@ struct rtp_plan {
 namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
+
+// An NVTX range named after the entry point for the duration of the call
+// (visible in a profiler's timeline; no cost when none is attached).
+struct CallRange {
+  explicit CallRange(const char* name) { nvtxRangePushA(name); }
+  ~CallRange() { nvtxRangePop(); }
+};
 
 // Self-test of the bounded wait used by every kernel: an mbarrier nobody
 // arrives on, waited for with a short limit.
@@ -270,6 +279,7 @@ rtp_status rtp_route_heads(const rtp_attn_cfg* cfg, const uint8_t* kind_host, vo
 
 rtp_status rtp_route_heads_range(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int q_begin, int q_end,
                                  void* stream, rtp_plan** out) {
+  CallRange range_("rtp_route_heads_range");
   if (!out) return RTP_ERR_INVALID_ARG;
   *out = nullptr;
   if (!cfg_prefill_ok(cfg) || !kind_host) return RTP_ERR_INVALID_ARG;
@@ -389,6 +399,7 @@ rtp_status rtp_plan_work_items(const rtp_plan* plan, int32_t* items_host) {
 
 rtp_status rtp_indexer_project(const rtp_plan* plan, const void* q, const void* k, const float* proj,
                                float* centroids, float* qbar, void* stream) {
+  CallRange range_("rtp_indexer_project");
   if (!plan) return RTP_ERR_INVALID_ARG;
   return indexer_run(plan, q, k, plan->q_end - plan->q_begin, proj, centroids, qbar, stream);
 }
@@ -396,6 +407,7 @@ rtp_status rtp_indexer_project(const rtp_plan* plan, const void* q, const void* 
 
 rtp_status rtp_block_select(const rtp_plan* plan, const float* qbar, const float* centroids, int32_t* sel,
                             int32_t* sel_cnt, void* stream) {
+  CallRange range_("rtp_block_select");
   if (!plan) return RTP_ERR_INVALID_ARG;
   if (plan->n_sparse == 0) return RTP_OK;
   if (!qbar || !centroids || !sel || !sel_cnt) return RTP_ERR_INVALID_ARG;
@@ -420,6 +432,7 @@ rtp_status rtp_block_select(const rtp_plan* plan, const float* qbar, const float
 
 rtp_status rtp_block_select_dynamic(const rtp_plan* plan, const float* qbar, const float* centroids, float mass,
                                     int min_k, float beta, int32_t* sel, int32_t* sel_cnt, void* stream) {
+  CallRange range_("rtp_block_select_dynamic");
   if (!plan) return RTP_ERR_INVALID_ARG;
   const rtp_attn_cfg& c = plan->cfg;
   if (!(mass > 0.f && mass <= 1.f) || !(beta >= 0.f) || !std::isfinite(beta)) return RTP_ERR_INVALID_ARG;
@@ -450,6 +463,7 @@ rtp_status rtp_block_select_dynamic(const rtp_plan* plan, const float* qbar, con
 
 rtp_status rtp_hybrid_prefill(const rtp_plan* plan, const void* q, const void* k, const void* v,
                               const int32_t* sel, const int32_t* sel_cnt, void* o, void* stream) {
+  CallRange range_("rtp_hybrid_prefill");
   if (!plan) return RTP_ERR_INVALID_ARG;
   return prefill_run(plan, q, plan->q_end - plan->q_begin, k, v, plan->q_end, sel, sel_cnt, o, stream);
 }
@@ -685,6 +699,7 @@ rtp_status rtp_sparse_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, 
                              const void* kcache, const void* vcache, const float* centroids, const float* proj,
                              void* o, void* workspace, size_t ws_bytes, int32_t* sel_out, int32_t* cnt_out,
                              void* stream) {
+  CallRange range_("rtp_sparse_decode");
   DecodeLayout L;
   DecodeArgs a;
   rtp_status st = prepare_decode(cfg, kind_host, cache_len, q, kcache, vcache, centroids, proj, nullptr, o, sel_out,
@@ -698,6 +713,7 @@ rtp_status rtp_sparse_decode_clustered(const rtp_attn_cfg* cfg, const uint8_t* k
                                        const void* q, const void* kcache, const void* vcache, const float* proj,
                                        const rtp_clusters* cl, void* o, void* workspace, size_t ws_bytes,
                                        int32_t* sel_out, int32_t* cnt_out, void* stream) {
+  CallRange range_("rtp_sparse_decode_clustered");
   if (!cl) return RTP_ERR_INVALID_ARG;
   DecodeLayout L;
   DecodeArgs a;
@@ -711,6 +727,7 @@ rtp_status rtp_sparse_decode_clustered(const rtp_attn_cfg* cfg, const uint8_t* k
 rtp_status rtp_sparse_decode_noalloc(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* q,
                                      const void* kcache, const void* vcache, const float* centroids,
                                      const float* proj, void* o, int32_t* sel_out, int32_t* cnt_out, void* stream) {
+  CallRange range_("rtp_sparse_decode_noalloc");
   DecodeLayout L;
   DecodeArgs a;
   rtp_status st = prepare_decode(cfg, kind_host, cache_len, q, kcache, vcache, centroids, proj, nullptr, o, sel_out,
@@ -734,6 +751,7 @@ size_t rtp_cache_cluster_workspace_bytes(const rtp_attn_cfg* cfg, int clu_end) {
 rtp_status rtp_cache_cluster(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int iters, const void* kcache,
                              const void* vcache, const float* proj, const rtp_clusters* cl, void* workspace,
                              size_t ws_bytes, void* stream) {
+  CallRange range_("rtp_cache_cluster");
   if (!cfg || !cl || iters < 1 || iters > 1000) return RTP_ERR_INVALID_ARG;
   if (!cluster_args_ok(cfg, kind_host, cl, decode_capacity(cfg, cl->clu_end))) return RTP_ERR_INVALID_ARG;
   if (!kcache || !vcache || !proj || !aligned16(kcache) || !aligned16(vcache) || !aligned16(proj))
@@ -772,6 +790,7 @@ rtp_status rtp_cache_cluster(const rtp_attn_cfg* cfg, const uint8_t* kind_host, 
 
 rtp_status rtp_cache_centroids(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* kcache,
                                const float* proj, float* centroids, void* stream) {
+  CallRange range_("rtp_cache_centroids");
   if (!cfg || cache_len < 1) return RTP_ERR_INVALID_ARG;
   CacheArgs a;
   const rtp_status st = cache_args(cfg, kind_host, decode_capacity(cfg, cache_len), kcache, proj, centroids, a);
@@ -783,6 +802,7 @@ rtp_status rtp_cache_centroids(const rtp_attn_cfg* cfg, const uint8_t* kind_host
 rtp_status rtp_cache_append(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int pos, const void* k_new,
                             const void* v_new, void* kcache, void* vcache, const float* proj, float* centroids,
                             void* stream) {
+  CallRange range_("rtp_cache_append");
   if (!cfg || pos < 0 || pos >= cfg->seq) return RTP_ERR_INVALID_ARG;
   CacheArgs a;
   const rtp_status st = cache_args(cfg, kind_host, cfg->seq, kcache, proj, centroids, a);
@@ -799,6 +819,7 @@ rtp_status rtp_cache_append(const rtp_attn_cfg* cfg, const uint8_t* kind_host, i
 // ------------------------------------------------------- host pipeline
 rtp_status rtp_pipeline_create(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int n_chunks, void* stream,
                                rtp_pipeline** out) {
+  CallRange range_("rtp_pipeline_create");
   if (!out) return RTP_ERR_INVALID_ARG;
   *out = nullptr;
   if (!cfg_prefill_ok(cfg) || !kind_host || n_chunks < 1 || n_chunks > 1024) return RTP_ERR_INVALID_ARG;
@@ -856,6 +877,7 @@ rtp_status rtp_hybrid_prefill_host(rtp_pipeline* pl, const void* q_host, const v
                                    const float* proj, void* o_host, void* q_dev, void* k_dev, void* v_dev,
                                    void* o_dev, float* centroids, float* qbar, int32_t* sel, int32_t* sel_cnt,
                                    void* stream) {
+  CallRange range_("rtp_hybrid_prefill_host");
   if (!pl || !q_host || !k_host || !v_host || !o_host || !q_dev || !k_dev || !v_dev || !o_dev)
     return RTP_ERR_INVALID_ARG;
   if (pl->n_sparse > 0 && (!proj || !centroids || !qbar || !sel || !sel_cnt)) return RTP_ERR_INVALID_ARG;
