@@ -776,7 +776,16 @@ def run_ours(args, rank, world, local):
         extra["dynamic"] = time_dynamic(rtp, w, res, device)
         extra["cp"] = time_cp_projection(rtp, w, res, device)
     if not args.no_e2e:
-        extra["e2e"] = time_e2e(rtp, w, res, max(2, min(args.steps, 3)), device, args.e2e_chunks)
+        e2e = time_e2e(rtp, w, res, max(2, min(args.steps, 3)), device, args.e2e_chunks)
+        # whole job: every rank's layer, over the slowest rank's time (every rank
+        # takes part in the reduction, also one whose pinned allocation failed)
+        t_max = max_over_ranks(e2e.get("ms_per_step", float("inf")), world)
+        if "error" not in e2e:
+            e2e["value"] = world * algo / (t_max * 1e-3) / 1e12
+            e2e["ms_per_step"] = t_max
+            e2e["h2d_bytes_per_step"] *= world
+            e2e["d2h_bytes_per_step"] *= world
+        extra["e2e"] = e2e
     for key in ("q", "k", "v", "o"):
         res[key] = None
     res["plan"].close()
