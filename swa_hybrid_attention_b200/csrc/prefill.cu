@@ -338,7 +338,9 @@ __device__ __forceinline__ bool issue_pv_chunked(Smem& s, int h, uint32_t parity
                                                  uint32_t* status) {
 #pragma unroll
   for (int q = 0; q < kPChunks; ++q) {
-    if (!mbar_wait_spin(&s.p_full[h][q], parity, abort, status)) return false;
+    // a suspending wait: a polling loop here would take issue slots from
+    // the two softmax warps that share this scheduler (measured ~1 % slower)
+    if (!mbar_wait(&s.p_full[h][q], parity, abort, status)) return false;
     tc_fence_after();
     issue_pv(d_tmem, p_tmem, vd, idesc, accumulate, q * (8 / kPChunks), (q + 1) * (8 / kPChunks));
   }
