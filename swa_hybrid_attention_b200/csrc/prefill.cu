@@ -19,7 +19,9 @@
 //    loaded into shared memory feeds two S = Q K^T and two O += P V MMAs.
 //    The four pairs of a group run on neighbouring CTAs at the same time,
 //    so K/V are re-read from L2, not HBM.
-//  * Warp roles: warp 0 = TMA producer (Q tiles, then a 2-stage K/V ring),
+//  * Warp roles: warp 0 = TMA producer (Q tiles, then a 2-stage K/V ring; a
+//    stage's K is released as soon as both heads' S MMAs have read it and its
+//    V after both P V MMAs, so the next K loads a tile earlier than V),
 //    warp 1 = single-thread tcgen05.mma issuer, warp 2 = TMEM allocator,
 //    warps 4-7 / 8-11 = softmax for head 0 / head 1 of the pair (one thread
 //    per query row, the whole S row in registers: no cross-thread reduction).
@@ -89,7 +91,9 @@ struct __align__(1024) Smem {
   uint8_t k[kStages][kTileBytes];
   uint8_t v[kStages][kTileBytes];
   uint64_t q_full[2], q_empty[2];
-  uint64_t k_full[kStages], v_full[kStages], kv_empty[kStages];
+  uint64_t k_full[kStages], v_full[kStages];
+  uint64_t k_empty[kStages];  // released once both heads' S MMAs of the tile have read K
+  uint64_t v_empty[kStages];  // released once both heads' P V MMAs have read V
   uint64_t s_full[2], o_full[2];
   uint64_t p_full[2][kPChunks];  // [head][chunk of keys]: that part of P is in TMEM
   uint64_t drain;
@@ -277,12 +281,13 @@ __device__ __noinline__ void run_producer(Smem& s, const CUtensorMap* mq, const 
         TileRef tr = ti.next();
         const int st = gt & 1;
         const uint32_t use = gt >> 1;
-        if (!mbar_wait(&s.kv_empty[st], (use & 1u) ^ 1u, abort, a.status)) goto drain;
+        if (!mbar_wait(&s.k_empty[st], (use & 1u) ^ 1u, abort, a.status)) goto drain;
         mbar_arrive_expect_tx(&s.k_full[st], kTileBytes);
         for (int c = 0; c < 2; ++c) {
           tma_load_3d(s.k[st] + c * kChunkBytes, mk, &s.k_full[st], 64 * c, tr.row0, item.bkv);
           tma_load_3d(s.k[st] + c * kChunkBytes + kChunkBytes / 2, mk, &s.k_full[st], 64 * c, tr.row1, item.bkv);
         }
+        if (!mbar_wait(&s.v_empty[st], (use & 1u) ^ 1u, abort, a.status)) goto drain;
         mbar_arrive_expect_tx(&s.v_full[st], kTileBytes);
         for (int c = 0; c < 2; ++c) {
           tma_load_3d(s.v[st] + c * kChunkBytes, mv, &s.v_full[st], 64 * c, tr.row0, item.bkv);
@@ -373,6 +378,7 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
       umma_commit(&s.s_full[0]);
       issue_qk(tS[1], qd1, sk, id_qk);
       umma_commit(&s.s_full[1]);
+      umma_commit(&s.k_empty[st0]);
       if (n == 1) {
         umma_commit(&s.q_empty[0]);
         umma_commit(&s.q_empty[1]);
@@ -399,12 +405,13 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
       }
       // head 1
       if (!issue_pv_chunked(s, 1, pc & 1u, tO[1], tS[1], sv, id_pv, j > 0, abort, a.status)) goto drain;
-      umma_commit(&s.kv_empty[st]);
+      umma_commit(&s.v_empty[st]);
       if (!has_next) {
         umma_commit(&s.o_full[1]);
       } else {
         issue_qk(tS[1], qd1, sk2, id_qk);
         umma_commit(&s.s_full[1]);
+        umma_commit(&s.k_empty[st2]);
         if (j + 2 == n) umma_commit(&s.q_empty[1]);
       }
       ++pc;
@@ -562,7 +569,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int st = 0; st < kStages; ++st) {
       mbar_init(&s.k_full[st], 1);
       mbar_init(&s.v_full[st], 1);
-      mbar_init(&s.kv_empty[st], 1);
+      mbar_init(&s.k_empty[st], 1);
+      mbar_init(&s.v_empty[st], 1);
     }
     mbar_init(&s.drain, 1);
     s.abort_flag = 0;
