@@ -310,6 +310,26 @@ drain:
 }
 
 // ---------------------------------------------------------------- MMA issue
+// The MMA thread's waits: a non-blocking test first (most phases it waits for
+// have completed already, and the suspending try_wait costs ~150 cycles even
+// then; this thread is the serial link between the softmax warps and the
+// tensor pipe, so its own latencies add up), the bounded suspending wait
+// otherwise.
+__device__ __forceinline__ bool mbar_test_nb(uint64_t* bar, uint32_t parity) {  // test_wait: never suspends
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mma_wait(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t* status) {
+  if (mbar_test_nb(bar, parity)) return true;
+  return mbar_wait(bar, parity, abort, status);
+}
 // The single issuing thread shares its scheduler with two busy softmax warps
 // and the tensor pipe buffers very few MMAs, so the issue path is kept short:
 // operand descriptors are built once per kernel and an operand at base + off
@@ -343,9 +363,9 @@ __device__ __forceinline__ bool issue_pv_chunked(Smem& s, int h, uint32_t parity
                                                  uint32_t* status) {
 #pragma unroll
   for (int q = 0; q < kPChunks; ++q) {
-    // a suspending wait: a polling loop here would take issue slots from
-    // the two softmax warps that share this scheduler (measured ~1 % slower)
-    if (!mbar_wait(&s.p_full[h][q], parity, abort, status)) return false;
+    // a polling loop here would take issue slots from the two softmax warps
+    // that share this scheduler (measured ~1 % slower than suspending)
+    if (!mma_wait(&s.p_full[h][q], parity, abort, status)) return false;
     tc_fence_after();
     issue_pv(d_tmem, p_tmem, vd, idesc, accumulate, q * (8 / kPChunks), (q + 1) * (8 / kPChunks));
   }
@@ -367,11 +387,11 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
     TileIter ti;
     ti.init(item, a);
     const int n = ti.n;
-    if (!mbar_wait(&s.q_full[0], it & 1u, abort, a.status)) goto drain;
-    if (!mbar_wait(&s.q_full[1], it & 1u, abort, a.status)) goto drain;
+    if (!mma_wait(&s.q_full[0], it & 1u, abort, a.status)) goto drain;
+    if (!mma_wait(&s.q_full[1], it & 1u, abort, a.status)) goto drain;
     {
       const int st0 = gt & 1;
-      if (!mbar_wait(&s.k_full[st0], (gt >> 1) & 1u, abort, a.status)) goto drain;
+      if (!mma_wait(&s.k_full[st0], (gt >> 1) & 1u, abort, a.status)) goto drain;
       tc_fence_after();
       const uint64_t sk = st0 ? kd1 : kd0;
       issue_qk(tS[0], qd0, sk, id_qk);
@@ -391,13 +411,13 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
       const int st2 = (g + 1) & 1;
       const uint64_t sv = st ? vd1 : vd0;
       const uint64_t sk2 = st2 ? kd1 : kd0;
-      if (!mbar_wait(&s.v_full[st], (g >> 1) & 1u, abort, a.status)) goto drain;
+      if (!mma_wait(&s.v_full[st], (g >> 1) & 1u, abort, a.status)) goto drain;
       // head 0: O0 += P0 V ; then S0 for the next tile
       if (!issue_pv_chunked(s, 0, pc & 1u, tO[0], tS[0], sv, id_pv, j > 0, abort, a.status)) goto drain;
       if (!has_next) {
         umma_commit(&s.o_full[0]);
       } else {
-        if (!mbar_wait(&s.k_full[st2], ((g + 1) >> 1) & 1u, abort, a.status)) goto drain;
+        if (!mma_wait(&s.k_full[st2], ((g + 1) >> 1) & 1u, abort, a.status)) goto drain;
         tc_fence_after();
         issue_qk(tS[0], qd0, sk2, id_qk);
         umma_commit(&s.s_full[0]);
