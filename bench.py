@@ -528,6 +528,7 @@ def time_decode(rtp, steps, device):
     torch.cuda.synchronize()
     ms = statistics.median(a.elapsed_time(b) for a, b in times)
     status = rtp.rtp_last_device_status(stream)
+    graph = time_decode_graph(rtp, w, d, C, o, flush, flush_read, steps)
     upkeep = time_cache_upkeep(rtp, w, d, C, cfg, flush, flush_read, steps, stream)
     clustered = time_clustered_decode(rtp, w, d, flush, flush_read, steps, stream)
     G = w.group
@@ -539,8 +540,49 @@ def time_decode(rtp, steps, device):
     flops = w.batch * keys * G * 4 * 128
     return {"workload": w.name, "ms_per_step": ms, "algorithmic_bytes": bytes_, "gb_s": bytes_ / (ms * 1e-3) / 1e9,
             "tflops_effective": flops / (ms * 1e-3) / 1e12, "l2": "flushed before each step (256 MB write, then 256 MB read)",
-            "launches_per_step": 3, "status": rtp.status_str(status), "cache_upkeep": upkeep,
+            "launches_per_step": 3, "status": rtp.status_str(status), "graph": graph, "cache_upkeep": upkeep,
             "clustered": clustered}
+
+
+def time_decode_graph(rtp, w, d, C, o_ref, flush, flush_read, steps):
+    """The same step as a serving loop would run it: the allocation-free
+    entry point captured once in a CUDA graph (its three launches and their
+    programmatic dependencies) and replayed; L2 flushed before each replay
+    as for the direct launches.  The replay's output must equal theirs."""
+    kinds, Lc = d["kinds"], d["cache_len"]
+    cfg = rtp.AttnConfig(w.batch, 1, w.n_q_heads, w.n_kv_heads, w.window, w.block, w.topk, w.n_local)
+    o = torch.empty_like(o_ref)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+
+    def step():
+        rtp.rtp_sparse_decode_noalloc(cfg, kinds, Lc, d["q"], d["kcache"], d["vcache"], C, d["proj"], o, stream=s)
+
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    torch.cuda.synchronize()
+    times = []
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            g.replay()
+        for _ in range(steps):
+            flush.zero_()
+            flush_read.sum()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(s)
+            g.replay()
+            b.record(s)
+            times.append((a, b))
+    torch.cuda.synchronize()
+    same = bool(torch.equal(o, o_ref))
+    del g
+    return {"ms_per_step": statistics.median(a.elapsed_time(b) for a, b in times), "equal_to_direct": same,
+            "note": "rtp_sparse_decode_noalloc captured once in a CUDA graph and replayed"}
 
 
 def time_clustered_decode(rtp, w, d, flush, flush_read, steps, stream, n_clusters=2048, iters=8):

@@ -100,3 +100,41 @@ def test_decode_full_size(rtp, cuda_device):
     w = inputs.workload(4)
     d = inputs.decode_step(w, cuda_device)
     check_decode(rtp, d, w.kinds[0], w.window, w.block, w.topk, w.n_local, cuda_device)
+
+
+def test_decode_workspace_reuse_and_arbitrary_contents(rtp, cuda_device):
+    """The workspace holds only scratch of the step that uses it: one
+    workspace, first filled with arbitrary bytes, then reused for steps on
+    alternating inputs, gives every step exactly the output and selection of
+    a call on a fresh workspace (nothing of the previous step is taken for
+    this step's)."""
+    kinds, B, hq, hkv, Lc, window, block, topk, n_local = [2, 0, 2, 2], 2, 16, 4, 8192, 1024, 128, 12, 3
+    steps = []
+    for seed in (7, 8):
+        w = inputs.Workload(60 + seed, "t", B, 1, hq, hkv, 1, window, block, topk, n_local, "lowfreq", 0, [kinds],
+                            cache_len=Lc, decode=True)
+        d = inputs.decode_step(w, "cpu")
+        d = {k: (v.to(cuda_device) if torch.is_tensor(v) else v) for k, v in d.items()}
+        d["C"] = oracle_centroids(d["kcache"], kinds, block, d["proj"]).to(cuda_device)
+        ref = rtp.sparse_decode_step(d["q"], d["kcache"], d["vcache"], d["C"], d["proj"], kinds, window=window,
+                                     block=block, topk=topk, n_local=n_local, return_selection=True)
+        steps.append((d, ref))
+    cfg = rtp.AttnConfig(B, Lc, hq, hkv, window, block, topk, n_local)
+    ws_bytes = rtp.rtp_decode_workspace_bytes(cfg, kinds, Lc)
+    g = torch.Generator(device="cpu").manual_seed(3)
+    for fill in ("random", "ones"):
+        if fill == "random":
+            ws = torch.randint(0, 256, (ws_bytes,), dtype=torch.uint8, generator=g).to(cuda_device)
+        else:
+            ws = torch.full((ws_bytes,), 0xFF, dtype=torch.uint8, device=cuda_device)
+        for i in (0, 1, 0, 1, 1, 0):
+            d, (ro, rsel, rcnt) = steps[i]
+            o = torch.empty_like(d["q"])
+            sel = torch.full((B, hkv, cfg.kmax), -1, dtype=torch.int32, device=cuda_device)
+            cnt = torch.zeros(B, hkv, dtype=torch.int32, device=cuda_device)
+            rtp.rtp_sparse_decode(cfg, kinds, Lc, d["q"], d["kcache"], d["vcache"], d["C"], d["proj"], o, ws,
+                                  ws_bytes, sel, cnt)
+            torch.cuda.synchronize()
+            assert torch.equal(o, ro), (fill, i)
+            assert torch.equal(cnt, rcnt) and torch.equal(sel, rsel), (fill, i)
+    assert rtp.rtp_last_device_status() == rtp.RTP_OK
