@@ -456,9 +456,10 @@ def time_e2e(rtp, w, res, steps, device, chunks=16):
             "serial_note": "uploads, layer and download one after another on one stream"}
 
 
-def time_secondary_128k(rtp, steps, device):
-    """48-layer 128K V2 prefill pass (one pass = all layers, buffers per layer)."""
-    w = inputs.workload(2)
+def time_layers(rtp, wid, steps, device):
+    """A 48-layer prefill pass (one pass = all layers, buffers per layer):
+    the 128K V2 model (workload 2) or the 32K V1 model (workload 1)."""
+    w = inputs.workload(wid)
     layers = []
     for l in range(w.layers):
         d, plan, bufs = make_layer(rtp, w, l, device)
@@ -841,7 +842,8 @@ def run_ours(args, rank, world, local):
         torch.cuda.empty_cache()
     secondary = {}
     if not args.no_secondary and world == 1:
-        secondary["v2_128k_48_layers"] = time_secondary_128k(rtp, 2, device)
+        secondary["v2_128k_48_layers"] = time_layers(rtp, 2, 2, device)
+        secondary["v1_32k_48_layers"] = time_layers(rtp, 1, 3, device)
         secondary["decode_8x256k"] = time_decode(rtp, args.decode_steps, device)
         if extra.get("dynamic"):
             secondary["dynamic_selection"] = extra["dynamic"]
