@@ -55,13 +55,15 @@ def _load():
         _lib.oracle_scores.argtypes = [P, P, L, I, P]
         _lib.oracle_select.argtypes = [P, P, L, I, P, L, I, I, I, P, P, P]
         _lib.oracle_select_dynamic.argtypes = [P, P, L, I, P, L, I, I, I, D, I, D, P, P, P, P]
+        _lib.oracle_rowmax_scores.argtypes = [P, I, L, I, I, P, I, P, L, L, P]
+        _lib.oracle_select_rowmax.argtypes = [P, I, L, I, I, P, I, P, L, P, L, I, I, I, P, P, P]
         _lib.oracle_kmeans.argtypes = [P, L, I, I, I, P, P]
         _lib.oracle_attention_keys.argtypes = [P, I, P, P, I, P, L, D, P]
         _lib.oracle_attention_rows.argtypes = [P, P, L, P, P, L, I, I, L, I, P, P, I, D, P]
         _lib.oracle_attention_probs.argtypes = [P, L, P, L, I, I, L, I, P, P, I, D, P]
         _lib.oracle_decode_head.argtypes = [P, I, P, P, L, I, P, L, P, I, I, L, I, I, I, I, I, P, P, P, D, P]
         for f in ("oracle_project_rows", "oracle_centroids", "oracle_qbar", "oracle_scores", "oracle_select",
-                  "oracle_select_dynamic", "oracle_kmeans", "oracle_attention_keys",
+                  "oracle_select_dynamic", "oracle_rowmax_scores", "oracle_select_rowmax", "oracle_kmeans", "oracle_attention_keys",
                   "oracle_attention_rows", "oracle_attention_probs", "oracle_decode_head"):
             getattr(_lib, f).restype = None
     return _lib
@@ -149,6 +151,41 @@ def select(qbar_rows: np.ndarray, C: np.ndarray, t_list, topk: int, n_local: int
     kth = np.empty(nq, dtype=np.float64)
     _load().oracle_select(_ptr(q), _ptr(c), c.shape[0], c.shape[1], _ptr(t), nq, topk, n_local, kmax, _ptr(sel),
                           _ptr(cnt), _ptr(kth))
+    return sel, cnt, kth
+
+
+def rowmax_scores(q_group, proj, C: np.ndarray, t: int, block: int) -> np.ndarray:
+    """Row-max scores of query block t (the alternative to the block mean as
+    the query-side aggregate of the RTPurboV2 indexer): u_i = sum_h P^T q_{h,i}
+    over the block's rows, s_j = max_i u_i . c_j for every block j (fp64).
+    q_group: the group's heads [G, N, 128] bf16; C: [nb, 16]."""
+    qb = _bf16_bits(q_group)
+    G = qb.shape[0]
+    qb = qb.reshape(G, -1, 128)
+    p = _f32(proj)
+    c = np.ascontiguousarray(C, dtype=np.float64)
+    out = np.empty(c.shape[0], dtype=np.float64)
+    _load().oracle_rowmax_scores(_ptr(qb), G, qb.shape[1], 128, block, _ptr(p), p.shape[1], _ptr(c), c.shape[0],
+                                 int(t), _ptr(out))
+    return out
+
+
+def select_rowmax(q_group, proj, C: np.ndarray, t_list, block: int, topk: int, n_local: int):
+    """Block selection with row-max scores and the fixed rule (sink + top-k by
+    (score desc, index asc) + local).  Returns (sel, cnt, kth_score) as select."""
+    qb = _bf16_bits(q_group)
+    G = qb.shape[0]
+    qb = qb.reshape(G, -1, 128)
+    p = _f32(proj)
+    c = np.ascontiguousarray(C, dtype=np.float64)
+    t = np.ascontiguousarray(t_list, dtype=np.int32)
+    nq = t.shape[0]
+    kmax = topk + 1 + n_local
+    sel = np.empty((nq, kmax), dtype=np.int32)
+    cnt = np.empty(nq, dtype=np.int32)
+    kth = np.empty(nq, dtype=np.float64)
+    _load().oracle_select_rowmax(_ptr(qb), G, qb.shape[1], 128, block, _ptr(p), p.shape[1], _ptr(c), c.shape[0],
+                                 _ptr(t), nq, topk, n_local, kmax, _ptr(sel), _ptr(cnt), _ptr(kth))
     return sel, cnt, kth
 
 

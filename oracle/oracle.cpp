@@ -44,6 +44,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <thread>
+#include <limits>
 #include <vector>
 
 namespace {
@@ -153,12 +154,11 @@ void oracle_scores(const double* qbar, const double* C, long nb, int r, double* 
 // written to sel[q][0..cnt-1] (the rest of the row is set to -1).
 // kth_score[q] receives the score of the k-th kept candidate, or NaN when
 // every candidate was kept (no cut was made).
-void oracle_select(const double* qbar, const double* C, long nb, int r, const int32_t* t_list, long nq, int topk,
-                   int n_local, int kmax, int32_t* sel, int32_t* cnt, double* kth_score) {
-  parallel_for(nq, [&](long q) {
-    long t = t_list[q];
-    std::vector<double> s(nb);
-    oracle_scores(qbar + q * r, C, nb, r, s.data());
+// The selection rule given the scores s[0..nb) of query block t: one output
+// row sel[0..kmax), its count and the k-th kept score (NaN without a cut).
+static void select_row(const std::vector<double>& s, long t, int topk, int n_local, int kmax, int32_t* sel,
+                       int32_t* cnt, double* kth_score) {
+  {
     long last_cand = t - n_local;  // candidates are 1..last_cand
     std::vector<long> cand;
     for (long j = 1; j <= last_cand; ++j) cand.push_back(j);
@@ -176,9 +176,54 @@ void oracle_select(const double* qbar, const double* C, long nb, int r, const in
     for (long j = std::max<long>(0, t - n_local + 1); j <= t; ++j) all.push_back(j);
     std::sort(all.begin(), all.end());
     all.erase(std::unique(all.begin(), all.end()), all.end());
-    for (int i = 0; i < kmax; ++i) sel[q * kmax + i] = i < static_cast<int>(all.size()) ? static_cast<int32_t>(all[i]) : -1;
-    cnt[q] = static_cast<int32_t>(all.size());
-    kth_score[q] = kth;
+    for (int i = 0; i < kmax; ++i) sel[i] = i < static_cast<int>(all.size()) ? static_cast<int32_t>(all[i]) : -1;
+    *cnt = static_cast<int32_t>(all.size());
+    *kth_score = kth;
+  }
+}
+
+void oracle_select(const double* qbar, const double* C, long nb, int r, const int32_t* t_list, long nq, int topk,
+                   int n_local, int kmax, int32_t* sel, int32_t* cnt, double* kth_score) {
+  parallel_for(nq, [&](long q) {
+    std::vector<double> s(nb);
+    oracle_scores(qbar + q * r, C, nb, r, s.data());
+    select_row(s, t_list[q], topk, n_local, kmax, sel + q * kmax, cnt + q, kth_score + q);
+  });
+}
+
+// Row-max scores of query block t (the per-query-block aggregate of the
+// [P2] indexer is left open by the pages; this is the alternative to the
+// mean): u_i = sum_{h in group} P^T q_{h,i} for every row i of the block,
+// s_j = max_i u_i . c_j (fp64).  q: the group's heads, [G][N][D] bf16;
+// C: [nb][r]; out: [nb].
+void oracle_rowmax_scores(const uint16_t* q, int G, long N, int D, int B, const float* P, int r, const double* C,
+                          long nb, long t, double* out) {
+  std::vector<double> u(static_cast<size_t>(B) * r, 0.0), qt(r);
+  for (int i = 0; i < B; ++i)
+    for (int h = 0; h < G; ++h) {
+      project_row(q + (static_cast<long>(h) * N + t * B + i) * D, D, P, r, qt.data());
+      for (int c = 0; c < r; ++c) u[static_cast<size_t>(i) * r + c] += qt[c];
+    }
+  for (long j = 0; j < nb; ++j) {
+    double best = -std::numeric_limits<double>::infinity();
+    for (int i = 0; i < B; ++i) {
+      double s = 0.0;
+      for (int c = 0; c < r; ++c) s += u[static_cast<size_t>(i) * r + c] * C[j * r + c];
+      best = std::max(best, s);
+    }
+    out[j] = best;
+  }
+}
+
+// The fixed selection rule (as oracle_select) on row-max scores, for the
+// query blocks t_list[0..nq).
+void oracle_select_rowmax(const uint16_t* q, int G, long N, int D, int B, const float* P, int r, const double* C,
+                          long nb, const int32_t* t_list, long nq, int topk, int n_local, int kmax, int32_t* sel,
+                          int32_t* cnt, double* kth_score) {
+  parallel_for(nq, [&](long x) {
+    std::vector<double> s(nb);
+    oracle_rowmax_scores(q, G, N, D, B, P, r, C, nb, t_list[x], s.data());
+    select_row(s, t_list[x], topk, n_local, kmax, sel + x * kmax, cnt + x, kth_score + x);
   });
 }
 

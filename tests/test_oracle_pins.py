@@ -277,6 +277,67 @@ def test_selection_small_t_is_full_causal():
         assert list(sel[t, : cnt[t]]) == list(range(t + 1))
 
 
+# ------------------------------------------------------------ row-max scores
+
+
+def brute_rowmax_scores(q_group, proj, C, t, block):
+    """u_i = sum_h q_{h,i} P (fp64, numpy), s_j = max_i u_i . c_j."""
+    qg = widen(q_group)[:, t * block:(t + 1) * block]  # [G, B, 128]
+    U = qg.sum(axis=0) @ np.asarray(proj, dtype=np.float64)
+    return (U @ np.asarray(C, dtype=np.float64).T).max(axis=0)
+
+
+@pytest.mark.parametrize("G,n,block,topk,n_local", [(2, 512, 64, 3, 1), (4, 1024, 128, 2, 2), (1, 640, 64, 20, 1)])
+def test_rowmax_selection_matches_bruteforce(G, n, block, topk, n_local):
+    g = torch.Generator().manual_seed(G * 1000 + n)
+    q = torch.randn(G, n, 128, generator=g).to(torch.bfloat16)
+    k = torch.randn(n, 128, generator=g).to(torch.bfloat16)
+    proj = torch.randn(128, 16, generator=g) / 11.3
+    C = oracle.centroids(k, block, proj)
+    nb = n // block
+    sel, cnt, kth = oracle.select_rowmax(q, proj, C, np.arange(nb), block, topk, n_local)
+    for t in range(nb):
+        s = brute_rowmax_scores(q, proj, C, t, block)
+        np.testing.assert_allclose(oracle.rowmax_scores(q, proj, C, t, block), s, rtol=1e-12, atol=1e-12)
+        cands = list(range(1, t - n_local + 1))
+        if len(cands) > topk:
+            cands = sorted(cands, key=lambda j: (-s[j], j))[:topk]
+        ref = sorted(set(cands) | {0} | set(range(max(0, t - n_local + 1), t + 1)))
+        assert list(sel[t, :cnt[t]]) == ref and np.all(sel[t, cnt[t]:] == -1)
+
+
+def test_rowmax_with_identical_rows_equals_mean_selection():
+    # every row of a block equal (per head): the row maximum is the block mean,
+    # so the scores and the selection are those of the query-block summaries
+    G, n, block, topk, n_local = 3, 768, 64, 4, 2
+    g = torch.Generator().manual_seed(5)
+    rows = torch.randn(G, n // block, 1, 128, generator=g).expand(G, n // block, block, 128)
+    q = rows.reshape(G, n, 128).to(torch.bfloat16)
+    k = torch.randn(n, 128, generator=g).to(torch.bfloat16)
+    proj = torch.randn(128, 16, generator=g) / 11.3
+    C = oracle.centroids(k, block, proj)
+    qb = oracle.qbar(q, block, proj)
+    nb = n // block
+    for t in range(nb):
+        np.testing.assert_allclose(oracle.rowmax_scores(q, proj, C, t, block), oracle.scores(qb[t], C),
+                                   rtol=1e-12, atol=1e-12)
+    a = oracle.select_rowmax(q, proj, C, np.arange(nb), block, topk, n_local)
+    b = oracle.select(qb, C, np.arange(nb), topk, n_local)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
+def test_rowmax_score_bounds_the_mean_score():
+    G, n, block = 2, 512, 128
+    g = torch.Generator().manual_seed(6)
+    q = torch.randn(G, n, 128, generator=g).to(torch.bfloat16)
+    k = torch.randn(n, 128, generator=g).to(torch.bfloat16)
+    proj = torch.randn(128, 16, generator=g) / 11.3
+    C = oracle.centroids(k, block, proj)
+    qb = oracle.qbar(q, block, proj)
+    for t in range(n // block):
+        assert np.all(oracle.rowmax_scores(q, proj, C, t, block) >= oracle.scores(qb[t], C) - 1e-12)
+
+
 # --------------------------------------------------------------------- decode
 
 
