@@ -340,6 +340,25 @@ def time_dynamic(rtp, w, res, device, points=((0.9, None), (0.99, None), (0.9, 1
             "fixed_blocks_per_query_block": float(np.mean([selected_count(t, w.topk, w.n_local) for t in range(nb)])),
             "algorithmic_tflops": flops / (pre_ms * 1e-3) / 1e12,
             "needle_recall": needle_recall(res["needles"], slot_of, sel, cnt, B)}
+    # the fixed top-k on row-max scores (largest low-rank logit over a query
+    # block's rows instead of the block mean); same budget, so the prefill
+    # time only moves with the tiles' masks
+    sel, cnt = torch.empty_like(bufs["sel"]), torch.empty_like(bufs["sel_cnt"])
+    for _ in range(2):
+        rtp.rtp_block_select_rowmax(plan.handle, q, res["proj"], bufs["centroids"], sel, cnt, stream)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    torch.cuda.synchronize()
+    for e in ev:
+        e[0].record(stream)
+        rtp.rtp_block_select_rowmax(plan.handle, q, res["proj"], bufs["centroids"], sel, cnt, stream)
+        e[1].record(stream)
+        rtp.rtp_hybrid_prefill(plan.handle, q, k, v, sel, cnt, o, stream)
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    out["rowmax_scores"] = {
+        "select_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
+        "prefill_ms": statistics.mean(e[1].elapsed_time(e[2]) for e in ev),
+        "needle_recall": needle_recall(res["needles"], slot_of, sel, cnt, B)}
     return out
 
 

@@ -216,6 +216,31 @@ rtp_status rtp_block_select_dynamic(const rtp_plan* plan, const float* qbar, con
                                     int min_k, float beta, int32_t* sel, int32_t* sel_cnt, void* stream);
 
 /* ------------------------------------------------------------------------
+ * rtp_block_select_rowmax — the fixed top-k rule with another score: a
+ * query block scores a candidate by the largest low-rank logit over its rows
+ * instead of the mean (RTPurboV2 page: the query-side aggregate of the
+ * indexer is left open; one row pointing at a block is then enough to keep
+ * it):
+ *   s_j = max_{i in block t} u_i . c_j,  u_i = P^T sum_{h in group} q_{h,i}
+ *   (u_i in fp32: the group's bf16 rows summed in head order, projected with
+ *   a fixed summation order; each dot product in the order of
+ *   rtp_block_select); keep the topk best candidates 1..t-n_local by (score
+ *   desc, index asc), block 0 and the local blocks, as rtp_block_select.
+ *   q          the plan's query rows, as for rtp_hybrid_prefill
+ *   proj       fp32 [128][16]
+ *   centroids  as written by rtp_indexer_project
+ *   sel, sel_cnt  as in rtp_block_select (same layout), so the result feeds
+ *             rtp_hybrid_prefill unchanged
+ * Work: block x 16 FMA per candidate and query block (7.7 ms on B200 for
+ * the 1M-token retrieval head with block 128, against 0.96 ms for the mean
+ * scores) on top of one more read of the group's Q rows.
+ * Errors: RTP_ERR_INVALID_ARG (bad plan or pointer; nothing launched),
+ * RTP_ERR_CUDA.
+ * ---------------------------------------------------------------------- */
+rtp_status rtp_block_select_rowmax(const rtp_plan* plan, const void* q, const float* proj, const float* centroids,
+                                   int32_t* sel, int32_t* sel_cnt, void* stream);
+
+/* ------------------------------------------------------------------------
  * rtp_hybrid_prefill — causal prefill attention over the routing map.
  * RTPurbo page (streaming heads: SWA; full heads: dense causal) and
  * RTPurboV2 page / "Full Attention Strikes Back" summary (sparse heads:

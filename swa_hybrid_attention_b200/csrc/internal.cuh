@@ -52,6 +52,11 @@ struct SelectArgs {
   float mass;
   int min_k;
   float beta_log2;
+  // row-max scores only: the plan's query rows and the projector
+  const __nv_bfloat16* q;  // [batch][n_q_heads][q_slab][128], row 0 = query row q_row0
+  const float* proj;       // [128][16]
+  const int32_t* slot_heads;
+  int n_q_heads, n_kv_heads, group, block, q_row0, q_slab;
 };
 constexpr int kDynMaxCap = 1024;  // largest top-k cap of the dynamic selection
 
@@ -140,6 +145,7 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& mq, const CU
 cudaError_t launch_indexer(const IndexerArgs& a, cudaStream_t stream);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
 cudaError_t launch_select_dynamic(const SelectArgs& a, cudaStream_t stream);
+cudaError_t launch_select_rowmax(const SelectArgs& a, cudaStream_t stream);
 // mks / mvs: the cluster-ordered K/V of clustered mode (any valid map otherwise).
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mks,
                           const CUtensorMap& mvs, cudaStream_t stream);

@@ -461,6 +461,39 @@ rtp_status rtp_block_select_dynamic(const rtp_plan* plan, const float* qbar, con
   return cuda_status(launch_select_dynamic(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+rtp_status rtp_block_select_rowmax(const rtp_plan* plan, const void* q, const float* proj, const float* centroids,
+                                   int32_t* sel, int32_t* sel_cnt, void* stream) {
+  CallRange range_("rtp_block_select_rowmax");
+  if (!plan) return RTP_ERR_INVALID_ARG;
+  if (plan->n_sparse == 0) return RTP_OK;
+  if (!q || !proj || !centroids || !sel || !sel_cnt) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(proj) || !aligned16(centroids) || !aligned16(sel) || !aligned16(sel_cnt))
+    return RTP_ERR_INVALID_ARG;
+  const rtp_attn_cfg& c = plan->cfg;
+  SelectArgs a = {};
+  a.centroids = centroids;
+  a.sel = sel;
+  a.cnt = sel_cnt;
+  a.batch = c.batch;
+  a.n_sparse = plan->n_sparse;
+  a.nb = plan->nqb;
+  a.topk = c.topk;
+  a.n_local = c.n_local;
+  a.kmax = c.topk + 1 + c.n_local;
+  a.t0 = plan->q_begin / c.block;
+  a.n_rows = plan->q_end / c.block - a.t0;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.proj = proj;
+  a.slot_heads = plan->d_slot_heads;
+  a.n_q_heads = c.n_q_heads;
+  a.n_kv_heads = c.n_kv_heads;
+  a.group = c.n_q_heads / c.n_kv_heads;
+  a.block = c.block;
+  a.q_row0 = plan->q_begin;
+  a.q_slab = plan->q_end - plan->q_begin;
+  return cuda_status(launch_select_rowmax(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 rtp_status rtp_hybrid_prefill(const rtp_plan* plan, const void* q, const void* k, const void* v,
                               const int32_t* sel, const int32_t* sel_cnt, void* o, void* stream) {
   CallRange range_("rtp_hybrid_prefill");

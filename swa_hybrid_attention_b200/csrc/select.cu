@@ -19,6 +19,8 @@
 //     at T go to the lowest indices.
 // The centroids of one (slot, sequence) are 16 fp32 per block and stay in L2.
 
+#include <cuda_bf16.h>
+
 #include "internal.cuh"
 #include "select_common.cuh"
 
@@ -246,6 +248,113 @@ __global__ void __launch_bounds__(kSelThreads) block_select_dynamic_kernel(const
   for (int e = 1 + nstar + a.n_local + tid; e < a.kmax; e += kSelThreads) out[e] = -1;
 }
 
+// ------------------------------------------------------------ row-max scores
+//
+// The same page's criticism of one fixed policy also leaves open how a query
+// block should score a candidate.  Besides the mean (the summary qbar_t), the
+// library offers the largest low-rank logit over the block's rows:
+//   s_j = max_{i in block t} u_i . c_j,   u_i = P^T sum_{h in group} q_{h,i},
+// so that one query row pointing at a block is enough to keep it.  Selection
+// rule and output are those of the fixed policy (top-k by score desc, index
+// asc; sink and local blocks added).
+//
+// Per CTA (one query block): 1. u_i of the block's rows into shared memory
+// (16 threads per row sum the group's heads over 8 dims each and project;
+// the 16 partial dot products of a rank are added in a fixed butterfly, lane
+// 0's result kept); 2. one candidate per thread: its centroid in registers,
+// the rows' u_i read as shared-memory broadcasts, max over rows of the fixed-
+// order 16-term dot product; 3. the fixed kernel's radix select and ordered
+// compaction.
+
+constexpr int kRowmaxCands = 4;
+
+struct RowmaxScratch {
+  float proj[kHeadDim * kRank];
+  float u[128][kRank];  // block <= 128 rows
+};
+
+__global__ void __launch_bounds__(kSelThreads) block_select_rowmax_kernel(const SelectArgs a) {
+  extern __shared__ uint32_t keys[];
+  __shared__ SelectScratch sh;
+  __shared__ __align__(16) RowmaxScratch rs;
+  const int t = a.t0 + static_cast<int>(blockIdx.x), slot = blockIdx.y, b = blockIdx.z;
+  const size_t row = (static_cast<size_t>(b) * a.n_sparse + slot) * a.nb + t;
+  int32_t* out = a.sel + row * a.kmax;
+  const int tid = threadIdx.x;
+  if (const int n = select_without_scores(t, a.topk, a.n_local, a.kmax, out); n >= 0) {
+    if (tid == 0) a.cnt[row] = n;
+    return;
+  }
+  const int ncand = t - a.n_local;
+  const int kvh = a.slot_heads[slot];
+  for (int e = tid; e < kHeadDim * kRank; e += kSelThreads) rs.proj[e] = a.proj[e];
+  __syncthreads();
+  // 1. u_i
+  {
+    const int rg = tid >> 4, cg = tid & 15;
+    for (int i0 = 0; i0 < a.block; i0 += kSelThreads / 16) {
+      const int i = i0 + rg;
+      const size_t qrow = static_cast<size_t>(t) * a.block + i - a.q_row0;
+      float sum[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int h = 0; h < a.group; ++h) {
+        const __nv_bfloat16* qp =
+            a.q + ((static_cast<size_t>(b) * a.n_q_heads + kvh * a.group + h) * a.q_slab + qrow) * kHeadDim + 8 * cg;
+        const uint4 raw = *reinterpret_cast<const uint4*>(qp);
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(p2[e]);
+          sum[2 * e] += f.x;
+          sum[2 * e + 1] += f.y;
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < kRank; ++c) {
+        float v = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v = fmaf(rs.proj[(8 * cg + e) * kRank + c], sum[e], v);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        if (cg == 0) rs.u[i][c] = v;
+      }
+    }
+  }
+  __syncthreads();
+  // 2. scores -> order keys: kRowmaxCands candidates per thread share each
+  // row's shared-memory read
+  const float* C = a.centroids + (static_cast<size_t>(b) * a.n_sparse + slot) * a.nb * kRank;
+  for (int x0 = tid; x0 < ncand; x0 += kRowmaxCands * kSelThreads) {
+    float4 cv[kRowmaxCands][4];
+    float best[kRowmaxCands];
+#pragma unroll
+    for (int u = 0; u < kRowmaxCands; ++u) {
+      const int x = min(x0 + u * kSelThreads, ncand - 1);
+      const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + 1) * kRank);
+#pragma unroll
+      for (int w = 0; w < 4; ++w) cv[u][w] = __ldg(c4 + w);
+      best[u] = -INFINITY;
+    }
+    for (int i = 0; i < a.block; ++i) {
+      const float4* u4 = reinterpret_cast<const float4*>(rs.u[i]);
+      const float4 u0 = u4[0], u1 = u4[1], u2 = u4[2], u3 = u4[3];
+      const float uq[kRank] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w,
+                               u2.x, u2.y, u2.z, u2.w, u3.x, u3.y, u3.z, u3.w};
+#pragma unroll
+      for (int u = 0; u < kRowmaxCands; ++u) best[u] = fmaxf(best[u], score16(uq, cv[u]));
+    }
+#pragma unroll
+    for (int u = 0; u < kRowmaxCands; ++u) {
+      const int x = x0 + u * kSelThreads;
+      if (x < ncand) keys[x] = order_key(best[u]);
+    }
+  }
+  __syncthreads();
+  const int n = select_from_keys(keys, ncand, t, a.topk, a.n_local, a.kmax, sh, out);
+  if (tid == 0) a.cnt[row] = n;
+}
+
 }  // namespace
 
 cudaError_t launch_select_dynamic(const SelectArgs& a, cudaStream_t stream) {
@@ -259,6 +368,20 @@ cudaError_t launch_select_dynamic(const SelectArgs& a, cudaStream_t stream) {
   if (a.n_rows == 0) return cudaSuccess;
   dim3 grid(a.n_rows, a.n_sparse, a.batch);
   block_select_dynamic_kernel<<<grid, kSelThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select_rowmax(const SelectArgs& a, cudaStream_t stream) {
+  if (a.n_sparse == 0) return cudaSuccess;
+  const size_t smem = static_cast<size_t>(a.nb) * sizeof(uint32_t);
+  if (smem + sizeof(RowmaxScratch) + sizeof(SelectScratch) > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(block_select_rowmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  if (a.n_rows == 0) return cudaSuccess;
+  dim3 grid(a.n_rows, a.n_sparse, a.batch);
+  block_select_rowmax_kernel<<<grid, kSelThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 

@@ -165,6 +165,40 @@ __device__ __forceinline__ float score16(const float (&q)[kRank], const float4 (
   return s;
 }
 
+// Steps 2 and 3 of a selection once the candidates' order keys are in
+// shared memory (ncand > topk >= 1): the topk-th largest key, then the
+// ordered compaction into out[1..topk], plus the sink and the local blocks.
+// Must be called by all kSelThreads threads of the CTA.
+__device__ inline int select_from_keys(const uint32_t* keys, int ncand, int t, int topk, int n_local, int kmax,
+                                       SelectScratch& sh, int32_t* out) {
+  const int tid = threadIdx.x;
+  uint32_t T, need;
+  radix_threshold<kSelThreads>(keys, ncand, topk, sh, T, need);
+  ordered_select<kSelThreads>(keys, ncand, T, need, sh, [&](int r, int x) { out[1 + r] = x + 1; });
+  if (tid == 0) out[0] = 0;
+  for (int m = tid; m < n_local; m += kSelThreads) out[1 + topk + m] = t - n_local + 1 + m;
+  for (int e = 1 + topk + n_local + tid; e < kmax; e += kSelThreads) out[e] = -1;
+  return 1 + topk + n_local;
+}
+
+// The selections that need no scores: every block 0..t when there are at
+// most topk candidates, or only the sink and local blocks when topk is 0.
+// Returns the count, or -1 if scores are needed.
+__device__ inline int select_without_scores(int t, int topk, int n_local, int kmax, int32_t* out) {
+  const int tid = threadIdx.x;
+  const int ncand = t - n_local > 0 ? t - n_local : 0;
+  if (ncand <= topk) {
+    const int n = t + 1;
+    for (int e = tid; e < kmax; e += kSelThreads) out[e] = e < n ? e : -1;
+    return n;
+  }
+  if (topk == 0) {
+    for (int e = tid; e < kmax; e += kSelThreads) out[e] = e == 0 ? 0 : (e <= n_local ? t - n_local + e : -1);
+    return 1 + n_local;
+  }
+  return -1;
+}
+
 // Selects the blocks of query block t.  Must be called by all kSelThreads
 // threads of the CTA.  q: the query summary (16 fp32); C: centroids of this
 // (slot, sequence), [>= t-n_local+1][16] fp32; keys: shared scratch of at
@@ -174,15 +208,8 @@ __device__ inline int select_blocks(const float (&q)[kRank], const float* C, int
                                     uint32_t* keys, SelectScratch& sh, int32_t* out) {
   const int tid = threadIdx.x;
   const int ncand = t - n_local > 0 ? t - n_local : 0;  // candidates are blocks 1..ncand
-  if (ncand <= topk) {
-    const int n = t + 1;
-    for (int e = tid; e < kmax; e += kSelThreads) out[e] = e < n ? e : -1;
-    return n;
-  }
-  if (topk == 0) {  // sink and local blocks only (the radix select needs k >= 1)
-    for (int e = tid; e < kmax; e += kSelThreads) out[e] = e == 0 ? 0 : (e <= n_local ? t - n_local + e : -1);
-    return 1 + n_local;
-  }
+  // (top-k 0: sink and local blocks only; the radix select needs k >= 1)
+  if (const int n = select_without_scores(t, topk, n_local, kmax, out); n >= 0) return n;
   // 1. scores -> order keys.  Four candidates per round with all their
   // loads issued before any use, so a thread keeps 16 independent 16-byte
   // loads in flight.
@@ -202,14 +229,7 @@ __device__ inline int select_blocks(const float (&q)[kRank], const float* C, int
     }
   }
   __syncthreads();
-  // 2. the topk-th largest key; 3. ordered compaction into out[1..topk]
-  uint32_t T, need;
-  radix_threshold<kSelThreads>(keys, ncand, topk, sh, T, need);
-  ordered_select<kSelThreads>(keys, ncand, T, need, sh, [&](int r, int x) { out[1 + r] = x + 1; });
-  if (tid == 0) out[0] = 0;
-  for (int m = tid; m < n_local; m += kSelThreads) out[1 + topk + m] = t - n_local + 1 + m;
-  for (int e = 1 + topk + n_local + tid; e < kmax; e += kSelThreads) out[e] = -1;
-  return 1 + topk + n_local;
+  return select_from_keys(keys, ncand, t, topk, n_local, kmax, sh, out);
 }
 
 }  // namespace rtp

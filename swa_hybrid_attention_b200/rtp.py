@@ -65,6 +65,7 @@ def _load() -> ctypes.CDLL:
         "rtp_indexer_project": (I, [P, P, P, P, P, P, P]),
         "rtp_block_select": (I, [P, P, P, P, P, P]),
         "rtp_block_select_dynamic": (I, [P, P, P, ctypes.c_float, I, ctypes.c_float, P, P, P]),
+        "rtp_block_select_rowmax": (I, [P, P, P, P, P, P, P]),
         "rtp_hybrid_prefill": (I, [P, P, P, P, P, P, P, P]),
         "rtp_pipeline_create": (I, [cfgp, P, I, P, ctypes.POINTER(P)]),
         "rtp_pipeline_destroy": (None, [P]),
@@ -93,7 +94,7 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 EXPORTED = ("rtp_route_heads", "rtp_route_heads_range", "rtp_plan_destroy", "rtp_plan_num_sparse", "rtp_plan_num_items",
             "rtp_plan_sparse_heads", "rtp_plan_work_items", "rtp_indexer_project", "rtp_block_select",
-            "rtp_block_select_dynamic", "rtp_pipeline_create", "rtp_pipeline_destroy", "rtp_hybrid_prefill_host",
+            "rtp_block_select_dynamic", "rtp_block_select_rowmax", "rtp_pipeline_create", "rtp_pipeline_destroy", "rtp_hybrid_prefill_host",
             "rtp_hybrid_prefill", "rtp_decode_workspace_bytes", "rtp_sparse_decode", "rtp_sparse_decode_noalloc",
             "rtp_cache_centroids", "rtp_cache_append", "rtp_cache_cluster_workspace_bytes", "rtp_cache_cluster",
             "rtp_decode_clustered_workspace_bytes", "rtp_sparse_decode_clustered",
@@ -220,6 +221,12 @@ def rtp_block_select_dynamic(plan: int, qbar, centroids, mass: float, min_k: int
     _check("rtp_block_select_dynamic",
            _lib.rtp_block_select_dynamic(plan, _ptr(qbar), _ptr(centroids), float(mass), int(min_k), float(beta),
                                          _ptr(sel), _ptr(sel_cnt), _stream(stream)))
+
+
+def rtp_block_select_rowmax(plan: int, q, proj, centroids, sel, sel_cnt, stream=None) -> None:
+    _check("rtp_block_select_rowmax",
+           _lib.rtp_block_select_rowmax(plan, _ptr(q), _ptr(proj), _ptr(centroids), _ptr(sel), _ptr(sel_cnt),
+                                        _stream(stream)))
 
 
 def default_selection_beta(cfg: AttnConfig) -> float:
@@ -437,16 +444,25 @@ class Plan:
             sel_cnt=torch.empty(c.batch, ns, nb, dtype=torch.int32, device=device),
         )
 
-    def run(self, q, k, v, proj, o, bufs: dict, stream=None, dynamic: dict | None = None) -> None:
+    def run(self, q, k, v, proj, o, bufs: dict, stream=None, dynamic: dict | None = None,
+            score: str = "mean") -> None:
         """One layer: indexer + selection (if any retrieval slot) + prefill.
 
         dynamic: None for the fixed top-k selection, else a dict with `mass`
         and optionally `min_k` (default 0) and `beta` (default: softmax scale
         / group) for rtp_block_select_dynamic (topk is then the cap).
+        score: "mean" (the query-block summary) or "rowmax" (the largest
+        low-rank logit over the block's rows, rtp_block_select_rowmax) for the
+        fixed top-k selection.
         """
+        if score not in ("mean", "rowmax") or (score == "rowmax" and dynamic is not None):
+            raise RtpError("Plan.run", RTP_ERR_INVALID_ARG)
         if self.n_sparse > 0:
             rtp_indexer_project(self.handle, q, k, proj, bufs["centroids"], bufs["qbar"], stream)
-            if dynamic is None:
+            if score == "rowmax":
+                rtp_block_select_rowmax(self.handle, q, proj, bufs["centroids"], bufs["sel"], bufs["sel_cnt"],
+                                        stream)
+            elif dynamic is None:
                 rtp_block_select(self.handle, bufs["qbar"], bufs["centroids"], bufs["sel"], bufs["sel_cnt"], stream)
             else:
                 beta = dynamic.get("beta")
