@@ -359,6 +359,36 @@ def time_dynamic(rtp, w, res, device, points=((0.9, None), (0.99, None), (0.9, 1
         "select_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
         "prefill_ms": statistics.mean(e[1].elapsed_time(e[2]) for e in ev),
         "needle_recall": needle_recall(res["needles"], slot_of, sel, cnt, B)}
+    # one selection per query head (same top-k per head); the pair of heads
+    # in a CTA streams the union of its two lists
+    if B == 128 and G % 2 == 0:
+        qh = torch.empty(w.batch, plan.n_sparse, G, nb, 16, dtype=torch.float32, device=device)
+        sh = torch.empty(w.batch, plan.n_sparse, G, nb, plan.cfg.kmax, dtype=torch.int32, device=device)
+        ch = torch.empty(w.batch, plan.n_sparse, G, nb, dtype=torch.int32, device=device)
+        for _ in range(2):
+            rtp.rtp_indexer_project_heads(plan.handle, q, res["proj"], qh, stream)
+            rtp.rtp_block_select_heads(plan.handle, qh, bufs["centroids"], sh, ch, stream)
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+        torch.cuda.synchronize()
+        for e in ev:
+            e[0].record(stream)
+            rtp.rtp_indexer_project_heads(plan.handle, q, res["proj"], qh, stream)
+            rtp.rtp_block_select_heads(plan.handle, qh, bufs["centroids"], sh, ch, stream)
+            e[1].record(stream)
+            rtp.rtp_hybrid_prefill_heads(plan.handle, q, k, v, sh, ch, o, stream)
+            e[2].record(stream)
+        torch.cuda.synchronize()
+        hit = 0
+        sh_c, ch_c = sh.cpu(), ch.cpu()
+        for kvh, hq_, tq, j in res["needles"]:
+            t = tq // B
+            row = sh_c[0, slot_of[kvh], hq_ % G, t, :int(ch_c[0, slot_of[kvh], hq_ % G, t])]
+            hit += int((row == j // B).any())
+        out["per_head"] = {
+            "select_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
+            "prefill_ms": statistics.mean(e[1].elapsed_time(e[2]) for e in ev),
+            "needle_recall": hit / len(res["needles"]) if res["needles"] else None}
+        del qh, sh, ch
     return out
 
 

@@ -241,6 +241,40 @@ rtp_status rtp_block_select_rowmax(const rtp_plan* plan, const void* q, const fl
                                    int32_t* sel, int32_t* sel_cnt, void* stream);
 
 /* ------------------------------------------------------------------------
+ * Per-head selection — the other query-side alternative: every query head
+ * selects its own blocks instead of its group sharing one list (RTPurboV2
+ * page: the indexer scores query against key summaries; which query rows
+ * share a selection is left open).  Three calls, for a whole-sequence plan
+ * with block 128 and an even group (else RTP_ERR_UNSUPPORTED):
+ *
+ * rtp_indexer_project_heads — qbar_{h,t} = (1/B) sum_{i in block t} P^T q_{h,i}
+ *   for every head h of every retrieval slot's group:
+ *   qbar_heads  fp32 [batch][n_sparse][group][seq/block][16] (out); for a
+ *               group of one head it is rtp_indexer_project's qbar
+ *   (the centroids come from rtp_indexer_project, which is still needed)
+ *
+ * rtp_block_select_heads — the rule of rtp_block_select for each head's
+ *   summary against its slot's centroids:
+ *   sel      int32 [batch][n_sparse][group][seq/block][kmax] (out)
+ *   sel_cnt  int32 [batch][n_sparse][group][seq/block] (out)
+ *
+ * rtp_hybrid_prefill_heads — rtp_hybrid_prefill on per-head selections: head
+ *   h of a retrieval KV head attends to the blocks of its own list (with the
+ *   causal mask).  The two heads of a query-head pair share one stream of
+ *   K/V tiles, the union of their lists; a tile outside one head's list is
+ *   masked out for that head, so the work grows with how much the pair's
+ *   lists differ.
+ * Errors: RTP_ERR_INVALID_ARG (bad plan or pointer; nothing launched),
+ * RTP_ERR_UNSUPPORTED (ranged plan, block 64 or odd group), RTP_ERR_CUDA.
+ * ---------------------------------------------------------------------- */
+rtp_status rtp_indexer_project_heads(const rtp_plan* plan, const void* q, const float* proj, float* qbar_heads,
+                                     void* stream);
+rtp_status rtp_block_select_heads(const rtp_plan* plan, const float* qbar_heads, const float* centroids,
+                                  int32_t* sel, int32_t* sel_cnt, void* stream);
+rtp_status rtp_hybrid_prefill_heads(const rtp_plan* plan, const void* q, const void* k, const void* v,
+                                    const int32_t* sel, const int32_t* sel_cnt, void* o, void* stream);
+
+/* ------------------------------------------------------------------------
  * rtp_hybrid_prefill — causal prefill attention over the routing map.
  * RTPurbo page (streaming heads: SWA; full heads: dense causal) and
  * RTPurboV2 page / "Full Attention Strikes Back" summary (sparse heads:

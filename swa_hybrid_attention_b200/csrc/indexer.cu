@@ -84,7 +84,52 @@ __global__ void __launch_bounds__(kThreads) indexer_kernel(const IndexerArgs a) 
   }
 }
 
+// Per-head query summaries (selection per query head instead of per KV
+// head): qbar_{h,t} = (1/B) sum_{i in block t} P^T q_{h,i} for every head h
+// of every retrieval slot's group, written to qbar [batch][n_sparse][group]
+// [nb][16].  One CTA per (block, slot x head, sequence); the same row order,
+// row-group order and projection chain as the indexer, so for a group of one
+// head the summary is the indexer's number.
+__global__ void __launch_bounds__(kThreads) indexer_heads_kernel(const IndexerArgs a) {
+  __shared__ float part[kRowGroups][kHeadDim];
+  __shared__ float total[kHeadDim];
+  __shared__ float proj[kHeadDim * kRank];
+  const int blk = a.blk0 + static_cast<int>(blockIdx.x), b = blockIdx.z;
+  const int slot = static_cast<int>(blockIdx.y) / a.group, g = static_cast<int>(blockIdx.y) % a.group;
+  const int lrow = static_cast<int>(blockIdx.x) * a.block;
+  const int tid = threadIdx.x, rg = tid >> 4, cg = tid & 15;
+  const int hq = a.slot_heads[slot] * a.group + g;
+  for (int e = tid; e < kHeadDim * kRank; e += kThreads) proj[e] = a.proj[e];
+  float accq[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  const __nv_bfloat16* qbase =
+      a.q + ((static_cast<size_t>(b) * a.n_q_heads + hq) * a.rows + static_cast<size_t>(lrow)) * kHeadDim;
+  sum_rows(accq, qbase, a.block, rg, cg);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[rg][cg * 8 + e] = accq[e];
+  __syncthreads();
+  if (tid < kHeadDim) {
+    float s = 0.f;
+#pragma unroll
+    for (int r = 0; r < kRowGroups; ++r) s += part[r][tid];
+    total[tid] = s;
+  }
+  __syncthreads();
+  if (tid < kRank) {
+    float s = 0.f;
+    for (int d = 0; d < kHeadDim; ++d) s = fmaf(proj[d * kRank + tid], total[d], s);
+    s *= 1.0f / static_cast<float>(a.block);
+    a.qbar[(((static_cast<size_t>(b) * a.n_sparse + slot) * a.group + g) * (a.seq / a.block) + blk) * kRank + tid] = s;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_indexer_heads(const IndexerArgs& a, cudaStream_t stream) {
+  if (a.n_sparse == 0 || a.n_blocks == 0) return cudaSuccess;
+  dim3 grid(a.n_blocks, a.n_sparse * a.group, a.batch);
+  indexer_heads_kernel<<<grid, kThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_indexer(const IndexerArgs& a, cudaStream_t stream) {
   if (a.n_sparse == 0) return cudaSuccess;

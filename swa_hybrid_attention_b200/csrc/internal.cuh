@@ -26,6 +26,9 @@ struct PrefillArgs {
   int window, block, kmax, nqb;
   float scale_log2;  // softmax scale * log2(e)
   uint32_t* status;
+  // 0: one selection per (retrieval slot, query block), sel [batch][n_sparse][nqb][kmax];
+  // 1: one per query head, sel [batch][n_sparse][group][nqb][kmax] (block 128 only)
+  int sel_heads;
 };
 
 struct IndexerArgs {
@@ -48,6 +51,7 @@ struct SelectArgs {
   int32_t* cnt;
   int batch, n_sparse, nb, topk, n_local, kmax;
   int t0, n_rows;  // query blocks t0 .. t0 + n_rows - 1 are selected
+  int c_group;     // selection rows per centroid slot: 1, or the group size for per-head selection
   // dynamic selection only: mass fraction, minimum count, beta * log2(e)
   float mass;
   int min_k;
@@ -143,6 +147,7 @@ constexpr int kMaxClusters = 2048;
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                            int num_ctas, cudaStream_t stream);
 cudaError_t launch_indexer(const IndexerArgs& a, cudaStream_t stream);
+cudaError_t launch_indexer_heads(const IndexerArgs& a, cudaStream_t stream);
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t stream);
 cudaError_t launch_select_dynamic(const SelectArgs& a, cudaStream_t stream);
 cudaError_t launch_select_rowmax(const SelectArgs& a, cudaStream_t stream);

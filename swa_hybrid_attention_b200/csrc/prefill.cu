@@ -68,7 +68,7 @@ constexpr uint32_t kTileBytes = 128 * 128 * 2;  // one 128x128 bf16 operand tile
 constexpr uint32_t kChunkBytes = 128 * 128;     // 64 columns x 128 rows
 constexpr int kNoWindow = 1 << 30;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale when max grows > 2^8
-constexpr uint32_t kMemberAll = 0x1Eu;
+constexpr uint32_t kMemberAll = 0x1Eu | (3u << 5);
 // Column pairs (k mod 8) whose exponentials use the FMA-pipe polynomial
 // instead of the MUFU: bit k set => pair k.  Default: none — measured on B200
 // (1M-token layer) the polynomial costs more issue slots than the MUFU time
@@ -122,6 +122,8 @@ __device__ __forceinline__ Item load_item(const int4* items, long idx, int n_kv_
 // flags bit 0: the tile needs the element mask.  Bits 1..4: membership of
 // (half 0, query half 0), (half 0, query half 1), (half 1, query half 0),
 // (half 1, query half 1) — only block-64 sparse tiles clear any of them.
+// Bits 5..6: membership of the pair's head 0 / head 1 — only per-head
+// selections clear one of them (the tile is then the other head's).
 struct TileRef {
   int row0, row1;
   uint32_t flags;
@@ -129,13 +131,17 @@ struct TileRef {
 
 // Enumerates the KV tiles of one work item in ascending key order.  The
 // producer, the MMA issuer and the softmax warps each run their own copy.
+// kHeads: the selections are per query head (the pair's two lists are
+// merged); a separate instantiation, so the shared-selection kernel carries
+// none of its work.
+template <bool kHeads>
 struct TileIter {
   int kind, t, n, lo, q0, window, j;
   const int32_t* la;
   const int32_t* lb;
   int na, nb, ia, ib;
   int nblocks;  // valid block indices are < nblocks
-  bool b64;
+  bool b64, heads;
   uint32_t* status;
 
   __device__ void init(const Item& it, const PrefillArgs& a) {
@@ -145,6 +151,7 @@ struct TileIter {
     q0 = 128 * t;
     window = (kind == KIND_SWA) ? a.window : kNoWindow;
     b64 = false;
+    heads = false;
     status = a.status;
     nblocks = a.nqb;
     if (kind == KIND_FULL) {
@@ -154,6 +161,23 @@ struct TileIter {
       int first = q0 - a.window + 1;
       lo = first <= 0 ? 0 : first / 128;
       n = t - lo + 1;
+    } else if (kHeads && a.block == 128) {
+      // per-head selections: the union of the pair's two ascending lists
+      heads = true;
+      const long base = ((static_cast<long>(it.b) * a.n_sparse + it.slot) * a.group + 2 * it.pair) * a.nqb + t;
+      la = a.sel + base * a.kmax;
+      na = min(max(a.cnt[base], 0), a.kmax);
+      lb = la + static_cast<long>(a.nqb) * a.kmax;
+      nb = min(max(a.cnt[base + a.nqb], 0), a.kmax);
+      int x = 0, y = 0, u = 0;
+      while (x < na || y < nb) {
+        int va = x < na ? la[x] : INT_MAX, vb = y < nb ? lb[y] : INT_MAX;
+        if (va <= vb) ++x;
+        if (vb <= va) ++y;
+        ++u;
+      }
+      n = u;
+      ia = ib = 0;
     } else if (a.block == 128) {
       long base = (static_cast<long>(it.b) * a.n_sparse + it.slot) * a.nqb + t;
       la = a.sel + base * a.kmax;
@@ -220,6 +244,14 @@ struct TileIter {
       r.row1 = k0 + 64;
       bool full_visible = (k0 + 127 <= q0) && (k0 > q0 + 127 - window);
       r.flags = kMemberAll | (full_visible ? 0u : 1u);
+    } else if (kHeads && heads) {
+      int v = 0;
+      uint32_t m = 0;
+      pick(v, m);
+      const int blk = checked_block(v, t);
+      r.row0 = 128 * blk;
+      r.row1 = r.row0 + 64;
+      r.flags = 0x1Eu | (m << 5) | ((blk >= t || m != 3u) ? 1u : 0u);
     } else if (!b64) {
       int blk = checked_block(la[j], t);
       r.row0 = 128 * blk;
@@ -237,7 +269,7 @@ struct TileIter {
       v1 = checked_block(v1, 2 * t + 1);
       r.row0 = 64 * v0;
       r.row1 = 64 * v1;
-      r.flags = 1u | ((m0 & 1u) << 1) | ((m0 & 2u) << 1) | ((m1 & 1u) << 3) | ((m1 & 2u) << 3);
+      r.flags = 1u | ((m0 & 1u) << 1) | ((m0 & 2u) << 1) | ((m1 & 1u) << 3) | ((m1 & 2u) << 3) | (3u << 5);
     }
     ++j;
     return r;
@@ -259,6 +291,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // ------------------------------------------------------------------ producer
+template <bool kHeads>
 __device__ __noinline__ void run_producer(Smem& s, const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv,
                              const PrefillArgs& a, volatile int* abort) {
   uint32_t it = 0, gt = 0;
@@ -275,7 +308,7 @@ __device__ __noinline__ void run_producer(Smem& s, const CUtensorMap* mq, const 
       q_issued |= 1u << h;
     }
     {
-      TileIter ti;
+      TileIter<kHeads> ti;
       ti.init(item, a);
       for (int j = 0; j < ti.n; ++j, ++gt) {
         TileRef tr = ti.next();
@@ -372,6 +405,7 @@ __device__ __forceinline__ bool issue_pv_chunked(Smem& s, int h, uint32_t parity
   return true;
 }
 
+template <bool kHeads>
 __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& a, volatile int* abort) {
   const uint32_t id_qk = idesc_bf16_f32(128, 128, false);
   const uint32_t id_pv = idesc_bf16_f32(128, 128, true);
@@ -384,7 +418,7 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
   uint32_t it = 0, gt = 0, pc = 0;
   for (long idx = blockIdx.x; idx < a.n_items; idx += gridDim.x, ++it) {
     Item item = load_item(a.items, idx, a.n_kv_heads);
-    TileIter ti;
+    TileIter<kHeads> ti;
     ti.init(item, a);
     const int n = ti.n;
     if (!mma_wait(&s.q_full[0], it & 1u, abort, a.status)) goto drain;
@@ -445,6 +479,7 @@ drain:
 }
 
 // ------------------------------------------------------------------ softmax
+template <bool kHeads>
 __device__ __noinline__ void run_softmax(Smem& s, uint32_t tmem, int h, const PrefillArgs& a, volatile int* abort) {
   const int q4 = warp_id() & 3;
   const int row = q4 * 32 + lane_id();
@@ -455,7 +490,7 @@ __device__ __noinline__ void run_softmax(Smem& s, uint32_t tmem, int h, const Pr
   uint32_t it = 0, sc = 0;
   for (long idx = blockIdx.x; idx < a.n_items; idx += gridDim.x, ++it) {
     Item item = load_item(a.items, idx, a.n_kv_heads);
-    TileIter ti;
+    TileIter<kHeads> ti;
     ti.init(item, a);
     const int i = 128 * item.t + row;
     const int rh = row >> 6;
@@ -475,7 +510,8 @@ __device__ __noinline__ void run_softmax(Smem& s, uint32_t tmem, int h, const Pr
         for (int c = 0; c < 128; ++c) {
           const int half = c >> 6;
           const int key = (half ? tr.row1 : tr.row0) + (c & 63);
-          const bool member = (tr.flags >> (1 + 2 * half + rh)) & 1u;
+          const bool member = kHeads ? (((tr.flags >> (1 + 2 * half + rh)) & (tr.flags >> (5 + h))) & 1u) != 0
+                                     : ((tr.flags >> (1 + 2 * half + rh)) & 1u) != 0;
           if (!(member && key <= i && key > lo_key)) r[c] = __float_as_uint(-INFINITY);
         }
       }
@@ -572,6 +608,7 @@ __device__ __noinline__ void run_softmax(Smem& s, uint32_t tmem, int h, const Pr
   }
 }
 
+template <bool kHeads>
 __global__ void __launch_bounds__(kThreads, 1)
     hybrid_prefill_kernel(const __grid_constant__ CUtensorMap mq, const __grid_constant__ CUtensorMap mk,
                           const __grid_constant__ CUtensorMap mv, const __grid_constant__ PrefillArgs a) {
@@ -618,14 +655,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // barrier below converged.
   if (warp >= 4) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHighRegs));
-    run_softmax(s, tmem, (warp - 4) >> 2, a, abort);
+    run_softmax<kHeads>(s, tmem, (warp - 4) >> 2, a, abort);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kLowRegs));
     if (warp == 0) {
-      if (lane_id() == 0) run_producer(s, &mq, &mk, &mv, a, abort);
+      if (lane_id() == 0) run_producer<kHeads>(s, &mq, &mk, &mv, a, abort);
       __syncwarp();
     } else if (warp == 1) {
-      if (lane_id() == 0) run_mma(s, tmem, a, abort);
+      if (lane_id() == 0) run_mma<kHeads>(s, tmem, a, abort);
       __syncwarp();
     }
   }
@@ -642,8 +679,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t prefill_smem_bytes() { return sizeof(Smem) + 1024; }
 
-cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                           int num_ctas, cudaStream_t stream) {
+namespace {
+template <bool kHeads>
+cudaError_t launch_prefill_t(const PrefillArgs& a, const CUtensorMap& mq, const CUtensorMap& mk,
+                             const CUtensorMap& mv, int num_ctas, cudaStream_t stream) {
   static int configured_device = -1;
   int dev = 0;
   cudaGetDevice(&dev);
@@ -651,16 +690,23 @@ cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& mq, const CU
     // The setmaxnreg split is only valid for the register count it was sized
     // for; refuse to launch a build that compiled to anything else.
     cudaFuncAttributes attr;
-    cudaError_t e = cudaFuncGetAttributes(&attr, hybrid_prefill_kernel);
+    cudaError_t e = cudaFuncGetAttributes(&attr, hybrid_prefill_kernel<kHeads>);
     if (e != cudaSuccess) return e;
     if (attr.numRegs != kLaunchRegs) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(hybrid_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(hybrid_prefill_kernel<kHeads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(prefill_smem_bytes()));
     if (e != cudaSuccess) return e;
     configured_device = dev;
   }
-  hybrid_prefill_kernel<<<num_ctas, kThreads, prefill_smem_bytes(), stream>>>(mq, mk, mv, a);
+  hybrid_prefill_kernel<kHeads><<<num_ctas, kThreads, prefill_smem_bytes(), stream>>>(mq, mk, mv, a);
   return cudaGetLastError();
+}
+}  // namespace
+
+cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                           int num_ctas, cudaStream_t stream) {
+  return a.sel_heads ? launch_prefill_t<true>(a, mq, mk, mv, num_ctas, stream)
+                     : launch_prefill_t<false>(a, mq, mk, mv, num_ctas, stream);
 }
 
 }  // namespace rtp

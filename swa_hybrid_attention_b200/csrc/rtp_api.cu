@@ -213,7 +213,7 @@ rtp_status indexer_run(const rtp_plan* plan, const void* q, const void* k, int s
 // query row of slab 0, their slabs q_slab rows apart; k and v start at row 0,
 // their slabs kv_slab rows apart.
 rtp_status prefill_run(const rtp_plan* plan, const void* q, int q_slab, const void* k, const void* v, int kv_slab,
-                       const int32_t* sel, const int32_t* sel_cnt, void* o, void* stream) {
+                       const int32_t* sel, const int32_t* sel_cnt, void* o, void* stream, int sel_heads = 0) {
   if (!q || !k || !v || !o) return RTP_ERR_INVALID_ARG;
   if (plan->n_sparse > 0 && (!sel || !sel_cnt)) return RTP_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RTP_ERR_INVALID_ARG;
@@ -247,6 +247,7 @@ rtp_status prefill_run(const rtp_plan* plan, const void* q, int q_slab, const vo
   a.nqb = plan->nqb;
   a.scale_log2 = plan->scale * kLog2e;
   a.status = status_word(plan->device);
+  a.sel_heads = sel_heads;
   const int ctas = static_cast<int>(std::min<long>(plan->n_items, plan->num_sms));
   if (ctas <= 0) return RTP_OK;
   return cuda_status(launch_prefill(a, mq, mk, mv, ctas, reinterpret_cast<cudaStream_t>(stream)));
@@ -414,7 +415,8 @@ rtp_status rtp_block_select(const rtp_plan* plan, const float* qbar, const float
   if (!aligned16(qbar) || !aligned16(centroids) || !aligned16(sel) || !aligned16(sel_cnt))
     return RTP_ERR_INVALID_ARG;
   const rtp_attn_cfg& c = plan->cfg;
-  SelectArgs a;
+  SelectArgs a = {};
+  a.c_group = 1;
   a.qbar = qbar;
   a.centroids = centroids;
   a.sel = sel;
@@ -442,7 +444,8 @@ rtp_status rtp_block_select_dynamic(const rtp_plan* plan, const float* qbar, con
   if (!qbar || !centroids || !sel || !sel_cnt) return RTP_ERR_INVALID_ARG;
   if (!aligned16(qbar) || !aligned16(centroids) || !aligned16(sel) || !aligned16(sel_cnt))
     return RTP_ERR_INVALID_ARG;
-  SelectArgs a;
+  SelectArgs a = {};
+  a.c_group = 1;
   a.qbar = qbar;
   a.centroids = centroids;
   a.sel = sel;
@@ -471,6 +474,7 @@ rtp_status rtp_block_select_rowmax(const rtp_plan* plan, const void* q, const fl
     return RTP_ERR_INVALID_ARG;
   const rtp_attn_cfg& c = plan->cfg;
   SelectArgs a = {};
+  a.c_group = 1;
   a.centroids = centroids;
   a.sel = sel;
   a.cnt = sel_cnt;
@@ -492,6 +496,77 @@ rtp_status rtp_block_select_rowmax(const rtp_plan* plan, const void* q, const fl
   a.q_row0 = plan->q_begin;
   a.q_slab = plan->q_end - plan->q_begin;
   return cuda_status(launch_select_rowmax(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// Per-head selection: a whole-sequence plan with 128-key blocks and an even
+// group (the prefill pairs the heads of a group).
+static bool per_head_ok(const rtp_plan* plan) {
+  const rtp_attn_cfg& c = plan->cfg;
+  const int group = c.n_q_heads / c.n_kv_heads;
+  return plan->q_begin == 0 && plan->q_end == c.seq && c.block == 128 && group % 2 == 0;
+}
+
+rtp_status rtp_indexer_project_heads(const rtp_plan* plan, const void* q, const float* proj, float* qbar_heads,
+                                     void* stream) {
+  CallRange range_("rtp_indexer_project_heads");
+  if (!plan) return RTP_ERR_INVALID_ARG;
+  if (!per_head_ok(plan)) return RTP_ERR_UNSUPPORTED;
+  if (plan->n_sparse == 0) return RTP_OK;
+  if (!q || !proj || !qbar_heads || !aligned16(q) || !aligned16(proj) || !aligned16(qbar_heads))
+    return RTP_ERR_INVALID_ARG;
+  const rtp_attn_cfg& c = plan->cfg;
+  IndexerArgs a = {};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.proj = proj;
+  a.qbar = qbar_heads;
+  a.slot_heads = plan->d_slot_heads;
+  a.batch = c.batch;
+  a.seq = c.seq;
+  a.n_q_heads = c.n_q_heads;
+  a.n_kv_heads = c.n_kv_heads;
+  a.group = c.n_q_heads / c.n_kv_heads;
+  a.n_sparse = plan->n_sparse;
+  a.block = c.block;
+  a.blk0 = 0;
+  a.rows = c.seq;
+  a.n_blocks = c.seq / c.block;
+  return cuda_status(launch_indexer_heads(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rtp_status rtp_block_select_heads(const rtp_plan* plan, const float* qbar_heads, const float* centroids,
+                                  int32_t* sel, int32_t* sel_cnt, void* stream) {
+  CallRange range_("rtp_block_select_heads");
+  if (!plan) return RTP_ERR_INVALID_ARG;
+  if (!per_head_ok(plan)) return RTP_ERR_UNSUPPORTED;
+  if (plan->n_sparse == 0) return RTP_OK;
+  if (!qbar_heads || !centroids || !sel || !sel_cnt) return RTP_ERR_INVALID_ARG;
+  if (!aligned16(qbar_heads) || !aligned16(centroids) || !aligned16(sel) || !aligned16(sel_cnt))
+    return RTP_ERR_INVALID_ARG;
+  const rtp_attn_cfg& c = plan->cfg;
+  const int group = c.n_q_heads / c.n_kv_heads;
+  SelectArgs a = {};
+  a.c_group = group;  // selection row (slot, head) scores against the slot's centroids
+  a.qbar = qbar_heads;
+  a.centroids = centroids;
+  a.sel = sel;
+  a.cnt = sel_cnt;
+  a.batch = c.batch;
+  a.n_sparse = plan->n_sparse * group;
+  a.nb = plan->nqb;
+  a.topk = c.topk;
+  a.n_local = c.n_local;
+  a.kmax = c.topk + 1 + c.n_local;
+  a.t0 = 0;
+  a.n_rows = plan->nqb;
+  return cuda_status(launch_select(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+rtp_status rtp_hybrid_prefill_heads(const rtp_plan* plan, const void* q, const void* k, const void* v,
+                                    const int32_t* sel, const int32_t* sel_cnt, void* o, void* stream) {
+  CallRange range_("rtp_hybrid_prefill_heads");
+  if (!plan) return RTP_ERR_INVALID_ARG;
+  if (!per_head_ok(plan)) return RTP_ERR_UNSUPPORTED;
+  return prefill_run(plan, q, plan->q_end - plan->q_begin, k, v, plan->q_end, sel, sel_cnt, o, stream, 1);
 }
 
 rtp_status rtp_hybrid_prefill(const rtp_plan* plan, const void* q, const void* k, const void* v,

@@ -33,7 +33,8 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(const SelectA
   const int t = a.t0 + static_cast<int>(blockIdx.x), slot = blockIdx.y, b = blockIdx.z;
   const size_t row = (static_cast<size_t>(b) * a.n_sparse + slot) * a.nb + t;
   int32_t* out = a.sel + row * a.kmax;
-  const float* C = a.centroids + (static_cast<size_t>(b) * a.n_sparse + slot) * a.nb * kRank;
+  const float* C =
+      a.centroids + (static_cast<size_t>(b) * (a.n_sparse / a.c_group) + slot / a.c_group) * a.nb * kRank;
   float q[kRank];
 #pragma unroll
   for (int c = 0; c < kRank; ++c) q[c] = a.qbar[row * kRank + c];

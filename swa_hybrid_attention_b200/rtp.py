@@ -66,6 +66,9 @@ def _load() -> ctypes.CDLL:
         "rtp_block_select": (I, [P, P, P, P, P, P]),
         "rtp_block_select_dynamic": (I, [P, P, P, ctypes.c_float, I, ctypes.c_float, P, P, P]),
         "rtp_block_select_rowmax": (I, [P, P, P, P, P, P, P]),
+        "rtp_indexer_project_heads": (I, [P, P, P, P, P]),
+        "rtp_block_select_heads": (I, [P, P, P, P, P, P]),
+        "rtp_hybrid_prefill_heads": (I, [P, P, P, P, P, P, P, P]),
         "rtp_hybrid_prefill": (I, [P, P, P, P, P, P, P, P]),
         "rtp_pipeline_create": (I, [cfgp, P, I, P, ctypes.POINTER(P)]),
         "rtp_pipeline_destroy": (None, [P]),
@@ -94,7 +97,8 @@ def _load() -> ctypes.CDLL:
 _lib = _load()
 EXPORTED = ("rtp_route_heads", "rtp_route_heads_range", "rtp_plan_destroy", "rtp_plan_num_sparse", "rtp_plan_num_items",
             "rtp_plan_sparse_heads", "rtp_plan_work_items", "rtp_indexer_project", "rtp_block_select",
-            "rtp_block_select_dynamic", "rtp_block_select_rowmax", "rtp_pipeline_create", "rtp_pipeline_destroy", "rtp_hybrid_prefill_host",
+            "rtp_block_select_dynamic", "rtp_block_select_rowmax", "rtp_indexer_project_heads",
+            "rtp_block_select_heads", "rtp_hybrid_prefill_heads", "rtp_pipeline_create", "rtp_pipeline_destroy", "rtp_hybrid_prefill_host",
             "rtp_hybrid_prefill", "rtp_decode_workspace_bytes", "rtp_sparse_decode", "rtp_sparse_decode_noalloc",
             "rtp_cache_centroids", "rtp_cache_append", "rtp_cache_cluster_workspace_bytes", "rtp_cache_cluster",
             "rtp_decode_clustered_workspace_bytes", "rtp_sparse_decode_clustered",
@@ -227,6 +231,23 @@ def rtp_block_select_rowmax(plan: int, q, proj, centroids, sel, sel_cnt, stream=
     _check("rtp_block_select_rowmax",
            _lib.rtp_block_select_rowmax(plan, _ptr(q), _ptr(proj), _ptr(centroids), _ptr(sel), _ptr(sel_cnt),
                                         _stream(stream)))
+
+
+def rtp_indexer_project_heads(plan: int, q, proj, qbar_heads, stream=None) -> None:
+    _check("rtp_indexer_project_heads",
+           _lib.rtp_indexer_project_heads(plan, _ptr(q), _ptr(proj), _ptr(qbar_heads), _stream(stream)))
+
+
+def rtp_block_select_heads(plan: int, qbar_heads, centroids, sel, sel_cnt, stream=None) -> None:
+    _check("rtp_block_select_heads",
+           _lib.rtp_block_select_heads(plan, _ptr(qbar_heads), _ptr(centroids), _ptr(sel), _ptr(sel_cnt),
+                                       _stream(stream)))
+
+
+def rtp_hybrid_prefill_heads(plan: int, q, k, v, sel, sel_cnt, o, stream=None) -> None:
+    _check("rtp_hybrid_prefill_heads",
+           _lib.rtp_hybrid_prefill_heads(plan, _ptr(q), _ptr(k), _ptr(v), _ptr(sel), _ptr(sel_cnt), _ptr(o),
+                                         _stream(stream)))
 
 
 def default_selection_beta(cfg: AttnConfig) -> float:
@@ -432,17 +453,24 @@ class Plan:
         except Exception:
             pass
 
-    def buffers(self, device) -> dict:
-        """Indexer / selection buffers for this plan (allocated with torch)."""
+    def buffers(self, device, per_head: bool = False) -> dict:
+        """Indexer / selection buffers for this plan (allocated with torch);
+        per_head adds those of the per-head selection."""
         c = self.cfg
         nb = c.seq // c.block
         ns = max(self.n_sparse, 0)
-        return dict(
+        bufs = dict(
             centroids=torch.empty(c.batch, ns, nb, 16, dtype=torch.float32, device=device),
             qbar=torch.empty(c.batch, ns, nb, 16, dtype=torch.float32, device=device),
             sel=torch.empty(c.batch, ns, nb, c.kmax, dtype=torch.int32, device=device),
             sel_cnt=torch.empty(c.batch, ns, nb, dtype=torch.int32, device=device),
         )
+        if per_head:
+            G = c.n_q_heads // c.n_kv_heads
+            bufs["qbar_heads"] = torch.empty(c.batch, ns, G, nb, 16, dtype=torch.float32, device=device)
+            bufs["sel_heads"] = torch.empty(c.batch, ns, G, nb, c.kmax, dtype=torch.int32, device=device)
+            bufs["cnt_heads"] = torch.empty(c.batch, ns, G, nb, dtype=torch.int32, device=device)
+        return bufs
 
     def run(self, q, k, v, proj, o, bufs: dict, stream=None, dynamic: dict | None = None,
             score: str = "mean") -> None:
@@ -453,10 +481,19 @@ class Plan:
         / group) for rtp_block_select_dynamic (topk is then the cap).
         score: "mean" (the query-block summary) or "rowmax" (the largest
         low-rank logit over the block's rows, rtp_block_select_rowmax) for the
-        fixed top-k selection.
+        fixed top-k selection, or "heads" (one selection per query head:
+        rtp_indexer_project_heads, rtp_block_select_heads and
+        rtp_hybrid_prefill_heads; bufs from buffers(device, per_head=True)).
         """
-        if score not in ("mean", "rowmax") or (score == "rowmax" and dynamic is not None):
+        if score not in ("mean", "rowmax", "heads") or (score != "mean" and dynamic is not None):
             raise RtpError("Plan.run", RTP_ERR_INVALID_ARG)
+        if self.n_sparse > 0 and score == "heads":
+            rtp_indexer_project(self.handle, q, k, proj, bufs["centroids"], bufs["qbar"], stream)
+            rtp_indexer_project_heads(self.handle, q, proj, bufs["qbar_heads"], stream)
+            rtp_block_select_heads(self.handle, bufs["qbar_heads"], bufs["centroids"], bufs["sel_heads"],
+                                   bufs["cnt_heads"], stream)
+            rtp_hybrid_prefill_heads(self.handle, q, k, v, bufs["sel_heads"], bufs["cnt_heads"], o, stream)
+            return
         if self.n_sparse > 0:
             rtp_indexer_project(self.handle, q, k, proj, bufs["centroids"], bufs["qbar"], stream)
             if score == "rowmax":
