@@ -251,7 +251,9 @@ struct TileIter {
       const int blk = checked_block(v, t);
       r.row0 = 128 * blk;
       r.row1 = r.row0 + 64;
-      r.flags = 0x1Eu | (m << 5) | ((blk >= t || m != 3u) ? 1u : 0u);
+      // a head outside the tile's lists skips it whole (P = 0); the element
+      // mask is only needed on the diagonal, which both lists hold
+      r.flags = 0x1Eu | (m << 5) | (blk >= t ? 1u : 0u);
     } else if (!b64) {
       int blk = checked_block(la[j], t);
       r.row0 = 128 * blk;
@@ -500,6 +502,23 @@ __device__ __noinline__ void run_softmax(Smem& s, uint32_t tmem, int h, const Pr
       if (!warp_wait(&s.s_full[h], sc & 1u, abort, a.status)) return;
       ++sc;
       tc_fence_after();
+      if (kHeads && !((tr.flags >> (5 + h)) & 1u)) {
+        // a tile of the other head's list only: P = 0 (its keys get no
+        // weight), written over S as usual, and nothing else to do
+        uint32_t z[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) z[e] = 0u;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          tmem_st16(tS + 16 * c, z);
+          if ((c + 1) % (4 / kPChunks) == 0) {
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&s.p_full[h][c / (4 / kPChunks)]);
+          }
+        }
+        continue;
+      }
       uint32_t r[128];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
