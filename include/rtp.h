@@ -32,6 +32,12 @@
  *     kept;
  *   - causal masking j <= i applies inside every selected block;
  *   - SWA: key j is visible to query i iff i-window < j <= i.
+ * Three alternatives to this policy are offered beside it, each feeding the
+ * same prefill: a per-query-block budget (rtp_block_select_dynamic), the
+ * largest logit over a query block's rows as its score
+ * (rtp_block_select_rowmax), and one selection per query head
+ * (rtp_indexer_project_heads, rtp_block_select_heads,
+ * rtp_hybrid_prefill_heads).
  *
  * Conventions
  *   - Every tensor argument is a DEVICE pointer owned by the caller,
