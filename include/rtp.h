@@ -229,15 +229,15 @@ rtp_status rtp_block_select_dynamic(const rtp_plan* plan, const float* qbar, con
  * it):
  *   s_j = max_{i in block t} u_i . c_j,  u_i = P^T sum_{h in group} q_{h,i}
  *   (u_i in fp32: the group's bf16 rows summed in head order, projected with
- *   a fixed summation order; each dot product in the order of
- *   rtp_block_select); keep the topk best candidates 1..t-n_local by (score
+ *   a fixed summation order; each dot product as two fixed-order chains over
+ *   ranks 0-7 and 8-15, then their sum); keep the topk best candidates 1..t-n_local by (score
  *   desc, index asc), block 0 and the local blocks, as rtp_block_select.
  *   q          the plan's query rows, as for rtp_hybrid_prefill
  *   proj       fp32 [128][16]
  *   centroids  as written by rtp_indexer_project
  *   sel, sel_cnt  as in rtp_block_select (same layout), so the result feeds
  *             rtp_hybrid_prefill unchanged
- * Work: block x 16 FMA per candidate and query block (7.7 ms on B200 for
+ * Work: block x 16 FMA per candidate and query block (7.3 ms on B200 for
  * the 1M-token retrieval head with block 128, against 0.96 ms for the mean
  * scores) on top of one more read of the group's Q rows.
  * Errors: RTP_ERR_INVALID_ARG (bad plan or pointer; nothing launched),

@@ -262,12 +262,33 @@ __global__ void __launch_bounds__(kSelThreads) block_select_dynamic_kernel(const
 // Per CTA (one query block): 1. u_i of the block's rows into shared memory
 // (16 threads per row sum the group's heads over 8 dims each and project;
 // the 16 partial dot products of a rank are added in a fixed butterfly, lane
-// 0's result kept); 2. one candidate per thread: its centroid in registers,
-// the rows' u_i read as shared-memory broadcasts, max over rows of the fixed-
-// order 16-term dot product; 3. the fixed kernel's radix select and ordered
-// compaction.
+// 0's result kept); 2. four candidates per thread: their centroids in
+// registers, each row's u_i read once as a shared-memory broadcast, max over
+// rows of the 16-term dot product (two fixed-order chains of 8, then their
+// sum); 3. the fixed kernel's radix select and ordered compaction.
 
 constexpr int kRowmaxCands = 4;
+
+// u . c with ranks 0-7 and 8-15 in two fma chains (fixed order), added at
+// the end: half the dependent latency of one 16-long chain.
+__device__ __forceinline__ float score16_two_chains(const float (&u)[kRank], const float4 (&c)[4]) {
+  float s0 = u[0] * c[0].x, s1 = u[8] * c[2].x;
+  s0 = fmaf(u[1], c[0].y, s0);
+  s1 = fmaf(u[9], c[2].y, s1);
+  s0 = fmaf(u[2], c[0].z, s0);
+  s1 = fmaf(u[10], c[2].z, s1);
+  s0 = fmaf(u[3], c[0].w, s0);
+  s1 = fmaf(u[11], c[2].w, s1);
+  s0 = fmaf(u[4], c[1].x, s0);
+  s1 = fmaf(u[12], c[3].x, s1);
+  s0 = fmaf(u[5], c[1].y, s0);
+  s1 = fmaf(u[13], c[3].y, s1);
+  s0 = fmaf(u[6], c[1].z, s0);
+  s1 = fmaf(u[14], c[3].z, s1);
+  s0 = fmaf(u[7], c[1].w, s0);
+  s1 = fmaf(u[15], c[3].w, s1);
+  return s0 + s1;
+}
 
 struct RowmaxScratch {
   float proj[kHeadDim * kRank];
@@ -343,7 +364,7 @@ __global__ void __launch_bounds__(kSelThreads) block_select_rowmax_kernel(const 
       const float uq[kRank] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w,
                                u2.x, u2.y, u2.z, u2.w, u3.x, u3.y, u3.z, u3.w};
 #pragma unroll
-      for (int u = 0; u < kRowmaxCands; ++u) best[u] = fmaxf(best[u], score16(uq, cv[u]));
+      for (int u = 0; u < kRowmaxCands; ++u) best[u] = fmaxf(best[u], score16_two_chains(uq, cv[u]));
     }
 #pragma unroll
     for (int u = 0; u < kRowmaxCands; ++u) {
