@@ -392,6 +392,32 @@ def time_dynamic(rtp, w, res, device, points=((0.9, None), (0.99, None), (0.9, 1
     return out
 
 
+def time_selection_variants(rtp, w, device, reps=2):
+    """The selection variants alone on the layer (profiling entry): the
+    indexer, then `reps` times each of the row-max selection and the per-head
+    summaries + selection; mean ms per call."""
+    d, plan, _ = make_layer(rtp, w, 0, device)
+    bufs = plan.buffers(device, per_head=True)
+    q, proj = d["q"], d["proj"]
+    stream = torch.cuda.current_stream()
+    rtp.rtp_indexer_project(plan.handle, q, d["k"], proj, bufs["centroids"], bufs["qbar"], stream)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    for e in ev:
+        e[0].record(stream)
+        rtp.rtp_block_select_rowmax(plan.handle, q, proj, bufs["centroids"], bufs["sel"], bufs["sel_cnt"], stream)
+        e[1].record(stream)
+        rtp.rtp_indexer_project_heads(plan.handle, q, proj, bufs["qbar_heads"], stream)
+        rtp.rtp_block_select_heads(plan.handle, bufs["qbar_heads"], bufs["centroids"], bufs["sel_heads"],
+                                   bufs["cnt_heads"], stream)
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    out = {"workload": w.name, "rowmax_select_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
+           "per_head_summaries_and_select_ms": statistics.mean(e[1].elapsed_time(e[2]) for e in ev),
+           "status": rtp.status_str(rtp.rtp_last_device_status(stream))}
+    plan.close()
+    return out
+
+
 def time_cp_projection(rtp, w, res, device, world=8, link_gbs=770.0):
     """Context-parallel prefill of the main layer split over `world` ranks,
     projected from one GPU: each rank's ranged prefill is timed here on its own
@@ -853,6 +879,10 @@ def run_ours(args, rank, world, local):
         w.seq = args.seq
         w.name = f"{w.name}@{args.seq}"
         w.needles = max(1, w.needles * args.seq // 1048576)
+    if args.only == "selection":
+        if rank == 0:
+            print(json.dumps({"selection_variants": time_selection_variants(rtp, w, device)}), flush=True)
+        return
     res = time_primary(rtp, w, rank_layer(rank), args.steps, args.warmup, device, world)
     algo, execd = layer_flops(w, res["kinds"])
     step_ms = max_over_ranks(res["total_ms"] / args.steps, world)
@@ -945,7 +975,8 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=10.0)
     ap.add_argument("--decode-steps", type=int, default=256)
     ap.add_argument("--seq", type=int, default=0, help="override the primary workload's length (profiling)")
-    ap.add_argument("--only", choices=["all", "decode"], default="all", help="run only part of the bench")
+    ap.add_argument("--only", choices=["all", "decode", "selection"], default="all",
+                    help="run only part of the bench (decode step; selection variants, for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
