@@ -97,6 +97,7 @@ struct __align__(1024) Smem {
   uint64_t s_full[2], o_full[2];
   uint64_t p_full[2][kPChunks];  // [head][chunk of keys]: that part of P is in TMEM
   uint64_t drain;
+  uint32_t tile_mem[kStages];  // per-head selections: the pair's membership of the tile in each K stage
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -317,6 +318,7 @@ __device__ __noinline__ void run_producer(Smem& s, const CUtensorMap* mq, const 
         const int st = gt & 1;
         const uint32_t use = gt >> 1;
         if (!mbar_wait(&s.k_empty[st], (use & 1u) ^ 1u, abort, a.status)) goto drain;
+        if constexpr (kHeads) s.tile_mem[st] = (tr.flags >> 5) & 3u;  // published by the arrive below
         mbar_arrive_expect_tx(&s.k_full[st], kTileBytes);
         for (int c = 0; c < 2; ++c) {
           tma_load_3d(s.k[st] + c * kChunkBytes, mk, &s.k_full[st], 64 * c, tr.row0, item.bkv);
@@ -407,6 +409,19 @@ __device__ __forceinline__ bool issue_pv_chunked(Smem& s, int h, uint32_t parity
   return true;
 }
 
+// Head h's O += P V for the tile or, for a head outside the tile's lists
+// (per-head selections), only the wait for its P handshake.
+template <bool kHeads>
+__device__ __forceinline__ bool pv_or_skip(Smem& s, int h, bool member, uint32_t parity, uint32_t d_tmem,
+                                          uint32_t p_tmem, uint64_t vd, uint32_t idesc, bool accumulate,
+                                          volatile int* abort, uint32_t* status) {
+  if (!kHeads || member) return issue_pv_chunked(s, h, parity, d_tmem, p_tmem, vd, idesc, accumulate, abort, status);
+#pragma unroll
+  for (int q = 0; q < kPChunks; ++q)
+    if (!mma_wait(&s.p_full[h][q], parity, abort, status)) return false;
+  return true;
+}
+
 template <bool kHeads>
 __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& a, volatile int* abort) {
   const uint32_t id_qk = idesc_bf16_f32(128, 128, false);
@@ -425,14 +440,20 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
     const int n = ti.n;
     if (!mma_wait(&s.q_full[0], it & 1u, abort, a.status)) goto drain;
     if (!mma_wait(&s.q_full[1], it & 1u, abort, a.status)) goto drain;
+    // per-head selections: membership of the tile in flight; a head's S and
+    // P V are issued only for its own tiles (its s_full is still committed,
+    // so the handshakes keep their phases), and its first P V overwrites O
+    uint32_t mem_cur = 3u;
+    bool started0 = false, started1 = false;
     {
       const int st0 = gt & 1;
       if (!mma_wait(&s.k_full[st0], (gt >> 1) & 1u, abort, a.status)) goto drain;
       tc_fence_after();
+      if constexpr (kHeads) mem_cur = s.tile_mem[st0];
       const uint64_t sk = st0 ? kd1 : kd0;
-      issue_qk(tS[0], qd0, sk, id_qk);
+      if (!kHeads || (mem_cur & 1u)) issue_qk(tS[0], qd0, sk, id_qk);
       umma_commit(&s.s_full[0]);
-      issue_qk(tS[1], qd1, sk, id_qk);
+      if (!kHeads || (mem_cur & 2u)) issue_qk(tS[1], qd1, sk, id_qk);
       umma_commit(&s.s_full[1]);
       umma_commit(&s.k_empty[st0]);
       if (n == 1) {
@@ -448,28 +469,37 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
       const uint64_t sv = st ? vd1 : vd0;
       const uint64_t sk2 = st2 ? kd1 : kd0;
       if (!mma_wait(&s.v_full[st], (g >> 1) & 1u, abort, a.status)) goto drain;
+      uint32_t mem_next = 3u;
       // head 0: O0 += P0 V ; then S0 for the next tile
-      if (!issue_pv_chunked(s, 0, pc & 1u, tO[0], tS[0], sv, id_pv, j > 0, abort, a.status)) goto drain;
+      if (!pv_or_skip<kHeads>(s, 0, (mem_cur & 1u) != 0, pc & 1u, tO[0], tS[0], sv, id_pv, kHeads ? started0 : j > 0,
+                              abort, a.status))
+        goto drain;
+      if (kHeads && (mem_cur & 1u)) started0 = true;
       if (!has_next) {
         umma_commit(&s.o_full[0]);
       } else {
         if (!mma_wait(&s.k_full[st2], ((g + 1) >> 1) & 1u, abort, a.status)) goto drain;
         tc_fence_after();
-        issue_qk(tS[0], qd0, sk2, id_qk);
+        if constexpr (kHeads) mem_next = s.tile_mem[st2];
+        if (!kHeads || (mem_next & 1u)) issue_qk(tS[0], qd0, sk2, id_qk);
         umma_commit(&s.s_full[0]);
         if (j + 2 == n) umma_commit(&s.q_empty[0]);
       }
       // head 1
-      if (!issue_pv_chunked(s, 1, pc & 1u, tO[1], tS[1], sv, id_pv, j > 0, abort, a.status)) goto drain;
+      if (!pv_or_skip<kHeads>(s, 1, (mem_cur & 2u) != 0, pc & 1u, tO[1], tS[1], sv, id_pv, kHeads ? started1 : j > 0,
+                              abort, a.status))
+        goto drain;
+      if (kHeads && (mem_cur & 2u)) started1 = true;
       umma_commit(&s.v_empty[st]);
       if (!has_next) {
         umma_commit(&s.o_full[1]);
       } else {
-        issue_qk(tS[1], qd1, sk2, id_qk);
+        if (!kHeads || (mem_next & 2u)) issue_qk(tS[1], qd1, sk2, id_qk);
         umma_commit(&s.s_full[1]);
         umma_commit(&s.k_empty[st2]);
         if (j + 2 == n) umma_commit(&s.q_empty[1]);
       }
+      mem_cur = mem_next;
       ++pc;
     }
     gt += n;
@@ -503,20 +533,10 @@ __device__ __noinline__ void run_softmax(Smem& s, uint32_t tmem, int h, const Pr
       ++sc;
       tc_fence_after();
       if (kHeads && !((tr.flags >> (5 + h)) & 1u)) {
-        // a tile of the other head's list only: P = 0 (its keys get no
-        // weight), written over S as usual, and nothing else to do
-        uint32_t z[16];
+        // a tile of the other head's list only: no S was computed for this
+        // head and no P V will read its P; the handshake keeps the phases
 #pragma unroll
-        for (int e = 0; e < 16; ++e) z[e] = 0u;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          tmem_st16(tS + 16 * c, z);
-          if ((c + 1) % (4 / kPChunks) == 0) {
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&s.p_full[h][c / (4 / kPChunks)]);
-          }
-        }
+        for (int q = 0; q < kPChunks; ++q) mbar_arrive(&s.p_full[h][q]);
         continue;
       }
       uint32_t r[128];
