@@ -338,6 +338,25 @@ def test_rowmax_score_bounds_the_mean_score():
         assert np.all(oracle.rowmax_scores(q, proj, C, t, block) >= oracle.scores(qb[t], C) - 1e-12)
 
 
+def test_per_head_selection_with_identical_heads_equals_the_shared_one():
+    # every head of the group the same: the shared summary is G times each
+    # head's own, so every head's own selection is the shared selection
+    G, n, block, topk, n_local = 4, 1024, 64, 3, 2
+    g = torch.Generator().manual_seed(9)
+    q1 = torch.randn(1, n, 128, generator=g).to(torch.bfloat16)
+    q = q1.expand(G, n, 128).contiguous()
+    k = torch.randn(n, 128, generator=g).to(torch.bfloat16)
+    proj = torch.randn(128, 16, generator=g) / 11.3
+    C = oracle.centroids(k, block, proj)
+    nb = n // block
+    shared = oracle.qbar(q, block, proj)
+    own = oracle.qbar(q[:1], block, proj)
+    np.testing.assert_allclose(shared, G * own, rtol=1e-12, atol=1e-12)
+    a = oracle.select(shared, C, np.arange(nb), topk, n_local)
+    b = oracle.select(own, C, np.arange(nb), topk, n_local)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[1], b[1])
+
+
 # --------------------------------------------------------------------- decode
 
 
