@@ -268,7 +268,8 @@ rtp_status rtp_block_select_rowmax(const rtp_plan* plan, const void* q, const fl
  *   h of a retrieval KV head attends to the blocks of its own list (with the
  *   causal mask).  The two heads of a query-head pair share one stream of
  *   K/V tiles, the union of their lists; a tile outside one head's list is
- *   masked out for that head, so the work grows with how much the pair's
+ *   skipped for that head (no MMAs, no softmax), but the pair's pipeline
+ *   still walks the whole union, so the time grows with how much the pair's
  *   lists differ.
  * Errors: RTP_ERR_INVALID_ARG (bad plan or pointer; nothing launched),
  * RTP_ERR_UNSUPPORTED (ranged plan, block 64 or odd group), RTP_ERR_CUDA.
