@@ -415,11 +415,15 @@ template <bool kHeads>
 __device__ __forceinline__ bool pv_or_skip(Smem& s, int h, bool member, uint32_t parity, uint32_t d_tmem,
                                           uint32_t p_tmem, uint64_t vd, uint32_t idesc, bool accumulate,
                                           volatile int* abort, uint32_t* status) {
-  if (!kHeads || member) return issue_pv_chunked(s, h, parity, d_tmem, p_tmem, vd, idesc, accumulate, abort, status);
+  if constexpr (kHeads) {
+    if (!member) {
 #pragma unroll
-  for (int q = 0; q < kPChunks; ++q)
-    if (!mma_wait(&s.p_full[h][q], parity, abort, status)) return false;
-  return true;
+      for (int q = 0; q < kPChunks; ++q)
+        if (!mma_wait(&s.p_full[h][q], parity, abort, status)) return false;
+      return true;
+    }
+  }
+  return issue_pv_chunked(s, h, parity, d_tmem, p_tmem, vd, idesc, accumulate, abort, status);
 }
 
 template <bool kHeads>

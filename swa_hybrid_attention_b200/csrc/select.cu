@@ -262,12 +262,13 @@ __global__ void __launch_bounds__(kSelThreads) block_select_dynamic_kernel(const
 // Per CTA (one query block): 1. u_i of the block's rows into shared memory
 // (16 threads per row sum the group's heads over 8 dims each and project;
 // the 16 partial dot products of a rank are added in a fixed butterfly, lane
-// 0's result kept); 2. four candidates per thread: their centroids in
-// registers, each row's u_i read once as a shared-memory broadcast, max over
+// 0's result kept); 2. two candidates per thread (80 registers: three CTAs
+// an SM): their centroids in registers, each row's u_i read once as a
+// shared-memory broadcast, max over
 // rows of the 16-term dot product (two fixed-order chains of 8, then their
 // sum); 3. the fixed kernel's radix select and ordered compaction.
 
-constexpr int kRowmaxCands = 4;
+constexpr int kRowmaxCands = 2;
 
 // u . c with ranks 0-7 and 8-15 in two fma chains (fixed order), added at
 // the end: half the dependent latency of one 16-long chain.
@@ -295,7 +296,7 @@ struct RowmaxScratch {
   float u[128][kRank];  // block <= 128 rows
 };
 
-__global__ void __launch_bounds__(kSelThreads) block_select_rowmax_kernel(const SelectArgs a) {
+__global__ void __launch_bounds__(kSelThreads, 3) block_select_rowmax_kernel(const SelectArgs a) {
   extern __shared__ uint32_t keys[];
   __shared__ SelectScratch sh;
   __shared__ __align__(16) RowmaxScratch rs;
