@@ -5,14 +5,20 @@ path computes, used to check the CUDA library.  Only the tests, the package
 smoke check and the CPU-baseline leg of the benchmark import this module;
 the library never does, and this module never imports the library.
 
-The arithmetic lives in oracle.cpp (C++17, fp64, std::thread); this file
-compiles it with g++ on first use and marshals numpy arrays through ctypes.
+Most of the arithmetic lives in oracle.cpp (C++17, fp64, std::thread); this
+file compiles it with g++ on first use and marshals numpy arrays through
+ctypes.  Two functions are written here instead: attention_rows_mm, the same
+exact attention as attention_rows with the logits and weighted sums of each
+query block's rows taken as fp64 matrix products (torch on the CPU, fast
+enough for tens of thousands of rows at 1M keys), and round_bf16, the
+single rounding of an fp64 result to bf16 for comparison.
 Each function states the passage of the RTPurbo / RTPurboV2 pages it
 follows (see the header of oracle.cpp for the page titles).
 
 Pinned by the not-gpu tests (tests/test_oracle_pins.py) against brute-force
-masked attention, torch's scaled-dot-product attention in fp64 on CPU,
-closed forms and invariants.  The pages print no worked example, so no
+masked attention (both attention statements), torch's scaled-dot-product
+attention in fp64 on CPU, exact nearest-even rounding by rational
+arithmetic, full sorts, closed forms and invariants.  The pages print no worked example, so no
 value here is tied to the authors' own implementation.
 """
 
@@ -393,9 +399,88 @@ def topk_chunks(qbar_row: np.ndarray, chunk_centroids: np.ndarray, topk: int) ->
     return np.sort(order[:topk])
 
 
+# Largest finite bf16: fraction 1.1111111b, exponent 127.
+_BF16_MAX = (2.0 - 2.0 ** -7) * 2.0 ** 127
+
+
 def round_bf16(x: np.ndarray) -> np.ndarray:
-    """Round fp64 values to the nearest bf16 (ties to even), returned as fp64."""
-    f = np.asarray(x, dtype=np.float64).astype(np.float32)
-    u = f.view(np.uint32).astype(np.uint64)
-    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
-    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+    """Round fp64 values to the nearest bf16 in one step (ties to even), returned as fp64.
+
+    bf16 has fp32's 8-bit exponent and 7 fraction bits.  A normal value keeps
+    the top 7 of fp64's 52 fraction bits, rounded half-to-even on the 45 bits
+    dropped; a value below the smallest normal bf16 (2^-126) is rounded to a
+    multiple of 2^-133 (the subnormal spacing); a value whose rounding exceeds
+    the largest finite bf16 becomes infinite; NaN stays NaN.  (Rounding to
+    fp32 first and then to bf16 would round twice, which differs when the
+    first rounding lands exactly half-way between two bf16 values.)
+    """
+    a = np.array(x, dtype=np.float64, copy=True)
+    u = a.view(np.uint64)
+    keep = np.uint64(45)
+    lsb = (u >> keep) & np.uint64(1)
+    r = ((u + np.uint64((1 << 44) - 1) + lsb) >> keep) << keep
+    out = r.view(np.float64).copy()
+    tiny = np.abs(a) < 2.0 ** -126
+    out[tiny] = np.round(a[tiny] * 2.0 ** 133) * 2.0 ** -133  # np.round: half to even
+    over = np.isfinite(a) & (np.abs(out) > _BF16_MAX)
+    out[over] = np.copysign(np.inf, a[over])
+    out[np.isnan(a)] = np.nan
+    return out
+
+
+def attention_rows_mm(q_rows, pos, k_head, v_head, mode: int, window: int = 0, block: int = 64, sel=None,
+                      cnt=None, scale: float | None = None) -> np.ndarray:
+    """Exact softmax attention for given rows of one query head -> fp64 [n, 128].
+
+    The same definition as attention_rows (RTPurbo page, opening section:
+    streaming heads keep a window, full heads every earlier token; the "Full
+    Attention Strikes Back" summary: exact softmax over the selected set),
+    computed with fp64 matrix products: the rows are taken in groups that
+    share a query block t = i // block, and for each group
+      J      = a key range (or the selected blocks of t) holding every key
+               visible to any row of the group,
+      s_ij   = scale * q_i . k_j for j in J         (one fp64 matmul),
+      s_ij   = -inf where j is not visible to i      (i-W < j <= i for SWA,
+               j <= i for full and, inside the selected blocks, sparse),
+      O_i    = sum_j p_ij v_j / sum_j p_ij,  p_ij = exp(s_ij - max_j s_ij)
+                                                     (one fp64 matmul).
+    mode 0 = SWA, 1 = full causal, 2 = sparse over sel[t] (first cnt[t]
+    entries).  A row with no visible key gets zeros.
+    """
+    import torch
+
+    qb = torch.from_numpy(_bf16_bits(q_rows).reshape(-1, 128).view(np.int16)).view(torch.bfloat16)
+    kb = torch.from_numpy(_bf16_bits(k_head).reshape(-1, 128).view(np.int16)).view(torch.bfloat16)
+    vb = torch.from_numpy(_bf16_bits(v_head).reshape(-1, 128).view(np.int16)).view(torch.bfloat16)
+    pp = np.ascontiguousarray(pos, dtype=np.int64)
+    sc = 1.0 / np.sqrt(128.0) if scale is None else float(scale)
+    out = np.zeros((qb.shape[0], 128), dtype=np.float64)
+    tq = pp // block
+    for t in np.unique(tq):
+        idx = np.nonzero(tq == t)[0]
+        i = torch.from_numpy(pp[idx])
+        hi = int(pp[idx].max())
+        if mode == SWA:
+            keys = torch.arange(max(0, int(pp[idx].min()) - window + 1), hi + 1)
+        elif mode == FULL:
+            keys = torch.arange(0, hi + 1)
+        else:
+            blocks = [int(b) for b in np.asarray(sel)[t, :int(np.asarray(cnt)[t])]]
+            keys = torch.cat([torch.arange(b * block, (b + 1) * block) for b in blocks]) if blocks else \
+                torch.zeros(0, dtype=torch.int64)
+            keys = keys[keys <= hi]
+        if keys.numel() == 0:
+            continue
+        visible = keys[None, :] <= i[:, None]
+        if mode == SWA:
+            visible &= keys[None, :] > i[:, None] - window
+        qd = qb[torch.from_numpy(idx)].double()
+        s = (qd @ kb[keys].double().T) * sc
+        s = s.masked_fill(~visible, float("-inf"))
+        m = s.max(dim=1, keepdim=True).values
+        ok = torch.isfinite(m[:, 0])
+        p = torch.exp(s - torch.where(torch.isfinite(m), m, torch.zeros_like(m)))
+        o = (p @ vb[keys].double()) / p.sum(dim=1, keepdim=True)
+        o[~ok] = 0.0
+        out[idx] = o.numpy()
+    return out

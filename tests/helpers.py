@@ -82,9 +82,10 @@ def check_prefill_rows(o_gpu, q, k, v, kinds, group, window, block, sel_gpu, cnt
         if mode == oracle.SPARSE:
             sel = cpu(sel_gpu[0, slot_of[kvh]]).numpy()
             cnt = cpu(cnt_gpu[0, slot_of[kvh]]).numpy()
+        if rows.size == 0:
+            continue
         qr = cpu(q[0, hq][torch.from_numpy(rows).to(q.device)])
-        ref = oracle.attention_rows(qr, rows, k_h, v_h, mode, window, block, sel, cnt,
-                                    scale)
+        ref = oracle.attention_rows_mm(qr, rows, k_h, v_h, mode, window, block, sel, cnt, scale)
         ref = oracle.round_bf16(ref)
         got = cpu(o_gpu[0, hq][torch.from_numpy(rows).to(o_gpu.device)]).double().numpy()
         err = np.abs(got - ref)

@@ -77,29 +77,37 @@ def small():
     return inputs.small_prefill(384, 2, 1, [oracle.FULL], seed=7)
 
 
+# The two statements of exact attention: per row (C++) and per query-block
+# group with fp64 matrix products (torch).  Every brute-force pin runs on both.
+ATTENTION = {"rows": oracle.attention_rows, "mm": oracle.attention_rows_mm}
+
+
+@pytest.mark.parametrize("impl", sorted(ATTENTION))
 @pytest.mark.parametrize("n", [128, 384, 1024])
 @pytest.mark.parametrize("mode,window", [(oracle.FULL, 0), (oracle.SWA, 100), (oracle.SWA, 1), (oracle.SWA, 256)])
-def test_attention_matches_bruteforce(n, mode, window):
+def test_attention_matches_bruteforce(n, mode, window, impl):
     d = inputs.small_prefill(n, 1, 1, [mode], seed=11 + n)
     q, k, v = d["q"][0, 0], d["k"][0, 0], d["v"][0, 0]
     rows = np.arange(n)
-    got = oracle.attention_rows(q, rows, k, v, mode, window)
+    got = ATTENTION[impl](q, rows, k, v, mode, window)
     ref = dense_reference(widen(q), widen(k), widen(v), mask_matrix(n, mode, window))
     assert np.max(np.abs(got - ref)) <= 1e-12
 
 
+@pytest.mark.parametrize("impl", sorted(ATTENTION))
 @pytest.mark.parametrize("n,block", [(384, 64), (1024, 128), (1024, 64)])
-def test_sparse_attention_matches_bruteforce(n, block):
+def test_sparse_attention_matches_bruteforce(n, block, impl):
     rng = np.random.default_rng(n + block)
     d = inputs.small_prefill(n, 1, 1, [oracle.SPARSE], seed=3)
     q, k, v = d["q"][0, 0], d["k"][0, 0], d["v"][0, 0]
     sel, cnt = random_selection(n, block, 5, rng)
-    got = oracle.attention_rows(q, np.arange(n), k, v, oracle.SPARSE, 0, block, sel, cnt)
+    got = ATTENTION[impl](q, np.arange(n), k, v, oracle.SPARSE, 0, block, sel, cnt)
     ref = dense_reference(widen(q), widen(k), widen(v), mask_matrix(n, oracle.SPARSE, 0, block, sel, cnt))
     assert np.max(np.abs(got - ref)) <= 1e-12
 
 
-def test_attention_matches_torch_sdpa_fp64():
+@pytest.mark.parametrize("impl", sorted(ATTENTION))
+def test_attention_matches_torch_sdpa_fp64(impl):
     n, block = 512, 64
     rng = np.random.default_rng(5)
     d = inputs.small_prefill(n, 1, 1, [oracle.SPARSE], seed=21)
@@ -110,8 +118,24 @@ def test_attention_matches_torch_sdpa_fp64():
         ref = torch.nn.functional.scaled_dot_product_attention(
             q.double()[None, None], k.double()[None, None], v.double()[None, None],
             attn_mask=torch.from_numpy(m)[None, None], scale=SCALE)[0, 0].numpy()
-        got = oracle.attention_rows(q, np.arange(n), k, v, mode, window, block, sel, cnt)
+        got = ATTENTION[impl](q, np.arange(n), k, v, mode, window, block, sel, cnt)
         assert np.max(np.abs(got - ref)) <= 1e-12
+
+
+@pytest.mark.parametrize("mode,window,block", [(oracle.FULL, 0, 64), (oracle.SWA, 300, 64), (oracle.SWA, 1, 128),
+                                               (oracle.SPARSE, 0, 64), (oracle.SPARSE, 0, 128)])
+def test_grouped_attention_equals_row_attention_on_scattered_rows(mode, window, block):
+    """Rows in random order from scattered query blocks (several per block,
+    one alone, the last ragged block), with a scale: both statements agree."""
+    n = 1000
+    rng = np.random.default_rng(block + window)
+    d = inputs.small_prefill(n, 1, 1, [mode], seed=61)
+    q, k, v = d["q"][0, 0], d["k"][0, 0], d["v"][0, 0]
+    sel, cnt = random_selection(n + block, block, 6, rng)
+    rows = rng.permutation(np.concatenate([rng.choice(n, 40, replace=False), [0, n - 1, 130]]))
+    a = oracle.attention_rows(q[rows], rows, k, v, mode, window, block, sel, cnt, 0.07)
+    b = oracle.attention_rows_mm(q[rows], rows, k, v, mode, window, block, sel, cnt, 0.07)
+    assert np.max(np.abs(a - b)) <= 1e-12
 
 
 def test_swa_with_window_ge_seq_is_full_bitwise(small):
@@ -406,11 +430,56 @@ def test_decode_full_head_sees_whole_cache():
         assert np.max(np.abs(out[h] - ref[0])) <= 1e-12
 
 
-def test_round_bf16():
-    x = np.array([1.0, 1.00390625, 1.005859375, -3.14159, 0.0, 65504.0])
+def _bf16_grid():
+    """Every non-negative finite bf16 value (bit patterns 0x0000..0x7F7F) and
+    2^128 standing for the next value up (infinity), as fp64."""
+    bits = np.arange(0, 0x7F81, dtype=np.uint32) << 16
+    vals = bits.view(np.float32).astype(np.float64)
+    vals[-1] = 2.0 ** 128
+    return vals
+
+
+def brute_round_bf16(x, grid):
+    """Nearest grid value by exact rational distance, ties to the even bit pattern."""
+    from fractions import Fraction
+
+    if np.isnan(x):
+        return np.nan
+    a = abs(x)
+    j = int(np.searchsorted(grid, a, side="left"))
+    if j == grid.size:  # beyond 2^128
+        r = grid[-1]
+    elif grid[j] == a:
+        r = grid[j]
+    else:
+        lo, hi = grid[j - 1], grid[j]
+        dl, dh = Fraction(a) - Fraction(lo), Fraction(hi) - Fraction(a)
+        r = lo if dl < dh or (dl == dh and (j - 1) % 2 == 0) else hi
+    r = np.inf if r == 2.0 ** 128 else r
+    return -r if x < 0 else r
+
+
+def test_round_bf16_matches_exact_nearest_even():
+    grid = _bf16_grid()
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal(3000) * np.exp2(rng.integers(-140, 130, 3000))
+    # exact half-way points between neighbouring bf16 values, and just off them
+    mids = (grid[1:-1:97] + grid[2::97]) / 2.0
+    x = np.concatenate([x, mids, -mids, np.nextafter(mids, 0), np.nextafter(mids, np.inf), grid[:-1:211],
+                        [0.0, -0.0, 2.0 ** -133, 3 * 2.0 ** -134, 2.0 ** -134, np.inf, -np.inf, np.nan,
+                         (2.0 - 2.0 ** -8) * 2.0 ** 127, 3.4e38, 1e300]])
     got = oracle.round_bf16(x)
-    ref = torch.tensor(x, dtype=torch.float64).to(torch.bfloat16).double().numpy()
-    assert np.array_equal(got, ref)
+    want = np.array([brute_round_bf16(v, grid) for v in x])
+    assert np.array_equal(got, want, equal_nan=True)
+    assert np.array_equal(np.signbit(got[x == 0]), np.signbit(x[x == 0]))
+
+
+def test_round_bf16_rounds_once():
+    # 1 + 2^-8 + 2^-30 lies above the half-way point between the bf16 values 1
+    # and 1 + 2^-7; rounding to fp32 first would land exactly on that point and
+    # then tie to 1.
+    x = np.array([1 + 2.0 ** -8 + 2.0 ** -30, -(1 + 2.0 ** -8 + 2.0 ** -30), 1 + 2.0 ** -8])
+    assert np.array_equal(oracle.round_bf16(x), [1 + 2.0 ** -7, -(1 + 2.0 ** -7), 1.0])
 
 
 def test_selection_ties_at_the_cut_take_lower_indices():
@@ -652,3 +721,65 @@ def test_attention_over_key_list_matches_bruteforce_and_full_row():
     for h in range(G):
         full = oracle.attention_rows(q[h, Lc - 1:Lc], np.array([Lc - 1]), k, v, oracle.FULL)
         assert np.max(np.abs(allk[h] - full[0])) <= 1e-12
+
+
+def _python_scores(qb, C):
+    """q . c_j as a plain fp64 sum in coordinate order, one chunk at a time."""
+    out = []
+    for row in C:
+        acc = 0.0
+        for a, b in zip(qb, row):
+            acc += float(a) * float(b)
+        out.append(acc)
+    return out
+
+
+@pytest.mark.parametrize("n,topk", [(50, 7), (50, 0), (12, 12), (12, 30), (1, 1), (300, 32)])
+def test_topk_chunks_matches_full_sort(n, topk):
+    """The clustered decode keeps the topk chunks by (score desc, chunk index
+    asc), listed ascending: a full Python sort of exact ties and negative
+    scores included."""
+    rng = np.random.default_rng(n + topk)
+    C = rng.standard_normal((n, 16))
+    dup = rng.integers(0, n, size=n // 3)
+    if dup.size:
+        C[dup] = C[dup[0]]  # a crowd of exactly equal scores
+    C[-1] = -C[0]
+    qb = rng.standard_normal(16)
+    s = _python_scores(qb, C)
+    want = sorted(sorted(range(n), key=lambda j: (-s[j], j))[:topk])
+    got = oracle.topk_chunks(qb, C, topk)
+    assert got.tolist() == want
+
+
+def test_topk_chunks_tie_order_is_by_index():
+    C = np.ones((10, 16))
+    C[6] = 2.0
+    got = oracle.topk_chunks(np.ones(16), C, 4)
+    assert got.tolist() == [0, 1, 2, 6]
+
+
+@pytest.mark.parametrize("cache_len,clu_end,n_chosen", [(900, 700, 3), (900, 900, 3), (900, 700, 0),
+                                                         (640, 640, 0), (1000, 128, 0)])
+def test_decode_clustered_keys_is_sink_chunks_and_tail(cache_len, clu_end, n_chosen):
+    """Brute force by a boolean mask over the cache: the sink block, every
+    member of the chosen chunks and the unclustered tail [clu_end, cache_len),
+    each key once."""
+    block, nc = 128, 6
+    rng = np.random.default_rng(cache_len + clu_end + n_chosen)
+    n = clu_end - block
+    assign = rng.integers(0, nc, size=max(n, 0))
+    members, offsets, chunks = oracle.cluster_chunks(assign, block, nc, chunk=16)
+    chosen = sorted(rng.choice(len(chunks), size=min(n_chosen, len(chunks)), replace=False).tolist()) \
+        if len(chunks) else []
+    mask = np.zeros(cache_len, dtype=bool)
+    mask[:min(block, cache_len)] = True
+    for x in chosen:
+        _, s0, m = chunks[x]
+        for key in members[s0:s0 + m]:
+            assert block <= key < clu_end
+            mask[key] = True
+    mask[clu_end:cache_len] = True
+    got = oracle.decode_clustered_keys(members, chunks, chosen, block, clu_end, cache_len)
+    assert got.tolist() == np.nonzero(mask)[0].tolist()
+    assert len(set(got.tolist())) == got.size
