@@ -381,13 +381,19 @@ rtp_status rtp_sparse_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, 
  *   cudaMalloc, cudaFree or allocating library call on this path.
  *   The array is looked up once per device, on the first call made with
  *   that device current; make that first call before any stream capture.
- *   Every call shares the one array and it keeps the last call's contents
- *   (every word a call reads is written earlier in the same call, so
- *   nothing needs clearing); calls that overlap on the GPU — on different
- *   streams, or from several host threads — race on it and must be
- *   serialised by the caller.
- *   Unlike rtp_sparse_decode this path has no device status word: an
- *   out-of-range block index in the selection is skipped without a report.
+ *   Every call shares the one array and it keeps the last call's contents;
+ *   a call writes every word it reads earlier in the same call (selection
+ *   lists, then per-split partial results), so nothing needs clearing —
+ *   unless one of its bounded waits gives up, in which case that call's
+ *   output is undefined and the time-out is reported as below.  Calls that
+ *   overlap on the GPU — on different streams, or from several host
+ *   threads — race on the array and must be serialised by the caller.
+ *   Errors on the device: this path reports in its own status word, a
+ *   second fixed device word beside the array (looked up with it), not in
+ *   the allocated word of the other entry points.  rtp_last_device_status
+ *   reads and clears both and allocates nothing itself, so a caller of this
+ *   path reads RTP_ERR_TIMEOUT (a bounded wait gave up) or
+ *   RTP_ERR_INVALID_ARG (an out-of-range block index was skipped) there.
  * ---------------------------------------------------------------------- */
 rtp_status rtp_sparse_decode_noalloc(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* q,
                                      const void* kcache, const void* vcache, const float* centroids,
@@ -515,10 +521,12 @@ rtp_status rtp_sparse_decode_clustered(const rtp_attn_cfg* cfg, const uint8_t* k
 
 /* ------------------------------------------------------------------------
  * rtp_last_device_status — synchronise `stream`, then read and clear the
- * device status word of the current device.  Returns RTP_OK, RTP_ERR_TIMEOUT
- * (a bounded wait gave up), RTP_ERR_INVALID_ARG (a kernel met an
- * out-of-range block index and skipped it) or RTP_ERR_CUDA (the stream
- * reported an error).
+ * device status words of the current device: the word the entry points
+ * allocate on first use (if one has) and the fixed word of
+ * rtp_sparse_decode_noalloc (if that has run).  Creates neither, so it
+ * allocates nothing.  Returns RTP_OK, RTP_ERR_TIMEOUT (a bounded wait gave
+ * up), RTP_ERR_INVALID_ARG (a kernel met an out-of-range block index and
+ * skipped it) or RTP_ERR_CUDA (the stream reported an error).
  * ---------------------------------------------------------------------- */
 rtp_status rtp_last_device_status(void* stream);
 

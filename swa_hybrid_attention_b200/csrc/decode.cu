@@ -988,29 +988,46 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(const _
 }
 
 // Scratch of the allocation-free decode entry point: a file-scope device
-// array that every GPU loading this library holds until the process exits.
+// array that every GPU loading this library holds until the process exits,
+// and the device status word its kernels report bounded-wait time-outs and
+// skipped indices in (the other entry points use an allocated word).
 static __device__ __align__(256) unsigned char g_decode_static_scratch[kDecodeStaticScratchBytes];
+static __device__ uint32_t g_decode_static_status;
+
+std::mutex g_static_mu;
+void* g_static_scratch_addr[64] = {nullptr};
+uint32_t* g_static_status_addr[64] = {nullptr};
 
 }  // namespace
 
-cudaError_t decode_static_scratch(void** ptr) {
-  // Host code may not use the array's name as a device address; look up the
-  // address once per device, with that device current, and reuse it.
-  static std::mutex mu;
-  static void* addr[64] = {nullptr};
+cudaError_t decode_static_scratch(void** ptr, uint32_t** status) {
+  // Host code may not use the arrays' names as device addresses; look the
+  // addresses up once per device, with that device current, and reuse them.
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lk(mu);
-  if (!addr[dev]) {
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  if (!g_static_scratch_addr[dev]) {
     void* p = nullptr;
+    void* w = nullptr;
     e = cudaGetSymbolAddress(&p, g_decode_static_scratch);
     if (e != cudaSuccess) return e;
-    addr[dev] = p;
+    e = cudaGetSymbolAddress(&w, g_decode_static_status);
+    if (e != cudaSuccess) return e;
+    g_static_status_addr[dev] = static_cast<uint32_t*>(w);
+    g_static_scratch_addr[dev] = p;
   }
-  *ptr = addr[dev];
+  *ptr = g_static_scratch_addr[dev];
+  *status = g_static_status_addr[dev];
   return cudaSuccess;
+}
+
+uint32_t* decode_static_status_if_used() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_static_mu);
+  return g_static_status_addr[dev];
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mks,

@@ -160,9 +160,13 @@ cudaError_t launch_cache_centroids(const CacheArgs& a, cudaStream_t stream);
 
 // Fixed-size device scratch used by the allocation-free decode entry point.
 constexpr size_t kDecodeStaticScratchBytes = size_t(16) << 20;
-// Device address of that scratch on the current device (looked up once per
-// device with cudaGetSymbolAddress; no allocation).
-cudaError_t decode_static_scratch(void** ptr);
+// Device addresses of that scratch and of its status word on the current
+// device (looked up once per device with cudaGetSymbolAddress; no
+// allocation).
+cudaError_t decode_static_scratch(void** ptr, uint32_t** status);
+// The status word of the allocation-free decode on the current device, or
+// NULL if that entry point has not run on it (no lookup, no allocation).
+uint32_t* decode_static_status_if_used();
 
 // Shared-memory bytes the prefill kernel needs (host side, for the opt-in).
 size_t prefill_smem_bytes();

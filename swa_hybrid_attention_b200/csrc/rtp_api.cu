@@ -95,6 +95,13 @@ uint32_t* status_word(int dev) {
   return g_status[dev];
 }
 
+// The status word of `dev` if it has been created, else NULL (no allocation).
+uint32_t* existing_status_word(int dev) {
+  if (dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_status_mu);
+  return g_status[dev];
+}
+
 // ------------------------------------------------------------- TMA encoding
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -733,16 +740,15 @@ rtp_status prepare_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int
 }
 
 // Scratch pointers, status word, TMA maps and the launch.
+// `status`: the device word the kernels report in; NULL = the library's
+// allocated status word of the current device.
 rtp_status run_decode(DecodeArgs& a, const DecodeLayout& L, char* ws, int32_t* sel_out, int32_t* cnt_out,
-                      bool with_status, const rtp_clusters* cl, void* stream) {
+                      uint32_t* status, const rtp_clusters* cl, void* stream) {
   a.sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(ws + L.sel_off);
   a.cnt = cnt_out ? cnt_out : reinterpret_cast<int32_t*>(ws + L.cnt_off);
   a.partial = reinterpret_cast<float*>(ws + L.part_off);
-  a.status = nullptr;
-  if (with_status) {
-    a.status = status_word(current_device());
-    if (!a.status) return RTP_ERR_NO_MEMORY;
-  }
+  a.status = status ? status : status_word(current_device());
+  if (!a.status) return RTP_ERR_NO_MEMORY;
   const long slabs = static_cast<long>(a.batch) * a.n_kv_heads;
   CUtensorMap mk, mv, mks, mvs;
   if (!encode_bf16_3d(&mk, a.kcache, a.cache_len, slabs, 64, a.cache_cap) ||
@@ -814,7 +820,7 @@ rtp_status rtp_sparse_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, 
                                  cnt_out, L, a);
   if (st != RTP_OK) return st;
   if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return RTP_ERR_INVALID_ARG;
-  return run_decode(a, L, static_cast<char*>(workspace), sel_out, cnt_out, true, nullptr, stream);
+  return run_decode(a, L, static_cast<char*>(workspace), sel_out, cnt_out, nullptr, nullptr, stream);
 }
 
 rtp_status rtp_sparse_decode_clustered(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len,
@@ -829,7 +835,7 @@ rtp_status rtp_sparse_decode_clustered(const rtp_attn_cfg* cfg, const uint8_t* k
       prepare_decode(cfg, kind_host, cache_len, q, kcache, vcache, nullptr, proj, cl, o, sel_out, cnt_out, L, a);
   if (st != RTP_OK) return st;
   if (!workspace || ws_bytes < L.total || !aligned16(workspace)) return RTP_ERR_INVALID_ARG;
-  return run_decode(a, L, static_cast<char*>(workspace), sel_out, cnt_out, true, cl, stream);
+  return run_decode(a, L, static_cast<char*>(workspace), sel_out, cnt_out, nullptr, cl, stream);
 }
 
 rtp_status rtp_sparse_decode_noalloc(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int cache_len, const void* q,
@@ -843,9 +849,10 @@ rtp_status rtp_sparse_decode_noalloc(const rtp_attn_cfg* cfg, const uint8_t* kin
   if (st != RTP_OK) return st;
   if (L.total > kDecodeStaticScratchBytes) return RTP_ERR_INVALID_ARG;  // beyond the fixed scratch
   void* scratch = nullptr;
-  if (decode_static_scratch(&scratch) != cudaSuccess || !scratch) return RTP_ERR_CUDA;
-  // no status word: getting one may allocate
-  return run_decode(a, L, static_cast<char*>(scratch), sel_out, cnt_out, false, nullptr, stream);
+  uint32_t* status = nullptr;
+  if (decode_static_scratch(&scratch, &status) != cudaSuccess || !scratch || !status) return RTP_ERR_CUDA;
+  // the kernels report in the static status word, not the allocated one
+  return run_decode(a, L, static_cast<char*>(scratch), sel_out, cnt_out, status, nullptr, stream);
 }
 
 size_t rtp_cache_cluster_workspace_bytes(const rtp_attn_cfg* cfg, int clu_end) {
@@ -1047,11 +1054,18 @@ rtp_status rtp_selftest_bounded_wait(unsigned limit_ms, void* stream) {
 rtp_status rtp_last_device_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return RTP_ERR_CUDA;
-  uint32_t* w = status_word(current_device());
-  if (!w) return RTP_ERR_NO_MEMORY;
+  // Read (and clear) the words that exist on this device: the allocated one
+  // once any entry point has created it, the static one of the
+  // allocation-free decode once that has run.  Reading creates neither.
+  uint32_t* words[2] = {existing_status_word(current_device()), decode_static_status_if_used()};
   uint32_t v = 0;
-  if (cudaMemcpy(&v, w, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return RTP_ERR_CUDA;
-  if (v != 0 && cudaMemset(w, 0, sizeof(uint32_t)) != cudaSuccess) return RTP_ERR_CUDA;
+  for (uint32_t* w : words) {
+    if (!w) continue;
+    uint32_t x = 0;
+    if (cudaMemcpy(&x, w, sizeof(x), cudaMemcpyDeviceToHost) != cudaSuccess) return RTP_ERR_CUDA;
+    if (x != 0 && cudaMemset(w, 0, sizeof(uint32_t)) != cudaSuccess) return RTP_ERR_CUDA;
+    v |= x;
+  }
   if (v & RTP_DEVERR_TIMEOUT) return RTP_ERR_TIMEOUT;
   if (v) return RTP_ERR_INVALID_ARG;
   return RTP_OK;

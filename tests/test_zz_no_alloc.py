@@ -78,6 +78,29 @@ def test_noalloc_matches_workspace_path_on_two_calls(rtp, cuda_device):
     assert rtp.rtp_last_device_status() == rtp.RTP_OK
 
 
+def test_noalloc_calls_and_status_read_change_no_free_memory(rtp, cuda_device):
+    """Once the first call on the device has looked up the array's address,
+    further calls, and reading the status words back, leave the device's free
+    memory exactly as it was: nothing is allocated or freed."""
+    cfg = rtp.AttnConfig(2, 1, 16, 4, WINDOW, BLOCK, TOPK, N_LOCAL)
+    d = make_case(5, cuda_device)
+    o = torch.empty_like(d["q"])
+
+    def call():
+        rtp.rtp_sparse_decode_noalloc(cfg, KINDS, 4096, d["q"], d["kcache"], d["vcache"], d["C"], d["proj"], o)
+
+    call()
+    assert rtp.rtp_last_device_status() == rtp.RTP_OK
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        call()
+    status = rtp.rtp_last_device_status()
+    torch.cuda.synchronize()
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert status == rtp.RTP_OK
+
+
 def test_noalloc_rejects_shapes_beyond_its_scratch(rtp, cuda_device):
     # 64 sequences x 4 heads x 64 splits x 8 heads of partials is ~35 MB > 16 MiB
     cfg = rtp.AttnConfig(64, 1, 32, 4, 8192, 128, 32, 4)
@@ -106,6 +129,8 @@ def test_noalloc_step_replayed_from_a_cuda_graph(rtp, cuda_device):
         step()  # first call on the device: the scratch address lookup happens outside the capture
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
+    # torch captures in the default "global" mode, in which a cudaMalloc made
+    # during the capture fails it.
     with torch.cuda.graph(graph, stream=s):
         step()
     torch.cuda.synchronize()
