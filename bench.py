@@ -418,59 +418,86 @@ def time_selection_variants(rtp, w, device, reps=2):
     return out
 
 
-def time_cp_projection(rtp, w, res, device, world=8, link_gbs=770.0):
+def time_cp_projection(rtp, w, res, device, world=8, link_gbs=770.0, reserve_sms=16):
     """Context-parallel prefill of the main layer split over `world` ranks,
-    projected from one GPU: each rank's ranged prefill is timed here on its own
-    rows (its K/V buffer holds every row it may read), and the K/V bytes it
-    would receive are counted from the row needs of its heads and selection.
-    Transfer time = bytes / the measured peer-copy bandwidth.  Not a
-    multi-GPU measurement."""
+    projected from one GPU.  Each rank's work is timed here on its own rows
+    (its K/V buffer holds every row it may read), as one ranged launch and as
+    the overlapped driver runs it (context_parallel.cp_prefill_layer): the
+    split plan's local tiles (the first on reserve_sms fewer CTAs, sized to
+    the exchange), then the tiles that need fetched rows.  The K/V bytes a
+    rank would receive are counted from its heads' row needs and selection;
+    transfer time = bytes / the measured peer-copy bandwidth.  With overlap a
+    rank takes local + remote + the part of the transfer its local tiles do
+    not hide.  Not a multi-GPU measurement."""
     from swa_hybrid_attention_b200 import context_parallel as cp
 
     plan, bufs = res["plan"], res["bufs"]
     q, k, v = res["q"], res["k"], res["v"]
     cfg = plan.cfg
     stream = torch.cuda.current_stream()
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
     slot_of = {h: s for s, h in enumerate(plan.slot_heads)}
     sel = bufs["sel"].cpu() if plan.n_sparse else None
     cnt = bufs["sel_cnt"].cpu() if plan.n_sparse else None
+    sel_d = bufs["sel"] if plan.n_sparse else None
+    cnt_d = bufs["sel_cnt"] if plan.n_sparse else None
     # every rank's inputs first, then all ranks' launches back to back, twice
     # (the second pass is timed), so that each launch runs at the clocks of a
     # long busy stretch like the single-GPU layer rather than as a short burst
     setup = []
     for qb, qe in cp.cp_ranges(cfg.seq, world):
-        pr = rtp.Plan(cfg, res["kinds"], q_range=(qb, qe))
+        pr = rtp.Plan(cfg, res["kinds"], q_range=(qb, qe), key_begin=qb)
         needs = cp.kv_needs(res["kinds"], cfg.window, cfg.block, (qb, qe), cfg.batch, sel, cnt, slot_of)
         kv_bytes = sum(hi - lo for iv in needs.values() for lo, hi in iv) * 2 * 128 * 2
+        transfer_s = kv_bytes / (link_gbs * 1e9)
+        head = cp.overlap_head_items(rtp.rtp_plan_work_items(pr.handle), pr.n_local, cfg, transfer_s,
+                                     sms - reserve_sms) if qb > 0 else 0
         # the rank's own Q rows and the K/V rows before its end (a rank's buffer)
         tensors = (q[:, :, qb:qe].contiguous(), k[:, :, :qe].contiguous(), v[:, :, :qe].contiguous())
-        setup.append((pr, qb, qe, kv_bytes, tensors, torch.empty_like(tensors[0])))
+        setup.append((pr, qb, qe, kv_bytes, head, tensors, torch.empty_like(tensors[0])))
     ranks = []
     for pass_ in range(2):
         evs = []
-        for pr, qb, qe, kv_bytes, (q_loc, k_loc, v_loc), o_loc in setup:
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            rtp.rtp_hybrid_prefill(pr.handle, q_loc, k_loc, v_loc, bufs["sel"] if plan.n_sparse else None,
-                                   bufs["sel_cnt"] if plan.n_sparse else None, o_loc, stream)
-            b.record(stream)
-            evs.append((a, b))
+        for pr, qb, qe, kv_bytes, head, (q_loc, k_loc, v_loc), o_loc in setup:
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            e[0].record(stream)
+            rtp.rtp_hybrid_prefill(pr.handle, q_loc, k_loc, v_loc, sel_d, cnt_d, o_loc, stream)
+            e[1].record(stream)
+            rtp.rtp_hybrid_prefill_items(pr.handle, q_loc, k_loc, v_loc, sel_d, cnt_d, o_loc, 0, head,
+                                         sms - reserve_sms, stream)
+            e[2].record(stream)
+            rtp.rtp_hybrid_prefill_items(pr.handle, q_loc, k_loc, v_loc, sel_d, cnt_d, o_loc, head, pr.n_local, 0,
+                                         stream)
+            e[3].record(stream)
+            rtp.rtp_hybrid_prefill_items(pr.handle, q_loc, k_loc, v_loc, sel_d, cnt_d, o_loc, pr.n_local,
+                                         pr.n_items, 0, stream)
+            e[4].record(stream)
+            evs.append(e)
         torch.cuda.synchronize()
         if pass_ == 1:
-            for (pr, qb, qe, kv_bytes, _, _), (a, b) in zip(setup, evs):
-                ranks.append({"q_rows": qe - qb, "prefill_ms": a.elapsed_time(b), "kv_bytes_in": kv_bytes,
-                              "transfer_ms": kv_bytes / (link_gbs * 1e9) * 1e3})
+            for (pr, qb, qe, kv_bytes, head, _, _), e in zip(setup, evs):
+                transfer = kv_bytes / (link_gbs * 1e9) * 1e3
+                head_ms, tail_ms, remote_ms = e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]), e[3].elapsed_time(e[4])
+                local_ms = head_ms + tail_ms
+                ranks.append({"q_rows": qe - qb, "prefill_ms": e[0].elapsed_time(e[1]), "kv_bytes_in": kv_bytes,
+                              "transfer_ms": transfer, "items": pr.n_items, "local_items": pr.n_local,
+                              "head_items": head, "head_ms": head_ms, "local_ms": local_ms, "remote_ms": remote_ms,
+                              "exposed_transfer_ms": max(0.0, transfer - local_ms),
+                              "overlapped_ms": local_ms + remote_ms + max(0.0, transfer - local_ms)})
     for pr, *_ in setup:
         pr.close()
     del setup
     torch.cuda.empty_cache()
-    worst = max(r["prefill_ms"] + r["transfer_ms"] for r in ranks)
     return {"world": world, "ranks": ranks, "compute_ms_max": max(r["prefill_ms"] for r in ranks),
             "kv_bytes_in_max": max(r["kv_bytes_in"] for r in ranks), "link_gbs": link_gbs,
-            "projected_ms_no_overlap": worst,
+            "reserve_sms": reserve_sms,
+            "projected_ms_no_overlap": max(r["prefill_ms"] + r["transfer_ms"] for r in ranks),
+            "projected_ms_overlap": max(r["overlapped_ms"] for r in ranks),
+            "exposed_transfer_ms_max": max(r["exposed_transfer_ms"] for r in ranks),
             "note": "projection from one GPU: per-rank prefill timed on its own rows (all ranks back to back, "
-                    "second pass); K/V transfer = bytes / measured 770 GB/s peer copy; the indexer, selection "
-                    "and centroid all-gather (<1 ms) are not included"}
+                    "second pass), as one launch and as the overlapped split (local tiles: capped head launch + "
+                    "tail; then remote tiles); K/V transfer = bytes / measured 770 GB/s peer copy; the indexer, "
+                    "selection and centroid all-gather (<1 ms) are not included"}
 
 
 def time_e2e(rtp, w, res, steps, device, chunks=16):
@@ -671,13 +698,24 @@ def time_clustered_decode(rtp, w, d, flush, flush_read, steps, stream, n_cluster
     B = w.block
     clu_end = (Lc // B - w.n_local) * B
     ns = sum(1 for k in kinds if k == inputs.SPARSE)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    cl = rtp.cluster_cache(d["kcache"], d["vcache"], d["proj"], kinds, clu_end=clu_end, n_clusters=n_clusters,
-                           iters=iters, block=B, stream=stream)
-    b.record(stream)
-    torch.cuda.synchronize()
-    km_ms = a.elapsed_time(b)
+    # k-means, warm: the clusters' arrays and the workspace are allocated once,
+    # outside the timed region; the median of 5 timed runs after a warm-up
+    ccfg = rtp.AttnConfig(w.batch, Lc, w.n_kv_heads, w.n_kv_heads, 1, B, 0, 1)
+    cl = rtp.Clusters(w.batch, w.n_kv_heads, clu_end, n_clusters, B, d["kcache"].device)
+    km_ws_bytes = rtp.rtp_cache_cluster_workspace_bytes(ccfg, clu_end)
+    km_ws = torch.empty(km_ws_bytes, dtype=torch.uint8, device=d["kcache"].device)
+    km_runs = []
+    for i in range(6):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        rtp.rtp_cache_cluster(ccfg, kinds, iters, d["kcache"], d["vcache"], d["proj"], cl, km_ws, km_ws_bytes,
+                              stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i > 0:
+            km_runs.append(a.elapsed_time(b))
+    km_ms = statistics.median(km_runs)
+    del km_ws
     cfg = rtp.AttnConfig(w.batch, Lc, w.n_q_heads, w.n_kv_heads, w.window, B, w.topk, w.n_local)
     ws_bytes = rtp.rtp_decode_clustered_workspace_bytes(cfg, kinds, Lc, clu_end)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=d["q"].device)
@@ -717,6 +755,7 @@ def time_clustered_decode(rtp, w, d, flush, flush_read, steps, stream, n_cluster
     bytes_ = keys * 128 * 2 * 2 + w.batch * ns * cl.max_chunks * 16 * 4 + w.batch * w.n_q_heads * 128 * 2 * 2
     chunks = cl.n_chunks.cpu()[:, [h for h, k in enumerate(kinds) if k == inputs.SPARSE]].float()
     return {"n_clusters": n_clusters, "iters": iters, "clu_end": clu_end, "kmeans_ms": km_ms,
+            "kmeans_ms_runs": km_runs,
             "mean_chunks_per_head": float(chunks.mean()), "ms_per_step": ms, "algorithmic_bytes": bytes_,
             "gb_s": bytes_ / (ms * 1e-3) / 1e9, "status": rtp.status_str(status)}
 
@@ -859,6 +898,36 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def secondary_summary(sec: dict) -> dict:
+    """The secondary figures in a few short keys (ms unless named _us)."""
+    out = {}
+    d = sec.get("decode_8x256k") or {}
+    if "ms_per_step" in d:
+        out["decode_8x256k_us"] = round(d["ms_per_step"] * 1e3, 2)
+        out["decode_hbm_frac"] = round(d["gb_s"] / 6552.6, 3) if "gb_s" in d else None
+        if d.get("graph"):
+            out["decode_graph_us"] = round(d["graph"]["ms_per_step"] * 1e3, 2)
+        c = d.get("clustered") or {}
+        if "ms_per_step" in c:
+            out["clustered_decode_us"] = round(c["ms_per_step"] * 1e3, 2)
+        if "kmeans_ms" in c:
+            out["kmeans_ms"] = round(c["kmeans_ms"], 2)
+    for key, name in (("v2_128k_48_layers", "v2_128k_ms_per_layer"), ("v1_32k_48_layers", "v1_32k_ms_per_layer")):
+        if "ms_per_layer" in sec.get(key, {}):
+            out[name] = round(sec[key]["ms_per_layer"], 3)
+            out[name.replace("ms_per_layer", "tflops_executed")] = round(sec[key]["tflops_executed"], 1)
+    cp = sec.get("context_parallel_projection") or {}
+    for key in ("projected_ms_no_overlap", "projected_ms_overlap", "exposed_transfer_ms_max"):
+        if key in cp:
+            out["cp8_" + key] = round(cp[key], 3)
+    dyn = sec.get("dynamic_selection") or {}
+    for key in ("rowmax_scores", "per_head"):
+        if key in dyn:
+            out[key + "_select_ms"] = round(dyn[key]["select_ms"], 3)
+            out[key + "_prefill_ms"] = round(dyn[key]["prefill_ms"], 2)
+    return out
+
+
 def run_ours(args, rank, world, local):
     from swa_hybrid_attention_b200 import build
 
@@ -894,6 +963,10 @@ def run_ours(args, rank, world, local):
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     traffic = prefill_traffic(w)
     extra = {}
+    if args.only == "cp":
+        if rank == 0:
+            print(json.dumps({"context_parallel_projection": time_cp_projection(rtp, w, res, device)}), flush=True)
+        return
     if not args.no_secondary and world == 1:
         extra["dynamic"] = time_dynamic(rtp, w, res, device)
         extra["cp"] = time_cp_projection(rtp, w, res, device)
@@ -958,6 +1031,7 @@ def run_ours(args, rank, world, local):
         line["cpu_baseline"] = cpu_base
     if secondary:
         line["secondary"] = secondary
+        line["summary"] = secondary_summary(secondary)  # last, short: the end of the line carries the key figures
     print(json.dumps(line), flush=True)
 
 
@@ -975,7 +1049,7 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=10.0)
     ap.add_argument("--decode-steps", type=int, default=256)
     ap.add_argument("--seq", type=int, default=0, help="override the primary workload's length (profiling)")
-    ap.add_argument("--only", choices=["all", "decode", "selection"], default="all",
+    ap.add_argument("--only", choices=["all", "decode", "selection", "cp"], default="all",
                     help="run only part of the bench (decode step; selection variants, for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:

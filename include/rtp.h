@@ -144,6 +144,29 @@ rtp_status rtp_route_heads(const rtp_attn_cfg* cfg, const uint8_t* kind_host, vo
  * ---------------------------------------------------------------------- */
 rtp_status rtp_route_heads_range(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int q_begin, int q_end,
                                  void* stream, rtp_plan** out);
+
+/* ------------------------------------------------------------------------
+ * rtp_route_heads_split — rtp_route_heads_range with the work list in two
+ * parts, so that a context-parallel rank can start attention while the
+ * earlier K/V rows it needs are still arriving (RTPurbo page, "RTP-LLM：
+ * RTPurbo 在长文上的极致性能优化": context parallelism with communication
+ * overlapped by computation).
+ *   key_begin  0 <= key_begin <= q_begin: the first K/V row present locally
+ *   The first rtp_plan_num_local_items(plan) items are the tiles whose
+ *   visible keys all lie at or after key_begin (streaming heads whose window
+ *   starts there; a full or sparse head always sees row 0, so its tiles are
+ *   local only when key_begin = 0); the other items follow.  Each part is
+ *   ordered longest first.  Run the parts with rtp_hybrid_prefill_items;
+ *   rtp_hybrid_prefill runs them all.  Every other call works as with
+ *   rtp_route_heads_range.
+ * Errors: as rtp_route_heads_range, and RTP_ERR_INVALID_ARG for key_begin
+ * outside [0, q_begin].
+ * ---------------------------------------------------------------------- */
+rtp_status rtp_route_heads_split(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int q_begin, int q_end,
+                                 int key_begin, void* stream, rtp_plan** out);
+/* Items of a split plan that see only local keys (the whole list for a plan
+ * made by rtp_route_heads / rtp_route_heads_range); -1 for NULL. */
+long rtp_plan_num_local_items(const rtp_plan* plan);
 void rtp_plan_destroy(rtp_plan* plan);
 
 /* Number of retrieval slots (KV heads of kind RTP_HEAD_SPARSE). */
@@ -296,6 +319,21 @@ rtp_status rtp_hybrid_prefill_heads(const rtp_plan* plan, const void* q, const v
  * ---------------------------------------------------------------------- */
 rtp_status rtp_hybrid_prefill(const rtp_plan* plan, const void* q, const void* k, const void* v,
                               const int32_t* sel, const int32_t* sel_cnt, void* o, void* stream);
+
+/* ------------------------------------------------------------------------
+ * rtp_hybrid_prefill_items — rtp_hybrid_prefill for the work items
+ * [item_begin, item_end) of the plan's list only (the order of
+ * rtp_plan_work_items), on at most max_ctas persistent CTAs (0 = one per
+ * SM).  Tiles are computed exactly as in rtp_hybrid_prefill (same result bit
+ * for bit), so launches over disjoint item ranges fill disjoint tiles of o.
+ * A cap below the SM count leaves SMs free for kernels that must run
+ * alongside, e.g. the collectives of a K/V exchange.
+ *   0 <= item_begin <= item_end <= rtp_plan_num_items(plan); max_ctas >= 0
+ * Errors: as rtp_hybrid_prefill, and RTP_ERR_INVALID_ARG for a bad range.
+ * ---------------------------------------------------------------------- */
+rtp_status rtp_hybrid_prefill_items(const rtp_plan* plan, const void* q, const void* k, const void* v,
+                                    const int32_t* sel, const int32_t* sel_cnt, void* o, long item_begin,
+                                    long item_end, int max_ctas, void* stream);
 
 /* ------------------------------------------------------------------------
  * rtp_hybrid_prefill_host — the prefill of one layer whose Q, K, V and O are

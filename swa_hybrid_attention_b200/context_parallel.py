@@ -17,9 +17,18 @@ tiles) and holds Q, K and V of those rows.  Its attention needs, for every
 The rows are requested from their owners and delivered with two all-to-alls
 (request lists, then payload); received rows land in this GPU's memory
 before any kernel reads them (no kernel reads another GPU's memory).  The
-attention itself is the library's prefill on a ranged plan
-(rtp_route_heads_range), so a rank computes exactly the tiles the
+attention itself is the library's prefill on a split ranged plan
+(rtp_route_heads_split), so a rank computes exactly the tiles the
 single-GPU prefill would compute for its rows, bit for bit.
+
+Overlap: the plan's work list starts with the tiles whose visible keys are
+all this rank's own rows (streaming heads whose window starts inside the
+range).  Those run on the compute stream while the exchange runs on a side
+stream; the first of them on all but a few SMs, so that the collectives'
+kernels have SMs to run on (a prefill CTA holds an SM's registers), the rest
+on every SM.  The tiles that need fetched rows (full and sparse heads always
+see row 0; streaming tiles near the range's start) run once the exchange is
+done.
 
 This module is host-side orchestration: which rows to fetch, and the
 collectives (torch.distributed, NCCL on GPUs; gloo with host staging where
@@ -145,16 +154,17 @@ def _all_gather(parts: list, x: torch.Tensor, group) -> None:
 
 
 def exchange_kv(k_loc: torch.Tensor, v_loc: torch.Tensor, needs: dict, ranges: list, rank: int, kf: torch.Tensor,
-                vf: torch.Tensor, group=None) -> int:
-    """Fill kf / vf ([batch][H][>= end][128]) with this rank's own rows and
-    the rows in `needs`, fetched from their owners.  k_loc / v_loc hold this
-    rank's rows [begin, end).  Every rank of the group must call it (it runs
-    three all-to-alls).  Returns the payload bytes received."""
+                vf: torch.Tensor, group=None, copy_own: bool = True) -> int:
+    """Fill kf / vf ([batch][H][>= end][128]) with the rows in `needs`,
+    fetched from their owners, and (copy_own) this rank's own rows.  k_loc /
+    v_loc hold this rank's rows [begin, end).  Every rank of the group must
+    call it (it runs three all-to-alls).  Returns the payload bytes received."""
     world = len(ranges)
     dev = k_loc.device
     qb, qe = ranges[rank]
-    kf[:, :, qb:qe].copy_(k_loc)
-    vf[:, :, qb:qe].copy_(v_loc)
+    if copy_own:
+        kf[:, :, qb:qe].copy_(k_loc)
+        vf[:, :, qb:qe].copy_(v_loc)
     reqs = split_by_owner(needs, ranges)
     assert reqs[rank].numel() == 0, "a rank never needs rows it owns from itself"
     # 1. how many requests go to / come from each rank
@@ -214,14 +224,46 @@ def gather_centroids(centroids: torch.Tensor, ranges: list, rank: int, block: in
 # ------------------------------------------------------------------ layer
 
 
+# Planner cost of one work item, in KV tiles of 128 keys (the same count the
+# library's longest-first ordering uses), for sizing the overlapped launch.
+def _item_tiles(item, cfg: rtp.AttnConfig) -> int:
+    kind, t = int(item[0]) & 0xFF, int(item[3])
+    if kind == FULL:
+        return t + 1
+    if kind == SWA:
+        first = 128 * t - cfg.window + 1
+        return t - (0 if first <= 0 else first // 128) + 1
+    return min(t + 1, cfg.topk + 1 + cfg.n_local)
+
+
+def overlap_head_items(items, n_local: int, cfg: rtp.AttnConfig, exchange_s: float, ctas: int,
+                       tile_s: float = 2.4e-6) -> int:
+    """How many of the first local items the capped launch should run so that
+    it lasts about as long as the exchange: ctas CTAs, each taking a KV tile
+    of one query-head pair in about tile_s seconds (the prefill kernel's
+    measured rate on B200: ~2.4 us per pair-tile per SM)."""
+    budget = exchange_s / tile_s * ctas
+    acc = 0
+    for i in range(n_local):
+        if acc >= budget:
+            return i
+        acc += _item_tiles(items[i], cfg)
+    return n_local
+
+
 def cp_prefill_layer(q_loc, k_loc, v_loc, kinds, proj, cfg: rtp.AttnConfig, group=None, dynamic: dict | None = None,
-                     stream=None) -> tuple:
+                     stream=None, overlap: bool = True, reserve_sms: int = 16, link_gbs: float = 770.0) -> tuple:
     """One layer of context-parallel prefill on this rank.
 
     cfg describes the whole sequence (cfg.seq = total tokens); q_loc, k_loc,
     v_loc hold this rank's rows of cp_ranges(cfg.seq, world)[rank].  Returns
     (o_loc, info) with o_loc the attention output of this rank's rows and
-    info the bytes received and the rows fetched.
+    info the bytes received, the rows fetched and the work split.
+    overlap: run the tiles that need no fetched row while the exchange is in
+    flight (side stream); the first of them on reserve_sms fewer CTAs, sized
+    to the exchange's duration at link_gbs.  stream: a torch.cuda.Stream
+    (None: the current stream); everything this rank queues goes on it, the
+    exchange on a side stream joined before the remote tiles.
     """
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
@@ -229,32 +271,55 @@ def cp_prefill_layer(q_loc, k_loc, v_loc, kinds, proj, cfg: rtp.AttnConfig, grou
     qb, qe = ranges[rank]
     assert q_loc.shape[2] == qe - qb and k_loc.shape[2] == qe - qb
     dev = q_loc.device
-    plan = rtp.Plan(cfg, kinds, stream, q_range=(qb, qe))
+    comp = torch.cuda.current_stream(dev) if stream is None else stream
+    plan = rtp.Plan(cfg, kinds, comp, q_range=(qb, qe), key_begin=qb)
     try:
-        bufs = plan.buffers(dev)
-        slot_of = {h: s for s, h in enumerate(plan.slot_heads)}
-        sel = cnt = None
-        if plan.n_sparse:
-            rtp.rtp_indexer_project(plan.handle, q_loc, k_loc, proj, bufs["centroids"], bufs["qbar"], stream)
-            gather_centroids(bufs["centroids"], ranges, rank, cfg.block, group)
-            if dynamic is None:
-                rtp.rtp_block_select(plan.handle, bufs["qbar"], bufs["centroids"], bufs["sel"], bufs["sel_cnt"],
-                                     stream)
+        with torch.cuda.stream(comp):
+            bufs = plan.buffers(dev)
+            slot_of = {h: s for s, h in enumerate(plan.slot_heads)}
+            sel = cnt = None
+            if plan.n_sparse:
+                rtp.rtp_indexer_project(plan.handle, q_loc, k_loc, proj, bufs["centroids"], bufs["qbar"], comp)
+                gather_centroids(bufs["centroids"], ranges, rank, cfg.block, group)
+                if dynamic is None:
+                    rtp.rtp_block_select(plan.handle, bufs["qbar"], bufs["centroids"], bufs["sel"],
+                                         bufs["sel_cnt"], comp)
+                else:
+                    beta = dynamic.get("beta")
+                    rtp.rtp_block_select_dynamic(plan.handle, bufs["qbar"], bufs["centroids"], dynamic["mass"],
+                                                 dynamic.get("min_k", 0),
+                                                 rtp.default_selection_beta(cfg) if beta is None else beta,
+                                                 bufs["sel"], bufs["sel_cnt"], comp)
+                sel, cnt = bufs["sel"].cpu(), bufs["sel_cnt"].cpu()
+            needs = kv_needs(kinds, cfg.window, cfg.block, (qb, qe), cfg.batch, sel, cnt, slot_of)
+            rows = sum(hi - lo for iv in needs.values() for lo, hi in iv)
+            kf = torch.empty(cfg.batch, cfg.n_kv_heads, qe, 128, dtype=k_loc.dtype, device=dev)
+            vf = torch.empty_like(kf)
+            kf[:, :, qb:qe].copy_(k_loc)
+            vf[:, :, qb:qe].copy_(v_loc)
+            o_loc = torch.empty_like(q_loc)
+            sel_d = bufs["sel"] if plan.n_sparse else None
+            cnt_d = bufs["sel_cnt"] if plan.n_sparse else None
+            n_loc, n_all = plan.n_local, plan.n_items
+            n_head = 0
+            if overlap and world > 1 and n_loc > 0:
+                sms = torch.cuda.get_device_properties(dev).multi_processor_count
+                ctas = max(1, sms - reserve_sms)
+                exchange_s = 2 * rows * 128 * k_loc.element_size() / (link_gbs * 1e9)
+                n_head = overlap_head_items(rtp.rtp_plan_work_items(plan.handle), n_loc, cfg, exchange_s, ctas)
+                side = torch.cuda.Stream(dev)
+                side.wait_stream(comp)
+                # queued before the exchange, whose host side blocks on its own stream only
+                rtp.rtp_hybrid_prefill_items(plan.handle, q_loc, kf, vf, sel_d, cnt_d, o_loc, 0, n_head, ctas, comp)
+                rtp.rtp_hybrid_prefill_items(plan.handle, q_loc, kf, vf, sel_d, cnt_d, o_loc, n_head, n_loc, 0, comp)
+                with torch.cuda.stream(side):
+                    received = exchange_kv(k_loc, v_loc, needs, ranges, rank, kf, vf, group, copy_own=False)
+                comp.wait_stream(side)
+                rtp.rtp_hybrid_prefill_items(plan.handle, q_loc, kf, vf, sel_d, cnt_d, o_loc, n_loc, n_all, 0, comp)
             else:
-                beta = dynamic.get("beta")
-                rtp.rtp_block_select_dynamic(plan.handle, bufs["qbar"], bufs["centroids"], dynamic["mass"],
-                                             dynamic.get("min_k", 0),
-                                             rtp.default_selection_beta(cfg) if beta is None else beta, bufs["sel"],
-                                             bufs["sel_cnt"], stream)
-            sel, cnt = bufs["sel"].cpu(), bufs["sel_cnt"].cpu()
-        needs = kv_needs(kinds, cfg.window, cfg.block, (qb, qe), cfg.batch, sel, cnt, slot_of)
-        kf = torch.empty(cfg.batch, cfg.n_kv_heads, qe, 128, dtype=k_loc.dtype, device=dev)
-        vf = torch.empty_like(kf)
-        received = exchange_kv(k_loc, v_loc, needs, ranges, rank, kf, vf, group)
-        o_loc = torch.empty_like(q_loc)
-        rtp.rtp_hybrid_prefill(plan.handle, q_loc, kf, vf, bufs["sel"] if plan.n_sparse else None,
-                               bufs["sel_cnt"] if plan.n_sparse else None, o_loc, stream)
-        rows = sum(hi - lo for iv in needs.values() for lo, hi in iv)
-        return o_loc, {"bytes_received": received, "rows_fetched": rows, "q_range": (qb, qe)}
+                received = exchange_kv(k_loc, v_loc, needs, ranges, rank, kf, vf, group, copy_own=False)
+                rtp.rtp_hybrid_prefill(plan.handle, q_loc, kf, vf, sel_d, cnt_d, o_loc, comp)
+        return o_loc, {"bytes_received": received, "rows_fetched": rows, "q_range": (qb, qe), "items": n_all,
+                       "local_items": n_loc, "head_items": n_head}
     finally:
         plan.close()

@@ -44,6 +44,8 @@ struct rtp_plan {
   std::vector<int32_t> slot_heads;
   std::vector<int32_t> items_host;  // [n_items][4]
   long n_items = 0;
+  long n_local = 0;  // items [0, n_local) see only keys at or after key_begin
+  int key_begin = 0;
   void* d_mem = nullptr;
   int4* d_items = nullptr;
   int32_t* d_slot_heads = nullptr;
@@ -219,8 +221,14 @@ rtp_status indexer_run(const rtp_plan* plan, const void* q, const void* k, int s
 // The prefill of a (possibly ranged) plan.  q and o point at the plan's first
 // query row of slab 0, their slabs q_slab rows apart; k and v start at row 0,
 // their slabs kv_slab rows apart.
+// Work items [item_begin, item_end) of the plan's list (item_end < 0: to the
+// end) run on at most max_ctas persistent CTAs (0: one per SM).
 rtp_status prefill_run(const rtp_plan* plan, const void* q, int q_slab, const void* k, const void* v, int kv_slab,
-                       const int32_t* sel, const int32_t* sel_cnt, void* o, void* stream, int sel_heads = 0) {
+                       const int32_t* sel, const int32_t* sel_cnt, void* o, void* stream, int sel_heads = 0,
+                       long item_begin = 0, long item_end = -1, int max_ctas = 0) {
+  if (item_end < 0) item_end = plan->n_items;
+  if (item_begin < 0 || item_begin > item_end || item_end > plan->n_items || max_ctas < 0)
+    return RTP_ERR_INVALID_ARG;
   if (!q || !k || !v || !o) return RTP_ERR_INVALID_ARG;
   if (plan->n_sparse > 0 && (!sel || !sel_cnt)) return RTP_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return RTP_ERR_INVALID_ARG;
@@ -234,8 +242,8 @@ rtp_status prefill_run(const rtp_plan* plan, const void* q, int q_slab, const vo
       !encode_bf16_3d(&mv, v, plan->q_end, static_cast<long>(c.batch) * c.n_kv_heads, 64, kv_slab))
     return RTP_ERR_CUDA;
   PrefillArgs a;
-  a.items = plan->d_items;
-  a.n_items = plan->n_items;
+  a.items = plan->d_items + item_begin;
+  a.n_items = item_end - item_begin;
   a.sel = sel;
   a.cnt = sel_cnt;
   a.o = static_cast<__nv_bfloat16*>(o);
@@ -255,10 +263,13 @@ rtp_status prefill_run(const rtp_plan* plan, const void* q, int q_slab, const vo
   a.scale_log2 = plan->scale * kLog2e;
   a.status = status_word(plan->device);
   a.sel_heads = sel_heads;
-  const int ctas = static_cast<int>(std::min<long>(plan->n_items, plan->num_sms));
+  const int ctas = static_cast<int>(
+      std::min<long>(a.n_items, max_ctas > 0 ? std::min(max_ctas, plan->num_sms) : plan->num_sms));
   if (ctas <= 0) return RTP_OK;
   return cuda_status(launch_prefill(a, mq, mk, mv, ctas, reinterpret_cast<cudaStream_t>(stream)));
 }
+rtp_status route_heads(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int q_begin, int q_end, int key_begin,
+                       void* stream, rtp_plan** out);
 }  // namespace
 
 extern "C" {
@@ -288,6 +299,29 @@ rtp_status rtp_route_heads(const rtp_attn_cfg* cfg, const uint8_t* kind_host, vo
 rtp_status rtp_route_heads_range(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int q_begin, int q_end,
                                  void* stream, rtp_plan** out) {
   CallRange range_("rtp_route_heads_range");
+  return route_heads(cfg, kind_host, q_begin, q_end, 0, stream, out);
+}
+
+rtp_status rtp_route_heads_split(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int q_begin, int q_end,
+                                 int key_begin, void* stream, rtp_plan** out) {
+  CallRange range_("rtp_route_heads_split");
+  if (!cfg || key_begin < 0 || key_begin > q_begin) {
+    if (out) *out = nullptr;
+    return RTP_ERR_INVALID_ARG;
+  }
+  return route_heads(cfg, kind_host, q_begin, q_end, key_begin, stream, out);
+}
+
+long rtp_plan_num_local_items(const rtp_plan* plan) { return plan ? plan->n_local : -1; }
+
+}  // extern "C"
+
+namespace {
+// The planner behind rtp_route_heads(_range/_split): work items of the query
+// rows [q_begin, q_end), those whose visible keys all lie at or after
+// key_begin first, each part longest first.
+rtp_status route_heads(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int q_begin, int q_end, int key_begin,
+                       void* stream, rtp_plan** out) {
   if (!out) return RTP_ERR_INVALID_ARG;
   *out = nullptr;
   if (!cfg_prefill_ok(cfg) || !kind_host) return RTP_ERR_INVALID_ARG;
@@ -322,6 +356,7 @@ rtp_status rtp_route_heads_range(const rtp_attn_cfg* cfg, const uint8_t* kind_ho
   // Work items with their cost (KV tiles visited), then longest first.
   struct W {
     long cost;
+    bool local;
     int32_t v[4];
   };
   std::vector<W> work;
@@ -345,10 +380,21 @@ rtp_status rtp_route_heads_range(const rtp_attn_cfg* cfg, const uint8_t* kind_ho
           cost = (c0 + c1 + 1) / 2;
         }
         const int slot = kind == RTP_HEAD_SPARSE ? slot_of[h] : 0;
+        // The earliest key the tile can see: the window's first row for a
+        // streaming head; row 0 for a full head and for a sparse head (its
+        // selection always holds the sink block).
+        const long first_key = kind == RTP_HEAD_SWA ? std::max(0L, 128L * t - cfg->window + 1) : 0L;
+        const bool local = first_key >= key_begin;
         for (int pr = 0; pr < pairs; ++pr)
-          work.push_back(W{cost, {kind | (slot << 8), b * cfg->n_kv_heads + h, pr, t}});
+          work.push_back(W{cost, local, {kind | (slot << 8), b * cfg->n_kv_heads + h, pr, t}});
       }
-  std::stable_sort(work.begin(), work.end(), [](const W& a, const W& b) { return a.cost > b.cost; });
+  std::stable_sort(work.begin(), work.end(), [](const W& a, const W& b) {
+    if (a.local != b.local) return a.local;
+    return a.cost > b.cost;
+  });
+  p->key_begin = key_begin;
+  p->n_local = 0;
+  for (const W& w : work) p->n_local += w.local ? 1 : 0;
   p->n_items = static_cast<long>(work.size());
   p->items_host.resize(work.size() * 4);
   for (size_t i = 0; i < work.size(); ++i) std::memcpy(&p->items_host[i * 4], work[i].v, sizeof(work[i].v));
@@ -382,6 +428,9 @@ rtp_status rtp_route_heads_range(const rtp_attn_cfg* cfg, const uint8_t* kind_ho
   *out = p;
   return RTP_OK;
 }
+}  // namespace
+
+extern "C" {
 
 void rtp_plan_destroy(rtp_plan* plan) {
   if (!plan) return;
@@ -581,6 +630,15 @@ rtp_status rtp_hybrid_prefill(const rtp_plan* plan, const void* q, const void* k
   CallRange range_("rtp_hybrid_prefill");
   if (!plan) return RTP_ERR_INVALID_ARG;
   return prefill_run(plan, q, plan->q_end - plan->q_begin, k, v, plan->q_end, sel, sel_cnt, o, stream);
+}
+
+rtp_status rtp_hybrid_prefill_items(const rtp_plan* plan, const void* q, const void* k, const void* v,
+                                    const int32_t* sel, const int32_t* sel_cnt, void* o, long item_begin,
+                                    long item_end, int max_ctas, void* stream) {
+  CallRange range_("rtp_hybrid_prefill_items");
+  if (!plan || item_end < 0) return RTP_ERR_INVALID_ARG;
+  return prefill_run(plan, q, plan->q_end - plan->q_begin, k, v, plan->q_end, sel, sel_cnt, o, stream, 0,
+                     item_begin, item_end, max_ctas);
 }
 
 

@@ -57,6 +57,8 @@ def _load() -> ctypes.CDLL:
     sig = {
         "rtp_route_heads": (I, [cfgp, P, P, ctypes.POINTER(P)]),
         "rtp_route_heads_range": (I, [cfgp, P, I, I, P, ctypes.POINTER(P)]),
+        "rtp_route_heads_split": (I, [cfgp, P, I, I, I, P, ctypes.POINTER(P)]),
+        "rtp_plan_num_local_items": (L, [P]),
         "rtp_plan_destroy": (None, [P]),
         "rtp_plan_num_sparse": (I, [P]),
         "rtp_plan_num_items": (L, [P]),
@@ -70,6 +72,7 @@ def _load() -> ctypes.CDLL:
         "rtp_block_select_heads": (I, [P, P, P, P, P, P]),
         "rtp_hybrid_prefill_heads": (I, [P, P, P, P, P, P, P, P]),
         "rtp_hybrid_prefill": (I, [P, P, P, P, P, P, P, P]),
+        "rtp_hybrid_prefill_items": (I, [P, P, P, P, P, P, P, L, L, I, P]),
         "rtp_pipeline_create": (I, [cfgp, P, I, P, ctypes.POINTER(P)]),
         "rtp_pipeline_destroy": (None, [P]),
         "rtp_hybrid_prefill_host": (I, [P] * 15),
@@ -95,7 +98,8 @@ def _load() -> ctypes.CDLL:
 
 
 _lib = _load()
-EXPORTED = ("rtp_route_heads", "rtp_route_heads_range", "rtp_plan_destroy", "rtp_plan_num_sparse", "rtp_plan_num_items",
+EXPORTED = ("rtp_route_heads", "rtp_route_heads_range", "rtp_route_heads_split", "rtp_plan_num_local_items",
+            "rtp_hybrid_prefill_items", "rtp_plan_destroy", "rtp_plan_num_sparse", "rtp_plan_num_items",
             "rtp_plan_sparse_heads", "rtp_plan_work_items", "rtp_indexer_project", "rtp_block_select",
             "rtp_block_select_dynamic", "rtp_block_select_rowmax", "rtp_indexer_project_heads",
             "rtp_block_select_heads", "rtp_hybrid_prefill_heads", "rtp_pipeline_create", "rtp_pipeline_destroy", "rtp_hybrid_prefill_host",
@@ -182,6 +186,20 @@ def rtp_route_heads_range(cfg: AttnConfig, kinds, q_begin: int, q_end: int, stre
     return out.value
 
 
+def rtp_route_heads_split(cfg: AttnConfig, kinds, q_begin: int, q_end: int, key_begin: int, stream=None) -> int:
+    """A ranged plan whose work list puts the tiles that see only keys >= key_begin first."""
+    out = ctypes.c_void_p()
+    c = cfg.c()
+    _check("rtp_route_heads_split", _lib.rtp_route_heads_split(ctypes.byref(c), _kinds(kinds), int(q_begin),
+                                                                 int(q_end), int(key_begin), _stream(stream),
+                                                                 ctypes.byref(out)))
+    return out.value
+
+
+def rtp_plan_num_local_items(plan: int) -> int:
+    return _lib.rtp_plan_num_local_items(plan)
+
+
 def rtp_plan_destroy(plan: int) -> None:
     _lib.rtp_plan_destroy(plan)
 
@@ -259,6 +277,13 @@ def default_selection_beta(cfg: AttnConfig) -> float:
 def rtp_hybrid_prefill(plan: int, q, k, v, sel, sel_cnt, o, stream=None) -> None:
     _check("rtp_hybrid_prefill", _lib.rtp_hybrid_prefill(plan, _ptr(q), _ptr(k), _ptr(v), _ptr(sel), _ptr(sel_cnt),
                                                          _ptr(o), _stream(stream)))
+
+
+def rtp_hybrid_prefill_items(plan: int, q, k, v, sel, sel_cnt, o, item_begin: int, item_end: int,
+                             max_ctas: int = 0, stream=None) -> None:
+    _check("rtp_hybrid_prefill_items",
+           _lib.rtp_hybrid_prefill_items(plan, _ptr(q), _ptr(k), _ptr(v), _ptr(sel), _ptr(sel_cnt), _ptr(o),
+                                         int(item_begin), int(item_end), int(max_ctas), _stream(stream)))
 
 
 def rtp_pipeline_create(cfg: AttnConfig, kinds, n_chunks: int, stream=None) -> int:
@@ -431,14 +456,22 @@ def rtp_version() -> int:
 class Plan:
     """Owns a routing plan (rtp_route_heads / rtp_plan_destroy)."""
 
-    def __init__(self, cfg: AttnConfig, kinds, stream=None, q_range: tuple | None = None):
+    def __init__(self, cfg: AttnConfig, kinds, stream=None, q_range: tuple | None = None,
+                 key_begin: int | None = None):
+        """q_range: a ranged plan (rtp_route_heads_range); with key_begin as
+        well, a split plan (rtp_route_heads_split) whose first n_local items
+        see only keys >= key_begin."""
         self.cfg = cfg
         self.kinds = list(kinds)
         self.q_range = (0, cfg.seq) if q_range is None else (int(q_range[0]), int(q_range[1]))
-        if q_range is None:
+        if key_begin is not None:
+            self.handle = rtp_route_heads_split(cfg, kinds, self.q_range[0], self.q_range[1], key_begin, stream)
+        elif q_range is None:
             self.handle = rtp_route_heads(cfg, kinds, stream)
         else:
             self.handle = rtp_route_heads_range(cfg, kinds, self.q_range[0], self.q_range[1], stream)
+        self.n_items = rtp_plan_num_items(self.handle)
+        self.n_local = rtp_plan_num_local_items(self.handle)
         self.n_sparse = rtp_plan_num_sparse(self.handle)
         self.slot_heads = rtp_plan_sparse_heads(self.handle)
 

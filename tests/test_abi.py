@@ -100,6 +100,18 @@ def test_null_plan_is_rejected(rtp):
     for fn, nargs in [(rtp._lib.rtp_indexer_project, 7), (rtp._lib.rtp_block_select, 6),
                       (rtp._lib.rtp_hybrid_prefill, 8)]:
         assert fn(*([None] * nargs)) == rtp.RTP_ERR_INVALID_ARG
+    assert rtp._lib.rtp_hybrid_prefill_items(None, None, None, None, None, None, None, 0, 0, 0,
+                                             None) == rtp.RTP_ERR_INVALID_ARG
+    assert rtp._lib.rtp_plan_num_local_items(None) == -1
+
+
+def test_split_plan_rejects_key_begin_outside_the_range_start(rtp):
+    """key_begin must lie in [0, q_begin]; refused before any device call."""
+    cfg = rtp.AttnConfig(1, 1024, 8, 2, 256, 64, 4, 2)
+    for q_begin, key_begin in [(256, 257), (256, -1), (0, 1)]:
+        with pytest.raises(rtp.RtpError) as e:
+            rtp.rtp_route_heads_split(cfg, [2, 0], q_begin, 512, key_begin)
+        assert e.value.status == rtp.RTP_ERR_INVALID_ARG
 
 
 def test_cache_calls_validate_before_launch(rtp):

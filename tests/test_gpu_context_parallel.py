@@ -53,9 +53,13 @@ def reference(rtp, q, k, v, proj, cfg, kinds, dynamic):
     return o, bufs
 
 
-def emulate(rtp, cp, q, k, v, proj, cfg, kinds, world, dynamic):
+def emulate(rtp, cp, q, k, v, proj, cfg, kinds, world, dynamic, split=False):
+    """split: each rank's plan is split at its first row (rtp_route_heads_split)
+    and run as the overlapped driver runs it: its local items (the first on a
+    capped grid) while every row outside its own is still garbage, then the
+    fetched rows arrive and the remaining items run."""
     ranges = cp.cp_ranges(cfg.seq, world)
-    plans = [rtp.Plan(cfg, kinds, q_range=r) for r in ranges]
+    plans = [rtp.Plan(cfg, kinds, q_range=r, key_begin=r[0] if split else None) for r in ranges]
     bufs = plans[0].buffers(q.device)  # whole-sequence layout, shared: each rank writes only its own part
     for b in bufs.values():
         b.fill_(-9)
@@ -80,20 +84,48 @@ def emulate(rtp, cp, q, k, v, proj, cfg, kinds, world, dynamic):
         vf = kf.clone()
         kf[:, :, qb:qe] = k[:, :, qb:qe]
         vf[:, :, qb:qe] = v[:, :, qb:qe]
+        fetched.append(sum(hi - lo for iv in needs.values() for lo, hi in iv))
+        o_loc = torch.empty_like(q[:, :, qb:qe])
+        q_loc = q[:, :, qb:qe].contiguous()
+        sel_d = bufs["sel"] if p.n_sparse else None
+        cnt_d = bufs["sel_cnt"] if p.n_sparse else None
+        if split:
+            check_split(rtp, p, cfg, kinds, qb)
+            head = p.n_local // 3
+            rtp.rtp_hybrid_prefill_items(p.handle, q_loc, kf, vf, sel_d, cnt_d, o_loc, 0, head, 5)
+            rtp.rtp_hybrid_prefill_items(p.handle, q_loc, kf, vf, sel_d, cnt_d, o_loc, head, p.n_local, 0)
         for (b, h), iv in needs.items():
             for lo, hi in iv:
                 kf[b, h, lo:hi] = k[b, h, lo:hi]
                 vf[b, h, lo:hi] = v[b, h, lo:hi]
-        fetched.append(sum(hi - lo for iv in needs.values() for lo, hi in iv))
-        o_loc = torch.empty_like(q[:, :, qb:qe])
-        rtp.rtp_hybrid_prefill(p.handle, q[:, :, qb:qe].contiguous(), kf, vf,
-                               bufs["sel"] if p.n_sparse else None, bufs["sel_cnt"] if p.n_sparse else None, o_loc)
+        if split:
+            rtp.rtp_hybrid_prefill_items(p.handle, q_loc, kf, vf, sel_d, cnt_d, o_loc, p.n_local, p.n_items, 0)
+        else:
+            rtp.rtp_hybrid_prefill(p.handle, q_loc, kf, vf, sel_d, cnt_d, o_loc)
         o[:, :, qb:qe] = o_loc
     torch.cuda.synchronize()
     assert rtp.rtp_last_device_status() == rtp.RTP_OK
     for p in plans:
         p.close()
     return o, bufs, fetched
+
+
+def check_split(rtp, p, cfg, kinds, key_begin):
+    """The split plan holds the ranged plan's items; the first n_local are
+    exactly those whose earliest visible key is at or after key_begin."""
+    items = rtp.rtp_plan_work_items(p.handle)
+    ranged = rtp.Plan(cfg, kinds, q_range=p.q_range)
+    ref = rtp.rtp_plan_work_items(ranged.handle)
+    ranged.close()
+    assert sorted(map(tuple, items.tolist())) == sorted(map(tuple, ref.tolist()))
+
+    def local(it):
+        kind, t = int(it[0]) & 0xFF, int(it[3])
+        first = max(0, 128 * t - cfg.window + 1) if kind == 0 else 0
+        return first >= key_begin
+
+    flags = [local(it) for it in items]
+    assert flags == [True] * p.n_local + [False] * (p.n_items - p.n_local)
 
 
 CASES = [
@@ -107,8 +139,9 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("split", [False, True], ids=["whole", "split"])
 @pytest.mark.parametrize("case", CASES)
-def test_emulated_ranks_equal_single_gpu_bit_for_bit(rtp, cp, cuda_device, case):
+def test_emulated_ranks_equal_single_gpu_bit_for_bit(rtp, cp, cuda_device, case, split):
     seq, hq, hkv, kinds, window, block, topk, n_local, world, dynamic = case
     d = inputs.small_prefill(seq, hq, hkv, kinds, seed=seq + world, device=cuda_device)
     d["k"] = torch.cat([d["k"], torch.roll(d["k"], 5, dims=2)])  # two sequences
@@ -118,7 +151,7 @@ def test_emulated_ranks_equal_single_gpu_bit_for_bit(rtp, cp, cuda_device, case)
     proj = inputs.random_projector(7, cuda_device)
     cfg = rtp.AttnConfig(2, seq, hq, hkv, window, block, topk, n_local)
     o_ref, b_ref = reference(rtp, q, k, v, proj, cfg, kinds, dynamic)
-    o, bufs, fetched = emulate(rtp, cp, q, k, v, proj, cfg, kinds, world, dynamic)
+    o, bufs, fetched = emulate(rtp, cp, q, k, v, proj, cfg, kinds, world, dynamic, split)
     if 2 in kinds:
         assert torch.equal(bufs["centroids"], b_ref["centroids"]) and torch.equal(bufs["qbar"], b_ref["qbar"])
         assert torch.equal(bufs["sel"], b_ref["sel"]) and torch.equal(bufs["sel_cnt"], b_ref["sel_cnt"])
@@ -126,7 +159,7 @@ def test_emulated_ranks_equal_single_gpu_bit_for_bit(rtp, cp, cuda_device, case)
     assert fetched[0] == 0 and all(f > 0 for f in fetched[1:])
 
 
-def _worker(rank, world, port, seq, q_out):
+def _worker(rank, world, port, seq, q_out, overlap):
     import sys
 
     sys.path.insert(0, ROOT)
@@ -146,7 +179,7 @@ def _worker(rank, world, port, seq, q_out):
         qb, qe = cp.cp_ranges(seq, world)[rank]
         o_loc, info = cp.cp_prefill_layer(d["q"][:, :, qb:qe].contiguous(), d["k"][:, :, qb:qe].contiguous(),
                                           d["v"][:, :, qb:qe].contiguous(), [2, 0, 1, 0],
-                                          inp.random_projector(7, "cuda"), cfg)
+                                          inp.random_projector(7, "cuda"), cfg, overlap=overlap)
         torch.cuda.synchronize()
         q_out.put((rank, o_loc.cpu().view(torch.int16).numpy(), info["bytes_received"],
                    rtp.rtp_last_device_status()))
@@ -155,7 +188,8 @@ def _worker(rank, world, port, seq, q_out):
         dist.destroy_process_group()
 
 
-def test_two_processes_with_gloo_staging(rtp, cp, cuda_device):
+@pytest.mark.parametrize("overlap", [True, False], ids=["overlap", "serial"])
+def test_two_processes_with_gloo_staging(rtp, cp, cuda_device, overlap):
     seq, world = 2048, 2
     d = inputs.small_prefill(seq, 8, 4, [2, 0, 1, 0], seed=77, device=cuda_device)
     cfg = rtp.AttnConfig(1, seq, 8, 4, 300, 64, 4, 2)
@@ -168,7 +202,7 @@ def test_two_processes_with_gloo_staging(rtp, cp, cuda_device):
 
     ctx = mp.get_context("spawn")
     q_out = ctx.Queue()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, seq, q_out)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, seq, q_out, overlap)) for r in range(world)]
     for p in procs:
         p.start()
     res = {}
