@@ -394,14 +394,16 @@ def time_dynamic(rtp, w, res, device, points=((0.9, None), (0.99, None), (0.9, 1
 
 def time_selection_variants(rtp, w, device, reps=2):
     """The selection variants alone on the layer (profiling entry): the
-    indexer, then `reps` times each of the row-max selection and the per-head
-    summaries + selection; mean ms per call."""
+    indexer, then `reps` times each of the row-max selection, the per-head
+    summaries + selection, the fixed top-k selection and the dynamic
+    (mass 0.9, default beta, cap = top-k) selection; mean ms per call."""
     d, plan, _ = make_layer(rtp, w, 0, device)
     bufs = plan.buffers(device, per_head=True)
     q, proj = d["q"], d["proj"]
     stream = torch.cuda.current_stream()
+    beta = rtp.default_selection_beta(plan.cfg)
     rtp.rtp_indexer_project(plan.handle, q, d["k"], proj, bufs["centroids"], bufs["qbar"], stream)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(reps)]
     for e in ev:
         e[0].record(stream)
         rtp.rtp_block_select_rowmax(plan.handle, q, proj, bufs["centroids"], bufs["sel"], bufs["sel_cnt"], stream)
@@ -410,9 +412,16 @@ def time_selection_variants(rtp, w, device, reps=2):
         rtp.rtp_block_select_heads(plan.handle, bufs["qbar_heads"], bufs["centroids"], bufs["sel_heads"],
                                    bufs["cnt_heads"], stream)
         e[2].record(stream)
+        rtp.rtp_block_select(plan.handle, bufs["qbar"], bufs["centroids"], bufs["sel"], bufs["sel_cnt"], stream)
+        e[3].record(stream)
+        rtp.rtp_block_select_dynamic(plan.handle, bufs["qbar"], bufs["centroids"], 0.9, 0, beta, bufs["sel"],
+                                     bufs["sel_cnt"], stream)
+        e[4].record(stream)
     torch.cuda.synchronize()
     out = {"workload": w.name, "rowmax_select_ms": statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
            "per_head_summaries_and_select_ms": statistics.mean(e[1].elapsed_time(e[2]) for e in ev),
+           "fixed_select_ms": statistics.mean(e[2].elapsed_time(e[3]) for e in ev),
+           "dynamic_select_ms": statistics.mean(e[3].elapsed_time(e[4]) for e in ev),
            "status": rtp.status_str(rtp.rtp_last_device_status(stream))}
     plan.close()
     return out
@@ -422,13 +431,13 @@ def time_cp_projection(rtp, w, res, device, world=8, link_gbs=770.0, reserve_sms
     """Context-parallel prefill of the main layer split over `world` ranks,
     projected from one GPU.  Each rank's work is timed here on its own rows
     (its K/V buffer holds every row it may read), as one ranged launch and as
-    the overlapped driver runs it (context_parallel.cp_prefill_layer): the
-    split plan's local tiles (the first on reserve_sms fewer CTAs, sized to
-    the exchange), then the tiles that need fetched rows.  The K/V bytes a
-    rank would receive are counted from its heads' row needs and selection;
+    the overlapped driver runs it (context_parallel.cp_prefill_layer): a head
+    of the split plan's local tiles on reserve_sms fewer CTAs, sized to the
+    exchange, then every other tile in one launch.  The K/V bytes a rank
+    would receive are counted from its heads' row needs and selection;
     transfer time = bytes / the measured peer-copy bandwidth.  With overlap a
-    rank takes local + remote + the part of the transfer its local tiles do
-    not hide.  Not a multi-GPU measurement."""
+    rank takes head + rest + the part of the transfer the head does not
+    hide.  Not a multi-GPU measurement."""
     from swa_hybrid_attention_b200 import context_parallel as cp
 
     plan, bufs = res["plan"], res["bufs"]
@@ -459,31 +468,27 @@ def time_cp_projection(rtp, w, res, device, world=8, link_gbs=770.0, reserve_sms
     for pass_ in range(2):
         evs = []
         for pr, qb, qe, kv_bytes, head, (q_loc, k_loc, v_loc), o_loc in setup:
-            e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
             e[0].record(stream)
             rtp.rtp_hybrid_prefill(pr.handle, q_loc, k_loc, v_loc, sel_d, cnt_d, o_loc, stream)
             e[1].record(stream)
             rtp.rtp_hybrid_prefill_items(pr.handle, q_loc, k_loc, v_loc, sel_d, cnt_d, o_loc, 0, head,
                                          sms - reserve_sms, stream)
             e[2].record(stream)
-            rtp.rtp_hybrid_prefill_items(pr.handle, q_loc, k_loc, v_loc, sel_d, cnt_d, o_loc, head, pr.n_local, 0,
+            rtp.rtp_hybrid_prefill_items(pr.handle, q_loc, k_loc, v_loc, sel_d, cnt_d, o_loc, head, pr.n_items, 0,
                                          stream)
             e[3].record(stream)
-            rtp.rtp_hybrid_prefill_items(pr.handle, q_loc, k_loc, v_loc, sel_d, cnt_d, o_loc, pr.n_local,
-                                         pr.n_items, 0, stream)
-            e[4].record(stream)
             evs.append(e)
         torch.cuda.synchronize()
         if pass_ == 1:
             for (pr, qb, qe, kv_bytes, head, _, _), e in zip(setup, evs):
                 transfer = kv_bytes / (link_gbs * 1e9) * 1e3
-                head_ms, tail_ms, remote_ms = e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]), e[3].elapsed_time(e[4])
-                local_ms = head_ms + tail_ms
+                head_ms, rest_ms = e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])
+                exposed = max(0.0, transfer - head_ms)
                 ranks.append({"q_rows": qe - qb, "prefill_ms": e[0].elapsed_time(e[1]), "kv_bytes_in": kv_bytes,
                               "transfer_ms": transfer, "items": pr.n_items, "local_items": pr.n_local,
-                              "head_items": head, "head_ms": head_ms, "local_ms": local_ms, "remote_ms": remote_ms,
-                              "exposed_transfer_ms": max(0.0, transfer - local_ms),
-                              "overlapped_ms": local_ms + remote_ms + max(0.0, transfer - local_ms)})
+                              "head_items": head, "head_ms": head_ms, "rest_ms": rest_ms,
+                              "exposed_transfer_ms": exposed, "overlapped_ms": head_ms + exposed + rest_ms})
     for pr, *_ in setup:
         pr.close()
     del setup
@@ -495,9 +500,9 @@ def time_cp_projection(rtp, w, res, device, world=8, link_gbs=770.0, reserve_sms
             "projected_ms_overlap": max(r["overlapped_ms"] for r in ranks),
             "exposed_transfer_ms_max": max(r["exposed_transfer_ms"] for r in ranks),
             "note": "projection from one GPU: per-rank prefill timed on its own rows (all ranks back to back, "
-                    "second pass), as one launch and as the overlapped split (local tiles: capped head launch + "
-                    "tail; then remote tiles); K/V transfer = bytes / measured 770 GB/s peer copy; the indexer, "
-                    "selection and centroid all-gather (<1 ms) are not included"}
+                    "second pass), as one launch and as the overlapped split (a capped launch of local tiles "
+                    "during the exchange, then every other tile); K/V transfer = bytes / measured 770 GB/s peer "
+                    "copy; the indexer, selection and centroid all-gather (<1 ms) are not included"}
 
 
 def time_e2e(rtp, w, res, steps, device, chunks=16):

@@ -23,12 +23,13 @@ single-GPU prefill would compute for its rows, bit for bit.
 
 Overlap: the plan's work list starts with the tiles whose visible keys are
 all this rank's own rows (streaming heads whose window starts inside the
-range).  Those run on the compute stream while the exchange runs on a side
-stream; the first of them on all but a few SMs, so that the collectives'
-kernels have SMs to run on (a prefill CTA holds an SM's registers), the rest
-on every SM.  The tiles that need fetched rows (full and sparse heads always
-see row 0; streaming tiles near the range's start) run once the exchange is
-done.
+range).  The first of them run on the compute stream, on all but a few SMs
+so that the collectives' kernels have SMs to run on (a prefill CTA holds an
+SM's registers), while the exchange runs on a side stream; as many as take
+about as long as the exchange.  Every other tile — the remaining local ones
+and those that need fetched rows (full and sparse heads always see row 0;
+streaming tiles near the range's start) — runs in one launch once the
+exchange is done.
 
 This module is host-side orchestration: which rows to fetch, and the
 collectives (torch.distributed, NCCL on GPUs; gloo with host staging where
@@ -239,10 +240,10 @@ def _item_tiles(item, cfg: rtp.AttnConfig) -> int:
 def overlap_head_items(items, n_local: int, cfg: rtp.AttnConfig, exchange_s: float, ctas: int,
                        tile_s: float = 2.4e-6) -> int:
     """How many of the first local items the capped launch should run so that
-    it lasts about as long as the exchange: ctas CTAs, each taking a KV tile
-    of one query-head pair in about tile_s seconds (the prefill kernel's
-    measured rate on B200: ~2.4 us per pair-tile per SM)."""
-    budget = exchange_s / tile_s * ctas
+    it lasts a little longer than the exchange (a quarter more): ctas CTAs,
+    each taking a KV tile of one query-head pair in about tile_s seconds (the
+    prefill kernel's measured rate on B200: ~2.4 us per pair-tile per SM)."""
+    budget = 1.25 * exchange_s / tile_s * ctas
     acc = 0
     for i in range(n_local):
         if acc >= budget:
@@ -259,9 +260,9 @@ def cp_prefill_layer(q_loc, k_loc, v_loc, kinds, proj, cfg: rtp.AttnConfig, grou
     v_loc hold this rank's rows of cp_ranges(cfg.seq, world)[rank].  Returns
     (o_loc, info) with o_loc the attention output of this rank's rows and
     info the bytes received, the rows fetched and the work split.
-    overlap: run the tiles that need no fetched row while the exchange is in
-    flight (side stream); the first of them on reserve_sms fewer CTAs, sized
-    to the exchange's duration at link_gbs.  stream: a torch.cuda.Stream
+    overlap: while the exchange is in flight (side stream), run tiles that
+    need no fetched row, on reserve_sms fewer CTAs, as many as the exchange's
+    duration at link_gbs allows; the rest after it.  stream: a torch.cuda.Stream
     (None: the current stream); everything this rank queues goes on it, the
     exchange on a side stream joined before the remote tiles.
     """
@@ -311,11 +312,11 @@ def cp_prefill_layer(q_loc, k_loc, v_loc, kinds, proj, cfg: rtp.AttnConfig, grou
                 side.wait_stream(comp)
                 # queued before the exchange, whose host side blocks on its own stream only
                 rtp.rtp_hybrid_prefill_items(plan.handle, q_loc, kf, vf, sel_d, cnt_d, o_loc, 0, n_head, ctas, comp)
-                rtp.rtp_hybrid_prefill_items(plan.handle, q_loc, kf, vf, sel_d, cnt_d, o_loc, n_head, n_loc, 0, comp)
                 with torch.cuda.stream(side):
                     received = exchange_kv(k_loc, v_loc, needs, ranges, rank, kf, vf, group, copy_own=False)
                 comp.wait_stream(side)
-                rtp.rtp_hybrid_prefill_items(plan.handle, q_loc, kf, vf, sel_d, cnt_d, o_loc, n_loc, n_all, 0, comp)
+                # the rest, local and remote tiles in one launch (one tail instead of two)
+                rtp.rtp_hybrid_prefill_items(plan.handle, q_loc, kf, vf, sel_d, cnt_d, o_loc, n_head, n_all, 0, comp)
             else:
                 received = exchange_kv(k_loc, v_loc, needs, ranges, rank, kf, vf, group, copy_own=False)
                 rtp.rtp_hybrid_prefill(plan.handle, q_loc, kf, vf, sel_d, cnt_d, o_loc, comp)
