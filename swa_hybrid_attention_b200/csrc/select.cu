@@ -259,16 +259,31 @@ __global__ void __launch_bounds__(kSelThreads) block_select_dynamic_kernel(const
 // rule and output are those of the fixed policy (top-k by score desc, index
 // asc; sink and local blocks added).
 //
-// Per CTA (one query block): 1. u_i of the block's rows into shared memory
-// (16 threads per row sum the group's heads over 8 dims each and project;
-// the 16 partial dot products of a rank are added in a fixed butterfly, lane
-// 0's result kept); 2. two candidates per thread (80 registers: three CTAs
-// an SM): their centroids in registers, each row's u_i read once as a
-// shared-memory broadcast, max over
-// rows of the 16-term dot product (two fixed-order chains of 8, then their
-// sum); 3. the fixed kernel's radix select and ordered compaction.
-
-constexpr int kRowmaxCands = 2;
+// Per CTA (one query block):
+//  1. u_i of the block's rows into shared memory (16 threads per row sum the
+//     group's heads over 8 dims each and project; the 16 partial dot
+//     products of a rank are added in a fixed butterfly, lane 0's result
+//     kept).
+//  2. Approximate scores on the tensor cores: the (rows x 16) . (16 x 8
+//     candidates) products are mma.sync m16n8k16 with both operands split
+//     into bf16 hi + lo parts (hi.hi + hi.lo + lo.hi, fp32 accumulation), the
+//     maximum over rows taken from the accumulator fragments.  Each split
+//     keeps 16 bits of mantissa, so an approximate dot product is within
+//     2^-14 |u_i| |c_j| of the exact one and the approximate row maximum a_j
+//     within E = 2^-12 max_i |u_i| max_j |c_j| (a 4x margin) of the exact
+//     fp32 score s_j of step 4.
+//  3. A lower bound b of the k-th largest approximate score a_(k) (two radix
+//     passes: the low edge of its 16-bit key bin).  At least k candidates
+//     have s >= a_(k) - E >= b - E, so a candidate with a_j < b - 2E has
+//     s_j < b - E and is not among the k best: only the others (the k best
+//     and those within 2E of the bin, 2^-7 relative wide) need their exact
+//     score.
+//  4. Those candidates are re-scored exactly (fp32, the 16-term dot product
+//     in two fixed-order chains of 8 then their sum, maximum over rows: the
+//     score every earlier version of this kernel computed for every
+//     candidate); the others get key 0, below every finite score's key.
+//  5. The fixed kernel's radix select and ordered compaction on those keys:
+//     the same selection as exact scores for every candidate.
 
 // u . c with ranks 0-7 and 8-15 in two fma chains (fixed order), added at
 // the end: half the dependent latency of one 16-long chain.
@@ -292,25 +307,57 @@ __device__ __forceinline__ float score16_two_chains(const float (&u)[kRank], con
 }
 
 struct RowmaxScratch {
-  float proj[kHeadDim * kRank];
+  // projector row 8 cg + e at projv[e][cg][0..16), rows padded to 20 words:
+  // the 16-byte loads of the 8 lanes of a phase (cg = 0..7 and 8..15) hit
+  // distinct banks (a dense [128][16] layout puts all 16 lanes of a row in
+  // one bank: a 16-way conflict on every load)
+  float projv[8][16][20];
   float u[128][kRank];  // block <= 128 rows
+  float red[2][kSelThreads / 32];
+  int n_poss;
 };
 
-__global__ void __launch_bounds__(kSelThreads, 3) block_select_rowmax_kernel(const SelectArgs a) {
-  extern __shared__ uint32_t keys[];
+// hi = bf16(x, y) (x in the low half), lo = bf16 of the remainders.
+__device__ __forceinline__ uint32_t bf16x2_bits(float x, float y) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(x, y);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+__device__ __forceinline__ void split_bf16x2(float x, float y, uint32_t& hi, uint32_t& lo) {
+  hi = bf16x2_bits(x, y);
+  lo = bf16x2_bits(x - __uint_as_float(hi << 16), y - __uint_as_float(hi & 0xFFFF0000u));
+}
+
+__device__ __forceinline__ void mma_m16n8k16_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Inverse of order_key.
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+__global__ void __launch_bounds__(kSelThreads, 2) block_select_rowmax_kernel(const SelectArgs a) {
+  extern __shared__ uint32_t keys[];  // [nb] order keys, then [nb] candidates to re-score
   __shared__ SelectScratch sh;
   __shared__ __align__(16) RowmaxScratch rs;
   const int t = a.t0 + static_cast<int>(blockIdx.x), slot = blockIdx.y, b = blockIdx.z;
   const size_t row = (static_cast<size_t>(b) * a.n_sparse + slot) * a.nb + t;
   int32_t* out = a.sel + row * a.kmax;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (const int n = select_without_scores(t, a.topk, a.n_local, a.kmax, out); n >= 0) {
     if (tid == 0) a.cnt[row] = n;
     return;
   }
   const int ncand = t - a.n_local;
   const int kvh = a.slot_heads[slot];
-  for (int e = tid; e < kHeadDim * kRank; e += kSelThreads) rs.proj[e] = a.proj[e];
+  for (int e = tid; e < kHeadDim * kRank; e += kSelThreads) {
+    const int d = e / kRank, c = e % kRank;
+    rs.projv[d & 7][d >> 3][c] = a.proj[e];
+  }
   __syncthreads();
   // 1. u_i
   {
@@ -319,61 +366,186 @@ __global__ void __launch_bounds__(kSelThreads, 3) block_select_rowmax_kernel(con
       const int i = i0 + rg;
       const size_t qrow = static_cast<size_t>(t) * a.block + i - a.q_row0;
       float sum[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-      for (int h = 0; h < a.group; ++h) {
-        const __nv_bfloat16* qp =
-            a.q + ((static_cast<size_t>(b) * a.n_q_heads + kvh * a.group + h) * a.q_slab + qrow) * kHeadDim + 8 * cg;
-        const uint4 raw = *reinterpret_cast<const uint4*>(qp);
-        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      // the heads' loads are issued 8 at a time (all in flight), then added
+      // in head order
+      const __nv_bfloat16* q0 =
+          a.q + ((static_cast<size_t>(b) * a.n_q_heads + kvh * a.group) * a.q_slab + qrow) * kHeadDim + 8 * cg;
+      const size_t head_stride = static_cast<size_t>(a.q_slab) * kHeadDim;
+      for (int h0 = 0; h0 < a.group; h0 += 8) {
+        uint4 raw[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(p2[e]);
-          sum[2 * e] += f.x;
-          sum[2 * e + 1] += f.y;
+        for (int hh = 0; hh < 8; ++hh)
+          if (h0 + hh < a.group) raw[hh] = *reinterpret_cast<const uint4*>(q0 + (h0 + hh) * head_stride);
+#pragma unroll
+        for (int hh = 0; hh < 8; ++hh) {
+          if (h0 + hh < a.group) {
+            const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw[hh]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(p2[e]);
+              sum[2 * e] += f.x;
+              sum[2 * e + 1] += f.y;
+            }
+          }
+        }
+      }
+      // rank c: sum over e of proj[8 cg + e][c] * sum[e] (fma chain in e order)
+      float v[kRank];
+#pragma unroll
+      for (int c = 0; c < kRank; ++c) v[c] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float4* pr = reinterpret_cast<const float4*>(rs.projv[e][cg]);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const float4 p4 = pr[w];
+          v[4 * w] = fmaf(p4.x, sum[e], v[4 * w]);
+          v[4 * w + 1] = fmaf(p4.y, sum[e], v[4 * w + 1]);
+          v[4 * w + 2] = fmaf(p4.z, sum[e], v[4 * w + 2]);
+          v[4 * w + 3] = fmaf(p4.w, sum[e], v[4 * w + 3]);
         }
       }
 #pragma unroll
       for (int c = 0; c < kRank; ++c) {
-        float v = 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v = fmaf(rs.proj[(8 * cg + e) * kRank + c], sum[e], v);
-        v += __shfl_xor_sync(0xffffffffu, v, 8);
-        v += __shfl_xor_sync(0xffffffffu, v, 4);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        if (cg == 0) rs.u[i][c] = v;
+        v[c] += __shfl_xor_sync(0xffffffffu, v[c], 8);
+        v[c] += __shfl_xor_sync(0xffffffffu, v[c], 4);
+        v[c] += __shfl_xor_sync(0xffffffffu, v[c], 2);
+        v[c] += __shfl_xor_sync(0xffffffffu, v[c], 1);
+        if (cg == 0) rs.u[i][c] = v[c];
       }
     }
   }
   __syncthreads();
-  // 2. scores -> order keys: kRowmaxCands candidates per thread share each
-  // row's shared-memory read
   const float* C = a.centroids + (static_cast<size_t>(b) * a.n_sparse + slot) * a.nb * kRank;
-  for (int x0 = tid; x0 < ncand; x0 += kRowmaxCands * kSelThreads) {
-    float4 cv[kRowmaxCands][4];
-    float best[kRowmaxCands];
+  const int mtiles = a.block / 16;  // 16-row tiles of u (4 or 8)
+  // 2. approximate scores, 8 candidates per warp step.  Fragments of
+  // m16n8k16 (g = lane / 4, q = lane % 4): A rows g and g+8 of the tile,
+  // dims 2q, 2q+1 and 2q+8, 2q+9; B column g (candidate 8 gi + g), the same
+  // dims; D rows g and g+8, candidates 2q and 2q+1.
+  float cn2_max = 0.f;
+  {
+    const int g = lane >> 2, q = lane & 3;
+    uint32_t ahi[8][4], alo[8][4];
 #pragma unroll
-    for (int u = 0; u < kRowmaxCands; ++u) {
-      const int x = min(x0 + u * kSelThreads, ncand - 1);
-      const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + 1) * kRank);
+    for (int mt = 0; mt < 8; ++mt) {
+      if (mt < mtiles) {
 #pragma unroll
-      for (int w = 0; w < 4; ++w) cv[u][w] = __ldg(c4 + w);
-      best[u] = -INFINITY;
+        for (int e = 0; e < 4; ++e) {
+          const int r = 16 * mt + g + 8 * (e & 1), k = 2 * q + 8 * (e >> 1);
+          split_bf16x2(rs.u[r][k], rs.u[r][k + 1], ahi[mt][e], alo[mt][e]);
+        }
+      }
     }
-    for (int i = 0; i < a.block; ++i) {
-      const float4* u4 = reinterpret_cast<const float4*>(rs.u[i]);
-      const float4 u0 = u4[0], u1 = u4[1], u2 = u4[2], u3 = u4[3];
-      const float uq[kRank] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w,
-                               u2.x, u2.y, u2.z, u2.w, u3.x, u3.y, u3.z, u3.w};
+    const int ngroups = (ncand + 7) / 8;
+    for (int gi = warp; gi < ngroups; gi += kSelThreads / 32) {
+      const int xg = 8 * gi + g;
+      const float* cp = C + static_cast<size_t>(min(xg, ncand - 1) + 1) * kRank;
+      const float2 c0 = __ldg(reinterpret_cast<const float2*>(cp + 2 * q));
+      const float2 c1 = __ldg(reinterpret_cast<const float2*>(cp + 2 * q + 8));
+      uint32_t bhi0, blo0, bhi1, blo1;
+      split_bf16x2(c0.x, c0.y, bhi0, blo0);
+      split_bf16x2(c1.x, c1.y, bhi1, blo1);
+      float n2 = c0.x * c0.x + c0.y * c0.y + c1.x * c1.x + c1.y * c1.y;
+      n2 += __shfl_xor_sync(0xffffffffu, n2, 1);
+      n2 += __shfl_xor_sync(0xffffffffu, n2, 2);
+      if (xg < ncand) cn2_max = fmaxf(cn2_max, n2);
+      float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-      for (int u = 0; u < kRowmaxCands; ++u) best[u] = fmaxf(best[u], score16_two_chains(uq, cv[u]));
+      for (int mt = 0; mt < 8; ++mt) {
+        if (mt < mtiles) {
+          float d[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_m16n8k16_bf16(d, alo[mt], bhi0, bhi1);
+          mma_m16n8k16_bf16(d, ahi[mt], blo0, blo1);
+          mma_m16n8k16_bf16(d, ahi[mt], bhi0, bhi1);
+          m0 = fmaxf(m0, fmaxf(d[0], d[2]));
+          m1 = fmaxf(m1, fmaxf(d[1], d[3]));
+        }
+      }
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, off));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, off));
+      }
+      if (g == 0) {
+        const int x0 = 8 * gi + 2 * q;
+        if (x0 < ncand) keys[x0] = order_key(m0);
+        if (x0 + 1 < ncand) keys[x0 + 1] = order_key(m1);
+      }
+    }
+  }
+  // the bound E from the largest |u_i| and |c_j|
+  {
+    float un2 = 0.f;
+    if (tid < a.block) {
+#pragma unroll
+      for (int c = 0; c < kRank; ++c) un2 = fmaf(rs.u[tid][c], rs.u[tid][c], un2);
     }
 #pragma unroll
-    for (int u = 0; u < kRowmaxCands; ++u) {
-      const int x = x0 + u * kSelThreads;
-      if (x < ncand) keys[x] = order_key(best[u]);
+    for (int off = 1; off < 32; off <<= 1) {
+      un2 = fmaxf(un2, __shfl_xor_sync(0xffffffffu, un2, off));
+      cn2_max = fmaxf(cn2_max, __shfl_xor_sync(0xffffffffu, cn2_max, off));
+    }
+    if (lane == 0) {
+      rs.red[0][warp] = un2;
+      rs.red[1][warp] = cn2_max;
     }
   }
   __syncthreads();
+  float u2 = 0.f, c2 = 0.f;
+#pragma unroll
+  for (int w = 0; w < kSelThreads / 32; ++w) {
+    u2 = fmaxf(u2, rs.red[0][w]);
+    c2 = fmaxf(c2, rs.red[1][w]);
+  }
+  const float E = 0x1p-12f * sqrtf(u2) * sqrtf(c2) * 1.001f;
+  // 3. a lower bound of the k-th largest approximate score (its 16-bit key
+  // bin: within 2^-7 of it), and the candidates within 2E of that bound
+  uint32_t T, need;
+  radix_threshold<kSelThreads>(keys, ncand, a.topk, sh, T, need, 2);
+  const float theta = key_value(T) - 2.0f * E;
+  uint32_t* poss = keys + a.nb;
+  {
+    const int per = (ncand + kSelThreads - 1) / kSelThreads;
+    const int x0 = min(ncand, tid * per), x1 = min(ncand, x0 + per);
+    uint32_t own = 0;
+    for (int x = x0; x < x1; ++x) own += key_value(keys[x]) >= theta;
+    uint32_t at = static_cast<uint32_t>(block_exclusive_scan<kSelThreads>(own, sh));
+    if (tid == kSelThreads - 1) rs.n_poss = static_cast<int>(at + own);
+    for (int x = x0; x < x1; ++x) {
+      if (key_value(keys[x]) >= theta) poss[at++] = static_cast<uint32_t>(x);
+      keys[x] = 0u;
+    }
+  }
+  __syncthreads();
+  // 4. exact scores of those: four threads per candidate, a quarter of the
+  // rows each (the maximum does not depend on how the rows are grouped)
+  {
+    const int n_poss = rs.n_poss, sub = tid & 3, rows_per = a.block / 4;
+    for (int p0 = 0; p0 < n_poss; p0 += kSelThreads / 4) {
+      const int p = p0 + (tid >> 2);
+      float best = -INFINITY;
+      int x = 0;
+      if (p < n_poss) {
+        x = static_cast<int>(poss[p]);
+        float4 cv[4];
+        const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + 1) * kRank);
+#pragma unroll
+        for (int w = 0; w < 4; ++w) cv[w] = __ldg(c4 + w);
+        for (int i = sub * rows_per; i < (sub + 1) * rows_per; ++i) {
+          const float4* u4 = reinterpret_cast<const float4*>(rs.u[i]);
+          const float4 u0 = u4[0], u1 = u4[1], u2v = u4[2], u3 = u4[3];
+          const float uq[kRank] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w,
+                                   u2v.x, u2v.y, u2v.z, u2v.w, u3.x, u3.y, u3.z, u3.w};
+          best = fmaxf(best, score16_two_chains(uq, cv));
+        }
+      }
+      best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 1));
+      best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 2));
+      if (sub == 0 && p < n_poss) keys[x] = order_key(best);
+    }
+  }
+  __syncthreads();
+  // 5. selection on the exact keys
   const int n = select_from_keys(keys, ncand, t, a.topk, a.n_local, a.kmax, sh, out);
   if (tid == 0) a.cnt[row] = n;
 }
@@ -396,7 +568,7 @@ cudaError_t launch_select_dynamic(const SelectArgs& a, cudaStream_t stream) {
 
 cudaError_t launch_select_rowmax(const SelectArgs& a, cudaStream_t stream) {
   if (a.n_sparse == 0) return cudaSuccess;
-  const size_t smem = static_cast<size_t>(a.nb) * sizeof(uint32_t);
+  const size_t smem = 2 * static_cast<size_t>(a.nb) * sizeof(uint32_t);
   if (smem + sizeof(RowmaxScratch) + sizeof(SelectScratch) > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(block_select_rowmax_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));

@@ -52,12 +52,15 @@ __device__ __forceinline__ unsigned long long block_exclusive_scan(unsigned long
 // Radix select, most significant byte first, over keys[0, n) in shared
 // memory (1 <= k <= n): T = the k-th largest key and `need` = how many keys
 // equal to T belong to the k largest.  Called by all NT threads of the CTA.
+// With passes < 4 only the top 8 * passes bits are resolved: T is then the
+// smallest key of the bin that holds the k-th largest (a lower bound of it)
+// and `need` counts within that bin.
 template <int NT>
 __device__ inline void radix_threshold(const uint32_t* keys, int n, int k, SelectScratchT<NT>& sh, uint32_t& T,
-                                       uint32_t& need_out) {
+                                       uint32_t& need_out, int passes = 4) {
   const int tid = threadIdx.x;
   uint32_t prefix = 0, need = static_cast<uint32_t>(k);
-  for (int pass = 0; pass < 4; ++pass) {
+  for (int pass = 0; pass < passes; ++pass) {
     const int shift = 24 - 8 * pass;
     const uint32_t hi_mask = pass == 0 ? 0u : (0xFFFFFFFFu << (shift + 8));
     for (int e = tid; e < 256; e += NT) sh.hist[e] = 0;

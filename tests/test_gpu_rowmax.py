@@ -53,6 +53,7 @@ CASES = [
     (3072, 8, 1, [S], 256, 64, 12, 1),
     (1536, 32, 4, [S, S, W, S], 300, 128, 3, 1),  # group of 8
     (640, 4, 1, [S], 128, 64, 16, 2),  # fewer candidates than top-k in every block
+    (32768, 16, 2, [S, W], 1024, 128, 32, 4),  # 256 blocks: many candidates per query block
 ]
 
 
@@ -132,3 +133,36 @@ def test_rowmax_finds_a_planted_needle_the_mean_misses(rtp, cuda_device):
     torch.cuda.synchronize()
     plan.close()
     assert mean_sel == {0, m, t} and row_sel == {0, j, t}, (sorted(mean_sel), sorted(row_sel))
+
+
+@pytest.mark.parametrize("tied", ["some", "all"])
+def test_rowmax_exact_ties_take_the_lower_blocks(rtp, cuda_device, tied):
+    """Blocks with identical keys have identical centroids and scores.  With
+    a crowd of them at the cut (or every block identical, so that every
+    candidate is re-scored exactly), the kept ones are the lowest-indexed, as
+    in the oracle."""
+    n, hq, hkv, block, topk, n_local = 8192, 8, 1, 128, 7, 2
+    d = inputs.small_prefill(n, hq, hkv, [S], seed=9)
+    k = d["k"].clone()
+    nb = n // block
+    src = k[0, 0, 3 * block:4 * block].clone()
+    copies = range(1, nb) if tied == "all" else range(5, nb, 3)
+    for b in copies:
+        k[0, 0, b * block:(b + 1) * block] = src
+    q, k, v, proj = (x.to(cuda_device) for x in (d["q"], k, d["v"], d["proj"]))
+    cfg = rtp.AttnConfig(1, n, hq, hkv, 256, block, topk, n_local)
+    plan = rtp.Plan(cfg, [S])
+    bufs = plan.buffers(cuda_device)
+    rtp.rtp_indexer_project(plan.handle, q, k, proj, bufs["centroids"], bufs["qbar"])
+    rtp.rtp_block_select_rowmax(plan.handle, q, proj, bufs["centroids"], bufs["sel"], bufs["sel_cnt"])
+    torch.cuda.synchronize()
+    assert rtp.rtp_last_device_status() == rtp.RTP_OK
+    C = oracle.centroids(cpu(k[0, 0]), block, cpu(proj))
+    check_rowmax_rows(cpu(bufs["sel"][0, 0]).numpy(), cpu(bufs["sel_cnt"][0, 0]).numpy(), cpu(q[0]), cpu(proj), C,
+                      np.arange(nb), block, topk, n_local)
+    if tied == "all":
+        # every candidate scores the same: blocks 1..topk are kept
+        for t in range(topk + n_local + 1, nb):
+            got = bufs["sel"][0, 0, t, :int(bufs["sel_cnt"][0, 0, t])].tolist()
+            assert got == [0] + list(range(1, topk + 1)) + list(range(t - n_local + 1, t + 1)), (t, got)
+    plan.close()
