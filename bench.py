@@ -720,6 +720,18 @@ def time_clustered_decode(rtp, w, d, flush, flush_read, steps, stream, n_cluster
         if i > 0:
             km_runs.append(a.elapsed_time(b))
     km_ms = statistics.median(km_runs)
+    # the same clustering in place (no cluster-ordered K/V copy written)
+    cl_in = rtp.Clusters(w.batch, w.n_kv_heads, clu_end, n_clusters, B, d["kcache"].device, in_place=True)
+    km_in_runs = []
+    for i in range(3):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        rtp.rtp_cache_cluster(ccfg, kinds, iters, d["kcache"], d["vcache"], d["proj"], cl_in, km_ws, km_ws_bytes,
+                              stream)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i > 0:
+            km_in_runs.append(a.elapsed_time(b))
     del km_ws
     cfg = rtp.AttnConfig(w.batch, Lc, w.n_q_heads, w.n_kv_heads, w.window, B, w.topk, w.n_local)
     ws_bytes = rtp.rtp_decode_clustered_workspace_bytes(cfg, kinds, Lc, clu_end)
@@ -745,6 +757,23 @@ def time_clustered_decode(rtp, w, d, flush, flush_read, steps, stream, n_cluster
         ev.append((e0, e1))
     torch.cuda.synchronize()
     ms = statistics.median(x.elapsed_time(y) for x, y in ev)
+    # in place: the decode gathers member rows from the cache
+    args_in = (cfg, kinds, Lc, d["q"], d["kcache"], d["vcache"], d["proj"], cl_in, o, ws, ws_bytes, sel, cnt)
+    for _ in range(5):
+        rtp.rtp_sparse_decode_clustered(*args_in, stream=stream)
+    torch.cuda.synchronize()
+    ev_in = []
+    for _ in range(steps):
+        flush.zero_()
+        flush_read.sum()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        rtp.rtp_sparse_decode_clustered(*args_in, stream=stream)
+        e1.record(stream)
+        ev_in.append((e0, e1))
+    torch.cuda.synchronize()
+    ms_in = statistics.median(x.elapsed_time(y) for x, y in ev_in)
+    rtp.rtp_sparse_decode_clustered(*args, stream=stream)  # leave the copy-based selection in sel / cnt
     status = rtp.rtp_last_device_status(stream)
     # keys read: every retrieval head's sink block, tail and selected chunks, every window head's window
     sel_c, cnt_c = sel.cpu(), cnt.cpu()
@@ -759,8 +788,12 @@ def time_clustered_decode(rtp, w, d, flush, flush_read, steps, stream, n_cluster
                 keys += min(w.window, Lc)
     bytes_ = keys * 128 * 2 * 2 + w.batch * ns * cl.max_chunks * 16 * 4 + w.batch * w.n_q_heads * 128 * 2 * 2
     chunks = cl.n_chunks.cpu()[:, [h for h, k in enumerate(kinds) if k == inputs.SPARSE]].float()
+    copy_bytes = 2 * w.batch * ns * (clu_end - B) * 128 * 2
     return {"n_clusters": n_clusters, "iters": iters, "clu_end": clu_end, "kmeans_ms": km_ms,
             "kmeans_ms_runs": km_runs,
+            "in_place": {"kmeans_ms": statistics.median(km_in_runs), "ms_per_step": ms_in,
+                         "copy_bytes_saved": copy_bytes,
+                         "note": "no cluster-ordered K/V copy: the decode gathers member rows (16-byte cp.async)"},
             "mean_chunks_per_head": float(chunks.mean()), "ms_per_step": ms, "algorithmic_bytes": bytes_,
             "gb_s": bytes_ / (ms * 1e-3) / 1e9, "status": rtp.status_str(status)}
 
@@ -915,6 +948,9 @@ def secondary_summary(sec: dict) -> dict:
         c = d.get("clustered") or {}
         if "ms_per_step" in c:
             out["clustered_decode_us"] = round(c["ms_per_step"] * 1e3, 2)
+        if "in_place" in c:
+            out["clustered_in_place_decode_us"] = round(c["in_place"]["ms_per_step"] * 1e3, 2)
+            out["kmeans_in_place_ms"] = round(c["in_place"]["kmeans_ms"], 2)
         if "kmeans_ms" in c:
             out["kmeans_ms"] = round(c["kmeans_ms"], 2)
     for key, name in (("v2_128k_48_layers", "v2_128k_ms_per_layer"), ("v1_32k_48_layers", "v1_32k_ms_per_layer")):

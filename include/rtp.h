@@ -499,6 +499,11 @@ rtp_status rtp_cache_append(const rtp_attn_cfg* cfg, const uint8_t* kind_host, i
  * All arrays are device memory owned by the caller; n = clu_end - block,
  * max_chunks = n / 128 + n_clusters (an upper bound on the chunks of a head).
  * Entries of non-retrieval heads are not written or read.
+ * With k_sorted and v_sorted NULL no cluster-ordered copy of K/V is made
+ * (2 x n x 256 bytes per head saved, and its writing): the decode step then
+ * gathers each selected chunk's member rows from the cache itself (16-byte
+ * asynchronous copies into the same shared-memory layout), with the same
+ * result bit for bit.
  * ---------------------------------------------------------------------- */
 typedef struct {
   int clu_end;             /* rows [block, clu_end) are clustered: multiple of block, > block */
@@ -506,8 +511,8 @@ typedef struct {
   float* centroids;        /* fp32 [batch][n_kv_heads][n_clusters][16] */
   int32_t* members;        /* [batch][n_kv_heads][n]: key rows grouped by cluster, ascending inside */
   int32_t* offsets;        /* [batch][n_kv_heads][n_clusters + 1]: cluster c = members[offsets[c] ..] */
-  void* k_sorted;          /* bf16 [batch][n_kv_heads][n][128]: K rows in `members` order */
-  void* v_sorted;          /* bf16, likewise for V */
+  void* k_sorted;          /* bf16 [batch][n_kv_heads][n][128]: K rows in `members` order, or NULL */
+  void* v_sorted;          /* bf16, likewise for V (NULL exactly when k_sorted is) */
   float* chunk_centroids;  /* fp32 [batch][n_kv_heads][max_chunks][16]: the centroid of the chunk's cluster */
   int32_t* chunk_start;    /* [batch][n_kv_heads][max_chunks]: first row of the chunk in k_sorted */
   int32_t* chunk_len;      /* [batch][n_kv_heads][max_chunks]: 1..128 */
@@ -523,7 +528,7 @@ typedef struct {
  * index), each centroid to the mean of its keys (an empty cluster keeps its
  * centroid).  Then the members, offsets, chunk table and the K/V rows in
  * cluster order are written.  Deterministic (fixed-order sums, a stable
- * counting sort).
+ * counting sort).  The K/V copy is skipped when cl->k_sorted is NULL.
  *   cfg        batch, n_kv_heads, head_dim, block, rank used; seq = cache
  *              capacity as for rtp_sparse_decode (must be >= clu_end)
  *   kind_host  HOST [n_kv_heads]; RTP_HEAD_SPARSE heads are clustered

@@ -520,13 +520,16 @@ __device__ __forceinline__ void attn_producer(DecSmem& sm, const CUtensorMap* mk
       const int s_end = min(s + static_cast<int>(run_end - x), cnt);
       const bool sparse = a.kind[kvh] == KIND_SPARSE;
       const int start = a.kind[kvh] == KIND_SWA ? max(0, a.cache_len - a.window) : 0;
-      // clustered list-1 spans come from the cluster-ordered K/V
-      const bool sorted_src = a.clustered && list == 1;
+      // clustered list-1 spans come from the cluster-ordered K/V, or are
+      // gathered row by row from the cache (member rows, in place)
+      const bool gather_src = a.clustered && a.gather && list == 1;
+      const bool sorted_src = a.clustered && !a.gather && list == 1;
       const __nv_bfloat16* kbase = sorted_src ? a.k_sorted + bk * static_cast<size_t>(a.clu_rows) * kHeadDim
                                               : a.kcache + bk * static_cast<size_t>(a.cache_cap) * kHeadDim;
       const __nv_bfloat16* vbase = sorted_src ? a.v_sorted + bk * static_cast<size_t>(a.clu_rows) * kHeadDim
                                               : a.vcache + bk * static_cast<size_t>(a.cache_cap) * kHeadDim;
-      const int src_rows = sorted_src ? a.clu_rows : a.cache_len;
+      // (no L2 prefetch for gathered spans: their rows are not contiguous)
+      const int src_rows = gather_src ? 0 : (sorted_src ? a.clu_rows : a.cache_len);
       const CUtensorMap* tk = sorted_src ? mks : mk;
       const CUtensorMap* tv = sorted_src ? mvs : mv;
       for (int s0 = s; s0 < s_end && ok; s0 += 32) {
@@ -582,6 +585,54 @@ __device__ __forceinline__ void attn_producer(DecSmem& sm, const CUtensorMap* mk
           if (lane == i + kPrefetchAhead && lane < m) prefetch_span();
           const uint32_t st = issued % kRingStages, ph = (issued / kRingStages) & 1u;
           int okl = 1;
+          if (gather_src) {
+            // The chunk's member rows, gathered from the cache with 16-byte
+            // cp.async copies into the consumers' 128-byte-swizzled layout
+            // (sw128): lanes 0-15 copy row 2i's sixteen 16-byte pieces, lanes
+            // 16-31 row 2i+1's.  Rows past the chunk repeat its first member
+            // (masked by nk).  Each lane's copies complete on the stage's
+            // barriers (cp.async.mbarrier.arrive raises their pending count
+            // when issued); lane 0's plain arrive is the phase's own arrival.
+            if (lane == 0) okl = mbar_wait(&sm.empty[st], ph ^ 1u, abort, a.status) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+            if (!ok) break;
+            if (lane == 0) sm.nk[st] = nk;
+            // lane l loads the positions of rows 4l .. 4l+3 (all four in flight)
+            const int32_t* mem = a.members + bk * static_cast<size_t>(a.clu_rows) + key0;
+            int pv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) pv[u] = mem[4 * lane + u < nk ? 4 * lane + u : 0];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              if (pv[u] < 0 || pv[u] >= a.cache_len) {  // not a cached row: recorded, row 0 read instead
+                flag_error(a.status, RTP_DEVERR_INDEX);
+                pv[u] = 0;
+              }
+            const int hi = lane >> 4, piece = lane & 15;
+            const uint32_t ks = smem_u32(sm.k[st]), vs = smem_u32(sm.v[st]);
+            const __nv_bfloat16* kslab = a.kcache + bk * static_cast<size_t>(a.cache_cap) * kHeadDim + 8 * piece;
+            const __nv_bfloat16* vslab = a.vcache + bk * static_cast<size_t>(a.cache_cap) * kHeadDim + 8 * piece;
+#pragma unroll 4
+            for (int k2 = 0; k2 < 64; ++k2) {
+              // rows 2 k2 (lanes 0-15) and 2 k2 + 1 (lanes 16-31): held by
+              // lane k2 / 2 in registers 2 (k2 & 1) and 2 (k2 & 1) + 1
+              const int e0 = __shfl_sync(0xffffffffu, (k2 & 1) ? pv[2] : pv[0], k2 >> 1);
+              const int e1 = __shfl_sync(0xffffffffu, (k2 & 1) ? pv[3] : pv[1], k2 >> 1);
+              const int r = 2 * k2 + hi;
+              const size_t off = static_cast<size_t>(hi ? e1 : e0) * kHeadDim;
+              cp_async16(sw128(ks, r, 8 * piece), kslab + off);
+              cp_async16(sw128(vs, r, 8 * piece), vslab + off);
+            }
+            cp_async_arrive(&sm.k_full[st]);
+            cp_async_arrive(&sm.v_full[st]);
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(&sm.k_full[st]);
+              mbar_arrive(&sm.v_full[st]);
+            }
+            ++issued;
+            continue;
+          }
           if (lane == 0) {
             okl = mbar_wait(&sm.empty[st], ph ^ 1u, abort, a.status) ? 1 : 0;
             if (okl) {

@@ -94,11 +94,14 @@ struct DecodeArgs {
   // Clustered retrieval heads (k-means of the cache; 0 = contiguous blocks):
   // a retrieval head attends to the sink block, the unclustered tail
   // [clu_end, cache_len) (both in list 0) and the top-k chunks of its
-  // clusters (list 1), streamed from the cluster-ordered copy of K/V.
+  // clusters (list 1), streamed from the cluster-ordered copy of K/V or,
+  // with `gather`, read in place: the chunk's member rows of the cache.
   int clustered;
+  int gather;
   int clu_end, clu_rows, max_chunks;
-  const __nv_bfloat16* k_sorted;    // [batch][n_kv_heads][clu_rows][128]
+  const __nv_bfloat16* k_sorted;    // [batch][n_kv_heads][clu_rows][128] (NULL with gather)
   const __nv_bfloat16* v_sorted;
+  const int32_t* members;           // [batch][n_kv_heads][clu_rows]: cache rows in cluster order
   const float* chunk_centroids;     // [batch][n_kv_heads][max_chunks][16]
   const int32_t* chunk_start;       // [batch][n_kv_heads][max_chunks]
   const int32_t* chunk_len;

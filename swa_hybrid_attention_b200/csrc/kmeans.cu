@@ -27,7 +27,9 @@
 //                 (each summed over its keys in position order)
 //   km_chunks     each cluster's keys cut into chunks of <= 128 (the units
 //                 the decode step selects), with the cluster's centroid
-//   km_permute    K and V rows copied into cluster order (one warp per row)
+//   km_permute    K and V rows copied into cluster order (one warp per row;
+//                 skipped when the caller asks for no copy: the decode then
+//                 gathers member rows in place)
 
 #include <cuda_bf16.h>
 
@@ -320,8 +322,10 @@ cudaError_t launch_kmeans(const KmeansArgs& a, int iters, cudaStream_t stream) {
     km_group_kernel<<<per_head, kGroupThreads, 0, stream>>>(a);
   }
   km_chunks_kernel<<<per_head, kGroupThreads, 0, stream>>>(a);
-  const dim3 per_row((a.n + kKmThreads / 32 - 1) / (kKmThreads / 32), a.n_kv_heads, a.batch);
-  km_permute_kernel<<<per_row, kKmThreads, 0, stream>>>(a);
+  if (a.k_sorted) {  // no cluster-ordered copy when the decode reads member rows in place
+    const dim3 per_row((a.n + kKmThreads / 32 - 1) / (kKmThreads / 32), a.n_kv_heads, a.batch);
+    km_permute_kernel<<<per_row, kKmThreads, 0, stream>>>(a);
+  }
   return cudaGetLastError();
 }
 

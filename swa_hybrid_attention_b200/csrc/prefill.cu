@@ -63,7 +63,11 @@ constexpr int kLaunchRegs = 168;
 constexpr int kLowRegs = 88;
 constexpr int kHighRegs = 200;
 static_assert(128 * kLowRegs + 256 * kHighRegs <= kThreads * kLaunchRegs, "register split must fit the launch");
-constexpr int kStages = 2;
+// K/V rings of two stages each.  (A third K stage, loading K two tiles
+// ahead, fits in shared memory but measured no faster on the 1M layer: the
+// wait for K it removes moves to the P handshakes of the same chain.)
+constexpr int kKStages = 2;
+constexpr int kVStages = 2;
 constexpr uint32_t kTileBytes = 128 * 128 * 2;  // one 128x128 bf16 operand tile
 constexpr uint32_t kChunkBytes = 128 * 128;     // 64 columns x 128 rows
 constexpr int kNoWindow = 1 << 30;
@@ -88,16 +92,16 @@ static_assert(kPChunks == 1 || kPChunks == 2 || kPChunks == 4, "P chunks must di
 
 struct __align__(1024) Smem {
   uint8_t q[2][kTileBytes];
-  uint8_t k[kStages][kTileBytes];
-  uint8_t v[kStages][kTileBytes];
+  uint8_t k[kKStages][kTileBytes];
+  uint8_t v[kVStages][kTileBytes];
   uint64_t q_full[2], q_empty[2];
-  uint64_t k_full[kStages], v_full[kStages];
-  uint64_t k_empty[kStages];  // released once both heads' S MMAs of the tile have read K
-  uint64_t v_empty[kStages];  // released once both heads' P V MMAs have read V
+  uint64_t k_full[kKStages], v_full[kVStages];
+  uint64_t k_empty[kKStages];  // released once both heads' S MMAs of the tile have read K
+  uint64_t v_empty[kVStages];  // released once both heads' P V MMAs have read V
   uint64_t s_full[2], o_full[2];
   uint64_t p_full[2][kPChunks];  // [head][chunk of keys]: that part of P is in TMEM
   uint64_t drain;
-  uint32_t tile_mem[kStages];  // per-head selections: the pair's membership of the tile in each K stage
+  uint32_t tile_mem[kKStages];  // per-head selections: the pair's membership of the tile in each K stage
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -298,6 +302,7 @@ template <bool kHeads>
 __device__ __noinline__ void run_producer(Smem& s, const CUtensorMap* mq, const CUtensorMap* mk, const CUtensorMap* mv,
                              const PrefillArgs& a, volatile int* abort) {
   uint32_t it = 0, gt = 0;
+  uint32_t k_issued = 0, v_issued = 0;  // K / V tiles whose copies were issued
   uint32_t q_issued = 0;  // bit h: Q of head h issued for the current item
   for (long idx = blockIdx.x; idx < a.n_items; idx += gridDim.x, ++it) {
     Item item = load_item(a.items, idx, a.n_kv_heads);
@@ -315,21 +320,23 @@ __device__ __noinline__ void run_producer(Smem& s, const CUtensorMap* mq, const 
       ti.init(item, a);
       for (int j = 0; j < ti.n; ++j, ++gt) {
         TileRef tr = ti.next();
-        const int st = gt & 1;
-        const uint32_t use = gt >> 1;
-        if (!mbar_wait(&s.k_empty[st], (use & 1u) ^ 1u, abort, a.status)) goto drain;
-        if constexpr (kHeads) s.tile_mem[st] = (tr.flags >> 5) & 3u;  // published by the arrive below
-        mbar_arrive_expect_tx(&s.k_full[st], kTileBytes);
+        const int sk = static_cast<int>(gt % kKStages), sv = static_cast<int>(gt % kVStages);
+        const uint32_t uk = gt / kKStages, uv = gt / kVStages;
+        if (!mbar_wait(&s.k_empty[sk], (uk & 1u) ^ 1u, abort, a.status)) goto drain;
+        if constexpr (kHeads) s.tile_mem[sk] = (tr.flags >> 5) & 3u;  // published by the arrive below
+        mbar_arrive_expect_tx(&s.k_full[sk], kTileBytes);
         for (int c = 0; c < 2; ++c) {
-          tma_load_3d(s.k[st] + c * kChunkBytes, mk, &s.k_full[st], 64 * c, tr.row0, item.bkv);
-          tma_load_3d(s.k[st] + c * kChunkBytes + kChunkBytes / 2, mk, &s.k_full[st], 64 * c, tr.row1, item.bkv);
+          tma_load_3d(s.k[sk] + c * kChunkBytes, mk, &s.k_full[sk], 64 * c, tr.row0, item.bkv);
+          tma_load_3d(s.k[sk] + c * kChunkBytes + kChunkBytes / 2, mk, &s.k_full[sk], 64 * c, tr.row1, item.bkv);
         }
-        if (!mbar_wait(&s.v_empty[st], (use & 1u) ^ 1u, abort, a.status)) goto drain;
-        mbar_arrive_expect_tx(&s.v_full[st], kTileBytes);
+        ++k_issued;
+        if (!mbar_wait(&s.v_empty[sv], (uv & 1u) ^ 1u, abort, a.status)) goto drain;
+        mbar_arrive_expect_tx(&s.v_full[sv], kTileBytes);
         for (int c = 0; c < 2; ++c) {
-          tma_load_3d(s.v[st] + c * kChunkBytes, mv, &s.v_full[st], 64 * c, tr.row0, item.bkv);
-          tma_load_3d(s.v[st] + c * kChunkBytes + kChunkBytes / 2, mv, &s.v_full[st], 64 * c, tr.row1, item.bkv);
+          tma_load_3d(s.v[sv] + c * kChunkBytes, mv, &s.v_full[sv], 64 * c, tr.row0, item.bkv);
+          tma_load_3d(s.v[sv] + c * kChunkBytes + kChunkBytes / 2, mv, &s.v_full[sv], 64 * c, tr.row1, item.bkv);
         }
+        ++v_issued;
       }
     }
   }
@@ -337,10 +344,13 @@ __device__ __noinline__ void run_producer(Smem& s, const CUtensorMap* mq, const 
 drain:
   // Give up: wait (bounded) for the copies already issued so that no TMA
   // write lands in shared memory after the CTA has exited.
-  for (uint32_t x = 0; x < 2 && x < gt; ++x) {
-    uint32_t g = gt - 1 - x;
-    drain_wait(&s.k_full[g & 1], (g >> 1) & 1u, a.status);
-    drain_wait(&s.v_full[g & 1], (g >> 1) & 1u, a.status);
+  for (uint32_t x = 0; x < kKStages && x < k_issued; ++x) {
+    const uint32_t g = k_issued - 1 - x;
+    drain_wait(&s.k_full[g % kKStages], (g / kKStages) & 1u, a.status);
+  }
+  for (uint32_t x = 0; x < kVStages && x < v_issued; ++x) {
+    const uint32_t g = v_issued - 1 - x;
+    drain_wait(&s.v_full[g % kVStages], (g / kVStages) & 1u, a.status);
   }
   for (int h = 0; h < 2; ++h)
     if (q_issued & (1u << h)) drain_wait(&s.q_full[h], it & 1u, a.status);
@@ -450,8 +460,8 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
     uint32_t mem_cur = 3u;
     bool started0 = false, started1 = false;
     {
-      const int st0 = gt & 1;
-      if (!mma_wait(&s.k_full[st0], (gt >> 1) & 1u, abort, a.status)) goto drain;
+      const int st0 = static_cast<int>(gt % kKStages);
+      if (!mma_wait(&s.k_full[st0], (gt / kKStages) & 1u, abort, a.status)) goto drain;
       tc_fence_after();
       if constexpr (kHeads) mem_cur = s.tile_mem[st0];
       const uint64_t sk = st0 ? kd1 : kd0;
@@ -467,12 +477,12 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
     }
     for (int j = 0; j < n; ++j) {
       const uint32_t g = gt + j;
-      const int st = g & 1;
+      const int st = static_cast<int>(g % kVStages);
       const bool has_next = j + 1 < n;
-      const int st2 = (g + 1) & 1;
+      const int st2 = static_cast<int>((g + 1) % kKStages);
       const uint64_t sv = st ? vd1 : vd0;
       const uint64_t sk2 = st2 ? kd1 : kd0;
-      if (!mma_wait(&s.v_full[st], (g >> 1) & 1u, abort, a.status)) goto drain;
+      if (!mma_wait(&s.v_full[st], (g / kVStages) & 1u, abort, a.status)) goto drain;
       uint32_t mem_next = 3u;
       // head 0: O0 += P0 V ; then S0 for the next tile
       if (!pv_or_skip<kHeads>(s, 0, (mem_cur & 1u) != 0, pc & 1u, tO[0], tS[0], sv, id_pv, kHeads ? started0 : j > 0,
@@ -482,7 +492,7 @@ __device__ __noinline__ void run_mma(Smem& s, uint32_t tmem, const PrefillArgs& 
       if (!has_next) {
         umma_commit(&s.o_full[0]);
       } else {
-        if (!mma_wait(&s.k_full[st2], ((g + 1) >> 1) & 1u, abort, a.status)) goto drain;
+        if (!mma_wait(&s.k_full[st2], ((g + 1) / kKStages) & 1u, abort, a.status)) goto drain;
         tc_fence_after();
         if constexpr (kHeads) mem_next = s.tile_mem[st2];
         if (!kHeads || (mem_next & 1u)) issue_qk(tS[0], qd0, sk2, id_qk);
@@ -666,10 +676,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int q = 0; q < kPChunks; ++q) mbar_init(&s.p_full[h][q], 128);
       mbar_init(&s.o_full[h], 1);
     }
-    for (int st = 0; st < kStages; ++st) {
+    for (int st = 0; st < kKStages; ++st) {
       mbar_init(&s.k_full[st], 1);
-      mbar_init(&s.v_full[st], 1);
       mbar_init(&s.k_empty[st], 1);
+    }
+    for (int st = 0; st < kVStages; ++st) {
+      mbar_init(&s.v_full[st], 1);
       mbar_init(&s.v_empty[st], 1);
     }
     mbar_init(&s.drain, 1);

@@ -739,9 +739,11 @@ bool cluster_args_ok(const rtp_attn_cfg* c, const uint8_t* kind, const rtp_clust
   if (cl->clu_end <= c->block || cl->clu_end % c->block != 0 || cl->clu_end > cap) return false;
   const int n = cl->clu_end - c->block;
   if (cl->n_clusters < 1 || cl->n_clusters > kMaxClusters || cl->n_clusters > n) return false;
-  if (!cl->centroids || !cl->members || !cl->offsets || !cl->k_sorted || !cl->v_sorted || !cl->chunk_centroids ||
-      !cl->chunk_start || !cl->chunk_len || !cl->n_chunks)
+  if (!cl->centroids || !cl->members || !cl->offsets || !cl->chunk_centroids || !cl->chunk_start || !cl->chunk_len ||
+      !cl->n_chunks)
     return false;
+  // k_sorted / v_sorted: both given (cluster-ordered copy) or both NULL (in place)
+  if ((cl->k_sorted == nullptr) != (cl->v_sorted == nullptr)) return false;
   return aligned16(cl->centroids) && aligned16(cl->k_sorted) && aligned16(cl->v_sorted) &&
          aligned16(cl->chunk_centroids);
 }
@@ -789,6 +791,8 @@ rtp_status prepare_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int
   a.max_chunks = cl ? a.clu_rows / 128 + cl->n_clusters : 0;
   a.k_sorted = cl ? static_cast<const __nv_bfloat16*>(cl->k_sorted) : nullptr;
   a.v_sorted = cl ? static_cast<const __nv_bfloat16*>(cl->v_sorted) : nullptr;
+  a.members = cl ? cl->members : nullptr;
+  a.gather = cl && !cl->k_sorted ? 1 : 0;
   a.chunk_centroids = cl ? cl->chunk_centroids : nullptr;
   a.chunk_start = cl ? cl->chunk_start : nullptr;
   a.chunk_len = cl ? cl->chunk_len : nullptr;
@@ -812,7 +816,10 @@ rtp_status run_decode(DecodeArgs& a, const DecodeLayout& L, char* ws, int32_t* s
   if (!encode_bf16_3d(&mk, a.kcache, a.cache_len, slabs, 64, a.cache_cap) ||
       !encode_bf16_3d(&mv, a.vcache, a.cache_len, slabs, 64, a.cache_cap))
     return RTP_ERR_CUDA;
-  if (cl) {
+  if (cl && a.gather) {
+    mks = mk;  // unused: gathered spans are copied with cp.async
+    mvs = mv;
+  } else if (cl) {
     if (!encode_bf16_3d(&mks, cl->k_sorted, a.clu_rows, slabs, 64) ||
         !encode_bf16_3d(&mvs, cl->v_sorted, a.clu_rows, slabs, 64))
       return RTP_ERR_CUDA;

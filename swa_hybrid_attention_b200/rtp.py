@@ -350,7 +350,10 @@ def rtp_cache_append(cfg: AttnConfig, kinds, pos: int, k_new, v_new, kcache, vca
 class Clusters:
     """Device arrays of a clustered KV cache (rtp_clusters), allocated with torch."""
 
-    def __init__(self, batch: int, n_kv_heads: int, clu_end: int, n_clusters: int, block: int, device):
+    def __init__(self, batch: int, n_kv_heads: int, clu_end: int, n_clusters: int, block: int, device,
+                 in_place: bool = False):
+        """in_place: no cluster-ordered copy of K/V (k_sorted / v_sorted NULL):
+        the clustered decode gathers each chunk's member rows from the cache."""
         n = clu_end - block
         self.clu_end, self.n_clusters, self.n = clu_end, n_clusters, n
         self.max_chunks = n // 128 + n_clusters
@@ -358,8 +361,11 @@ class Clusters:
         self.centroids = torch.zeros(batch, n_kv_heads, n_clusters, 16, dtype=torch.float32, device=device)
         self.members = torch.zeros(batch, n_kv_heads, n, **i32)
         self.offsets = torch.zeros(batch, n_kv_heads, n_clusters + 1, **i32)
-        self.k_sorted = torch.zeros(batch, n_kv_heads, n, 128, dtype=torch.bfloat16, device=device)
-        self.v_sorted = torch.zeros_like(self.k_sorted)
+        if in_place:
+            self.k_sorted = self.v_sorted = None
+        else:
+            self.k_sorted = torch.zeros(batch, n_kv_heads, n, 128, dtype=torch.bfloat16, device=device)
+            self.v_sorted = torch.zeros_like(self.k_sorted)
         self.chunk_centroids = torch.zeros(batch, n_kv_heads, self.max_chunks, 16, dtype=torch.float32,
                                            device=device)
         self.chunk_start = torch.zeros(batch, n_kv_heads, self.max_chunks, **i32)
@@ -401,12 +407,13 @@ def rtp_sparse_decode_clustered(cfg: AttnConfig, kinds, cache_len: int, q, kcach
 
 
 def cluster_cache(kcache, vcache, proj, kinds, *, clu_end: int, n_clusters: int, iters: int = 8, block: int = 128,
-                  stream=None) -> Clusters:
+                  stream=None, in_place: bool = False) -> Clusters:
     """k-means clustering of rows [block, clu_end) of the retrieval heads of a
-    cache [batch][n_kv_heads][capacity][128]; returns the Clusters arrays."""
+    cache [batch][n_kv_heads][capacity][128]; returns the Clusters arrays
+    (in_place: without the cluster-ordered copy of K/V)."""
     B, H, cap = kcache.shape[0], kcache.shape[1], kcache.shape[2]
     cfg = AttnConfig(B, cap, H, H, 1, block, 0, 1)
-    cl = Clusters(B, H, clu_end, n_clusters, block, kcache.device)
+    cl = Clusters(B, H, clu_end, n_clusters, block, kcache.device, in_place=in_place)
     ws_bytes = rtp_cache_cluster_workspace_bytes(cfg, clu_end)
     if ws_bytes == 0:
         raise RtpError("rtp_cache_cluster_workspace_bytes", RTP_ERR_INVALID_ARG)

@@ -133,10 +133,11 @@ def test_kmeans_recovers_planted_blobs_exactly(rtp, cuda_device):
     assert np.all(np.abs(mu - mu_o) <= IDX_ABS + IDX_REL * np.abs(mu_o))
 
 
-def clusters_from_oracle(rtp, k, v, proj, kinds, clu_end, nc, iters, block):
-    """The oracle's clustering, laid out in the rtp_clusters arrays."""
+def clusters_from_oracle(rtp, k, v, proj, kinds, clu_end, nc, iters, block, in_place=False):
+    """The oracle's clustering, laid out in the rtp_clusters arrays (in_place:
+    without the cluster-ordered K/V copy)."""
     B, H = k.shape[0], k.shape[1]
-    cl = rtp.Clusters(B, H, clu_end, nc, block, k.device)
+    cl = rtp.Clusters(B, H, clu_end, nc, block, k.device, in_place=in_place)
     per_head = {}
     for b in range(B):
         for h in range(H):
@@ -149,9 +150,10 @@ def clusters_from_oracle(rtp, k, v, proj, kinds, clu_end, nc, iters, block):
             cl.centroids[b, h] = mu32.to(k.device)
             cl.members[b, h] = torch.from_numpy(members.astype(np.int32)).to(k.device)
             cl.offsets[b, h] = torch.from_numpy(offsets.astype(np.int32)).to(k.device)
-            idx = torch.from_numpy(members).to(k.device)
-            cl.k_sorted[b, h] = k[b, h].index_select(0, idx)
-            cl.v_sorted[b, h] = v[b, h].index_select(0, idx)
+            if not in_place:
+                idx = torch.from_numpy(members).to(k.device)
+                cl.k_sorted[b, h] = k[b, h].index_select(0, idx)
+                cl.v_sorted[b, h] = v[b, h].index_select(0, idx)
             cc = np.zeros((cl.max_chunks, 16), dtype=np.float32)
             for i, (c, s0, m) in enumerate(chunks):
                 cl.chunk_start[b, h, i] = s0
@@ -184,8 +186,13 @@ def test_clustered_decode_matches_oracle(rtp, cuda_device, case):
     cl, per_head = clusters_from_oracle(rtp, k, v, proj, kinds, clu_end, nc, 3, block)
     o, sel, cnt = rtp.sparse_decode_clustered_step(q, k, v, proj, kinds, cl, window=window, block=block, topk=topk,
                                                    cache_len=Lc, return_selection=True)
+    # the same clustering without the K/V copy: member rows gathered in place
+    cl_in, _ = clusters_from_oracle(rtp, k, v, proj, kinds, clu_end, nc, 3, block, in_place=True)
+    o_in, sel_in, cnt_in = rtp.sparse_decode_clustered_step(q, k, v, proj, kinds, cl_in, window=window, block=block,
+                                                            topk=topk, cache_len=Lc, return_selection=True)
     torch.cuda.synchronize()
     assert rtp.rtp_last_device_status() == rtp.RTP_OK
+    assert torch.equal(o_in, o) and torch.equal(sel_in, sel) and torch.equal(cnt_in, cnt)
     sel, cnt, o = cpu(sel).numpy(), cpu(cnt).numpy(), cpu(o)
     n_tail = (Lc - clu_end + 127) // 128
     errs = []
@@ -229,8 +236,15 @@ def test_gpu_clustering_then_decode_runs_clean(rtp, cuda_device):
     cl = rtp.cluster_cache(k, v, proj, kinds, clu_end=clu_end, n_clusters=nc, iters=4, block=block)
     o, sel, cnt = rtp.sparse_decode_clustered_step(q, k, v, proj, kinds, cl, window=800, block=block, topk=topk,
                                                    cache_len=Lc, return_selection=True)
+    # in place: the same clustering (no K/V copy written) and the same step
+    cl_in = rtp.cluster_cache(k, v, proj, kinds, clu_end=clu_end, n_clusters=nc, iters=4, block=block, in_place=True)
+    o_in, sel_in, _ = rtp.sparse_decode_clustered_step(q, k, v, proj, kinds, cl_in, window=800, block=block,
+                                                       topk=topk, cache_len=Lc, return_selection=True)
     torch.cuda.synchronize()
     assert rtp.rtp_last_device_status() == rtp.RTP_OK
+    for name in ("centroids", "members", "offsets", "chunk_start", "chunk_len", "n_chunks", "chunk_centroids"):
+        assert torch.equal(getattr(cl, name), getattr(cl_in, name)), name
+    assert torch.equal(o_in, o) and torch.equal(sel_in, sel)
     G = Hq // Hkv
     for b in range(B):
         n_ch = int(cl.n_chunks[b, 0])
@@ -259,8 +273,11 @@ def test_clustered_decode_full_size_cache(rtp, cuda_device):
     cl, per_head = clusters_from_oracle(rtp, k, v, proj, kinds, clu_end, 256, 2, B)
     o, sel, cnt = rtp.sparse_decode_clustered_step(q, k, v, proj, kinds, cl, window=w.window, block=B, topk=w.topk,
                                                    return_selection=True)
+    cl.k_sorted = cl.v_sorted = None  # the same clustering, read in place
+    o_in = rtp.sparse_decode_clustered_step(q, k, v, proj, kinds, cl, window=w.window, block=B, topk=w.topk)
     torch.cuda.synchronize()
     assert rtp.rtp_last_device_status() == rtp.RTP_OK
+    assert torch.equal(o_in, o)
     sel, cnt, o = cpu(sel).numpy(), cpu(cnt).numpy(), cpu(o)
     G = w.group
     n_tail = (Lc - clu_end + 127) // 128
