@@ -312,7 +312,9 @@ struct RowmaxScratch {
   // distinct banks (a dense [128][16] layout puts all 16 lanes of a row in
   // one bank: a 16-way conflict on every load)
   float projv[8][16][20];
-  float u[128][kRank];  // block <= 128 rows
+  // block <= 128 rows, padded to 20 words so that the exact re-score's four
+  // threads of a candidate (rows 4i .. 4i+3 at a time) read distinct banks
+  float u[128][20];
   float red[2][kSelThreads / 32];
   int n_poss;
 };
@@ -335,10 +337,6 @@ __device__ __forceinline__ void mma_m16n8k16_bf16(float (&d)[4], const uint32_t 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Inverse of order_key.
-__device__ __forceinline__ float key_value(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
-}
 
 __global__ void __launch_bounds__(kSelThreads, 2) block_select_rowmax_kernel(const SelectArgs a) {
   extern __shared__ uint32_t keys[];  // [nb] order keys, then [nb] candidates to re-score
@@ -502,17 +500,17 @@ __global__ void __launch_bounds__(kSelThreads, 2) block_select_rowmax_kernel(con
   // bin: within 2^-7 of it), and the candidates within 2E of that bound
   uint32_t T, need;
   radix_threshold<kSelThreads>(keys, ncand, a.topk, sh, T, need, 2);
-  const float theta = key_value(T) - 2.0f * E;
+  const float theta = key_score(T) - 2.0f * E;
   uint32_t* poss = keys + a.nb;
   {
     const int per = (ncand + kSelThreads - 1) / kSelThreads;
     const int x0 = min(ncand, tid * per), x1 = min(ncand, x0 + per);
     uint32_t own = 0;
-    for (int x = x0; x < x1; ++x) own += key_value(keys[x]) >= theta;
+    for (int x = x0; x < x1; ++x) own += key_score(keys[x]) >= theta;
     uint32_t at = static_cast<uint32_t>(block_exclusive_scan<kSelThreads>(own, sh));
     if (tid == kSelThreads - 1) rs.n_poss = static_cast<int>(at + own);
     for (int x = x0; x < x1; ++x) {
-      if (key_value(keys[x]) >= theta) poss[at++] = static_cast<uint32_t>(x);
+      if (key_score(keys[x]) >= theta) poss[at++] = static_cast<uint32_t>(x);
       keys[x] = 0u;
     }
   }
@@ -521,7 +519,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) block_select_rowmax_kernel(con
   // rows each (the maximum does not depend on how the rows are grouped)
   {
     const int n_poss = rs.n_poss, sub = tid & 3, rows_per = a.block / 4;
-    for (int p0 = 0; p0 < n_poss; p0 += kSelThreads / 4) {
+    for (int p0 = 0; p0 < n_poss; p0 += kSelThreads / 4) {  // sub s takes rows 4i + s
       const int p = p0 + (tid >> 2);
       float best = -INFINITY;
       int x = 0;
@@ -531,8 +529,9 @@ __global__ void __launch_bounds__(kSelThreads, 2) block_select_rowmax_kernel(con
         const float4* c4 = reinterpret_cast<const float4*>(C + static_cast<size_t>(x + 1) * kRank);
 #pragma unroll
         for (int w = 0; w < 4; ++w) cv[w] = __ldg(c4 + w);
-        for (int i = sub * rows_per; i < (sub + 1) * rows_per; ++i) {
-          const float4* u4 = reinterpret_cast<const float4*>(rs.u[i]);
+#pragma unroll 4
+        for (int ii = 0; ii < rows_per; ++ii) {
+          const float4* u4 = reinterpret_cast<const float4*>(rs.u[4 * ii + sub]);
           const float4 u0 = u4[0], u1 = u4[1], u2v = u4[2], u3 = u4[3];
           const float uq[kRank] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w,
                                    u2v.x, u2v.y, u2v.z, u2v.w, u3.x, u3.y, u3.z, u3.w};
