@@ -20,6 +20,7 @@
 // The centroids of one (slot, sequence) are 16 fp32 per block and stay in L2.
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "internal.cuh"
 #include "select_common.cuh"
@@ -262,28 +263,33 @@ __global__ void __launch_bounds__(kSelThreads) block_select_dynamic_kernel(const
 // Per CTA (one query block):
 //  1. u_i of the block's rows into shared memory (16 threads per row sum the
 //     group's heads over 8 dims each and project; the 16 partial dot
-//     products of a rank are added in a fixed butterfly, lane 0's result
-//     kept).
+//     products of each rank are added by a fixed reduce-scatter tree, lane
+//     c ending with rank c).
 //  2. Approximate scores on the tensor cores: the (rows x 16) . (16 x 8
-//     candidates) products are mma.sync m16n8k16 with both operands split
-//     into bf16 hi + lo parts (hi.hi + hi.lo + lo.hi, fp32 accumulation), the
-//     maximum over rows taken from the accumulator fragments.  Each split
-//     keeps 16 bits of mantissa, so an approximate dot product is within
-//     2^-14 |u_i| |c_j| of the exact one and the approximate row maximum a_j
-//     within E = 2^-12 max_i |u_i| max_j |c_j| (a 4x margin) of the exact
-//     fp32 score s_j of step 4.
+//     candidates) products are mma.sync m16n8k16 on fp16 operands (u scaled
+//     by an exact power of two su so that every entry lies below 2^14; c as
+//     is), fp32 accumulation, the maximum over rows taken from the
+//     accumulator fragments.  Rounding each operand to fp16 costs at most
+//     2^-11 of it (plus 2^-25 below fp16's normal range), so an approximate
+//     row maximum a_j is within
+//       E = 2^-9 max|su u_i| max|c_j| + 2^-22 (max|su u_i| + max|c_j|)
+//     (about a 2x margin, the accumulation's rounding included) of su s_j,
+//     s_j the exact fp32 score of step 4.  If some |c_j| reaches 2^15 (fp16
+//     could overflow) no approximation is used: every candidate goes to step
+//     4.
 //  3. A lower bound b of the k-th largest approximate score a_(k) (two radix
 //     passes: the low edge of its 16-bit key bin).  At least k candidates
-//     have s >= a_(k) - E >= b - E, so a candidate with a_j < b - 2E has
-//     s_j < b - E and is not among the k best: only the others (the k best
-//     and those within 2E of the bin, 2^-7 relative wide) need their exact
-//     score.
-//  4. Those candidates are re-scored exactly (fp32, the 16-term dot product
-//     in two fixed-order chains of 8 then their sum, maximum over rows: the
-//     score every earlier version of this kernel computed for every
-//     candidate); the others get key 0, below every finite score's key.
-//  5. The fixed kernel's radix select and ordered compaction on those keys:
-//     the same selection as exact scores for every candidate.
+//     have su s >= a_(k) - E >= b - E, so a candidate with a_j < b - 2E has
+//     su s_j < b - E and is not among the k best: only the others (the k
+//     best and those within 2E of the bin, 2^-7 relative wide) need their
+//     exact score.
+//  4. Those candidates (listed in ascending order) are re-scored exactly
+//     (fp32, the 16-term dot product in two fixed-order chains of 8 then
+//     their sum, maximum over rows: the score every earlier version of this
+//     kernel computed for every candidate).
+//  5. The fixed kernel's radix select and ordered compaction over the listed
+//     candidates' exact keys: the same selection as exact scores for every
+//     candidate.
 
 // u . c with ranks 0-7 and 8-15 in two fma chains (fixed order), added at
 // the end: half the dependent latency of one 16-long chain.
@@ -319,19 +325,15 @@ struct RowmaxScratch {
   int n_poss;
 };
 
-// hi = bf16(x, y) (x in the low half), lo = bf16 of the remainders.
-__device__ __forceinline__ uint32_t bf16x2_bits(float x, float y) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(x, y);
+// fp16 pair (x in the low half), round to nearest.
+__device__ __forceinline__ uint32_t f16x2_bits(float x, float y) {
+  const __half2 v = __floats2half2_rn(x, y);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
-__device__ __forceinline__ void split_bf16x2(float x, float y, uint32_t& hi, uint32_t& lo) {
-  hi = bf16x2_bits(x, y);
-  lo = bf16x2_bits(x - __uint_as_float(hi << 16), y - __uint_as_float(hi & 0xFFFF0000u));
-}
 
-__device__ __forceinline__ void mma_m16n8k16_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+__device__ __forceinline__ void mma_m16n8k16_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
@@ -403,34 +405,77 @@ __global__ void __launch_bounds__(kSelThreads, 2) block_select_rowmax_kernel(con
           v[4 * w + 3] = fmaf(p4.w, sum[e], v[4 * w + 3]);
         }
       }
+      // reduce-scatter over the row's 16 lanes (a fixed tree): at each step a
+      // lane keeps the half of its ranks that matches its lane bit and adds
+      // the partner's copy of that half, so lane cg ends with rank cg summed
+      // over all 16 lanes
 #pragma unroll
-      for (int c = 0; c < kRank; ++c) {
-        v[c] += __shfl_xor_sync(0xffffffffu, v[c], 8);
-        v[c] += __shfl_xor_sync(0xffffffffu, v[c], 4);
-        v[c] += __shfl_xor_sync(0xffffffffu, v[c], 2);
-        v[c] += __shfl_xor_sync(0xffffffffu, v[c], 1);
-        if (cg == 0) rs.u[i][c] = v[c];
+      for (int j = 0; j < 8; ++j) {
+        const bool up = (cg & 8) != 0;
+        const float send = up ? v[j] : v[j + 8], keep = up ? v[j + 8] : v[j];
+        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const bool up = (cg & 4) != 0;
+        const float send = up ? v[j] : v[j + 4], keep = up ? v[j + 4] : v[j];
+        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, 4);
+      }
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const bool up = (cg & 2) != 0;
+        const float send = up ? v[j] : v[j + 2], keep = up ? v[j + 2] : v[j];
+        v[j] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+      }
+      {
+        const bool up = (cg & 1) != 0;
+        const float send = up ? v[0] : v[1], keep = up ? v[1] : v[0];
+        rs.u[i][cg] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
       }
     }
   }
   __syncthreads();
   const float* C = a.centroids + (static_cast<size_t>(b) * a.n_sparse + slot) * a.nb * kRank;
   const int mtiles = a.block / 16;  // 16-row tiles of u (4 or 8)
-  // 2. approximate scores, 8 candidates per warp step.  Fragments of
-  // m16n8k16 (g = lane / 4, q = lane % 4): A rows g and g+8 of the tile,
-  // dims 2q, 2q+1 and 2q+8, 2q+9; B column g (candidate 8 gi + g), the same
-  // dims; D rows g and g+8, candidates 2q and 2q+1.
+  // the largest |u_i| sets u's scale for the fp16 products: su = 2^(14 - e)
+  // with max|u_i| in [2^(e-1), 2^e), so that every su u_i,d lies below 2^14
+  // (scaling by a power of two is exact; scores and bounds below are all in
+  // this scaled unit, so the comparisons do not change)
+  {
+    float un2 = 0.f;
+    if (tid < a.block) {
+#pragma unroll
+      for (int c = 0; c < kRank; ++c) un2 = fmaf(rs.u[tid][c], rs.u[tid][c], un2);
+    }
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) un2 = fmaxf(un2, __shfl_xor_sync(0xffffffffu, un2, off));
+    if (lane == 0) rs.red[0][warp] = un2;
+  }
+  __syncthreads();
+  float u2 = 0.f;
+#pragma unroll
+  for (int w = 0; w < kSelThreads / 32; ++w) u2 = fmaxf(u2, rs.red[0][w]);
+  const float umax = sqrtf(u2) * 1.001f;
+  int ue = 0;
+  frexpf(umax, &ue);
+  const float su = umax > 0.f ? ldexpf(1.f, 14 - ue) : 1.f;
+  // 2. approximate scores, 8 candidates per warp step: the
+  // (rows x 16) . (16 x 8 candidates) products as mma.sync m16n8k16 on fp16
+  // operands (su u and c), fp32 accumulation.  Fragments (g = lane / 4,
+  // q = lane % 4): A rows g and g+8 of the tile, dims 2q, 2q+1 and 2q+8,
+  // 2q+9; B column g (candidate 8 gi + g), the same dims; D rows g and g+8,
+  // candidates 2q and 2q+1.
   float cn2_max = 0.f;
   {
     const int g = lane >> 2, q = lane & 3;
-    uint32_t ahi[8][4], alo[8][4];
+    uint32_t af[8][4];
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
       if (mt < mtiles) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int r = 16 * mt + g + 8 * (e & 1), k = 2 * q + 8 * (e >> 1);
-          split_bf16x2(rs.u[r][k], rs.u[r][k + 1], ahi[mt][e], alo[mt][e]);
+          af[mt][e] = f16x2_bits(su * rs.u[r][k], su * rs.u[r][k + 1]);
         }
       }
     }
@@ -440,9 +485,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) block_select_rowmax_kernel(con
       const float* cp = C + static_cast<size_t>(min(xg, ncand - 1) + 1) * kRank;
       const float2 c0 = __ldg(reinterpret_cast<const float2*>(cp + 2 * q));
       const float2 c1 = __ldg(reinterpret_cast<const float2*>(cp + 2 * q + 8));
-      uint32_t bhi0, blo0, bhi1, blo1;
-      split_bf16x2(c0.x, c0.y, bhi0, blo0);
-      split_bf16x2(c1.x, c1.y, bhi1, blo1);
+      const uint32_t b0 = f16x2_bits(c0.x, c0.y), b1 = f16x2_bits(c1.x, c1.y);
       float n2 = c0.x * c0.x + c0.y * c0.y + c1.x * c1.x + c1.y * c1.y;
       n2 += __shfl_xor_sync(0xffffffffu, n2, 1);
       n2 += __shfl_xor_sync(0xffffffffu, n2, 2);
@@ -452,9 +495,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) block_select_rowmax_kernel(con
       for (int mt = 0; mt < 8; ++mt) {
         if (mt < mtiles) {
           float d[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_m16n8k16_bf16(d, alo[mt], bhi0, bhi1);
-          mma_m16n8k16_bf16(d, ahi[mt], blo0, blo1);
-          mma_m16n8k16_bf16(d, ahi[mt], bhi0, bhi1);
+          mma_m16n8k16_f16(d, af[mt], b0, b1);
           m0 = fmaxf(m0, fmaxf(d[0], d[2]));
           m1 = fmaxf(m1, fmaxf(d[1], d[3]));
         }
@@ -471,48 +512,34 @@ __global__ void __launch_bounds__(kSelThreads, 2) block_select_rowmax_kernel(con
       }
     }
   }
-  // the bound E from the largest |u_i| and |c_j|
-  {
-    float un2 = 0.f;
-    if (tid < a.block) {
+  // the bound E (scaled unit) from the largest |su u_i| and |c_j|
 #pragma unroll
-      for (int c = 0; c < kRank; ++c) un2 = fmaf(rs.u[tid][c], rs.u[tid][c], un2);
-    }
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      un2 = fmaxf(un2, __shfl_xor_sync(0xffffffffu, un2, off));
-      cn2_max = fmaxf(cn2_max, __shfl_xor_sync(0xffffffffu, cn2_max, off));
-    }
-    if (lane == 0) {
-      rs.red[0][warp] = un2;
-      rs.red[1][warp] = cn2_max;
-    }
-  }
+  for (int off = 1; off < 32; off <<= 1) cn2_max = fmaxf(cn2_max, __shfl_xor_sync(0xffffffffu, cn2_max, off));
+  if (lane == 0) rs.red[1][warp] = cn2_max;
   __syncthreads();
-  float u2 = 0.f, c2 = 0.f;
+  float c2 = 0.f;
 #pragma unroll
-  for (int w = 0; w < kSelThreads / 32; ++w) {
-    u2 = fmaxf(u2, rs.red[0][w]);
-    c2 = fmaxf(c2, rs.red[1][w]);
-  }
-  const float E = 0x1p-12f * sqrtf(u2) * sqrtf(c2) * 1.001f;
+  for (int w = 0; w < kSelThreads / 32; ++w) c2 = fmaxf(c2, rs.red[1][w]);
+  const float cmax = sqrtf(c2) * 1.001f, sumax = su * umax;
+  // a centroid entry at or above 2^15 could overflow fp16 (65504): then no
+  // approximate score is trusted and every candidate is scored exactly
+  const bool trusted = cmax < 32768.f;
+  const float E = 0x1p-9f * sumax * cmax + 0x1p-22f * (sumax + cmax);
   // 3. a lower bound of the k-th largest approximate score (its 16-bit key
   // bin: within 2^-7 of it), and the candidates within 2E of that bound
   uint32_t T, need;
   radix_threshold<kSelThreads>(keys, ncand, a.topk, sh, T, need, 2);
-  const float theta = key_score(T) - 2.0f * E;
+  const float theta = trusted ? key_score(T) - 2.0f * E : -INFINITY;
   uint32_t* poss = keys + a.nb;
   {
     const int per = (ncand + kSelThreads - 1) / kSelThreads;
     const int x0 = min(ncand, tid * per), x1 = min(ncand, x0 + per);
     uint32_t own = 0;
-    for (int x = x0; x < x1; ++x) own += key_score(keys[x]) >= theta;
+    for (int x = x0; x < x1; ++x) own += !trusted || key_score(keys[x]) >= theta;
     uint32_t at = static_cast<uint32_t>(block_exclusive_scan<kSelThreads>(own, sh));
     if (tid == kSelThreads - 1) rs.n_poss = static_cast<int>(at + own);
-    for (int x = x0; x < x1; ++x) {
-      if (key_score(keys[x]) >= theta) poss[at++] = static_cast<uint32_t>(x);
-      keys[x] = 0u;
-    }
+    for (int x = x0; x < x1; ++x)
+      if (!trusted || key_score(keys[x]) >= theta) poss[at++] = static_cast<uint32_t>(x);
   }
   __syncthreads();
   // 4. exact scores of those: four threads per candidate, a quarter of the
@@ -540,13 +567,24 @@ __global__ void __launch_bounds__(kSelThreads, 2) block_select_rowmax_kernel(con
       }
       best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 1));
       best = fmaxf(best, __shfl_xor_sync(0xffffffffu, best, 2));
-      if (sub == 0 && p < n_poss) keys[x] = order_key(best);
+      if (sub == 0 && p < n_poss) keys[p] = order_key(best);  // keys[p]: candidate poss[p]
     }
   }
   __syncthreads();
-  // 5. selection on the exact keys
-  const int n = select_from_keys(keys, ncand, t, a.topk, a.n_local, a.kmax, sh, out);
-  if (tid == 0) a.cnt[row] = n;
+  // 5. the k best of the re-scored candidates (the others cannot be): radix
+  // select and ordered compaction over their exact keys; poss is ascending,
+  // so the output is ascending and ties go to the lower block
+  {
+    const int n_poss = rs.n_poss;
+    uint32_t T2, need2;
+    radix_threshold<kSelThreads>(keys, n_poss, a.topk, sh, T2, need2);
+    ordered_select<kSelThreads>(keys, n_poss, T2, need2, sh,
+                                [&](int r, int p) { out[1 + r] = static_cast<int32_t>(poss[p]) + 1; });
+    if (tid == 0) out[0] = 0;
+    for (int m = tid; m < a.n_local; m += kSelThreads) out[1 + a.topk + m] = t - a.n_local + 1 + m;
+    for (int e = 1 + a.topk + a.n_local + tid; e < a.kmax; e += kSelThreads) out[e] = -1;
+    if (tid == 0) a.cnt[row] = 1 + a.topk + a.n_local;
+  }
 }
 
 }  // namespace

@@ -166,3 +166,25 @@ def test_rowmax_exact_ties_take_the_lower_blocks(rtp, cuda_device, tied):
             got = bufs["sel"][0, 0, t, :int(bufs["sel_cnt"][0, 0, t])].tolist()
             assert got == [0] + list(range(1, topk + 1)) + list(range(t - n_local + 1, t + 1)), (t, got)
     plan.close()
+
+
+def test_rowmax_centroids_beyond_fp16_range(rtp, cuda_device):
+    """Keys scaled so that centroid entries exceed fp16's range (2^15 and
+    more): the tensor-core approximation is not used and every candidate is
+    scored exactly; the selection still equals the oracle's."""
+    n, hq, hkv, block, topk, n_local = 4096, 8, 1, 128, 5, 2
+    d = inputs.small_prefill(n, hq, hkv, [S], seed=13)
+    k = (d["k"].float() * 1.0e5).to(torch.bfloat16)
+    q, k, proj = d["q"].to(cuda_device), k.to(cuda_device), d["proj"].to(cuda_device)
+    cfg = rtp.AttnConfig(1, n, hq, hkv, 256, block, topk, n_local)
+    plan = rtp.Plan(cfg, [S])
+    bufs = plan.buffers(cuda_device)
+    rtp.rtp_indexer_project(plan.handle, q, k, proj, bufs["centroids"], bufs["qbar"])
+    assert float(bufs["centroids"].abs().max()) >= 32768.0
+    rtp.rtp_block_select_rowmax(plan.handle, q, proj, bufs["centroids"], bufs["sel"], bufs["sel_cnt"])
+    torch.cuda.synchronize()
+    assert rtp.rtp_last_device_status() == rtp.RTP_OK
+    C = oracle.centroids(cpu(k[0, 0]), block, cpu(proj))
+    check_rowmax_rows(cpu(bufs["sel"][0, 0]).numpy(), cpu(bufs["sel_cnt"][0, 0]).numpy(), cpu(q[0]), cpu(proj), C,
+                      np.arange(n // block), block, topk, n_local)
+    plan.close()
