@@ -589,6 +589,25 @@ def time_layers(rtp, wid, steps, device):
     b.record(stream)
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / steps
+    # each kernel separately: one more pass with events between the calls
+    evs = []
+    for d, plan, bufs in layers:
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        sel = bufs["sel"] if plan.n_sparse else None
+        cnt = bufs["sel_cnt"] if plan.n_sparse else None
+        e[0].record(stream)
+        if plan.n_sparse:
+            rtp.rtp_indexer_project(plan.handle, d["q"], d["k"], d["proj"], bufs["centroids"], bufs["qbar"], stream)
+        e[1].record(stream)
+        if plan.n_sparse:
+            rtp.rtp_block_select(plan.handle, bufs["qbar"], bufs["centroids"], sel, cnt, stream)
+        e[2].record(stream)
+        rtp.rtp_hybrid_prefill(plan.handle, d["q"], d["k"], d["v"], sel, cnt, o, stream)
+        e[3].record(stream)
+        evs.append(e)
+    torch.cuda.synchronize()
+    kernels = {name: sum(e[i].elapsed_time(e[i + 1]) for e in evs) for i, name in
+               enumerate(("indexer", "select", "prefill"))}
     algo = sum(layer_flops(w, w.kinds[l])[0] for l in range(w.layers))
     execd = sum(layer_flops(w, w.kinds[l])[1] for l in range(w.layers))
     status = rtp.rtp_last_device_status(stream)
@@ -597,6 +616,7 @@ def time_layers(rtp, wid, steps, device):
     del layers
     torch.cuda.empty_cache()
     return {"workload": w.name, "layers": w.layers, "ms_per_pass": ms, "ms_per_layer": ms / w.layers,
+            "kernels_ms_per_pass": kernels,
             "tflops_effective": algo / (ms * 1e-3) / 1e12, "tflops_executed": execd / (ms * 1e-3) / 1e12,
             "status": rtp.status_str(status)}
 
