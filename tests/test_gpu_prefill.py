@@ -97,6 +97,19 @@ def test_batch_two_and_scale(rtp, cuda_device):
     plan.close()
 
 
+@pytest.mark.parametrize("scale", [0.5, 2.0])
+def test_growing_maximum(rtp, cuda_device, scale):
+    """Key norms ramp up along the sequence and the softmax scale is large, so
+    a row's maximum keeps growing, also between the two 64-key halves of a
+    tile: every reference move, O rescale and recomputed chunk of P is taken,
+    including the one that waits for the tile's first half to pass its P V."""
+    n = 1024
+    d = inputs.small_prefill(n, 6, 3, [2, 0, 1], seed=9)
+    ramp = torch.linspace(0.25, 2.0, n).view(1, 1, n, 1)
+    d["k"] = (d["k"].float() * ramp).to(torch.bfloat16)
+    full_check(rtp, d, 300, 128, 2, 1, cuda_device, scale=scale)
+
+
 def test_deterministic(rtp, cuda_device):
     w = inputs.workload(0)
     d = inputs.prefill_layer(w, 0, "cpu")
