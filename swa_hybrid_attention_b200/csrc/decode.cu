@@ -244,8 +244,18 @@ __global__ void __launch_bounds__(kDecSelThreads, 8) __cluster_dims__(kSelCluste
   float q[kRank];
   {
     const __nv_bfloat16* qg = a.q + (static_cast<size_t>(b) * a.n_q_heads + kvh * a.group) * kHeadDim + tid;
+    // The group's values of this dimension are loaded eight at a time, all
+    // in flight together (one memory round trip per eight heads rather than
+    // one per head), then added in head order.
     float qs = 0.f;
-    for (int h = 0; h < a.group; ++h) qs += __bfloat162float(qg[h * kHeadDim]);
+    for (int h0 = 0; h0 < a.group; h0 += 8) {
+      float qv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) qv[u] = h0 + u < a.group ? __bfloat162float(qg[(h0 + u) * kHeadDim]) : 0.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (h0 + u < a.group) qs += qv[u];
+    }
     const float prow[kRank] = {pr[0].x, pr[0].y, pr[0].z, pr[0].w, pr[1].x, pr[1].y, pr[1].z, pr[1].w,
                                pr[2].x, pr[2].y, pr[2].z, pr[2].w, pr[3].x, pr[3].y, pr[3].z, pr[3].w};
 #pragma unroll
