@@ -529,6 +529,11 @@ typedef struct {
  * centroid).  Then the members, offsets, chunk table and the K/V rows in
  * cluster order are written.  Deterministic (fixed-order sums, a stable
  * counting sort).  The K/V copy is skipped when cl->k_sorted is NULL.
+ * The distances are computed on tensor cores in fp16 where that provably
+ * decides a key's nearest centroid, and in fp32 otherwise; the result is
+ * the fp32 evaluation's for every key.  Setting the environment variable
+ * RTP_KMEANS_EXACT_ASSIGN=1 (read once per process) makes every key take
+ * the fp32 path (a diagnostic: the results are the same).
  *   cfg        batch, n_kv_heads, head_dim, block, rank used; seq = cache
  *              capacity as for rtp_sparse_decode (must be >= clu_end)
  *   kind_host  HOST [n_kv_heads]; RTP_HEAD_SPARSE heads are clustered

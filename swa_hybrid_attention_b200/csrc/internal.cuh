@@ -141,6 +141,8 @@ struct KmeansArgs {
   int32_t* chunk_start;         // [batch][n_kv_heads][max_chunks]: first row in the sorted K/V
   int32_t* chunk_len;
   int32_t* n_chunks;            // [batch][n_kv_heads]
+  int32_t* amb_list;            // workspace [batch][n_kv_heads][n]: keys the tensor-core pass left to the exact one
+  int32_t* amb_count;           // workspace [batch][n_kv_heads]
   uint8_t kind[kMaxDecodeKvHeads];
   int batch, n_kv_heads, cache_cap, block, clu_end, n, nc, max_chunks;
 };

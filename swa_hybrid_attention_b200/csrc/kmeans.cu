@@ -19,8 +19,15 @@
 // Kernels (retrieval heads only; CTAs of other heads leave at once):
 //   km_project    one thread per key: X = P^T k (fixed order over d)
 //   km_seed       the evenly spaced seeds
-//   km_assign     four keys per thread against every centroid, the centroids
-//                 in shared memory
+//   km_assign_mma the distances of 32 keys per warp to every centroid by
+//                 mma.sync (fp16 operands, fp32 accumulation, |mu|^2 as the
+//                 accumulator's start); a key whose two smallest distances
+//                 differ by more than twice the pass's proven error bound is
+//                 assigned there, every other key is queued
+//   km_rescore    the queued keys by the exact fp32 path (the same operations
+//                 in the same order as km_assign, which does every key when
+//                 RTP_KMEANS_EXACT_ASSIGN=1), so the assignment is the fp32
+//                 path's, key for key
 //   km_group      one CTA of 1024 threads per (sequence, head): cluster sizes,
 //                 offsets (scan), stable placement of the keys (one warp,
 //                 32 keys per step with match_any), and the new centroids
@@ -32,6 +39,9 @@
 //                 gathers member rows in place)
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdlib>
 
 #include "internal.cuh"
 
@@ -79,6 +89,7 @@ __global__ void __launch_bounds__(kKmThreads) km_project_kernel(const KmeansArgs
 __global__ void __launch_bounds__(kKmThreads) km_seed_kernel(const KmeansArgs a) {
   if (a.kind[blockIdx.y] != KIND_SPARSE) return;
   const size_t bk = head_index(a);
+  if (threadIdx.x == 0) a.amb_count[bk] = 0;
   for (int e = threadIdx.x; e < a.nc * kRank; e += kKmThreads) {
     const int c = e / kRank, d = e % kRank;
     const long j = (static_cast<long>(2 * c + 1) * a.n) / (2L * a.nc);
@@ -90,10 +101,17 @@ __global__ void __launch_bounds__(kKmThreads) km_seed_kernel(const KmeansArgs a)
 // serves this many keys (the loop is bound by shared-memory loads otherwise).
 constexpr int kAssignKeys = 4;
 
-__global__ void __launch_bounds__(kKmThreads) km_assign_kernel(const KmeansArgs a) {
+// The exact assignment: each key against every centroid in fp32 with the
+// fixed operation order (|mu|^2 by fma over the 16 dims, x.mu by fma over
+// the 16 dims, |mu|^2 - 2 x.mu, first minimum over ascending c).  Used for
+// every key (km_assign_kernel) or for the keys the tensor-core pass could
+// not decide (km_rescore_kernel); a key's result does not depend on which.
+// kList: the CTA's keys are entries [first, first + kKmThreads*kAssignKeys)
+// of the head's list of undecided keys (count entries); otherwise keys
+// first + ... directly.
+template <bool kList>
+__device__ __forceinline__ void exact_assign(const KmeansArgs& a, size_t bk, int first, int count) {
   extern __shared__ float4 mu4[];  // [nc][4] centroids, then [nc] squared norms
-  if (a.kind[blockIdx.y] != KIND_SPARSE) return;
-  const size_t bk = head_index(a);
   float* nrm = reinterpret_cast<float*>(mu4 + 4 * a.nc);
   const float4* src = reinterpret_cast<const float4*>(a.centroids + bk * a.nc * kRank);
   for (int e = threadIdx.x; e < 4 * a.nc; e += kKmThreads) mu4[e] = src[e];
@@ -111,12 +129,18 @@ __global__ void __launch_bounds__(kKmThreads) km_assign_kernel(const KmeansArgs 
     nrm[c] = s;
   }
   __syncthreads();
-  // keys j0 + u * kKmThreads, u < kAssignKeys (coalesced over the CTA)
-  const int j0 = blockIdx.x * kKmThreads * kAssignKeys + threadIdx.x;
+  // keys of entries e0 + u * kKmThreads, u < kAssignKeys (coalesced over the CTA)
+  const int e0 = first + threadIdx.x;
+  int jk[kAssignKeys];
+#pragma unroll
+  for (int u = 0; u < kAssignKeys; ++u) {
+    const int e = e0 + u * kKmThreads;
+    jk[u] = e < count ? (kList ? a.amb_list[bk * a.n + e] : e) : -1;
+  }
   float x[kAssignKeys][kRank];
 #pragma unroll
   for (int u = 0; u < kAssignKeys; ++u) {
-    const int j = min(j0 + u * kKmThreads, a.n - 1);
+    const int j = min(max(jk[u], 0), a.n - 1);
     const float4* xr = reinterpret_cast<const float4*>(a.X + (bk * a.n + j) * kRank);
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
@@ -153,8 +177,275 @@ __global__ void __launch_bounds__(kKmThreads) km_assign_kernel(const KmeansArgs 
   }
 #pragma unroll
   for (int u = 0; u < kAssignKeys; ++u) {
-    const int j = j0 + u * kKmThreads;
-    if (j < a.n) a.assign[bk * a.n + j] = bc[u];
+    const int j = jk[u];
+    if (j >= 0 && j < a.n) a.assign[bk * a.n + j] = bc[u];
+  }
+}
+
+__global__ void __launch_bounds__(kKmThreads) km_assign_kernel(const KmeansArgs a) {
+  if (a.kind[blockIdx.y] != KIND_SPARSE) return;
+  exact_assign<false>(a, head_index(a), blockIdx.x * kKmThreads * kAssignKeys, a.n);
+}
+
+// gridDim.x CTAs per head walk the head's list in chunks of
+// kKmThreads * kAssignKeys keys (the centroids are loaded once per chunk).
+__global__ void __launch_bounds__(kKmThreads) km_rescore_kernel(const KmeansArgs a) {
+  if (a.kind[blockIdx.y] != KIND_SPARSE) return;
+  const size_t bk = head_index(a);
+  const int count = min(a.amb_count[bk], a.n);
+  for (int first = blockIdx.x * kKmThreads * kAssignKeys; first < count;
+       first += gridDim.x * kKmThreads * kAssignKeys) {  // (uniform over the CTA)
+    exact_assign<true>(a, bk, first, count);
+    __syncthreads();  // the shared centroids are loaded again for the next chunk
+  }
+}
+
+// ------------------------------------------------ tensor-core assignment
+// The distances of 16 keys to 8 centroids are one mma.sync m16n8k16: A = the
+// keys' projections in fp16, B = -2 mu in fp16, C = |mu|^2 (fp32, the exact
+// path's value), so D = |mu|^2 - 2 x~.mu~.  Each thread keeps, per key row,
+// the smallest D, its centroid and the second smallest D.  D differs from the
+// exact path's fp32 distance by at most
+//   E = 1.125 * 2^-9 |x| M + 2^-16 M^2 + 2^-20 (|x| + M),   M = max_c |mu_c|
+// (fp16 rounding of x and mu: 2^-11 relative each, products exact; fp32
+// accumulation of 17 terms; the exact path's own fp32 rounding; with margin).
+// A key whose second smallest D exceeds its smallest by more than 2E has the
+// exact path's nearest centroid, unique; every other key (and any key with
+// non-finite values, |x| >= 30000 or M > 8192, outside fp16's safe range) is
+// appended to the head's undecided list, which km_rescore_kernel assigns by
+// the exact path.  The result is the exact path's, key for key.
+constexpr int kMmaWarps = 8;
+constexpr int kMmaThreads = 32 * kMmaWarps;
+constexpr int kMmaGroups = 4;                              // 32-key groups per warp
+constexpr int kMmaKeysPerCta = kMmaThreads * kMmaGroups;  // 1024
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1, float c0,
+                                        float c1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%11,%12,%13};"
+      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(c0), "f"(c1), "f"(c0), "f"(c1));
+}
+
+__device__ __forceinline__ void ldsm_x4_b16(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t half2_bits(float lo, float hi) {
+  const __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Running smallest distance m1 of one key row, a lower bound L of its second
+// smallest, and the 16-centroid tile pair where m1 was found, updated with
+// the four distances this thread sees in pair p: (d0, d1) from the first
+// 8-centroid tile, (e0, e1) from the second.  L stays <= the true second
+// smallest: the group's two smallest are exact, and the second smallest of
+// the union is min(max(m1, g1), min(L, g2)).
+__device__ __forceinline__ void top2_group(float& m1, float& L, int& pb, float d0, float d1, float e0, float e1,
+                                           int p) {
+  const float a0 = fminf(d0, d1), b0 = fmaxf(d0, d1), a1 = fminf(e0, e1), b1 = fmaxf(e0, e1);
+  const float g1 = fminf(a0, a1), g2 = fminf(fmaxf(a0, a1), fminf(b0, b1));
+  L = fminf(fmaxf(m1, g1), fminf(L, g2));
+  if (g1 < m1) pb = p;
+  m1 = fminf(m1, g1);
+}
+
+// Merge with the quad neighbour at lane ^ mask (the same rows, other
+// centroids); owner = the quad lane whose centroids hold m1.
+__device__ __forceinline__ void top2_merge(float& m1, float& L, int& pb, int& owner, int mask) {
+  const float om1 = __shfl_xor_sync(0xffffffffu, m1, mask);
+  const float oL = __shfl_xor_sync(0xffffffffu, L, mask);
+  const int opb = __shfl_xor_sync(0xffffffffu, pb, mask);
+  const int oown = __shfl_xor_sync(0xffffffffu, owner, mask);
+  L = fminf(fmaxf(m1, om1), fminf(L, oL));
+  if (om1 < m1) {
+    m1 = om1;
+    pb = opb;
+    owner = oown;
+  }
+}
+
+// The exact path's distance of key x to centroid c (the same fp32 operations
+// in the same order as exact_assign).
+__device__ __forceinline__ float exact_dist(const float (&x)[kRank], const float* mu, float nc2) {
+  float dot = 0.f;
+#pragma unroll
+  for (int d = 0; d < kRank; ++d) dot = fmaf(x[d], mu[d], dot);
+  return fmaf(-2.f, dot, nc2);
+}
+
+__global__ void __launch_bounds__(kMmaThreads) km_assign_mma_kernel(const KmeansArgs a) {
+  // dynamic: -2 mu as fp16 [ncp][16] (32 bytes per centroid, its two 16-byte
+  // halves swapped when bit 2 of c is set, so that the eight rows of an
+  // ldmatrix tile fall in distinct bank groups), then |mu|^2 [ncp] (fp32,
+  // +inf for the padding centroids c >= nc)
+  extern __shared__ __align__(16) uint8_t km_smem[];
+  __shared__ float wmax[kMmaWarps];
+  if (a.kind[blockIdx.y] != KIND_SPARSE) return;
+  const size_t bk = head_index(a);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int npairs = (a.nc + 15) / 16, ncp = 16 * npairs;
+  uint8_t* mu16 = km_smem;
+  float* nrm = reinterpret_cast<float*>(km_smem + static_cast<size_t>(ncp) * 32);
+  const float* src = a.centroids + bk * a.nc * kRank;
+  float mymax = 0.f;
+  for (int c = tid; c < ncp; c += kMmaThreads) {
+    float v[kRank];
+    if (c < a.nc) {
+      const float4* c4 = reinterpret_cast<const float4*>(src + static_cast<size_t>(c) * kRank);
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float4 m = c4[w];
+        v[4 * w] = m.x;
+        v[4 * w + 1] = m.y;
+        v[4 * w + 2] = m.z;
+        v[4 * w + 3] = m.w;
+      }
+    } else {
+#pragma unroll
+      for (int d = 0; d < kRank; ++d) v[d] = 0.f;
+    }
+    float sq = 0.f;  // the exact path's |mu|^2: fma over the dims in order
+#pragma unroll
+    for (int d = 0; d < kRank; ++d) sq = fmaf(v[d], v[d], sq);
+    nrm[c] = c < a.nc ? sq : INFINITY;
+    if (c < a.nc) mymax = fmaxf(mymax, sq);  // (a NaN norm is caught below: M is then NaN)
+    if (c < a.nc && !(sq <= INFINITY)) mymax = NAN;
+    uint4* row = reinterpret_cast<uint4*>(mu16 + static_cast<size_t>(c) * 32);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const float* q = v + 8 * h;
+      row[h ^ ((c >> 2) & 1)] = make_uint4(half2_bits(-2.f * q[0], -2.f * q[1]), half2_bits(-2.f * q[2], -2.f * q[3]),
+                                           half2_bits(-2.f * q[4], -2.f * q[5]), half2_bits(-2.f * q[6], -2.f * q[7]));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float o = __shfl_xor_sync(0xffffffffu, mymax, off);
+    mymax = (mymax != mymax || o != o) ? NAN : fmaxf(mymax, o);
+  }
+  if (lane == 0) wmax[warp] = mymax;
+  __syncthreads();
+  float M2 = 0.f;
+#pragma unroll
+  for (int w = 0; w < kMmaWarps; ++w) M2 = (M2 != M2 || wmax[w] != wmax[w]) ? NAN : fmaxf(M2, wmax[w]);
+  const float M = sqrtf(M2);
+  const bool m_ok = M <= 8192.f;  // false for NaN
+
+  const int g = lane >> 2, q4 = lane & 3;
+  const uint32_t mu_base = static_cast<uint32_t>(__cvta_generic_to_shared(mu16));
+  // ldmatrix row address of this lane: matrix lane/8 = (centroid half-tile
+  // lane/16, dim half (lane/8)&1), row lane%8
+  const int lrow = 8 * (lane >> 4) + (lane & 7), lhalf = (lane >> 3) & 1;
+  const float* Xh = a.X + bk * a.n * kRank;
+  for (int grp = 0; grp < kMmaGroups; ++grp) {
+    const int base = blockIdx.x * kMmaKeysPerCta + (grp * kMmaWarps + warp) * 32;
+    if (base >= a.n) break;  // (uniform over the warp)
+    // A fragments: rows base + 16 mt + g (+8), dims 2q4, 2q4+1 and 2q4+8, 2q4+9
+    uint32_t af[2][4];
+    float xsq[2][2];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int j = min(base + 16 * mt + g + 8 * rr, a.n - 1);
+        const float* xr = Xh + static_cast<size_t>(j) * kRank;
+        const float2 lo = *reinterpret_cast<const float2*>(xr + 2 * q4);
+        const float2 hi = *reinterpret_cast<const float2*>(xr + 2 * q4 + 8);
+        af[mt][rr] = half2_bits(lo.x, lo.y);
+        af[mt][2 + rr] = half2_bits(hi.x, hi.y);
+        xsq[mt][rr] = fmaf(lo.x, lo.x, fmaf(lo.y, lo.y, fmaf(hi.x, hi.x, hi.y * hi.y)));
+      }
+    float m1[2][2], L[2][2];
+    int pb[2][2];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        m1[mt][rr] = INFINITY;
+        L[mt][rr] = INFINITY;
+        pb[mt][rr] = 0;
+      }
+    for (int p = 0; p < npairs; ++p) {
+      const int n0 = 16 * p;
+      const int cr = n0 + lrow;
+      uint32_t b00, b01, b10, b11;  // [centroid tile][dim half]
+      ldsm_x4_b16(mu_base + cr * 32 + ((lhalf ^ ((cr >> 2) & 1)) << 4), b00, b01, b10, b11);
+      const float2 c0 = *reinterpret_cast<const float2*>(nrm + n0 + 2 * q4);
+      const float2 c1 = *reinterpret_cast<const float2*>(nrm + n0 + 8 + 2 * q4);
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        float d0[4], d1[4];
+        mma_f16(d0, af[mt], b00, b01, c0.x, c0.y);
+        mma_f16(d1, af[mt], b10, b11, c1.x, c1.y);
+        top2_group(m1[mt][0], L[mt][0], pb[mt][0], d0[0], d0[1], d1[0], d1[1], p);
+        top2_group(m1[mt][1], L[mt][1], pb[mt][1], d0[2], d0[3], d1[2], d1[3], p);
+      }
+    }
+    // the four threads of a quad saw different centroids of the same rows
+    int own[2][2];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        own[mt][rr] = q4;
+        top2_merge(m1[mt][rr], L[mt][rr], pb[mt][rr], own[mt][rr], 1);
+        top2_merge(m1[mt][rr], L[mt][rr], pb[mt][rr], own[mt][rr], 2);
+        xsq[mt][rr] += __shfl_xor_sync(0xffffffffu, xsq[mt][rr], 1);
+        xsq[mt][rr] += __shfl_xor_sync(0xffffffffu, xsq[mt][rr], 2);
+      }
+    // lane (g, q4) decides row 16 (q4 >> 1) + g + 8 (q4 & 1) of the group
+    const int mt = q4 >> 1, rr = q4 & 1;
+    const float bm1 = mt ? (rr ? m1[1][1] : m1[1][0]) : (rr ? m1[0][1] : m1[0][0]);
+    const float bm2 = mt ? (rr ? L[1][1] : L[1][0]) : (rr ? L[0][1] : L[0][0]);
+    const int bpb = mt ? (rr ? pb[1][1] : pb[1][0]) : (rr ? pb[0][1] : pb[0][0]);
+    const int bown = mt ? (rr ? own[1][1] : own[1][0]) : (rr ? own[0][1] : own[0][0]);
+    const float bx2 = mt ? (rr ? xsq[1][1] : xsq[1][0]) : (rr ? xsq[0][1] : xsq[0][0]);
+    const int j = base + 16 * mt + g + 8 * rr;
+    const float xn = sqrtf(bx2);
+    const float E = 0x1.2p-9f * xn * M + 0x1p-16f * M * M + 0x1p-20f * (xn + M);
+    const bool sure = m_ok && xn < 30000.f && (bm2 - bm1) > 2.f * E;  // false for any NaN
+    const bool valid = j < a.n;
+    if (valid && sure) {
+      // The nearest centroid is unique and is one of the four that the
+      // owning lane saw in pair bpb (the one that gave m1): the smallest of
+      // their exact distances (ascending order) is it.
+      float xr[kRank];
+      const float4* x4 = reinterpret_cast<const float4*>(Xh + static_cast<size_t>(j) * kRank);
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float4 v = x4[w];
+        xr[4 * w] = v.x;
+        xr[4 * w + 1] = v.y;
+        xr[4 * w + 2] = v.z;
+        xr[4 * w + 3] = v.w;
+      }
+      float best = INFINITY;
+      int bc = 16 * bpb + 2 * bown;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int c = 16 * bpb + 8 * (k >> 1) + 2 * bown + (k & 1);
+        if (c < a.nc) {
+          const float dist = exact_dist(xr, src + static_cast<size_t>(c) * kRank, nrm[c]);
+          if (dist < best) {
+            best = dist;
+            bc = c;
+          }
+        }
+      }
+      a.assign[bk * a.n + j] = bc;
+    }
+    const uint32_t undecided = __ballot_sync(0xffffffffu, valid && !sure);
+    if (undecided) {
+      int slot0 = 0;
+      if (lane == 0) slot0 = atomicAdd(a.amb_count + bk, __popc(undecided));
+      slot0 = __shfl_sync(0xffffffffu, slot0, 0);
+      if (valid && !sure) a.amb_list[bk * a.n + slot0 + __popc(undecided & ((1u << lane) - 1u))] = j;
+    }
   }
 }
 
@@ -202,6 +493,7 @@ __global__ void __launch_bounds__(kGroupThreads) km_group_kernel(const KmeansArg
   const size_t bk = head_index(a);
   const int tid = threadIdx.x, lane = tid & 31;
   const int32_t* asg = a.assign + bk * a.n;
+  if (tid == 0) a.amb_count[bk] = 0;  // the undecided list of the next round starts empty
   for (int c = tid; c < a.nc; c += kGroupThreads) {
     cnt[c] = 0;
     running[c] = 0;
@@ -312,13 +604,32 @@ cudaError_t launch_kmeans(const KmeansArgs& a, int iters, cudaStream_t stream) {
   km_project_kernel<<<per_key, kKmThreads, 0, stream>>>(a);
   km_seed_kernel<<<per_head, kKmThreads, 0, stream>>>(a);
   const size_t smem = static_cast<size_t>(a.nc) * (kRank + 1) * sizeof(float);
-  if (smem > 48 * 1024) {
-    cudaError_t e =
-        cudaFuncSetAttribute(km_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-  }
+  const size_t ncp = 16 * static_cast<size_t>((a.nc + 15) / 16);
+  const size_t smem_mma = ncp * (32 + sizeof(float));
+  // RTP_KMEANS_EXACT_ASSIGN=1 (diagnostic): every key by the exact fp32 path,
+  // which the tensor-core pass must reproduce key for key.
+  static const bool exact_only = [] {
+    const char* e = std::getenv("RTP_KMEANS_EXACT_ASSIGN");
+    return e && e[0] == '1';
+  }();
+  cudaError_t e = cudaFuncSetAttribute(km_assign_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(km_rescore_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(km_assign_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem_mma));
+  if (e != cudaSuccess) return e;
+  const dim3 per_mma((a.n + kMmaKeysPerCta - 1) / kMmaKeysPerCta, a.n_kv_heads, a.batch);
+  // one CTA per chunk of a full list; those beyond the list's end leave at once
+  const dim3 per_rescore = per_keys;
   for (int it = 0; it < iters; ++it) {
-    km_assign_kernel<<<per_keys, kKmThreads, smem, stream>>>(a);
+    if (exact_only) {
+      km_assign_kernel<<<per_keys, kKmThreads, smem, stream>>>(a);
+    } else {
+      km_assign_mma_kernel<<<per_mma, kMmaThreads, smem_mma, stream>>>(a);
+      km_rescore_kernel<<<per_rescore, kKmThreads, smem, stream>>>(a);
+    }
     km_group_kernel<<<per_head, kGroupThreads, 0, stream>>>(a);
   }
   km_chunks_kernel<<<per_head, kGroupThreads, 0, stream>>>(a);

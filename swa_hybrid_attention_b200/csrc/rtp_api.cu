@@ -925,7 +925,7 @@ size_t rtp_cache_cluster_workspace_bytes(const rtp_attn_cfg* cfg, int clu_end) {
   const size_t bk = static_cast<size_t>(cfg->batch) * cfg->n_kv_heads;
   const size_t n = static_cast<size_t>(clu_end - cfg->block);
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-  return up(bk * n * kRank * sizeof(float)) + up(bk * n * sizeof(int32_t));
+  return up(bk * n * kRank * sizeof(float)) + 2 * up(bk * n * sizeof(int32_t)) + up(bk * sizeof(int32_t));
 }
 
 rtp_status rtp_cache_cluster(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int iters, const void* kcache,
@@ -954,8 +954,15 @@ rtp_status rtp_cache_cluster(const rtp_attn_cfg* cfg, const uint8_t* kind_host, 
   a.max_chunks = a.n / 128 + a.nc;
   const size_t bk = static_cast<size_t>(cfg->batch) * cfg->n_kv_heads;
   a.X = static_cast<float*>(workspace);
-  a.assign = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) +
-                                        (bk * a.n * kRank * sizeof(float) + 255) / 256 * 256);
+  {
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    char* w = static_cast<char*>(workspace) + up(bk * a.n * kRank * sizeof(float));
+    a.assign = reinterpret_cast<int32_t*>(w);
+    w += up(bk * a.n * sizeof(int32_t));
+    a.amb_list = reinterpret_cast<int32_t*>(w);
+    w += up(bk * a.n * sizeof(int32_t));
+    a.amb_count = reinterpret_cast<int32_t*>(w);
+  }
   a.centroids = cl->centroids;
   a.members = cl->members;
   a.offsets = cl->offsets;

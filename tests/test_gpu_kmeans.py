@@ -107,6 +107,32 @@ def test_kmeans_valid_and_agrees_with_oracle(rtp, cuda_device, block, nc, iters)
         assert torch.equal(getattr(cl, name), getattr(cl2, name)), name
 
 
+def test_tensor_core_assignment_equals_exact_path(rtp, cuda_device, tmp_path):
+    """The assignment pass on tensor cores (fp16 distances, keys it cannot
+    decide within its error bound re-scored in fp32) gives, key for key, the
+    exact fp32 path's nearest centroid: whole clusterings are bit-identical to
+    a run with RTP_KMEANS_EXACT_ASSIGN=1 (every key by the fp32 path), also
+    with exact ties (duplicated keys) and values beyond fp16's range."""
+    import os
+    import subprocess
+    import sys
+
+    import kmeans_cases
+
+    here = kmeans_cases.run_all(rtp, cuda_device)
+    out = tmp_path / "exact.pt"
+    env = dict(os.environ, RTP_KMEANS_EXACT_ASSIGN="1")
+    r = subprocess.run([sys.executable, kmeans_cases.__file__, str(out)], env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    exact = torch.load(out)
+    for name, fields in here.items():
+        assert fields["status"] == rtp.RTP_OK and exact[name]["status"] == rtp.RTP_OK, name
+        for f, t in fields.items():
+            if f != "status":
+                assert torch.equal(t, exact[name][f]), (name, f)
+
+
 def test_kmeans_recovers_planted_blobs_exactly(rtp, cuda_device):
     block, nc, per = 128, 16, 96
     n = nc * per
