@@ -143,10 +143,13 @@ struct KmeansArgs {
   int32_t* n_chunks;            // [batch][n_kv_heads]
   int32_t* amb_list;            // workspace [batch][n_kv_heads][n]: keys the tensor-core pass left to the exact one
   int32_t* amb_count;           // workspace [batch][n_kv_heads]
+  int32_t* seg;                 // workspace [batch][n_kv_heads][n_seg][nc]: per key segment, counts then starts
+  int n_seg;                    // key segments of kKmSegKeys keys
   uint8_t kind[kMaxDecodeKvHeads];
   int batch, n_kv_heads, cache_cap, block, clu_end, n, nc, max_chunks;
 };
 constexpr int kMaxClusters = 2048;
+constexpr int kKmSegKeys = 4096;  // keys per segment of the k-means grouping
 
 // Launchers (return the launch error, never synchronise).
 cudaError_t launch_prefill(const PrefillArgs& a, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,

@@ -28,10 +28,11 @@
 //                 in the same order as km_assign, which does every key when
 //                 RTP_KMEANS_EXACT_ASSIGN=1), so the assignment is the fp32
 //                 path's, key for key
-//   km_group      one CTA of 1024 threads per (sequence, head): cluster sizes,
-//                 offsets (scan), stable placement of the keys (one warp,
-//                 32 keys per step with match_any), and the new centroids
-//                 (each summed over its keys in position order)
+//   km_hist / km_scan / km_place / km_means  the keys grouped by cluster:
+//                 per-segment counts, offsets and segment starts, stable
+//                 placement (a warp per segment, 32 keys per step with
+//                 match_any), and the new centroids (each summed over its
+//                 keys in position order)
 //   km_chunks     each cluster's keys cut into chunks of <= 128 (the units
 //                 the decode step selects), with the cluster's centroid
 //   km_permute    K and V rows copied into cluster order (one warp per row;
@@ -486,72 +487,122 @@ __device__ __forceinline__ void scan_counts(const int* cnt, int* off, int nc, in
   if (c0 + 1 < nc) off[c0 + 1] = base + v0;
 }
 
-__global__ void __launch_bounds__(kGroupThreads) km_group_kernel(const KmeansArgs a) {
-  __shared__ int cnt[kMaxClusters], off[kMaxClusters], running[kMaxClusters];
+// Grouping of the keys by cluster, in four steps over many CTAs; the result
+// is that of one walk over the keys in order: members of a cluster ascend,
+// and each centroid is the sum of its members' projections in member order,
+// divided by their number (an empty cluster keeps its centroid).
+//   km_hist   per segment of kKmSegKeys keys: the count of each cluster
+//   km_scan   per (sequence, head): the offsets of the clusters and, for each
+//             segment, where its keys of each cluster start
+//   km_place  one warp per segment: its keys to their places, in key order
+//   km_means  one half-warp per cluster: lane d sums dimension d
+constexpr int kHistThreads = 256;
+constexpr int kPlaceWarps = 4;
+constexpr int kMeansThreads = 256;
+
+__global__ void __launch_bounds__(kHistThreads) km_hist_kernel(const KmeansArgs a) {
+  __shared__ int cnt[kMaxClusters];
+  if (a.kind[blockIdx.y] != KIND_SPARSE) return;
+  const size_t bk = head_index(a);
+  const int tid = threadIdx.x, sg = blockIdx.x;
+  const int32_t* asg = a.assign + bk * a.n;
+  for (int c = tid; c < a.nc; c += kHistThreads) cnt[c] = 0;
+  __syncthreads();
+  const int j1 = min(a.n, (sg + 1) * kKmSegKeys);
+  for (int j = sg * kKmSegKeys + tid; j < j1; j += kHistThreads) atomicAdd(&cnt[asg[j]], 1);
+  __syncthreads();
+  int32_t* seg = a.seg + (bk * a.n_seg + sg) * a.nc;
+  for (int c = tid; c < a.nc; c += kHistThreads) seg[c] = cnt[c];
+}
+
+__global__ void __launch_bounds__(kGroupThreads) km_scan_kernel(const KmeansArgs a) {
+  __shared__ int cnt[kMaxClusters], off[kMaxClusters];
   __shared__ int warp_tot[32];
   if (a.kind[blockIdx.y] != KIND_SPARSE) return;
   const size_t bk = head_index(a);
-  const int tid = threadIdx.x, lane = tid & 31;
-  const int32_t* asg = a.assign + bk * a.n;
+  const int tid = threadIdx.x;
   if (tid == 0) a.amb_count[bk] = 0;  // the undecided list of the next round starts empty
+  int32_t* seg = a.seg + bk * a.n_seg * a.nc;
+  // per cluster: each segment's start relative to the cluster, and its size
   for (int c = tid; c < a.nc; c += kGroupThreads) {
-    cnt[c] = 0;
-    running[c] = 0;
+    int run = 0;
+#pragma unroll 4
+    for (int sg = 0; sg < a.n_seg; ++sg) {
+      const int v = seg[static_cast<size_t>(sg) * a.nc + c];
+      seg[static_cast<size_t>(sg) * a.nc + c] = run;
+      run += v;
+    }
+    cnt[c] = run;
   }
-  __syncthreads();
-  for (int j = tid; j < a.n; j += kGroupThreads) atomicAdd(&cnt[asg[j]], 1);
   __syncthreads();
   scan_counts(cnt, off, a.nc, warp_tot);
   __syncthreads();
   int32_t* offs = a.offsets + bk * (a.nc + 1);
-  for (int c = tid; c < a.nc; c += kGroupThreads) offs[c] = off[c];
-  if (tid == 0) offs[a.nc] = a.n;
-  // stable placement: one warp walks the keys in order, 32 at a time
-  int32_t* mem = a.members + bk * a.n;
-  if (tid < 32) {
-    const uint32_t lt = (1u << lane) - 1u;
-    for (int j0 = 0; j0 < a.n; j0 += 32 * 8) {
-      int cj[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int j = j0 + 32 * u + lane;
-        cj[u] = j < a.n ? asg[j] : -1;
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int c = cj[u];
-        const uint32_t peers = __match_any_sync(0xffffffffu, c);
-        if (c >= 0) mem[off[c] + running[c] + __popc(peers & lt)] = a.block + j0 + 32 * u + lane;
-        __syncwarp();
-        if (c >= 0 && lane == __ffs(peers) - 1) running[c] += __popc(peers);
-        __syncwarp();
-      }
-    }
-  }
-  __syncthreads();
-  // new centroids: the mean of each cluster's keys, summed in position order
   for (int c = tid; c < a.nc; c += kGroupThreads) {
-    const int size = cnt[c];
-    if (size == 0) continue;
-    float s[kRank];
-#pragma unroll
-    for (int d = 0; d < kRank; ++d) s[d] = 0.f;
-    for (int e = 0; e < size; ++e) {
-      const int j = mem[off[c] + e] - a.block;
-      const float4* xr = reinterpret_cast<const float4*>(a.X + (bk * a.n + j) * kRank);
-#pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float4 v = xr[w];
-        s[4 * w] += v.x;
-        s[4 * w + 1] += v.y;
-        s[4 * w + 2] += v.z;
-        s[4 * w + 3] += v.w;
-      }
-    }
-    float* mu = a.centroids + (bk * a.nc + c) * kRank;
-#pragma unroll
-    for (int d = 0; d < kRank; ++d) mu[d] = s[d] / static_cast<float>(size);
+    offs[c] = off[c];
+#pragma unroll 4
+    for (int sg = 0; sg < a.n_seg; ++sg) seg[static_cast<size_t>(sg) * a.nc + c] += off[c];
   }
+  if (tid == 0) offs[a.nc] = a.n;
+}
+
+__global__ void __launch_bounds__(32 * kPlaceWarps) km_place_kernel(const KmeansArgs a) {
+  __shared__ int running[kPlaceWarps][kMaxClusters];
+  if (a.kind[blockIdx.y] != KIND_SPARSE) return;
+  const size_t bk = head_index(a);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int sg = blockIdx.x * kPlaceWarps + w;
+  if (sg >= a.n_seg) return;  // (warp-uniform; the warps share no barrier)
+  const int32_t* start = a.seg + (bk * a.n_seg + sg) * a.nc;
+  for (int c = lane; c < a.nc; c += 32) running[w][c] = start[c];
+  __syncwarp();
+  const int32_t* asg = a.assign + bk * a.n;
+  int32_t* mem = a.members + bk * a.n;
+  const uint32_t lt = (1u << lane) - 1u;
+  const int j1 = min(a.n, (sg + 1) * kKmSegKeys);
+  for (int j0 = sg * kKmSegKeys; j0 < j1; j0 += 32 * 8) {
+    int cj[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + 32 * u + lane;
+      cj[u] = j < j1 ? asg[j] : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int c = cj[u];
+      const uint32_t peers = __match_any_sync(0xffffffffu, c);
+      if (c >= 0) mem[running[w][c] + __popc(peers & lt)] = a.block + j0 + 32 * u + lane;
+      __syncwarp();
+      if (c >= 0 && lane == __ffs(peers) - 1) running[w][c] += __popc(peers);
+      __syncwarp();
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kMeansThreads) km_means_kernel(const KmeansArgs a) {
+  if (a.kind[blockIdx.y] != KIND_SPARSE) return;
+  const size_t bk = head_index(a);
+  const int c = (blockIdx.x * kMeansThreads + threadIdx.x) >> 4, d = threadIdx.x & 15;
+  if (c >= a.nc) return;  // (no barriers or shuffles below)
+  const int32_t* offs = a.offsets + bk * (a.nc + 1);
+  const int o0 = offs[c], size = offs[c + 1] - o0;
+  if (size == 0) return;
+  const int32_t* mem = a.members + bk * a.n + o0;
+  const float* Xd = a.X + bk * a.n * kRank + d;
+  float s = 0.f;
+  int e = 0;
+  for (; e + 4 <= size; e += 4) {  // four members' loads in flight, added in order
+    int jj[4];
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) jj[u] = mem[e + u] - a.block;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = Xd[static_cast<size_t>(jj[u]) * kRank];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) s += v[u];
+  }
+  for (; e < size; ++e) s += Xd[static_cast<size_t>(mem[e] - a.block) * kRank];
+  a.centroids[(bk * a.nc + c) * kRank + d] = s / static_cast<float>(size);
 }
 
 __global__ void __launch_bounds__(kGroupThreads) km_chunks_kernel(const KmeansArgs a) {
@@ -621,6 +672,9 @@ cudaError_t launch_kmeans(const KmeansArgs& a, int iters, cudaStream_t stream) {
                              static_cast<int>(smem_mma));
   if (e != cudaSuccess) return e;
   const dim3 per_mma((a.n + kMmaKeysPerCta - 1) / kMmaKeysPerCta, a.n_kv_heads, a.batch);
+  const dim3 per_seg(a.n_seg, a.n_kv_heads, a.batch);
+  const dim3 per_place((a.n_seg + kPlaceWarps - 1) / kPlaceWarps, a.n_kv_heads, a.batch);
+  const dim3 per_means((a.nc * 16 + kMeansThreads - 1) / kMeansThreads, a.n_kv_heads, a.batch);
   // one CTA per chunk of a full list; those beyond the list's end leave at once
   const dim3 per_rescore = per_keys;
   for (int it = 0; it < iters; ++it) {
@@ -630,7 +684,10 @@ cudaError_t launch_kmeans(const KmeansArgs& a, int iters, cudaStream_t stream) {
       km_assign_mma_kernel<<<per_mma, kMmaThreads, smem_mma, stream>>>(a);
       km_rescore_kernel<<<per_rescore, kKmThreads, smem, stream>>>(a);
     }
-    km_group_kernel<<<per_head, kGroupThreads, 0, stream>>>(a);
+    km_hist_kernel<<<per_seg, kHistThreads, 0, stream>>>(a);
+    km_scan_kernel<<<per_head, kGroupThreads, 0, stream>>>(a);
+    km_place_kernel<<<per_place, 32 * kPlaceWarps, 0, stream>>>(a);
+    km_means_kernel<<<per_means, kMeansThreads, 0, stream>>>(a);
   }
   km_chunks_kernel<<<per_head, kGroupThreads, 0, stream>>>(a);
   if (a.k_sorted) {  // no cluster-ordered copy when the decode reads member rows in place

@@ -925,7 +925,9 @@ size_t rtp_cache_cluster_workspace_bytes(const rtp_attn_cfg* cfg, int clu_end) {
   const size_t bk = static_cast<size_t>(cfg->batch) * cfg->n_kv_heads;
   const size_t n = static_cast<size_t>(clu_end - cfg->block);
   auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-  return up(bk * n * kRank * sizeof(float)) + 2 * up(bk * n * sizeof(int32_t)) + up(bk * sizeof(int32_t));
+  const size_t n_seg = (n + kKmSegKeys - 1) / kKmSegKeys;
+  return up(bk * n * kRank * sizeof(float)) + 2 * up(bk * n * sizeof(int32_t)) + up(bk * sizeof(int32_t)) +
+         up(bk * n_seg * kMaxClusters * sizeof(int32_t));
 }
 
 rtp_status rtp_cache_cluster(const rtp_attn_cfg* cfg, const uint8_t* kind_host, int iters, const void* kcache,
@@ -962,6 +964,9 @@ rtp_status rtp_cache_cluster(const rtp_attn_cfg* cfg, const uint8_t* kind_host, 
     a.amb_list = reinterpret_cast<int32_t*>(w);
     w += up(bk * a.n * sizeof(int32_t));
     a.amb_count = reinterpret_cast<int32_t*>(w);
+    w += up(bk * sizeof(int32_t));
+    a.seg = reinterpret_cast<int32_t*>(w);
+    a.n_seg = (a.n + kKmSegKeys - 1) / kKmSegKeys;
   }
   a.centroids = cl->centroids;
   a.members = cl->members;

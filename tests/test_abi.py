@@ -162,8 +162,10 @@ def test_cluster_calls_validate_before_launch(rtp):
     kinds = rtp._kinds([2, 0])
     ws = rtp.rtp_cache_cluster_workspace_bytes(cfg, 2048)
     up = lambda x: (x + 255) // 256 * 256  # noqa: E731
-    # projected keys, assignment, undecided-key list, one counter per head
-    assert ws == up(2 * 2 * 1920 * 16 * 4) + 2 * up(2 * 2 * 1920 * 4) + up(2 * 2 * 4)
+    # projected keys, assignment, undecided-key list, one counter per head,
+    # per-segment cluster counts (segments of 4096 keys, up to 2048 clusters)
+    assert ws == (up(2 * 2 * 1920 * 16 * 4) + 2 * up(2 * 2 * 1920 * 4) + up(2 * 2 * 4) +
+                  up(2 * 2 * 1 * 2048 * 4))
     for bad in (dict(clu_end=128), dict(clu_end=2000), dict(clu_end=8192), dict(n_clusters=0),
                 dict(n_clusters=4096)):
         x = cl(**bad)
