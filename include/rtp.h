@@ -338,7 +338,10 @@ rtp_status rtp_hybrid_prefill_items(const rtp_plan* plan, const void* q, const v
 /* ------------------------------------------------------------------------
  * rtp_hybrid_prefill_host — the prefill of one layer whose Q, K, V and O are
  * in host memory (a serving engine's view of a request).  The layer is cut
- * into n_chunks runs of query rows (whole 128-row tiles); chunk c's Q, K and
+ * into n_chunks runs of query rows (whole 128-row tiles; equal runs, except
+ * that with four or more the last two are a half and a quarter of the others,
+ * since that chunk's kernels and download follow the last upload and overlap
+ * nothing; every run has at least one tile); chunk c's Q, K and
  * V rows go to the device on an upload stream, its indexer, selection and
  * attention run on `stream` as soon as they have arrived (the attention of
  * rows [begin, end) only reads K/V rows < end, all of them uploaded by then),

@@ -1025,9 +1025,29 @@ rtp_status rtp_pipeline_create(const rtp_attn_cfg* cfg, const uint8_t* kind_host
     rtp_pipeline_destroy(pl);
     return st;
   };
+  // Chunk boundaries in tiles: equal chunks, except that with four or more
+  // the last two are a half and a quarter of the others (what follows the
+  // last upload -- that chunk's kernels and its download -- is the part of
+  // the pipeline nothing overlaps); every chunk keeps at least one tile.
+  std::vector<int> tb(n_chunks + 1, 0);
+  {
+    std::vector<double> w(n_chunks, 1.0);
+    if (n_chunks >= 4) {
+      w[n_chunks - 2] = 0.5;
+      w[n_chunks - 1] = 0.25;
+    }
+    double total = 0.0, run = 0.0;
+    for (double x : w) total += x;
+    tb[n_chunks] = tiles;
+    for (int c = 1; c < n_chunks; ++c) {
+      run += w[c - 1];
+      const int t = static_cast<int>(std::llround(run / total * tiles));
+      tb[c] = std::min(std::max(t, tb[c - 1] + 1), tiles - (n_chunks - c));
+    }
+  }
   for (int c = 0; c < n_chunks; ++c) {
-    const int b = 128 * static_cast<int>(static_cast<long>(c) * tiles / n_chunks);
-    const int e = std::min(cfg->seq, 128 * static_cast<int>(static_cast<long>(c + 1) * tiles / n_chunks));
+    const int b = 128 * tb[c];
+    const int e = std::min(cfg->seq, 128 * tb[c + 1]);
     rtp_plan* p = nullptr;
     const rtp_status st = rtp_route_heads_range(cfg, kind_host, b, e, stream, &p);
     if (st != RTP_OK) return fail(st);
