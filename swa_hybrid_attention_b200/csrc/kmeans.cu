@@ -28,8 +28,8 @@
 //                 in the same order as km_assign, which does every key when
 //                 RTP_KMEANS_EXACT_ASSIGN=1), so the assignment is the fp32
 //                 path's, key for key
-//   km_hist / km_scan / km_place / km_means  the keys grouped by cluster:
-//                 per-segment counts, offsets and segment starts, stable
+//   km_hist / km_segscan / km_scan / km_place / km_means  the keys grouped
+//                 by cluster: per-segment counts, segment starts, offsets, stable
 //                 placement (a warp per segment, 32 keys per step with
 //                 match_any), and the new centroids (each summed over its
 //                 keys in position order)
@@ -492,8 +492,9 @@ __device__ __forceinline__ void scan_counts(const int* cnt, int* off, int nc, in
 // and each centroid is the sum of its members' projections in member order,
 // divided by their number (an empty cluster keeps its centroid).
 //   km_hist   per segment of kKmSegKeys keys: the count of each cluster
-//   km_scan   per (sequence, head): the offsets of the clusters and, for each
-//             segment, where its keys of each cluster start
+//   km_segscan per cluster: where each segment's keys start inside it, and
+//             its size
+//   km_scan   per (sequence, head): the offsets of the clusters
 //   km_place  one warp per segment: its keys to their places, in key order
 //   km_means  one half-warp per cluster: lane d sums dimension d
 constexpr int kHistThreads = 256;
@@ -515,6 +516,26 @@ __global__ void __launch_bounds__(kHistThreads) km_hist_kernel(const KmeansArgs 
   for (int c = tid; c < a.nc; c += kHistThreads) seg[c] = cnt[c];
 }
 
+// One thread per cluster: each segment's start relative to the cluster (in
+// place over the counts) and the cluster's size (into its offsets entry).
+constexpr int kSegScanThreads = 256;
+__global__ void __launch_bounds__(kSegScanThreads) km_segscan_kernel(const KmeansArgs a) {
+  if (a.kind[blockIdx.y] != KIND_SPARSE) return;
+  const size_t bk = head_index(a);
+  const int c = blockIdx.x * kSegScanThreads + threadIdx.x;
+  if (c >= a.nc) return;
+  int32_t* seg = a.seg + bk * a.n_seg * a.nc + c;
+  int run = 0;
+#pragma unroll 4
+  for (int sg = 0; sg < a.n_seg; ++sg) {
+    const int v = seg[static_cast<size_t>(sg) * a.nc];
+    seg[static_cast<size_t>(sg) * a.nc] = run;
+    run += v;
+  }
+  a.offsets[bk * (a.nc + 1) + c] = run;
+}
+
+// One CTA per (sequence, head): the clusters' offsets from their sizes.
 __global__ void __launch_bounds__(kGroupThreads) km_scan_kernel(const KmeansArgs a) {
   __shared__ int cnt[kMaxClusters], off[kMaxClusters];
   __shared__ int warp_tot[32];
@@ -522,27 +543,12 @@ __global__ void __launch_bounds__(kGroupThreads) km_scan_kernel(const KmeansArgs
   const size_t bk = head_index(a);
   const int tid = threadIdx.x;
   if (tid == 0) a.amb_count[bk] = 0;  // the undecided list of the next round starts empty
-  int32_t* seg = a.seg + bk * a.n_seg * a.nc;
-  // per cluster: each segment's start relative to the cluster, and its size
-  for (int c = tid; c < a.nc; c += kGroupThreads) {
-    int run = 0;
-#pragma unroll 4
-    for (int sg = 0; sg < a.n_seg; ++sg) {
-      const int v = seg[static_cast<size_t>(sg) * a.nc + c];
-      seg[static_cast<size_t>(sg) * a.nc + c] = run;
-      run += v;
-    }
-    cnt[c] = run;
-  }
+  int32_t* offs = a.offsets + bk * (a.nc + 1);
+  for (int c = tid; c < a.nc; c += kGroupThreads) cnt[c] = offs[c];
   __syncthreads();
   scan_counts(cnt, off, a.nc, warp_tot);
   __syncthreads();
-  int32_t* offs = a.offsets + bk * (a.nc + 1);
-  for (int c = tid; c < a.nc; c += kGroupThreads) {
-    offs[c] = off[c];
-#pragma unroll 4
-    for (int sg = 0; sg < a.n_seg; ++sg) seg[static_cast<size_t>(sg) * a.nc + c] += off[c];
-  }
+  for (int c = tid; c < a.nc; c += kGroupThreads) offs[c] = off[c];
   if (tid == 0) offs[a.nc] = a.n;
 }
 
@@ -553,8 +559,9 @@ __global__ void __launch_bounds__(32 * kPlaceWarps) km_place_kernel(const Kmeans
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const int sg = blockIdx.x * kPlaceWarps + w;
   if (sg >= a.n_seg) return;  // (warp-uniform; the warps share no barrier)
-  const int32_t* start = a.seg + (bk * a.n_seg + sg) * a.nc;
-  for (int c = lane; c < a.nc; c += 32) running[w][c] = start[c];
+  const int32_t* start = a.seg + (bk * a.n_seg + sg) * a.nc;  // relative to the cluster
+  const int32_t* offs = a.offsets + bk * (a.nc + 1);
+  for (int c = lane; c < a.nc; c += 32) running[w][c] = offs[c] + start[c];
   __syncwarp();
   const int32_t* asg = a.assign + bk * a.n;
   int32_t* mem = a.members + bk * a.n;
@@ -673,6 +680,7 @@ cudaError_t launch_kmeans(const KmeansArgs& a, int iters, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const dim3 per_mma((a.n + kMmaKeysPerCta - 1) / kMmaKeysPerCta, a.n_kv_heads, a.batch);
   const dim3 per_seg(a.n_seg, a.n_kv_heads, a.batch);
+  const dim3 per_segscan((a.nc + kSegScanThreads - 1) / kSegScanThreads, a.n_kv_heads, a.batch);
   const dim3 per_place((a.n_seg + kPlaceWarps - 1) / kPlaceWarps, a.n_kv_heads, a.batch);
   const dim3 per_means((a.nc * 16 + kMeansThreads - 1) / kMeansThreads, a.n_kv_heads, a.batch);
   // one CTA per chunk of a full list; those beyond the list's end leave at once
@@ -685,6 +693,7 @@ cudaError_t launch_kmeans(const KmeansArgs& a, int iters, cudaStream_t stream) {
       km_rescore_kernel<<<per_rescore, kKmThreads, smem, stream>>>(a);
     }
     km_hist_kernel<<<per_seg, kHistThreads, 0, stream>>>(a);
+    km_segscan_kernel<<<per_segscan, kSegScanThreads, 0, stream>>>(a);
     km_scan_kernel<<<per_head, kGroupThreads, 0, stream>>>(a);
     km_place_kernel<<<per_place, 32 * kPlaceWarps, 0, stream>>>(a);
     km_means_kernel<<<per_means, kMeansThreads, 0, stream>>>(a);

@@ -50,10 +50,29 @@ def run_all(rtp, device):
     return out
 
 
+def run_full(rtp, device):
+    """The decode workload's whole cache (8 sequences x 262,144 rows, 3 of 4
+    heads clustered), 2048 clusters, 8 rounds: the bench's clustering."""
+    from swa_hybrid_attention_b200 import inputs
+
+    w = inputs.workload(4)
+    d = inputs.decode_step(w, device)
+    Lc = d["cache_len"]
+    clu_end = (Lc // w.block - w.n_local) * w.block
+    cl = rtp.cluster_cache(d["kcache"], d["vcache"], d["proj"], d["kinds"], clu_end=clu_end, n_clusters=2048,
+                           iters=8, block=w.block, in_place=True)
+    torch.cuda.synchronize()
+    out = {f: getattr(cl, f).cpu() for f in ("centroids", "members", "offsets", "n_chunks", "chunk_start",
+                                             "chunk_len", "chunk_centroids")}
+    out["status"] = int(rtp.rtp_last_device_status())
+    return {"full": out}
+
+
 if __name__ == "__main__":
     from swa_hybrid_attention_b200 import build
 
     build.build()
     from swa_hybrid_attention_b200 import rtp as mod
 
-    torch.save(run_all(mod, torch.device("cuda:0")), sys.argv[1])
+    run = run_full if "--full" in sys.argv[2:] else run_all
+    torch.save(run(mod, torch.device("cuda:0")), sys.argv[1])

@@ -107,23 +107,17 @@ def test_kmeans_valid_and_agrees_with_oracle(rtp, cuda_device, block, nc, iters)
         assert torch.equal(getattr(cl, name), getattr(cl2, name)), name
 
 
-def test_tensor_core_assignment_equals_exact_path(rtp, cuda_device, tmp_path):
-    """The assignment pass on tensor cores (fp16 distances, keys it cannot
-    decide within its error bound re-scored in fp32) gives, key for key, the
-    exact fp32 path's nearest centroid: whole clusterings are bit-identical to
-    a run with RTP_KMEANS_EXACT_ASSIGN=1 (every key by the fp32 path), also
-    with exact ties (duplicated keys) and values beyond fp16's range."""
+def _against_exact_path(rtp, here, tmp_path, extra):
     import os
     import subprocess
     import sys
 
     import kmeans_cases
 
-    here = kmeans_cases.run_all(rtp, cuda_device)
     out = tmp_path / "exact.pt"
     env = dict(os.environ, RTP_KMEANS_EXACT_ASSIGN="1")
-    r = subprocess.run([sys.executable, kmeans_cases.__file__, str(out)], env=env, capture_output=True, text=True,
-                       timeout=600)
+    r = subprocess.run([sys.executable, kmeans_cases.__file__, str(out)] + extra, env=env, capture_output=True,
+                       text=True, timeout=900)
     assert r.returncode == 0, r.stderr[-2000:]
     exact = torch.load(out)
     for name, fields in here.items():
@@ -131,6 +125,26 @@ def test_tensor_core_assignment_equals_exact_path(rtp, cuda_device, tmp_path):
         for f, t in fields.items():
             if f != "status":
                 assert torch.equal(t, exact[name][f]), (name, f)
+
+
+def test_tensor_core_assignment_equals_exact_path(rtp, cuda_device, tmp_path):
+    """The assignment pass on tensor cores (fp16 distances, keys it cannot
+    decide within its error bound re-scored in fp32) gives, key for key, the
+    exact fp32 path's nearest centroid: whole clusterings are bit-identical to
+    a run with RTP_KMEANS_EXACT_ASSIGN=1 (every key by the fp32 path), also
+    with exact ties (duplicated keys) and values beyond fp16's range."""
+    import kmeans_cases
+
+    _against_exact_path(rtp, kmeans_cases.run_all(rtp, cuda_device), tmp_path, [])
+
+
+@pytest.mark.slow
+def test_tensor_core_assignment_equals_exact_path_full_size(rtp, cuda_device, tmp_path):
+    """The same at the decode workload's full size: 8 x 262,144-row cache, 3
+    clustered heads, 2048 clusters, 8 rounds (6.28M keys a round)."""
+    import kmeans_cases
+
+    _against_exact_path(rtp, kmeans_cases.run_full(rtp, cuda_device), tmp_path, ["--full"])
 
 
 def test_kmeans_recovers_planted_blobs_exactly(rtp, cuda_device):
