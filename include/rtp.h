@@ -413,7 +413,8 @@ rtp_status rtp_sparse_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, 
  * while a CUDA graph is being captured or replayed elsewhere in the
  * process, real-time loops that must not enter the allocator (cudaMalloc
  * synchronises the device), or hosts whose memory pools are owned by
- * another runtime.  The paper has no counterpart to this entry point.
+ * another runtime.  The method itself has no counterpart to this entry
+ * point; it is a variant of rtp_sparse_decode for such callers.
  *   Arguments are those of rtp_sparse_decode without workspace/ws_bytes.
  *   The split-K scratch (selection lists and per-split partial results)
  *   lives in a fixed 16 MiB device array inside the library

@@ -110,14 +110,14 @@ constexpr int kAssignKeys = 4;
 // kList: the CTA's keys are entries [first, first + kKmThreads*kAssignKeys)
 // of the head's list of undecided keys (count entries); otherwise keys
 // first + ... directly.
-template <bool kList>
+template <bool kList, int kThreads, int kKeys>
 __device__ __forceinline__ void exact_assign(const KmeansArgs& a, size_t bk, int first, int count) {
   extern __shared__ float4 mu4[];  // [nc][4] centroids, then [nc] squared norms
   float* nrm = reinterpret_cast<float*>(mu4 + 4 * a.nc);
   const float4* src = reinterpret_cast<const float4*>(a.centroids + bk * a.nc * kRank);
-  for (int e = threadIdx.x; e < 4 * a.nc; e += kKmThreads) mu4[e] = src[e];
+  for (int e = threadIdx.x; e < 4 * a.nc; e += kThreads) mu4[e] = src[e];
   __syncthreads();
-  for (int c = threadIdx.x; c < a.nc; c += kKmThreads) {
+  for (int c = threadIdx.x; c < a.nc; c += kThreads) {
     float s = 0.f;
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
@@ -130,17 +130,17 @@ __device__ __forceinline__ void exact_assign(const KmeansArgs& a, size_t bk, int
     nrm[c] = s;
   }
   __syncthreads();
-  // keys of entries e0 + u * kKmThreads, u < kAssignKeys (coalesced over the CTA)
+  // keys of entries e0 + u * kThreads, u < kKeys (coalesced over the CTA)
   const int e0 = first + threadIdx.x;
-  int jk[kAssignKeys];
+  int jk[kKeys];
 #pragma unroll
-  for (int u = 0; u < kAssignKeys; ++u) {
-    const int e = e0 + u * kKmThreads;
+  for (int u = 0; u < kKeys; ++u) {
+    const int e = e0 + u * kThreads;
     jk[u] = e < count ? (kList ? a.amb_list[bk * a.n + e] : e) : -1;
   }
-  float x[kAssignKeys][kRank];
+  float x[kKeys][kRank];
 #pragma unroll
-  for (int u = 0; u < kAssignKeys; ++u) {
+  for (int u = 0; u < kKeys; ++u) {
     const int j = min(max(jk[u], 0), a.n - 1);
     const float4* xr = reinterpret_cast<const float4*>(a.X + (bk * a.n + j) * kRank);
 #pragma unroll
@@ -152,10 +152,10 @@ __device__ __forceinline__ void exact_assign(const KmeansArgs& a, size_t bk, int
       x[u][4 * w + 3] = v.w;
     }
   }
-  float best[kAssignKeys];
-  int bc[kAssignKeys];
+  float best[kKeys];
+  int bc[kKeys];
 #pragma unroll
-  for (int u = 0; u < kAssignKeys; ++u) {
+  for (int u = 0; u < kKeys; ++u) {
     best[u] = INFINITY;
     bc[u] = 0;
   }
@@ -165,7 +165,7 @@ __device__ __forceinline__ void exact_assign(const KmeansArgs& a, size_t bk, int
     const float m[kRank] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w,
                             m2.x, m2.y, m2.z, m2.w, m3.x, m3.y, m3.z, m3.w};
 #pragma unroll
-    for (int u = 0; u < kAssignKeys; ++u) {
+    for (int u = 0; u < kKeys; ++u) {
       float dot = 0.f;
 #pragma unroll
       for (int d = 0; d < kRank; ++d) dot = fmaf(x[u][d], m[d], dot);
@@ -177,7 +177,7 @@ __device__ __forceinline__ void exact_assign(const KmeansArgs& a, size_t bk, int
     }
   }
 #pragma unroll
-  for (int u = 0; u < kAssignKeys; ++u) {
+  for (int u = 0; u < kKeys; ++u) {
     const int j = jk[u];
     if (j >= 0 && j < a.n) a.assign[bk * a.n + j] = bc[u];
   }
@@ -185,7 +185,7 @@ __device__ __forceinline__ void exact_assign(const KmeansArgs& a, size_t bk, int
 
 __global__ void __launch_bounds__(kKmThreads) km_assign_kernel(const KmeansArgs a) {
   if (a.kind[blockIdx.y] != KIND_SPARSE) return;
-  exact_assign<false>(a, head_index(a), blockIdx.x * kKmThreads * kAssignKeys, a.n);
+  exact_assign<false, kKmThreads, kAssignKeys>(a, head_index(a), blockIdx.x * kKmThreads * kAssignKeys, a.n);
 }
 
 // gridDim.x CTAs per head walk the head's list in chunks of
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kKmThreads) km_rescore_kernel(const KmeansArgs
   const int count = min(a.amb_count[bk], a.n);
   for (int first = blockIdx.x * kKmThreads * kAssignKeys; first < count;
        first += gridDim.x * kKmThreads * kAssignKeys) {  // (uniform over the CTA)
-    exact_assign<true>(a, bk, first, count);
+    exact_assign<true, kKmThreads, kAssignKeys>(a, bk, first, count);
     __syncthreads();  // the shared centroids are loaded again for the next chunk
   }
 }
@@ -526,11 +526,16 @@ __global__ void __launch_bounds__(kSegScanThreads) km_segscan_kernel(const Kmean
   if (c >= a.nc) return;
   int32_t* seg = a.seg + bk * a.n_seg * a.nc + c;
   int run = 0;
-#pragma unroll 4
-  for (int sg = 0; sg < a.n_seg; ++sg) {
-    const int v = seg[static_cast<size_t>(sg) * a.nc];
-    seg[static_cast<size_t>(sg) * a.nc] = run;
-    run += v;
+  for (int sg0 = 0; sg0 < a.n_seg; sg0 += 8) {  // eight segments' counts in flight, then their starts
+    int v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = sg0 + u < a.n_seg ? seg[static_cast<size_t>(sg0 + u) * a.nc] : 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (sg0 + u < a.n_seg) {
+        seg[static_cast<size_t>(sg0 + u) * a.nc] = run;
+        run += v[u];
+      }
   }
   a.offsets[bk * (a.nc + 1) + c] = run;
 }
