@@ -720,6 +720,29 @@ def time_decode_rotating(rtp, w, d, C, cfg, steps, stream, n_problems=4):
             "l2": "no flush: four independent problems in turn, ~285 MB of other K/V between two visits of one"}
 
 
+def time_kmeans_one_sequence(rtp, device, n_clusters=2048, iters=8):
+    """k-means of one sequence of the decode workload's cache (3 clustered
+    heads, 262,144 rows each): a small case for profiling the clustering
+    kernels; warm, median of 5 runs after one, in place (no K/V copy)."""
+    w = inputs.workload(4)
+    d = inputs.decode_step(w, device, batch=1)
+    Lc = d["cache_len"]
+    clu_end = (Lc // w.block - w.n_local) * w.block
+    runs = []
+    for i in range(6):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        rtp.cluster_cache(d["kcache"], d["vcache"], d["proj"], d["kinds"], clu_end=clu_end, n_clusters=n_clusters,
+                          iters=iters, block=w.block, in_place=True)
+        b.record()
+        torch.cuda.synchronize()
+        if i > 0:
+            runs.append(a.elapsed_time(b))
+    return {"ms": statistics.median(runs), "clusters": n_clusters, "rounds": iters, "keys_per_head": clu_end - w.block,
+            "heads": sum(1 for k in d["kinds"] if k == inputs.SPARSE), "status": rtp.status_str(rtp.rtp_last_device_status()),
+            "note": "includes the arrays' allocation by cluster_cache (outside the kernels)"}
+
+
 def time_decode_graph(rtp, w, d, C, o_ref, flush, flush_read, steps):
     """The same step as a serving loop would run it: the allocation-free
     entry point captured once in a CUDA graph (its three launches and their
@@ -1053,6 +1076,10 @@ def run_ours(args, rank, world, local):
         if rank == 0:
             print(json.dumps({"decode_8x256k": time_decode(rtp, args.decode_steps, device)}), flush=True)
         return
+    if args.only == "kmeans":
+        if rank == 0:
+            print(json.dumps({"kmeans_one_sequence": time_kmeans_one_sequence(rtp, device)}), flush=True)
+        return
     w = inputs.workload(3)
     if args.seq:
         # same head structure at a shorter length (profiling runs)
@@ -1160,7 +1187,7 @@ def main():
     ap.add_argument("--ref-step-seconds", type=float, default=10.0)
     ap.add_argument("--decode-steps", type=int, default=256)
     ap.add_argument("--seq", type=int, default=0, help="override the primary workload's length (profiling)")
-    ap.add_argument("--only", choices=["all", "decode", "selection", "cp"], default="all",
+    ap.add_argument("--only", choices=["all", "decode", "selection", "cp", "kmeans"], default="all",
                     help="run only part of the bench (decode step; selection variants, for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:

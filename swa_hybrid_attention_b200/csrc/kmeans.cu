@@ -205,16 +205,19 @@ __global__ void __launch_bounds__(kKmThreads) km_rescore_kernel(const KmeansArgs
 // The distances of 16 keys to 8 centroids are one mma.sync m16n8k16: A = the
 // keys' projections in fp16, B = -2 mu in fp16, C = |mu|^2 (fp32, the exact
 // path's value), so D = |mu|^2 - 2 x~.mu~.  Each thread keeps, per key row,
-// the smallest D, its centroid and the second smallest D.  D differs from the
-// exact path's fp32 distance by at most
+// the smallest D, the group (four centroids of one tile pair) holding it and
+// the smallest D among the other groups.  D differs from the exact path's fp32
+// distance by at most
 //   E = 1.125 * 2^-9 |x| M + 2^-16 M^2 + 2^-20 (|x| + M),   M = max_c |mu_c|
 // (fp16 rounding of x and mu: 2^-11 relative each, products exact; fp32
 // accumulation of 17 terms; the exact path's own fp32 rounding; with margin).
-// A key whose second smallest D exceeds its smallest by more than 2E has the
-// exact path's nearest centroid, unique; every other key (and any key with
-// non-finite values, |x| >= 30000 or M > 8192, outside fp16's safe range) is
-// appended to the head's undecided list, which km_rescore_kernel assigns by
-// the exact path.  The result is the exact path's, key for key.
+// A key whose other groups all lie more than 2E above its smallest D has the
+// exact path's nearest centroid in its best group, found by the group's four
+// exact distances (ascending, first minimum: the exact path's tie rule); every
+// other key (and any key with non-finite values, |x| >= 30000 or M > 8192,
+// outside fp16's safe range) is appended to the head's undecided list, which
+// km_rescore_kernel assigns by the exact path.  The result is the exact
+// path's, key for key.
 constexpr int kMmaWarps = 8;
 constexpr int kMmaThreads = 32 * kMmaWarps;
 constexpr int kMmaGroups = 4;                              // 32-key groups per warp
@@ -240,23 +243,29 @@ __device__ __forceinline__ uint32_t half2_bits(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Running smallest distance m1 of one key row, a lower bound L of its second
-// smallest, and the 16-centroid tile pair where m1 was found, updated with
-// the four distances this thread sees in pair p: (d0, d1) from the first
-// 8-centroid tile, (e0, e1) from the second.  L stays <= the true second
-// smallest: the group's two smallest are exact, and the second smallest of
-// the union is min(max(m1, g1), min(L, g2)).
+__device__ __forceinline__ float min3f(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Running smallest distance m1 of one key row, the smallest distance L among
+// the other groups (a group: the four centroids one thread sees in one
+// 16-centroid tile pair) and the tile pair holding m1, updated with this
+// thread's four distances of pair p: (d0, d1) from the first 8-centroid tile,
+// (e0, e1) from the second.  If L exceeds m1 by more than twice the error
+// bound, every centroid outside the group lies farther than the group's
+// nearest, so the exact nearest centroid is one of the group's four.
 __device__ __forceinline__ void top2_group(float& m1, float& L, int& pb, float d0, float d1, float e0, float e1,
                                            int p) {
-  const float a0 = fminf(d0, d1), b0 = fmaxf(d0, d1), a1 = fminf(e0, e1), b1 = fmaxf(e0, e1);
-  const float g1 = fminf(a0, a1), g2 = fminf(fmaxf(a0, a1), fminf(b0, b1));
-  L = fminf(fmaxf(m1, g1), fminf(L, g2));
+  const float g1 = min3f(fminf(d0, d1), e0, e1);
+  L = fminf(L, fmaxf(m1, g1));
   if (g1 < m1) pb = p;
   m1 = fminf(m1, g1);
 }
 
 // Merge with the quad neighbour at lane ^ mask (the same rows, other
-// centroids); owner = the quad lane whose centroids hold m1.
+// centroids, so other groups); owner = the quad lane whose group holds m1.
 __device__ __forceinline__ void top2_merge(float& m1, float& L, int& pb, int& owner, int mask) {
   const float om1 = __shfl_xor_sync(0xffffffffu, m1, mask);
   const float oL = __shfl_xor_sync(0xffffffffu, L, mask);
@@ -279,7 +288,7 @@ __device__ __forceinline__ float exact_dist(const float (&x)[kRank], const float
   return fmaf(-2.f, dot, nc2);
 }
 
-__global__ void __launch_bounds__(kMmaThreads) km_assign_mma_kernel(const KmeansArgs a) {
+__global__ void __launch_bounds__(kMmaThreads, 3) km_assign_mma_kernel(const KmeansArgs a) {
   // dynamic: -2 mu as fp16 [ncp][16] (32 bytes per centroid, its two 16-byte
   // halves swapped when bit 2 of c is set, so that the eight rows of an
   // ldmatrix tile fall in distinct bank groups), then |mu|^2 [ncp] (fp32,
