@@ -18,8 +18,10 @@ follows (see the header of oracle.cpp for the page titles).
 Pinned by the not-gpu tests (tests/test_oracle_pins.py) against brute-force
 masked attention (both attention statements), torch's scaled-dot-product
 attention in fp64 on CPU, exact nearest-even rounding by rational
-arithmetic, full sorts, closed forms and invariants.  The pages print no worked example, so no
-value here is tied to the authors' own implementation.
+arithmetic, full sorts, closed forms and invariants; tests/test_oracle_mutants.py
+checks that each of a list of planted mistakes in this package makes those pins
+fail.  The pages print no worked example, so no value here is tied to the
+authors' own implementation.
 """
 
 from __future__ import annotations

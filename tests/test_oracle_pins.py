@@ -384,14 +384,18 @@ def test_per_head_selection_with_identical_heads_equals_the_shared_one():
 # --------------------------------------------------------------------- decode
 
 
-def test_decode_equals_last_prefill_row():
-    Lc, block, G = 1024, 64, 4
+@pytest.mark.parametrize("Lc", [1024, 1025])
+def test_decode_equals_last_prefill_row(Lc):
+    """The decode step is the prefill's row L_c - 1, also when that row opens
+    a new query block (L_c = 1025: block 16, whose own centroid does not
+    exist yet)."""
+    block, G = 64, 4
     d = inputs.small_prefill(Lc, G, 1, [oracle.SPARSE], seed=31)
     q, k, v = d["q"][0], d["k"][0, 0], d["v"][0, 0]
     p = inputs.lowfreq_projector()
     C = oracle.centroids(k, block, p).astype(np.float32)
     out, sel, cnt, _ = oracle.decode_head(q[:, Lc - 1], k, v, C, p, oracle.SPARSE, 0, block, 4, 2)
-    nb = Lc // block
+    nb = (Lc + block - 1) // block
     t = nb - 1
     sel_full = np.full((nb, sel.shape[0]), -1, dtype=np.int32)
     cnt_full = np.ones(nb, dtype=np.int32)
@@ -688,6 +692,19 @@ def test_kmeans_degenerate_sizes():
     assert np.array_equal(assign, np.arange(9)) and np.array_equal(mu, X)
     mu0, _ = oracle.kmeans(X, 3, 0)  # no iteration: the evenly spaced seeds
     assert np.array_equal(mu0, X[[1, 4, 7]])
+
+
+def test_kmeans_ties_go_to_the_lower_index_and_an_empty_cluster_keeps_its_centroid():
+    # Six points on a line (integers, so every distance is exact); the seeds
+    # are rows 1, 3 and 5: the values 0, 4 and 4.  Clusters 1 and 2 start on
+    # the same point, so every point nearer 4 ties between them and goes to
+    # cluster 1, leaving cluster 2 empty; the point 2 ties between 0 and 4
+    # and goes to cluster 0.
+    X = np.zeros((6, 16))
+    X[:, 0] = [2, 0, 8, 4, 3, 4]
+    mu, assign = oracle.kmeans(X, 3, 1)
+    assert assign.tolist() == [0, 0, 1, 1, 1, 1]
+    assert mu[:, 0].tolist() == [1.0, 4.75, 4.0] and not mu[:, 1:].any()
 
 
 def test_cluster_chunks_cover_members_once():
