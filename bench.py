@@ -656,7 +656,6 @@ def time_decode(rtp, steps, device):
     torch.cuda.synchronize()
     ms = statistics.median(a.elapsed_time(b) for a, b in times)
     status = rtp.rtp_last_device_status(stream)
-    graph = time_decode_graph(rtp, w, d, C, o, flush, flush_read, steps)
     rotating = time_decode_rotating(rtp, w, d, C, cfg, steps, stream)
     upkeep = time_cache_upkeep(rtp, w, d, C, cfg, flush, flush_read, steps, stream)
     clustered = time_clustered_decode(rtp, w, d, flush, flush_read, steps, stream)
@@ -669,7 +668,7 @@ def time_decode(rtp, steps, device):
     flops = w.batch * keys * G * 4 * 128
     return {"workload": w.name, "ms_per_step": ms, "algorithmic_bytes": bytes_, "gb_s": bytes_ / (ms * 1e-3) / 1e9,
             "tflops_effective": flops / (ms * 1e-3) / 1e12, "l2": "flushed before each step (256 MB write, then 256 MB read)",
-            "launches_per_step": 3, "status": rtp.status_str(status), "graph": graph, "rotating": rotating,
+            "launches_per_step": 3, "status": rtp.status_str(status), "rotating": rotating,
             "cache_upkeep": upkeep, "clustered": clustered}
 
 
@@ -741,47 +740,6 @@ def time_kmeans_one_sequence(rtp, device, n_clusters=2048, iters=8):
     return {"ms": statistics.median(runs), "clusters": n_clusters, "rounds": iters, "keys_per_head": clu_end - w.block,
             "heads": sum(1 for k in d["kinds"] if k == inputs.SPARSE), "status": rtp.status_str(rtp.rtp_last_device_status()),
             "note": "includes the arrays' allocation by cluster_cache (outside the kernels)"}
-
-
-def time_decode_graph(rtp, w, d, C, o_ref, flush, flush_read, steps):
-    """The same step as a serving loop would run it: the allocation-free
-    entry point captured once in a CUDA graph (its three launches and their
-    programmatic dependencies) and replayed; L2 flushed before each replay
-    as for the direct launches.  The replay's output must equal theirs."""
-    kinds, Lc = d["kinds"], d["cache_len"]
-    cfg = rtp.AttnConfig(w.batch, 1, w.n_q_heads, w.n_kv_heads, w.window, w.block, w.topk, w.n_local)
-    o = torch.empty_like(o_ref)
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
-
-    def step():
-        rtp.rtp_sparse_decode_noalloc(cfg, kinds, Lc, d["q"], d["kcache"], d["vcache"], C, d["proj"], o, stream=s)
-
-    with torch.cuda.stream(s):
-        step()
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=s):
-        step()
-    torch.cuda.synchronize()
-    times = []
-    with torch.cuda.stream(s):
-        for _ in range(3):
-            g.replay()
-        for _ in range(steps):
-            flush.zero_()
-            flush_read.sum()
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            a.record(s)
-            g.replay()
-            b.record(s)
-            times.append((a, b))
-    torch.cuda.synchronize()
-    same = bool(torch.equal(o, o_ref))
-    del g
-    return {"ms_per_step": statistics.median(a.elapsed_time(b) for a, b in times), "equal_to_direct": same,
-            "note": "rtp_sparse_decode_noalloc captured once in a CUDA graph and replayed"}
 
 
 def time_clustered_decode(rtp, w, d, flush, flush_read, steps, stream, n_clusters=2048, iters=8):
@@ -1034,8 +992,6 @@ def secondary_summary(sec: dict) -> dict:
     if "ms_per_step" in d:
         out["decode_8x256k_us"] = round(d["ms_per_step"] * 1e3, 2)
         out["decode_hbm_frac"] = round(d["gb_s"] / 6552.6, 3) if "gb_s" in d else None
-        if d.get("graph"):
-            out["decode_graph_us"] = round(d["graph"]["ms_per_step"] * 1e3, 2)
         if (d.get("rotating") or {}).get("ms_per_step"):
             out["decode_rotating_us"] = round(d["rotating"]["ms_per_step"] * 1e3, 2)
         c = d.get("clustered") or {}

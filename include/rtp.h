@@ -409,20 +409,19 @@ rtp_status rtp_sparse_decode(const rtp_attn_cfg* cfg, const uint8_t* kind_host, 
 
 /* ------------------------------------------------------------------------
  * rtp_sparse_decode_noalloc — the decode step of rtp_sparse_decode for
- * callers that cannot allocate device memory at call time: code running
- * while a CUDA graph is being captured or replayed elsewhere in the
- * process, real-time loops that must not enter the allocator (cudaMalloc
- * synchronises the device), or hosts whose memory pools are owned by
- * another runtime.  The method itself has no counterpart to this entry
- * point; it is a variant of rtp_sparse_decode for such callers.
+ * callers that cannot allocate device memory at call time: real-time loops
+ * that must not enter the allocator (cudaMalloc synchronises the device),
+ * or hosts whose memory pools are owned by another runtime.  The method
+ * itself has no counterpart to this entry point; it is a variant of
+ * rtp_sparse_decode for such callers.
  *   Arguments are those of rtp_sparse_decode without workspace/ws_bytes.
  *   The split-K scratch (selection lists and per-split partial results)
  *   lives in a fixed 16 MiB device array inside the library
  *   (rtp_decode_workspace_bytes tells how much a shape needs); a shape that
  *   needs more returns RTP_ERR_INVALID_ARG.  Nothing is allocated: no
  *   cudaMalloc, cudaFree or allocating library call on this path.
- *   The array is looked up once per device, on the first call made with
- *   that device current; make that first call before any stream capture.
+ *   The array's address is looked up once per device, on the first call
+ *   made with that device current.
  *   Every call shares the one array and it keeps the last call's contents;
  *   a call writes every word it reads earlier in the same call (selection
  *   lists, then per-split partial results), so nothing needs clearing —
