@@ -109,6 +109,21 @@ MUTANTS = [
        "for (long j = std::max<long>(0, i - window); j <= i; ++j) keys.push_back(j);")]),
     ("decode full head misses the new token", CPP,
      [("for (long j = 0; j <= i; ++j) keys.push_back(j);", "for (long j = 0; j < i; ++j) keys.push_back(j);")]),
+    ("query summary rows read head-interleaved", CPP,
+     [("project_row(q + (static_cast<long>(h) * N + i) * D, D, P, r, qt.data());\n        for (int c = 0; c < r; ++c) mean[c]",
+       "project_row(q + (i * G + h) * D, D, P, r, qt.data());\n        for (int c = 0; c < r; ++c) mean[c]")]),
+    ("query summary drops the block's first row", CPP,
+     [("for (long i = t * B; i < (t + 1) * B; ++i) {", "for (long i = t * B + 1; i < (t + 1) * B; ++i) {")]),
+    ("row-max scores with the centroids transposed", CPP,
+     [("s += u[static_cast<size_t>(i) * r + c] * C[j * r + c];", "s += u[static_cast<size_t>(i) * r + c] * C[c * nb + j];")]),
+    ("dynamic covered fraction before the cut off by one", CPP,
+     [("cum_lo[q] = nstar >= 2 ? prefix[nstar - 2] / Z", "cum_lo[q] = nstar >= 2 ? prefix[nstar - 1] / Z")]),
+    ("k-means with an absolute-value distance", CPP, [("dist += e * e;", "dist += std::fabs(e);")]),
+    ("key-list attention ignores the list", CPP,
+     [("widen_bf16(kc[keys[e] * D + d]);\n      s[e] = acc * scale;", "widen_bf16(kc[e * D + d]);\n      s[e] = acc * scale;")]),
+    ("sparse rows read the first query block's selection", CPP,
+     [("long b = sel[t * static_cast<long>(kmax) + e];", "long b = sel[e];")]),
+    ("decode overrides a given selection", CPP, [("if (mode == 2 && !use_given_sel) {", "if (mode == 2) {")]),
     # --- Python statements ---
     ("chunk ties kept by higher index", PY,
      [("order = np.lexsort((np.arange(s.size), -s))", "order = np.lexsort((-np.arange(s.size), -s))")]),
@@ -128,6 +143,19 @@ MUTANTS = [
      [("r = ((u + np.uint64((1 << 44) - 1) + lsb) >> keep) << keep", "r = ((u + np.uint64(1 << 44)) >> keep) << keep")]),
     ("bf16 rounding truncates", PY,
      [("r = ((u + np.uint64((1 << 44) - 1) + lsb) >> keep) << keep", "r = (u >> keep) << keep")]),
+    ("chunk top-k keeps one fewer", PY, [("return np.sort(order[:topk])", "return np.sort(order[:topk - 1])")]),
+    ("cache centroids written for every head", PY,
+     [("if int(kinds[h]) == SPARSE and n > 0:", "if n > 0:")]),
+    ("append completes a block one row early", PY, [("if (pos + 1) % block == 0:", "if (pos + 2) % block == 0:")]),
+    ("append writes the next block's centroid", PY,
+     [("blk = (pos + 1) // block - 1", "blk = min((pos + 1) // block, Cn.shape[2] - 1)")]),
+    ("bf16 subnormals on the wrong spacing", PY,
+     [("out[tiny] = np.round(a[tiny] * 2.0 ** 133) * 2.0 ** -133", "out[tiny] = np.round(a[tiny] * 2.0 ** 132) * 2.0 ** -132")]),
+    ("bf16 overflow kept finite", PY,
+     [("out[over] = np.copysign(np.inf, a[over])", "out[over] = np.copysign(_BF16_MAX, a[over])")]),
+    ("matrix attention window starts one key late", PY,
+     [("keys = torch.arange(max(0, int(pp[idx].min()) - window + 1), hi + 1)",
+       "keys = torch.arange(max(0, int(pp[idx].min()) - window + 2), hi + 1)")]),
     ("matrix attention window one key wider", PY,
      [("visible &= keys[None, :] > i[:, None] - window", "visible &= keys[None, :] >= i[:, None] - window")]),
     ("matrix attention without the scale", PY,

@@ -411,6 +411,30 @@ def test_decode_equals_last_prefill_row(Lc):
     assert list(sel[:cnt]) == brute_select(qb, C.astype(np.float64), t, 4, 2)
 
 
+def test_decode_attends_to_a_given_selection_as_given():
+    """A selection handed to the decode step is used as it is (not replaced
+    by the oracle's own top-k): the output equals brute-force attention over
+    exactly those blocks."""
+    Lc, block, G, topk, n_local = 1000, 64, 2, 4, 2
+    d = inputs.small_prefill(Lc, G, 1, [oracle.SPARSE], seed=37)
+    q, k, v = d["q"][0], d["k"][0, 0], d["v"][0, 0]
+    p = inputs.lowfreq_projector()
+    C = oracle.centroids(k, block, p).astype(np.float32)
+    given = [0, 3, 7, 14, 15]  # t = 999 // 64 = 15; block 15 holds keys 960..999
+    _, own, own_cnt, _ = oracle.decode_head(q[:, Lc - 1], k, v, C, p, oracle.SPARSE, 0, block, topk, n_local)
+    assert list(own[:own_cnt]) != given
+    sel = np.full(topk + 1 + n_local, -1, dtype=np.int32)
+    sel[:len(given)] = given
+    out, sel_out, cnt_out, _ = oracle.decode_head(q[:, Lc - 1], k, v, C, p, oracle.SPARSE, 0, block, topk, n_local,
+                                                  sel=sel, cnt=len(given))
+    assert list(sel_out[:cnt_out]) == given
+    j = np.arange(Lc)
+    m = np.isin(j // block, given)[None, :]
+    for h in range(G):
+        ref = dense_reference(widen(q[h, Lc - 1:Lc]), widen(k), widen(v), m)
+        assert np.max(np.abs(out[h] - ref[0])) <= 1e-12
+
+
 def test_decode_swa_equals_window_row():
     Lc, G, W = 700, 2, 300
     d = inputs.small_prefill(Lc, G, 1, [oracle.SWA], seed=41)
