@@ -1,6 +1,10 @@
-"""The error bound behind the tensor-core k-means assignment, checked on the CPU.
+"""The error bounds behind the two fp16 tensor-core scorers, checked on the CPU.
 
-km_assign_mma_kernel (csrc/kmeans.cu) computes D = |mu|^2 - 2 x~.mu~ with an
+Two kernels score with fp16 mma.sync and keep exactness by re-scoring, in
+fp32, everything a proven bound cannot decide: the k-means assignment and
+the row-max block selection.  Both bounds are checked here.
+
+k-means.  km_assign_mma_kernel (csrc/kmeans.cu) computes D = |mu|^2 - 2 x~.mu~ with an
 mma.sync m16n8k16: x and -2 mu rounded to fp16, the accumulator seeded with
 the exact path's fp32 |mu|^2.  It decides a key only when the other groups'
 smallest D exceeds its smallest D by more than 2E, with
@@ -21,6 +25,16 @@ correctly rounded fma.  Inputs are adversarial: magnitudes from fp16's
 subnormal range up to the kernel's limits (|x| < 30000, M <= 8192),
 components placed on fp16 half-way points, mixed scales and near-cancelling
 distances.  Every model must stay within E.
+
+Row-max selection.  block_select_rowmax_kernel (csrc/select.cu) scores the
+rows u_i of a query block against candidate centroids c_j as fp16 MMAs of
+su u (su a power of two putting every entry below 2^14) and c, accumulated
+from zero in fp32, and keeps for exact re-scoring every candidate whose
+approximate row maximum lies within 2E of the k-th, with
+    E = 2^-9 max|su u_i| max|c_j| + 2^-22 (max|su u_i| + max|c_j|)
+(the maxima as the kernel forms them in fp32, with a 1.001 factor).  The
+exact score is u_i . c_j in two fp32 fma chains of eight ranks, then their
+sum; each approximate product must lie within E of su times it.
 """
 
 from __future__ import annotations
@@ -182,3 +196,87 @@ def test_round32_matches_numpy():
     for v in np.concatenate([rng.standard_normal(200) * np.exp2(rng.integers(-140, 120, 200)),
                              [1.0 + 2.0 ** -24, 1.0 + 3 * 2.0 ** -24, 2.0 ** -149 * 1.5, 2.0 ** -149 * 2.5]]):
         assert float(round32(Fraction(float(v)))) == float(np.float32(v))
+
+
+# ------------------------------------------------------------ row-max scores
+
+
+def two_chains(u, c):
+    """score16_two_chains: ranks 0-7 and 8-15 in two fp32 fma chains, then added."""
+    s0 = round32(F(u[0]) * F(c[0]))
+    s1 = round32(F(u[8]) * F(c[8]))
+    for d in range(1, 8):
+        s0 = fma32(u[d], c[d], s0)
+        s1 = fma32(u[8 + d], c[8 + d], s1)
+    return round32(s0 + s1)
+
+
+def rowmax_scale_and_bound(U, Cs):
+    """su, and E in the scaled unit, as block_select_rowmax_kernel forms them."""
+    un2 = []
+    for u in U:
+        t = Fraction(0)
+        for d in range(R):
+            t = fma32(u[d], u[d], t)
+        un2.append(t)
+    umax = np.float32(math.sqrt(float(max(un2)))) * np.float32(1.001)
+    _, ue = math.frexp(float(umax))
+    su = 2.0 ** (14 - ue) if umax > 0 else 1.0
+    cn2 = [sum(float(np.float32(c[d]) * np.float32(c[d])) for d in range(R)) for c in Cs]
+    cmax = float(np.float32(math.sqrt(max(cn2))) * np.float32(1.001))
+    sumax = su * float(umax)
+    return su, 2.0 ** -9 * sumax * cmax + 2.0 ** -22 * (sumax + cmax), cmax
+
+
+def mma_models_from_zero(a, b):
+    """sum_d fp16(a_d) fp16(b_d) accumulated from zero under the same models."""
+    p = [to_f16(a[d]) * to_f16(b[d]) for d in range(R)]
+    out = {"exact_sum": round32(sum(p))}
+    for tz in (False, True):
+        acc = Fraction(0)
+        for v in p:
+            acc = round32(acc + v, tz)
+        out[f"chain_{'rz' if tz else 'rn'}"] = acc
+        level = p
+        while len(level) > 1:
+            level = [round32(level[i] + level[i + 1], tz) for i in range(0, len(level), 2)]
+        out[f"tree_{'rz' if tz else 'rn'}"] = level[0]
+    return out
+
+
+def rowmax_cases(rng):
+    out = []
+    for su_, sc in [(1.0, 1.0), (1e-4, 3.0), (30.0, 1e-3), (1e-7, 1e-7), (500.0, 2000.0)]:
+        for _ in range(5):
+            out.append(((rng.standard_normal((4, R)) * su_).astype(np.float32),
+                        (rng.standard_normal((6, R)) * sc).astype(np.float32)))
+    for lo, hi in [(-24, -14), (-6, 2), (6, 12)]:
+        for _ in range(5):
+            out.append((f16_halfway(rng, 4 * R, lo, hi).reshape(4, R), f16_halfway(rng, 6 * R, lo, hi).reshape(6, R)))
+
+    def up(e):
+        return np.nextafter(np.float32((1.0 + 2.0 ** -11) * 2.0 ** e), np.float32(np.inf))
+    for eu, ec in [(0, 0), (-9, 5), (7, -3), (3, 12)]:  # coherent: every fp16 rounding upward
+        out.append((np.full((4, R), up(eu), np.float32), np.full((6, R), up(ec), np.float32)))
+    return out
+
+
+def test_rowmax_approximate_scores_stay_within_the_bound():
+    rng = np.random.default_rng(77)
+    worst, checked = 0.0, 0
+    for U, Cs in rowmax_cases(rng):
+        su, E, cmax = rowmax_scale_and_bound(U, Cs)
+        if not cmax < 32768.0:  # the kernel then scores every candidate exactly
+            continue
+        checked += 1
+        for u in U:
+            su_u = [np.float32(su * float(u[d])) for d in range(R)]
+            assert max(abs(float(v)) for v in su_u) < 2.0 ** 14
+            for c in Cs:
+                ex = Fraction(su) * two_chains(u, c)  # scaling by a power of two is exact
+                for name, D in mma_models_from_zero(su_u, c).items():
+                    err = abs(float(D - ex))
+                    worst = max(worst, err / E)
+                    assert err <= E, (name, err, E)
+    print(f"row-max: largest |a - su s| / E: {worst:.3f} over {checked} blocks")
+    assert checked >= 35 and worst > 0.3  # the coherent cases come close to half the bound
