@@ -517,7 +517,7 @@ typedef struct {
   void* k_sorted;          /* bf16 [batch][n_kv_heads][n][128]: K rows in `members` order, or NULL */
   void* v_sorted;          /* bf16, likewise for V (NULL exactly when k_sorted is) */
   float* chunk_centroids;  /* fp32 [batch][n_kv_heads][max_chunks][16]: the centroid of the chunk's cluster */
-  int32_t* chunk_start;    /* [batch][n_kv_heads][max_chunks]: first row of the chunk in k_sorted */
+  int32_t* chunk_start;    /* [batch][n_kv_heads][max_chunks]: first row of the chunk in `members` order */
   int32_t* chunk_len;      /* [batch][n_kv_heads][max_chunks]: 1..128 */
   int32_t* n_chunks;       /* [batch][n_kv_heads]: chunks in use, cluster-major order */
 } rtp_clusters;
