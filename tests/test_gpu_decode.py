@@ -24,11 +24,12 @@ def rtp(cuda_device):
 def oracle_centroids(kc, kinds, block, proj):
     """Cached centroids of every retrieval head, computed by the oracle."""
     B, H, Lc = kc.shape[0], kc.shape[1], kc.shape[2]
-    C = torch.zeros(B, H, Lc // block, 16, dtype=torch.float32)
+    n = Lc // block  # complete blocks (at least one row is allocated: the call wants a centroid array)
+    C = torch.zeros(B, H, max(1, n), 16, dtype=torch.float32)
     for b in range(B):
         for h in range(H):
-            if kinds[h] == 2:
-                C[b, h] = torch.from_numpy(oracle.centroids(cpu(kc[b, h]), block, cpu(proj)).astype(np.float32))
+            if kinds[h] == 2 and n:
+                C[b, h, :n] = torch.from_numpy(oracle.centroids(cpu(kc[b, h]), block, cpu(proj)).astype(np.float32))
     return C
 
 
@@ -88,6 +89,25 @@ DECODE_CASES = [
 
 @pytest.mark.parametrize("case", DECODE_CASES)
 def test_decode_small(rtp, cuda_device, case):
+    B, hq, hkv, kinds, Lc, window, block, topk, n_local = case
+    w = inputs.Workload(4, "t", B, 1, hq, hkv, 1, window, block, topk, n_local, "lowfreq", 0, [kinds],
+                        cache_len=Lc, decode=True)
+    d = inputs.decode_step(w, "cpu")
+    check_decode(rtp, d, kinds, window, block, topk, n_local, cuda_device)
+
+
+SHORT_CACHE_CASES = [
+    # batch, hq, hkv, kinds, cache_len, window, block, topk, n_local
+    (1, 8, 2, [2, 0], 1, 100, 64, 4, 2),    # a single cached token
+    (1, 8, 2, [2, 1], 63, 100, 64, 4, 2),   # no complete block yet; a full head
+    (1, 8, 2, [2, 0], 64, 32, 64, 4, 2),    # exactly one block; window shorter than the cache
+    (2, 8, 2, [2, 0], 65, 64, 64, 4, 1),    # the new token opens block 1
+    (1, 4, 1, [2], 300, 64, 64, 1, 1),      # top-k 1
+]
+
+
+@pytest.mark.parametrize("case", SHORT_CACHE_CASES, ids=[f"len{c[4]}-k{c[7]}" for c in SHORT_CACHE_CASES])
+def test_decode_short_caches(rtp, cuda_device, case):
     B, hq, hkv, kinds, Lc, window, block, topk, n_local = case
     w = inputs.Workload(4, "t", B, 1, hq, hkv, 1, window, block, topk, n_local, "lowfreq", 0, [kinds],
                         cache_len=Lc, decode=True)

@@ -60,6 +60,8 @@ def test_tiny_v2_layer(rtp, cuda_device):
 
 EDGE_CASES = [
     # seq, hq, hkv, kinds, window, block, topk, n_local
+    (64, 2, 1, [2], 64, 64, 2, 1),              # one block of 64: half a query tile, sink only
+    (64, 4, 2, [0, 1], 16, 64, 1, 1),           # one block of 64, SWA and full
     (128, 2, 1, [1], 64, 128, 2, 1),            # one tile, full
     (128, 2, 1, [0], 1, 128, 2, 1),             # window 1: each row sees itself
     (192, 2, 1, [2], 64, 64, 1, 1),             # ragged last 128-row tile, block 64
