@@ -84,6 +84,18 @@ def layer_flops(w, kinds) -> tuple[float, float]:
     return float(algo), float(tiles * G * TILE_FLOPS)
 
 
+def decode_work(w, kinds, Lc) -> tuple[int, int]:
+    """(algorithmic bytes, FLOPs) of one decode step: per sequence, the K/V
+    rows every head reads (kmax selected blocks of a retrieval head, the
+    window of a streaming head), the retrieval heads' cached centroids, and
+    q and o."""
+    ns = sum(1 for k in kinds if k == inputs.SPARSE)
+    nsw = len(kinds) - ns
+    keys = ns * w.kmax * w.block + nsw * min(w.window, Lc)
+    bytes_ = w.batch * (keys * 128 * 2 * 2 + ns * (Lc // w.block) * 16 * 4 + w.n_q_heads * 128 * 2 * 2)
+    return bytes_, w.batch * keys * w.group * 4 * 128
+
+
 def indexer_bytes(w, kinds) -> float:
     ns = sum(1 for k in kinds if k == inputs.SPARSE)
     nb = w.seq // w.block
@@ -659,13 +671,7 @@ def time_decode(rtp, steps, device):
     rotating = time_decode_rotating(rtp, w, d, C, cfg, steps, stream)
     upkeep = time_cache_upkeep(rtp, w, d, C, cfg, flush, flush_read, steps, stream)
     clustered = time_clustered_decode(rtp, w, d, flush, flush_read, steps, stream)
-    G = w.group
-    ns = sum(1 for k in kinds if k == inputs.SPARSE)
-    nsw = len(kinds) - ns
-    kmax = w.kmax
-    keys = ns * kmax * w.block + nsw * min(w.window, Lc)
-    bytes_ = w.batch * (keys * 128 * 2 * 2 + ns * (Lc // w.block) * 16 * 4 + w.n_q_heads * 128 * 2 * 2)
-    flops = w.batch * keys * G * 4 * 128
+    bytes_, flops = decode_work(w, kinds, Lc)
     return {"workload": w.name, "ms_per_step": ms, "algorithmic_bytes": bytes_, "gb_s": bytes_ / (ms * 1e-3) / 1e9,
             "tflops_effective": flops / (ms * 1e-3) / 1e12, "l2": "flushed before each step (256 MB write, then 256 MB read)",
             "launches_per_step": 3, "status": rtp.status_str(status), "rotating": rotating,

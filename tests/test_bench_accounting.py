@@ -55,3 +55,19 @@ def test_full_size_flops_match_the_published_figures(wid, layers, expected):
     w = inputs.workload(wid)
     total = sum(bench.layer_flops(w, w.kinds[layer])[0] for layer in layers)
     assert abs(total - expected) <= 1e-3 * expected, total
+
+
+def test_decode_and_indexer_bytes_match_the_published_figures():
+    """The byte counts behind the decode and indexer roofline fractions: 95.0 MB
+    and 7.3e8 FLOPs per 8 x 256K decode step (37 blocks of 128 keys for each of
+    three retrieval heads, the 8192-key window, centroids, q and o, per
+    sequence), and 2.42 GB per indexer launch on the 1M-token layer (K of the
+    retrieval head and Q of its group of eight, plus the centroids and
+    summaries)."""
+    w = inputs.workload(4)
+    bytes_, flops = bench.decode_work(w, w.kinds[0], w.cache_len)
+    assert abs(bytes_ - 95.0e6) <= 1e-3 * 95.0e6, bytes_
+    assert abs(flops - 7.3e8) <= 1e-2 * 7.3e8, flops
+    w3 = inputs.workload(3)
+    ib = bench.indexer_bytes(w3, w3.kinds[0])
+    assert abs(ib - 2.42e9) <= 5e-3 * 2.42e9, ib
