@@ -124,6 +124,15 @@ MUTANTS = [
     ("sparse rows read the first query block's selection", CPP,
      [("long b = sel[t * static_cast<long>(kmax) + e];", "long b = sel[e];")]),
     ("decode overrides a given selection", CPP, [("if (mode == 2 && !use_given_sel) {", "if (mode == 2) {")]),
+    ("k-means seeds one row late", CPP,
+     [("const long j = (static_cast<long>(2 * c + 1) * n) / (2L * nc);",
+       "const long j = std::min(n - 1, (static_cast<long>(2 * c + 1) * n) / (2L * nc) + 1);")]),
+    ("probabilities without the scale", CPP,
+     [("acc += widen_bf16(q_row[d]) * widen_bf16(k[keys[e] * D + d]);\n    s[e] = scale * acc;",
+       "acc += widen_bf16(q_row[d]) * widen_bf16(k[keys[e] * D + d]);\n    s[e] = acc;")]),
+    ("decode drops the new token's own key from its block", CPP,
+     [("        for (long j = b * B; j < (b + 1) * B; ++j)\n          if (j <= i) keys.push_back(j);",
+       "        for (long j = b * B; j < (b + 1) * B; ++j)\n          if (j < i) keys.push_back(j);")]),
     # --- Python statements ---
     ("chunk ties kept by higher index", PY,
      [("order = np.lexsort((np.arange(s.size), -s))", "order = np.lexsort((-np.arange(s.size), -s))")]),
@@ -156,6 +165,10 @@ MUTANTS = [
     ("matrix attention window starts one key late", PY,
      [("keys = torch.arange(max(0, int(pp[idx].min()) - window + 1), hi + 1)",
        "keys = torch.arange(max(0, int(pp[idx].min()) - window + 2), hi + 1)")]),
+    ("cluster sizes miss trailing empty clusters", PY,
+     [("counts = np.bincount(a, minlength=n_clusters)", "counts = np.bincount(a)")]),
+    ("matrix attention drops each selected block's last key", PY,
+     [("torch.arange(b * block, (b + 1) * block) for b in blocks", "torch.arange(b * block, (b + 1) * block - 1) for b in blocks")]),
     ("matrix attention window one key wider", PY,
      [("visible &= keys[None, :] > i[:, None] - window", "visible &= keys[None, :] >= i[:, None] - window")]),
     ("matrix attention without the scale", PY,

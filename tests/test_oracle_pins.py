@@ -162,7 +162,7 @@ def test_sparse_covering_all_blocks_is_full_bitwise(small):
 
 @pytest.mark.parametrize("mode,window", [(oracle.FULL, 0), (oracle.SWA, 50)])
 def test_rows_are_distributions(small, mode, window):
-    q, k = small["q"][0, 0], small["k"][0, 0]
+    q, k, v = small["q"][0, 0], small["k"][0, 0], small["v"][0, 0]
     n = q.shape[0]
     for i in (0, 1, 49, 50, 51, 200, n - 1):
         p = oracle.attention_probs(q[i], i, k, mode, window)
@@ -171,6 +171,9 @@ def test_rows_are_distributions(small, mode, window):
         if mode == oracle.SWA:
             vis &= np.arange(n) > i - window
         assert np.all(p[~vis] == 0.0) and np.all(p[vis] > 0.0)
+        # the same weights as the output row (same logits, same scale)
+        row = oracle.attention_rows(q[i:i + 1], np.array([i]), k, v, mode, window)[0]
+        assert np.max(np.abs(p @ widen(v) - row)) <= 1e-12
 
 
 def test_ones_value_gives_ones(small):
