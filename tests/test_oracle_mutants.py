@@ -133,6 +133,16 @@ MUTANTS = [
     ("decode drops the new token's own key from its block", CPP,
      [("        for (long j = b * B; j < (b + 1) * B; ++j)\n          if (j <= i) keys.push_back(j);",
        "        for (long j = b * B; j < (b + 1) * B; ++j)\n          if (j < i) keys.push_back(j);")]),
+    ("projection drops the last dimension", CPP,
+     [("for (int d = 0; d < D; ++d) s += static_cast<double>(P[d * r + c])",
+       "for (int d = 0; d < D - 1; ++d) s += static_cast<double>(P[d * r + c])")]),
+    ("k-means mean sums the first dimension only", CPP,
+     [("sum[assign[j] * r + d] += X[j * r + d];", "sum[assign[j] * r + d] += X[j * r];")]),
+    ("row attention reads the first query row for every row", CPP,
+     [("qd[d] = widen_bf16(q_rows[r * D + d]);", "qd[d] = widen_bf16(q_rows[d]);")]),
+    ("decode summary takes head 0 for every head", CPP,
+     [("project_row(q + h * D, D, P, r, qt.data());\n      for (int c = 0; c < r; ++c) qbar[c] += qt[c];",
+       "project_row(q, D, P, r, qt.data());\n      for (int c = 0; c < r; ++c) qbar[c] += qt[c];")]),
     # --- Python statements ---
     ("chunk ties kept by higher index", PY,
      [("order = np.lexsort((np.arange(s.size), -s))", "order = np.lexsort((-np.arange(s.size), -s))")]),
@@ -169,6 +179,12 @@ MUTANTS = [
      [("counts = np.bincount(a, minlength=n_clusters)", "counts = np.bincount(a)")]),
     ("matrix attention drops each selected block's last key", PY,
      [("torch.arange(b * block, (b + 1) * block) for b in blocks", "torch.arange(b * block, (b + 1) * block - 1) for b in blocks")]),
+    ("bf16 rounding loses NaN", PY, [("    out[np.isnan(a)] = np.nan\n", "")]),
+    ("chunk top-k left in score order", PY, [("return np.sort(order[:topk])", "return order[:topk]")]),
+    ("clustered decode takes the previous chunk", PY,
+     [("_, s0, n = chunks[int(x)]", "_, s0, n = chunks[int(x) - 1]")]),
+    ("matrix attention uses the next row's query block", PY,
+     [("tq = pp // block", "tq = np.minimum((pp + 1) // block, pp.max() // block)")]),
     ("matrix attention window one key wider", PY,
      [("visible &= keys[None, :] > i[:, None] - window", "visible &= keys[None, :] >= i[:, None] - window")]),
     ("matrix attention without the scale", PY,

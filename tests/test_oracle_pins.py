@@ -499,6 +499,10 @@ def test_round_bf16_matches_exact_nearest_even():
     x = np.concatenate([x, mids, -mids, np.nextafter(mids, 0), np.nextafter(mids, np.inf), grid[:-1:211],
                         [0.0, -0.0, 2.0 ** -133, 3 * 2.0 ** -134, 2.0 ** -134, np.inf, -np.inf, np.nan,
                          (2.0 - 2.0 ** -8) * 2.0 ** 127, 3.4e38, 1e300]])
+    # NaNs whose payload lies only in the low fraction bits (rounding the bits
+    # alone would turn them into infinities)
+    low_nan = np.array([0x7FF0000000000001, 0xFFF0000000000010, 0x7FF00000000FFFFF], dtype=np.uint64).view(np.float64)
+    x = np.concatenate([x, low_nan])
     got = oracle.round_bf16(x)
     want = np.array([brute_round_bf16(v, grid) for v in x])
     assert np.array_equal(got, want, equal_nan=True)
