@@ -167,3 +167,43 @@ def test_exchange_delivers_exactly_the_requested_rows(cp, world):
         assert p.exitcode == 0
     res = dict(q.get(timeout=10) for _ in range(world))
     assert all(res[r] for r in range(world)), res
+
+
+def test_overlapped_launch_is_the_shortest_prefix_covering_the_exchange(cp):
+    """overlap_head_items picks how many of a rank's first local items the
+    capped launch runs while the K/V exchange is in flight: the shortest
+    prefix whose planned KV tiles reach 1.25 x the exchange time at the
+    per-tile rate on the given number of CTAs (all local items if none
+    does).  Item costs are the planner's tile counts: t + 1 for a full head,
+    the window's tiles for a streaming head, min(t + 1, 1 + k + L) for a
+    sparse head (the selected block count)."""
+    from swa_hybrid_attention_b200 import rtp
+
+    cfg = rtp.AttnConfig(1, 1 << 20, 32, 4, 8192, 128, 128, 8)
+    rng = np.random.default_rng(3)
+    kinds = rng.integers(0, 3, 400)
+    ts = rng.integers(0, 8192, 400)
+    items = np.stack([kinds, np.zeros(400), np.zeros(400), ts], axis=1).astype(np.int64)
+    cost = []
+    for kind, t in zip(kinds, ts):
+        if kind == 1:
+            cost.append(t + 1)
+        elif kind == 0:
+            lo = max(0, (128 * t - cfg.window + 1)) // 128
+            cost.append(t - lo + 1)
+        else:
+            sel = t + 1 if t - cfg.n_local <= cfg.topk else 1 + cfg.topk + cfg.n_local
+            cost.append(sel)
+    tile_s, ctas = 2.4e-6, 132
+    for exchange_s in (0.0, 1e-5, 3e-4, 5.7e-4, 1e-3, 1.0):
+        n_local = 300
+        n = cp.overlap_head_items(items, n_local, cfg, exchange_s, ctas, tile_s)
+        budget = 1.25 * exchange_s / tile_s * ctas
+        prefix = np.concatenate([[0], np.cumsum(cost[:n_local])])
+        assert 0 <= n <= n_local
+        if n < n_local:
+            assert prefix[n] >= budget and (n == 0 or prefix[n - 1] < budget), (exchange_s, n)
+        else:
+            assert prefix[n_local - 1] < budget
+    assert cp.overlap_head_items(items, 300, cfg, 0.0, ctas, tile_s) == 0
+    assert cp.overlap_head_items(items, 300, cfg, 1.0, ctas, tile_s) == 300
