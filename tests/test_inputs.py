@@ -64,3 +64,26 @@ def test_generation_is_seeded_and_values_are_not_rotated():
     plain = inputs.small_prefill(256, 4, 2, [SPARSE, SWA], seed=9, rotate=False)
     assert torch.equal(plain["v"], a["v"])  # V is never rotated
     assert not torch.equal(plain["k"], a["k"]) and torch.equal(plain["k"][:, :, 0], a["k"][:, :, 0])  # position 0
+
+
+def test_rotary_encoding_rotates_pairs_i_and_i_plus_64():
+    """Rotate-half pairs (i, i + 64) turned by position * 1e6^(-2i/128): as
+    complex numbers x_i + 1j x_(i+64) multiplied by exp(1j * angle); the
+    rotation keeps each pair's norm, and the scores q.k of two rotated rows
+    depend only on the difference of their positions."""
+    torch.manual_seed(0)
+    n = 300
+    x = torch.randn(n, 128, dtype=torch.float64)
+    cos, sin = inputs.rope_tables(n, "cpu")
+    y = inputs.apply_rope_fp32(x.float(), cos, sin).double()
+    i = torch.arange(64, dtype=torch.float64)
+    ang = torch.arange(n, dtype=torch.float64)[:, None] * 1e6 ** (-2.0 * i / 128)[None, :]
+    z = torch.complex(x[:, :64], x[:, 64:]) * torch.exp(1j * ang)
+    assert torch.allclose(y[:, :64], z.real, atol=1e-5) and torch.allclose(y[:, 64:], z.imag, atol=1e-5)
+    assert torch.allclose(y[:, :64] ** 2 + y[:, 64:] ** 2, x[:, :64] ** 2 + x[:, 64:] ** 2, rtol=1e-5, atol=1e-5)
+    q, k = torch.randn(128, dtype=torch.float64), torch.randn(128, dtype=torch.float64)
+    qs = inputs.apply_rope_fp32(q.float().expand(n, 128), cos, sin).double()
+    ks = inputs.apply_rope_fp32(k.float().expand(n, 128), cos, sin).double()
+    s1 = (qs[200] * ks[150]).sum()  # offset 50
+    s2 = (qs[80] * ks[30]).sum()
+    assert abs(float(s1 - s2)) <= 1e-4
