@@ -1,5 +1,6 @@
-"""The C-ABI library loads, exports every symbol include/rtp.h declares, and
-rejects bad arguments before touching the GPU (runs without a GPU)."""
+"""The C-ABI library loads, exports every symbol include/rtp.h declares, the
+ctypes binding declares every one with the header's argument list, and the
+library rejects bad arguments before touching the GPU (runs without a GPU)."""
 
 import ctypes
 import os
@@ -180,3 +181,49 @@ def test_cluster_calls_validate_before_launch(rtp):
     assert rtp.rtp_decode_clustered_workspace_bytes(cfg, [2, 0], 3000, 2048) > 0
     assert lib.rtp_sparse_decode_clustered(ctypes.byref(c), kinds, 3000, fake, fake, fake, fake, None, fake, fake,
                                            1 << 30, None, None, None) == inv
+
+
+def declared_prototypes():
+    """{name: (return type, [parameter types])} of every function in include/rtp.h."""
+    text = open(os.path.join(ROOT, "include", "rtp.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    out = {}
+    for ret, name, params in re.findall(r"([A-Za-z_][\w \*]*?)\s*\b(rtp_[a-z_]+)\s*\(([^;{]*?)\)\s*;", text):
+        ps = [p.strip() for p in params.split(",") if p.strip()]
+        if ps == ["void"]:
+            ps = []
+        types = [re.sub(r"\s*\b\w+$", "", p) if not p.endswith("*") else p for p in ps]
+        out[name] = (ret.strip(), types)
+    return out
+
+
+def _kind_of_c(t: str) -> str:
+    t = t.replace("const", "").strip()
+    if "*" in t:
+        return "ptr"
+    return {"int": "int", "long": "long", "size_t": "size_t", "float": "float", "double": "double",
+            "unsigned": "uint", "rtp_status": "int", "void": "void"}[t]
+
+
+def _kind_of_ctypes(t) -> str:
+    if t is None:
+        return "void"
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+        return "ptr"
+    return {ctypes.c_int: "int", ctypes.c_long: "long", ctypes.c_size_t: "size_t", ctypes.c_float: "float",
+            ctypes.c_double: "double", ctypes.c_uint: "uint"}[t]
+
+
+def test_binding_signatures_match_the_header(rtp):
+    """ctypes does not check a call against the C prototype, so the binding's
+    argument list is compared with rtp.h here: same count, and each argument
+    of the same kind (pointer, int, long, size_t, float, unsigned), and the
+    same kind of result."""
+    protos = declared_prototypes()
+    assert set(protos) == set(rtp.EXPORTED)
+    for name, (ret, params) in protos.items():
+        f = getattr(rtp._lib, name)
+        got = [_kind_of_ctypes(t) for t in (f.argtypes or [])]
+        assert got == [_kind_of_c(p) for p in params], (name, got, params)
+        assert _kind_of_ctypes(f.restype) == _kind_of_c(ret), (name, f.restype, ret)
