@@ -227,3 +227,31 @@ def test_binding_signatures_match_the_header(rtp):
         got = [_kind_of_ctypes(t) for t in (f.argtypes or [])]
         assert got == [_kind_of_c(p) for p in params], (name, got, params)
         assert _kind_of_ctypes(f.restype) == _kind_of_c(ret), (name, f.restype, ret)
+
+
+def declared_structs():
+    """{typedef name: [(field type, field name)]} of the header's plain structs."""
+    text = open(os.path.join(ROOT, "include", "rtp.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = {}
+    for body, name in re.findall(r"typedef struct\s*\{(.*?)\}\s*(\w+)\s*;", text, flags=re.S):
+        fields = []
+        for decl in body.split(";"):
+            decl = " ".join(decl.split())
+            if decl:
+                m = re.match(r"(.*?)(\w+)$", decl)
+                fields.append((m.group(1).strip(), m.group(2)))
+        out[name] = fields
+    return out
+
+
+def test_binding_structs_match_the_header(rtp):
+    """The ctypes structures passed by pointer have the header's fields, in
+    its order and of its kinds, and the same size."""
+    structs = declared_structs()
+    assert set(structs) == {"rtp_attn_cfg", "rtp_clusters"}
+    for name, fields in structs.items():
+        cls = getattr(rtp, name)
+        got = [(n, _kind_of_ctypes(t)) for n, t in cls._fields_]
+        assert got == [(n, _kind_of_c(t)) for t, n in fields], name
+    assert ctypes.sizeof(rtp.rtp_attn_cfg) == 12 * 4
